@@ -1,0 +1,434 @@
+/*
+ * pararnn_oracle.c -- plain fp64 CPU oracle for the ParaRNN hot path.
+ *
+ * TEST INFRASTRUCTURE ONLY.  The test suite, the smoke check and the CPU
+ * baseline leg of the benchmark call this code; the CUDA library never does,
+ * and this file includes nothing from it.
+ *
+ * What it computes (all in double precision, one channel at a time, with no
+ * scan, no blocking and no fusion):
+ *
+ *   - the sequential unroll s_t = f(s_{t-1}, x_t), s_{-1} = h0
+ *     ("sequential_apply" / ".eval() keeps the one-step recurrence",
+ *      pararnn-torch PyPI page, Quickstart and API overview sections);
+ *   - K Newton iterations on the whole-trajectory system
+ *     F(H)_t = h_t - f(h_{t-1}, x_t) = 0 (pararnn-torch PyPI page, Method
+ *     section; ParaRNN thread, tweet [3/8]), starting from the warm start
+ *     h_t^(0) = f(0, x_t) (Method section, "paper App. A"), each linear
+ *     system J delta = -F solved by a plain forward substitution in time;
+ *   - the adjoint of the recurrence at a given trajectory H: the reverse
+ *     recursion lambda_t = g_t + A_{t+1}^T lambda_{t+1} and the parameter
+ *     gradients it implies (Method section, "Backward follows paper eq. 2.6";
+ *     the equation itself is not printed, so this is the plain adjoint of the
+ *     triangular system F(H) = 0).
+ *
+ * Cells (state width S, gate count G, pre-activations p_g, diagonal
+ * recurrent weights a_g, one channel):
+ *   0 linear   S=1 G=2  f = p_a * h + p_b                     (no weights)
+ *   1 diag GRU S=1 G=3  z = sig(p_z + a_z h), r = sig(p_r + a_r h),
+ *                       c = tanh(p_c + a_c r h), f = (1 - z) h + z c
+ *   2 diag LSTM S=2 G=4 state (c, h), gates (i, f, o, c):
+ *                       i = sig(p_i + a_i h), f = sig(p_f + a_f h + 1),
+ *                       o = sig(p_o + a_o h), g = tanh(p_c + a_c h),
+ *                       c' = f c + i g, h' = o tanh(c')
+ * GRU and LSTM are the diagonal (per-channel) forms of the ParaGRU / ParaLSTM
+ * cells listed on the pararnn-torch page (Models, Usage); the linear cell is
+ * the affine recurrence that the News section says needs no Newton iteration
+ * beyond one exact scan.
+ *
+ * Layouts (row-major, D fastest): px (B,T,G,D), w (G,D), h0 (B,S,D),
+ * H / dL_dH (B,T,S,D), dL_dpx (B,T,G,D), dL_da (G,D), dL_dh0 (B,S,D).
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define MAXS 2
+#define MAXG 4
+
+static int ncell_gates(int cell) { return cell == 0 ? 2 : cell == 1 ? 3 : cell == 2 ? 4 : -1; }
+static int ncell_state(int cell) { return cell == 0 ? 1 : cell == 1 ? 1 : cell == 2 ? 2 : -1; }
+
+int oracle_num_gates(int cell) { return ncell_gates(cell); }
+int oracle_state_width(int cell) { return ncell_state(cell); }
+
+static double sig(double x) { return 1.0 / (1.0 + exp(-x)); }
+
+/* max that lets a NaN through, so that a non-finite residual is visible */
+static double nanmax(double a, double b) {
+    if (a != a) return a;
+    if (b != b) return b;
+    return a > b ? a : b;
+}
+
+/* ---- one cell application and its derivatives ------------------------- */
+
+/* s' = f(s, p) for one channel.  p: G pre-activations, w: G weights (may be
+ * NULL for the linear cell), s: S state values. */
+void oracle_cell_step(int cell, const double* p, const double* w, const double* s, double* out) {
+    if (cell == 0) {
+        out[0] = p[0] * s[0] + p[1];
+    } else if (cell == 1) {
+        double h = s[0];
+        double z = sig(p[0] + w[0] * h);
+        double r = sig(p[1] + w[1] * h);
+        double c = tanh(p[2] + w[2] * r * h);
+        out[0] = (1.0 - z) * h + z * c;
+    } else {
+        double c = s[0], h = s[1];
+        double ig = sig(p[0] + w[0] * h);
+        double fg = sig(p[1] + w[1] * h + 1.0);
+        double og = sig(p[2] + w[2] * h);
+        double gg = tanh(p[3] + w[3] * h);
+        double cn = fg * c + ig * gg;
+        out[0] = cn;
+        out[1] = og * tanh(cn);
+    }
+}
+
+/* A = d f / d s at (s, p), S x S row-major: A[i*S + j] = d s'_i / d s_j. */
+void oracle_cell_jacobian(int cell, const double* p, const double* w, const double* s, double* A) {
+    if (cell == 0) {
+        A[0] = p[0];
+    } else if (cell == 1) {
+        double h = s[0];
+        double z = sig(p[0] + w[0] * h);
+        double r = sig(p[1] + w[1] * h);
+        double c = tanh(p[2] + w[2] * r * h);
+        /* d f/d p_z, d f/d p_c, d f/d p_r by the chain rule */
+        double Gz = (c - h) * z * (1.0 - z);
+        double Gc = z * (1.0 - c * c);
+        double Gr = Gc * w[2] * h * r * (1.0 - r);
+        /* h enters directly through (1 - z) h, and through each gate's
+         * pre-activation: a_z h, a_r h and a_c r h (d(r h)/dh = r + h dr/dh) */
+        A[0] = (1.0 - z) + w[0] * Gz + w[1] * Gr + w[2] * r * Gc;
+    } else {
+        double c = s[0], h = s[1];
+        double ig = sig(p[0] + w[0] * h);
+        double fg = sig(p[1] + w[1] * h + 1.0);
+        double og = sig(p[2] + w[2] * h);
+        double gg = tanh(p[3] + w[3] * h);
+        double cn = fg * c + ig * gg;
+        double tn = tanh(cn);
+        double dcn_dh = c * fg * (1.0 - fg) * w[1] + gg * ig * (1.0 - ig) * w[0] + ig * (1.0 - gg * gg) * w[3];
+        A[0] = fg;                                   /* dc'/dc */
+        A[1] = dcn_dh;                               /* dc'/dh */
+        A[2] = og * (1.0 - tn * tn) * fg;            /* dh'/dc */
+        A[3] = og * (1.0 - og) * w[2] * tn + og * (1.0 - tn * tn) * dcn_dh; /* dh'/dh */
+    }
+}
+
+/* dp[i*G + g] = d s'_i / d p_g and da[i*G + g] = d s'_i / d a_g at (s, p). */
+void oracle_cell_param_grads(int cell, const double* p, const double* w, const double* s, double* dp, double* da) {
+    if (cell == 0) {
+        dp[0] = s[0];
+        dp[1] = 1.0;
+        da[0] = 0.0;
+        da[1] = 0.0;
+    } else if (cell == 1) {
+        double h = s[0];
+        double z = sig(p[0] + w[0] * h);
+        double r = sig(p[1] + w[1] * h);
+        double c = tanh(p[2] + w[2] * r * h);
+        double Gz = (c - h) * z * (1.0 - z);
+        double Gc = z * (1.0 - c * c);
+        double Gr = Gc * w[2] * h * r * (1.0 - r);
+        dp[0] = Gz;
+        dp[1] = Gr;
+        dp[2] = Gc;
+        da[0] = Gz * h;
+        da[1] = Gr * h;
+        da[2] = Gc * r * h;
+    } else {
+        double c = s[0], h = s[1];
+        double ig = sig(p[0] + w[0] * h);
+        double fg = sig(p[1] + w[1] * h + 1.0);
+        double og = sig(p[2] + w[2] * h);
+        double gg = tanh(p[3] + w[3] * h);
+        double cn = fg * c + ig * gg;
+        double tn = tanh(cn);
+        double dc[4], dh[4];
+        dc[0] = gg * ig * (1.0 - ig);     /* dc'/dp_i */
+        dc[1] = c * fg * (1.0 - fg);      /* dc'/dp_f */
+        dc[2] = 0.0;                      /* dc'/dp_o */
+        dc[3] = ig * (1.0 - gg * gg);     /* dc'/dp_c */
+        for (int g = 0; g < 4; ++g) dh[g] = og * (1.0 - tn * tn) * dc[g];
+        dh[2] = og * (1.0 - og) * tn;     /* dh'/dp_o */
+        for (int g = 0; g < 4; ++g) {
+            dp[0 * 4 + g] = dc[g];
+            dp[1 * 4 + g] = dh[g];
+            /* every gate's pre-activation carries a_g * h */
+            da[0 * 4 + g] = dc[g] * h;
+            da[1 * 4 + g] = dh[g] * h;
+        }
+    }
+}
+
+/* ---- per-channel drivers ----------------------------------------------- */
+
+typedef struct {
+    int cell, S, G;
+    int64_t B, T, D;
+    int K;
+    const double* px;
+    const double* w;
+    const double* h0;
+    const double* H_in;   /* adjoint: trajectory to linearise at */
+    const double* dLdH;
+    double* H;            /* unroll / newton output */
+    double* dLdpx;
+    double* dLda_b;       /* adjoint: per-batch partial (B,G,D) */
+    double* dLdh0;
+    int mode;             /* 0 unroll, 1 newton, 2 adjoint */
+    int nthreads;
+    int tid;
+    double resid[64];     /* per-thread residual history (K+1 <= 64) */
+} job_t;
+
+static void load_p(const job_t* j, int64_t b, int64_t t, int64_t d, double* p) {
+    for (int g = 0; g < j->G; ++g) p[g] = j->px[((b * j->T + t) * j->G + g) * j->D + d];
+}
+static void load_w(const job_t* j, int64_t d, double* w) {
+    for (int g = 0; g < j->G; ++g) w[g] = j->w ? j->w[g * j->D + d] : 0.0;
+}
+static void load_h0(const job_t* j, int64_t b, int64_t d, double* s) {
+    for (int i = 0; i < j->S; ++i) s[i] = j->h0 ? j->h0[(b * j->S + i) * j->D + d] : 0.0;
+}
+static double* Hat(double* H, const job_t* j, int64_t b, int64_t t, int i, int64_t d) {
+    return &H[((b * j->T + t) * j->S + i) * j->D + d];
+}
+static double Hget(const double* H, const job_t* j, int64_t b, int64_t t, int i, int64_t d) {
+    return H[((b * j->T + t) * j->S + i) * j->D + d];
+}
+
+static void channel_unroll(job_t* j, int64_t b, int64_t d) {
+    double w[MAXG], p[MAXG], s[MAXS], sn[MAXS];
+    load_w(j, d, w);
+    load_h0(j, b, d, s);
+    for (int64_t t = 0; t < j->T; ++t) {
+        load_p(j, b, t, d, p);
+        oracle_cell_step(j->cell, p, w, s, sn);
+        for (int i = 0; i < j->S; ++i) {
+            s[i] = sn[i];
+            *Hat(j->H, j, b, t, i, d) = s[i];
+        }
+    }
+}
+
+/* max_t |h_t - f(h_{t-1}, x_t)| of the trajectory currently stored in H */
+static double channel_residual(job_t* j, int64_t b, int64_t d) {
+    double w[MAXG], p[MAXG], prev[MAXS], cur[MAXS], fv[MAXS];
+    double r = 0.0;
+    load_w(j, d, w);
+    load_h0(j, b, d, prev);
+    for (int64_t t = 0; t < j->T; ++t) {
+        load_p(j, b, t, d, p);
+        oracle_cell_step(j->cell, p, w, prev, fv);
+        for (int i = 0; i < j->S; ++i) {
+            cur[i] = Hget(j->H, j, b, t, i, d);
+            r = nanmax(r, fabs(cur[i] - fv[i]));
+        }
+        for (int i = 0; i < j->S; ++i) prev[i] = cur[i];
+    }
+    return r;
+}
+
+static void channel_newton(job_t* j, int64_t b, int64_t d) {
+    const int S = j->S;
+    double w[MAXG], p[MAXG], zero[MAXS] = {0.0, 0.0}, fv[MAXS];
+    load_w(j, d, w);
+    /* warm start: h_t^(0) = f(0, x_t) */
+    for (int64_t t = 0; t < j->T; ++t) {
+        load_p(j, b, t, d, p);
+        oracle_cell_step(j->cell, p, w, zero, fv);
+        for (int i = 0; i < S; ++i) *Hat(j->H, j, b, t, i, d) = fv[i];
+    }
+    for (int k = 0; k < j->K; ++k) {
+        /* Newton step: J(H) delta = -F(H).  J is lower block-bidiagonal with
+         * identity on the diagonal and -A_t below it, so the solve is the
+         * forward substitution delta_t = A_t delta_{t-1} - F_t, delta_{-1} = 0. */
+        double prev_old[MAXS], cur_old[MAXS], delta[MAXS] = {0.0, 0.0}, nd[MAXS], A[MAXS * MAXS];
+        double rk = 0.0;
+        load_h0(j, b, d, prev_old);
+        for (int64_t t = 0; t < j->T; ++t) {
+            load_p(j, b, t, d, p);
+            for (int i = 0; i < S; ++i) cur_old[i] = Hget(j->H, j, b, t, i, d);
+            oracle_cell_step(j->cell, p, w, prev_old, fv);
+            oracle_cell_jacobian(j->cell, p, w, prev_old, A);
+            for (int i = 0; i < S; ++i) {
+                double F = cur_old[i] - fv[i];
+                rk = nanmax(rk, fabs(F));
+                double acc = -F;
+                for (int m = 0; m < S; ++m) acc += A[i * S + m] * delta[m];
+                nd[i] = acc;
+            }
+            for (int i = 0; i < S; ++i) {
+                delta[i] = nd[i];
+                *Hat(j->H, j, b, t, i, d) = cur_old[i] + delta[i];
+                prev_old[i] = cur_old[i];
+            }
+        }
+        j->resid[k] = nanmax(j->resid[k], rk);
+    }
+    j->resid[j->K] = nanmax(j->resid[j->K], channel_residual(j, b, d));
+}
+
+static void channel_adjoint(job_t* j, int64_t b, int64_t d) {
+    const int S = j->S, G = j->G;
+    double w[MAXG], p[MAXG], pn[MAXG], s[MAXS], sp[MAXS], A[MAXS * MAXS];
+    double dp[MAXS * MAXG], da[MAXS * MAXG];
+    double lam[MAXS] = {0.0, 0.0}, acc_a[MAXG] = {0.0, 0.0, 0.0, 0.0};
+    load_w(j, d, w);
+    for (int64_t t = j->T - 1; t >= 0; --t) {
+        /* lambda_t = g_t + A_{t+1}^T lambda_{t+1}, A_{t+1} = df/ds at (h_t, x_{t+1}) */
+        double nl[MAXS];
+        for (int i = 0; i < S; ++i) nl[i] = j->dLdH[((b * j->T + t) * S + i) * j->D + d];
+        if (t + 1 < j->T) {
+            load_p(j, b, t + 1, d, pn);
+            for (int i = 0; i < S; ++i) s[i] = Hget(j->H_in, j, b, t, i, d);
+            oracle_cell_jacobian(j->cell, pn, w, s, A);
+            for (int i = 0; i < S; ++i)
+                for (int m = 0; m < S; ++m) nl[i] += A[m * S + i] * lam[m];
+        }
+        for (int i = 0; i < S; ++i) lam[i] = nl[i];
+        /* parameter gradients of row t, linearised at (h_{t-1}, x_t) */
+        load_p(j, b, t, d, p);
+        if (t > 0)
+            for (int i = 0; i < S; ++i) sp[i] = Hget(j->H_in, j, b, t - 1, i, d);
+        else
+            load_h0(j, b, d, sp);
+        oracle_cell_param_grads(j->cell, p, w, sp, dp, da);
+        for (int g = 0; g < G; ++g) {
+            double gp = 0.0, ga = 0.0;
+            for (int i = 0; i < S; ++i) {
+                gp += lam[i] * dp[i * G + g];
+                ga += lam[i] * da[i * G + g];
+            }
+            j->dLdpx[((b * j->T + t) * G + g) * j->D + d] = gp;
+            acc_a[g] += ga;
+        }
+    }
+    for (int g = 0; g < G; ++g) j->dLda_b[(b * G + g) * j->D + d] = acc_a[g];
+    if (j->dLdh0) {
+        /* dL/dh0 = A_0^T lambda_0 with A_0 = df/ds at (h0, x_0) */
+        load_p(j, b, 0, d, p);
+        load_h0(j, b, d, sp);
+        oracle_cell_jacobian(j->cell, p, w, sp, A);
+        for (int i = 0; i < S; ++i) {
+            double acc = 0.0;
+            for (int m = 0; m < S; ++m) acc += A[m * S + i] * lam[m];
+            j->dLdh0[(b * S + i) * j->D + d] = acc;
+        }
+    }
+}
+
+static void* worker(void* arg) {
+    job_t* j = (job_t*)arg;
+    int64_t nch = j->B * j->D;
+    int64_t per = (nch + j->nthreads - 1) / j->nthreads;
+    int64_t lo = (int64_t)j->tid * per, hi = lo + per < nch ? lo + per : nch;
+    for (int64_t c = lo; c < hi; ++c) {
+        int64_t b = c / j->D, d = c % j->D;
+        if (j->mode == 0) channel_unroll(j, b, d);
+        else if (j->mode == 1) channel_newton(j, b, d);
+        else channel_adjoint(j, b, d);
+    }
+    return NULL;
+}
+
+static int run(job_t* proto, int nthreads) {
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > 256) nthreads = 256;
+    job_t* jobs = (job_t*)calloc((size_t)nthreads, sizeof(job_t));
+    pthread_t* th = (pthread_t*)calloc((size_t)nthreads, sizeof(pthread_t));
+    if (!jobs || !th) { free(jobs); free(th); return -2; }
+    for (int i = 0; i < nthreads; ++i) {
+        jobs[i] = *proto;
+        jobs[i].nthreads = nthreads;
+        jobs[i].tid = i;
+        for (int k = 0; k < 64; ++k) jobs[i].resid[k] = 0.0;
+    }
+    for (int i = 1; i < nthreads; ++i) pthread_create(&th[i], NULL, worker, &jobs[i]);
+    worker(&jobs[0]);
+    for (int i = 1; i < nthreads; ++i) pthread_join(th[i], NULL);
+    for (int k = 0; k < 64; ++k) {
+        double r = 0.0;
+        for (int i = 0; i < nthreads; ++i) r = nanmax(r, jobs[i].resid[k]);
+        proto->resid[k] = r;
+    }
+    free(jobs);
+    free(th);
+    return 0;
+}
+
+static int check(int cell, int64_t B, int64_t T, int64_t D, const double* px) {
+    if (ncell_gates(cell) < 0 || B < 0 || T < 0 || D < 0 || (B * T * D > 0 && !px)) return -1;
+    return 0;
+}
+
+/* Sequential unroll.  Returns 0 on success, negative on bad arguments. */
+int oracle_unroll(int cell, int64_t B, int64_t T, int64_t D, const double* px, const double* w,
+                  const double* h0, double* H, int nthreads) {
+    if (check(cell, B, T, D, px) || (cell != 0 && !w)) return -1;
+    job_t j;
+    memset(&j, 0, sizeof j);
+    j.cell = cell; j.S = ncell_state(cell); j.G = ncell_gates(cell);
+    j.B = B; j.T = T; j.D = D; j.px = px; j.w = w; j.h0 = h0; j.H = H; j.mode = 0;
+    return run(&j, nthreads);
+}
+
+/* K Newton iterations from the warm start.  resid (K+1 doubles, may be NULL)
+ * receives max |F(H^(k))| over the whole batch for k = 0..K. */
+int oracle_newton(int cell, int64_t B, int64_t T, int64_t D, const double* px, const double* w,
+                  const double* h0, int K, double* H, double* resid, int nthreads) {
+    if (check(cell, B, T, D, px) || (cell != 0 && !w) || K < 0 || K > 62) return -1;
+    job_t j;
+    memset(&j, 0, sizeof j);
+    j.cell = cell; j.S = ncell_state(cell); j.G = ncell_gates(cell);
+    j.B = B; j.T = T; j.D = D; j.K = K; j.px = px; j.w = w; j.h0 = h0; j.H = H; j.mode = 1;
+    int rc = run(&j, nthreads);
+    if (rc == 0 && resid)
+        for (int k = 0; k <= K; ++k) resid[k] = j.resid[k];
+    return rc;
+}
+
+/* max |F(H)| of a given trajectory H */
+double oracle_residual(int cell, int64_t B, int64_t T, int64_t D, const double* px, const double* w,
+                       const double* h0, const double* H) {
+    job_t j;
+    memset(&j, 0, sizeof j);
+    j.cell = cell; j.S = ncell_state(cell); j.G = ncell_gates(cell);
+    j.B = B; j.T = T; j.D = D; j.px = px; j.w = w; j.h0 = h0; j.H = (double*)H;
+    double r = 0.0;
+    for (int64_t c = 0; c < B * D; ++c) r = nanmax(r, channel_residual(&j, c / D, c % D));
+    return r;
+}
+
+/* Adjoint at trajectory H: dL_dpx (B,T,G,D), dL_da (G,D) summed over b then
+ * t in natural order (may be NULL), dL_dh0 (B,S,D, may be NULL). */
+int oracle_adjoint(int cell, int64_t B, int64_t T, int64_t D, const double* px, const double* w,
+                   const double* h0, const double* H, const double* dLdH, double* dLdpx, double* dLda,
+                   double* dLdh0, int nthreads) {
+    if (check(cell, B, T, D, px) || (cell != 0 && !w) || !H || !dLdH || !dLdpx) return -1;
+    int G = ncell_gates(cell);
+    double* part = (double*)calloc((size_t)(B * G * D > 0 ? B * G * D : 1), sizeof(double));
+    if (!part) return -2;
+    job_t j;
+    memset(&j, 0, sizeof j);
+    j.cell = cell; j.S = ncell_state(cell); j.G = G;
+    j.B = B; j.T = T; j.D = D; j.px = px; j.w = w; j.h0 = h0; j.H_in = H; j.dLdH = dLdH;
+    j.dLdpx = dLdpx; j.dLda_b = part; j.dLdh0 = dLdh0; j.mode = 2;
+    int rc = run(&j, nthreads);
+    if (rc == 0 && dLda) {
+        for (int g = 0; g < G; ++g)
+            for (int64_t d = 0; d < D; ++d) {
+                double acc = 0.0;
+                for (int64_t b = 0; b < B; ++b) acc += part[(b * G + g) * D + d];
+                dLda[g * D + d] = acc;
+            }
+    }
+    free(part);
+    return rc;
+}
