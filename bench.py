@@ -1,0 +1,506 @@
+"""Benchmark: Newton-solve B*T*D elements per second on B200, through the C ABI.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+                    [--workload NAME] [--no-extra]
+
+A step is one pass of the hot path over one batch of the workload: one
+``pararnn_newton_forward`` call (all K Newton iterations; the linear workload
+is one exact scan), plus ``pararnn_newton_backward`` for workloads that carry
+a backward pass.  Inputs are resident in HBM before timing and are larger
+than L2, so no flush is needed between steps.  The device time of the K
+timed steps is measured with CUDA events on the launching stream between a
+barrier and a synchronize on both sides; with N > 1 processes (one per GPU,
+launched by torchrun) each rank solves its own independent problem of the
+full workload size (channels never interact), the time is the max over ranks,
+and ``value`` counts the elements of all ranks (weak scaling).
+
+``--impl reference`` times the fp64 CPU oracle -- the slow, obviously correct
+program every GPU result is checked against -- on a bounded sample of the same
+workload on this machine's host cores (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "Newton-solve B·T·D elements/sec at K iters; achieved HBM GB/s vs B200 peak"
+UNIT = "elem/s"
+
+# Algorithmic HBM bytes per (b,t,d) element for one call, by what the fused
+# kernels must move at minimum: every pre-activation read once, every output
+# written once (the Newton iterate never leaves the chip between iterations).
+#   linear f32 fwd: a, b read (8) + h written (4)                         = 12
+#   GRU fwd: px read (3 x 4 f32 | 3 x 2 bf16) + h written (4)            = 16 | 10
+#   LSTM fwd f32: px read (4 x 4) + (c, h) written (8)                    = 24
+#   GRU bwd: px (3 x 4 | 3 x 2) + H (4) + dL/dH (4) read, dL/dpx (3 x 4) written
+#                                                                        = 32 | 26
+ALGO_BYTES = {
+    ("linear", "f32", "fwd"): 12, ("diag_gru", "f32", "fwd"): 16, ("diag_gru", "bf16", "fwd"): 10,
+    ("diag_lstm", "f32", "fwd"): 24, ("diag_lstm", "bf16", "fwd"): 16,
+    ("linear", "f32", "bwd"): 24, ("diag_gru", "f32", "bwd"): 32, ("diag_gru", "bf16", "bwd"): 26,
+    ("diag_lstm", "f32", "bwd"): 48, ("diag_lstm", "bf16", "bwd"): 40,
+}
+KERNEL_SOURCES = ["newton_fwd.cuh", "adjoint_bwd.cuh", "lookback.cuh", "cells.cuh", "common.cuh", "pararnn_abi.cu"]
+
+
+# --------------------------------------------------------------------------
+# distributed plumbing (host only; testable with gloo on CPU)
+# --------------------------------------------------------------------------
+
+def dist_env():
+    return int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")), int(os.environ.get("WORLD_SIZE", "1"))
+
+
+def dist_init(backend, world):
+    import torch.distributed as dist
+
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist if world > 1 else None
+
+
+def barrier(dist, device=None):
+    if dist is not None:
+        if device is not None and dist.get_backend() == "nccl":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def reduce_max(dist, value, device):
+    """Max of a float over ranks (the timing rule: the slowest rank counts)."""
+    if dist is None:
+        return value
+    import torch
+
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_seed(base_seed, rank):
+    """Each rank draws an independent problem of the full workload size."""
+    return base_seed + 1000 * rank
+
+
+def aggregate_throughput(elements_per_rank, world, steps, max_ms):
+    """Whole-job units/s: every rank's elements over the slowest rank's time."""
+    return elements_per_rank * world * steps / (max_ms / 1e3)
+
+
+# --------------------------------------------------------------------------
+# measurement helpers
+# --------------------------------------------------------------------------
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "nonlinear_rnn_iteration_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "source": "of measured"}
+    return {"hbm_gbs": 6650.0, "source": "of fallback"}
+
+
+def recorded_traffic(kernel, workload):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel sources; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    e = rec.get("%s/%s" % (kernel, workload))
+    if not e or e.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.QUERY,
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        if self.path and os.path.exists(self.path):
+            for line in open(self.path):
+                f = [x.strip() for x in line.split(",")]
+                if len(f) >= 9:
+                    try:
+                        rows.append((float(f[1]), float(f[2]), float(f[3]), f[4], f[5], f[6], f[7], f[8]))
+                    except ValueError:
+                        pass
+            os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        loaded = [r for r in rows if r[2] > 200.0] or rows
+        sm = sorted(r[0] for r in loaded)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in loaded for i in range(4) if r[4 + i].lower() == "active"})
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
+                "samples": len(rows)}
+
+
+# --------------------------------------------------------------------------
+# the native arm
+# --------------------------------------------------------------------------
+
+class Problem:
+    """One workload's device buffers and its C-ABI step."""
+
+    def __init__(self, w, device, seed):
+        import torch
+
+        from nonlinear_rnn_iteration_b200 import binding, workloads
+
+        self.w, self.dev, self.b = w, device, binding
+        x = workloads.device_inputs(w, device, seed=seed, with_grad=w.backward)
+        self.px, self.a = x["px"], x["a"]
+        self.g = x.get("dLdH")
+        del x
+        self.H = torch.empty((w.B, w.T, w.S, w.D), dtype=torch.float32, device=device)
+        self.ws = binding.workspace_for(w.cell_id, w.B, w.T, w.D, w.K, device)
+        if w.backward:
+            self.dpx = torch.empty((w.B, w.T, w.G, w.D), dtype=torch.float32, device=device)
+            self.da = torch.empty((w.G, w.D), dtype=torch.float32, device=device)
+        self.code = binding.BF16 if w.px_dtype == "bf16" else binding.F32
+        self.stream = torch.cuda.current_stream(device)
+
+    def forward(self, px=None, H=None):
+        w = self.w
+        st = self.b.pararnn_newton_forward(w.cell_id, w.B, w.T, w.D, self.code, self.px if px is None else px,
+                                           self.a, None, w.K, self.H if H is None else H, self.ws,
+                                           self.ws.numel(), None, self.stream)
+        if st != 0:
+            raise RuntimeError("forward: %s %s" % (self.b.STATUS[st], self.b.pararnn_last_error()))
+
+    def backward(self):
+        w = self.w
+        st = self.b.pararnn_newton_backward(w.cell_id, w.B, w.T, w.D, self.code, self.px, self.a, None, self.H,
+                                            self.g, self.dpx, self.da, None, self.ws, self.ws.numel(), self.stream)
+        if st != 0:
+            raise RuntimeError("backward: %s %s" % (self.b.STATUS[st], self.b.pararnn_last_error()))
+
+    def step(self):
+        self.forward()
+        if self.w.backward:
+            self.backward()
+
+    def launches_per_step(self):
+        return 1 + (2 if self.w.backward else 0)
+
+    def check_status(self):
+        st = self.b.pararnn_status_sync(self.ws, self.stream)
+        if st != 0:
+            raise RuntimeError("device status %s" % self.b.STATUS[st])
+
+
+def time_device(prob, steps, warmup, dist, device, per_call=True):
+    """Returns (ms_per_step max over ranks, fwd_ms, bwd_ms) with CUDA events."""
+    import torch
+
+    for _ in range(warmup):
+        prob.step()
+    prob.check_status()
+    barrier(dist, device)
+    torch.cuda.synchronize(device)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(prob.stream)
+    for i in range(steps):
+        ev[i][0].record(prob.stream)
+        prob.forward()
+        ev[i][1].record(prob.stream)
+        if prob.w.backward:
+            prob.backward()
+        ev[i][2].record(prob.stream)
+    t1.record(prob.stream)
+    torch.cuda.synchronize(device)
+    barrier(dist, device)
+    total = t0.elapsed_time(t1)
+    fwd = sum(a.elapsed_time(b) for a, b, _ in ev) / steps
+    bwd = sum(b.elapsed_time(c) for _, b, c in ev) / steps
+    prob.check_status()
+    return reduce_max(dist, total, device) / steps, fwd, bwd
+
+
+def time_e2e(prob, steps):
+    """Same step through the public API with host buffers: pinned host ->
+    device copy of the pre-activations, the forward (and backward) call, device
+    -> host copy of the result, all inside the timed region."""
+    import torch
+
+    w = prob.w
+    px_host = torch.empty(prob.px.shape, dtype=prob.px.dtype, pin_memory=True)
+    px_host.copy_(prob.px)
+    H_host = torch.empty(prob.H.shape, dtype=torch.float32, pin_memory=True)
+    outs = [H_host]
+    if w.backward:
+        g_host = torch.empty(prob.g.shape, dtype=torch.float32, pin_memory=True)
+        g_host.copy_(prob.g)
+        dpx_host = torch.empty(prob.dpx.shape, dtype=torch.float32, pin_memory=True)
+        outs.append(dpx_host)
+    px_dev = torch.empty_like(prob.px)
+    s = prob.stream
+
+    def one():
+        px_dev.copy_(px_host, non_blocking=True)
+        if w.backward:
+            prob.g.copy_(g_host, non_blocking=True)
+        prob.forward(px=px_dev)
+        if w.backward:
+            prob.backward()
+        H_host.copy_(prob.H, non_blocking=True)
+        if w.backward:
+            dpx_host.copy_(prob.dpx, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(s)
+    for _ in range(steps):
+        one()
+    t1.record(s)
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1) / steps
+    h2d = px_host.numel() * px_host.element_size() + (g_host.numel() * 4 if w.backward else 0)
+    d2h = sum(o.numel() * o.element_size() for o in outs)
+    return ms, h2d, d2h
+
+
+def cpu_baseline(w, device, seed, target_s=12.0):
+    """The oracle as it stands, on a bounded sample of the workload's channels
+    (full length T each), on this host's cores."""
+    import numpy as np
+
+    import oracle
+    from nonlinear_rnn_iteration_b200 import workloads
+
+    threads = os.cpu_count() or 1
+    x = workloads.device_inputs(w, device, seed=seed)
+
+    def run(n):
+        chans = workloads.sample_channels(w, n, seed=5)
+        bs = [b for b, _ in chans]
+        ds = [d for _, d in chans]
+        import torch
+
+        bi, di = torch.tensor(bs, device=device), torch.tensor(ds, device=device)
+        px = x["px"][bi, :, :, di].float().cpu().numpy().astype(np.float64).transpose(1, 2, 0)[None]
+        a = None if x["a"] is None else x["a"][:, di].cpu().numpy().astype(np.float64)
+        t = time.perf_counter()
+        if w.cell == "linear":
+            oracle.unroll(w.cell_id, px, a, None, nthreads=threads)
+        else:
+            oracle.newton(w.cell_id, px, a, None, K=w.K, nthreads=threads)
+        return time.perf_counter() - t, n * w.T
+
+    n = max(threads, 8)
+    dt, el = run(n)
+    while dt < 1.0 and n < w.B * w.D:
+        n = min(w.B * w.D, n * 4)
+        dt, el = run(n)
+    n_final = int(min(w.B * w.D, max(n, n * target_s / max(dt, 1e-3))))
+    if n_final > n:
+        dt, el = run(n_final)
+        n = n_final
+    del x
+    kind = "sequential unroll" if w.cell == "linear" else "Newton K=%d with sequential solves" % w.K
+    return {"value": el / dt, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": "%d of %d channels at full T=%d (%s, fp64), %.1f s" % (n, w.B * w.D, w.T, kind, dt)}
+
+
+def extra_workloads(names, device, seed_base):
+    """Device-time lines for the other workloads (parity cases, not bench lines)."""
+    import torch
+
+    from nonlinear_rnn_iteration_b200 import workloads
+
+    peak = measured_peaks()["hbm_gbs"]
+    out = {}
+    for name in names:
+        w = workloads.WORKLOADS[name]
+        prob = Problem(w, device, seed_base + w.seed)
+        ms, fwd, bwd = time_device(prob, steps=5, warmup=3, dist=None, device=device)
+        fb = ALGO_BYTES[(w.cell, w.px_dtype, "fwd")] * w.elements
+        rec = {"ms_per_step": round(ms, 4), "elem_per_s": w.elements / (ms / 1e3),
+               "fwd_ms": round(fwd, 4), "fwd_algo_gbs": round(fb / (fwd / 1e3) / 1e9, 1),
+               "fwd_frac_hbm": round(fb / (fwd / 1e3) / 1e9 / peak, 3), "fwd_bytes_per_elem": fb // w.elements}
+        if w.backward:
+            bb = ALGO_BYTES[(w.cell, w.px_dtype, "bwd")] * w.elements
+            rec.update(bwd_ms=round(bwd, 4), bwd_algo_gbs=round(bb / (bwd / 1e3) / 1e9, 1),
+                       bwd_frac_hbm=round(bb / (bwd / 1e3) / 1e9 / peak, 3), bwd_bytes_per_elem=bb // w.elements)
+        out[name] = rec
+        del prob
+        torch.cuda.empty_cache()
+    return out
+
+
+def run_native(args):
+    import torch
+
+    from nonlinear_rnn_iteration_b200 import workloads
+
+    rank, local, world = dist_env()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    dist = dist_init("nccl", world)
+    w = workloads.WORKLOADS[args.workload]
+    prob = Problem(w, device, rank_seed(w.seed, rank))
+    with ClockSampler(local) as clk:
+        ms, fwd_ms, bwd_ms = time_device(prob, args.steps, args.warmup, dist, device)
+    clocks = clk.summary()
+    value = aggregate_throughput(w.elements, world, 1, ms)
+    peaks = measured_peaks()
+    dir_ = "fwd"
+    algo = ALGO_BYTES[(w.cell, w.px_dtype, dir_)] * w.elements
+    achieved = algo / (fwd_ms / 1e3) / 1e9
+    roof = {"bound": "hbm", "kernel": "newton_fwd_kernel", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
+            "peak_source": peaks["source"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+            "traffic": recorded_traffic("newton_fwd_kernel", w.name),
+            "algorithmic_bytes_per_launch": algo, "bytes_per_elem": algo // w.elements,
+            "launch_ms": round(fwd_ms, 4)}
+    e2e_ms, h2d, d2h = time_e2e(prob, steps=3)
+    e2e = {"value": w.elements / (e2e_ms / 1e3) * world, "unit": UNIT, "h2d_bytes_per_step": h2d,
+           "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 3)}
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32" if w.px_dtype == "f32" else "bf16 px / f32 state", "data": "synthetic",
+        "config": {"workload": w.name, "cell": w.cell, "B": w.B, "T": w.T, "D": w.D, "K": w.K,
+                   "px_dtype": w.px_dtype, "backward": w.backward,
+                   "l2": "inputs larger than L2 (%.2f GB pre-activations per rank), no flush"
+                         % (prob.px.numel() * prob.px.element_size() / 1e9),
+                   "parallelism": "replicas%d" % world},
+        "roofline": roof, "e2e": e2e, "gpu_launches": prob.launches_per_step() * args.steps, "clocks": clocks,
+    }
+    del prob
+    torch.cuda.empty_cache()
+    if rank == 0 and world == 1:
+        line["cpu_baseline"] = cpu_baseline(w, device, rank_seed(w.seed, rank))
+        if not args.no_extra:
+            line["workloads"] = extra_workloads([n for n in workloads.WORKLOADS if n != w.name], device, 0)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+def run_reference(args):
+    """The oracle as the reference arm, rank 0 only, on the host cores."""
+    rank, local, world = dist_env()
+    if rank != 0:
+        return
+    import numpy as np
+
+    import oracle
+    from nonlinear_rnn_iteration_b200 import workloads
+
+    w = workloads.WORKLOADS[args.workload]
+    threads = os.cpu_count() or 1
+    # a bounded sample per step: whole channels (full T), sized so that one step
+    # takes a few seconds on this host
+    n = max(threads, 8)
+    per_step = []
+    x = workloads.host_inputs(w.with_shape(B=1, D=n), seed=w.seed)
+
+    def one():
+        t = time.perf_counter()
+        if w.cell == "linear":
+            oracle.unroll(w.cell_id, x["px"], x["a"], None, nthreads=threads)
+        else:
+            oracle.newton(w.cell_id, x["px"], x["a"], None, K=w.K, nthreads=threads)
+        return time.perf_counter() - t
+
+    probe = one()
+    scale = max(1, int(2.0 / max(probe, 1e-3)))
+    n = min(w.B * w.D, n * scale)
+    x = workloads.host_inputs(w.with_shape(B=1, D=n), seed=w.seed)
+    for _ in range(args.warmup):
+        one()
+    for _ in range(args.steps):
+        per_step.append(one())
+    ms = 1e3 * sum(per_step) / len(per_step)
+    value = n * w.T / (ms / 1e3)
+    sample = "%d of %d channels at full T=%d per step (fp64 oracle)" % (n, w.B * w.D, w.T)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "cell": w.cell, "B": w.B, "T": w.T, "D": w.D, "K": w.K,
+                   "px_dtype": w.px_dtype, "parallelism": "host threads"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    del np
+
+
+def main(argv=None):
+    from nonlinear_rnn_iteration_b200 import workloads
+
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--workload", default=workloads.HEADLINE, choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--no-extra", action="store_true", help="skip the other workloads' lines")
+    args = ap.parse_args(argv)
+    args.warmup = max(3, args.warmup)
+    args.steps = max(1, args.steps)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_native(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,165 @@
+/*
+ * pararnn_b200.h -- C ABI of libpararnn_b200, the B200 (sm_100a) hot path of
+ * ParaRNN: Newton iterations on a whole-trajectory nonlinear system, each
+ * linear solve done as a parallel associative scan over time, and the
+ * reverse-time adjoint scan for the backward pass.
+ *
+ * The method (pararnn-torch PyPI page, Method section; ParaRNN thread, tweet
+ * [3/8]; ParaRNN abstract on the Hugging Face paper search page):
+ *   the recurrence h_t = f(h_{t-1}, x_t), t = 0..T-1, h_{-1} = h0, is the
+ *   system F(H)_t = h_t - f(h_{t-1}, x_t) = 0.  Starting from the warm start
+ *   h_t^(0) = f(0, x_t) (Method section, "App. A"), each Newton iteration
+ *   evaluates f and its Jacobian A_t = df/dh_{t-1} at the current iterate and
+ *   solves the lower block-bidiagonal system
+ *       delta_t = A_t delta_{t-1} - F_t,  delta_{-1} = 0,
+ *   by an associative scan over time with the operator
+ *       (A2, b2) o (A1, b1) = (A2 A1, A2 b1 + b2)
+ *   (Method section: "each linear solve is an associative scan over time").
+ *   The library solves the equivalent direct form
+ *       h_t^(k+1) = A_t h_{t-1}^(k+1) + (f(h_{t-1}^(k), x_t) - A_t h_{t-1}^(k)),
+ *   h_{-1} = h0, which is the same update without reading h^(k)_t.
+ *
+ * Cells (diagonal: every channel d is an independent recurrence; p_g are the
+ * gate pre-activations, a_g the per-gate, per-channel recurrent weights):
+ *   PARARNN_CELL_LINEAR     S=1, G=2 (a, b):   h' = a h + b
+ *                           (the affine case the News section says needs no
+ *                           Newton iteration beyond one exact scan)
+ *   PARARNN_CELL_DIAG_GRU   S=1, G=3 (z, r, c): z = sig(p_z + a_z h),
+ *                           r = sig(p_r + a_r h), c = tanh(p_c + a_c r h),
+ *                           h' = (1 - z) h + z c          (ParaGRU, Models)
+ *   PARARNN_CELL_DIAG_LSTM  S=2 state (c, h), G=4 (i, f, o, c):
+ *                           i = sig(p_i + a_i h), f = sig(p_f + a_f h + 1),
+ *                           o = sig(p_o + a_o h), g = tanh(p_c + a_c h),
+ *                           c' = f c + i g, h' = o tanh(c')  (ParaLSTM)
+ *
+ * Layouts (row-major, channels fastest, all device memory owned by the
+ * caller):
+ *   preacts  (B, T, G, D)  float32 or bfloat16 (px_dtype)
+ *   diag_w   (G, D)        float32, or NULL for all-zero weights (ignored by
+ *                          the linear cell)
+ *   h0       (B, S, D)     float32, or NULL for a zero initial state
+ *   H        (B, T, S, D)  float32 (LSTM: state order c, h)
+ *   dL_dH    (B, T, S, D)  float32
+ *   dL_dpx   (B, T, G, D)  float32
+ *   dL_da    (G, D)        float32
+ *   dL_dh0   (B, S, D)     float32
+ * Every pointer must be aligned to its element size; rows are read with
+ * 16-byte (f32) or 8-byte (bf16) vector loads when D is a multiple of 4 and
+ * every pointer is 16-byte aligned, and element by element otherwise.
+ *
+ * Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ * default stream).  Argument errors are detected on the host before anything
+ * is launched and return PARARNN_EINVAL (nothing is written).  Conditions the
+ * GPU detects -- a non-finite value in the output, a wait between thread
+ * blocks that ran past its time limit -- are recorded in the workspace and
+ * returned by pararnn_status_sync().  A CUDA launch or copy failure returns
+ * PARARNN_ECUDA.  The library allocates no memory and keeps no state between
+ * calls; pararnn_last_error() describes the last failure on the calling
+ * thread.  Results are deterministic: the same inputs give the same bits,
+ * whatever the order in which thread blocks run.
+ */
+#ifndef PARARNN_B200_H
+#define PARARNN_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    PARARNN_OK = 0,
+    PARARNN_EINVAL = 1,     /* bad argument; nothing launched */
+    PARARNN_ENONFINITE = 2, /* a NaN or Inf reached the output */
+    PARARNN_ETIMEOUT = 3,   /* a bounded inter-block wait gave up; outputs invalid */
+    PARARNN_ECUDA = 4       /* a CUDA runtime call failed */
+} pararnn_status;
+
+typedef enum {
+    PARARNN_CELL_LINEAR = 0,
+    PARARNN_CELL_DIAG_GRU = 1,
+    PARARNN_CELL_DIAG_LSTM = 2
+} pararnn_cell;
+
+typedef enum {
+    PARARNN_F32 = 0,
+    PARARNN_BF16 = 1
+} pararnn_dtype;
+
+/* Gate count G (2, 3, 4) and state width S (1, 1, 2) of a cell; -1 if the
+ * cell is unknown.  Pure host functions. */
+int pararnn_num_gates(pararnn_cell cell);
+int pararnn_state_width(pararnn_cell cell);
+
+/* Bytes of device workspace that pararnn_newton_forward (with this K) and
+ * pararnn_newton_backward need for a (B, T, D) problem; the same buffer
+ * serves both.  0 for an unknown cell or a negative size.  Pure host
+ * function.  The workspace holds the inter-block scan carries, a status
+ * word and per-block gradient partials; its contents need no initialisation
+ * (each call resets what it uses on `stream`). */
+size_t pararnn_workspace_bytes(pararnn_cell cell, int64_t B, int64_t T, int64_t D, int K);
+
+/* Newton forward: K >= 1 iterations from the warm start, output H = h^(K).
+ * (Method section; NewtonConfig(max_iters=K), API overview section.)
+ *   preacts    (B,T,G,D) in px_dtype, read only
+ *   diag_w     (G,D) f32 or NULL (zeros)
+ *   h0         (B,S,D) f32 or NULL (zeros)
+ *   K          1..64 Newton iterations; the linear cell is exact after one,
+ *              and performs exactly one scan for any K
+ *   H_out      (B,T,S,D) f32, written
+ *   workspace  >= pararnn_workspace_bytes(cell,B,T,D,K) bytes, 256-byte aligned
+ *   resid_hist NULL, or K+1 floats of device memory that receive
+ *              max_{b,t,s,d} |F(H^(k))| for k = 0..K (the residual history a
+ *              NewtonDivergenceError carries, Evaluation section)
+ * B, T or D equal to 0 is an empty problem: nothing is launched except the
+ * zeroing of resid_hist. */
+pararnn_status pararnn_newton_forward(pararnn_cell cell, int64_t B, int64_t T, int64_t D,
+                                      pararnn_dtype px_dtype, const void* preacts, const float* diag_w,
+                                      const float* h0, int K, float* H_out, void* workspace,
+                                      size_t ws_bytes, float* resid_hist, void* stream);
+
+/* Adjoint (backward) at the trajectory H (normally the forward's output):
+ *   lambda_t = dL/dH_t + A_{t+1}^T lambda_{t+1},  lambda_{T-1} = dL/dH_{T-1},
+ * with A_{t+1} = df/dh at (h_t, x_{t+1}), a reverse-time scan under the same
+ * operator (Method section: "Backward follows paper eq. 2.6"; the ParaRNN
+ * thread's "custom parallel reductions").  Then
+ *   dL_dpx[b,t,g,d] = lambda_t . df/dp_g at (h_{t-1}, x_t)
+ *   dL_da[g,d]      = sum_{b,t} lambda_t . df/da_g at (h_{t-1}, x_t)
+ *   dL_dh0[b,:,d]   = A_0^T lambda_0
+ * dL_da is reduced in a fixed order without floating-point atomics
+ * (Compatibility section: the packed VJP is deterministic).
+ *   dL_dpx  (B,T,G,D) f32, written (required)
+ *   dL_da   (G,D) f32 or NULL; not written for the linear cell (no weights)
+ *   dL_dh0  (B,S,D) f32 or NULL */
+pararnn_status pararnn_newton_backward(pararnn_cell cell, int64_t B, int64_t T, int64_t D,
+                                       pararnn_dtype px_dtype, const void* preacts, const float* diag_w,
+                                       const float* h0, const float* H, const float* dL_dH, float* dL_dpx,
+                                       float* dL_da, float* dL_dh0, void* workspace, size_t ws_bytes,
+                                       void* stream);
+
+/* Waits for `stream` and returns what the GPU recorded for the last forward
+ * or backward call that used `workspace`: PARARNN_OK, PARARNN_ENONFINITE or
+ * PARARNN_ETIMEOUT (ETIMEOUT wins if both happened); PARARNN_ECUDA if the copy
+ * or the synchronisation fails. */
+pararnn_status pararnn_status_sync(const void* workspace, void* stream);
+
+/* Static, NUL-terminated name of a status code ("PARARNN_OK", ...). */
+const char* pararnn_status_string(pararnn_status status);
+
+/* Static, NUL-terminated description of the last EINVAL or ECUDA returned on
+ * the calling thread ("" if none). */
+const char* pararnn_last_error(void);
+
+/* Runs the library's bounded inter-block wait on a flag that nothing sets,
+ * with a limit of timeout_ns nanoseconds, so that a test can see the time-out
+ * path end cleanly: the kernel records PARARNN_ETIMEOUT in the workspace and
+ * returns; pararnn_status_sync() then reports it.  workspace needs at least
+ * pararnn_workspace_bytes(PARARNN_CELL_LINEAR, 1, 1, 1, 1) bytes. */
+pararnn_status pararnn_probe_wait_timeout(void* workspace, size_t ws_bytes, uint64_t timeout_ns, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PARARNN_B200_H */

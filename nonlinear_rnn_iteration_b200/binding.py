@@ -1,0 +1,202 @@
+"""ctypes binding of libpararnn_b200 -- argument marshalling only.
+
+The ``pararnn_*`` functions here have the names and argument order of the C
+ABI in ``include/pararnn_b200.h``; pointer arguments accept a torch tensor
+(its ``data_ptr()``), an int address, or None (NULL).  ``stream`` accepts a
+``torch.cuda.Stream``, an int handle or None (the legacy default stream).
+
+Above them, :func:`newton_forward` and :func:`newton_backward` allocate the
+outputs and the workspace with torch (device memory is torch's job here) and
+raise :class:`PararnnError` on a non-OK status.  Every step of the
+computation runs in the library's CUDA kernels; nothing here computes.  If
+the library cannot be loaded, this module raises: there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+from . import build as _build
+
+LINEAR, DIAG_GRU, DIAG_LSTM = 0, 1, 2
+F32, BF16 = 0, 1
+CELLS = {"linear": LINEAR, "diag_gru": DIAG_GRU, "diag_lstm": DIAG_LSTM}
+STATUS = {0: "PARARNN_OK", 1: "PARARNN_EINVAL", 2: "PARARNN_ENONFINITE", 3: "PARARNN_ETIMEOUT", 4: "PARARNN_ECUDA"}
+OK, EINVAL, ENONFINITE, ETIMEOUT, ECUDA = 0, 1, 2, 3, 4
+
+# every exported symbol of include/pararnn_b200.h, with its C signature
+_P, _I64, _I, _SZ, _U64 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t, ctypes.c_uint64
+SIGNATURES = {
+    "pararnn_num_gates": (_I, [_I]),
+    "pararnn_state_width": (_I, [_I]),
+    "pararnn_workspace_bytes": (_SZ, [_I, _I64, _I64, _I64, _I]),
+    "pararnn_newton_forward": (_I, [_I, _I64, _I64, _I64, _I, _P, _P, _P, _I, _P, _P, _SZ, _P, _P]),
+    "pararnn_newton_backward": (_I, [_I, _I64, _I64, _I64, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "pararnn_status_sync": (_I, [_P, _P]),
+    "pararnn_status_string": (ctypes.c_char_p, [_I]),
+    "pararnn_last_error": (ctypes.c_char_p, []),
+    "pararnn_probe_wait_timeout": (_I, [_P, _SZ, _U64, _P]),
+}
+
+_lib = None
+
+
+class PararnnError(RuntimeError):
+    def __init__(self, status: int, where: str, detail: str = ""):
+        self.status = status
+        msg = "%s returned %s" % (where, STATUS.get(status, status))
+        if detail:
+            msg += ": " + detail
+        super().__init__(msg)
+
+
+def load(path: str | None = None):
+    """Load (building first if missing or stale) the in-tree library."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    so = path or _build.build()
+    if not os.path.exists(so):
+        raise RuntimeError("libpararnn_b200.so not found at %s" % so)
+    lib = ctypes.CDLL(so)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def _ptr(x):
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(s):
+    if s is None:
+        return None
+    if isinstance(s, int):
+        return s
+    return s.cuda_stream
+
+
+# ---- the C ABI, one to one -------------------------------------------------
+
+def pararnn_num_gates(cell):
+    return load().pararnn_num_gates(cell)
+
+
+def pararnn_state_width(cell):
+    return load().pararnn_state_width(cell)
+
+
+def pararnn_workspace_bytes(cell, B, T, D, K):
+    return load().pararnn_workspace_bytes(cell, B, T, D, K)
+
+
+def pararnn_newton_forward(cell, B, T, D, px_dtype, preacts, diag_w, h0, K, H_out, workspace, ws_bytes,
+                           resid_hist, stream):
+    return load().pararnn_newton_forward(cell, B, T, D, px_dtype, _ptr(preacts), _ptr(diag_w), _ptr(h0), K,
+                                         _ptr(H_out), _ptr(workspace), ws_bytes, _ptr(resid_hist), _stream(stream))
+
+
+def pararnn_newton_backward(cell, B, T, D, px_dtype, preacts, diag_w, h0, H, dL_dH, dL_dpx, dL_da, dL_dh0,
+                            workspace, ws_bytes, stream):
+    return load().pararnn_newton_backward(cell, B, T, D, px_dtype, _ptr(preacts), _ptr(diag_w), _ptr(h0), _ptr(H),
+                                          _ptr(dL_dH), _ptr(dL_dpx), _ptr(dL_da), _ptr(dL_dh0), _ptr(workspace),
+                                          ws_bytes, _stream(stream))
+
+
+def pararnn_status_sync(workspace, stream):
+    return load().pararnn_status_sync(_ptr(workspace), _stream(stream))
+
+
+def pararnn_status_string(status):
+    return load().pararnn_status_string(status).decode()
+
+
+def pararnn_last_error():
+    return load().pararnn_last_error().decode()
+
+
+def pararnn_probe_wait_timeout(workspace, ws_bytes, timeout_ns, stream):
+    return load().pararnn_probe_wait_timeout(_ptr(workspace), ws_bytes, timeout_ns, _stream(stream))
+
+
+# ---- tensor-level helpers (allocation through torch, compute in the library) ----
+
+def _check(status, where):
+    if status != OK:
+        raise PararnnError(status, where, pararnn_last_error())
+
+
+def _dtype_code(t):
+    import torch
+
+    if t.dtype == torch.float32:
+        return F32
+    if t.dtype == torch.bfloat16:
+        return BF16
+    raise TypeError("pre-activations must be float32 or bfloat16, got %s" % t.dtype)
+
+
+def _shape(cell, px):
+    G = pararnn_num_gates(cell)
+    if px.dim() != 4 or px.shape[2] != G:
+        raise ValueError("preacts must be (B, T, %d, D), got %s" % (G, tuple(px.shape)))
+    if not px.is_contiguous():
+        raise ValueError("preacts must be contiguous")
+    B, T, _, D = px.shape
+    return B, T, D
+
+
+def workspace_for(cell, B, T, D, K, device):
+    import torch
+
+    n = pararnn_workspace_bytes(cell, B, T, D, K)
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def newton_forward(cell, px, diag_w=None, h0=None, K=1, out=None, workspace=None, resid_hist=None, stream=None,
+                   sync_status=True):
+    """H = h^(K) of shape (B,T,S,D), float32, on px's device."""
+    import torch
+
+    cell = CELLS.get(cell, cell)
+    B, T, D = _shape(cell, px)
+    S = pararnn_state_width(cell)
+    if out is None:
+        out = torch.empty((B, T, S, D), dtype=torch.float32, device=px.device)
+    if workspace is None:
+        workspace = workspace_for(cell, B, T, D, K, px.device)
+    st = stream if stream is not None else torch.cuda.current_stream(px.device)
+    _check(pararnn_newton_forward(cell, B, T, D, _dtype_code(px), px, diag_w, h0, K, out, workspace,
+                                  workspace.numel(), resid_hist, st), "pararnn_newton_forward")
+    if sync_status:
+        _check(pararnn_status_sync(workspace, st), "pararnn_newton_forward (device status)")
+    return out
+
+
+def newton_backward(cell, px, H, dL_dH, diag_w=None, h0=None, workspace=None, want_da=True, want_dh0=False,
+                    stream=None, sync_status=True):
+    """Returns (dL_dpx (B,T,G,D), dL_da (G,D) or None, dL_dh0 (B,S,D) or None), float32."""
+    import torch
+
+    cell = CELLS.get(cell, cell)
+    B, T, D = _shape(cell, px)
+    G, S = pararnn_num_gates(cell), pararnn_state_width(cell)
+    dpx = torch.empty((B, T, G, D), dtype=torch.float32, device=px.device)
+    da = torch.empty((G, D), dtype=torch.float32, device=px.device) if (want_da and cell != LINEAR) else None
+    dh0 = torch.empty((B, S, D), dtype=torch.float32, device=px.device) if want_dh0 else None
+    if workspace is None:
+        workspace = workspace_for(cell, B, T, D, 1, px.device)
+    st = stream if stream is not None else torch.cuda.current_stream(px.device)
+    _check(pararnn_newton_backward(cell, B, T, D, _dtype_code(px), px, diag_w, h0, H, dL_dH, dpx, da, dh0,
+                                   workspace, workspace.numel(), st), "pararnn_newton_backward")
+    if sync_status:
+        _check(pararnn_status_sync(workspace, st), "pararnn_newton_backward (device status)")
+    return dpx, da, dh0

@@ -1,0 +1,238 @@
+// cells.cuh -- the three diagonal cells, one channel at a time, in float32.
+//
+// Each cell provides
+//   warm(p, w, f)                  f = f(0, x): the Newton warm start
+//                                  (pararnn-torch PyPI page, Method section,
+//                                  "h^(0) = f(0, x)")
+//   elem(p, w, sp, f, A, beta)     f = f(sp, x), A = df/dsp (S x S, row-major),
+//                                  beta = f - A sp: the scan element of the
+//                                  direct-form Newton update
+//                                  h_t = A_t h_{t-1} + beta_t
+//   bwd(p, w, sp, A, sens)         A and the sensitivities the adjoint needs
+//   grads(sens, lam, dp, da)       dL/dp_g and dL/da_g of one row given
+//                                  lambda_t (the adjoint state)
+// Cell equations: diagonal GRU (gates z, r, c) and diagonal LSTM (gates i, f,
+// o, c; forget bias +1; state (c, h)) as listed for ParaGRU / ParaLSTM on the
+// pararnn-torch page; the linear cell h' = a h + b is the affine recurrence
+// the News section calls an exact parallel scan.
+#pragma once
+
+#include "common.cuh"
+
+namespace pararnn {
+
+struct CellLinear {
+    static constexpr int G = 2, S = 1, NSENS = 1;
+    static constexpr bool kNonlinear = false;  // one scan is exact
+
+    static __device__ __forceinline__ void warm(const float (&p)[G], const float (&)[G], float (&f)[S]) {
+        f[0] = p[1];
+    }
+    static __device__ __forceinline__ void elem(const float (&p)[G], const float (&)[G], const float (&sp)[S],
+                                                float (&f)[S], float (&A)[S * S], float (&beta)[S]) {
+        A[0] = p[0];
+        beta[0] = p[1];
+        f[0] = __fmaf_rn(p[0], sp[0], p[1]);
+    }
+    static __device__ __forceinline__ void bwd(const float (&p)[G], const float (&)[G], const float (&sp)[S],
+                                               float (&A)[S * S], float (&sens)[NSENS]) {
+        A[0] = p[0];
+        sens[0] = sp[0];
+    }
+    static __device__ __forceinline__ void grads(const float (&sens)[NSENS], const float (&lam)[S], float (&dp)[G],
+                                                 float (&da)[G]) {
+        dp[0] = lam[0] * sens[0];
+        dp[1] = lam[0];
+        da[0] = 0.0f;
+        da[1] = 0.0f;
+    }
+};
+
+struct CellGRU {
+    static constexpr int G = 3, S = 1, NSENS = 5;
+    static constexpr bool kNonlinear = true;
+
+    static __device__ __forceinline__ void warm(const float (&p)[G], const float (&)[G], float (&f)[S]) {
+        // h = 0: z = sig(p_z), c = tanh(p_c), f = z c
+        f[0] = sigmoid_f(p[0]) * tanh_f(p[2]);
+    }
+    // z, r, c and the chain-rule factors G_z = df/dp_z, G_r = df/dp_r, G_c = df/dp_c
+    static __device__ __forceinline__ void gates(const float (&p)[G], const float (&w)[G], float h, float& z,
+                                                 float& r, float& c, float& Gz, float& Gr, float& Gc) {
+        z = sigmoid_f(__fmaf_rn(w[0], h, p[0]));
+        r = sigmoid_f(__fmaf_rn(w[1], h, p[1]));
+        c = tanh_f(__fmaf_rn(w[2] * r, h, p[2]));
+        Gz = (c - h) * (z - z * z);
+        Gc = z * __fmaf_rn(-c, c, 1.0f);
+        Gr = Gc * w[2] * h * (r - r * r);
+    }
+    static __device__ __forceinline__ void elem(const float (&p)[G], const float (&w)[G], const float (&sp)[S],
+                                                float (&f)[S], float (&A)[S * S], float (&beta)[S]) {
+        const float h = sp[0];
+        float z, r, c, Gz, Gr, Gc;
+        gates(p, w, h, z, r, c, Gz, Gr, Gc);
+        f[0] = __fmaf_rn(z, c - h, h);  // (1 - z) h + z c
+        // df/dh: the direct (1 - z) plus each gate's pre-activation term
+        float a = 1.0f - z;
+        a = __fmaf_rn(w[0], Gz, a);
+        a = __fmaf_rn(w[1], Gr, a);
+        a = __fmaf_rn(w[2] * r, Gc, a);
+        A[0] = a;
+        beta[0] = __fmaf_rn(-a, h, f[0]);
+    }
+    static __device__ __forceinline__ void bwd(const float (&p)[G], const float (&w)[G], const float (&sp)[S],
+                                               float (&A)[S * S], float (&sens)[NSENS]) {
+        const float h = sp[0];
+        float z, r, c, Gz, Gr, Gc;
+        gates(p, w, h, z, r, c, Gz, Gr, Gc);
+        float a = 1.0f - z;
+        a = __fmaf_rn(w[0], Gz, a);
+        a = __fmaf_rn(w[1], Gr, a);
+        a = __fmaf_rn(w[2] * r, Gc, a);
+        A[0] = a;
+        sens[0] = Gz;
+        sens[1] = Gr;
+        sens[2] = Gc;
+        sens[3] = r * h;
+        sens[4] = h;
+    }
+    static __device__ __forceinline__ void grads(const float (&sens)[NSENS], const float (&lam)[S], float (&dp)[G],
+                                                 float (&da)[G]) {
+        dp[0] = lam[0] * sens[0];
+        dp[1] = lam[0] * sens[1];
+        dp[2] = lam[0] * sens[2];
+        da[0] = dp[0] * sens[4];
+        da[1] = dp[1] * sens[4];
+        da[2] = dp[2] * sens[3];
+    }
+};
+
+struct CellLSTM {
+    static constexpr int G = 4, S = 2, NSENS = 6;
+    static constexpr bool kNonlinear = true;
+
+    static __device__ __forceinline__ void warm(const float (&p)[G], const float (&)[G], float (&f)[S]) {
+        // (c, h) = 0: c' = i g, h' = o tanh(c')
+        const float i = sigmoid_f(p[0]);
+        const float o = sigmoid_f(p[2]);
+        const float g = tanh_f(p[3]);
+        const float cn = i * g;
+        f[0] = cn;
+        f[1] = o * tanh_f(cn);
+    }
+    struct Terms {
+        float i, fg, o, g, cn, tn, dcn_dh;
+    };
+    static __device__ __forceinline__ Terms terms(const float (&p)[G], const float (&w)[G], float c, float h) {
+        Terms q;
+        q.i = sigmoid_f(__fmaf_rn(w[0], h, p[0]));
+        q.fg = sigmoid_f(__fmaf_rn(w[1], h, p[1]) + 1.0f);
+        q.o = sigmoid_f(__fmaf_rn(w[2], h, p[2]));
+        q.g = tanh_f(__fmaf_rn(w[3], h, p[3]));
+        q.cn = __fmaf_rn(q.fg, c, q.i * q.g);
+        q.tn = tanh_f(q.cn);
+        // dc'/dh through the f, i and c gates' pre-activations
+        float d = c * (q.fg - q.fg * q.fg) * w[1];
+        d = __fmaf_rn(q.g * (q.i - q.i * q.i), w[0], d);
+        d = __fmaf_rn(q.i * __fmaf_rn(-q.g, q.g, 1.0f), w[3], d);
+        q.dcn_dh = d;
+        return q;
+    }
+    static __device__ __forceinline__ void elem(const float (&p)[G], const float (&w)[G], const float (&sp)[S],
+                                                float (&f)[S], float (&A)[S * S], float (&beta)[S]) {
+        const float c = sp[0], h = sp[1];
+        const Terms q = terms(p, w, c, h);
+        const float k = q.o * __fmaf_rn(-q.tn, q.tn, 1.0f);  // dh'/dc'
+        f[0] = q.cn;
+        f[1] = q.o * q.tn;
+        A[0] = q.fg;                                            // dc'/dc
+        A[1] = q.dcn_dh;                                        // dc'/dh
+        A[2] = k * q.fg;                                        // dh'/dc
+        A[3] = __fmaf_rn((q.o - q.o * q.o) * w[2], q.tn, k * q.dcn_dh);  // dh'/dh
+        beta[0] = f[0] - __fmaf_rn(A[0], c, A[1] * h);
+        beta[1] = f[1] - __fmaf_rn(A[2], c, A[3] * h);
+    }
+    static __device__ __forceinline__ void bwd(const float (&p)[G], const float (&w)[G], const float (&sp)[S],
+                                               float (&A)[S * S], float (&sens)[NSENS]) {
+        const float c = sp[0], h = sp[1];
+        const Terms q = terms(p, w, c, h);
+        const float k = q.o * __fmaf_rn(-q.tn, q.tn, 1.0f);
+        const float dho = (q.o - q.o * q.o) * q.tn;
+        A[0] = q.fg;
+        A[1] = q.dcn_dh;
+        A[2] = k * q.fg;
+        A[3] = __fmaf_rn(dho, w[2], k * q.dcn_dh);
+        sens[0] = q.g * (q.i - q.i * q.i);               // dc'/dp_i
+        sens[1] = c * (q.fg - q.fg * q.fg);              // dc'/dp_f
+        sens[2] = q.i * __fmaf_rn(-q.g, q.g, 1.0f);      // dc'/dp_c
+        sens[3] = k;                                     // dh'/dc'
+        sens[4] = dho;                                   // dh'/dp_o
+        sens[5] = h;
+    }
+    static __device__ __forceinline__ void grads(const float (&sens)[NSENS], const float (&lam)[S], float (&dp)[G],
+                                                 float (&da)[G]) {
+        // lambda . df/dp_g with h' depending on p_i, p_f, p_c only through c'
+        const float m = __fmaf_rn(lam[1], sens[3], lam[0]);
+        dp[0] = m * sens[0];
+        dp[1] = m * sens[1];
+        dp[2] = lam[1] * sens[4];
+        dp[3] = m * sens[2];
+#pragma unroll
+        for (int g = 0; g < G; ++g) da[g] = dp[g] * sens[5];
+    }
+};
+
+// ---- scan element algebra (S = 1 scalar, S = 2 2x2 block) -----------------
+// element e = (A, b) acts on a state x as e(x) = A x + b; composition
+// (A2, b2) o (A1, b1) = (A2 A1, A2 b1 + b2) applies e1 first.  Every
+// application goes through apply(), so the same product is rounded the same
+// way wherever it is formed.
+
+template <int S>
+struct Elem {
+    float A[S * S];
+    float b[S];
+};
+
+template <int S>
+__device__ __forceinline__ void elem_identity(Elem<S>& e) {
+#pragma unroll
+    for (int i = 0; i < S * S; ++i) e.A[i] = (i % (S + 1) == 0) ? 1.0f : 0.0f;
+#pragma unroll
+    for (int i = 0; i < S; ++i) e.b[i] = 0.0f;
+}
+
+// y = A x + b
+template <int S>
+__device__ __forceinline__ void apply(const float (&A)[S * S], const float (&b)[S], const float (&x)[S],
+                                      float (&y)[S]) {
+    if constexpr (S == 1) {
+        y[0] = __fmaf_rn(A[0], x[0], b[0]);
+    } else {
+        y[0] = __fmaf_rn(A[0], x[0], __fmaf_rn(A[1], x[1], b[0]));
+        y[1] = __fmaf_rn(A[2], x[0], __fmaf_rn(A[3], x[1], b[1]));
+    }
+}
+
+// acc <- e o acc  (e applied after acc)
+template <int S>
+__device__ __forceinline__ void compose_after(const float (&A)[S * S], const float (&b)[S], Elem<S>& acc) {
+    if constexpr (S == 1) {
+        acc.b[0] = __fmaf_rn(A[0], acc.b[0], b[0]);
+        acc.A[0] = A[0] * acc.A[0];
+    } else {
+        float nb[2];
+        apply<2>(A, b, acc.b, nb);
+        float nA[4];
+        nA[0] = __fmaf_rn(A[0], acc.A[0], A[1] * acc.A[2]);
+        nA[1] = __fmaf_rn(A[0], acc.A[1], A[1] * acc.A[3]);
+        nA[2] = __fmaf_rn(A[2], acc.A[0], A[3] * acc.A[2]);
+        nA[3] = __fmaf_rn(A[2], acc.A[1], A[3] * acc.A[3]);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc.A[i] = nA[i];
+        acc.b[0] = nb[0];
+        acc.b[1] = nb[1];
+    }
+}
+
+}  // namespace pararnn

@@ -1,0 +1,133 @@
+// common.cuh -- device helpers shared by the forward and backward kernels:
+// vectorised row loads/stores, the release/acquire flag protocol used by the
+// decoupled look-back between thread blocks, and the bounded wait.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace pararnn {
+
+// ---- workspace header (first 256 bytes of every workspace) -------------
+// word 0: status bits, word 1: tile ticket counter.  The rest is padding.
+constexpr unsigned kStatusNonFinite = 1u;
+constexpr unsigned kStatusTimeout = 2u;
+constexpr size_t kHeaderBytes = 256;
+
+// look-back flag values (one 32-bit flag per tile and Newton iteration)
+constexpr unsigned kFlagEmpty = 0u;
+constexpr unsigned kFlagAggregate = 1u;   // the tile's own composed element is published
+constexpr unsigned kFlagInclusive = 2u;   // the state after the tile's last row is published
+
+// ---- element loads -------------------------------------------------------
+
+template <typename T>
+struct PxTraits;
+
+template <>
+struct PxTraits<float> {
+    static __device__ __forceinline__ float cvt(float x) { return x; }
+};
+template <>
+struct PxTraits<__nv_bfloat16> {
+    static __device__ __forceinline__ float cvt(__nv_bfloat16 x) { return __bfloat162float(x); }
+};
+
+// Load V consecutive values starting at p (p is V-element aligned when V > 1).
+// Streaming data: read once, so the load asks L1 not to keep the line.
+template <int V>
+__device__ __forceinline__ void load_row(const float* p, float (&out)[V]) {
+    if constexpr (V == 4) {
+        float4 v;
+        asm volatile("ld.global.nc.L1::no_allocate.v4.f32 {%0,%1,%2,%3}, [%4];"
+                     : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                     : "l"(p));
+        out[0] = v.x; out[1] = v.y; out[2] = v.z; out[3] = v.w;
+    } else if constexpr (V == 2) {
+        float2 v;
+        asm volatile("ld.global.nc.L1::no_allocate.v2.f32 {%0,%1}, [%2];" : "=f"(v.x), "=f"(v.y) : "l"(p));
+        out[0] = v.x; out[1] = v.y;
+    } else {
+#pragma unroll
+        for (int i = 0; i < V; ++i) out[i] = __ldg(p + i);
+    }
+}
+
+template <int V>
+__device__ __forceinline__ void load_row(const __nv_bfloat16* p, float (&out)[V]) {
+    if constexpr (V == 4) {
+        uint2 v;
+        asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
+        out[0] = __uint_as_float(v.x << 16);
+        out[1] = __uint_as_float(v.x & 0xffff0000u);
+        out[2] = __uint_as_float(v.y << 16);
+        out[3] = __uint_as_float(v.y & 0xffff0000u);
+    } else if constexpr (V == 2) {
+        unsigned v;
+        asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
+        out[0] = __uint_as_float(v << 16);
+        out[1] = __uint_as_float(v & 0xffff0000u);
+    } else {
+#pragma unroll
+        for (int i = 0; i < V; ++i) out[i] = __bfloat162float(p[i]);
+    }
+}
+
+template <int V>
+__device__ __forceinline__ void store_row(float* p, const float (&v)[V]) {
+    if constexpr (V == 4) {
+        *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+    } else if constexpr (V == 2) {
+        *reinterpret_cast<float2*>(p) = make_float2(v[0], v[1]);
+    } else {
+#pragma unroll
+        for (int i = 0; i < V; ++i) p[i] = v[i];
+    }
+}
+
+// ---- inter-block protocol ------------------------------------------------
+// A tile publishes a payload (plain stores by several lanes of one warp),
+// every writing lane fences, the warp synchronises, and one lane stores the
+// flag with release semantics at GPU scope.  A reader loads the flag with
+// acquire semantics, synchronises its warp, and loads the payload with
+// relaxed GPU-scope loads, which are served by L2 and never by a stale L1
+// line.
+
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void st_release_gpu(unsigned* p, unsigned v) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ float ld_relaxed_gpu(const float* p) {
+    float v;
+    asm volatile("ld.relaxed.gpu.global.f32 %0, [%1];" : "=f"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// ---- numerics --------------------------------------------------------------
+
+__device__ __forceinline__ float sigmoid_f(float x) { return __fdividef(1.0f, 1.0f + __expf(-x)); }
+__device__ __forceinline__ float tanh_f(float x) { return tanhf(x); }
+
+// max that keeps a NaN (so a non-finite residual is reported, not hidden)
+__device__ __forceinline__ float nanmax_f(float a, float b) { return (a != a || a > b) ? a : b; }
+
+// Non-negative floats order like their bit patterns, and a NaN's bits sort
+// above +Inf, so an integer atomicMax on the bits is a deterministic max.
+__device__ __forceinline__ void atomic_max_nonneg(float* addr, float v) {
+    atomicMax(reinterpret_cast<unsigned*>(addr), __float_as_uint(fabsf(v)) & 0x7fffffffu);
+}
+
+}  // namespace pararnn

@@ -1,0 +1,206 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle.
+
+Tolerances (relative error with a 1e-2*max floor, see gpu_util.rel_err):
+  H from f32 pre-activations             <= 1e-4
+  gradients (dL/dpx, dL/da, dL/dh0)      <= 1e-3
+  H from bf16 pre-activations vs the oracle on the same bf16 values
+                                         <= 1e-4
+  H from bf16 pre-activations vs the oracle on the unrounded f32 draws
+                                         <= 2e-2 normwise (gpu_util.norm_err):
+    the rounding of the inputs themselves moves outputs near zero by more
+    than 2e-2 of their own size, for any solver
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_util import gather_channels, norm_err, rel_err, to_np
+from nonlinear_rnn_iteration_b200 import binding, workloads
+
+pytestmark = pytest.mark.gpu
+
+TOL_H, TOL_G, TOL_BF16_F32 = 1e-4, 1e-3, 2e-2
+DEV = "cuda:0"
+
+
+def _inputs(cell, B, T, D, seed, h0=False, bf16=False, grad=False):
+    rng = np.random.default_rng(seed)
+    G, S = oracle.NUM_GATES[cell], oracle.STATE_WIDTH[cell]
+    px = rng.standard_normal((B, T, G, D)).astype(np.float32)
+    if cell == oracle.LINEAR:
+        px[:, :, 0, :] = 1.0 / (1.0 + np.exp(-px[:, :, 0, :]))
+        w = None
+    else:
+        w = rng.uniform(-0.5, 0.5, (G, D)).astype(np.float32)
+    hz = (0.5 * rng.standard_normal((B, S, D))).astype(np.float32) if h0 else None
+    g = rng.standard_normal((B, T, S, D)).astype(np.float32) if grad else None
+    px_used = workloads.round_bf16(px) if bf16 else px
+    t = lambda a: None if a is None else torch.from_numpy(np.ascontiguousarray(a)).to(DEV)
+    pxt = t(px).to(torch.bfloat16) if bf16 else t(px)
+    return dict(px=px, px_used=px_used, w=w, h0=hz, g=g, pxt=pxt, wt=t(w), h0t=t(hz), gt=t(g))
+
+
+# (cell, B, T, D, K): several tiles along T and D, ragged tails, vector (D % 4 == 0)
+# and element-wise (odd D) paths
+SMALL = [
+    (oracle.LINEAR, 2, 300, 136, 1),
+    (oracle.LINEAR, 1, 97, 37, 1),
+    (oracle.DIAG_GRU, 2, 200, 100, 3),
+    (oracle.DIAG_GRU, 1, 131, 37, 2),
+    (oracle.DIAG_GRU, 1, 1024, 64, 3),
+    (oracle.DIAG_LSTM, 2, 150, 72, 4),
+    (oracle.DIAG_LSTM, 1, 77, 13, 3),
+]
+
+
+@pytest.mark.parametrize("case", SMALL, ids=lambda c: "cell%d_B%dT%dD%dK%d" % c)
+@pytest.mark.parametrize("h0", [False, True])
+def test_forward_small(case, h0, cuda_device):
+    cell, B, T, D, K = case
+    x = _inputs(cell, B, T, D, seed=T * 7 + D, h0=h0)
+    resid = torch.zeros(K + 1, device=DEV)
+    H = binding.newton_forward(cell, x["pxt"], x["wt"], x["h0t"], K=K, resid_hist=resid)
+    Ho, ro = oracle.newton(cell, x["px"], x["w"], x["h0"], K=K)
+    assert rel_err(to_np(H), Ho) <= TOL_H
+    # residual history: f32 residuals agree with the fp64 ones up to rounding-level noise
+    r = to_np(resid)
+    assert np.all(np.abs(r - ro) <= 1e-4 * max(1.0, ro[0]) + 1e-5 * ro), (r, ro)
+
+
+@pytest.mark.parametrize("cell", [oracle.DIAG_GRU, oracle.DIAG_LSTM])
+def test_forward_bf16_small(cell, cuda_device):
+    B, T, D, K = 2, 180, 68, 3
+    x = _inputs(cell, B, T, D, seed=5, bf16=True)
+    H = to_np(binding.newton_forward(cell, x["pxt"], x["wt"], None, K=K))
+    Hb, _ = oracle.newton(cell, x["px_used"], x["w"], None, K=K)
+    Hf, _ = oracle.newton(cell, x["px"], x["w"], None, K=K)
+    assert rel_err(H, Hb) <= TOL_H
+    assert norm_err(H, Hf) <= TOL_BF16_F32
+
+
+@pytest.mark.parametrize("case", [(oracle.LINEAR, 2, 150, 68), (oracle.LINEAR, 1, 61, 5),
+                                  (oracle.DIAG_GRU, 2, 200, 100), (oracle.DIAG_GRU, 1, 97, 37),
+                                  (oracle.DIAG_LSTM, 2, 120, 72), (oracle.DIAG_LSTM, 1, 45, 9)],
+                         ids=lambda c: "cell%d_B%dT%dD%d" % c)
+@pytest.mark.parametrize("bf16", [False, True])
+def test_backward_small(case, bf16, cuda_device):
+    cell, B, T, D = case
+    K = 3
+    x = _inputs(cell, B, T, D, seed=B + T + D, h0=True, bf16=bf16, grad=True)
+    H = binding.newton_forward(cell, x["pxt"], x["wt"], x["h0t"], K=K)
+    dpx, da, dh0 = binding.newton_backward(cell, x["pxt"], H, x["gt"], x["wt"], x["h0t"], want_dh0=True)
+    Ho, _ = oracle.newton(cell, x["px_used"], x["w"], x["h0"], K=K)
+    dpxo, dao, dh0o = oracle.adjoint(cell, x["px_used"], x["w"], x["h0"], Ho, x["g"])
+    assert rel_err(to_np(dpx), dpxo) <= TOL_G
+    assert rel_err(to_np(dh0), dh0o) <= TOL_G
+    if cell != oracle.LINEAR:
+        assert rel_err(to_np(da), dao) <= TOL_G
+    else:
+        assert da is None
+
+
+def test_linear_any_k_is_one_scan(cuda_device):
+    x = _inputs(oracle.LINEAR, 1, 100, 64, seed=3)
+    r1 = torch.zeros(2, device=DEV)
+    r4 = torch.zeros(5, device=DEV)
+    H1 = binding.newton_forward(oracle.LINEAR, x["pxt"], None, None, K=1, resid_hist=r1)
+    H4 = binding.newton_forward(oracle.LINEAR, x["pxt"], None, None, K=4, resid_hist=r4)
+    assert torch.equal(H1, H4)
+    assert np.all(to_np(r4)[1:] == to_np(r1)[1])
+
+
+def test_newton_reaches_unroll(cuda_device):
+    # prefix exactness: K = T Newton steps reproduce the sequential unroll
+    for cell in (oracle.DIAG_GRU, oracle.DIAG_LSTM):
+        x = _inputs(cell, 1, 12, 8, seed=11)
+        H = binding.newton_forward(cell, x["pxt"], x["wt"], None, K=12)
+        U = oracle.unroll(cell, x["px"], x["w"], None)
+        assert rel_err(to_np(H), U) <= TOL_H
+
+
+def test_edge_shapes(cuda_device):
+    # T = 1, D = 1, B = 1, and a T that is one past a tile boundary
+    for cell in (oracle.LINEAR, oracle.DIAG_GRU, oracle.DIAG_LSTM):
+        for (B, T, D) in [(1, 1, 1), (3, 1, 5), (1, 65, 1), (2, 33, 4), (1, 129, 64)]:
+            x = _inputs(cell, B, T, D, seed=B * 100 + T + D, h0=True, grad=True)
+            K = 2
+            H = binding.newton_forward(cell, x["pxt"], x["wt"], x["h0t"], K=K)
+            Ho, _ = oracle.newton(cell, x["px"], x["w"], x["h0"], K=K)
+            assert rel_err(to_np(H), Ho) <= TOL_H, (cell, B, T, D)
+            dpx, da, dh0 = binding.newton_backward(cell, x["pxt"], H, x["gt"], x["wt"], x["h0t"], want_dh0=True)
+            dpxo, dao, dh0o = oracle.adjoint(cell, x["px"], x["w"], x["h0"], Ho, x["g"])
+            assert rel_err(to_np(dpx), dpxo) <= TOL_G, (cell, B, T, D)
+            assert rel_err(to_np(dh0), dh0o) <= TOL_G, (cell, B, T, D)
+            if da is not None:
+                assert rel_err(to_np(da), dao) <= TOL_G, (cell, B, T, D)
+
+
+def test_empty_problems(cuda_device):
+    for (B, T, D) in [(0, 5, 8), (2, 0, 8), (2, 5, 0)]:
+        px = torch.empty((B, T, 3, D), device=DEV)
+        resid = torch.full((4,), 7.0, device=DEV)
+        H = binding.newton_forward(oracle.DIAG_GRU, px, None, None, K=3, resid_hist=resid)
+        assert H.shape == (B, T, 1, D)
+        assert torch.all(resid == 0)
+        g = torch.empty((B, T, 1, D), device=DEV)
+        dpx, da, dh0 = binding.newton_backward(oracle.DIAG_GRU, px, H, g, want_dh0=True)
+        assert dpx.shape == (B, T, 3, D)
+        assert torch.all(da == 0) and torch.all(dh0 == 0)
+
+
+def test_deterministic(cuda_device):
+    # the same inputs give the same bits, run after run
+    for cell in (oracle.DIAG_GRU, oracle.DIAG_LSTM):
+        x = _inputs(cell, 4, 2048, 256, seed=9, grad=True)
+        outs = []
+        for _ in range(3):
+            H = binding.newton_forward(cell, x["pxt"], x["wt"], None, K=3)
+            dpx, da, _ = binding.newton_backward(cell, x["pxt"], H, x["gt"], x["wt"])
+            outs.append((H.clone(), dpx.clone(), da.clone()))
+        for o in outs[1:]:
+            for a, b in zip(o, outs[0]):
+                assert torch.equal(a, b)
+
+
+# ---- full-size workloads, checked on a seeded sample of channels ----------
+
+@pytest.mark.parametrize("name", [n for n in workloads.WORKLOADS])
+def test_workload_full_size_sampled(name, cuda_device):
+    w = workloads.WORKLOADS[name]
+    x = workloads.device_inputs(w, DEV, with_grad=w.backward)
+    resid = torch.zeros(w.K + 1, device=DEV)
+    H = binding.newton_forward(w.cell_id, x["px"], x["a"], None, K=w.K, resid_hist=resid)
+    # sample channels; for the weight gradient, take every batch row of the sampled d
+    n_d = 24 if w.T <= 16384 else 12
+    ds = sorted(set(d for _, d in workloads.sample_channels(w, n_d, seed=99)))
+    chans = [(b, d) for d in ds for b in range(w.B)] if w.backward else workloads.sample_channels(w, 48, seed=7)
+    a_np = None if x["a"] is None else to_np(x["a"])
+    # full tensors stay on the device; only the sampled channels move to the host
+    Hs = gather_channels(H, chans)
+    pxs_dev = gather_channels(x["px"], chans)  # (T,G,n): values the GPU read (bf16 upcast exactly)
+    # oracle on the sampled channels: a (1,T,G,n) problem from the gathered values
+    px1 = pxs_dev[None]
+    w1 = None if a_np is None else a_np[:, [d for _, d in chans]]
+    Ho, ro = oracle.newton(w.cell_id, px1, w1, None, K=w.K)
+    assert rel_err(Hs, Ho[0]) <= TOL_H, name
+    if w.px_dtype == "bf16":
+        px32s = gather_channels(x["px32"], chans)[None]
+        Hf, _ = oracle.newton(w.cell_id, px32s, w1, None, K=w.K)
+        assert norm_err(Hs, Hf[0]) <= TOL_BF16_F32, name
+    # the residual history is a max over the whole batch: the sample's is a lower bound
+    r = to_np(resid)
+    assert np.all(r[:-1] + 1e-5 >= ro[:-1] * (1 - 1e-3)), (r, ro)
+    assert np.all(np.diff(r) < 0), r
+    if w.backward:
+        g = x["dLdH"]
+        dpx, da, _ = binding.newton_backward(w.cell_id, x["px"], H, g, x["a"])
+        gs = gather_channels(g, chans)[None]
+        dpxo, dao, _ = oracle.adjoint(w.cell_id, px1, w1, None, Ho, gs)
+        assert rel_err(gather_channels(dpx, chans), dpxo[0]) <= TOL_G, name
+        # dL/da[g, d] sums over every batch row of channel d; the sample holds all of them
+        da_np = to_np(da)
+        ref = np.zeros((w.G, len(ds)))
+        for i, (b, d) in enumerate(chans):
+            ref[:, ds.index(d)] += dao[:, i]
+        assert rel_err(da_np[:, ds], ref) <= TOL_G, name
