@@ -43,9 +43,10 @@
  *   dL_dpx   (B, T, G, D)  float32
  *   dL_da    (G, D)        float32
  *   dL_dh0   (B, S, D)     float32
- * Every pointer must be aligned to its element size; rows are read with
- * 16-byte (f32) or 8-byte (bf16) vector loads when D is a multiple of 4 and
- * every pointer is 16-byte aligned, and element by element otherwise.
+ * Every pointer must be aligned to its element size.  When D times the
+ * pre-activation element size is a multiple of 16 bytes and the row buffers
+ * are 16-byte aligned, tiles are staged by the tensor memory accelerator;
+ * otherwise the same kernels copy them element by element.
  *
  * Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
  * default stream).  Argument errors are detected on the host before anything
@@ -53,9 +54,10 @@
  * GPU detects -- a non-finite value in the output, a wait between thread
  * blocks that ran past its time limit -- are recorded in the workspace and
  * returned by pararnn_status_sync().  A CUDA launch or copy failure returns
- * PARARNN_ECUDA.  The library allocates no memory and keeps no state between
- * calls; pararnn_last_error() describes the last failure on the calling
- * thread.  Results are deterministic: the same inputs give the same bits,
+ * PARARNN_ECUDA.  The library allocates no memory; the only state it keeps
+ * between calls is a process-wide call counter that tags the scan carries it
+ * leaves in a workspace.  pararnn_last_error() describes the last failure on
+ * the calling thread.  Results are deterministic: the same inputs give the same bits,
  * whatever the order in which thread blocks run.
  */
 #ifndef PARARNN_B200_H
@@ -95,9 +97,13 @@ int pararnn_state_width(pararnn_cell cell);
 /* Bytes of device workspace that pararnn_newton_forward (with this K) and
  * pararnn_newton_backward need for a (B, T, D) problem; the same buffer
  * serves both.  0 for an unknown cell or a negative size.  Pure host
- * function.  The workspace holds the inter-block scan carries, a status
- * word and per-block gradient partials; its contents need no initialisation
- * (each call resets what it uses on `stream`). */
+ * function.  The workspace holds a status word, a tile counter, the
+ * inter-block scan carries and per-block gradient partials.  Zero-fill it
+ * once after allocating it (cudaMemset); after that the library keeps it
+ * consistent from call to call: carries are tagged with a per-call number
+ * and words left by earlier calls never read as valid.  Calls that share a
+ * workspace must be ordered (the same stream, or synchronised); calls that
+ * overlap on the GPU with one workspace race. */
 size_t pararnn_workspace_bytes(pararnn_cell cell, int64_t B, int64_t T, int64_t D, int K);
 
 /* Newton forward: K >= 1 iterations from the warm start, output H = h^(K).
@@ -108,7 +114,8 @@ size_t pararnn_workspace_bytes(pararnn_cell cell, int64_t B, int64_t T, int64_t 
  *   K          1..64 Newton iterations; the linear cell is exact after one,
  *              and performs exactly one scan for any K
  *   H_out      (B,T,S,D) f32, written
- *   workspace  >= pararnn_workspace_bytes(cell,B,T,D,K) bytes, 256-byte aligned
+ *   workspace  >= pararnn_workspace_bytes(cell,B,T,D,K) bytes, 16-byte
+ *              aligned, zero-filled once after allocation
  *   resid_hist NULL, or K+1 floats of device memory that receive
  *              max_{b,t,s,d} |F(H^(k))| for k = 0..K (the residual history a
  *              NewtonDivergenceError carries, Evaluation section)

@@ -155,10 +155,11 @@ def _shape(cell, px):
 
 
 def workspace_for(cell, B, T, D, K, device):
+    """A zero-filled workspace (the one initialisation the C ABI asks for)."""
     import torch
 
     n = pararnn_workspace_bytes(cell, B, T, D, K)
-    return torch.empty(n, dtype=torch.uint8, device=device)
+    return torch.zeros(n, dtype=torch.uint8, device=device)
 
 
 def newton_forward(cell, px, diag_w=None, h0=None, K=1, out=None, workspace=None, resid_hist=None, stream=None,

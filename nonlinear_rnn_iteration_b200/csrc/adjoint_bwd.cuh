@@ -1,14 +1,14 @@
 // adjoint_bwd.cuh -- the backward pass: a reverse-time scan for the adjoint
-// state and the gradient epilogue, fused in one kernel, plus a fixed-order
-// reduction of the per-tile weight-gradient partials.
+// state and the gradient epilogue, fused in one persistent kernel, plus a
+// fixed-order reduction of the per-tile weight-gradient partials.
 //
 // At the trajectory H (the forward's output), with g_t = dL/dH_t:
 //     lambda_t = g_t + A_{t+1}^T lambda_{t+1},   lambda_{T-1} = g_{T-1},
 //     A_{t+1} = df/dh at (h_t, x_{t+1}),
 // which is the scan of the elements (M_t, g_t), M_t = A_{t+1}^T, in reverse
 // time under the same operator as the forward (pararnn-torch PyPI page,
-// Method section: the backward follows the paper's adjoint; this is the plain
-// adjoint of the lower-bidiagonal system F(H) = 0).  Then
+// Method section: the backward follows the paper's adjoint; here it is the
+// plain adjoint of the lower-bidiagonal system F(H) = 0).  Then
 //     dL/dp_g[t]  = lambda_t . df/dp_g   at (h_{t-1}, x_t)
 //     dL/da_g     = sum_{b,t} lambda_t . df/da_g
 //     dL/dh0      = A_0^T lambda_0.
@@ -21,6 +21,8 @@
 #include "cells.cuh"
 #include "common.cuh"
 #include "lookback.cuh"
+#include "newton_fwd.cuh"
+#include "tma.cuh"
 
 namespace pararnn {
 
@@ -33,271 +35,316 @@ struct BwdParams {
     float* dLdpx;       // (B,T,G,D)
     float* dLdh0;       // (B,S,D) or null
     float* part;        // per-tile dL/da partials [nTiles][G][W]
+    unsigned* ticket;
     int64_t B, T, D;
-    int64_t nCG, nChunks;
+    int64_t nCG, nChunks, nTiles;
     LookbackCtx lb;     // nSlots = 1
 };
 
+template <class Sh, typename PxT>
+struct BwdSmem {
+    alignas(128) PxT px[Sh::NSTAGE][Sh::L][Sh::G][Sh::W];
+    alignas(128) float H[Sh::NSTAGE][Sh::L][Sh::S][Sh::W];
+    alignas(128) float g[Sh::NSTAGE][Sh::L][Sh::S][Sh::W];
+    float agg[Sh::NSUB][Sh::NA][Sh::W];   // indexed by position in the reverse scan
+    float carry[Sh::NSUB][Sh::S][Sh::W];
+    float firstA[Sh::NSUB][Sh::S * Sh::S][Sh::W];  // each sub-chunk's first-row Jacobian
+    float hprev[Sh::S][Sh::W];            // state just before the tile
+    float w[Sh::G][Sh::W];
+    float da[Sh::NSUB][Sh::G][Sh::W];
+    uint64_t bar[Sh::NSTAGE];
+    unsigned ticket[Sh::NSTAGE];
+};
+
+template <class Sh>
+struct BwdMaps {
+    CUtensorMap px, H, g;
+};
+
 template <class Cell, typename PxT, class Sh>
-__global__ void __launch_bounds__(Sh::NT) adjoint_bwd_kernel(const BwdParams prm) {
-    constexpr int G = Sh::G, S = Sh::S, NA = Sh::NA, V = Sh::V, R = Sh::R, NS = Cell::NSENS;
+__device__ __forceinline__ void issue_bwd_load(const BwdMaps<Sh>* maps, BwdSmem<Sh, PxT>& sm, const BwdParams& prm,
+                                               unsigned tile, int stage) {
+    const int64_t pos = tile / prm.lb.nGroups;
+    const int64_t gid = tile - pos * prm.lb.nGroups;
+    const int64_t chunk = prm.nChunks - 1 - pos;
+    const int64_t b = gid / prm.nCG;
+    const int64_t d0 = (gid - b * prm.nCG) * Sh::W;
+    const int row = (int)(b * prm.T + chunk * Sh::L);
+    constexpr uint32_t bytes = Sh::L * Sh::W * (Sh::G * sizeof(PxT) + 2 * Sh::S * sizeof(float));
+    mbar_arrive_expect_tx(&sm.bar[stage], bytes);
+    tma_load_3d(&sm.px[stage][0][0][0], &maps->px, &sm.bar[stage], (int)d0, 0, row);
+    tma_load_3d(&sm.H[stage][0][0][0], &maps->H, &sm.bar[stage], (int)d0, 0, row);
+    tma_load_3d(&sm.g[stage][0][0][0], &maps->g, &sm.bar[stage], (int)d0, 0, row);
+}
+
+template <class Cell, typename PxT, class Sh>
+__global__ void __launch_bounds__(Sh::NT, Sh::MINB)
+    adjoint_bwd_kernel(const __grid_constant__ BwdMaps<Sh> maps, const BwdParams prm) {
+    constexpr int G = Sh::G, S = Sh::S, V = Sh::V, R = Sh::R, NS = Cell::NSENS;
     constexpr int TPW = Sh::TPW, NSUB = Sh::NSUB, W = Sh::W, L = Sh::L, LC = Sh::LC, NT = Sh::NT;
     constexpr int CPL = W / 32;
-    static_assert(G * W <= NT, "one thread per (gate, channel) in the partial reduction");
-
-    __shared__ float s_agg[NSUB][NA][W];    // indexed by position in the reverse scan
-    __shared__ float s_carry[NSUB][S][W];
-    __shared__ float s_edge[NSUB][S][W];    // each sub-chunk's last state h
-    __shared__ float s_firstA[NSUB][S * S][W];  // each sub-chunk's first-row Jacobian
-    __shared__ float s_da[NSUB][G][W];
-    __shared__ unsigned s_ticket;
+    using SM = BwdSmem<Sh, PxT>;
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    SM& sm = *reinterpret_cast<SM*>(smem_raw);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int sub = warp * TPW + lane / LC;
     const int rs = NSUB - 1 - sub;  // this sub-chunk's position in the reverse scan
     const int cc = (lane % LC) * V;
-
-    if (tid == 0) s_ticket = atomicAdd(prm.lb.status + 1, 1u);
-    __syncthreads();
-    const int64_t tile = s_ticket;
-    const int64_t pos = tile / prm.lb.nGroups;
-    const int64_t gid = tile - pos * prm.lb.nGroups;
-    const int64_t chunk = prm.nChunks - 1 - pos;
-    const int64_t b = gid / prm.nCG;
-    const int64_t d0 = (gid - b * prm.nCG) * W;
-    const int64_t t0 = chunk * L;
-    const int64_t tb = t0 + (int64_t)sub * R;
     const int64_t T = prm.T, D = prm.D;
-    const bool cvalid = d0 + cc < D;
-    const PxT* px = static_cast<const PxT*>(prm.px);
+    const PxT* pxg = static_cast<const PxT*>(prm.px);
 
-    float w[V][G];
+    if (tid == 0) {
+        if constexpr (Sh::kTma) {
 #pragma unroll
-    for (int v = 0; v < V; ++v)
-#pragma unroll
-        for (int g = 0; g < G; ++g) w[v][g] = (prm.w && cvalid) ? __ldg(prm.w + g * D + d0 + cc + v) : 0.0f;
-
-    // ---- loads: pre-activations, states, upstream gradients ----
-    float p[R][G][V], hs[R][S][V], gr[R][S][V];
-#pragma unroll
-    for (int r = 0; r < R; ++r) {
-        const int64_t t = tb + r;
-        const bool ok = t < T && cvalid;
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-            if (ok) load_row<V>(px + ((b * T + t) * G + g) * D + d0 + cc, p[r][g]);
-            else
-#pragma unroll
-                for (int v = 0; v < V; ++v) p[r][g][v] = 0.0f;
+            for (int s = 0; s < Sh::NSTAGE; ++s) mbar_init(&sm.bar[s], 1);
+            mbar_fence_init();
         }
+        const unsigned t = atomicAdd(prm.ticket, 1u);
+        sm.ticket[0] = t;
+        if constexpr (Sh::kTma)
+            if (t < prm.nTiles) issue_bwd_load<Cell, PxT, Sh>(&maps, sm, prm, t, 0);
+    }
+    __syncthreads();
+
+    for (int it = 0;; ++it) {
+        const int st = it % Sh::NSTAGE;
+        const unsigned tile_u = sm.ticket[st];
+        if (tile_u >= prm.nTiles) break;
+        if (tid == 0) {
+            const unsigned t2 = atomicAdd(prm.ticket, 1u);
+            sm.ticket[(it + 1) % Sh::NSTAGE] = t2;
+            if constexpr (Sh::kTma)
+                if (t2 < prm.nTiles) issue_bwd_load<Cell, PxT, Sh>(&maps, sm, prm, t2, (it + 1) % Sh::NSTAGE);
+        }
+        const int64_t tile = tile_u;
+        const int64_t pos = tile / prm.lb.nGroups;
+        const int64_t gid = tile - pos * prm.lb.nGroups;
+        const int64_t chunk = prm.nChunks - 1 - pos;
+        const int64_t b = gid / prm.nCG;
+        const int64_t d0 = (gid - b * prm.nCG) * W;
+        const int64_t t0 = chunk * L;
+        const int64_t tb = t0 + (int64_t)sub * R;
+        const bool cvalid = d0 + cc < D;
+
+        for (int i = tid; i < G * W; i += NT) {
+            const int g = i / W, c = i - (i / W) * W;
+            sm.w[g][c] = (prm.w && d0 + c < D) ? __ldg(prm.w + g * D + d0 + c) : 0.0f;
+        }
+        if (tid < W) {
+            const int64_t d = d0 + tid;
 #pragma unroll
-        for (int s = 0; s < S; ++s) {
-            if (ok) {
-                load_row<V>(prm.H + ((b * T + t) * S + s) * D + d0 + cc, hs[r][s]);
-                load_row<V>(prm.dLdH + ((b * T + t) * S + s) * D + d0 + cc, gr[r][s]);
-            } else {
-#pragma unroll
-                for (int v = 0; v < V; ++v) {
-                    hs[r][s][v] = 0.0f;
-                    gr[r][s][v] = 0.0f;
+            for (int s = 0; s < S; ++s) {
+                float x = 0.0f;
+                if (d < D) {
+                    if (t0 > 0) x = prm.H[((b * T + t0 - 1) * S + s) * D + d];
+                    else if (prm.h0) x = prm.h0[(b * S + s) * D + d];
+                }
+                sm.hprev[s][tid] = x;
+            }
+        }
+        if constexpr (Sh::kTma) {
+            Deadline dl;
+            while (!mbar_try_wait(&sm.bar[st], (it / Sh::NSTAGE) & 1)) {
+                if (dl.expired(prm.lb.timeout_ns)) {
+                    if (tid == 0) atomicOr(prm.lb.status, kStatusTimeout);
+                    break;
                 }
             }
-        }
-    }
-#pragma unroll
-    for (int s = 0; s < S; ++s)
-#pragma unroll
-        for (int v = 0; v < V; ++v) s_edge[sub][s][cc + v] = hs[R - 1][s][v];
-    __syncthreads();
-
-    // ---- linearisation at (h_{t-1}, x_t) for every row ----
-    float sp[S][V];
-#pragma unroll
-    for (int v = 0; v < V; ++v)
-#pragma unroll
-        for (int s = 0; s < S; ++s) {
-            float x = 0.0f;
-            if (sub > 0) x = s_edge[sub - 1][s][cc + v];
-            else if (cvalid && t0 > 0) x = prm.H[((b * T + t0 - 1) * S + s) * D + d0 + cc + v];
-            else if (cvalid && prm.h0) x = prm.h0[(b * S + s) * D + d0 + cc + v];
-            sp[s][v] = x;
-        }
-    float jA[R][S * S][V], sens[R][NS][V];
-#pragma unroll
-    for (int r = 0; r < R; ++r)
-#pragma unroll
-        for (int v = 0; v < V; ++v) {
-            float pv[G], wv[G], spv[S], A[S * S], se[NS];
-#pragma unroll
-            for (int g = 0; g < G; ++g) {
-                pv[g] = p[r][g][v];
-                wv[g] = w[v][g];
+        } else {
+            for (int i = tid; i < L * G * W; i += NT) {
+                const int row = i / (G * W), rem = i - row * (G * W), g = rem / W, c = rem - g * W;
+                const int64_t t = t0 + row, d = d0 + c;
+                sm.px[st][row][g][c] = (t < T && d < D) ? pxg[((b * T + t) * G + g) * D + d] : PxT(0.0f);
             }
-#pragma unroll
-            for (int s = 0; s < S; ++s) spv[s] = sp[s][v];
-            Cell::bwd(pv, wv, spv, A, se);
-#pragma unroll
-            for (int a = 0; a < S * S; ++a) jA[r][a][v] = A[a];
-#pragma unroll
-            for (int n = 0; n < NS; ++n) sens[r][n][v] = se[n];
-#pragma unroll
-            for (int s = 0; s < S; ++s) sp[s][v] = hs[r][s][v];
+            for (int i = tid; i < L * S * W; i += NT) {
+                const int row = i / (S * W), rem = i - row * (S * W), s = rem / W, c = rem - s * W;
+                const int64_t t = t0 + row, d = d0 + c;
+                const bool ok = t < T && d < D;
+                sm.H[st][row][s][c] = ok ? prm.H[((b * T + t) * S + s) * D + d] : 0.0f;
+                sm.g[st][row][s][c] = ok ? prm.dLdH[((b * T + t) * S + s) * D + d] : 0.0f;
+            }
         }
-#pragma unroll
-    for (int a = 0; a < S * S; ++a)
-#pragma unroll
-        for (int v = 0; v < V; ++v) s_firstA[sub][a][cc + v] = jA[0][a][v];
+        __syncthreads();
 
-    // the last sub-chunk also needs A at the first row of the next tile
-    float nextA[S * S][V];
-    if (sub == NSUB - 1) {
-        const int64_t tn = t0 + L;
+        // ---- linearisation at (h_{t-1}, x_t) for every row ----
+        float jA[R][S * S][V], sens[R][NS][V];
 #pragma unroll
-        for (int v = 0; v < V; ++v) {
-            float A[S * S];
+        for (int r = 0; r < R; ++r)
 #pragma unroll
-            for (int a = 0; a < S * S; ++a) A[a] = 0.0f;
-            if (tn < T && cvalid) {
-                float pv[G], wv[G], spv[S], se[NS];
+            for (int v = 0; v < V; ++v) {
+                float pv[G], wv[G], spv[S], A[S * S], se[NS];
+                const int row = sub * R + r;
 #pragma unroll
                 for (int g = 0; g < G; ++g) {
-                    pv[g] = PxTraits<PxT>::cvt(px[((b * T + tn) * G + g) * D + d0 + cc + v]);
-                    wv[g] = w[v][g];
+                    pv[g] = PxTraits<PxT>::cvt(sm.px[st][row][g][cc + v]);
+                    wv[g] = sm.w[g][cc + v];
                 }
 #pragma unroll
-                for (int s = 0; s < S; ++s) spv[s] = hs[R - 1][s][v];
+                for (int s = 0; s < S; ++s) spv[s] = row > 0 ? sm.H[st][row - 1][s][cc + v] : sm.hprev[s][cc + v];
                 Cell::bwd(pv, wv, spv, A, se);
+#pragma unroll
+                for (int a = 0; a < S * S; ++a) jA[r][a][v] = A[a];
+#pragma unroll
+                for (int n = 0; n < NS; ++n) sens[r][n][v] = se[n];
             }
 #pragma unroll
-            for (int a = 0; a < S * S; ++a) nextA[a][v] = A[a];
-        }
-    }
-    __syncthreads();
-
-    // ---- reverse-scan elements (M_t, g_t), M_t = A_{t+1}^T ----
-    float eM[R][S * S][V];
+        for (int a = 0; a < S * S; ++a)
 #pragma unroll
-    for (int r = 0; r < R; ++r)
+            for (int v = 0; v < V; ++v) sm.firstA[sub][a][cc + v] = jA[0][a][v];
+        // the last sub-chunk also needs A at the first row of the next tile
+        float nextA[S * S][V];
+        if (sub == NSUB - 1) {
+            const int64_t tn = t0 + L;
+#pragma unroll
+            for (int v = 0; v < V; ++v) {
+                float A[S * S];
+#pragma unroll
+                for (int a = 0; a < S * S; ++a) A[a] = 0.0f;
+                if (tn < T && cvalid) {
+                    float pv[G], wv[G], spv[S], se[NS];
+#pragma unroll
+                    for (int g = 0; g < G; ++g) {
+                        pv[g] = PxTraits<PxT>::cvt(pxg[((b * T + tn) * G + g) * D + d0 + cc + v]);
+                        wv[g] = sm.w[g][cc + v];
+                    }
+#pragma unroll
+                    for (int s = 0; s < S; ++s) spv[s] = sm.H[st][L - 1][s][cc + v];
+                    Cell::bwd(pv, wv, spv, A, se);
+                }
+#pragma unroll
+                for (int a = 0; a < S * S; ++a) nextA[a][v] = A[a];
+            }
+        }
+        __syncthreads();
+
+        // ---- reverse-scan elements (M_t, g_t), M_t = A_{t+1}^T ----
+        float eM[R][S * S][V];
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+#pragma unroll
+            for (int v = 0; v < V; ++v) {
+                const int64_t t = tb + r;
+                float A[S * S];
+#pragma unroll
+                for (int a = 0; a < S * S; ++a) {
+                    if (r + 1 < R) A[a] = jA[r + 1][a][v];
+                    else if (sub + 1 < NSUB) A[a] = sm.firstA[sub + 1][a][cc + v];
+                    else A[a] = nextA[a][v];
+                }
+                const bool has_next = (t + 1 < T) && cvalid;
+                const bool rvalid = (t < T) && cvalid;
+#pragma unroll
+                for (int i = 0; i < S; ++i)
+#pragma unroll
+                    for (int m = 0; m < S; ++m) {
+                        float val = has_next ? A[m * S + i] : 0.0f;  // transpose
+                        if (!rvalid) val = (i == m) ? 1.0f : 0.0f;     // past the end: identity
+                        eM[r][i * S + m][v] = val;
+                    }
+            }
 #pragma unroll
         for (int v = 0; v < V; ++v) {
-            const int64_t t = tb + r;
-            float A[S * S];
+            Elem<S> acc;
+            elem_identity<S>(acc);
 #pragma unroll
-            for (int a = 0; a < S * S; ++a) {
-                if (r + 1 < R) A[a] = jA[r + 1][a][v];
-                else if (sub + 1 < NSUB) A[a] = s_firstA[sub + 1][a][cc + v];
-                else A[a] = nextA[a][v];
+            for (int r = R - 1; r >= 0; --r) {
+                float M[S * S], gv[S];
+#pragma unroll
+                for (int a = 0; a < S * S; ++a) M[a] = eM[r][a][v];
+#pragma unroll
+                for (int s = 0; s < S; ++s) gv[s] = (tb + r < T) ? sm.g[st][sub * R + r][s][cc + v] : 0.0f;
+                compose_after<S>(M, gv, acc);
             }
-            const bool has_next = (t + 1 < T) && cvalid;
-            const bool rvalid = (t < T) && cvalid;
 #pragma unroll
-            for (int i = 0; i < S; ++i)
+            for (int a = 0; a < S * S; ++a) sm.agg[rs][a][cc + v] = acc.A[a];
 #pragma unroll
-                for (int m = 0; m < S; ++m) {
-                    float val = has_next ? A[m * S + i] : 0.0f;  // transpose
-                    if (!rvalid) val = (i == m) ? 1.0f : 0.0f;     // past the end: identity
-                    eM[r][i * S + m][v] = val;
-                }
+            for (int s = 0; s < S; ++s) sm.agg[rs][S * S + s][cc + v] = acc.b[s];
         }
+        __syncthreads();
+
+        if (warp == 0) {
+            float zero[CPL][S], carry[CPL][S];
 #pragma unroll
-    for (int v = 0; v < V; ++v) {
-        Elem<S> acc;
-        elem_identity<S>(acc);
+            for (int j = 0; j < CPL; ++j)
 #pragma unroll
-        for (int r = R - 1; r >= 0; --r) {
-            float M[S * S], g[S];
-#pragma unroll
-            for (int a = 0; a < S * S; ++a) M[a] = eM[r][a][v];
-#pragma unroll
-            for (int s = 0; s < S; ++s) g[s] = gr[r][s][v];
-            compose_after<S>(M, g, acc);
+                for (int s = 0; s < S; ++s) zero[j][s] = 0.0f;  // lambda_T = 0
+            tile_scan_step<S, W, NSUB, Sh::P>(prm.lb, tile, pos, 0, lane, sm.agg, sm.carry, zero, carry);
         }
-#pragma unroll
-        for (int a = 0; a < S * S; ++a) s_agg[rs][a][cc + v] = acc.A[a];
-#pragma unroll
-        for (int s = 0; s < S; ++s) s_agg[rs][S * S + s][cc + v] = acc.b[s];
-    }
-    __syncthreads();
+        __syncthreads();
 
-    if (warp == 0) {
-        float zero[CPL][S], carry[CPL][S];
+        // ---- lambda and the gradient epilogue ----
+        float da_acc[G][V];
 #pragma unroll
-        for (int j = 0; j < CPL; ++j)
+        for (int g = 0; g < G; ++g)
 #pragma unroll
-            for (int s = 0; s < S; ++s) zero[j][s] = 0.0f;  // lambda_T = 0
-        tile_scan_step<S, W, NSUB>(prm.lb, tile, pos, 0, lane, s_agg, s_carry, zero, carry);
-    }
-    __syncthreads();
-
-    // ---- lambda and the gradient epilogue ----
-    float da_acc[G][V];
+            for (int v = 0; v < V; ++v) da_acc[g][v] = 0.0f;
+        float outp[R][G][V];
+        bool bad = false;
 #pragma unroll
-    for (int g = 0; g < G; ++g)
+        for (int v = 0; v < V; ++v) {
+            float x[S];
 #pragma unroll
-        for (int v = 0; v < V; ++v) da_acc[g][v] = 0.0f;
-    bool bad = false;
+            for (int s = 0; s < S; ++s) x[s] = sm.carry[rs][s][cc + v];
 #pragma unroll
-    for (int v = 0; v < V; ++v) {
-        float x[S];
+            for (int r = R - 1; r >= 0; --r) {
+                const bool rvalid = (tb + r < T) && cvalid;
+                float M[S * S], gv[S], y[S];
 #pragma unroll
-        for (int s = 0; s < S; ++s) x[s] = s_carry[rs][s][cc + v];
+                for (int a = 0; a < S * S; ++a) M[a] = eM[r][a][v];
 #pragma unroll
-        for (int r = R - 1; r >= 0; --r) {
-            float M[S * S], g[S], y[S];
+                for (int s = 0; s < S; ++s) gv[s] = (tb + r < T) ? sm.g[st][sub * R + r][s][cc + v] : 0.0f;
+                apply<S>(M, gv, x, y);
 #pragma unroll
-            for (int a = 0; a < S * S; ++a) M[a] = eM[r][a][v];
+                for (int s = 0; s < S; ++s) x[s] = y[s];
+                float se[NS], dp[G], da[G];
 #pragma unroll
-            for (int s = 0; s < S; ++s) g[s] = gr[r][s][v];
-            apply<S>(M, g, x, y);
-#pragma unroll
-            for (int s = 0; s < S; ++s) x[s] = y[s];
-            float se[NS], dp[G], da[G];
-#pragma unroll
-            for (int n = 0; n < NS; ++n) se[n] = sens[r][n][v];
-            Cell::grads(se, x, dp, da);
-            const bool rvalid = (tb + r < T) && cvalid;
-            if (rvalid) {
+                for (int n = 0; n < NS; ++n) se[n] = sens[r][n][v];
+                Cell::grads(se, x, dp, da);
 #pragma unroll
                 for (int g2 = 0; g2 < G; ++g2) {
-                    p[r][g2][v] = dp[g2];  // reuse the pre-activation registers for the output row
-                    da_acc[g2][v] += da[g2];
-                    bad |= !isfinite(dp[g2]);
+                    outp[r][g2][v] = dp[g2];
+                    if (rvalid) {
+                        da_acc[g2][v] += da[g2];
+                        bad |= !isfinite(dp[g2]);
+                    }
                 }
-            }
-            if (r == 0 && tb == 0 && rvalid && prm.dLdh0) {
-                // dL/dh0 = A_0^T lambda_0, A_0 at (h0, x_0)
+                if (r == 0 && tb == 0 && rvalid && prm.dLdh0) {
+                    // dL/dh0 = A_0^T lambda_0, A_0 at (h0, x_0)
 #pragma unroll
-                for (int i = 0; i < S; ++i) {
-                    float acc = 0.0f;
+                    for (int i = 0; i < S; ++i) {
+                        float acc = 0.0f;
 #pragma unroll
-                    for (int m = 0; m < S; ++m) acc = __fmaf_rn(jA[0][m * S + i][v], x[m], acc);
-                    prm.dLdh0[(b * S + i) * D + d0 + cc + v] = acc;
+                        for (int m = 0; m < S; ++m) acc = __fmaf_rn(jA[0][m * S + i][v], x[m], acc);
+                        prm.dLdh0[(b * S + i) * D + d0 + cc + v] = acc;
+                    }
                 }
             }
         }
-    }
 #pragma unroll
-    for (int r = 0; r < R; ++r) {
-        const int64_t t = tb + r;
-        if (t < T && cvalid) {
+        for (int r = 0; r < R; ++r) {
+            const int64_t t = tb + r;
+            if (t < T && cvalid) {
 #pragma unroll
-            for (int g = 0; g < G; ++g) store_row<V>(prm.dLdpx + ((b * T + t) * G + g) * D + d0 + cc, p[r][g]);
+                for (int g = 0; g < G; ++g) store_row<V>(prm.dLdpx + ((b * T + t) * G + g) * D + d0 + cc, outp[r][g]);
+            }
         }
-    }
-    if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(prm.lb.status, kStatusNonFinite);
+        if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(prm.lb.status, kStatusNonFinite);
 
-    // ---- per-tile dL/da partial, summed over sub-chunks in a fixed order ----
+        // ---- per-tile dL/da partial, summed over sub-chunks in a fixed order ----
 #pragma unroll
-    for (int g = 0; g < G; ++g)
+        for (int g = 0; g < G; ++g)
 #pragma unroll
-        for (int v = 0; v < V; ++v) s_da[sub][g][cc + v] = da_acc[g][v];
-    __syncthreads();
-    if (tid < G * W) {
-        const int g = tid / W, ch = tid - (tid / W) * W;
-        float acc = 0.0f;
+            for (int v = 0; v < V; ++v) sm.da[sub][g][cc + v] = da_acc[g][v];
+        __syncthreads();
+        for (int i = tid; i < G * W; i += NT) {
+            const int g = i / W, ch = i - (i / W) * W;
+            float acc = 0.0f;
 #pragma unroll 4
-        for (int sb = 0; sb < NSUB; ++sb) acc += s_da[sb][g][ch];
-        prm.part[(tile * G + g) * W + ch] = acc;
+            for (int sb = 0; sb < NSUB; ++sb) acc += sm.da[sb][g][ch];
+            prm.part[(tile * G + g) * W + ch] = acc;
+        }
+        __syncthreads();  // stage st, the ticket slot and the shared partials are free again
     }
 }
 

@@ -1,6 +1,6 @@
 // common.cuh -- device helpers shared by the forward and backward kernels:
-// vectorised row loads/stores, the release/acquire flag protocol used by the
-// decoupled look-back between thread blocks, and the bounded wait.
+// vectorised row loads/stores, the global timer for bounded waits, and the
+// activation functions.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -14,11 +14,6 @@ namespace pararnn {
 constexpr unsigned kStatusNonFinite = 1u;
 constexpr unsigned kStatusTimeout = 2u;
 constexpr size_t kHeaderBytes = 256;
-
-// look-back flag values (one 32-bit flag per tile and Newton iteration)
-constexpr unsigned kFlagEmpty = 0u;
-constexpr unsigned kFlagAggregate = 1u;   // the tile's own composed element is published
-constexpr unsigned kFlagInclusive = 2u;   // the state after the tile's last row is published
 
 // ---- element loads -------------------------------------------------------
 
@@ -84,30 +79,6 @@ __device__ __forceinline__ void store_row(float* p, const float (&v)[V]) {
 #pragma unroll
         for (int i = 0; i < V; ++i) p[i] = v[i];
     }
-}
-
-// ---- inter-block protocol ------------------------------------------------
-// A tile publishes a payload (plain stores by several lanes of one warp),
-// every writing lane fences, the warp synchronises, and one lane stores the
-// flag with release semantics at GPU scope.  A reader loads the flag with
-// acquire semantics, synchronises its warp, and loads the payload with
-// relaxed GPU-scope loads, which are served by L2 and never by a stale L1
-// line.
-
-__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
-    unsigned v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-
-__device__ __forceinline__ void st_release_gpu(unsigned* p, unsigned v) {
-    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
-__device__ __forceinline__ float ld_relaxed_gpu(const float* p) {
-    float v;
-    asm volatile("ld.relaxed.gpu.global.f32 %0, [%1];" : "=f"(v) : "l"(p) : "memory");
-    return v;
 }
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {

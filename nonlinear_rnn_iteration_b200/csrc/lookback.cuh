@@ -1,20 +1,27 @@
 // lookback.cuh -- decoupled look-back between the tiles of one channel group.
 //
-// Tiles are numbered by a ticket taken at block start (an atomic counter), in
-// scan order: ticket = position_along_the_scan * nGroups + group.  A tile
-// therefore waits only on tiles whose tickets were taken earlier, by blocks
-// that are already running, so every wait ends (forward progress does not
-// depend on the order in which the hardware schedules blocks).
+// Tiles are numbered by a ticket taken from an atomic counter, in scan
+// order: ticket = position_along_the_scan * nGroups + group.  A block
+// processes its tickets in increasing order, so the smallest unfinished
+// ticket always belongs to a running block and every wait ends (forward
+// progress does not depend on how the hardware schedules blocks).
 //
 // Per (tile, slot) -- slot = Newton iteration in the forward, 0 in the
-// backward -- the workspace holds one flag and two payloads, W channels wide:
-//   aggregate  the tile's composed scan element (A: S x S, b: S)   [flag 1]
-//   inclusive  the state after the tile's last row                  [flag 2]
+// backward -- and per channel, the workspace holds 64-bit words
+//     { high 32 bits: the call's epoch tag, low 32 bits: a float }
+//   aggregate  the tile's composed scan element (A: S x S, b: S)  NA words
+//   inclusive  the state after the tile's last row                 S words
+// A word is valid when its tag equals this call's epoch, so a value and its
+// "ready" flag travel in one single-copy-atomic store: publishing needs no
+// fence and reading needs one L2 round trip.  Words left by earlier calls
+// carry other tags and read as not ready; a zero-filled workspace never
+// matches (epochs start at 1).
+//
 // The carry into a tile is found by walking back to the nearest predecessor
 // with an inclusive value and applying the aggregates in between, in order,
-// to it.  Because an inclusive value is itself formed as
-// apply(aggregate, carry), the carry comes out bit-identical whichever
-// predecessors had already finished: results do not depend on timing.
+// to it.  An inclusive value is itself formed as apply(aggregate, carry), so
+// the carry is bit-identical whichever predecessors had finished: results do
+// not depend on timing.
 #pragma once
 
 #include "cells.cuh"
@@ -22,149 +29,201 @@
 
 namespace pararnn {
 
+typedef unsigned long long word_t;
+
 struct LookbackCtx {
-    unsigned* status;
-    unsigned* flags;     // [nTiles][nSlots]
-    float* agg;          // [nTiles][nSlots][NA][W]
-    float* inc;          // [nTiles][nSlots][S][W]
+    unsigned* status;  // workspace header word 0
+    word_t* agg;       // [nTiles][nSlots][NA][W]
+    word_t* inc;       // [nTiles][nSlots][S][W]
     int64_t nGroups;
     int nSlots;
+    uint32_t epoch;
     uint64_t timeout_ns;
 };
 
-// Bounded wait for a flag to reach `want` (or more).  Returns false if the
-// time limit passed first; the caller records the time-out and carries on, so
-// that the kernel always finishes.
-__device__ __forceinline__ bool wait_flag(const unsigned* flag, unsigned want, uint64_t timeout_ns, unsigned& seen) {
-    seen = ld_acquire_gpu(flag);
-    if (seen >= want) return true;
-    const uint64_t t0 = globaltimer_ns();
-    while (true) {
-        __nanosleep(64);
-        seen = ld_acquire_gpu(flag);
-        if (seen >= want) return true;
-        if (globaltimer_ns() - t0 > timeout_ns) return false;
-    }
+__device__ __forceinline__ void st_word(word_t* p, float v, uint32_t epoch) {
+    const word_t w = (static_cast<word_t>(epoch) << 32) | __float_as_uint(v);
+    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(w) : "memory");
 }
 
-// Publish one payload row set and then the flag.  Called by all 32 lanes of
-// one warp; lane l owns channels l, l+32, ... of the tile.
+__device__ __forceinline__ word_t ld_word(const word_t* p) {
+    word_t w;
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(w) : "l"(p) : "memory");
+    return w;
+}
+
+__device__ __forceinline__ bool word_ok(word_t w, uint32_t epoch) { return static_cast<uint32_t>(w >> 32) == epoch; }
+__device__ __forceinline__ float word_val(word_t w) { return __uint_as_float(static_cast<uint32_t>(w)); }
+
+// Bounded wait for an mbarrier phase or a flag: returns false once
+// `timeout_ns` has passed, so that the caller can record the time-out and
+// finish instead of spinning for ever.
+struct Deadline {
+    uint64_t start = 0;
+    __device__ __forceinline__ bool expired(uint64_t timeout_ns) {
+        const uint64_t now = globaltimer_ns();
+        if (start == 0) {
+            start = now | 1;
+            return false;
+        }
+        return now - start > timeout_ns;
+    }
+};
+
 template <int N, int W>
-__device__ __forceinline__ void publish(float* dst, const float (&vals)[W / 32][N], unsigned* flag, unsigned flag_value,
-                                        int lane) {
+__device__ __forceinline__ void publish_words(word_t* dst, const float (&vals)[W / 32][N], uint32_t epoch, int lane) {
 #pragma unroll
     for (int j = 0; j < W / 32; ++j)
 #pragma unroll
-        for (int n = 0; n < N; ++n) dst[n * W + lane + 32 * j] = vals[j][n];
-    __threadfence();
-    __syncwarp();
-    if (lane == 0) st_release_gpu(flag, flag_value);
+        for (int n = 0; n < N; ++n) st_word(dst + n * W + lane + 32 * j, vals[j][n], epoch);
+}
+
+// Rare path: the nearest inclusive value lies more than P tiles back.  Walk
+// back one predecessor at a time for one channel, then apply the aggregates.
+template <int S, int W>
+__device__ bool lookback_deep(const LookbackCtx& cx, int64_t tile, int64_t dist_max, int slot, int ch, float (&x)[S]) {
+    constexpr int NA = S * S + S;
+    Deadline dl;
+    int64_t found = -1;
+    for (int64_t d = 1; d <= dist_max && found < 0;) {
+        const int64_t tp = tile - d * cx.nGroups;
+        bool inc_ok = true, agg_ok = true;
+#pragma unroll
+        for (int s = 0; s < S; ++s) inc_ok &= word_ok(ld_word(cx.inc + ((tp * cx.nSlots + slot) * S + s) * W + ch), cx.epoch);
+        if (inc_ok) {
+            found = d;
+            break;
+        }
+#pragma unroll
+        for (int a = 0; a < NA; ++a) agg_ok &= word_ok(ld_word(cx.agg + ((tp * cx.nSlots + slot) * NA + a) * W + ch), cx.epoch);
+        if (agg_ok) {
+            ++d;
+            continue;
+        }
+        if (dl.expired(cx.timeout_ns)) return false;
+        __nanosleep(32);
+    }
+    if (found < 0) return false;
+    {
+        const int64_t tp = tile - found * cx.nGroups;
+#pragma unroll
+        for (int s = 0; s < S; ++s) x[s] = word_val(ld_word(cx.inc + ((tp * cx.nSlots + slot) * S + s) * W + ch));
+    }
+    for (int64_t d = found - 1; d >= 1; --d) {
+        const int64_t tp = tile - d * cx.nGroups;
+        float A[S * S], b[S], y[S];
+#pragma unroll
+        for (int a = 0; a < S * S; ++a) A[a] = word_val(ld_word(cx.agg + ((tp * cx.nSlots + slot) * NA + a) * W + ch));
+#pragma unroll
+        for (int s = 0; s < S; ++s) b[s] = word_val(ld_word(cx.agg + ((tp * cx.nSlots + slot) * NA + S * S + s) * W + ch));
+        apply<S>(A, b, x, y);
+#pragma unroll
+        for (int s = 0; s < S; ++s) x[s] = y[s];
+    }
+    return true;
 }
 
 // Carry into `tile` for scan slot `slot`: the state just before the tile's
-// first row.  `dist_max` = number of predecessors (the tile's position along
-// the scan).  Called by all 32 lanes of one warp.
-template <int S, int W>
+// first row, for the W/32 channels this lane owns.  `dist_max` = the tile's
+// position along the scan (its number of predecessors).  All 32 lanes of one
+// warp call this.  The words of the nearest P predecessors are fetched at
+// once, so the common case costs one L2 round trip.
+template <int S, int W, int P>
 __device__ void lookback_carry(const LookbackCtx& cx, int64_t tile, int64_t dist_max, int slot, int lane,
                                float (&carry)[W / 32][S]) {
     constexpr int NA = S * S + S;
     constexpr int CPL = W / 32;
-    // 1. find the nearest predecessor with an inclusive value; lanes read the
-    //    flags of 32 predecessors at once
-    int64_t base = 1, found = -1;
-    uint64_t t_start = 0;
-    bool timed_out = false;
+    const int depth = dist_max < P ? static_cast<int>(dist_max) : P;
+    Deadline dl;
     while (true) {
-        const int64_t j = base + lane;
-        unsigned f = kFlagAggregate;
-        if (j <= dist_max) f = ld_acquire_gpu(cx.flags + (tile - j * cx.nGroups) * cx.nSlots + slot);
-        const unsigned inc_mask = __ballot_sync(0xffffffffu, j <= dist_max && f == kFlagInclusive);
-        const unsigned empty_mask = __ballot_sync(0xffffffffu, j <= dist_max && f == kFlagEmpty);
-        if (inc_mask) {
-            const int first = __ffs(inc_mask) - 1;
-            const unsigned before = first ? (empty_mask & ((1u << first) - 1u)) : 0u;
-            if (!before) {
-                found = base + first;
-                break;
-            }
-        } else if (!empty_mask) {
-            base += 32;  // 32 aggregates in a row: look further back
-            if (base <= dist_max) continue;
-            // the first tile of the scan publishes only an inclusive value, so
-            // this is unreachable unless the workspace was overwritten
-            timed_out = true;
-            break;
-        }
-        if (t_start == 0) {
-            t_start = globaltimer_ns() | 1;
-        } else if (globaltimer_ns() - t_start > cx.timeout_ns) {
-            timed_out = true;
-            break;
-        }
-        __nanosleep(64);
-    }
-    __syncwarp();
-    if (timed_out) {
-        if (lane == 0) atomicOr(cx.status, kStatusTimeout);
+        int state_all = 0;  // bit 0: some channel must wait, bit 1: some channel needs the deep walk
 #pragma unroll
-        for (int j = 0; j < CPL; ++j)
+        for (int j = 0; j < CPL; ++j) {
+            const int ch = lane + 32 * j;
+            word_t wi[P][S], wa[P][NA];
 #pragma unroll
-            for (int s = 0; s < S; ++s) carry[j][s] = 0.0f;
-        return;
-    }
-    // 2. x = inclusive(found), then apply the aggregates of predecessors
-    //    found-1, ..., 1 in that order; loads are issued in batches so that
-    //    several L2 round trips overlap
-    constexpr int BATCH = 4;
-    float x[CPL][S];
-    {
-        const float* ip = cx.inc + ((tile - found * cx.nGroups) * cx.nSlots + slot) * S * W;
+            for (int d = 0; d < P; ++d) {
+                if (d < depth) {
+                    const int64_t tp = tile - (d + 1) * cx.nGroups;
 #pragma unroll
-        for (int j = 0; j < CPL; ++j)
+                    for (int s = 0; s < S; ++s) wi[d][s] = ld_word(cx.inc + ((tp * cx.nSlots + slot) * S + s) * W + ch);
 #pragma unroll
-            for (int s = 0; s < S; ++s) x[j][s] = ld_relaxed_gpu(ip + s * W + lane + 32 * j);
-    }
-    for (int64_t i = found - 1; i >= 1; i -= BATCH) {
-        float e[BATCH][CPL][NA];
-#pragma unroll
-        for (int m = 0; m < BATCH; ++m) {
-            if (i - m >= 1) {
-                const float* ap = cx.agg + ((tile - (i - m) * cx.nGroups) * cx.nSlots + slot) * NA * W;
-#pragma unroll
-                for (int j = 0; j < CPL; ++j)
-#pragma unroll
-                    for (int a = 0; a < NA; ++a) e[m][j][a] = ld_relaxed_gpu(ap + a * W + lane + 32 * j);
-            }
-        }
-#pragma unroll
-        for (int m = 0; m < BATCH; ++m) {
-            if (i - m >= 1) {
-#pragma unroll
-                for (int j = 0; j < CPL; ++j) {
-                    float A[S * S], b[S], y[S];
-#pragma unroll
-                    for (int a = 0; a < S * S; ++a) A[a] = e[m][j][a];
-#pragma unroll
-                    for (int s = 0; s < S; ++s) b[s] = e[m][j][S * S + s];
-                    apply<S>(A, b, x[j], y);
-#pragma unroll
-                    for (int s = 0; s < S; ++s) x[j][s] = y[s];
+                    for (int a = 0; a < NA; ++a) wa[d][a] = ld_word(cx.agg + ((tp * cx.nSlots + slot) * NA + a) * W + ch);
                 }
             }
+            int found = -1, state = 0;
+#pragma unroll
+            for (int d = 0; d < P; ++d) {
+                if (d < depth && found < 0 && state == 0) {
+                    bool inc_ok = true, agg_ok = true;
+#pragma unroll
+                    for (int s = 0; s < S; ++s) inc_ok &= word_ok(wi[d][s], cx.epoch);
+#pragma unroll
+                    for (int a = 0; a < NA; ++a) agg_ok &= word_ok(wa[d][a], cx.epoch);
+                    if (inc_ok) found = d;
+                    else if (!agg_ok) state = 1;
+                }
+            }
+            if (found < 0 && state == 0) state = (depth < dist_max) ? 2 : 1;
+            if (found >= 0) {
+                float x[S];
+#pragma unroll
+                for (int s = 0; s < S; ++s) x[s] = word_val(wi[0][s]);
+#pragma unroll
+                for (int d = P - 1; d >= 0; --d) {
+                    if (d == found) {
+#pragma unroll
+                        for (int s = 0; s < S; ++s) x[s] = word_val(wi[d][s]);
+                    } else if (d < found) {
+                        float A[S * S], b[S], y[S];
+#pragma unroll
+                        for (int a = 0; a < S * S; ++a) A[a] = word_val(wa[d][a]);
+#pragma unroll
+                        for (int s = 0; s < S; ++s) b[s] = word_val(wa[d][S * S + s]);
+                        apply<S>(A, b, x, y);
+#pragma unroll
+                        for (int s = 0; s < S; ++s) x[s] = y[s];
+                    }
+                }
+#pragma unroll
+                for (int s = 0; s < S; ++s) carry[j][s] = x[s];
+            }
+            state_all |= (found >= 0) ? 0 : state;
         }
+        const unsigned wait_any = __ballot_sync(0xffffffffu, state_all & 1);
+        const unsigned deep_any = __ballot_sync(0xffffffffu, state_all & 2);
+        if (!wait_any && !deep_any) return;
+        if (!wait_any && deep_any) {
+            // every unresolved channel has P aggregates in a row: walk further back
+            bool ok = true;
+#pragma unroll
+            for (int j = 0; j < CPL; ++j) {
+                float x[S];
+                if (lookback_deep<S, W>(cx, tile, dist_max, slot, lane + 32 * j, x)) {
+#pragma unroll
+                    for (int s = 0; s < S; ++s) carry[j][s] = x[s];
+                } else {
+                    ok = false;
+                }
+            }
+            if (__all_sync(0xffffffffu, ok)) return;
+            break;  // timed out
+        }
+        if (dl.expired(cx.timeout_ns)) break;
+        __nanosleep(32);
     }
+    if (lane == 0) atomicOr(cx.status, kStatusTimeout);
 #pragma unroll
     for (int j = 0; j < CPL; ++j)
 #pragma unroll
-        for (int s = 0; s < S; ++s) carry[j][s] = x[j][s];
+        for (int s = 0; s < S; ++s) carry[j][s] = 0.0f;
 }
 
-// The work warp 0 does between the two block barriers of one scan step:
-// compose the NSUB sub-chunk elements (s_agg, in scan order) into the tile's
-// element, publish it, find the carry, publish the inclusive state, and
-// write each sub-chunk's carry-in to s_carry.  Returns (in carry_out) the
-// carry into the tile.
-template <int S, int W, int NSUB>
+// Warp 0's work between two block barriers of one scan step: compose the
+// NSUB sub-chunk elements (s_agg, in scan order) into the tile's element,
+// publish it, find the carry, publish the state after the tile, and write
+// each sub-chunk's carry-in to s_carry.  Returns the carry into the tile.
+template <int S, int W, int NSUB, int P>
 __device__ __forceinline__ void tile_scan_step(const LookbackCtx& cx, int64_t tile, int64_t pos, int slot, int lane,
                                                const float (&s_agg)[NSUB][S * S + S][W], float (&s_carry)[NSUB][S][W],
                                                const float (&first_carry)[W / 32][S], float (&carry_out)[W / 32][S]) {
@@ -185,7 +244,6 @@ __device__ __forceinline__ void tile_scan_step(const LookbackCtx& cx, int64_t ti
             compose_after<S>(A, b, tot[j]);
         }
     }
-    unsigned* flag = cx.flags + tile * cx.nSlots + slot;
     float carry[CPL][S];
     if (pos == 0) {
 #pragma unroll
@@ -201,14 +259,14 @@ __device__ __forceinline__ void tile_scan_step(const LookbackCtx& cx, int64_t ti
 #pragma unroll
             for (int s = 0; s < S; ++s) vals[j][S * S + s] = tot[j].b[s];
         }
-        publish<NA, W>(cx.agg + (tile * cx.nSlots + slot) * NA * W, vals, flag, kFlagAggregate, lane);
-        lookback_carry<S, W>(cx, tile, pos, slot, lane, carry);
+        publish_words<NA, W>(cx.agg + (tile * cx.nSlots + slot) * NA * W, vals, cx.epoch, lane);
+        lookback_carry<S, W, P>(cx, tile, pos, slot, lane, carry);
     }
     {
         float vals[CPL][S];
 #pragma unroll
         for (int j = 0; j < CPL; ++j) apply<S>(tot[j].A, tot[j].b, carry[j], vals[j]);
-        publish<S, W>(cx.inc + (tile * cx.nSlots + slot) * S * W, vals, flag, kFlagInclusive, lane);
+        publish_words<S, W>(cx.inc + (tile * cx.nSlots + slot) * S * W, vals, cx.epoch, lane);
     }
 #pragma unroll
     for (int j = 0; j < CPL; ++j) {

@@ -1,8 +1,10 @@
 // pararnn_abi.cu -- the C ABI declared in include/pararnn_b200.h: argument
 // checks, workspace layout, choice of tile shape and kernel launches.
+#include <atomic>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include "pararnn_b200.h"
 
@@ -27,73 +29,89 @@ pararnn_status cuda_fail(cudaError_t e, const char* what) {
     return fail(PARARNN_ECUDA, "%s: %s", what, cudaGetErrorString(e));
 }
 
-// ---- tile shapes (V channels per thread, LC lanes across channels, warps, rows per thread) ----
-// vector path (D a multiple of 4, 16-byte aligned rows): 2 or 4 channels per thread, 64 channels per tile
-using FwdLinV = FwdShape<CellLinear, 4, 16, 8, 4>;
-using FwdGruV = FwdShape<CellGRU, 2, 32, 8, 4>;
-using FwdLstmV = FwdShape<CellLSTM, 2, 32, 8, 2>;
-using BwdLinV = FwdShape<CellLinear, 2, 32, 8, 4>;
-using BwdGruV = FwdShape<CellGRU, 2, 32, 8, 2>;
-using BwdLstmV = FwdShape<CellLSTM, 2, 32, 8, 1>;
-// scalar path (D not a multiple of 4, or unaligned pointers): 32 channels per tile
-using FwdLinS = FwdShape<CellLinear, 1, 32, 8, 8>;
-using FwdGruS = FwdShape<CellGRU, 1, 32, 8, 4>;
-using FwdLstmS = FwdShape<CellLSTM, 1, 32, 8, 2>;
-using BwdLinS = FwdShape<CellLinear, 1, 32, 8, 4>;
-using BwdGruS = FwdShape<CellGRU, 1, 32, 8, 2>;
-using BwdLstmS = FwdShape<CellLSTM, 1, 32, 8, 1>;
+// ---- tile shapes ------------------------------------------------------------
+// FwdShape<Cell, PxT, V channels/thread, LC lanes across channels, warps,
+//          R rows/thread, blocks/SM budget, TMA>
+// TMA path (D * element size a multiple of 16 bytes, 16-byte aligned rows):
+// 64 channels per tile.  Element-wise path otherwise: 32 channels per tile.
+template <typename PxT> using FwdLinT = FwdShape<CellLinear, PxT, 4, 16, 8, 4, 2, true>;
+template <typename PxT> using FwdGruT = FwdShape<CellGRU, PxT, 4, 16, 8, 4, 2, true>;
+template <typename PxT> using FwdLstmT = FwdShape<CellLSTM, PxT, 4, 16, 8, 2, 2, true>;
+template <typename PxT> using BwdLinT = FwdShape<CellLinear, PxT, 4, 16, 8, 2, 2, true>;
+template <typename PxT> using BwdGruT = FwdShape<CellGRU, PxT, 4, 16, 8, 2, 2, true>;
+template <typename PxT> using BwdLstmT = FwdShape<CellLSTM, PxT, 2, 32, 8, 2, 1, true>;
+template <typename PxT> using FwdLinS = FwdShape<CellLinear, PxT, 1, 32, 8, 4, 2, false>;
+template <typename PxT> using FwdGruS = FwdShape<CellGRU, PxT, 1, 32, 8, 4, 2, false>;
+template <typename PxT> using FwdLstmS = FwdShape<CellLSTM, PxT, 1, 32, 8, 2, 2, false>;
+template <typename PxT> using BwdLinS = FwdShape<CellLinear, PxT, 1, 32, 8, 2, 2, false>;
+template <typename PxT> using BwdGruS = FwdShape<CellGRU, PxT, 1, 32, 8, 2, 2, false>;
+template <typename PxT> using BwdLstmS = FwdShape<CellLSTM, PxT, 1, 32, 8, 2, 1, false>;
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far beyond any legitimate wait
 constexpr int kMaxK = 64;
+
+// Epoch tags of the look-back words: unique per call within this process and
+// never 0, so that words left by other calls (or a zero-filled workspace)
+// never read as ready.
+std::atomic<uint32_t> g_epoch{0};
+uint32_t next_epoch() {
+    uint32_t e;
+    do {
+        e = g_epoch.fetch_add(1, std::memory_order_relaxed) + 1;
+    } while (e == 0);
+    return e;
+}
 
 struct Geometry {
     int W = 0, L = 0, S = 0, G = 0, NA = 0, nSlots = 0;
 };
 
-Geometry geometry(pararnn_cell cell, bool fwd, bool vec, int K) {
+template <class Sh>
+Geometry geom_of(int nSlots) {
     Geometry g;
-    auto set = [&](auto sh) {
-        using Sh = decltype(sh);
-        g.W = Sh::W;
-        g.L = Sh::L;
-        g.S = Sh::S;
-        g.G = Sh::G;
-        g.NA = Sh::NA;
-    };
-    if (cell == PARARNN_CELL_LINEAR) {
-        if (fwd) vec ? set(FwdLinV{}) : set(FwdLinS{});
-        else vec ? set(BwdLinV{}) : set(BwdLinS{});
-    } else if (cell == PARARNN_CELL_DIAG_GRU) {
-        if (fwd) vec ? set(FwdGruV{}) : set(FwdGruS{});
-        else vec ? set(BwdGruV{}) : set(BwdGruS{});
-    } else {
-        if (fwd) vec ? set(FwdLstmV{}) : set(FwdLstmS{});
-        else vec ? set(BwdLstmV{}) : set(BwdLstmS{});
-    }
-    g.nSlots = fwd ? (cell == PARARNN_CELL_LINEAR ? 1 : K) : 1;
+    g.W = Sh::W;
+    g.L = Sh::L;
+    g.S = Sh::S;
+    g.G = Sh::G;
+    g.NA = Sh::NA;
+    g.nSlots = nSlots;
     return g;
+}
+
+// The tile geometry does not depend on the pre-activation dtype.
+Geometry geometry(pararnn_cell cell, bool fwd, bool tma, int K) {
+    const int ns = fwd ? (cell == PARARNN_CELL_LINEAR ? 1 : K) : 1;
+    if (cell == PARARNN_CELL_LINEAR) {
+        if (fwd) return tma ? geom_of<FwdLinT<float>>(ns) : geom_of<FwdLinS<float>>(ns);
+        return tma ? geom_of<BwdLinT<float>>(ns) : geom_of<BwdLinS<float>>(ns);
+    }
+    if (cell == PARARNN_CELL_DIAG_GRU) {
+        if (fwd) return tma ? geom_of<FwdGruT<float>>(ns) : geom_of<FwdGruS<float>>(ns);
+        return tma ? geom_of<BwdGruT<float>>(ns) : geom_of<BwdGruS<float>>(ns);
+    }
+    if (fwd) return tma ? geom_of<FwdLstmT<float>>(ns) : geom_of<FwdLstmS<float>>(ns);
+    return tma ? geom_of<BwdLstmT<float>>(ns) : geom_of<BwdLstmS<float>>(ns);
 }
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct Plan {
     int64_t nCG = 0, nChunks = 0, nGroups = 0, nTiles = 0;
-    size_t off_flags = 0, off_agg = 0, off_inc = 0, off_part = 0, total = 0;
+    size_t off_agg = 0, off_inc = 0, off_part = 0, total = 0;
     Geometry g;
 };
 
-Plan make_plan(pararnn_cell cell, int64_t B, int64_t T, int64_t D, int K, bool fwd, bool vec) {
+Plan make_plan(pararnn_cell cell, int64_t B, int64_t T, int64_t D, int K, bool fwd, bool tma) {
     Plan p;
-    p.g = geometry(cell, fwd, vec, K);
+    p.g = geometry(cell, fwd, tma, K);
     p.nCG = (D + p.g.W - 1) / p.g.W;
     p.nChunks = (T + p.g.L - 1) / p.g.L;
     p.nGroups = B * p.nCG;
     p.nTiles = p.nGroups * p.nChunks;
     const size_t nt = (size_t)p.nTiles, ns = (size_t)p.g.nSlots, W = (size_t)p.g.W;
-    p.off_flags = kHeaderBytes;
-    p.off_agg = align256(p.off_flags + nt * ns * sizeof(unsigned));
-    p.off_inc = align256(p.off_agg + nt * ns * p.g.NA * W * sizeof(float));
-    p.off_part = align256(p.off_inc + nt * ns * p.g.S * W * sizeof(float));
+    p.off_agg = kHeaderBytes;
+    p.off_inc = align256(p.off_agg + nt * ns * p.g.NA * W * sizeof(word_t));
+    p.off_part = align256(p.off_inc + nt * ns * p.g.S * W * sizeof(word_t));
     p.total = fwd ? p.off_part : align256(p.off_part + nt * p.g.G * W * sizeof(float));
     return p;
 }
@@ -119,9 +137,61 @@ pararnn_status check_sizes(pararnn_cell cell, int64_t B, int64_t T, int64_t D) {
     if (!cell_ok(cell)) return fail(PARARNN_EINVAL, "unknown cell %d", (int)cell);
     if (B < 0 || T < 0 || D < 0) return fail(PARARNN_EINVAL, "negative size B=%lld T=%lld D=%lld", (long long)B,
                                              (long long)T, (long long)D);
-    const int64_t lim = int64_t(1) << 40;
-    if (B > lim || T > lim || D > lim || (B && T && D && (double)B * T * D * 4 > 9.0e18 / 16))
-        return fail(PARARNN_EINVAL, "problem too large");
+    if (B * T >= (int64_t(1) << 31) || D >= (int64_t(1) << 31) || (B && T && D && (double)B * T * D > 4.0e12))
+        return fail(PARARNN_EINVAL, "problem too large (B*T and D must be below 2^31)");
+    return PARARNN_OK;
+}
+
+// ---- TMA descriptors ------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+        else
+            cudaGetLastError();
+    });
+    return fn;
+}
+
+// 3-D map over a (rows, inner, D) row-major tensor: dims (D, inner, rows),
+// box (W, inner, L), zero fill outside.
+pararnn_status make_map(CUtensorMap* map, const void* base, bool bf16, int64_t D, int inner, int64_t rows, int W,
+                        int L) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return fail(PARARNN_ECUDA, "cuTensorMapEncodeTiled is unavailable");
+    const size_t esz = bf16 ? 2 : 4;
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)inner, (cuuint64_t)rows};
+    cuuint64_t strides[2] = {(cuuint64_t)(D * esz), (cuuint64_t)(D * esz * inner)};
+    cuuint32_t box[3] = {(cuuint32_t)W, (cuuint32_t)inner, (cuuint32_t)L};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3,
+                    const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(PARARNN_ECUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return PARARNN_OK;
+}
+
+// ---- launches --------------------------------------------------------------
+template <class Kern>
+pararnn_status persistent_grid(Kern kern, int threads, size_t smem, int64_t nTiles, unsigned& grid) {
+    int dev = 0, sms = 0, per_sm = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem);
+    if (e != cudaSuccess) return cuda_fail(e, "occupancy query");
+    if (per_sm < 1) return fail(PARARNN_ECUDA, "kernel does not fit on an SM");
+    const int64_t want = (int64_t)sms * per_sm;
+    grid = (unsigned)(nTiles < want ? nTiles : want);
     return PARARNN_OK;
 }
 
@@ -129,7 +199,28 @@ template <class Cell, typename PxT, class Sh>
 pararnn_status launch_fwd(const Plan& pl, FwdParams prm, cudaStream_t st) {
     prm.nCG = pl.nCG;
     prm.nChunks = pl.nChunks;
-    newton_fwd_kernel<Cell, PxT, Sh><<<(unsigned)pl.nTiles, Sh::NT, 0, st>>>(prm);
+    prm.nTiles = pl.nTiles;
+    CUtensorMap map;
+    memset(&map, 0, sizeof map);
+    if (Sh::kTma) {
+        pararnn_status s = make_map(&map, prm.px, sizeof(PxT) == 2, prm.D, Sh::G, prm.B * prm.T, Sh::W, Sh::L);
+        if (s != PARARNN_OK) return s;
+    }
+    const size_t smem = sizeof(FwdSmem<Sh, PxT>);
+    const bool lean = !Cell::kNonlinear && prm.resid == nullptr;
+    unsigned grid = 0;
+    pararnn_status s;
+    if (lean) {
+        auto kern = newton_fwd_kernel<Cell, PxT, Sh, true>;
+        s = persistent_grid(kern, Sh::NT, smem, pl.nTiles, grid);
+        if (s != PARARNN_OK) return s;
+        kern<<<grid, Sh::NT, smem, st>>>(map, prm);
+    } else {
+        auto kern = newton_fwd_kernel<Cell, PxT, Sh, false>;
+        s = persistent_grid(kern, Sh::NT, smem, pl.nTiles, grid);
+        if (s != PARARNN_OK) return s;
+        kern<<<grid, Sh::NT, smem, st>>>(map, prm);
+    }
     cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? PARARNN_OK : cuda_fail(e, "forward kernel launch");
 }
@@ -138,7 +229,22 @@ template <class Cell, typename PxT, class Sh>
 pararnn_status launch_bwd(const Plan& pl, BwdParams prm, float* dLda, cudaStream_t st) {
     prm.nCG = pl.nCG;
     prm.nChunks = pl.nChunks;
-    adjoint_bwd_kernel<Cell, PxT, Sh><<<(unsigned)pl.nTiles, Sh::NT, 0, st>>>(prm);
+    prm.nTiles = pl.nTiles;
+    BwdMaps<Sh> maps;
+    memset(&maps, 0, sizeof maps);
+    if (Sh::kTma) {
+        const int64_t rows = prm.B * prm.T;
+        pararnn_status s = make_map(&maps.px, prm.px, sizeof(PxT) == 2, prm.D, Sh::G, rows, Sh::W, Sh::L);
+        if (s == PARARNN_OK) s = make_map(&maps.H, prm.H, false, prm.D, Sh::S, rows, Sh::W, Sh::L);
+        if (s == PARARNN_OK) s = make_map(&maps.g, prm.dLdH, false, prm.D, Sh::S, rows, Sh::W, Sh::L);
+        if (s != PARARNN_OK) return s;
+    }
+    const size_t smem = sizeof(BwdSmem<Sh, PxT>);
+    auto kern = adjoint_bwd_kernel<Cell, PxT, Sh>;
+    unsigned grid = 0;
+    pararnn_status s = persistent_grid(kern, Sh::NT, smem, pl.nTiles, grid);
+    if (s != PARARNN_OK) return s;
+    kern<<<grid, Sh::NT, smem, st>>>(maps, prm);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "backward kernel launch");
     if (dLda) {
@@ -160,9 +266,16 @@ pararnn_status launch_bwd(const Plan& pl, BwdParams prm, float* dLda, cudaStream
     return PARARNN_OK;
 }
 
-__global__ void probe_wait_kernel(unsigned* status, const unsigned* flag, uint64_t timeout_ns) {
-    unsigned seen;
-    if (threadIdx.x == 0 && !wait_flag(flag, kFlagInclusive, timeout_ns, seen)) atomicOr(status, kStatusTimeout);
+__global__ void probe_wait_kernel(unsigned* status, const word_t* word, uint32_t epoch, uint64_t timeout_ns) {
+    if (threadIdx.x != 0) return;
+    Deadline dl;
+    while (!word_ok(ld_word(word), epoch)) {
+        if (dl.expired(timeout_ns)) {
+            atomicOr(status, kStatusTimeout);
+            return;
+        }
+        __nanosleep(256);
+    }
 }
 
 }  // namespace
@@ -183,8 +296,8 @@ size_t pararnn_workspace_bytes(pararnn_cell cell, int64_t B, int64_t T, int64_t 
     if (K > kMaxK) K = kMaxK;
     size_t m = kHeaderBytes + 256;
     for (int fwd = 0; fwd < 2; ++fwd)
-        for (int vec = 0; vec < 2; ++vec) {
-            const Plan p = make_plan(cell, B, T, D, K, fwd != 0, vec != 0);
+        for (int tma = 0; tma < 2; ++tma) {
+            const Plan p = make_plan(cell, B, T, D, K, fwd != 0, tma != 0);
             if (p.total > m) m = p.total;
         }
     return m;
@@ -218,13 +331,14 @@ pararnn_status pararnn_newton_forward(pararnn_cell cell, int64_t B, int64_t T, i
         return fail(PARARNN_EINVAL, "resid_hist is not device-accessible float memory");
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const bool vec = (D % 4 == 0) && aligned(preacts, 16) && aligned(H_out, 16);
+    // TMA staging needs 16-byte rows of pre-activations and 16-byte stores of H
+    const bool tma = ((D * (int64_t)esz) % 16 == 0) && aligned(preacts, 16) && aligned(H_out, 16);
     const int Keff = cell == PARARNN_CELL_LINEAR ? 1 : K;
-    const Plan pl = make_plan(cell, B, T, D, Keff, true, vec);
+    const Plan pl = make_plan(cell, B, T, D, Keff, true, tma);
     if (pl.nTiles >= (int64_t(1) << 31)) return fail(PARARNN_EINVAL, "too many tiles");
 
     char* ws = static_cast<char*>(workspace);
-    cudaError_t e = cudaMemsetAsync(ws, 0, empty ? kHeaderBytes : pl.off_agg, s);
+    cudaError_t e = cudaMemsetAsync(ws, 0, kHeaderBytes, s);
     if (e != cudaSuccess) return cuda_fail(e, "workspace reset");
     if (resid_hist) {
         e = cudaMemsetAsync(resid_hist, 0, sizeof(float) * (K + 1), s);
@@ -243,24 +357,26 @@ pararnn_status pararnn_newton_forward(pararnn_cell cell, int64_t B, int64_t T, i
     prm.T = T;
     prm.D = D;
     prm.K = Keff;
+    prm.ticket = reinterpret_cast<unsigned*>(ws) + 1;
     prm.lb.status = reinterpret_cast<unsigned*>(ws);
-    prm.lb.flags = reinterpret_cast<unsigned*>(ws + pl.off_flags);
-    prm.lb.agg = reinterpret_cast<float*>(ws + pl.off_agg);
-    prm.lb.inc = reinterpret_cast<float*>(ws + pl.off_inc);
+    prm.lb.agg = reinterpret_cast<word_t*>(ws + pl.off_agg);
+    prm.lb.inc = reinterpret_cast<word_t*>(ws + pl.off_inc);
     prm.lb.nGroups = pl.nGroups;
     prm.lb.nSlots = pl.g.nSlots;
+    prm.lb.epoch = next_epoch();
     prm.lb.timeout_ns = kWaitLimitNs;
 
+    typedef __nv_bfloat16 bf16;
     const bool bf = px_dtype == PARARNN_BF16;
     if (cell == PARARNN_CELL_LINEAR) {
-        if (vec) st = bf ? launch_fwd<CellLinear, __nv_bfloat16, FwdLinV>(pl, prm, s) : launch_fwd<CellLinear, float, FwdLinV>(pl, prm, s);
-        else st = bf ? launch_fwd<CellLinear, __nv_bfloat16, FwdLinS>(pl, prm, s) : launch_fwd<CellLinear, float, FwdLinS>(pl, prm, s);
+        if (tma) st = bf ? launch_fwd<CellLinear, bf16, FwdLinT<bf16>>(pl, prm, s) : launch_fwd<CellLinear, float, FwdLinT<float>>(pl, prm, s);
+        else st = bf ? launch_fwd<CellLinear, bf16, FwdLinS<bf16>>(pl, prm, s) : launch_fwd<CellLinear, float, FwdLinS<float>>(pl, prm, s);
     } else if (cell == PARARNN_CELL_DIAG_GRU) {
-        if (vec) st = bf ? launch_fwd<CellGRU, __nv_bfloat16, FwdGruV>(pl, prm, s) : launch_fwd<CellGRU, float, FwdGruV>(pl, prm, s);
-        else st = bf ? launch_fwd<CellGRU, __nv_bfloat16, FwdGruS>(pl, prm, s) : launch_fwd<CellGRU, float, FwdGruS>(pl, prm, s);
+        if (tma) st = bf ? launch_fwd<CellGRU, bf16, FwdGruT<bf16>>(pl, prm, s) : launch_fwd<CellGRU, float, FwdGruT<float>>(pl, prm, s);
+        else st = bf ? launch_fwd<CellGRU, bf16, FwdGruS<bf16>>(pl, prm, s) : launch_fwd<CellGRU, float, FwdGruS<float>>(pl, prm, s);
     } else {
-        if (vec) st = bf ? launch_fwd<CellLSTM, __nv_bfloat16, FwdLstmV>(pl, prm, s) : launch_fwd<CellLSTM, float, FwdLstmV>(pl, prm, s);
-        else st = bf ? launch_fwd<CellLSTM, __nv_bfloat16, FwdLstmS>(pl, prm, s) : launch_fwd<CellLSTM, float, FwdLstmS>(pl, prm, s);
+        if (tma) st = bf ? launch_fwd<CellLSTM, bf16, FwdLstmT<bf16>>(pl, prm, s) : launch_fwd<CellLSTM, float, FwdLstmT<float>>(pl, prm, s);
+        else st = bf ? launch_fwd<CellLSTM, bf16, FwdLstmS<bf16>>(pl, prm, s) : launch_fwd<CellLSTM, float, FwdLstmS<float>>(pl, prm, s);
     }
     if (st != PARARNN_OK) return st;
     if (resid_hist && Keff < K) {
@@ -304,13 +420,13 @@ pararnn_status pararnn_newton_backward(pararnn_cell cell, int64_t B, int64_t T, 
         return fail(PARARNN_EINVAL, "dL_da is not device-accessible float memory");
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const bool vec = (D % 4 == 0) && aligned(preacts, 16) && aligned(H, 16) && aligned(dL_dH, 16) &&
-                     aligned(dL_dpx, 16);
-    const Plan pl = make_plan(cell, B, T, D, 1, false, vec);
+    const bool tma = ((D * (int64_t)esz) % 16 == 0) && (D % 4 == 0) && aligned(preacts, 16) && aligned(H, 16) &&
+                     aligned(dL_dH, 16) && aligned(dL_dpx, 16);
+    const Plan pl = make_plan(cell, B, T, D, 1, false, tma);
     if (pl.nTiles >= (int64_t(1) << 31)) return fail(PARARNN_EINVAL, "too many tiles");
 
     char* ws = static_cast<char*>(workspace);
-    cudaError_t e = cudaMemsetAsync(ws, 0, empty ? kHeaderBytes : pl.off_agg, s);
+    cudaError_t e = cudaMemsetAsync(ws, 0, kHeaderBytes, s);
     if (e != cudaSuccess) return cuda_fail(e, "workspace reset");
     if (empty) {
         const int G = pararnn_num_gates(cell);
@@ -338,24 +454,26 @@ pararnn_status pararnn_newton_backward(pararnn_cell cell, int64_t B, int64_t T, 
     prm.B = B;
     prm.T = T;
     prm.D = D;
+    prm.ticket = reinterpret_cast<unsigned*>(ws) + 1;
     prm.lb.status = reinterpret_cast<unsigned*>(ws);
-    prm.lb.flags = reinterpret_cast<unsigned*>(ws + pl.off_flags);
-    prm.lb.agg = reinterpret_cast<float*>(ws + pl.off_agg);
-    prm.lb.inc = reinterpret_cast<float*>(ws + pl.off_inc);
+    prm.lb.agg = reinterpret_cast<word_t*>(ws + pl.off_agg);
+    prm.lb.inc = reinterpret_cast<word_t*>(ws + pl.off_inc);
     prm.lb.nGroups = pl.nGroups;
     prm.lb.nSlots = 1;
+    prm.lb.epoch = next_epoch();
     prm.lb.timeout_ns = kWaitLimitNs;
 
+    typedef __nv_bfloat16 bf16;
     const bool bf = px_dtype == PARARNN_BF16;
     if (cell == PARARNN_CELL_LINEAR) {
-        if (vec) st = bf ? launch_bwd<CellLinear, __nv_bfloat16, BwdLinV>(pl, prm, dL_da, s) : launch_bwd<CellLinear, float, BwdLinV>(pl, prm, dL_da, s);
-        else st = bf ? launch_bwd<CellLinear, __nv_bfloat16, BwdLinS>(pl, prm, dL_da, s) : launch_bwd<CellLinear, float, BwdLinS>(pl, prm, dL_da, s);
+        if (tma) st = bf ? launch_bwd<CellLinear, bf16, BwdLinT<bf16>>(pl, prm, dL_da, s) : launch_bwd<CellLinear, float, BwdLinT<float>>(pl, prm, dL_da, s);
+        else st = bf ? launch_bwd<CellLinear, bf16, BwdLinS<bf16>>(pl, prm, dL_da, s) : launch_bwd<CellLinear, float, BwdLinS<float>>(pl, prm, dL_da, s);
     } else if (cell == PARARNN_CELL_DIAG_GRU) {
-        if (vec) st = bf ? launch_bwd<CellGRU, __nv_bfloat16, BwdGruV>(pl, prm, dL_da, s) : launch_bwd<CellGRU, float, BwdGruV>(pl, prm, dL_da, s);
-        else st = bf ? launch_bwd<CellGRU, __nv_bfloat16, BwdGruS>(pl, prm, dL_da, s) : launch_bwd<CellGRU, float, BwdGruS>(pl, prm, dL_da, s);
+        if (tma) st = bf ? launch_bwd<CellGRU, bf16, BwdGruT<bf16>>(pl, prm, dL_da, s) : launch_bwd<CellGRU, float, BwdGruT<float>>(pl, prm, dL_da, s);
+        else st = bf ? launch_bwd<CellGRU, bf16, BwdGruS<bf16>>(pl, prm, dL_da, s) : launch_bwd<CellGRU, float, BwdGruS<float>>(pl, prm, dL_da, s);
     } else {
-        if (vec) st = bf ? launch_bwd<CellLSTM, __nv_bfloat16, BwdLstmV>(pl, prm, dL_da, s) : launch_bwd<CellLSTM, float, BwdLstmV>(pl, prm, dL_da, s);
-        else st = bf ? launch_bwd<CellLSTM, __nv_bfloat16, BwdLstmS>(pl, prm, dL_da, s) : launch_bwd<CellLSTM, float, BwdLstmS>(pl, prm, dL_da, s);
+        if (tma) st = bf ? launch_bwd<CellLSTM, bf16, BwdLstmT<bf16>>(pl, prm, dL_da, s) : launch_bwd<CellLSTM, float, BwdLstmT<float>>(pl, prm, dL_da, s);
+        else st = bf ? launch_bwd<CellLSTM, bf16, BwdLstmS<bf16>>(pl, prm, dL_da, s) : launch_bwd<CellLSTM, float, BwdLstmS<float>>(pl, prm, dL_da, s);
     }
     return st;
 }
@@ -397,7 +515,7 @@ pararnn_status pararnn_probe_wait_timeout(void* workspace, size_t ws_bytes, uint
     cudaError_t e = cudaMemsetAsync(ws, 0, kHeaderBytes + 256, s);
     if (e != cudaSuccess) return cuda_fail(e, "workspace reset");
     probe_wait_kernel<<<1, 32, 0, s>>>(reinterpret_cast<unsigned*>(ws),
-                                         reinterpret_cast<const unsigned*>(ws + kHeaderBytes), timeout_ns);
+                                         reinterpret_cast<const word_t*>(ws + kHeaderBytes), next_epoch(), timeout_ns);
     e = cudaGetLastError();
     return e == cudaSuccess ? PARARNN_OK : cuda_fail(e, "probe launch");
 }

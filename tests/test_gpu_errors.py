@@ -34,7 +34,7 @@ def test_nonfinite_residual_is_visible(cuda_device):
 
 def test_wait_time_out_ends_cleanly(cuda_device):
     n = binding.pararnn_workspace_bytes(binding.LINEAR, 1, 1, 1, 1)
-    ws = torch.empty(n, dtype=torch.uint8, device=DEV)
+    ws = torch.zeros(n, dtype=torch.uint8, device=DEV)
     st = torch.cuda.current_stream()
     assert binding.pararnn_probe_wait_timeout(ws, n, 20_000_000, st) == binding.OK  # 20 ms
     assert binding.pararnn_status_sync(ws, st) == binding.ETIMEOUT
@@ -49,7 +49,7 @@ def test_host_memory_is_rejected(cuda_device):
     host = np.zeros((1, 8, 3, 8), dtype=np.float32)
     H = torch.empty(1, 8, 1, 8, device=DEV)
     n = binding.pararnn_workspace_bytes(1, 1, 8, 8, 2)
-    ws = torch.empty(n, dtype=torch.uint8, device=DEV)
+    ws = torch.zeros(n, dtype=torch.uint8, device=DEV)
     st = binding.pararnn_newton_forward(1, 1, 8, 8, 0, host.ctypes.data, None, None, 2, H, ws, n, None, None)
     assert st == binding.EINVAL
     assert "device-accessible" in binding.pararnn_last_error()
@@ -59,6 +59,6 @@ def test_misaligned_pointer_is_rejected(cuda_device):
     buf = torch.zeros(1 + 8 * 3 * 8, device=DEV)
     H = torch.empty(1, 8, 1, 8, device=DEV)
     n = binding.pararnn_workspace_bytes(1, 1, 8, 8, 2)
-    ws = torch.empty(n, dtype=torch.uint8, device=DEV)
+    ws = torch.zeros(n, dtype=torch.uint8, device=DEV)
     st = binding.pararnn_newton_forward(1, 1, 8, 8, 0, buf.data_ptr() + 2, None, None, 2, H, ws, n, None, None)
     assert st == binding.EINVAL
