@@ -393,6 +393,9 @@ def run_native(args):
     torch.cuda.set_device(device)
     dist = dist_init("nccl", world)
     w = workloads.WORKLOADS[args.workload]
+    if args.B or args.T or args.D:
+        w = w.with_shape(B=args.B, T=args.T, D=args.D, name="%s@B%dT%dD%d" % (w.name, args.B or w.B, args.T or w.T,
+                                                                           args.D or w.D))
     prob = Problem(w, device, rank_seed(w.seed, rank))
     with ClockSampler(local) as clk:
         ms, fwd_ms, bwd_ms = time_device(prob, args.steps, args.warmup, dist, device)
@@ -407,9 +410,12 @@ def run_native(args):
             "traffic": recorded_traffic("newton_fwd_kernel", w.name),
             "algorithmic_bytes_per_launch": algo, "bytes_per_elem": algo // w.elements,
             "launch_ms": round(fwd_ms, 4)}
-    e2e_ms, h2d, d2h = time_e2e(prob, steps=3)
-    e2e = {"value": w.elements / (e2e_ms / 1e3) * world, "unit": UNIT, "h2d_bytes_per_step": h2d,
-           "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 3)}
+    if args.quick:
+        e2e = None
+    else:
+        e2e_ms, h2d, d2h = time_e2e(prob, steps=3)
+        e2e = {"value": w.elements / (e2e_ms / 1e3) * world, "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 3)}
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
@@ -423,7 +429,7 @@ def run_native(args):
     }
     del prob
     torch.cuda.empty_cache()
-    if rank == 0 and world == 1:
+    if rank == 0 and world == 1 and not args.quick:
         line["cpu_baseline"] = cpu_baseline(w, device, rank_seed(w.seed, rank))
         if not args.no_extra:
             line["workloads"] = extra_workloads([n for n in workloads.WORKLOADS if n != w.name], device, 0)
@@ -493,6 +499,11 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--workload", default=workloads.HEADLINE, choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--no-extra", action="store_true", help="skip the other workloads' lines")
+    ap.add_argument("--quick", action="store_true",
+                    help="device timing only (no e2e, CPU baseline or other workloads): for profiling runs")
+    ap.add_argument("--B", type=int, default=None, help="override the workload's batch (profiling cases)")
+    ap.add_argument("--T", type=int, default=None, help="override the workload's length (profiling cases)")
+    ap.add_argument("--D", type=int, default=None, help="override the workload's channels (profiling cases)")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)
     args.steps = max(1, args.steps)

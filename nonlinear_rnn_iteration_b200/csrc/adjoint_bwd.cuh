@@ -46,10 +46,10 @@ struct BwdSmem {
     alignas(128) PxT px[Sh::NSTAGE][Sh::L][Sh::G][Sh::W];
     alignas(128) float H[Sh::NSTAGE][Sh::L][Sh::S][Sh::W];
     alignas(128) float g[Sh::NSTAGE][Sh::L][Sh::S][Sh::W];
-    float agg[Sh::NSUB][Sh::NA][Sh::W];   // indexed by position in the reverse scan
-    float carry[Sh::NSUB][Sh::S][Sh::W];
+    float wagg[Sh::NWARPS][Sh::NA][Sh::W];       // each warp's composed element
+    float cin[Sh::S][Sh::W];                     // lambda just after the tile (the carry)
     float firstA[Sh::NSUB][Sh::S * Sh::S][Sh::W];  // each sub-chunk's first-row Jacobian
-    float hprev[Sh::S][Sh::W];            // state just before the tile
+    float hprev[Sh::S][Sh::W];                   // state just before the tile
     float w[Sh::G][Sh::W];
     float da[Sh::NSUB][Sh::G][Sh::W];
     uint64_t bar[Sh::NSTAGE];
@@ -80,43 +80,39 @@ __device__ __forceinline__ void issue_bwd_load(const BwdMaps<Sh>* maps, BwdSmem<
 template <class Cell, typename PxT, class Sh>
 __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
     adjoint_bwd_kernel(const __grid_constant__ BwdMaps<Sh> maps, const BwdParams prm) {
-    constexpr int G = Sh::G, S = Sh::S, V = Sh::V, R = Sh::R, NS = Cell::NSENS;
-    constexpr int TPW = Sh::TPW, NSUB = Sh::NSUB, W = Sh::W, L = Sh::L, LC = Sh::LC, NT = Sh::NT;
+    constexpr int G = Sh::G, S = Sh::S, V = Sh::V, R = Sh::R, NS = Cell::NSENS, NW = Sh::NWARPS;
+    constexpr int TPW = Sh::TPW, NSUB = Sh::NSUB, W = Sh::W, L = Sh::L, LC = Sh::LC, NTC = Sh::NTC;
+    constexpr int NSTAGE = Sh::NSTAGE;
     constexpr int CPL = W / 32;
     using SM = BwdSmem<Sh, PxT>;
     extern __shared__ __align__(128) unsigned char smem_raw[];
     SM& sm = *reinterpret_cast<SM*>(smem_raw);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int sub = warp * TPW + lane / LC;
-    const int rs = NSUB - 1 - sub;  // this sub-chunk's position in the reverse scan
-    const int cc = (lane % LC) * V;
+    const bool is_scan = warp == NW;
     const int64_t T = prm.T, D = prm.D;
     const PxT* pxg = static_cast<const PxT*>(prm.px);
 
-    if (tid == 0) {
+    if (is_scan && lane == 0) {
         if constexpr (Sh::kTma) {
 #pragma unroll
-            for (int s = 0; s < Sh::NSTAGE; ++s) mbar_init(&sm.bar[s], 1);
+            for (int s = 0; s < NSTAGE; ++s) mbar_init(&sm.bar[s], 1);
             mbar_fence_init();
         }
-        const unsigned t = atomicAdd(prm.ticket, 1u);
-        sm.ticket[0] = t;
-        if constexpr (Sh::kTma)
-            if (t < prm.nTiles) issue_bwd_load<Cell, PxT, Sh>(&maps, sm, prm, t, 0);
+#pragma unroll
+        for (int s = 0; s < NSTAGE - 1; ++s) {
+            const unsigned t = atomicAdd(prm.ticket, 1u);
+            sm.ticket[s] = t;
+            if constexpr (Sh::kTma)
+                if (t < prm.nTiles) issue_bwd_load<Cell, PxT, Sh>(&maps, sm, prm, t, s);
+        }
     }
-    __syncthreads();
+    block_sync();
 
     for (int it = 0;; ++it) {
-        const int st = it % Sh::NSTAGE;
+        const int st = it % NSTAGE;
         const unsigned tile_u = sm.ticket[st];
         if (tile_u >= prm.nTiles) break;
-        if (tid == 0) {
-            const unsigned t2 = atomicAdd(prm.ticket, 1u);
-            sm.ticket[(it + 1) % Sh::NSTAGE] = t2;
-            if constexpr (Sh::kTma)
-                if (t2 < prm.nTiles) issue_bwd_load<Cell, PxT, Sh>(&maps, sm, prm, t2, (it + 1) % Sh::NSTAGE);
-        }
         const int64_t tile = tile_u;
         const int64_t pos = tile / prm.lb.nGroups;
         const int64_t gid = tile - pos * prm.lb.nGroups;
@@ -124,227 +120,261 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
         const int64_t b = gid / prm.nCG;
         const int64_t d0 = (gid - b * prm.nCG) * W;
         const int64_t t0 = chunk * L;
-        const int64_t tb = t0 + (int64_t)sub * R;
-        const bool cvalid = d0 + cc < D;
 
-        for (int i = tid; i < G * W; i += NT) {
-            const int g = i / W, c = i - (i / W) * W;
-            sm.w[g][c] = (prm.w && d0 + c < D) ? __ldg(prm.w + g * D + d0 + c) : 0.0f;
-        }
-        if (tid < W) {
-            const int64_t d = d0 + tid;
-#pragma unroll
-            for (int s = 0; s < S; ++s) {
-                float x = 0.0f;
-                if (d < D) {
-                    if (t0 > 0) x = prm.H[((b * T + t0 - 1) * S + s) * D + d];
-                    else if (prm.h0) x = prm.h0[(b * S + s) * D + d];
-                }
-                sm.hprev[s][tid] = x;
+        if (is_scan) {
+            // ================= scan warp =================
+            if (lane == 0) {
+                const int sn = (it + NSTAGE - 1) % NSTAGE;
+                const unsigned prev_t = sm.ticket[(it + NSTAGE - 2) % NSTAGE];
+                unsigned t2 = prev_t;
+                if (prev_t < prm.nTiles) t2 = atomicAdd(prm.ticket, 1u);
+                sm.ticket[sn] = t2;
+                if constexpr (Sh::kTma)
+                    if (t2 < prm.nTiles && prev_t < prm.nTiles) issue_bwd_load<Cell, PxT, Sh>(&maps, sm, prm, t2, sn);
             }
-        }
-        if constexpr (Sh::kTma) {
-            Deadline dl;
-            while (!mbar_try_wait(&sm.bar[st], (it / Sh::NSTAGE) & 1)) {
-                if (dl.expired(prm.lb.timeout_ns)) {
-                    if (tid == 0) atomicOr(prm.lb.status, kStatusTimeout);
-                    break;
-                }
-            }
-        } else {
-            for (int i = tid; i < L * G * W; i += NT) {
-                const int row = i / (G * W), rem = i - row * (G * W), g = rem / W, c = rem - g * W;
-                const int64_t t = t0 + row, d = d0 + c;
-                sm.px[st][row][g][c] = (t < T && d < D) ? pxg[((b * T + t) * G + g) * D + d] : PxT(0.0f);
-            }
-            for (int i = tid; i < L * S * W; i += NT) {
-                const int row = i / (S * W), rem = i - row * (S * W), s = rem / W, c = rem - s * W;
-                const int64_t t = t0 + row, d = d0 + c;
-                const bool ok = t < T && d < D;
-                sm.H[st][row][s][c] = ok ? prm.H[((b * T + t) * S + s) * D + d] : 0.0f;
-                sm.g[st][row][s][c] = ok ? prm.dLdH[((b * T + t) * S + s) * D + d] : 0.0f;
-            }
-        }
-        __syncthreads();
-
-        // ---- linearisation at (h_{t-1}, x_t) for every row ----
-        float jA[R][S * S][V], sens[R][NS][V];
-#pragma unroll
-        for (int r = 0; r < R; ++r)
-#pragma unroll
-            for (int v = 0; v < V; ++v) {
-                float pv[G], wv[G], spv[S], A[S * S], se[NS];
-                const int row = sub * R + r;
-#pragma unroll
-                for (int g = 0; g < G; ++g) {
-                    pv[g] = PxTraits<PxT>::cvt(sm.px[st][row][g][cc + v]);
-                    wv[g] = sm.w[g][cc + v];
-                }
-#pragma unroll
-                for (int s = 0; s < S; ++s) spv[s] = row > 0 ? sm.H[st][row - 1][s][cc + v] : sm.hprev[s][cc + v];
-                Cell::bwd(pv, wv, spv, A, se);
-#pragma unroll
-                for (int a = 0; a < S * S; ++a) jA[r][a][v] = A[a];
-#pragma unroll
-                for (int n = 0; n < NS; ++n) sens[r][n][v] = se[n];
-            }
-#pragma unroll
-        for (int a = 0; a < S * S; ++a)
-#pragma unroll
-            for (int v = 0; v < V; ++v) sm.firstA[sub][a][cc + v] = jA[0][a][v];
-        // the last sub-chunk also needs A at the first row of the next tile
-        float nextA[S * S][V];
-        if (sub == NSUB - 1) {
-            const int64_t tn = t0 + L;
-#pragma unroll
-            for (int v = 0; v < V; ++v) {
-                float A[S * S];
-#pragma unroll
-                for (int a = 0; a < S * S; ++a) A[a] = 0.0f;
-                if (tn < T && cvalid) {
-                    float pv[G], wv[G], spv[S], se[NS];
-#pragma unroll
-                    for (int g = 0; g < G; ++g) {
-                        pv[g] = PxTraits<PxT>::cvt(pxg[((b * T + tn) * G + g) * D + d0 + cc + v]);
-                        wv[g] = sm.w[g][cc + v];
-                    }
-#pragma unroll
-                    for (int s = 0; s < S; ++s) spv[s] = sm.H[st][L - 1][s][cc + v];
-                    Cell::bwd(pv, wv, spv, A, se);
-                }
-#pragma unroll
-                for (int a = 0; a < S * S; ++a) nextA[a][v] = A[a];
-            }
-        }
-        __syncthreads();
-
-        // ---- reverse-scan elements (M_t, g_t), M_t = A_{t+1}^T ----
-        float eM[R][S * S][V];
-#pragma unroll
-        for (int r = 0; r < R; ++r)
-#pragma unroll
-            for (int v = 0; v < V; ++v) {
-                const int64_t t = tb + r;
-                float A[S * S];
-#pragma unroll
-                for (int a = 0; a < S * S; ++a) {
-                    if (r + 1 < R) A[a] = jA[r + 1][a][v];
-                    else if (sub + 1 < NSUB) A[a] = sm.firstA[sub + 1][a][cc + v];
-                    else A[a] = nextA[a][v];
-                }
-                const bool has_next = (t + 1 < T) && cvalid;
-                const bool rvalid = (t < T) && cvalid;
-#pragma unroll
-                for (int i = 0; i < S; ++i)
-#pragma unroll
-                    for (int m = 0; m < S; ++m) {
-                        float val = has_next ? A[m * S + i] : 0.0f;  // transpose
-                        if (!rvalid) val = (i == m) ? 1.0f : 0.0f;     // past the end: identity
-                        eM[r][i * S + m][v] = val;
-                    }
-            }
-#pragma unroll
-        for (int v = 0; v < V; ++v) {
-            Elem<S> acc;
-            elem_identity<S>(acc);
-#pragma unroll
-            for (int r = R - 1; r >= 0; --r) {
-                float M[S * S], gv[S];
-#pragma unroll
-                for (int a = 0; a < S * S; ++a) M[a] = eM[r][a][v];
-#pragma unroll
-                for (int s = 0; s < S; ++s) gv[s] = (tb + r < T) ? sm.g[st][sub * R + r][s][cc + v] : 0.0f;
-                compose_after<S>(M, gv, acc);
-            }
-#pragma unroll
-            for (int a = 0; a < S * S; ++a) sm.agg[rs][a][cc + v] = acc.A[a];
-#pragma unroll
-            for (int s = 0; s < S; ++s) sm.agg[rs][S * S + s][cc + v] = acc.b[s];
-        }
-        __syncthreads();
-
-        if (warp == 0) {
-            float zero[CPL][S], carry[CPL][S];
+            float zero[CPL][S];
 #pragma unroll
             for (int j = 0; j < CPL; ++j)
 #pragma unroll
                 for (int s = 0; s < S; ++s) zero[j][s] = 0.0f;  // lambda_T = 0
-            tile_scan_step<S, W, NSUB, Sh::P>(prm.lb, tile, pos, 0, lane, sm.agg, sm.carry, zero, carry);
-        }
-        __syncthreads();
+            block_sync();  // tile set up
+            block_sync();  // first-row Jacobians shared
+            block_sync();  // warp totals ready
+            tile_lookback<S, W, NW, Sh::P, true>(prm.lb, tile, pos, 0, lane, sm.wagg, zero, sm.cin);
+            block_sync();  // carry ready
+            block_sync();  // per-sub-chunk dL/da partials ready
+        } else {
+            // ================= compute warps =================
+            const int sub = warp * TPW + lane / LC;
+            const int cc = (lane % LC) * V;
+            const int64_t tb = t0 + (int64_t)sub * R;
+            const bool cvalid = d0 + cc < D;
 
-        // ---- lambda and the gradient epilogue ----
-        float da_acc[G][V];
+            for (int i = tid; i < G * W; i += NTC) {
+                const int g = i / W, c = i - (i / W) * W;
+                sm.w[g][c] = (prm.w && d0 + c < D) ? __ldg(prm.w + g * D + d0 + c) : 0.0f;
+            }
+            if (tid < W) {
+                const int64_t d = d0 + tid;
 #pragma unroll
-        for (int g = 0; g < G; ++g)
-#pragma unroll
-            for (int v = 0; v < V; ++v) da_acc[g][v] = 0.0f;
-        float outp[R][G][V];
-        bool bad = false;
-#pragma unroll
-        for (int v = 0; v < V; ++v) {
-            float x[S];
-#pragma unroll
-            for (int s = 0; s < S; ++s) x[s] = sm.carry[rs][s][cc + v];
-#pragma unroll
-            for (int r = R - 1; r >= 0; --r) {
-                const bool rvalid = (tb + r < T) && cvalid;
-                float M[S * S], gv[S], y[S];
-#pragma unroll
-                for (int a = 0; a < S * S; ++a) M[a] = eM[r][a][v];
-#pragma unroll
-                for (int s = 0; s < S; ++s) gv[s] = (tb + r < T) ? sm.g[st][sub * R + r][s][cc + v] : 0.0f;
-                apply<S>(M, gv, x, y);
-#pragma unroll
-                for (int s = 0; s < S; ++s) x[s] = y[s];
-                float se[NS], dp[G], da[G];
-#pragma unroll
-                for (int n = 0; n < NS; ++n) se[n] = sens[r][n][v];
-                Cell::grads(se, x, dp, da);
-#pragma unroll
-                for (int g2 = 0; g2 < G; ++g2) {
-                    outp[r][g2][v] = dp[g2];
-                    if (rvalid) {
-                        da_acc[g2][v] += da[g2];
-                        bad |= !isfinite(dp[g2]);
+                for (int s = 0; s < S; ++s) {
+                    float x = 0.0f;
+                    if (d < D) {
+                        if (t0 > 0) x = prm.H[((b * T + t0 - 1) * S + s) * D + d];
+                        else if (prm.h0) x = prm.h0[(b * S + s) * D + d];
+                    }
+                    sm.hprev[s][tid] = x;
+                }
+            }
+            if constexpr (Sh::kTma) {
+                Deadline dl;
+                while (!mbar_try_wait(&sm.bar[st], (it / NSTAGE) & 1)) {
+                    if (dl.expired(prm.lb.timeout_ns)) {
+                        if (tid == 0) atomicOr(prm.lb.status, kStatusTimeout);
+                        break;
                     }
                 }
-                if (r == 0 && tb == 0 && rvalid && prm.dLdh0) {
-                    // dL/dh0 = A_0^T lambda_0, A_0 at (h0, x_0)
+            } else {
+                for (int i = tid; i < L * G * W; i += NTC) {
+                    const int row = i / (G * W), rem = i - row * (G * W), g = rem / W, c = rem - g * W;
+                    const int64_t t = t0 + row, d = d0 + c;
+                    sm.px[st][row][g][c] = (t < T && d < D) ? pxg[((b * T + t) * G + g) * D + d] : PxT(0.0f);
+                }
+                for (int i = tid; i < L * S * W; i += NTC) {
+                    const int row = i / (S * W), rem = i - row * (S * W), s = rem / W, c = rem - s * W;
+                    const int64_t t = t0 + row, d = d0 + c;
+                    const bool ok = t < T && d < D;
+                    sm.H[st][row][s][c] = ok ? prm.H[((b * T + t) * S + s) * D + d] : 0.0f;
+                    sm.g[st][row][s][c] = ok ? prm.dLdH[((b * T + t) * S + s) * D + d] : 0.0f;
+                }
+            }
+            block_sync();  // tile set up
+
+            // ---- linearisation at (h_{t-1}, x_t) for every row ----
+            float jA[R][S * S][V], sens[R][NS][V];
 #pragma unroll
-                    for (int i = 0; i < S; ++i) {
-                        float acc = 0.0f;
+            for (int r = 0; r < R; ++r) {
+                const int row = sub * R + r;
+                float pv[G][V], hv[S][V];
 #pragma unroll
-                        for (int m = 0; m < S; ++m) acc = __fmaf_rn(jA[0][m * S + i][v], x[m], acc);
-                        prm.dLdh0[(b * S + i) * D + d0 + cc + v] = acc;
+                for (int g = 0; g < G; ++g) lds_row<V>(&sm.px[st][row][g][cc], pv[g]);
+#pragma unroll
+                for (int s = 0; s < S; ++s) lds_row<V>(row > 0 ? &sm.H[st][row - 1][s][cc] : &sm.hprev[s][cc], hv[s]);
+#pragma unroll
+                for (int v = 0; v < V; ++v) {
+                    float pg[G], wv[G], spv[S], A[S * S], se[NS];
+#pragma unroll
+                    for (int g = 0; g < G; ++g) {
+                        pg[g] = pv[g][v];
+                        wv[g] = sm.w[g][cc + v];
+                    }
+#pragma unroll
+                    for (int s = 0; s < S; ++s) spv[s] = hv[s][v];
+                    Cell::bwd(pg, wv, spv, A, se);
+#pragma unroll
+                    for (int a = 0; a < S * S; ++a) jA[r][a][v] = A[a];
+#pragma unroll
+                    for (int n = 0; n < NS; ++n) sens[r][n][v] = se[n];
+                }
+            }
+#pragma unroll
+            for (int a = 0; a < S * S; ++a)
+#pragma unroll
+                for (int v = 0; v < V; ++v) sm.firstA[sub][a][cc + v] = jA[0][a][v];
+            // the last sub-chunk also needs A at the first row of the next tile
+            float nextA[S * S][V];
+            if (sub == NSUB - 1) {
+                const int64_t tn = t0 + L;
+#pragma unroll
+                for (int v = 0; v < V; ++v) {
+                    float A[S * S];
+#pragma unroll
+                    for (int a = 0; a < S * S; ++a) A[a] = 0.0f;
+                    if (tn < T && cvalid) {
+                        float pv[G], wv[G], spv[S], se[NS];
+#pragma unroll
+                        for (int g = 0; g < G; ++g) {
+                            pv[g] = PxTraits<PxT>::cvt(pxg[((b * T + tn) * G + g) * D + d0 + cc + v]);
+                            wv[g] = sm.w[g][cc + v];
+                        }
+#pragma unroll
+                        for (int s = 0; s < S; ++s) spv[s] = sm.H[st][L - 1][s][cc + v];
+                        Cell::bwd(pv, wv, spv, A, se);
+                    }
+#pragma unroll
+                    for (int a = 0; a < S * S; ++a) nextA[a][v] = A[a];
+                }
+            }
+            block_sync();  // first-row Jacobians shared
+
+            // ---- reverse-scan elements (M_t, g_t), M_t = A_{t+1}^T ----
+            float eM[R][S * S][V];
+#pragma unroll
+            for (int r = 0; r < R; ++r)
+#pragma unroll
+                for (int v = 0; v < V; ++v) {
+                    const int64_t t = tb + r;
+                    float A[S * S];
+#pragma unroll
+                    for (int a = 0; a < S * S; ++a) {
+                        if (r + 1 < R) A[a] = jA[r + 1][a][v];
+                        else if (sub + 1 < NSUB) A[a] = sm.firstA[sub + 1][a][cc + v];
+                        else A[a] = nextA[a][v];
+                    }
+                    const bool has_next = (t + 1 < T) && cvalid;
+                    const bool rvalid = (t < T) && cvalid;
+#pragma unroll
+                    for (int i = 0; i < S; ++i)
+#pragma unroll
+                        for (int m = 0; m < S; ++m) {
+                            float val = has_next ? A[m * S + i] : 0.0f;  // transpose
+                            if (!rvalid) val = (i == m) ? 1.0f : 0.0f;     // past the end: identity
+                            eM[r][i * S + m][v] = val;
+                        }
+                }
+            ElemV<S, V> mine, excl, pre;
+            float gr[R][S][V];
+#pragma unroll
+            for (int r = 0; r < R; ++r)
+#pragma unroll
+                for (int s = 0; s < S; ++s) {
+                    lds_row<V>(&sm.g[st][sub * R + r][s][cc], gr[r][s]);
+                    if (tb + r >= T)
+#pragma unroll
+                        for (int v = 0; v < V; ++v) gr[r][s][v] = 0.0f;
+                }
+#pragma unroll
+            for (int v = 0; v < V; ++v) {
+                elem_identity<S>(mine.e[v]);
+#pragma unroll
+                for (int r = R - 1; r >= 0; --r) {
+                    float M[S * S], gv[S];
+#pragma unroll
+                    for (int a = 0; a < S * S; ++a) M[a] = eM[r][a][v];
+#pragma unroll
+                    for (int s = 0; s < S; ++s) gv[s] = gr[r][s][v];
+                    compose_after<S>(M, gv, mine.e[v]);
+                }
+            }
+            warp_prefix<S, V, LC, W, NW, true>(mine, excl, warp, lane, sm.wagg);
+            block_sync();  // warp totals ready
+            sub_prefix<S, V, LC, W, NW, true>(excl, warp, lane, sm.wagg, pre);
+            block_sync();  // carry ready
+
+            // ---- lambda and the gradient epilogue ----
+            float da_acc[G][V];
+#pragma unroll
+            for (int g = 0; g < G; ++g)
+#pragma unroll
+                for (int v = 0; v < V; ++v) da_acc[g][v] = 0.0f;
+            float outp[R][G][V];
+            bool bad = false;
+#pragma unroll
+            for (int v = 0; v < V; ++v) {
+                float x[S], cv[S];
+#pragma unroll
+                for (int s = 0; s < S; ++s) cv[s] = sm.cin[s][cc + v];
+                apply<S>(pre.e[v].A, pre.e[v].b, cv, x);
+#pragma unroll
+                for (int r = R - 1; r >= 0; --r) {
+                    const bool rvalid = (tb + r < T) && cvalid;
+                    float M[S * S], gv[S], y[S];
+#pragma unroll
+                    for (int a = 0; a < S * S; ++a) M[a] = eM[r][a][v];
+#pragma unroll
+                    for (int s = 0; s < S; ++s) gv[s] = gr[r][s][v];
+                    apply<S>(M, gv, x, y);
+#pragma unroll
+                    for (int s = 0; s < S; ++s) x[s] = y[s];
+                    float se[NS], dp[G], da[G];
+#pragma unroll
+                    for (int n = 0; n < NS; ++n) se[n] = sens[r][n][v];
+                    Cell::grads(se, x, dp, da);
+#pragma unroll
+                    for (int g2 = 0; g2 < G; ++g2) {
+                        outp[r][g2][v] = dp[g2];
+                        if (rvalid) {
+                            da_acc[g2][v] += da[g2];
+                            bad |= !isfinite(dp[g2]);
+                        }
+                    }
+                    if (r == 0 && tb == 0 && rvalid && prm.dLdh0) {
+                        // dL/dh0 = A_0^T lambda_0, A_0 at (h0, x_0)
+#pragma unroll
+                        for (int i = 0; i < S; ++i) {
+                            float acc = 0.0f;
+#pragma unroll
+                            for (int m = 0; m < S; ++m) acc = __fmaf_rn(jA[0][m * S + i][v], x[m], acc);
+                            prm.dLdh0[(b * S + i) * D + d0 + cc + v] = acc;
+                        }
                     }
                 }
             }
-        }
 #pragma unroll
-        for (int r = 0; r < R; ++r) {
-            const int64_t t = tb + r;
-            if (t < T && cvalid) {
+            for (int r = 0; r < R; ++r) {
+                const int64_t t = tb + r;
+                if (t < T && cvalid) {
 #pragma unroll
-                for (int g = 0; g < G; ++g) store_row<V>(prm.dLdpx + ((b * T + t) * G + g) * D + d0 + cc, outp[r][g]);
+                    for (int g = 0; g < G; ++g) store_row<V>(prm.dLdpx + ((b * T + t) * G + g) * D + d0 + cc, outp[r][g]);
+                }
             }
-        }
-        if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(prm.lb.status, kStatusNonFinite);
+            if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(prm.lb.status, kStatusNonFinite);
 
-        // ---- per-tile dL/da partial, summed over sub-chunks in a fixed order ----
+            // ---- per-tile dL/da partial, summed over sub-chunks in a fixed order ----
 #pragma unroll
-        for (int g = 0; g < G; ++g)
+            for (int g = 0; g < G; ++g)
 #pragma unroll
-            for (int v = 0; v < V; ++v) sm.da[sub][g][cc + v] = da_acc[g][v];
-        __syncthreads();
-        for (int i = tid; i < G * W; i += NT) {
-            const int g = i / W, ch = i - (i / W) * W;
-            float acc = 0.0f;
+                for (int v = 0; v < V; ++v) sm.da[sub][g][cc + v] = da_acc[g][v];
+            block_sync();  // per-sub-chunk dL/da partials ready
+            for (int i = tid; i < G * W; i += NTC) {
+                const int g = i / W, ch = i - (i / W) * W;
+                float acc = 0.0f;
 #pragma unroll 4
-            for (int sb = 0; sb < NSUB; ++sb) acc += sm.da[sb][g][ch];
-            prm.part[(tile * G + g) * W + ch] = acc;
+                for (int sb = 0; sb < NSUB; ++sb) acc += sm.da[sb][g][ch];
+                prm.part[(tile * G + g) * W + ch] = acc;
+            }
         }
-        __syncthreads();  // stage st, the ticket slot and the shared partials are free again
+        block_sync();  // stage st, the ticket slot and the shared partials are free again
     }
 }
 

@@ -69,6 +69,39 @@ __device__ __forceinline__ void load_row(const __nv_bfloat16* p, float (&out)[V]
     }
 }
 
+// Shared-memory row reads of V consecutive values (one vector access per lane).
+template <int V>
+__device__ __forceinline__ void lds_row(const float* p, float (&out)[V]) {
+    if constexpr (V == 4) {
+        const float4 v = *reinterpret_cast<const float4*>(p);
+        out[0] = v.x; out[1] = v.y; out[2] = v.z; out[3] = v.w;
+    } else if constexpr (V == 2) {
+        const float2 v = *reinterpret_cast<const float2*>(p);
+        out[0] = v.x; out[1] = v.y;
+    } else {
+#pragma unroll
+        for (int i = 0; i < V; ++i) out[i] = p[i];
+    }
+}
+
+template <int V>
+__device__ __forceinline__ void lds_row(const __nv_bfloat16* p, float (&out)[V]) {
+    if constexpr (V == 4) {
+        const uint2 v = *reinterpret_cast<const uint2*>(p);
+        out[0] = __uint_as_float(v.x << 16);
+        out[1] = __uint_as_float(v.x & 0xffff0000u);
+        out[2] = __uint_as_float(v.y << 16);
+        out[3] = __uint_as_float(v.y & 0xffff0000u);
+    } else if constexpr (V == 2) {
+        const unsigned v = *reinterpret_cast<const unsigned*>(p);
+        out[0] = __uint_as_float(v << 16);
+        out[1] = __uint_as_float(v & 0xffff0000u);
+    } else {
+#pragma unroll
+        for (int i = 0; i < V; ++i) out[i] = __bfloat162float(p[i]);
+    }
+}
+
 template <int V>
 __device__ __forceinline__ void store_row(float* p, const float (&v)[V]) {
     if constexpr (V == 4) {
@@ -86,6 +119,11 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
     return t;
 }
+
+// Block-wide barrier usable from warp-uniform divergent code paths (the
+// compute warps and the scan warp arrive at it from different code); it
+// orders shared- and global-memory accesses like __syncthreads.
+__device__ __forceinline__ void block_sync() { asm volatile("bar.sync 0;" ::: "memory"); }
 
 // ---- numerics --------------------------------------------------------------
 

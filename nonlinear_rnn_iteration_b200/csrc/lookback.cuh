@@ -219,28 +219,121 @@ __device__ void lookback_carry(const LookbackCtx& cx, int64_t tile, int64_t dist
         for (int s = 0; s < S; ++s) carry[j][s] = 0.0f;
 }
 
-// Warp 0's work between two block barriers of one scan step: compose the
-// NSUB sub-chunk elements (s_agg, in scan order) into the tile's element,
-// publish it, find the carry, publish the state after the tile, and write
-// each sub-chunk's carry-in to s_carry.  Returns the carry into the tile.
-template <int S, int W, int NSUB, int P>
-__device__ __forceinline__ void tile_scan_step(const LookbackCtx& cx, int64_t tile, int64_t pos, int slot, int lane,
-                                               const float (&s_agg)[NSUB][S * S + S][W], float (&s_carry)[NSUB][S][W],
-                                               const float (&first_carry)[W / 32][S], float (&carry_out)[W / 32][S]) {
+// ---- the block-level part of one scan step --------------------------------
+// Thread (warp w, lane l) owns sub-chunk sub = w * TPW + l / LC of the tile
+// and the V channels cc .. cc+V-1, cc = (l % LC) * V.  Scan order is time
+// order (forward) or reverse time order (backward).
+
+// A scan element of V channels held by one thread.
+template <int S, int V>
+struct ElemV {
+    Elem<S> e[V];
+};
+
+template <int S>
+__device__ __forceinline__ Elem<S> shfl_elem(const Elem<S>& x, int src_lane_delta, bool up) {
+    Elem<S> y;
+#pragma unroll
+    for (int a = 0; a < S * S; ++a)
+        y.A[a] = up ? __shfl_up_sync(0xffffffffu, x.A[a], src_lane_delta) : __shfl_down_sync(0xffffffffu, x.A[a], src_lane_delta);
+#pragma unroll
+    for (int s = 0; s < S; ++s)
+        y.b[s] = up ? __shfl_up_sync(0xffffffffu, x.b[s], src_lane_delta) : __shfl_down_sync(0xffffffffu, x.b[s], src_lane_delta);
+    return y;
+}
+
+// acc <- x o acc
+template <int S>
+__device__ __forceinline__ void compose_elem(const Elem<S>& x, Elem<S>& acc) {
+    compose_after<S>(x.A, x.b, acc);
+}
+
+// Step 1 (all threads, between the local composition and the first barrier):
+// scan the TPW sub-chunks of each warp with shuffles.  Returns in `excl` the
+// composition of the sub-chunks before this one inside its warp (identity for
+// the first), and writes each warp's total to wagg[w] (by the lanes of the
+// warp's last sub-chunk in scan order).
+template <int S, int V, int LC, int W, int NW, bool kReverse>
+__device__ __forceinline__ void warp_prefix(const ElemV<S, V>& mine, ElemV<S, V>& excl, int warp, int lane,
+                                            float (&wagg)[NW][S * S + S][W]) {
+    constexpr int TPW = 32 / LC;
+    const int q = lane / LC;                          // sub-chunk index inside the warp, time order
+    const int qs = kReverse ? (TPW - 1 - q) : q;      // ... in scan order
+    const int cc = (lane % LC) * V;
+#pragma unroll
+    for (int v = 0; v < V; ++v) {
+        Elem<S> incl = mine.e[v];
+#pragma unroll
+        for (int d = 1; d < TPW; d *= 2) {
+            // the sub-chunk d places earlier in scan order sits d*LC lanes below
+            // (forward) or above (reverse)
+            const Elem<S> other = shfl_elem<S>(incl, d * LC, !kReverse);
+            if (qs >= d) {
+                Elem<S> t = other;   // incl <- incl o other (other first)
+                compose_elem<S>(incl, t);
+                incl = t;
+            }
+        }
+        Elem<S> ex = shfl_elem<S>(incl, LC, !kReverse);
+        if (qs == 0) elem_identity<S>(ex);
+        excl.e[v] = ex;
+        if (qs == TPW - 1) {
+#pragma unroll
+            for (int a = 0; a < S * S; ++a) wagg[warp][a][cc + v] = incl.A[a];
+#pragma unroll
+            for (int s = 0; s < S; ++s) wagg[warp][S * S + s][cc + v] = incl.b[s];
+        }
+    }
+}
+
+// Step 2a (all threads, after the first barrier): the composition of every
+// earlier warp (scan order) followed by the earlier sub-chunks of this warp:
+// the element that maps the tile's carry-in to this sub-chunk's carry-in.
+template <int S, int V, int LC, int W, int NW, bool kReverse>
+__device__ __forceinline__ void sub_prefix(const ElemV<S, V>& excl, int warp, int lane,
+                                           const float (&wagg)[NW][S * S + S][W], ElemV<S, V>& pre) {
+    const int cc = (lane % LC) * V;
+    const int ws = kReverse ? (NW - 1 - warp) : warp;  // this warp's position in scan order
+#pragma unroll
+    for (int v = 0; v < V; ++v) {
+        Elem<S> acc;
+        elem_identity<S>(acc);
+        for (int k = 0; k < ws; ++k) {
+            const int wk = kReverse ? (NW - 1 - k) : k;
+            float A[S * S], b[S];
+#pragma unroll
+            for (int a = 0; a < S * S; ++a) A[a] = wagg[wk][a][cc + v];
+#pragma unroll
+            for (int s = 0; s < S; ++s) b[s] = wagg[wk][S * S + s][cc + v];
+            compose_after<S>(A, b, acc);
+        }
+        compose_elem<S>(excl.e[v], acc);
+        pre.e[v] = acc;
+    }
+}
+
+// Step 2b (warp 0, after the first barrier): compose the warp totals into
+// the tile's element, publish it, find the carry by look-back, publish the
+// state after the tile, and write the carry-in to cin.
+template <int S, int W, int NW, int P, bool kReverse>
+__device__ __forceinline__ void tile_lookback(const LookbackCtx& cx, int64_t tile, int64_t pos, int slot, int lane,
+                                              const float (&wagg)[NW][S * S + S][W],
+                                              const float (&first_carry)[W / 32][S], float (&cin)[S][W]) {
     constexpr int NA = S * S + S;
     constexpr int CPL = W / 32;
     Elem<S> tot[CPL];
 #pragma unroll
     for (int j = 0; j < CPL; ++j) elem_identity<S>(tot[j]);
-#pragma unroll 4
-    for (int sb = 0; sb < NSUB; ++sb) {
+#pragma unroll
+    for (int k = 0; k < NW; ++k) {
+        const int wk = kReverse ? (NW - 1 - k) : k;
 #pragma unroll
         for (int j = 0; j < CPL; ++j) {
             float A[S * S], b[S];
 #pragma unroll
-            for (int a = 0; a < S * S; ++a) A[a] = s_agg[sb][a][lane + 32 * j];
+            for (int a = 0; a < S * S; ++a) A[a] = wagg[wk][a][lane + 32 * j];
 #pragma unroll
-            for (int s = 0; s < S; ++s) b[s] = s_agg[sb][S * S + s][lane + 32 * j];
+            for (int s = 0; s < S; ++s) b[s] = wagg[wk][S * S + s][lane + 32 * j];
             compose_after<S>(A, b, tot[j]);
         }
     }
@@ -262,33 +355,14 @@ __device__ __forceinline__ void tile_scan_step(const LookbackCtx& cx, int64_t ti
         publish_words<NA, W>(cx.agg + (tile * cx.nSlots + slot) * NA * W, vals, cx.epoch, lane);
         lookback_carry<S, W, P>(cx, tile, pos, slot, lane, carry);
     }
-    {
-        float vals[CPL][S];
+    float vals[CPL][S];
 #pragma unroll
-        for (int j = 0; j < CPL; ++j) apply<S>(tot[j].A, tot[j].b, carry[j], vals[j]);
-        publish_words<S, W>(cx.inc + (tile * cx.nSlots + slot) * S * W, vals, cx.epoch, lane);
-    }
+    for (int j = 0; j < CPL; ++j) apply<S>(tot[j].A, tot[j].b, carry[j], vals[j]);
+    publish_words<S, W>(cx.inc + (tile * cx.nSlots + slot) * S * W, vals, cx.epoch, lane);
 #pragma unroll
-    for (int j = 0; j < CPL; ++j) {
-        float x[S];
+    for (int j = 0; j < CPL; ++j)
 #pragma unroll
-        for (int s = 0; s < S; ++s) x[s] = carry[j][s];
-#pragma unroll 4
-        for (int sb = 0; sb < NSUB; ++sb) {
-            float A[S * S], b[S], y[S];
-#pragma unroll
-            for (int s = 0; s < S; ++s) s_carry[sb][s][lane + 32 * j] = x[s];
-#pragma unroll
-            for (int a = 0; a < S * S; ++a) A[a] = s_agg[sb][a][lane + 32 * j];
-#pragma unroll
-            for (int s = 0; s < S; ++s) b[s] = s_agg[sb][S * S + s][lane + 32 * j];
-            apply<S>(A, b, x, y);
-#pragma unroll
-            for (int s = 0; s < S; ++s) x[s] = y[s];
-        }
-#pragma unroll
-        for (int s = 0; s < S; ++s) carry_out[j][s] = carry[j][s];
-    }
+        for (int s = 0; s < S; ++s) cin[s][lane + 32 * j] = carry[j][s];
 }
 
 }  // namespace pararnn

@@ -1,6 +1,7 @@
 // pararnn_abi.cu -- the C ABI declared in include/pararnn_b200.h: argument
 // checks, workspace layout, choice of tile shape and kernel launches.
 #include <atomic>
+#include <cstdlib>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -31,21 +32,21 @@ pararnn_status cuda_fail(cudaError_t e, const char* what) {
 
 // ---- tile shapes ------------------------------------------------------------
 // FwdShape<Cell, PxT, V channels/thread, LC lanes across channels, warps,
-//          R rows/thread, blocks/SM budget, TMA>
+//          R rows/thread, blocks/SM budget, shared-memory stages, TMA>
 // TMA path (D * element size a multiple of 16 bytes, 16-byte aligned rows):
 // 64 channels per tile.  Element-wise path otherwise: 32 channels per tile.
-template <typename PxT> using FwdLinT = FwdShape<CellLinear, PxT, 4, 16, 8, 4, 2, true>;
-template <typename PxT> using FwdGruT = FwdShape<CellGRU, PxT, 4, 16, 8, 4, 2, true>;
-template <typename PxT> using FwdLstmT = FwdShape<CellLSTM, PxT, 4, 16, 8, 2, 2, true>;
-template <typename PxT> using BwdLinT = FwdShape<CellLinear, PxT, 4, 16, 8, 2, 2, true>;
-template <typename PxT> using BwdGruT = FwdShape<CellGRU, PxT, 4, 16, 8, 2, 2, true>;
-template <typename PxT> using BwdLstmT = FwdShape<CellLSTM, PxT, 2, 32, 8, 2, 1, true>;
-template <typename PxT> using FwdLinS = FwdShape<CellLinear, PxT, 1, 32, 8, 4, 2, false>;
-template <typename PxT> using FwdGruS = FwdShape<CellGRU, PxT, 1, 32, 8, 4, 2, false>;
-template <typename PxT> using FwdLstmS = FwdShape<CellLSTM, PxT, 1, 32, 8, 2, 2, false>;
-template <typename PxT> using BwdLinS = FwdShape<CellLinear, PxT, 1, 32, 8, 2, 2, false>;
-template <typename PxT> using BwdGruS = FwdShape<CellGRU, PxT, 1, 32, 8, 2, 2, false>;
-template <typename PxT> using BwdLstmS = FwdShape<CellLSTM, PxT, 1, 32, 8, 2, 1, false>;
+template <typename PxT> using FwdLinT = FwdShape<CellLinear, PxT, 4, 16, 8, 4, 2, 3, true>;
+template <typename PxT> using FwdGruT = FwdShape<CellGRU, PxT, 4, 16, 8, 4, 2, 2, true>;
+template <typename PxT> using FwdLstmT = FwdShape<CellLSTM, PxT, 4, 16, 8, 2, 2, 2, true>;
+template <typename PxT> using BwdLinT = FwdShape<CellLinear, PxT, 4, 16, 8, 2, 2, 2, true>;
+template <typename PxT> using BwdGruT = FwdShape<CellGRU, PxT, 4, 16, 8, 2, 2, 2, true>;
+template <typename PxT> using BwdLstmT = FwdShape<CellLSTM, PxT, 2, 32, 8, 2, 1, 2, true>;
+template <typename PxT> using FwdLinS = FwdShape<CellLinear, PxT, 1, 32, 8, 4, 2, 2, false>;
+template <typename PxT> using FwdGruS = FwdShape<CellGRU, PxT, 1, 32, 8, 4, 2, 2, false>;
+template <typename PxT> using FwdLstmS = FwdShape<CellLSTM, PxT, 1, 32, 8, 2, 2, 2, false>;
+template <typename PxT> using BwdLinS = FwdShape<CellLinear, PxT, 1, 32, 8, 2, 2, 2, false>;
+template <typename PxT> using BwdGruS = FwdShape<CellGRU, PxT, 1, 32, 8, 2, 2, 2, false>;
+template <typename PxT> using BwdLstmS = FwdShape<CellLSTM, PxT, 1, 32, 8, 2, 1, 2, false>;
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far beyond any legitimate wait
 constexpr int kMaxK = 64;
@@ -181,8 +182,18 @@ pararnn_status make_map(CUtensorMap* map, const void* base, bool bf16, int64_t D
 }
 
 // ---- launches --------------------------------------------------------------
+// PARARNN_LOG=1 in the environment prints each launch's configuration to stderr.
+bool log_enabled() {
+    static const bool on = [] {
+        const char* e = getenv("PARARNN_LOG");
+        return e && *e && *e != '0';
+    }();
+    return on;
+}
+
 template <class Kern>
-pararnn_status persistent_grid(Kern kern, int threads, size_t smem, int64_t nTiles, unsigned& grid) {
+pararnn_status persistent_grid(Kern kern, int threads, size_t smem, int64_t nTiles, unsigned& grid,
+                               const char* what) {
     int dev = 0, sms = 0, per_sm = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -192,6 +203,9 @@ pararnn_status persistent_grid(Kern kern, int threads, size_t smem, int64_t nTil
     if (per_sm < 1) return fail(PARARNN_ECUDA, "kernel does not fit on an SM");
     const int64_t want = (int64_t)sms * per_sm;
     grid = (unsigned)(nTiles < want ? nTiles : want);
+    if (log_enabled())
+        fprintf(stderr, "pararnn: %s grid=%u blocks/SM=%d SMs=%d threads=%d smem=%zu tiles=%lld\n", what, grid,
+                per_sm, sms, threads, smem, (long long)nTiles);
     return PARARNN_OK;
 }
 
@@ -207,17 +221,21 @@ pararnn_status launch_fwd(const Plan& pl, FwdParams prm, cudaStream_t st) {
         if (s != PARARNN_OK) return s;
     }
     const size_t smem = sizeof(FwdSmem<Sh, PxT>);
-    const bool lean = !Cell::kNonlinear && prm.resid == nullptr;
     unsigned grid = 0;
     pararnn_status s;
-    if (lean) {
-        auto kern = newton_fwd_kernel<Cell, PxT, Sh, true>;
-        s = persistent_grid(kern, Sh::NT, smem, pl.nTiles, grid);
-        if (s != PARARNN_OK) return s;
-        kern<<<grid, Sh::NT, smem, st>>>(map, prm);
-    } else {
+    bool launched = false;
+    if constexpr (!Cell::kNonlinear) {
+        if (prm.resid == nullptr) {  // the linear cell with no residual wanted: the lean single scan
+            auto kern = newton_fwd_kernel<Cell, PxT, Sh, true>;
+            s = persistent_grid(kern, Sh::NT, smem, pl.nTiles, grid, "newton_fwd(lean)");
+            if (s != PARARNN_OK) return s;
+            kern<<<grid, Sh::NT, smem, st>>>(map, prm);
+            launched = true;
+        }
+    }
+    if (!launched) {
         auto kern = newton_fwd_kernel<Cell, PxT, Sh, false>;
-        s = persistent_grid(kern, Sh::NT, smem, pl.nTiles, grid);
+        s = persistent_grid(kern, Sh::NT, smem, pl.nTiles, grid, "newton_fwd");
         if (s != PARARNN_OK) return s;
         kern<<<grid, Sh::NT, smem, st>>>(map, prm);
     }
@@ -242,7 +260,7 @@ pararnn_status launch_bwd(const Plan& pl, BwdParams prm, float* dLda, cudaStream
     const size_t smem = sizeof(BwdSmem<Sh, PxT>);
     auto kern = adjoint_bwd_kernel<Cell, PxT, Sh>;
     unsigned grid = 0;
-    pararnn_status s = persistent_grid(kern, Sh::NT, smem, pl.nTiles, grid);
+    pararnn_status s = persistent_grid(kern, Sh::NT, smem, pl.nTiles, grid, "adjoint_bwd");
     if (s != PARARNN_OK) return s;
     kern<<<grid, Sh::NT, smem, st>>>(maps, prm);
     cudaError_t e = cudaGetLastError();
