@@ -54,9 +54,11 @@
  * GPU detects -- a non-finite value in the output, a wait between thread
  * blocks that ran past its time limit -- are recorded in the workspace and
  * returned by pararnn_status_sync().  A CUDA launch or copy failure returns
- * PARARNN_ECUDA.  The library allocates no memory; the only state it keeps
- * between calls is a process-wide call counter that tags the scan carries it
- * leaves in a workspace.  pararnn_last_error() describes the last failure on
+ * PARARNN_ECUDA.  Apart from the fixed scratch array that
+ * pararnn_newton_forward_noalloc uses (part of the library's device image),
+ * the library allocates no memory; the only state it keeps between calls is a
+ * process-wide call counter that tags the scan carries it leaves in a
+ * workspace.  pararnn_last_error() describes the last failure on
  * the calling thread.  Results are deterministic: the same inputs give the same bits,
  * whatever the order in which thread blocks run.
  */
@@ -164,6 +166,32 @@ const char* pararnn_last_error(void);
  * returns; pararnn_status_sync() then reports it.  workspace needs at least
  * pararnn_workspace_bytes(PARARNN_CELL_LINEAR, 1, 1, 1, 1) bytes. */
 pararnn_status pararnn_probe_wait_timeout(void* workspace, size_t ws_bytes, uint64_t timeout_ns, void* stream);
+
+/* The Newton forward for callers that cannot allocate device memory.  (The
+ * ParaRNN pages have no counterpart: this is a deployment convenience.)
+ * Some callers cannot call cudaMalloc when they run the forward -- a host
+ * framework that owns every device allocation through its own pool, a
+ * latency-bound loop that cannot afford cudaMalloc's implicit
+ * synchronisation, a process with a device-memory budget fixed at start-up.
+ * This entry point computes exactly what pararnn_newton_forward computes, with
+ * the same kernels, but keeps its scratch memory (the workspace) in a fixed
+ * 32 MiB array inside the library's device image, so it allocates nothing.
+ * Every GPU that loads the library holds that array until the process exits.
+ *   Arguments are those of pararnn_newton_forward without workspace/ws_bytes.
+ *   wait_status  0: return once launched (device-detected conditions are then
+ *                not reported); non-zero: wait for `stream` and return the
+ *                device status as pararnn_status_sync would.
+ * Problems whose pararnn_workspace_bytes(cell, B, T, D, K) exceeds 32 MiB
+ * return PARARNN_EINVAL with an explanation in pararnn_last_error().  The
+ * first call on a device sets that device up (it looks up the array's device
+ * address and clears the array once, synchronising the device): make that
+ * first call before any stream capture.  All calls share the one array, which
+ * keeps the last call's contents: calls that overlap on the GPU race, so
+ * order them (one stream, or synchronise between them). */
+pararnn_status pararnn_newton_forward_noalloc(pararnn_cell cell, int64_t B, int64_t T, int64_t D,
+                                              pararnn_dtype px_dtype, const void* preacts, const float* diag_w,
+                                              const float* h0, int K, float* H_out, float* resid_hist,
+                                              int wait_status, void* stream);
 
 #ifdef __cplusplus
 }

@@ -36,6 +36,7 @@ SIGNATURES = {
     "pararnn_status_string": (ctypes.c_char_p, [_I]),
     "pararnn_last_error": (ctypes.c_char_p, []),
     "pararnn_probe_wait_timeout": (_I, [_P, _SZ, _U64, _P]),
+    "pararnn_newton_forward_noalloc": (_I, [_I, _I64, _I64, _I64, _I, _P, _P, _P, _I, _P, _P, _I, _P]),
 }
 
 _lib = None
@@ -125,6 +126,12 @@ def pararnn_last_error():
 
 def pararnn_probe_wait_timeout(workspace, ws_bytes, timeout_ns, stream):
     return load().pararnn_probe_wait_timeout(_ptr(workspace), ws_bytes, timeout_ns, _stream(stream))
+
+
+def pararnn_newton_forward_noalloc(cell, B, T, D, px_dtype, preacts, diag_w, h0, K, H_out, resid_hist, wait_status,
+                                   stream):
+    return load().pararnn_newton_forward_noalloc(cell, B, T, D, px_dtype, _ptr(preacts), _ptr(diag_w), _ptr(h0), K,
+                                                 _ptr(H_out), _ptr(resid_hist), int(wait_status), _stream(stream))
 
 
 # ---- tensor-level helpers (allocation through torch, compute in the library) ----

@@ -298,6 +298,11 @@ __global__ void probe_wait_kernel(unsigned* status, const word_t* word, uint32_t
 
 }  // namespace
 
+namespace pararnn {
+// lets the other translation unit of the library (noalloc.cu) report through pararnn_last_error()
+void set_last_error(const char* msg) { fail(PARARNN_OK, "%s", msg); }
+}  // namespace pararnn
+
 extern "C" {
 
 int pararnn_num_gates(pararnn_cell cell) {
