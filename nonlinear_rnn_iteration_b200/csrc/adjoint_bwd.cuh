@@ -123,7 +123,14 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
 
         if (is_scan) {
             // ================= scan warp =================
+            float zero[CPL][S];
+#pragma unroll
+            for (int j = 0; j < CPL; ++j)
+#pragma unroll
+                for (int s = 0; s < S; ++s) zero[j][s] = 0.0f;  // lambda_T = 0
+            block_sync();  // tile set up
             if (lane == 0) {
+                // claim the tile NSTAGE-1 ahead and start streaming it in
                 const int sn = (it + NSTAGE - 1) % NSTAGE;
                 const unsigned prev_t = sm.ticket[(it + NSTAGE - 2) % NSTAGE];
                 unsigned t2 = prev_t;
@@ -132,15 +139,9 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
                 if constexpr (Sh::kTma)
                     if (t2 < prm.nTiles && prev_t < prm.nTiles) issue_bwd_load<Cell, PxT, Sh>(&maps, sm, prm, t2, sn);
             }
-            float zero[CPL][S];
-#pragma unroll
-            for (int j = 0; j < CPL; ++j)
-#pragma unroll
-                for (int s = 0; s < S; ++s) zero[j][s] = 0.0f;  // lambda_T = 0
-            block_sync();  // tile set up
             block_sync();  // first-row Jacobians shared
             block_sync();  // warp totals ready
-            tile_lookback<S, W, NW, Sh::P, true>(prm.lb, tile, pos, 0, lane, sm.wagg, zero, sm.cin);
+            tile_lookback<S, W, NW, true>(prm.lb, tile, pos, 0, lane, sm.wagg, zero, sm.cin);
             block_sync();  // carry ready
             block_sync();  // per-sub-chunk dL/da partials ready
         } else {

@@ -7,15 +7,18 @@
 // progress does not depend on how the hardware schedules blocks).
 //
 // Per (tile, slot) -- slot = Newton iteration in the forward, 0 in the
-// backward -- and per channel, the workspace holds 64-bit words
-//     { high 32 bits: the call's epoch tag, low 32 bits: a float }
-//   aggregate  the tile's composed scan element (A: S x S, b: S)  NA words
-//   inclusive  the state after the tile's last row                 S words
+// backward -- the workspace holds 64-bit words
+//     { high 32 bits: the call's epoch tag, low 32 bits: a value }
+//   status     one word: 1 = aggregate published, 2 = inclusive published
+//   aggregate  per channel, the tile's composed scan element (A, b)  NA words
+//   inclusive  per channel, the state after the tile's last row      S words
 // A word is valid when its tag equals this call's epoch, so a value and its
-// "ready" flag travel in one single-copy-atomic store: publishing needs no
-// fence and reading needs one L2 round trip.  Words left by earlier calls
-// carry other tags and read as not ready; a zero-filled workspace never
-// matches (epochs start at 1).
+// "ready" flag travel in one single-copy-atomic store: no fence is needed.
+// Words left by earlier calls carry other tags and read as not ready; a
+// zero-filled workspace never matches (epochs start at 1).  The status word
+// lets one warp read 32 predecessors' states in one round trip; payload
+// words are checked again when they are read, so a status seen before its
+// payload costs a retry, never a wrong value.
 //
 // The carry into a tile is found by walking back to the nearest predecessor
 // with an inclusive value and applying the aggregates in between, in order,
@@ -33,6 +36,7 @@ typedef unsigned long long word_t;
 
 struct LookbackCtx {
     unsigned* status;  // workspace header word 0
+    word_t* tstat;     // [nTiles][nSlots] tile status words
     word_t* agg;       // [nTiles][nSlots][NA][W]
     word_t* inc;       // [nTiles][nSlots][S][W]
     int64_t nGroups;
@@ -78,145 +82,149 @@ __device__ __forceinline__ void publish_words(word_t* dst, const float (&vals)[W
         for (int n = 0; n < N; ++n) st_word(dst + n * W + lane + 32 * j, vals[j][n], epoch);
 }
 
-// Rare path: the nearest inclusive value lies more than P tiles back.  Walk
-// back one predecessor at a time for one channel, then apply the aggregates.
-template <int S, int W>
-__device__ bool lookback_deep(const LookbackCtx& cx, int64_t tile, int64_t dist_max, int slot, int ch, float (&x)[S]) {
-    constexpr int NA = S * S + S;
-    Deadline dl;
-    int64_t found = -1;
-    for (int64_t d = 1; d <= dist_max && found < 0;) {
-        const int64_t tp = tile - d * cx.nGroups;
-        bool inc_ok = true, agg_ok = true;
-#pragma unroll
-        for (int s = 0; s < S; ++s) inc_ok &= word_ok(ld_word(cx.inc + ((tp * cx.nSlots + slot) * S + s) * W + ch), cx.epoch);
-        if (inc_ok) {
-            found = d;
-            break;
-        }
-#pragma unroll
-        for (int a = 0; a < NA; ++a) agg_ok &= word_ok(ld_word(cx.agg + ((tp * cx.nSlots + slot) * NA + a) * W + ch), cx.epoch);
-        if (agg_ok) {
-            ++d;
-            continue;
-        }
-        if (dl.expired(cx.timeout_ns)) return false;
-        __nanosleep(32);
-    }
-    if (found < 0) return false;
-    {
-        const int64_t tp = tile - found * cx.nGroups;
-#pragma unroll
-        for (int s = 0; s < S; ++s) x[s] = word_val(ld_word(cx.inc + ((tp * cx.nSlots + slot) * S + s) * W + ch));
-    }
-    for (int64_t d = found - 1; d >= 1; --d) {
-        const int64_t tp = tile - d * cx.nGroups;
-        float A[S * S], b[S], y[S];
-#pragma unroll
-        for (int a = 0; a < S * S; ++a) A[a] = word_val(ld_word(cx.agg + ((tp * cx.nSlots + slot) * NA + a) * W + ch));
-#pragma unroll
-        for (int s = 0; s < S; ++s) b[s] = word_val(ld_word(cx.agg + ((tp * cx.nSlots + slot) * NA + S * S + s) * W + ch));
-        apply<S>(A, b, x, y);
-#pragma unroll
-        for (int s = 0; s < S; ++s) x[s] = y[s];
-    }
-    return true;
+constexpr uint32_t kTileAggregate = 1u, kTileInclusive = 2u;
+
+__device__ __forceinline__ void st_status(word_t* p, uint32_t state, uint32_t epoch) {
+    const word_t w = (static_cast<word_t>(epoch) << 32) | state;
+    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(w) : "memory");
 }
 
 // Carry into `tile` for scan slot `slot`: the state just before the tile's
 // first row, for the W/32 channels this lane owns.  `dist_max` = the tile's
 // position along the scan (its number of predecessors).  All 32 lanes of one
-// warp call this.  The words of the nearest P predecessors are fetched at
-// once, so the common case costs one L2 round trip.
-template <int S, int W, int P>
+// warp call this.
+//   1. lane j reads the status of predecessor base+j; the nearest one with an
+//      inclusive value, with only aggregates between it and this tile, ends
+//      the walk (32 predecessors per round trip);
+//   2. the payload words of that inclusive value and of the aggregates in
+//      between are read in batches of NB predecessors, and the aggregates are
+//      applied to the inclusive value in order, nearest last.
+// The inclusive words of the first predecessor are fetched with step 1, so
+// the common case costs one round trip.
+template <int S, int W>
 __device__ void lookback_carry(const LookbackCtx& cx, int64_t tile, int64_t dist_max, int slot, int lane,
                                float (&carry)[W / 32][S]) {
     constexpr int NA = S * S + S;
     constexpr int CPL = W / 32;
-    const int depth = dist_max < P ? static_cast<int>(dist_max) : P;
+    constexpr int NB = S == 1 ? 4 : 2;  // aggregates read per batch
     Deadline dl;
+    int64_t base = 1, found = -1;
+    bool ok = true;
+    // ---- 1. walk the status words ----
     while (true) {
-        int state_all = 0;  // bit 0: some channel must wait, bit 1: some channel needs the deep walk
+        const int64_t j = base + lane;
+        uint32_t state = 0;
+        if (j <= dist_max) {
+            const word_t w = ld_word(cx.tstat + (tile - j * cx.nGroups) * cx.nSlots + slot);
+            if (word_ok(w, cx.epoch)) state = static_cast<uint32_t>(w);
+        }
+        float spec[CPL][S];  // inclusive words of the nearest predecessor, fetched speculatively
+        bool spec_ok = true;
+        if (base == 1) {
+            const float* dummy = nullptr;
+            (void)dummy;
 #pragma unroll
-        for (int j = 0; j < CPL; ++j) {
-            const int ch = lane + 32 * j;
-            word_t wi[P][S], wa[P][NA];
+            for (int jj = 0; jj < CPL; ++jj)
 #pragma unroll
-            for (int d = 0; d < P; ++d) {
-                if (d < depth) {
-                    const int64_t tp = tile - (d + 1) * cx.nGroups;
-#pragma unroll
-                    for (int s = 0; s < S; ++s) wi[d][s] = ld_word(cx.inc + ((tp * cx.nSlots + slot) * S + s) * W + ch);
-#pragma unroll
-                    for (int a = 0; a < NA; ++a) wa[d][a] = ld_word(cx.agg + ((tp * cx.nSlots + slot) * NA + a) * W + ch);
+                for (int s = 0; s < S; ++s) {
+                    const word_t w = ld_word(cx.inc + (((tile - cx.nGroups) * cx.nSlots + slot) * S + s) * W + lane + 32 * jj);
+                    spec_ok &= word_ok(w, cx.epoch);
+                    spec[jj][s] = word_val(w);
                 }
-            }
-            int found = -1, state = 0;
+        }
+        const unsigned inc_mask = __ballot_sync(0xffffffffu, j <= dist_max && state == kTileInclusive);
+        const unsigned not_ready = __ballot_sync(0xffffffffu, j <= dist_max && state == 0);
+        if (inc_mask) {
+            const int first = __ffs(inc_mask) - 1;
+            const unsigned before = first ? (not_ready & ((1u << first) - 1u)) : 0u;
+            if (!before) {
+                found = base + first;
+                if (found == 1 && __all_sync(0xffffffffu, spec_ok)) {
 #pragma unroll
-            for (int d = 0; d < P; ++d) {
-                if (d < depth && found < 0 && state == 0) {
-                    bool inc_ok = true, agg_ok = true;
+                    for (int jj = 0; jj < CPL; ++jj)
 #pragma unroll
-                    for (int s = 0; s < S; ++s) inc_ok &= word_ok(wi[d][s], cx.epoch);
-#pragma unroll
-                    for (int a = 0; a < NA; ++a) agg_ok &= word_ok(wa[d][a], cx.epoch);
-                    if (inc_ok) found = d;
-                    else if (!agg_ok) state = 1;
+                        for (int s = 0; s < S; ++s) carry[jj][s] = spec[jj][s];
+                    return;
                 }
+                break;
             }
-            if (found < 0 && state == 0) state = (depth < dist_max) ? 2 : 1;
-            if (found >= 0) {
-                float x[S];
+        } else if (!not_ready) {
+            // 32 aggregates in a row: look further back
+            base += 32;
+            if (base <= dist_max) continue;
+            ok = false;  // the first tile of the scan never publishes an aggregate only
+            break;
+        }
+        if (dl.expired(cx.timeout_ns)) {
+            ok = false;
+            break;
+        }
+        __nanosleep(20);
+    }
+    // ---- 2. payloads: inclusive(found), then aggregates found-1 .. 1 ----
+    if (ok) {
+        float x[CPL][S];
+        Deadline dl2;
+        while (true) {
+            bool good = true;
 #pragma unroll
-                for (int s = 0; s < S; ++s) x[s] = word_val(wi[0][s]);
+            for (int jj = 0; jj < CPL; ++jj)
 #pragma unroll
-                for (int d = P - 1; d >= 0; --d) {
-                    if (d == found) {
+                for (int s = 0; s < S; ++s) {
+                    const word_t w = ld_word(cx.inc + (((tile - found * cx.nGroups) * cx.nSlots + slot) * S + s) * W + lane + 32 * jj);
+                    good &= word_ok(w, cx.epoch);
+                    x[jj][s] = word_val(w);
+                }
+            for (int64_t i = found - 1; i >= 1 && good; i -= NB) {
+                word_t e[NB][CPL][NA];
 #pragma unroll
-                        for (int s = 0; s < S; ++s) x[s] = word_val(wi[d][s]);
-                    } else if (d < found) {
-                        float A[S * S], b[S], y[S];
+                for (int m = 0; m < NB; ++m)
+                    if (i - m >= 1) {
+                        const word_t* ap = cx.agg + ((tile - (i - m) * cx.nGroups) * cx.nSlots + slot) * NA * W;
 #pragma unroll
-                        for (int a = 0; a < S * S; ++a) A[a] = word_val(wa[d][a]);
+                        for (int jj = 0; jj < CPL; ++jj)
 #pragma unroll
-                        for (int s = 0; s < S; ++s) b[s] = word_val(wa[d][S * S + s]);
-                        apply<S>(A, b, x, y);
-#pragma unroll
-                        for (int s = 0; s < S; ++s) x[s] = y[s];
+                            for (int a = 0; a < NA; ++a) e[m][jj][a] = ld_word(ap + a * W + lane + 32 * jj);
                     }
-                }
 #pragma unroll
-                for (int s = 0; s < S; ++s) carry[j][s] = x[s];
+                for (int m = 0; m < NB; ++m)
+                    if (i - m >= 1) {
+#pragma unroll
+                        for (int jj = 0; jj < CPL; ++jj) {
+                            float A[S * S], b[S], y[S];
+#pragma unroll
+                            for (int a = 0; a < S * S; ++a) {
+                                good &= word_ok(e[m][jj][a], cx.epoch);
+                                A[a] = word_val(e[m][jj][a]);
+                            }
+#pragma unroll
+                            for (int s = 0; s < S; ++s) {
+                                good &= word_ok(e[m][jj][S * S + s], cx.epoch);
+                                b[s] = word_val(e[m][jj][S * S + s]);
+                            }
+                            apply<S>(A, b, x[jj], y);
+#pragma unroll
+                            for (int s = 0; s < S; ++s) x[jj][s] = y[s];
+                        }
+                    }
             }
-            state_all |= (found >= 0) ? 0 : state;
-        }
-        const unsigned wait_any = __ballot_sync(0xffffffffu, state_all & 1);
-        const unsigned deep_any = __ballot_sync(0xffffffffu, state_all & 2);
-        if (!wait_any && !deep_any) return;
-        if (!wait_any && deep_any) {
-            // every unresolved channel has P aggregates in a row: walk further back
-            bool ok = true;
+            if (__all_sync(0xffffffffu, good)) {
 #pragma unroll
-            for (int j = 0; j < CPL; ++j) {
-                float x[S];
-                if (lookback_deep<S, W>(cx, tile, dist_max, slot, lane + 32 * j, x)) {
+                for (int jj = 0; jj < CPL; ++jj)
 #pragma unroll
-                    for (int s = 0; s < S; ++s) carry[j][s] = x[s];
-                } else {
-                    ok = false;
-                }
+                    for (int s = 0; s < S; ++s) carry[jj][s] = x[jj][s];
+                return;
             }
-            if (__all_sync(0xffffffffu, ok)) return;
-            break;  // timed out
+            // a status word became visible before its payload: read again
+            if (dl2.expired(cx.timeout_ns)) break;
+            __nanosleep(20);
         }
-        if (dl.expired(cx.timeout_ns)) break;
-        __nanosleep(32);
     }
     if (lane == 0) atomicOr(cx.status, kStatusTimeout);
 #pragma unroll
-    for (int j = 0; j < CPL; ++j)
+    for (int jj = 0; jj < CPL; ++jj)
 #pragma unroll
-        for (int s = 0; s < S; ++s) carry[j][s] = 0.0f;
+        for (int s = 0; s < S; ++s) carry[jj][s] = 0.0f;
 }
 
 // ---- the block-level part of one scan step --------------------------------
@@ -315,7 +323,7 @@ __device__ __forceinline__ void sub_prefix(const ElemV<S, V>& excl, int warp, in
 // Step 2b (warp 0, after the first barrier): compose the warp totals into
 // the tile's element, publish it, find the carry by look-back, publish the
 // state after the tile, and write the carry-in to cin.
-template <int S, int W, int NW, int P, bool kReverse>
+template <int S, int W, int NW, bool kReverse>
 __device__ __forceinline__ void tile_lookback(const LookbackCtx& cx, int64_t tile, int64_t pos, int slot, int lane,
                                               const float (&wagg)[NW][S * S + S][W],
                                               const float (&first_carry)[W / 32][S], float (&cin)[S][W]) {
@@ -353,12 +361,16 @@ __device__ __forceinline__ void tile_lookback(const LookbackCtx& cx, int64_t til
             for (int s = 0; s < S; ++s) vals[j][S * S + s] = tot[j].b[s];
         }
         publish_words<NA, W>(cx.agg + (tile * cx.nSlots + slot) * NA * W, vals, cx.epoch, lane);
-        lookback_carry<S, W, P>(cx, tile, pos, slot, lane, carry);
+        __syncwarp();
+        if (lane == 0) st_status(cx.tstat + tile * cx.nSlots + slot, kTileAggregate, cx.epoch);
+        lookback_carry<S, W>(cx, tile, pos, slot, lane, carry);
     }
     float vals[CPL][S];
 #pragma unroll
     for (int j = 0; j < CPL; ++j) apply<S>(tot[j].A, tot[j].b, carry[j], vals[j]);
     publish_words<S, W>(cx.inc + (tile * cx.nSlots + slot) * S * W, vals, cx.epoch, lane);
+    __syncwarp();
+    if (lane == 0) st_status(cx.tstat + tile * cx.nSlots + slot, kTileInclusive, cx.epoch);
 #pragma unroll
     for (int j = 0; j < CPL; ++j)
 #pragma unroll

@@ -68,7 +68,6 @@ struct FwdShape {
     static constexpr int L = NSUB * R;            // time steps per tile
     static constexpr int NTC = NWARPS * 32;       // compute threads
     static constexpr int NT = NTC + 32;           // + the scan warp
-    static constexpr int P = S == 1 ? 4 : 2;      // predecessors fetched at once by the look-back
     static constexpr uint32_t kStageBytes = L * G * W * sizeof(PxT);
     static_assert(NSTAGE >= 2, "at least one stage in flight while another is used");
     static_assert(32 % LC == 0 && W % 32 == 0, "tile width must be a multiple of 32 channels");
@@ -144,17 +143,6 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
 
         if (is_scan) {
             // ================= scan warp =================
-            if (lane == 0) {
-                // claim the tile NSTAGE-1 ahead; its stage was freed by the
-                // previous iteration's last barrier
-                const int sn = (it + NSTAGE - 1) % NSTAGE;
-                const unsigned prev_t = sm.ticket[(it + NSTAGE - 2) % NSTAGE];
-                unsigned t2 = prev_t;
-                if (prev_t < prm.nTiles) t2 = atomicAdd(prm.ticket, 1u);
-                sm.ticket[sn] = t2;
-                if constexpr (Sh::kTma)
-                    if (t2 < prm.nTiles && prev_t < prm.nTiles) issue_tile_load<Cell, PxT, Sh>(&tmap, sm, prm, t2, sn);
-            }
             float first_carry[CPL][S];  // h_{-1} = h0 for every iterate
 #pragma unroll
             for (int j = 0; j < CPL; ++j)
@@ -164,9 +152,20 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
                     first_carry[j][s] = (prm.h0 && d < D) ? prm.h0[(b * S + s) * D + d] : 0.0f;
                 }
             block_sync();  // tile set up
+            if (lane == 0) {
+                // claim the tile NSTAGE-1 ahead and start streaming it in; its
+                // stage was freed by the previous iteration's last barrier
+                const int sn = (it + NSTAGE - 1) % NSTAGE;
+                const unsigned prev_t = sm.ticket[(it + NSTAGE - 2) % NSTAGE];
+                unsigned t2 = prev_t;
+                if (prev_t < prm.nTiles) t2 = atomicAdd(prm.ticket, 1u);
+                sm.ticket[sn] = t2;
+                if constexpr (Sh::kTma)
+                    if (t2 < prm.nTiles && prev_t < prm.nTiles) issue_tile_load<Cell, PxT, Sh>(&tmap, sm, prm, t2, sn);
+            }
             if constexpr (kLean) {
                 block_sync();  // warp totals ready
-                tile_lookback<S, W, NW, Sh::P, false>(prm.lb, tile, chunk, 0, lane, sm.wagg, first_carry, sm.cin);
+                tile_lookback<S, W, NW, false>(prm.lb, tile, chunk, 0, lane, sm.wagg, first_carry, sm.cin);
                 block_sync();  // carry ready
             } else {
                 const int K = prm.K;
@@ -174,7 +173,7 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
                     block_sync();  // edges ready
                     if (k == K) break;
                     block_sync();  // warp totals ready
-                    tile_lookback<S, W, NW, Sh::P, false>(prm.lb, tile, chunk, k, lane, sm.wagg, first_carry, sm.cin);
+                    tile_lookback<S, W, NW, false>(prm.lb, tile, chunk, k, lane, sm.wagg, first_carry, sm.cin);
                     block_sync();  // carry ready
                     if (k + 1 == K && !prm.resid) break;
                 }

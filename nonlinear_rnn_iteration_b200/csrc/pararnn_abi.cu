@@ -34,13 +34,14 @@ pararnn_status cuda_fail(cudaError_t e, const char* what) {
 // FwdShape<Cell, PxT, V channels/thread, LC lanes across channels, warps,
 //          R rows/thread, blocks/SM budget, shared-memory stages, TMA>
 // TMA path (D * element size a multiple of 16 bytes, 16-byte aligned rows):
-// 64 channels per tile.  Element-wise path otherwise: 32 channels per tile.
-template <typename PxT> using FwdLinT = FwdShape<CellLinear, PxT, 4, 16, 8, 4, 2, 3, true>;
+// 32 or 64 channels per tile, chosen by measurement on the workloads.
+// Element-wise path otherwise: 32 channels per tile.
+template <typename PxT> using FwdLinT = FwdShape<CellLinear, PxT, 4, 8, 4, 8, 2, 3, true>;
 template <typename PxT> using FwdGruT = FwdShape<CellGRU, PxT, 4, 16, 8, 4, 2, 2, true>;
-template <typename PxT> using FwdLstmT = FwdShape<CellLSTM, PxT, 4, 16, 8, 2, 2, 2, true>;
-template <typename PxT> using BwdLinT = FwdShape<CellLinear, PxT, 4, 16, 8, 2, 2, 2, true>;
-template <typename PxT> using BwdGruT = FwdShape<CellGRU, PxT, 4, 16, 8, 2, 2, 2, true>;
-template <typename PxT> using BwdLstmT = FwdShape<CellLSTM, PxT, 2, 32, 8, 2, 1, 2, true>;
+template <typename PxT> using FwdLstmT = FwdShape<CellLSTM, PxT, 2, 16, 8, 2, 2, 2, true>;
+template <typename PxT> using BwdLinT = FwdShape<CellLinear, PxT, 2, 16, 8, 4, 2, 2, true>;
+template <typename PxT> using BwdGruT = FwdShape<CellGRU, PxT, 2, 16, 8, 4, 2, 2, true>;
+template <typename PxT> using BwdLstmT = FwdShape<CellLSTM, PxT, 2, 16, 8, 2, 1, 2, true>;
 template <typename PxT> using FwdLinS = FwdShape<CellLinear, PxT, 1, 32, 8, 4, 2, 2, false>;
 template <typename PxT> using FwdGruS = FwdShape<CellGRU, PxT, 1, 32, 8, 4, 2, 2, false>;
 template <typename PxT> using FwdLstmS = FwdShape<CellLSTM, PxT, 1, 32, 8, 2, 2, 2, false>;
@@ -98,7 +99,7 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct Plan {
     int64_t nCG = 0, nChunks = 0, nGroups = 0, nTiles = 0;
-    size_t off_agg = 0, off_inc = 0, off_part = 0, total = 0;
+    size_t off_tstat = 0, off_agg = 0, off_inc = 0, off_part = 0, total = 0;
     Geometry g;
 };
 
@@ -110,7 +111,8 @@ Plan make_plan(pararnn_cell cell, int64_t B, int64_t T, int64_t D, int K, bool f
     p.nGroups = B * p.nCG;
     p.nTiles = p.nGroups * p.nChunks;
     const size_t nt = (size_t)p.nTiles, ns = (size_t)p.g.nSlots, W = (size_t)p.g.W;
-    p.off_agg = kHeaderBytes;
+    p.off_tstat = kHeaderBytes;
+    p.off_agg = align256(p.off_tstat + nt * ns * sizeof(word_t));
     p.off_inc = align256(p.off_agg + nt * ns * p.g.NA * W * sizeof(word_t));
     p.off_part = align256(p.off_inc + nt * ns * p.g.S * W * sizeof(word_t));
     p.total = fwd ? p.off_part : align256(p.off_part + nt * p.g.G * W * sizeof(float));
@@ -382,6 +384,7 @@ pararnn_status pararnn_newton_forward(pararnn_cell cell, int64_t B, int64_t T, i
     prm.K = Keff;
     prm.ticket = reinterpret_cast<unsigned*>(ws) + 1;
     prm.lb.status = reinterpret_cast<unsigned*>(ws);
+    prm.lb.tstat = reinterpret_cast<word_t*>(ws + pl.off_tstat);
     prm.lb.agg = reinterpret_cast<word_t*>(ws + pl.off_agg);
     prm.lb.inc = reinterpret_cast<word_t*>(ws + pl.off_inc);
     prm.lb.nGroups = pl.nGroups;
@@ -479,6 +482,7 @@ pararnn_status pararnn_newton_backward(pararnn_cell cell, int64_t B, int64_t T, 
     prm.D = D;
     prm.ticket = reinterpret_cast<unsigned*>(ws) + 1;
     prm.lb.status = reinterpret_cast<unsigned*>(ws);
+    prm.lb.tstat = reinterpret_cast<word_t*>(ws + pl.off_tstat);
     prm.lb.agg = reinterpret_cast<word_t*>(ws + pl.off_agg);
     prm.lb.inc = reinterpret_cast<word_t*>(ws + pl.off_inc);
     prm.lb.nGroups = pl.nGroups;
