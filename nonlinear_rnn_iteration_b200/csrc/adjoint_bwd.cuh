@@ -191,6 +191,11 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
             }
             block_sync();  // tile set up
 
+            float wr[V][G];  // the recurrent weights of this thread's channels
+#pragma unroll
+            for (int v = 0; v < V; ++v)
+#pragma unroll
+                for (int g = 0; g < G; ++g) wr[v][g] = sm.w[g][cc + v];
             // ---- linearisation at (h_{t-1}, x_t) for every row ----
             float jA[R][S * S][V], sens[R][NS][V];
 #pragma unroll
@@ -203,15 +208,12 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
                 for (int s = 0; s < S; ++s) lds_row<V>(row > 0 ? &sm.H[st][row - 1][s][cc] : &sm.hprev[s][cc], hv[s]);
 #pragma unroll
                 for (int v = 0; v < V; ++v) {
-                    float pg[G], wv[G], spv[S], A[S * S], se[NS];
+                    float pg[G], spv[S], A[S * S], se[NS];
 #pragma unroll
-                    for (int g = 0; g < G; ++g) {
-                        pg[g] = pv[g][v];
-                        wv[g] = sm.w[g][cc + v];
-                    }
+                    for (int g = 0; g < G; ++g) pg[g] = pv[g][v];
 #pragma unroll
                     for (int s = 0; s < S; ++s) spv[s] = hv[s][v];
-                    Cell::bwd(pg, wv, spv, A, se);
+                    Cell::bwd(pg, wr[v], spv, A, se);
 #pragma unroll
                     for (int a = 0; a < S * S; ++a) jA[r][a][v] = A[a];
 #pragma unroll
@@ -232,15 +234,12 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
 #pragma unroll
                     for (int a = 0; a < S * S; ++a) A[a] = 0.0f;
                     if (tn < T && cvalid) {
-                        float pv[G], wv[G], spv[S], se[NS];
+                        float pv[G], spv[S], se[NS];
 #pragma unroll
-                        for (int g = 0; g < G; ++g) {
-                            pv[g] = PxTraits<PxT>::cvt(pxg[((b * T + tn) * G + g) * D + d0 + cc + v]);
-                            wv[g] = sm.w[g][cc + v];
-                        }
+                        for (int g = 0; g < G; ++g) pv[g] = PxTraits<PxT>::cvt(pxg[((b * T + tn) * G + g) * D + d0 + cc + v]);
 #pragma unroll
                         for (int s = 0; s < S; ++s) spv[s] = sm.H[st][L - 1][s][cc + v];
-                        Cell::bwd(pv, wv, spv, A, se);
+                        Cell::bwd(pv, wr[v], spv, A, se);
                     }
 #pragma unroll
                     for (int a = 0; a < S * S; ++a) nextA[a][v] = A[a];

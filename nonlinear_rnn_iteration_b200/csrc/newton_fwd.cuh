@@ -278,6 +278,12 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
                 if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(prm.lb.status, kStatusNonFinite);
             } else {
                 // ---- general path: warm start, K Newton iterations ----
+                const bool want_resid = prm.resid != nullptr;
+                float wr[V][G];  // the recurrent weights of this thread's channels
+#pragma unroll
+                for (int v = 0; v < V; ++v)
+#pragma unroll
+                    for (int g = 0; g < G; ++g) wr[v][g] = sm.w[g][cc + v];
                 float h[R][S][V];
 #pragma unroll
                 for (int r = 0; r < R; ++r) {
@@ -285,13 +291,10 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
                     load_p(r, pv);
 #pragma unroll
                     for (int v = 0; v < V; ++v) {
-                        float pg[G], wv[G], f[S];
+                        float pg[G], f[S];
 #pragma unroll
-                        for (int g = 0; g < G; ++g) {
-                            pg[g] = pv[g][v];
-                            wv[g] = sm.w[g][cc + v];
-                        }
-                        Cell::warm(pg, wv, f);
+                        for (int g = 0; g < G; ++g) pg[g] = pv[g][v];
+                        Cell::warm(pg, wr[v], f);
 #pragma unroll
                         for (int s = 0; s < S; ++s) h[r][s][v] = f[s];
                     }
@@ -321,23 +324,20 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
                         load_p(r, pv);
 #pragma unroll
                         for (int v = 0; v < V; ++v) {
-                            float pg[G], wv[G], spv[S], f[S], A[S * S], be[S];
+                            float pg[G], spv[S], f[S], A[S * S], be[S];
 #pragma unroll
-                            for (int g = 0; g < G; ++g) {
-                                pg[g] = pv[g][v];
-                                wv[g] = sm.w[g][cc + v];
-                            }
+                            for (int g = 0; g < G; ++g) pg[g] = pv[g][v];
 #pragma unroll
                             for (int s = 0; s < S; ++s) spv[s] = sp[s][v];
-                            Cell::elem(pg, wv, spv, f, A, be);
-                            if (rvalid) {
-#pragma unroll
-                                for (int s = 0; s < S; ++s) res = nanmax_f(res, fabsf(h[r][s][v] - f[s]));
-                            } else {
+                            Cell::elem(pg, wr[v], spv, f, A, be);
+                            if (!rvalid) {
 #pragma unroll
                                 for (int a = 0; a < S * S; ++a) A[a] = (a % (S + 1) == 0) ? 1.0f : 0.0f;
 #pragma unroll
                                 for (int s = 0; s < S; ++s) be[s] = 0.0f;
+                            } else if (want_resid) {
+#pragma unroll
+                                for (int s = 0; s < S; ++s) res = nanmax_f(res, fabsf(h[r][s][v] - f[s]));
                             }
 #pragma unroll
                             for (int a = 0; a < S * S; ++a) eA[r][a][v] = A[a];

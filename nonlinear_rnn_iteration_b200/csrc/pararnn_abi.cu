@@ -37,7 +37,7 @@ pararnn_status cuda_fail(cudaError_t e, const char* what) {
 // 32 or 64 channels per tile, chosen by measurement on the workloads.
 // Element-wise path otherwise: 32 channels per tile.
 template <typename PxT> using FwdLinT = FwdShape<CellLinear, PxT, 4, 8, 4, 8, 2, 3, true>;
-template <typename PxT> using FwdGruT = FwdShape<CellGRU, PxT, 4, 16, 8, 4, 2, 2, true>;
+template <typename PxT> using FwdGruT = FwdShape<CellGRU, PxT, 4, 8, 8, 4, 2, 2, true>;
 template <typename PxT> using FwdLstmT = FwdShape<CellLSTM, PxT, 2, 16, 8, 2, 2, 2, true>;
 template <typename PxT> using BwdLinT = FwdShape<CellLinear, PxT, 2, 16, 8, 4, 2, 2, true>;
 template <typename PxT> using BwdGruT = FwdShape<CellGRU, PxT, 2, 16, 8, 4, 2, 2, true>;
