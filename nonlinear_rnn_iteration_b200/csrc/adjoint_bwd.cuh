@@ -41,15 +41,26 @@ struct BwdParams {
     LookbackCtx lb;     // nSlots = 1
 };
 
+// Stage rows: px row i is time t0 + i (one row past the tile, for the
+// Jacobian at the next tile's first row); H row i is time t0 - 1 + i (one row
+// before the tile, the state the first row is linearised at); dL/dH row i is
+// time t0 + i.
+// One stage of TMA destinations, each array 128-byte aligned (a tensor copy
+// writes to a 128-byte aligned shared address).
+template <class Sh, typename PxT>
+struct alignas(128) BwdStage {
+    alignas(128) PxT px[Sh::L + 1][Sh::G][Sh::W];
+    alignas(128) float H[Sh::L + 1][Sh::S][Sh::W];
+    alignas(128) float g[Sh::L][Sh::S][Sh::W];
+};
+
 template <class Sh, typename PxT>
 struct BwdSmem {
-    alignas(128) PxT px[Sh::NSTAGE][Sh::L][Sh::G][Sh::W];
-    alignas(128) float H[Sh::NSTAGE][Sh::L][Sh::S][Sh::W];
-    alignas(128) float g[Sh::NSTAGE][Sh::L][Sh::S][Sh::W];
+    BwdStage<Sh, PxT> stg[Sh::NSTAGE];
     float wagg[Sh::NWARPS][Sh::NA][Sh::W];       // each warp's composed element
     float cin[Sh::S][Sh::W];                     // lambda just after the tile (the carry)
     float firstA[Sh::NSUB][Sh::S * Sh::S][Sh::W];  // each sub-chunk's first-row Jacobian
-    float hprev[Sh::S][Sh::W];                   // state just before the tile
+    float hprev[Sh::S][Sh::W];                   // h0 (for the first tile of a row)
     float w[Sh::G][Sh::W];
     float da[Sh::NSUB][Sh::G][Sh::W];
     uint64_t bar[Sh::NSTAGE];
@@ -70,11 +81,13 @@ __device__ __forceinline__ void issue_bwd_load(const BwdMaps<Sh>* maps, BwdSmem<
     const int64_t b = gid / prm.nCG;
     const int64_t d0 = (gid - b * prm.nCG) * Sh::W;
     const int row = (int)(b * prm.T + chunk * Sh::L);
-    constexpr uint32_t bytes = Sh::L * Sh::W * (Sh::G * sizeof(PxT) + 2 * Sh::S * sizeof(float));
+    constexpr uint32_t bytes = (Sh::L + 1) * Sh::W * Sh::G * sizeof(PxT) + (Sh::L + 1) * Sh::W * Sh::S * sizeof(float) +
+                               Sh::L * Sh::W * Sh::S * sizeof(float);
     mbar_arrive_expect_tx(&sm.bar[stage], bytes);
-    tma_load_3d(&sm.px[stage][0][0][0], &maps->px, &sm.bar[stage], (int)d0, 0, row);
-    tma_load_3d(&sm.H[stage][0][0][0], &maps->H, &sm.bar[stage], (int)d0, 0, row);
-    tma_load_3d(&sm.g[stage][0][0][0], &maps->g, &sm.bar[stage], (int)d0, 0, row);
+    tma_load_3d(&sm.stg[stage].px[0][0][0], &maps->px, &sm.bar[stage], (int)d0, 0, row);
+    // row - 1 may be -1 (first tile of the first batch row): TMA fills zeros there
+    tma_load_3d(&sm.stg[stage].H[0][0][0], &maps->H, &sm.bar[stage], (int)d0, 0, row - 1);
+    tma_load_3d(&sm.stg[stage].g[0][0][0], &maps->g, &sm.bar[stage], (int)d0, 0, row);
 }
 
 template <class Cell, typename PxT, class Sh>
@@ -155,17 +168,10 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
                 const int g = i / W, c = i - (i / W) * W;
                 sm.w[g][c] = (prm.w && d0 + c < D) ? __ldg(prm.w + g * D + d0 + c) : 0.0f;
             }
-            if (tid < W) {
+            if (t0 == 0 && tid < W) {
                 const int64_t d = d0 + tid;
 #pragma unroll
-                for (int s = 0; s < S; ++s) {
-                    float x = 0.0f;
-                    if (d < D) {
-                        if (t0 > 0) x = prm.H[((b * T + t0 - 1) * S + s) * D + d];
-                        else if (prm.h0) x = prm.h0[(b * S + s) * D + d];
-                    }
-                    sm.hprev[s][tid] = x;
-                }
+                for (int s = 0; s < S; ++s) sm.hprev[s][tid] = (prm.h0 && d < D) ? prm.h0[(b * S + s) * D + d] : 0.0f;
             }
             if constexpr (Sh::kTma) {
                 Deadline dl;
@@ -176,17 +182,16 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
                     }
                 }
             } else {
-                for (int i = tid; i < L * G * W; i += NTC) {
+                for (int i = tid; i < (L + 1) * G * W; i += NTC) {
                     const int row = i / (G * W), rem = i - row * (G * W), g = rem / W, c = rem - g * W;
                     const int64_t t = t0 + row, d = d0 + c;
-                    sm.px[st][row][g][c] = (t < T && d < D) ? pxg[((b * T + t) * G + g) * D + d] : PxT(0.0f);
+                    sm.stg[st].px[row][g][c] = (t < T && d < D) ? pxg[((b * T + t) * G + g) * D + d] : PxT(0.0f);
                 }
-                for (int i = tid; i < L * S * W; i += NTC) {
+                for (int i = tid; i < (L + 1) * S * W; i += NTC) {
                     const int row = i / (S * W), rem = i - row * (S * W), s = rem / W, c = rem - s * W;
-                    const int64_t t = t0 + row, d = d0 + c;
-                    const bool ok = t < T && d < D;
-                    sm.H[st][row][s][c] = ok ? prm.H[((b * T + t) * S + s) * D + d] : 0.0f;
-                    sm.g[st][row][s][c] = ok ? prm.dLdH[((b * T + t) * S + s) * D + d] : 0.0f;
+                    const int64_t th = t0 - 1 + row, tg = t0 + row, d = d0 + c;
+                    sm.stg[st].H[row][s][c] = (th >= 0 && th < T && d < D) ? prm.H[((b * T + th) * S + s) * D + d] : 0.0f;
+                    if (row < L) sm.stg[st].g[row][s][c] = (tg < T && d < D) ? prm.dLdH[((b * T + tg) * S + s) * D + d] : 0.0f;
                 }
             }
             block_sync();  // tile set up
@@ -203,9 +208,9 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
                 const int row = sub * R + r;
                 float pv[G][V], hv[S][V];
 #pragma unroll
-                for (int g = 0; g < G; ++g) lds_row<V>(&sm.px[st][row][g][cc], pv[g]);
+                for (int g = 0; g < G; ++g) lds_row<V>(&sm.stg[st].px[row][g][cc], pv[g]);
 #pragma unroll
-                for (int s = 0; s < S; ++s) lds_row<V>(row > 0 ? &sm.H[st][row - 1][s][cc] : &sm.hprev[s][cc], hv[s]);
+                for (int s = 0; s < S; ++s) lds_row<V>((t0 == 0 && row == 0) ? &sm.hprev[s][cc] : &sm.stg[st].H[row][s][cc], hv[s]);
 #pragma unroll
                 for (int v = 0; v < V; ++v) {
                     float pg[G], spv[S], A[S * S], se[NS];
@@ -236,9 +241,9 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
                     if (tn < T && cvalid) {
                         float pv[G], spv[S], se[NS];
 #pragma unroll
-                        for (int g = 0; g < G; ++g) pv[g] = PxTraits<PxT>::cvt(pxg[((b * T + tn) * G + g) * D + d0 + cc + v]);
+                        for (int g = 0; g < G; ++g) pv[g] = PxTraits<PxT>::cvt(sm.stg[st].px[L][g][cc + v]);
 #pragma unroll
-                        for (int s = 0; s < S; ++s) spv[s] = sm.H[st][L - 1][s][cc + v];
+                        for (int s = 0; s < S; ++s) spv[s] = sm.stg[st].H[L][s][cc + v];
                         Cell::bwd(pv, wr[v], spv, A, se);
                     }
 #pragma unroll
@@ -278,7 +283,7 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
             for (int r = 0; r < R; ++r)
 #pragma unroll
                 for (int s = 0; s < S; ++s) {
-                    lds_row<V>(&sm.g[st][sub * R + r][s][cc], gr[r][s]);
+                    lds_row<V>(&sm.stg[st].g[sub * R + r][s][cc], gr[r][s]);
                     if (tb + r >= T)
 #pragma unroll
                         for (int v = 0; v < V; ++v) gr[r][s][v] = 0.0f;

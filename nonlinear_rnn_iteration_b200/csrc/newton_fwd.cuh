@@ -68,16 +68,28 @@ struct FwdShape {
     static constexpr int L = NSUB * R;            // time steps per tile
     static constexpr int NTC = NWARPS * 32;       // compute threads
     static constexpr int NT = NTC + 32;           // + the scan warp
-    static constexpr uint32_t kStageBytes = L * G * W * sizeof(PxT);
+    // forward stage rows: a nonlinear cell's tile also carries the row just
+    // before it (the warm start there is the first row's previous state)
+    static constexpr int ROW0 = Cell::kNonlinear ? 1 : 0;
+    static constexpr int LF = L + ROW0;
+    static constexpr uint32_t kStageBytes = LF * G * W * sizeof(PxT);
     static_assert(NSTAGE >= 2, "at least one stage in flight while another is used");
     static_assert(32 % LC == 0 && W % 32 == 0, "tile width must be a multiple of 32 channels");
     static_assert(!kTma || (W * sizeof(PxT)) % 16 == 0, "TMA box rows must be whole 16-byte units");
-    static_assert(W <= 256 && L <= 256 && G <= 256, "TMA box dimensions are at most 256");
+    static_assert(W <= 256 && L + 1 <= 256 && G <= 256, "TMA box dimensions are at most 256");
+};
+
+// One TMA destination: a tensor copy writes to a 128-byte aligned shared
+// address, so every stage is padded to a multiple of 128 bytes.
+template <class Sh, typename PxT>
+struct alignas(128) FwdStage {
+    PxT v[Sh::LF][Sh::G][Sh::W];  // row i is time t0 - ROW0 + i
 };
 
 template <class Sh, typename PxT>
 struct FwdSmem {
-    alignas(128) PxT px[Sh::NSTAGE][Sh::L][Sh::G][Sh::W];  // TMA destination
+    static_assert(sizeof(FwdStage<Sh, PxT>) % 128 == 0, "each TMA stage starts 128-byte aligned");
+    FwdStage<Sh, PxT> px[Sh::NSTAGE];
     float wagg[Sh::NWARPS][Sh::NA][Sh::W];  // each compute warp's composed element
     float edge[Sh::NSUB][Sh::S][Sh::W];     // each sub-chunk's last state (current iterate)
     float cin[Sh::S][Sh::W];                // the state just before the tile (current iterate)
@@ -94,7 +106,9 @@ __device__ __forceinline__ void issue_tile_load(const CUtensorMap* map, FwdSmem<
     const int64_t b = gid / prm.nCG;
     const int64_t d0 = (gid - b * prm.nCG) * Sh::W;
     mbar_arrive_expect_tx(&sm.bar[stage], Sh::kStageBytes);
-    tma_load_3d(&sm.px[stage][0][0][0], map, &sm.bar[stage], (int)d0, 0, (int)(b * prm.T + chunk * Sh::L));
+    // the row coordinate may be -1 (first tile of the first batch row): TMA fills zeros there
+    tma_load_3d(&sm.px[stage].v[0][0][0], map, &sm.bar[stage], (int)d0, 0,
+                (int)(b * prm.T + chunk * Sh::L) - Sh::ROW0);
 }
 
 template <class Cell, typename PxT, class Sh, bool kLean>
@@ -189,7 +203,26 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
                 const int g = i / W, c = i - (i / W) * W;
                 sm.w[g][c] = (prm.w && d0 + c < D) ? __ldg(prm.w + g * D + d0 + c) : 0.0f;
             }
-            // h^(0) just before the tile: h0 for the first tile, else the warm start of the previous row
+            // the tile's pre-activations: TMA (already in flight) or a cooperative copy
+            if constexpr (Sh::kTma) {
+                Deadline dl;
+                while (!mbar_try_wait(&sm.bar[st], (it / NSTAGE) & 1)) {
+                    if (dl.expired(prm.lb.timeout_ns)) {
+                        if (tid == 0) atomicOr(prm.lb.status, kStatusTimeout);
+                        break;
+                    }
+                }
+            } else {
+                for (int i = tid; i < Sh::LF * G * W; i += NTC) {
+                    const int row = i / (G * W), rem = i - row * (G * W), g = rem / W, c = rem - g * W;
+                    const int64_t t = t0 - Sh::ROW0 + row, d = d0 + c;
+                    sm.px[st].v[row][g][c] = (t >= 0 && t < T && d < D) ? pxg[((b * T + t) * G + g) * D + d] : PxT(0.0f);
+                }
+            }
+            block_sync();  // tile set up
+            // h^(0) just before the tile: h0 for the first tile, else the warm
+            // start of the previous row (row 0 of a nonlinear cell's stage);
+            // read by sub-chunk 0 after the next barrier
             if (need_prev && tid < W) {
                 const int64_t d = d0 + tid;
                 float f[S] = {};
@@ -201,8 +234,9 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
                         float pv[G], wv[G];
 #pragma unroll
                         for (int g = 0; g < G; ++g) {
-                            pv[g] = PxTraits<PxT>::cvt(pxg[((b * T + t0 - 1) * G + g) * D + d]);
-                            wv[g] = prm.w ? __ldg(prm.w + g * D + d) : 0.0f;
+                            pv[g] = Sh::ROW0 ? PxTraits<PxT>::cvt(sm.px[st].v[0][g][tid])
+                                             : PxTraits<PxT>::cvt(pxg[((b * T + t0 - 1) * G + g) * D + d]);
+                            wv[g] = sm.w[g][tid];
                         }
                         Cell::warm(pv, wv, f);
                     }
@@ -210,28 +244,11 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
 #pragma unroll
                 for (int s = 0; s < S; ++s) sm.cin[s][tid] = f[s];
             }
-            // the tile's pre-activations: TMA (already in flight) or a cooperative copy
-            if constexpr (Sh::kTma) {
-                Deadline dl;
-                while (!mbar_try_wait(&sm.bar[st], (it / NSTAGE) & 1)) {
-                    if (dl.expired(prm.lb.timeout_ns)) {
-                        if (tid == 0) atomicOr(prm.lb.status, kStatusTimeout);
-                        break;
-                    }
-                }
-            } else {
-                for (int i = tid; i < L * G * W; i += NTC) {
-                    const int row = i / (G * W), rem = i - row * (G * W), g = rem / W, c = rem - g * W;
-                    const int64_t t = t0 + row, d = d0 + c;
-                    sm.px[st][row][g][c] = (t < T && d < D) ? pxg[((b * T + t) * G + g) * D + d] : PxT(0.0f);
-                }
-            }
-            block_sync();  // tile set up
 
             // pre-activations of row r of this thread, V channels per gate
             auto load_p = [&](int r, float (&pv)[G][V]) {
 #pragma unroll
-                for (int g = 0; g < G; ++g) lds_row<V>(&sm.px[st][sub * R + r][g][cc], pv[g]);
+                for (int g = 0; g < G; ++g) lds_row<V>(&sm.px[st].v[Sh::ROW0 + sub * R + r][g][cc], pv[g]);
             };
 
             if constexpr (kLean) {

@@ -219,7 +219,7 @@ pararnn_status launch_fwd(const Plan& pl, FwdParams prm, cudaStream_t st) {
     CUtensorMap map;
     memset(&map, 0, sizeof map);
     if (Sh::kTma) {
-        pararnn_status s = make_map(&map, prm.px, sizeof(PxT) == 2, prm.D, Sh::G, prm.B * prm.T, Sh::W, Sh::L);
+        pararnn_status s = make_map(&map, prm.px, sizeof(PxT) == 2, prm.D, Sh::G, prm.B * prm.T, Sh::W, Sh::LF);
         if (s != PARARNN_OK) return s;
     }
     const size_t smem = sizeof(FwdSmem<Sh, PxT>);
@@ -254,8 +254,8 @@ pararnn_status launch_bwd(const Plan& pl, BwdParams prm, float* dLda, cudaStream
     memset(&maps, 0, sizeof maps);
     if (Sh::kTma) {
         const int64_t rows = prm.B * prm.T;
-        pararnn_status s = make_map(&maps.px, prm.px, sizeof(PxT) == 2, prm.D, Sh::G, rows, Sh::W, Sh::L);
-        if (s == PARARNN_OK) s = make_map(&maps.H, prm.H, false, prm.D, Sh::S, rows, Sh::W, Sh::L);
+        pararnn_status s = make_map(&maps.px, prm.px, sizeof(PxT) == 2, prm.D, Sh::G, rows, Sh::W, Sh::L + 1);
+        if (s == PARARNN_OK) s = make_map(&maps.H, prm.H, false, prm.D, Sh::S, rows, Sh::W, Sh::L + 1);
         if (s == PARARNN_OK) s = make_map(&maps.g, prm.dLdH, false, prm.D, Sh::S, rows, Sh::W, Sh::L);
         if (s != PARARNN_OK) return s;
     }
