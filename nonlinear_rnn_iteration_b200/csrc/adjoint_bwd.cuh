@@ -141,6 +141,8 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
             for (int j = 0; j < CPL; ++j)
 #pragma unroll
                 for (int s = 0; s < S; ++s) zero[j][s] = 0.0f;  // lambda_T = 0
+            Probe<S, W> pr;  // no early probe: the single pass is too short to hide one
+            pr.st = 0;
             block_sync();  // tile set up
             if (lane == 0) {
                 // claim the tile NSTAGE-1 ahead and start streaming it in
@@ -154,7 +156,7 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
             }
             block_sync();  // first-row Jacobians shared
             block_sync();  // warp totals ready
-            tile_lookback<S, W, NW, true>(prm.lb, tile, pos, 0, lane, sm.wagg, zero, sm.cin);
+            tile_lookback<S, W, NW, true>(prm.lb, tile, pos, 0, lane, sm.wagg, zero, pr, sm.cin);
             block_sync();  // carry ready
             block_sync();  // per-sub-chunk dL/da partials ready
         } else {

@@ -227,6 +227,28 @@ __device__ void lookback_carry(const LookbackCtx& cx, int64_t tile, int64_t dist
         for (int s = 0; s < S; ++s) carry[jj][s] = 0.0f;
 }
 
+// The predecessor's status and inclusive words, loaded early (while the
+// compute warps evaluate) and used after they have composed the tile: when
+// the predecessor had already finished, the carry costs no waiting at all.
+template <int S, int W>
+struct Probe {
+    word_t st;
+    word_t inc[W / 32][S];
+};
+
+template <int S, int W>
+__device__ __forceinline__ void probe_issue(const LookbackCtx& cx, int64_t tile, int64_t pos, int slot, int lane,
+                                            Probe<S, W>& pr) {
+    pr.st = 0;
+    if (pos == 0) return;
+    const int64_t tp = tile - cx.nGroups;
+    pr.st = ld_word(cx.tstat + tp * cx.nSlots + slot);
+#pragma unroll
+    for (int j = 0; j < W / 32; ++j)
+#pragma unroll
+        for (int s = 0; s < S; ++s) pr.inc[j][s] = ld_word(cx.inc + ((tp * cx.nSlots + slot) * S + s) * W + lane + 32 * j);
+}
+
 // ---- the block-level part of one scan step --------------------------------
 // Thread (warp w, lane l) owns sub-chunk sub = w * TPW + l / LC of the tile
 // and the V channels cc .. cc+V-1, cc = (l % LC) * V.  Scan order is time
@@ -326,7 +348,8 @@ __device__ __forceinline__ void sub_prefix(const ElemV<S, V>& excl, int warp, in
 template <int S, int W, int NW, bool kReverse>
 __device__ __forceinline__ void tile_lookback(const LookbackCtx& cx, int64_t tile, int64_t pos, int slot, int lane,
                                               const float (&wagg)[NW][S * S + S][W],
-                                              const float (&first_carry)[W / 32][S], float (&cin)[S][W]) {
+                                              const float (&first_carry)[W / 32][S], const Probe<S, W>& pr,
+                                              float (&cin)[S][W]) {
     constexpr int NA = S * S + S;
     constexpr int CPL = W / 32;
     Elem<S> tot[CPL];
@@ -346,12 +369,27 @@ __device__ __forceinline__ void tile_lookback(const LookbackCtx& cx, int64_t til
         }
     }
     float carry[CPL][S];
+    bool probed = false;
+    if (pos > 0) {
+        // the predecessor's inclusive state, if the early probe found it published
+        bool ok = word_ok(pr.st, cx.epoch) && static_cast<uint32_t>(pr.st) == kTileInclusive;
+#pragma unroll
+        for (int j = 0; j < CPL; ++j)
+#pragma unroll
+            for (int s = 0; s < S; ++s) {
+                ok &= word_ok(pr.inc[j][s], cx.epoch);
+                carry[j][s] = word_val(pr.inc[j][s]);
+            }
+        probed = __all_sync(0xffffffffu, ok);
+    }
     if (pos == 0) {
 #pragma unroll
         for (int j = 0; j < CPL; ++j)
 #pragma unroll
             for (int s = 0; s < S; ++s) carry[j][s] = first_carry[j][s];
     } else {
+        // publish the aggregate first, so that successors never wait on this
+        // tile's look-back (it costs a few stores)
         float vals[CPL][NA];
 #pragma unroll
         for (int j = 0; j < CPL; ++j) {
@@ -363,7 +401,7 @@ __device__ __forceinline__ void tile_lookback(const LookbackCtx& cx, int64_t til
         publish_words<NA, W>(cx.agg + (tile * cx.nSlots + slot) * NA * W, vals, cx.epoch, lane);
         __syncwarp();
         if (lane == 0) st_status(cx.tstat + tile * cx.nSlots + slot, kTileAggregate, cx.epoch);
-        lookback_carry<S, W>(cx, tile, pos, slot, lane, carry);
+        if (!probed) lookback_carry<S, W>(cx, tile, pos, slot, lane, carry);
     }
     float vals[CPL][S];
 #pragma unroll

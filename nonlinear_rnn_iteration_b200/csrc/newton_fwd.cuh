@@ -165,6 +165,13 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
                     const int64_t d = d0 + lane + 32 * j;
                     first_carry[j][s] = (prm.h0 && d < D) ? prm.h0[(b * S + s) * D + d] : 0.0f;
                 }
+            // early probe of the predecessor: only where a long evaluation
+            // phase hides its round trip (the Newton iterations of a
+            // nonlinear cell); elsewhere a probe that misses costs more than
+            // it saves
+            Probe<S, W> pr;
+            pr.st = 0;
+            if constexpr (!kLean) probe_issue<S, W>(prm.lb, tile, chunk, 0, lane, pr);
             block_sync();  // tile set up
             if (lane == 0) {
                 // claim the tile NSTAGE-1 ahead and start streaming it in; its
@@ -179,15 +186,16 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
             }
             if constexpr (kLean) {
                 block_sync();  // warp totals ready
-                tile_lookback<S, W, NW, false>(prm.lb, tile, chunk, 0, lane, sm.wagg, first_carry, sm.cin);
+                tile_lookback<S, W, NW, false>(prm.lb, tile, chunk, 0, lane, sm.wagg, first_carry, pr, sm.cin);
                 block_sync();  // carry ready
             } else {
                 const int K = prm.K;
                 for (int k = 0; k <= K; ++k) {
                     block_sync();  // edges ready
                     if (k == K) break;
+                    if (k > 0) probe_issue<S, W>(prm.lb, tile, chunk, k, lane, pr);
                     block_sync();  // warp totals ready
-                    tile_lookback<S, W, NW, false>(prm.lb, tile, chunk, k, lane, sm.wagg, first_carry, sm.cin);
+                    tile_lookback<S, W, NW, false>(prm.lb, tile, chunk, k, lane, sm.wagg, first_carry, pr, sm.cin);
                     block_sync();  // carry ready
                     if (k + 1 == K && !prm.resid) break;
                 }
