@@ -333,8 +333,10 @@ def cpu_baseline(w, device, seed, target_s=12.0):
         import torch
 
         bi, di = torch.tensor(bs, device=device), torch.tensor(ds, device=device)
-        px = x["px"][bi, :, :, di].float().cpu().numpy().astype(np.float64).transpose(1, 2, 0)[None]
-        a = None if x["a"] is None else x["a"][:, di].cpu().numpy().astype(np.float64)
+        # (1, T, G, n) contiguous fp64, prepared outside the timed region
+        px = np.ascontiguousarray(x["px"][bi, :, :, di].float().cpu().numpy().transpose(1, 2, 0)[None],
+                                  dtype=np.float64)
+        a = None if x["a"] is None else np.ascontiguousarray(x["a"][:, di].cpu().numpy(), dtype=np.float64)
         t = time.perf_counter()
         if w.cell == "linear":
             oracle.unroll(w.cell_id, px, a, None, nthreads=threads)
@@ -457,6 +459,12 @@ def run_reference(args):
     per_step = []
     x = workloads.host_inputs(w.with_shape(B=1, D=n), seed=w.seed)
 
+    def prepare(xx):
+        # fp64 contiguous inputs, converted outside the timed region
+        return {k: (None if v is None else np.ascontiguousarray(v, dtype=np.float64)) for k, v in xx.items()}
+
+    x = prepare(x)
+
     def one():
         t = time.perf_counter()
         if w.cell == "linear":
@@ -468,7 +476,7 @@ def run_reference(args):
     probe = one()
     scale = max(1, int(2.0 / max(probe, 1e-3)))
     n = min(w.B * w.D, n * scale)
-    x = workloads.host_inputs(w.with_shape(B=1, D=n), seed=w.seed)
+    x = prepare(workloads.host_inputs(w.with_shape(B=1, D=n), seed=w.seed))
     for _ in range(args.warmup):
         one()
     for _ in range(args.steps):
@@ -486,7 +494,6 @@ def run_reference(args):
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
-    del np
 
 
 def main(argv=None):
