@@ -50,7 +50,7 @@ ALGO_BYTES = {
     ("linear", "f32", "bwd"): 24, ("diag_gru", "f32", "bwd"): 32, ("diag_gru", "bf16", "bwd"): 26,
     ("diag_lstm", "f32", "bwd"): 48, ("diag_lstm", "bf16", "bwd"): 40,
 }
-KERNEL_SOURCES = ["newton_fwd.cuh", "adjoint_bwd.cuh", "lookback.cuh", "cells.cuh", "common.cuh", "pararnn_abi.cu"]
+KERNEL_SOURCES = ["newton_fwd.cuh", "adjoint_bwd.cuh", "lookback.cuh", "cells.cuh", "common.cuh", "tma.cuh", "pararnn_abi.cu"]
 
 
 # --------------------------------------------------------------------------

@@ -2,16 +2,20 @@
 // state and the gradient epilogue, fused in one persistent kernel, plus a
 // fixed-order reduction of the per-tile weight-gradient partials.
 //
-// At the trajectory H (the forward's output), with g_t = dL/dH_t:
+// At the trajectory H (the forward's output), with g_t = dL/dH_t, the adjoint
+// of the lower-bidiagonal system F(H) = 0 is
 //     lambda_t = g_t + A_{t+1}^T lambda_{t+1},   lambda_{T-1} = g_{T-1},
-//     A_{t+1} = df/dh at (h_t, x_{t+1}),
-// which is the scan of the elements (M_t, g_t), M_t = A_{t+1}^T, in reverse
-// time under the same operator as the forward (pararnn-torch PyPI page,
-// Method section: the backward follows the paper's adjoint; here it is the
-// plain adjoint of the lower-bidiagonal system F(H) = 0).  Then
+//     A_t = df/dh at (h_{t-1}, x_t)
+// (pararnn-torch PyPI page, Method section: the backward follows the paper's
+// adjoint).  The kernel scans the propagated adjoint mu_t = A_t^T lambda_t
+// instead of lambda itself:
+//     mu_t = A_t^T (g_t + mu_{t+1}),   mu_T = 0,   lambda_t = g_t + mu_{t+1},
+// a reverse-time scan of the elements (A_t^T, A_t^T g_t) under the same
+// operator as the forward.  Each element needs only its own row's Jacobian
+// (no neighbouring row), and dL/dh0 = A_0^T lambda_0 = mu_0 is the scan's
+// last state.  Then
 //     dL/dp_g[t]  = lambda_t . df/dp_g   at (h_{t-1}, x_t)
-//     dL/da_g     = sum_{b,t} lambda_t . df/da_g
-//     dL/dh0      = A_0^T lambda_0.
+//     dL/da_g     = sum_{b,t} lambda_t . df/da_g.
 // dL/da is summed within a tile in a fixed order, written per tile, and
 // reduced over tiles in a fixed order by a second kernel: no floating-point
 // atomics, so the result does not depend on scheduling (Compatibility
@@ -41,28 +45,24 @@ struct BwdParams {
     LookbackCtx lb;     // nSlots = 1
 };
 
-// Stage rows: px row i is time t0 + i (one row past the tile, for the
-// Jacobian at the next tile's first row); H row i is time t0 - 1 + i (one row
-// before the tile, the state the first row is linearised at); dL/dH row i is
-// time t0 + i.
-// One stage of TMA destinations, each array 128-byte aligned (a tensor copy
-// writes to a 128-byte aligned shared address).
+// Stage rows: px and dL/dH row i are time t0 + i; H row i is time t0 - 1 + i
+// (the state row i is linearised at).  Each array is 128-byte aligned (a
+// tensor copy writes to a 128-byte aligned shared address).
 template <class Sh, typename PxT>
 struct alignas(128) BwdStage {
-    alignas(128) PxT px[Sh::L + 1][Sh::G][Sh::W];
-    alignas(128) float H[Sh::L + 1][Sh::S][Sh::W];
+    alignas(128) PxT px[Sh::L][Sh::G][Sh::W];
+    alignas(128) float H[Sh::L][Sh::S][Sh::W];
     alignas(128) float g[Sh::L][Sh::S][Sh::W];
 };
 
 template <class Sh, typename PxT>
 struct BwdSmem {
     BwdStage<Sh, PxT> stg[Sh::NSTAGE];
-    float wagg[Sh::NWARPS][Sh::NA][Sh::W];       // each warp's composed element
-    float cin[Sh::S][Sh::W];                     // lambda just after the tile (the carry)
-    float firstA[Sh::NSUB][Sh::S * Sh::S][Sh::W];  // each sub-chunk's first-row Jacobian
-    float hprev[Sh::S][Sh::W];                   // h0 (for the first tile of a row)
+    float wagg[Sh::NWARPS][Sh::NA][Sh::W];  // each warp's composed element
+    float cin[Sh::S][Sh::W];                // mu just after the tile (the carry)
+    float hprev[Sh::S][Sh::W];              // h0 (for the first tile of a row)
     float w[Sh::G][Sh::W];
-    float da[Sh::NSUB][Sh::G][Sh::W];
+    float da[2][Sh::NSUB][Sh::G][Sh::W];    // per-sub-chunk dL/da partials, two tiles in turn
     uint64_t bar[Sh::NSTAGE];
     unsigned ticket[Sh::NSTAGE];
 };
@@ -81,8 +81,7 @@ __device__ __forceinline__ void issue_bwd_load(const BwdMaps<Sh>* maps, BwdSmem<
     const int64_t b = gid / prm.nCG;
     const int64_t d0 = (gid - b * prm.nCG) * Sh::W;
     const int row = (int)(b * prm.T + chunk * Sh::L);
-    constexpr uint32_t bytes = (Sh::L + 1) * Sh::W * Sh::G * sizeof(PxT) + (Sh::L + 1) * Sh::W * Sh::S * sizeof(float) +
-                               Sh::L * Sh::W * Sh::S * sizeof(float);
+    constexpr uint32_t bytes = Sh::L * Sh::W * (Sh::G * sizeof(PxT) + 2 * Sh::S * sizeof(float));
     mbar_arrive_expect_tx(&sm.bar[stage], bytes);
     tma_load_3d(&sm.stg[stage].px[0][0][0], &maps->px, &sm.bar[stage], (int)d0, 0, row);
     // row - 1 may be -1 (first tile of the first batch row): TMA fills zeros there
@@ -90,11 +89,37 @@ __device__ __forceinline__ void issue_bwd_load(const BwdMaps<Sh>* maps, BwdSmem<
     tma_load_3d(&sm.stg[stage].g[0][0][0], &maps->g, &sm.bar[stage], (int)d0, 0, row);
 }
 
+// y = A^T v
+template <int S>
+__device__ __forceinline__ void mat_t_vec(const float (&A)[S * S], const float (&v)[S], float (&y)[S]) {
+    if constexpr (S == 1) {
+        y[0] = A[0] * v[0];
+    } else {
+        y[0] = __fmaf_rn(A[0], v[0], A[2] * v[1]);
+        y[1] = __fmaf_rn(A[1], v[0], A[3] * v[1]);
+    }
+}
+
+// The dL/da partial of one tile: the sum of its sub-chunks' partials in
+// sub-chunk order, written by the scan warp.
+template <class Sh, typename PxT>
+__device__ __forceinline__ void store_tile_partial(const BwdSmem<Sh, PxT>& sm, int buf, const BwdParams& prm,
+                                                   int64_t tile, int lane) {
+    constexpr int G = Sh::G, W = Sh::W;
+    for (int i = lane; i < G * W; i += 32) {
+        const int g = i / W, ch = i - (i / W) * W;
+        float acc = 0.0f;
+#pragma unroll
+        for (int sb = 0; sb < Sh::NSUB; ++sb) acc += sm.da[buf][sb][g][ch];
+        prm.part[(tile * G + g) * W + ch] = acc;
+    }
+}
+
 template <class Cell, typename PxT, class Sh>
 __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
     adjoint_bwd_kernel(const __grid_constant__ BwdMaps<Sh> maps, const BwdParams prm) {
     constexpr int G = Sh::G, S = Sh::S, V = Sh::V, R = Sh::R, NS = Cell::NSENS, NW = Sh::NWARPS;
-    constexpr int TPW = Sh::TPW, NSUB = Sh::NSUB, W = Sh::W, L = Sh::L, LC = Sh::LC, NTC = Sh::NTC;
+    constexpr int TPW = Sh::TPW, W = Sh::W, L = Sh::L, LC = Sh::LC, NTC = Sh::NTC;
     constexpr int NSTAGE = Sh::NSTAGE;
     constexpr int CPL = W / 32;
     using SM = BwdSmem<Sh, PxT>;
@@ -122,7 +147,15 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
     }
     block_sync();
 
-    for (int it = 0;; ++it) {
+    // Three block barriers per tile: (1) tile set up, (2) warp totals ready,
+    // (3) carry ready.  Nothing is shared across the end of a tile without
+    // one of them in between: the next tile's stage is refilled only after
+    // its barrier (1), the dL/da partials alternate between two buffers and
+    // the scan warp reduces a tile's partials between barriers (1) and (2)
+    // of the block's next tile.
+    int64_t prev_tile = -1;  // scan warp: the tile whose partials sit in da[(it - 1) & 1]
+    int it = 0;
+    for (;; ++it) {
         const int st = it % NSTAGE;
         const unsigned tile_u = sm.ticket[st];
         if (tile_u >= prm.nTiles) break;
@@ -140,10 +173,10 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
 #pragma unroll
             for (int j = 0; j < CPL; ++j)
 #pragma unroll
-                for (int s = 0; s < S; ++s) zero[j][s] = 0.0f;  // lambda_T = 0
+                for (int s = 0; s < S; ++s) zero[j][s] = 0.0f;  // mu_T = 0
             Probe<S, W> pr;  // no early probe: the single pass is too short to hide one
             pr.st = 0;
-            block_sync();  // tile set up
+            block_sync();  // (1) tile set up
             if (lane == 0) {
                 // claim the tile NSTAGE-1 ahead and start streaming it in
                 const int sn = (it + NSTAGE - 1) % NSTAGE;
@@ -154,11 +187,11 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
                 if constexpr (Sh::kTma)
                     if (t2 < prm.nTiles && prev_t < prm.nTiles) issue_bwd_load<Cell, PxT, Sh>(&maps, sm, prm, t2, sn);
             }
-            block_sync();  // first-row Jacobians shared
-            block_sync();  // warp totals ready
+            if (prev_tile >= 0) store_tile_partial<Sh, PxT>(sm, (it - 1) & 1, prm, prev_tile, lane);
+            prev_tile = tile;
+            block_sync();  // (2) warp totals ready
             tile_lookback<S, W, NW, true>(prm.lb, tile, pos, 0, lane, sm.wagg, zero, pr, sm.cin);
-            block_sync();  // carry ready
-            block_sync();  // per-sub-chunk dL/da partials ready
+            block_sync();  // (3) carry ready
         } else {
             // ================= compute warps =================
             const int sub = warp * TPW + lane / LC;
@@ -184,35 +217,43 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
                     }
                 }
             } else {
-                for (int i = tid; i < (L + 1) * G * W; i += NTC) {
+                for (int i = tid; i < L * G * W; i += NTC) {
                     const int row = i / (G * W), rem = i - row * (G * W), g = rem / W, c = rem - g * W;
                     const int64_t t = t0 + row, d = d0 + c;
                     sm.stg[st].px[row][g][c] = (t < T && d < D) ? pxg[((b * T + t) * G + g) * D + d] : PxT(0.0f);
                 }
-                for (int i = tid; i < (L + 1) * S * W; i += NTC) {
+                for (int i = tid; i < L * S * W; i += NTC) {
                     const int row = i / (S * W), rem = i - row * (S * W), s = rem / W, c = rem - s * W;
                     const int64_t th = t0 - 1 + row, tg = t0 + row, d = d0 + c;
                     sm.stg[st].H[row][s][c] = (th >= 0 && th < T && d < D) ? prm.H[((b * T + th) * S + s) * D + d] : 0.0f;
-                    if (row < L) sm.stg[st].g[row][s][c] = (tg < T && d < D) ? prm.dLdH[((b * T + tg) * S + s) * D + d] : 0.0f;
+                    sm.stg[st].g[row][s][c] = (tg < T && d < D) ? prm.dLdH[((b * T + tg) * S + s) * D + d] : 0.0f;
                 }
             }
-            block_sync();  // tile set up
+            block_sync();  // (1) tile set up
 
             float wr[V][G];  // the recurrent weights of this thread's channels
 #pragma unroll
             for (int v = 0; v < V; ++v)
 #pragma unroll
                 for (int g = 0; g < G; ++g) wr[v][g] = sm.w[g][cc + v];
-            // ---- linearisation at (h_{t-1}, x_t) for every row ----
-            float jA[R][S * S][V], sens[R][NS][V];
+
+            // ---- linearisation at (h_{t-1}, x_t) and the sub-chunk's element,
+            //      composed in scan order (latest row first) ----
+            float jA[R][S * S][V], sens[R][NS][V], gr[R][S][V];
+            ElemV<S, V> mine, excl, pre;
 #pragma unroll
-            for (int r = 0; r < R; ++r) {
+            for (int v = 0; v < V; ++v) elem_identity<S>(mine.e[v]);
+#pragma unroll
+            for (int r = R - 1; r >= 0; --r) {
                 const int row = sub * R + r;
+                const bool rvalid = (tb + r < T) && cvalid;
                 float pv[G][V], hv[S][V];
 #pragma unroll
                 for (int g = 0; g < G; ++g) lds_row<V>(&sm.stg[st].px[row][g][cc], pv[g]);
 #pragma unroll
                 for (int s = 0; s < S; ++s) lds_row<V>((t0 == 0 && row == 0) ? &sm.hprev[s][cc] : &sm.stg[st].H[row][s][cc], hv[s]);
+#pragma unroll
+                for (int s = 0; s < S; ++s) lds_row<V>(&sm.stg[st].g[row][s][cc], gr[r][s]);
 #pragma unroll
                 for (int v = 0; v < V; ++v) {
                     float pg[G], spv[S], A[S * S], se[NS];
@@ -221,92 +262,32 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
 #pragma unroll
                     for (int s = 0; s < S; ++s) spv[s] = hv[s][v];
                     Cell::bwd(pg, wr[v], spv, A, se);
+                    if (!rvalid) {
+                        // past the end of the sequence: the identity element
+#pragma unroll
+                        for (int a = 0; a < S * S; ++a) A[a] = (a % (S + 1) == 0) ? 1.0f : 0.0f;
+#pragma unroll
+                        for (int s = 0; s < S; ++s) gr[r][s][v] = 0.0f;
+                    }
 #pragma unroll
                     for (int a = 0; a < S * S; ++a) jA[r][a][v] = A[a];
 #pragma unroll
                     for (int n = 0; n < NS; ++n) sens[r][n][v] = se[n];
-                }
-            }
-#pragma unroll
-            for (int a = 0; a < S * S; ++a)
-#pragma unroll
-                for (int v = 0; v < V; ++v) sm.firstA[sub][a][cc + v] = jA[0][a][v];
-            // the last sub-chunk also needs A at the first row of the next tile
-            float nextA[S * S][V];
-            if (sub == NSUB - 1) {
-                const int64_t tn = t0 + L;
-#pragma unroll
-                for (int v = 0; v < V; ++v) {
-                    float A[S * S];
-#pragma unroll
-                    for (int a = 0; a < S * S; ++a) A[a] = 0.0f;
-                    if (tn < T && cvalid) {
-                        float pv[G], spv[S], se[NS];
-#pragma unroll
-                        for (int g = 0; g < G; ++g) pv[g] = PxTraits<PxT>::cvt(sm.stg[st].px[L][g][cc + v]);
-#pragma unroll
-                        for (int s = 0; s < S; ++s) spv[s] = sm.stg[st].H[L][s][cc + v];
-                        Cell::bwd(pv, wr[v], spv, A, se);
-                    }
-#pragma unroll
-                    for (int a = 0; a < S * S; ++a) nextA[a][v] = A[a];
-                }
-            }
-            block_sync();  // first-row Jacobians shared
-
-            // ---- reverse-scan elements (M_t, g_t), M_t = A_{t+1}^T ----
-            float eM[R][S * S][V];
-#pragma unroll
-            for (int r = 0; r < R; ++r)
-#pragma unroll
-                for (int v = 0; v < V; ++v) {
-                    const int64_t t = tb + r;
-                    float A[S * S];
-#pragma unroll
-                    for (int a = 0; a < S * S; ++a) {
-                        if (r + 1 < R) A[a] = jA[r + 1][a][v];
-                        else if (sub + 1 < NSUB) A[a] = sm.firstA[sub + 1][a][cc + v];
-                        else A[a] = nextA[a][v];
-                    }
-                    const bool has_next = (t + 1 < T) && cvalid;
-                    const bool rvalid = (t < T) && cvalid;
+                    float M[S * S], gv[S], bv[S];
 #pragma unroll
                     for (int i = 0; i < S; ++i)
 #pragma unroll
-                        for (int m = 0; m < S; ++m) {
-                            float val = has_next ? A[m * S + i] : 0.0f;  // transpose
-                            if (!rvalid) val = (i == m) ? 1.0f : 0.0f;     // past the end: identity
-                            eM[r][i * S + m][v] = val;
-                        }
-                }
-            ElemV<S, V> mine, excl, pre;
-            float gr[R][S][V];
-#pragma unroll
-            for (int r = 0; r < R; ++r)
-#pragma unroll
-                for (int s = 0; s < S; ++s) {
-                    lds_row<V>(&sm.stg[st].g[sub * R + r][s][cc], gr[r][s]);
-                    if (tb + r >= T)
-#pragma unroll
-                        for (int v = 0; v < V; ++v) gr[r][s][v] = 0.0f;
-                }
-#pragma unroll
-            for (int v = 0; v < V; ++v) {
-                elem_identity<S>(mine.e[v]);
-#pragma unroll
-                for (int r = R - 1; r >= 0; --r) {
-                    float M[S * S], gv[S];
-#pragma unroll
-                    for (int a = 0; a < S * S; ++a) M[a] = eM[r][a][v];
+                        for (int m = 0; m < S; ++m) M[i * S + m] = A[m * S + i];  // A^T
 #pragma unroll
                     for (int s = 0; s < S; ++s) gv[s] = gr[r][s][v];
-                    compose_after<S>(M, gv, mine.e[v]);
+                    mat_t_vec<S>(A, gv, bv);
+                    compose_after<S>(M, bv, mine.e[v]);
                 }
             }
             warp_prefix<S, V, LC, W, NW, true>(mine, excl, warp, lane, sm.wagg);
-            block_sync();  // warp totals ready
+            block_sync();  // (2) warp totals ready
             sub_prefix<S, V, LC, W, NW, true>(excl, warp, lane, sm.wagg, pre);
-            block_sync();  // carry ready
+            block_sync();  // (3) carry ready
 
             // ---- lambda and the gradient epilogue ----
             float da_acc[G][V];
@@ -318,25 +299,23 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
             bool bad = false;
 #pragma unroll
             for (int v = 0; v < V; ++v) {
-                float x[S], cv[S];
+                float x[S], cv[S];  // x = mu_{t+1}, the propagated adjoint after row t
 #pragma unroll
                 for (int s = 0; s < S; ++s) cv[s] = sm.cin[s][cc + v];
                 apply<S>(pre.e[v].A, pre.e[v].b, cv, x);
 #pragma unroll
                 for (int r = R - 1; r >= 0; --r) {
                     const bool rvalid = (tb + r < T) && cvalid;
-                    float M[S * S], gv[S], y[S];
+                    float lam[S], A[S * S];
 #pragma unroll
-                    for (int a = 0; a < S * S; ++a) M[a] = eM[r][a][v];
+                    for (int s = 0; s < S; ++s) lam[s] = gr[r][s][v] + x[s];
 #pragma unroll
-                    for (int s = 0; s < S; ++s) gv[s] = gr[r][s][v];
-                    apply<S>(M, gv, x, y);
-#pragma unroll
-                    for (int s = 0; s < S; ++s) x[s] = y[s];
+                    for (int a = 0; a < S * S; ++a) A[a] = jA[r][a][v];
+                    mat_t_vec<S>(A, lam, x);  // mu_t
                     float se[NS], dp[G], da[G];
 #pragma unroll
                     for (int n = 0; n < NS; ++n) se[n] = sens[r][n][v];
-                    Cell::grads(se, x, dp, da);
+                    Cell::grads(se, lam, dp, da);
 #pragma unroll
                     for (int g2 = 0; g2 < G; ++g2) {
                         outp[r][g2][v] = dp[g2];
@@ -346,14 +325,9 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
                         }
                     }
                     if (r == 0 && tb == 0 && rvalid && prm.dLdh0) {
-                        // dL/dh0 = A_0^T lambda_0, A_0 at (h0, x_0)
+                        // dL/dh0 = A_0^T lambda_0 = mu_0
 #pragma unroll
-                        for (int i = 0; i < S; ++i) {
-                            float acc = 0.0f;
-#pragma unroll
-                            for (int m = 0; m < S; ++m) acc = __fmaf_rn(jA[0][m * S + i][v], x[m], acc);
-                            prm.dLdh0[(b * S + i) * D + d0 + cc + v] = acc;
-                        }
+                        for (int s = 0; s < S; ++s) prm.dLdh0[(b * S + s) * D + d0 + cc + v] = x[s];
                     }
                 }
             }
@@ -366,23 +340,14 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
                 }
             }
             if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(prm.lb.status, kStatusNonFinite);
-
-            // ---- per-tile dL/da partial, summed over sub-chunks in a fixed order ----
 #pragma unroll
             for (int g = 0; g < G; ++g)
 #pragma unroll
-                for (int v = 0; v < V; ++v) sm.da[sub][g][cc + v] = da_acc[g][v];
-            block_sync();  // per-sub-chunk dL/da partials ready
-            for (int i = tid; i < G * W; i += NTC) {
-                const int g = i / W, ch = i - (i / W) * W;
-                float acc = 0.0f;
-#pragma unroll 4
-                for (int sb = 0; sb < NSUB; ++sb) acc += sm.da[sb][g][ch];
-                prm.part[(tile * G + g) * W + ch] = acc;
-            }
+                for (int v = 0; v < V; ++v) sm.da[it & 1][sub][g][cc + v] = da_acc[g][v];
         }
-        block_sync();  // stage st, the ticket slot and the shared partials are free again
     }
+    block_sync();  // the last tile's partials are in place
+    if (is_scan && prev_tile >= 0) store_tile_partial<Sh, PxT>(sm, (it - 1) & 1, prm, prev_tile, lane);
 }
 
 // dL/da[g][d] = sum over batch rows b, then over tiles along time, of the

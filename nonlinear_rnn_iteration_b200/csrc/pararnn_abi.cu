@@ -34,20 +34,23 @@ pararnn_status cuda_fail(cudaError_t e, const char* what) {
 // FwdShape<Cell, PxT, V channels/thread, LC lanes across channels, warps,
 //          R rows/thread, blocks/SM budget, shared-memory stages, TMA>
 // TMA path (D * element size a multiple of 16 bytes, 16-byte aligned rows):
-// 32 or 64 channels per tile, chosen by measurement on the workloads.
-// Element-wise path otherwise: 32 channels per tile.
+// 32 channels per tile, shapes chosen by measurement on the workloads.
+// Element-wise path otherwise: 32 channels per tile.  Blocks of 8 warps
+// (7 compute + the scan warp) or 6 warps let two blocks share an SM with
+// 128 or 168 registers per thread; a 9-warp block puts 5 warps of two blocks
+// on one of the SM's four schedulers and caps registers at 96.
 template <typename PxT> using FwdLinT = FwdShape<CellLinear, PxT, 4, 8, 4, 8, 2, 3, true>;
 template <typename PxT> using FwdGruT = FwdShape<CellGRU, PxT, 4, 8, 8, 4, 2, 2, true>;
-template <typename PxT> using FwdLstmT = FwdShape<CellLSTM, PxT, 2, 16, 8, 2, 2, 2, true>;
-template <typename PxT> using BwdLinT = FwdShape<CellLinear, PxT, 2, 16, 8, 4, 2, 2, true>;
-template <typename PxT> using BwdGruT = FwdShape<CellGRU, PxT, 2, 16, 8, 4, 2, 2, true>;
-template <typename PxT> using BwdLstmT = FwdShape<CellLSTM, PxT, 2, 16, 8, 2, 1, 2, true>;
-template <typename PxT> using FwdLinS = FwdShape<CellLinear, PxT, 1, 32, 8, 4, 2, 2, false>;
-template <typename PxT> using FwdGruS = FwdShape<CellGRU, PxT, 1, 32, 8, 4, 2, 2, false>;
-template <typename PxT> using FwdLstmS = FwdShape<CellLSTM, PxT, 1, 32, 8, 2, 2, 2, false>;
-template <typename PxT> using BwdLinS = FwdShape<CellLinear, PxT, 1, 32, 8, 2, 2, 2, false>;
-template <typename PxT> using BwdGruS = FwdShape<CellGRU, PxT, 1, 32, 8, 2, 2, 2, false>;
-template <typename PxT> using BwdLstmS = FwdShape<CellLSTM, PxT, 1, 32, 8, 2, 1, 2, false>;
+template <typename PxT> using FwdLstmT = FwdShape<CellLSTM, PxT, 2, 16, 7, 4, 2, 2, true>;
+template <typename PxT> using BwdLinT = FwdShape<CellLinear, PxT, 2, 16, 5, 8, 2, 2, true>;
+template <typename PxT> using BwdGruT = FwdShape<CellGRU, PxT, 2, 16, 5, 8, 2, 2, true>;
+template <typename PxT> using BwdLstmT = FwdShape<CellLSTM, PxT, 2, 16, 5, 4, 2, 2, true>;
+template <typename PxT> using FwdLinS = FwdShape<CellLinear, PxT, 1, 32, 7, 4, 2, 2, false>;
+template <typename PxT> using FwdGruS = FwdShape<CellGRU, PxT, 1, 32, 7, 4, 2, 2, false>;
+template <typename PxT> using FwdLstmS = FwdShape<CellLSTM, PxT, 1, 32, 7, 4, 2, 2, false>;
+template <typename PxT> using BwdLinS = FwdShape<CellLinear, PxT, 1, 32, 7, 4, 2, 2, false>;
+template <typename PxT> using BwdGruS = FwdShape<CellGRU, PxT, 1, 32, 7, 4, 2, 2, false>;
+template <typename PxT> using BwdLstmS = FwdShape<CellLSTM, PxT, 1, 32, 7, 2, 2, 2, false>;
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far beyond any legitimate wait
 constexpr int kMaxK = 64;
@@ -254,8 +257,8 @@ pararnn_status launch_bwd(const Plan& pl, BwdParams prm, float* dLda, cudaStream
     memset(&maps, 0, sizeof maps);
     if (Sh::kTma) {
         const int64_t rows = prm.B * prm.T;
-        pararnn_status s = make_map(&maps.px, prm.px, sizeof(PxT) == 2, prm.D, Sh::G, rows, Sh::W, Sh::L + 1);
-        if (s == PARARNN_OK) s = make_map(&maps.H, prm.H, false, prm.D, Sh::S, rows, Sh::W, Sh::L + 1);
+        pararnn_status s = make_map(&maps.px, prm.px, sizeof(PxT) == 2, prm.D, Sh::G, rows, Sh::W, Sh::L);
+        if (s == PARARNN_OK) s = make_map(&maps.H, prm.H, false, prm.D, Sh::S, rows, Sh::W, Sh::L);
         if (s == PARARNN_OK) s = make_map(&maps.g, prm.dLdH, false, prm.D, Sh::S, rows, Sh::W, Sh::L);
         if (s != PARARNN_OK) return s;
     }
