@@ -16,10 +16,8 @@
 //   * one scan warp takes tile tickets, issues the tensor-memory-accelerator
 //     loads of the tiles ahead, and does each tile's decoupled look-back.
 // Per Newton iteration of a tile:
-//   1. compute warps evaluate f, A_t, beta_t on their rows (the previous
-//      row's state comes from the neighbouring sub-chunk through shared
-//      memory), compose them, and combine the sub-chunks of each warp with a
-//      shuffle scan;                                                 [barrier]
+//   1. compute warps evaluate f, A_t, beta_t on their rows, compose them,
+//      and combine the sub-chunks of each warp with a shuffle scan;  [barrier]
 //   2. the scan warp composes the warp totals into the tile's element,
 //      publishes it, finds the carry by look-back over earlier tiles of the
 //      same channels and publishes the state after the tile; meanwhile each
@@ -27,9 +25,14 @@
 //                                                                    [barrier]
 //   3. compute warps apply that prefix to the carry and re-walk their rows:
 //      h^(k+1).
-// Iteration k+1 needs h^(k) just before the tile: that is the carry found in
-// iteration k.  HBM traffic is the minimum: pre-activations read once, h^(K)
-// written once.
+// The first row of a sub-chunk is linearised at the state just before it.
+// For the warm start each thread evaluates f(0, x) on that row itself; after
+// iteration k it is h^(k+1) just before the sub-chunk, which is the value the
+// re-walk starts from (the prefix applied to the carry), so no state crosses
+// between sub-chunks and two block barriers per iteration suffice.  The same
+// value is also produced, rounded along a different path, as the last row of
+// the sub-chunk before; the two agree to rounding.  HBM traffic is the
+// minimum: pre-activations read once, h^(K) written once.
 #pragma once
 
 #include "cells.cuh"
@@ -91,7 +94,6 @@ struct FwdSmem {
     static_assert(sizeof(FwdStage<Sh, PxT>) % 128 == 0, "each TMA stage starts 128-byte aligned");
     FwdStage<Sh, PxT> px[Sh::NSTAGE];
     float wagg[Sh::NWARPS][Sh::NA][Sh::W];  // each compute warp's composed element
-    float edge[Sh::NSUB][Sh::S][Sh::W];     // each sub-chunk's last state (current iterate)
     float cin[Sh::S][Sh::W];                // the state just before the tile (current iterate)
     float w[Sh::G][Sh::W];                  // the tile's recurrent weights
     uint64_t bar[Sh::NSTAGE];
@@ -190,14 +192,11 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
                 block_sync();  // carry ready
             } else {
                 const int K = prm.K;
-                for (int k = 0; k <= K; ++k) {
-                    block_sync();  // edges ready
-                    if (k == K) break;
+                for (int k = 0; k < K; ++k) {
                     if (k > 0) probe_issue<S, W>(prm.lb, tile, chunk, k, lane, pr);
                     block_sync();  // warp totals ready
                     tile_lookback<S, W, NW, false>(prm.lb, tile, chunk, k, lane, sm.wagg, first_carry, pr, sm.cin);
                     block_sync();  // carry ready
-                    if (k + 1 == K && !prm.resid) break;
                 }
             }
         } else {
@@ -228,31 +227,6 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
                 }
             }
             block_sync();  // tile set up
-            // h^(0) just before the tile: h0 for the first tile, else the warm
-            // start of the previous row (row 0 of a nonlinear cell's stage);
-            // read by sub-chunk 0 after the next barrier
-            if (need_prev && tid < W) {
-                const int64_t d = d0 + tid;
-                float f[S] = {};
-                if (d < D) {
-                    if (t0 == 0) {
-#pragma unroll
-                        for (int s = 0; s < S; ++s) f[s] = prm.h0 ? prm.h0[(b * S + s) * D + d] : 0.0f;
-                    } else {
-                        float pv[G], wv[G];
-#pragma unroll
-                        for (int g = 0; g < G; ++g) {
-                            pv[g] = Sh::ROW0 ? PxTraits<PxT>::cvt(sm.px[st].v[0][g][tid])
-                                             : PxTraits<PxT>::cvt(pxg[((b * T + t0 - 1) * G + g) * D + d]);
-                            wv[g] = sm.w[g][tid];
-                        }
-                        Cell::warm(pv, wv, f);
-                    }
-                }
-#pragma unroll
-                for (int s = 0; s < S; ++s) sm.cin[s][tid] = f[s];
-            }
-
             // pre-activations of row r of this thread, V channels per gate
             auto load_p = [&](int r, float (&pv)[G][V]) {
 #pragma unroll
@@ -324,22 +298,52 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
                         for (int s = 0; s < S; ++s) h[r][s][v] = f[s];
                     }
                 }
-                if (need_prev) {
+                // h^(0) just before the sub-chunk: h0 at the start of a row,
+                // else the warm start of the row before (in the stage, except
+                // for the linear cell's first sub-chunk)
+                float hin[S][V];
 #pragma unroll
-                    for (int s = 0; s < S; ++s)
+                for (int s = 0; s < S; ++s)
 #pragma unroll
-                        for (int v = 0; v < V; ++v) sm.edge[sub][s][cc + v] = h[R - 1][s][v];
+                    for (int v = 0; v < V; ++v) hin[s][v] = 0.0f;
+                if (need_prev && cvalid) {
+                    if (tb == 0) {
+                        if (prm.h0)
+#pragma unroll
+                            for (int s = 0; s < S; ++s)
+#pragma unroll
+                                for (int v = 0; v < V; ++v) hin[s][v] = prm.h0[(b * S + s) * D + d0 + cc + v];
+                    } else {
+                        float pv[G][V];
+                        if (Sh::ROW0 + sub * R - 1 >= 0) {
+#pragma unroll
+                            for (int g = 0; g < G; ++g) lds_row<V>(&sm.px[st].v[Sh::ROW0 + sub * R - 1][g][cc], pv[g]);
+                        } else {
+#pragma unroll
+                            for (int g = 0; g < G; ++g)
+#pragma unroll
+                                for (int v = 0; v < V; ++v)
+                                    pv[g][v] = PxTraits<PxT>::cvt(pxg[((b * T + tb - 1) * G + g) * D + d0 + cc + v]);
+                        }
+#pragma unroll
+                        for (int v = 0; v < V; ++v) {
+                            float pg[G], f[S];
+#pragma unroll
+                            for (int g = 0; g < G; ++g) pg[g] = pv[g][v];
+                            Cell::warm(pg, wr[v], f);
+#pragma unroll
+                            for (int s = 0; s < S; ++s) hin[s][v] = f[s];
+                        }
+                    }
                 }
                 const int K = prm.K;
                 for (int k = 0; k <= K; ++k) {
-                    block_sync();  // edges ready
                     // ---- 1. elements of iteration k+1 and the residual of iterate k ----
                     float sp[S][V];
 #pragma unroll
                     for (int s = 0; s < S; ++s)
 #pragma unroll
-                        for (int v = 0; v < V; ++v)
-                            sp[s][v] = !need_prev ? 0.0f : (sub == 0 ? sm.cin[s][cc + v] : sm.edge[sub - 1][s][cc + v]);
+                        for (int v = 0; v < V; ++v) sp[s][v] = hin[s][v];
                     float eA[R][S * S][V], eb[R][S][V];
                     float res = 0.0f;
 #pragma unroll
@@ -406,6 +410,8 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
                         for (int s = 0; s < S; ++s) cv[s] = sm.cin[s][cc + v];
                         apply<S>(pre.e[v].A, pre.e[v].b, cv, x);
 #pragma unroll
+                        for (int s = 0; s < S; ++s) hin[s][v] = x[s];  // h^(k+1) just before the sub-chunk
+#pragma unroll
                         for (int r = 0; r < R; ++r) {
                             float A[S * S], be[S], y[S];
 #pragma unroll
@@ -419,12 +425,6 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
                                 h[r][s][v] = y[s];
                             }
                         }
-                    }
-                    if (need_prev) {
-#pragma unroll
-                        for (int s = 0; s < S; ++s)
-#pragma unroll
-                            for (int v = 0; v < V; ++v) sm.edge[sub][s][cc + v] = h[R - 1][s][v];
                     }
                     if (k + 1 == K && !prm.resid) break;  // no residual pass wanted
                 }
@@ -445,7 +445,10 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
                 if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(prm.lb.status, kStatusNonFinite);
             }
         }
-        block_sync();  // stage st and the ticket slot are free again
+        // No barrier here: the next tile's barrier (tile set up) comes before
+        // its scan warp refills a stage or rewrites a ticket slot, and every
+        // other shared array is rewritten only after a barrier that all of
+        // this tile's readers have passed.
     }
 }
 

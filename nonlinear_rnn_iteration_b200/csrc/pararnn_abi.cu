@@ -41,7 +41,7 @@ pararnn_status cuda_fail(cudaError_t e, const char* what) {
 // on one of the SM's four schedulers and caps registers at 96.
 template <typename PxT> using FwdLinT = FwdShape<CellLinear, PxT, 4, 8, 4, 8, 2, 3, true>;
 template <typename PxT> using FwdGruT = FwdShape<CellGRU, PxT, 4, 8, 8, 4, 2, 2, true>;
-template <typename PxT> using FwdLstmT = FwdShape<CellLSTM, PxT, 2, 16, 7, 4, 2, 2, true>;
+template <typename PxT> using FwdLstmT = FwdShape<CellLSTM, PxT, 2, 16, 7, 5, 2, 2, true>;
 template <typename PxT> using BwdLinT = FwdShape<CellLinear, PxT, 2, 16, 5, 8, 2, 2, true>;
 template <typename PxT> using BwdGruT = FwdShape<CellGRU, PxT, 2, 16, 5, 8, 2, 2, true>;
 template <typename PxT> using BwdLstmT = FwdShape<CellLSTM, PxT, 2, 16, 5, 4, 2, 2, true>;
