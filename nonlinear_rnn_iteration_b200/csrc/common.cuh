@@ -127,20 +127,35 @@ __device__ __forceinline__ void block_sync() { asm volatile("bar.sync 0;" ::: "m
 
 // ---- numerics --------------------------------------------------------------
 
-__device__ __forceinline__ float sigmoid_f(float x) { return __fdividef(1.0f, 1.0f + __expf(-x)); }
+// e^x = 2^(x log2 e) with the PTX approximate base-2 exponential, and the
+// PTX approximate reciprocal (both flush subnormal results to zero; the
+// state and gates here never need them).  e^x overflowing to +inf and
+// 1/inf = 0 give the saturated limits below exactly.
+__device__ __forceinline__ float exp2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float rcp_approx(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+constexpr float kLog2e = 1.4426950408889634f;
 
-// tanh from its definition, tanh|x| = 1 - 2 / (e^{2|x|} + 1), with the odd
+// sigma(x) = 1 / (1 + e^{-x})
+__device__ __forceinline__ float sigmoid_f(float x) { return rcp_approx(1.0f + exp2_approx(x * -kLog2e)); }
+
+// tanh from its definition, tanh x = 1 - 2 / (e^{2x} + 1), with the odd
 // Taylor series x - x^3/3 + 2x^5/15 - 17x^7/315 below |x| = 1/16, where the
 // subtraction would cancel (the first omitted term is below 1e-12 of tanh
-// there); odd symmetry restores the sign.  e^{2|x|} overflowing to +inf gives
-// exactly 1.  Relative error a few 1e-7 over the whole range.
+// there).  e^{2x} overflowing to +inf gives exactly 1, underflowing to 0
+// exactly -1.
 __device__ __forceinline__ float tanh_f(float x) {
-    const float ax = fabsf(x);
-    const float e = __expf(2.0f * ax);
-    const float big = 1.0f - __fdividef(2.0f, e + 1.0f);
-    const float x2 = ax * ax;
-    const float poly = ax * __fmaf_rn(x2, __fmaf_rn(x2, __fmaf_rn(x2, -17.0f / 315.0f, 2.0f / 15.0f), -1.0f / 3.0f), 1.0f);
-    return copysignf(ax < 0.0625f ? poly : big, x);
+    const float big = __fmaf_rn(-2.0f, rcp_approx(exp2_approx(x * (2.0f * kLog2e)) + 1.0f), 1.0f);
+    const float x2 = x * x;
+    const float poly = x * __fmaf_rn(x2, __fmaf_rn(x2, __fmaf_rn(x2, -17.0f / 315.0f, 2.0f / 15.0f), -1.0f / 3.0f), 1.0f);
+    return fabsf(x) < 0.0625f ? poly : big;
 }
 
 // max that keeps a NaN (so a non-finite residual is reported, not hidden)
