@@ -190,8 +190,10 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
             if (prev_tile >= 0) store_tile_partial<Sh, PxT>(sm, (it - 1) & 1, prm, prev_tile, lane);
             prev_tile = tile;
             block_sync();  // (2) warp totals ready
-            tile_lookback<S, W, NW, true>(prm.lb, tile, pos, 0, lane, sm.wagg, zero, pr, sm.cin);
+            Inclusive<S, W> inc;
+            tile_lookback<S, W, NW, true>(prm.lb, tile, pos, 0, lane, sm.wagg, zero, pr, sm.cin, inc);
             block_sync();  // (3) carry ready
+            publish_inclusive<S, W>(prm.lb, tile, 0, lane, inc);
         } else {
             // ================= compute warps =================
             const int sub = warp * TPW + lane / LC;

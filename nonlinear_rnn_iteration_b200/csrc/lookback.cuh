@@ -342,14 +342,25 @@ __device__ __forceinline__ void sub_prefix(const ElemV<S, V>& excl, int warp, in
     }
 }
 
-// Step 2b (warp 0, after the first barrier): compose the warp totals into
-// the tile's element, publish it, find the carry by look-back, publish the
-// state after the tile, and write the carry-in to cin.
+// The state after a tile, for the W/32 channels of one scan-warp lane,
+// computed before the carry barrier and published after it.
+template <int S, int W>
+struct Inclusive {
+    float v[W / 32][S];
+};
+
+// Step 2b (the scan warp, after the first barrier): compose the warp totals
+// into the tile's element, find the carry and write it to cin; return the
+// state after the tile in `out`, to be published by publish_inclusive once
+// the compute warps have been released.  When the early probe found the
+// predecessor's state, nobody waits on this tile's aggregate -- its own
+// state follows within a barrier's time -- so the aggregate is published
+// only before a real look-back, where successors may need it meanwhile.
 template <int S, int W, int NW, bool kReverse>
 __device__ __forceinline__ void tile_lookback(const LookbackCtx& cx, int64_t tile, int64_t pos, int slot, int lane,
                                               const float (&wagg)[NW][S * S + S][W],
                                               const float (&first_carry)[W / 32][S], const Probe<S, W>& pr,
-                                              float (&cin)[S][W]) {
+                                              float (&cin)[S][W], Inclusive<S, W>& out) {
     constexpr int NA = S * S + S;
     constexpr int CPL = W / 32;
     Elem<S> tot[CPL];
@@ -369,8 +380,12 @@ __device__ __forceinline__ void tile_lookback(const LookbackCtx& cx, int64_t til
         }
     }
     float carry[CPL][S];
-    bool probed = false;
-    if (pos > 0) {
+    if (pos == 0) {
+#pragma unroll
+        for (int j = 0; j < CPL; ++j)
+#pragma unroll
+            for (int s = 0; s < S; ++s) carry[j][s] = first_carry[j][s];
+    } else {
         // the predecessor's inclusive state, if the early probe found it published
         bool ok = word_ok(pr.st, cx.epoch) && static_cast<uint32_t>(pr.st) == kTileInclusive;
 #pragma unroll
@@ -380,39 +395,39 @@ __device__ __forceinline__ void tile_lookback(const LookbackCtx& cx, int64_t til
                 ok &= word_ok(pr.inc[j][s], cx.epoch);
                 carry[j][s] = word_val(pr.inc[j][s]);
             }
-        probed = __all_sync(0xffffffffu, ok);
-    }
-    if (pos == 0) {
+        if (!__all_sync(0xffffffffu, ok)) {
+            // publish the aggregate first, so that successors never wait on
+            // this tile's look-back
+            float vals[CPL][NA];
 #pragma unroll
-        for (int j = 0; j < CPL; ++j)
+            for (int j = 0; j < CPL; ++j) {
 #pragma unroll
-            for (int s = 0; s < S; ++s) carry[j][s] = first_carry[j][s];
-    } else {
-        // publish the aggregate first, so that successors never wait on this
-        // tile's look-back (it costs a few stores)
-        float vals[CPL][NA];
+                for (int a = 0; a < S * S; ++a) vals[j][a] = tot[j].A[a];
 #pragma unroll
-        for (int j = 0; j < CPL; ++j) {
-#pragma unroll
-            for (int a = 0; a < S * S; ++a) vals[j][a] = tot[j].A[a];
-#pragma unroll
-            for (int s = 0; s < S; ++s) vals[j][S * S + s] = tot[j].b[s];
+                for (int s = 0; s < S; ++s) vals[j][S * S + s] = tot[j].b[s];
+            }
+            publish_words<NA, W>(cx.agg + (tile * cx.nSlots + slot) * NA * W, vals, cx.epoch, lane);
+            __syncwarp();
+            if (lane == 0) st_status(cx.tstat + tile * cx.nSlots + slot, kTileAggregate, cx.epoch);
+            lookback_carry<S, W>(cx, tile, pos, slot, lane, carry);
         }
-        publish_words<NA, W>(cx.agg + (tile * cx.nSlots + slot) * NA * W, vals, cx.epoch, lane);
-        __syncwarp();
-        if (lane == 0) st_status(cx.tstat + tile * cx.nSlots + slot, kTileAggregate, cx.epoch);
-        if (!probed) lookback_carry<S, W>(cx, tile, pos, slot, lane, carry);
     }
-    float vals[CPL][S];
 #pragma unroll
-    for (int j = 0; j < CPL; ++j) apply<S>(tot[j].A, tot[j].b, carry[j], vals[j]);
-    publish_words<S, W>(cx.inc + (tile * cx.nSlots + slot) * S * W, vals, cx.epoch, lane);
-    __syncwarp();
-    if (lane == 0) st_status(cx.tstat + tile * cx.nSlots + slot, kTileInclusive, cx.epoch);
-#pragma unroll
-    for (int j = 0; j < CPL; ++j)
+    for (int j = 0; j < CPL; ++j) {
+        apply<S>(tot[j].A, tot[j].b, carry[j], out.v[j]);
 #pragma unroll
         for (int s = 0; s < S; ++s) cin[s][lane + 32 * j] = carry[j][s];
+    }
+}
+
+// Step 3 (the scan warp, after the carry barrier): publish the state after
+// the tile (inclusive words, then the status word).
+template <int S, int W>
+__device__ __forceinline__ void publish_inclusive(const LookbackCtx& cx, int64_t tile, int slot, int lane,
+                                                  const Inclusive<S, W>& out) {
+    publish_words<S, W>(cx.inc + (tile * cx.nSlots + slot) * S * W, out.v, cx.epoch, lane);
+    __syncwarp();
+    if (lane == 0) st_status(cx.tstat + tile * cx.nSlots + slot, kTileInclusive, cx.epoch);
 }
 
 }  // namespace pararnn

@@ -177,7 +177,8 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
             block_sync();  // tile set up
             if (lane == 0) {
                 // claim the tile NSTAGE-1 ahead and start streaming it in; its
-                // stage was freed by the previous iteration's last barrier
+                // stage was last read by the previous tile, whose readers have
+                // all passed this tile's set-up barrier
                 const int sn = (it + NSTAGE - 1) % NSTAGE;
                 const unsigned prev_t = sm.ticket[(it + NSTAGE - 2) % NSTAGE];
                 unsigned t2 = prev_t;
@@ -186,17 +187,20 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
                 if constexpr (Sh::kTma)
                     if (t2 < prm.nTiles && prev_t < prm.nTiles) issue_tile_load<Cell, PxT, Sh>(&tmap, sm, prm, t2, sn);
             }
+            Inclusive<S, W> inc;
             if constexpr (kLean) {
                 block_sync();  // warp totals ready
-                tile_lookback<S, W, NW, false>(prm.lb, tile, chunk, 0, lane, sm.wagg, first_carry, pr, sm.cin);
+                tile_lookback<S, W, NW, false>(prm.lb, tile, chunk, 0, lane, sm.wagg, first_carry, pr, sm.cin, inc);
                 block_sync();  // carry ready
+                publish_inclusive<S, W>(prm.lb, tile, 0, lane, inc);
             } else {
                 const int K = prm.K;
                 for (int k = 0; k < K; ++k) {
                     if (k > 0) probe_issue<S, W>(prm.lb, tile, chunk, k, lane, pr);
                     block_sync();  // warp totals ready
-                    tile_lookback<S, W, NW, false>(prm.lb, tile, chunk, k, lane, sm.wagg, first_carry, pr, sm.cin);
+                    tile_lookback<S, W, NW, false>(prm.lb, tile, chunk, k, lane, sm.wagg, first_carry, pr, sm.cin, inc);
                     block_sync();  // carry ready
+                    publish_inclusive<S, W>(prm.lb, tile, k, lane, inc);
                 }
             }
         } else {
