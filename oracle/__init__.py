@@ -19,10 +19,15 @@ Functions and what they follow:
   weights and the initial state (Method section, backward pass).
 * :func:`cell_step`, :func:`cell_jacobian`, :func:`cell_param_grads` -- one
   cell application and its closed-form derivatives, exposed for the pins.
+* :func:`head_gru_unroll`, :func:`head_gru_newton`, :func:`head_gru_step`,
+  :func:`head_gru_jacobian` -- the same for the head-wise GRU
+  (``ParaGRU(mix='head', n_heads)`` on the pararnn-torch page: block-diagonal
+  recurrent weights, one dense d x d block per head, d = D / n_heads).
 
 Cells: ``LINEAR`` (S=1, gates a,b), ``DIAG_GRU`` (S=1, gates z,r,c),
 ``DIAG_LSTM`` (S=2 state (c,h), gates i,f,o,c).  Layouts are row-major with
-channels fastest: px (B,T,G,D), w (G,D), h0 (B,S,D), H (B,T,S,D).
+channels fastest: px (B,T,G,D), w (G,D), h0 (B,S,D), H (B,T,S,D).  The
+head-wise GRU: px (B,T,3,D), U (3, n_heads, d, d), h0 (B,D), H (B,T,D).
 
 Every function here is pinned by ``tests/test_oracle_pins.py`` against
 library routines (torch.nn.GRU / LSTMCell, autograd, dense linear solves),
@@ -101,6 +106,13 @@ def _bind(so_path):
     lib.oracle_residual.restype = ctypes.c_double
     lib.oracle_adjoint.argtypes = [ci, i64, i64, i64, P, P, P, P, P, P, P, P, ci]
     lib.oracle_adjoint.restype = ci
+    for name in ("oracle_head_gru_step", "oracle_head_gru_jacobian"):
+        getattr(lib, name).argtypes = [ci, P, P, P, P]
+        getattr(lib, name).restype = None
+    lib.oracle_head_gru_unroll.argtypes = [i64, i64, i64, ci, P, P, P, P, ci]
+    lib.oracle_head_gru_unroll.restype = ci
+    lib.oracle_head_gru_newton.argtypes = [i64, i64, i64, ci, P, P, P, ci, P, P, ci]
+    lib.oracle_head_gru_newton.restype = ci
     return lib
 
 
@@ -200,3 +212,59 @@ def adjoint(cell, px, w, h0, H, dLdH, nthreads=None):
     if rc:
         raise ValueError("oracle_adjoint rejected its arguments (%d)" % rc)
     return dpx, da, dh0
+
+
+# ---- head-wise GRU ---------------------------------------------------------
+
+def _head_shape(px, U):
+    if px.ndim != 4 or px.shape[2] != 3:
+        raise ValueError("px must be (B,T,3,D), got %s" % (px.shape,))
+    B, T, _, D = px.shape
+    if U.ndim != 4 or U.shape[0] != 3 or U.shape[2] != U.shape[3] or U.shape[1] * U.shape[2] != D:
+        raise ValueError("U must be (3, n_heads, d, d) with n_heads * d = D, got %s" % (U.shape,))
+    return B, T, D, U.shape[1]
+
+
+def head_gru_step(p, U, s):
+    """One head: p (3, d) = (p_z, p_r, p_c), U (3, d, d), s (d,) -> f (d,)."""
+    lib = _load()
+    p, U, s = _f64(p), _f64(U), _f64(s)
+    d = s.shape[0]
+    out = np.zeros(d)
+    lib.oracle_head_gru_step(d, _ptr(p), _ptr(U), _ptr(s), _ptr(out))
+    return out
+
+
+def head_gru_jacobian(p, U, s):
+    """One head: d f / d s, (d, d)."""
+    lib = _load()
+    p, U, s = _f64(p), _f64(U), _f64(s)
+    d = s.shape[0]
+    A = np.zeros((d, d))
+    lib.oracle_head_gru_jacobian(d, _ptr(p), _ptr(U), _ptr(s), _ptr(A))
+    return A
+
+
+def head_gru_unroll(px, U, h0=None, nthreads=None):
+    lib = _load()
+    px, U, h0 = _f64(px), _f64(U), _f64(h0)
+    B, T, D, nh = _head_shape(px, U)
+    H = np.zeros((B, T, D))
+    rc = lib.oracle_head_gru_unroll(B, T, D, nh, _ptr(px), _ptr(U), _ptr(h0), _ptr(H), _threads(nthreads))
+    if rc:
+        raise ValueError("oracle_head_gru_unroll: bad arguments")
+    return H
+
+
+def head_gru_newton(px, U, h0=None, K=1, nthreads=None):
+    """Returns (H^(K), resid) with resid[k] = max |F(H^(k))| for k = 0..K."""
+    lib = _load()
+    px, U, h0 = _f64(px), _f64(U), _f64(h0)
+    B, T, D, nh = _head_shape(px, U)
+    H = np.zeros((B, T, D))
+    resid = np.zeros(K + 1)
+    rc = lib.oracle_head_gru_newton(B, T, D, nh, _ptr(px), _ptr(U), _ptr(h0), K, _ptr(H), _ptr(resid),
+                                    _threads(nthreads))
+    if rc:
+        raise ValueError("oracle_head_gru_newton: bad arguments")
+    return H, resid

@@ -432,3 +432,216 @@ int oracle_adjoint(int cell, int64_t B, int64_t T, int64_t D, const double* px, 
     free(part);
     return rc;
 }
+
+/* ==== head-wise GRU (block-diagonal recurrent weights) ====================
+ *
+ * The ParaGRU(mix='head', n_heads) variant of the pararnn-torch page
+ * (Models / Usage, "Dreamer-style block GRU": block-diagonal A, one dense
+ * block per head).  The page prints no equations; the reading here is the
+ * GRU of torch.nn.GRUCell with its recurrent weight restricted to
+ * block-diagonal form, written with this file's gate convention.  For one
+ * head of width d, state s (d values), pre-activations p = (p_z, p_r, p_c)
+ * (3 x d) and recurrent weights U_z, U_r, U_c (d x d each):
+ *     z = sig(p_z + U_z s),  r = sig(p_r + U_r s),  n = U_c s,
+ *     c = tanh(p_c + r * n), f = (1 - z) * s + z * c        (elementwise *)
+ * which is the diagonal GRU above when the U_g are diagonal.  Its Jacobian
+ * with respect to s is the dense d x d block
+ *     A = diag(1 - z) + diag(alpha) U_z + diag(beta) U_r + diag(gamma) U_c,
+ *     alpha = (c - s) z (1 - z),  beta = z (1 - c^2) n r (1 - r),
+ *     gamma = z (1 - c^2) r.
+ * Layouts (row-major): px (B,T,3,D) with D = n_heads * d and head h owning
+ * channels h*d .. h*d+d-1; U (3, n_heads, d, d) with U[g][h][i][j] the
+ * weight of state j in gate pre-activation i; h0 (B,D); H (B,T,D).
+ */
+
+/* one head, one step: out = f(s, p); p holds p_z[0..d), p_r[0..d), p_c[0..d);
+ * U holds U_z, U_r, U_c of the head, each d x d */
+void oracle_head_gru_step(int d, const double* p, const double* U, const double* s, double* out) {
+    const double* Uz = U;
+    const double* Ur = U + (size_t)d * d;
+    const double* Uc = U + 2 * (size_t)d * d;
+    for (int i = 0; i < d; ++i) {
+        double az = p[i], ar = p[d + i], n = 0.0;
+        for (int j = 0; j < d; ++j) {
+            az += Uz[(size_t)i * d + j] * s[j];
+            ar += Ur[(size_t)i * d + j] * s[j];
+            n += Uc[(size_t)i * d + j] * s[j];
+        }
+        double z = sig(az), r = sig(ar), c = tanh(p[2 * d + i] + r * n);
+        out[i] = (1.0 - z) * s[i] + z * c;
+    }
+}
+
+/* A[i*d + j] = d f_i / d s_j at (s, p) */
+void oracle_head_gru_jacobian(int d, const double* p, const double* U, const double* s, double* A) {
+    const double* Uz = U;
+    const double* Ur = U + (size_t)d * d;
+    const double* Uc = U + 2 * (size_t)d * d;
+    for (int i = 0; i < d; ++i) {
+        double az = p[i], ar = p[d + i], n = 0.0;
+        for (int j = 0; j < d; ++j) {
+            az += Uz[(size_t)i * d + j] * s[j];
+            ar += Ur[(size_t)i * d + j] * s[j];
+            n += Uc[(size_t)i * d + j] * s[j];
+        }
+        double z = sig(az), r = sig(ar), c = tanh(p[2 * d + i] + r * n);
+        double alpha = (c - s[i]) * z * (1.0 - z);
+        double beta = z * (1.0 - c * c) * n * r * (1.0 - r);
+        double gamma = z * (1.0 - c * c) * r;
+        for (int j = 0; j < d; ++j)
+            A[(size_t)i * d + j] = (i == j ? 1.0 - z : 0.0) + alpha * Uz[(size_t)i * d + j] +
+                                   beta * Ur[(size_t)i * d + j] + gamma * Uc[(size_t)i * d + j];
+    }
+}
+
+typedef struct {
+    int64_t B, T, D;
+    int nh, d, K, mode, nthreads, tid;
+    const double *px, *U, *h0;
+    double* H;
+    double resid[64];
+} hjob_t;
+
+/* pre-activations of head h at (b, t), gathered as p_z, p_r, p_c */
+static void head_p(const hjob_t* j, int64_t b, int64_t t, int h, double* p) {
+    for (int g = 0; g < 3; ++g)
+        for (int i = 0; i < j->d; ++i) p[g * j->d + i] = j->px[((b * j->T + t) * 3 + g) * j->D + (int64_t)h * j->d + i];
+}
+
+static const double* head_U(const hjob_t* j, int h, double* buf) {
+    /* U_z, U_r, U_c of head h gathered contiguously */
+    size_t dd = (size_t)j->d * j->d;
+    for (int g = 0; g < 3; ++g) memcpy(buf + g * dd, j->U + ((size_t)g * j->nh + h) * dd, dd * sizeof(double));
+    return buf;
+}
+
+static void head_h0(const hjob_t* j, int64_t b, int h, double* s) {
+    for (int i = 0; i < j->d; ++i) s[i] = j->h0 ? j->h0[b * j->D + (int64_t)h * j->d + i] : 0.0;
+}
+
+static void head_seq(hjob_t* j, int64_t b, int h) {
+    const int d = j->d;
+    const int64_t T = j->T;
+    size_t dd = (size_t)d * d;
+    double* Ubuf = (double*)malloc(3 * dd * sizeof(double));
+    double* s = (double*)malloc((size_t)(T > 0 ? T : 1) * d * sizeof(double));   /* iterate, (T, d) */
+    double* del = (double*)malloc((size_t)d * sizeof(double));
+    double* F = (double*)malloc((size_t)d * sizeof(double));
+    double* A = (double*)malloc(dd * sizeof(double));
+    double* p = (double*)malloc(3 * (size_t)d * sizeof(double));
+    double* prev = (double*)malloc((size_t)d * sizeof(double));
+    double* fv = (double*)malloc((size_t)d * sizeof(double));
+    double* tmp = (double*)malloc((size_t)d * sizeof(double));
+    const double* U = head_U(j, h, Ubuf);
+    if (j->mode == 0) {
+        /* sequential unroll */
+        head_h0(j, b, h, prev);
+        for (int64_t t = 0; t < T; ++t) {
+            head_p(j, b, t, h, p);
+            oracle_head_gru_step(d, p, U, prev, s + t * d);
+            memcpy(prev, s + t * d, d * sizeof(double));
+        }
+    } else {
+        /* warm start s^(0)_t = f(0, x_t) */
+        for (int i = 0; i < d; ++i) tmp[i] = 0.0;
+        for (int64_t t = 0; t < T; ++t) {
+            head_p(j, b, t, h, p);
+            oracle_head_gru_step(d, p, U, tmp, s + t * d);
+        }
+        for (int k = 0; k <= j->K; ++k) {
+            /* residual F(s^(k)), then (k < K) the Newton step: A_t at s_{t-1},
+             * delta_t = A_t delta_{t-1} - F_t by forward substitution */
+            double rk = 0.0;
+            for (int i = 0; i < d; ++i) del[i] = 0.0;
+            head_h0(j, b, h, prev);
+            for (int64_t t = 0; t < T; ++t) {
+                head_p(j, b, t, h, p);
+                oracle_head_gru_step(d, p, U, prev, fv);
+                for (int i = 0; i < d; ++i) {
+                    F[i] = s[t * d + i] - fv[i];
+                    rk = nanmax(rk, fabs(F[i]));
+                }
+                if (k < j->K) {
+                    oracle_head_gru_jacobian(d, p, U, prev, A);
+                    for (int i = 0; i < d; ++i) {
+                        double acc = -F[i];
+                        for (int m = 0; m < d; ++m) acc += A[(size_t)i * d + m] * del[m];
+                        tmp[i] = acc;
+                    }
+                    memcpy(del, tmp, d * sizeof(double));
+                }
+                memcpy(prev, s + t * d, d * sizeof(double));   /* s^(k)_t, the next row's s_{t-1} */
+                if (k < j->K)
+                    for (int i = 0; i < d; ++i) s[t * d + i] += del[i];
+            }
+            j->resid[k] = nanmax(j->resid[k], rk);
+        }
+    }
+    for (int64_t t = 0; t < T; ++t)
+        for (int i = 0; i < d; ++i) j->H[(b * T + t) * j->D + (int64_t)h * d + i] = s[t * d + i];
+    free(Ubuf); free(s); free(del); free(F); free(A); free(p); free(prev); free(fv); free(tmp);
+}
+
+static void* head_worker(void* arg) {
+    hjob_t* j = (hjob_t*)arg;
+    int64_t nseq = j->B * j->nh;
+    int64_t per = (nseq + j->nthreads - 1) / j->nthreads;
+    int64_t lo = (int64_t)j->tid * per, hi = lo + per < nseq ? lo + per : nseq;
+    for (int64_t q = lo; q < hi; ++q) head_seq(j, q / j->nh, (int)(q % j->nh));
+    return NULL;
+}
+
+static int head_run(hjob_t* proto, int nthreads) {
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > 256) nthreads = 256;
+    hjob_t* jobs = (hjob_t*)calloc((size_t)nthreads, sizeof(hjob_t));
+    pthread_t* th = (pthread_t*)calloc((size_t)nthreads, sizeof(pthread_t));
+    if (!jobs || !th) { free(jobs); free(th); return -2; }
+    for (int i = 0; i < nthreads; ++i) {
+        jobs[i] = *proto;
+        jobs[i].nthreads = nthreads;
+        jobs[i].tid = i;
+        for (int k = 0; k < 64; ++k) jobs[i].resid[k] = 0.0;
+    }
+    for (int i = 1; i < nthreads; ++i) pthread_create(&th[i], NULL, head_worker, &jobs[i]);
+    head_worker(&jobs[0]);
+    for (int i = 1; i < nthreads; ++i) pthread_join(th[i], NULL);
+    for (int k = 0; k < 64; ++k) {
+        double r = 0.0;
+        for (int i = 0; i < nthreads; ++i) r = nanmax(r, jobs[i].resid[k]);
+        proto->resid[k] = r;
+    }
+    free(jobs);
+    free(th);
+    return 0;
+}
+
+static int head_check(int64_t B, int64_t T, int64_t D, int nh, const double* px, const double* U) {
+    if (B < 0 || T < 0 || D < 0 || nh < 1 || D % nh != 0 || (B * T * D > 0 && (!px || !U))) return -1;
+    return 0;
+}
+
+/* Sequential unroll of the head-wise GRU. */
+int oracle_head_gru_unroll(int64_t B, int64_t T, int64_t D, int nh, const double* px, const double* U,
+                           const double* h0, double* H, int nthreads) {
+    if (head_check(B, T, D, nh, px, U)) return -1;
+    hjob_t j;
+    memset(&j, 0, sizeof j);
+    j.B = B; j.T = T; j.D = D; j.nh = nh; j.d = (int)(D / nh); j.px = px; j.U = U; j.h0 = h0; j.H = H; j.mode = 0;
+    return head_run(&j, nthreads);
+}
+
+/* K Newton iterations of the head-wise GRU from the warm start; resid (K+1
+ * doubles, may be NULL) receives max |F(H^(k))| for k = 0..K. */
+int oracle_head_gru_newton(int64_t B, int64_t T, int64_t D, int nh, const double* px, const double* U,
+                           const double* h0, int K, double* H, double* resid, int nthreads) {
+    if (head_check(B, T, D, nh, px, U) || K < 0 || K > 62) return -1;
+    hjob_t j;
+    memset(&j, 0, sizeof j);
+    j.B = B; j.T = T; j.D = D; j.nh = nh; j.d = (int)(D / nh); j.K = K; j.px = px; j.U = U; j.h0 = h0; j.H = H;
+    j.mode = 1;
+    int rc = head_run(&j, nthreads);
+    if (rc == 0 && resid)
+        for (int k = 0; k <= K; ++k) resid[k] = j.resid[k];
+    return rc;
+}

@@ -304,6 +304,138 @@ def pin_residual_monotone():
         assert all(res[k + 1] < res[k] for k in range(w.K)), "%s residuals not decreasing: %s" % (name, res)
 
 
+# ---- head-wise GRU (block-diagonal recurrent weights) ----------------------
+# One head of width d is torch.nn.GRUCell(3d, d) with
+#   x = (p_z, p_r, p_c), all biases 0,
+#   weight_ih row blocks (r | z | n) = ([0 I 0] | [-I 0 0] | [0 0 I]),
+#   weight_hh row blocks (r | z | n) = (U_r | -U_z | U_c):
+# negating the z pre-activation turns torch's kept-state weight into our
+# (1 - z), and torch's candidate tanh(W_in x + r * (W_hn h)) is our
+# c = tanh(p_c + r * (U_c h)).
+
+
+def _torch_head_cell(U):
+    d = U.shape[-1]
+    cell = torch.nn.GRUCell(3 * d, d, bias=True).double()
+    I, Z = np.eye(d), np.zeros((d, d))
+    w_ih = np.block([[Z, I, Z], [-I, Z, Z], [Z, Z, I]])
+    w_hh = np.concatenate([U[1], -U[0], U[2]], axis=0)
+    with torch.no_grad():
+        cell.weight_ih.copy_(torch.tensor(w_ih))
+        cell.weight_hh.copy_(torch.tensor(w_hh))
+        cell.bias_ih.zero_()
+        cell.bias_hh.zero_()
+    return cell
+
+
+def _head_inputs(B, T, nh, d, seed, h0=False):
+    rng = _rng(seed)
+    D = nh * d
+    px = rng.standard_normal((B, T, 3, D))
+    U = rng.uniform(-1.0, 1.0, (3, nh, d, d)) / np.sqrt(d)
+    hz = rng.standard_normal((B, D)) * 0.5 if h0 else None
+    return px, U, hz
+
+
+def _torch_head_unroll(px, U, h0):
+    B, T, _, D = px.shape
+    nh, d = U.shape[1], U.shape[2]
+    out = np.zeros((B, T, D))
+    for h in range(nh):
+        cell = _torch_head_cell(U[:, h])
+        sl = slice(h * d, (h + 1) * d)
+        s = torch.zeros(B, d, dtype=torch.float64) if h0 is None else torch.tensor(h0[:, sl])
+        for t in range(T):
+            x = torch.tensor(px[:, t, :, sl].reshape(B, 3 * d))
+            s = cell(x, s)
+            out[:, t, sl] = s.detach().numpy()
+    return out
+
+
+def pin_head_step_and_jacobian():
+    rng = _rng(31)
+    for d in (1, 3, 8):
+        for _ in range(10):
+            p = rng.standard_normal((3, d)) * 2.0
+            U = rng.uniform(-1.0, 1.0, (3, d, d))
+            s = rng.standard_normal(d)
+            cell = _torch_head_cell(U)
+            f = lambda x: cell(torch.tensor(p.reshape(1, 3 * d)), x.reshape(1, d)).reshape(d)
+            _close(oracle.head_gru_step(p, U, s), f(torch.tensor(s)).detach().numpy(), 1e-14, "head step d=%d" % d)
+            J = torch.autograd.functional.jacobian(f, torch.tensor(s)).numpy()
+            _close(oracle.head_gru_jacobian(p, U, s), J, 1e-12, "head Jacobian d=%d" % d)
+
+
+def pin_head_unroll():
+    for h0 in (False, True):
+        px, U, hz = _head_inputs(2, 9, 3, 4, seed=32, h0=h0)
+        _close(oracle.head_gru_unroll(px, U, hz), _torch_head_unroll(px, U, hz), 1e-13, "head unroll h0=%s" % h0)
+
+
+def pin_head_newton_dense():
+    # dense Newton on the whole trajectory: F(X)_t = X_t - f(X_{t-1}, x_t),
+    # Jacobian by autograd, each step by torch.linalg.solve; heads at once
+    B, T, nh, d = 1, 5, 2, 3
+    D = nh * d
+    for h0 in (False, True):
+        px, U, hz = _head_inputs(B, T, nh, d, seed=33, h0=h0)
+        cells = [_torch_head_cell(U[:, h]) for h in range(nh)]
+        s0 = torch.zeros(D, dtype=torch.float64) if hz is None else torch.tensor(hz[0])
+
+        def f_all(prev, t):
+            outs = []
+            for h in range(nh):
+                sl = slice(h * d, (h + 1) * d)
+                x = torch.tensor(px[0, t, :, sl].reshape(1, 3 * d))
+                outs.append(cells[h](x, prev[sl].reshape(1, d)).reshape(d))
+            return torch.cat(outs)
+
+        def F(Xflat):
+            X = Xflat.reshape(T, D)
+            rows, prev = [], s0
+            for t in range(T):
+                rows.append(X[t] - f_all(prev, t))
+                prev = X[t]
+            return torch.cat(rows)
+
+        X = torch.cat([f_all(torch.zeros(D, dtype=torch.float64), t) for t in range(T)])  # warm start
+        for k in range(1, 4):
+            J = torch.autograd.functional.jacobian(F, X)
+            X = X - torch.linalg.solve(J, F(X))
+            H, resid = oracle.head_gru_newton(px, U, hz, K=k)
+            _close(H[0], X.detach().numpy().reshape(T, D), 1e-11, "head Newton k=%d h0=%s" % (k, h0))
+            _close(resid[k], float(torch.max(torch.abs(F(X)))), 1e-11, "head residual k=%d" % k)
+
+
+def pin_head_prefix_exact_and_diagonal():
+    # Newton on the lower block-bidiagonal system makes the first k rows exact
+    # after k steps and everything exact after T steps
+    px, U, hz = _head_inputs(1, 8, 2, 3, seed=34, h0=True)
+    ref = _torch_head_unroll(px, U, hz)
+    for k in (1, 3, 5):
+        H, _ = oracle.head_gru_newton(px, U, hz, K=k)
+        _close(H[:, :k], ref[:, :k], 1e-12, "head prefix exact k=%d" % k)
+        if k == 1:  # not vacuous: one step leaves the later rows inexact
+            assert np.max(np.abs(H[:, k:] - ref[:, k:])) > 1e-6, "head Newton exact everywhere after one step"
+    H, _ = oracle.head_gru_newton(px, U, hz, K=8)
+    _close(H, ref, 1e-12, "head exact after T steps")
+    # diagonal blocks: the diagonal GRU, computed by its own code path
+    rng = _rng(35)
+    B, T, nh, d = 2, 20, 2, 3
+    D = nh * d
+    px = rng.standard_normal((B, T, 3, D))
+    a = rng.uniform(-0.5, 0.5, (3, D))
+    U = np.zeros((3, nh, d, d))
+    for g in range(3):
+        for h in range(nh):
+            U[g, h] = np.diag(a[g, h * d:(h + 1) * d])
+    Hh, rh = oracle.head_gru_newton(px, U, K=3)
+    Hd, rd = oracle.newton(oracle.DIAG_GRU, px, a, K=3)
+    _close(Hh, Hd[:, :, 0, :], 1e-13, "head with diagonal blocks vs the diagonal GRU")
+    _close(rh, rd, 1e-13, "head vs diagonal residual history")
+
+
 ALL_PINS = [pin_cell_step, pin_jacobian, pin_param_grads, pin_unroll, pin_newton_dense, pin_affine_one_step,
             pin_prefix_exact, pin_lstm_zero_weights, pin_adjoint_dense, pin_adjoint_bptt, pin_adjoint_fd,
-            pin_residual_monotone]
+            pin_residual_monotone, pin_head_step_and_jacobian, pin_head_unroll, pin_head_newton_dense,
+            pin_head_prefix_exact_and_diagonal]

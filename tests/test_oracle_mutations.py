@@ -38,6 +38,24 @@ MUTATIONS = {
                            "for (int m = 0; m < S; ++m) nl[i] += A[i * S + m] * lam[m];"),
     "adjoint_wrong_time_index": ("load_p(j, b, t + 1, d, pn);", "load_p(j, b, t, d, pn);"),
     "adjoint_da_uses_dp": ("ga += lam[i] * da[i * G + g];", "ga += lam[i] * dp[i * G + g];"),
+    # head-wise GRU
+    "head_step_weight_transposed": ("            az += Uz[(size_t)i * d + j] * s[j];\n            ar += Ur[(size_t)i * d + j] * s[j];\n"
+                                    "            n += Uc[(size_t)i * d + j] * s[j];\n        }\n"
+                                    "        double z = sig(az), r = sig(ar), c = tanh(p[2 * d + i] + r * n);\n        out[i]",
+                                    "            az += Uz[(size_t)j * d + i] * s[j];\n            ar += Ur[(size_t)i * d + j] * s[j];\n"
+                                    "            n += Uc[(size_t)i * d + j] * s[j];\n        }\n"
+                                    "        double z = sig(az), r = sig(ar), c = tanh(p[2 * d + i] + r * n);\n        out[i]"),
+    "head_reset_gate_dropped": ("c = tanh(p[2 * d + i] + r * n);\n        out[i]", "c = tanh(p[2 * d + i] + n);\n        out[i]"),
+    "head_jacobian_term_dropped": ("beta * Ur[(size_t)i * d + j] +", "0.0 * Ur[(size_t)i * d + j] +"),
+    "head_jacobian_transposed": ("A[(size_t)i * d + j] = (i == j ? 1.0 - z : 0.0)", "A[(size_t)j * d + i] = (i == j ? 1.0 - z : 0.0)"),
+    "head_newton_sign": ("double acc = -F[i];", "double acc = F[i];"),
+    "head_newton_linearised_at_new_iterate": (
+        "memcpy(prev, s + t * d, d * sizeof(double));   /* s^(k)_t, the next row's s_{t-1} */\n"
+        "                if (k < j->K)\n                    for (int i = 0; i < d; ++i) s[t * d + i] += del[i];",
+        "if (k < j->K)\n                    for (int i = 0; i < d; ++i) s[t * d + i] += del[i];\n"
+        "                memcpy(prev, s + t * d, d * sizeof(double));"),
+    "head_no_warm_start": ("oracle_head_gru_step(d, p, U, tmp, s + t * d);",
+                           "for (int i = 0; i < d; ++i) s[t * d + i] = 0.0;"),
 }
 
 
