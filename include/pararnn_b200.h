@@ -193,6 +193,50 @@ pararnn_status pararnn_newton_forward_noalloc(pararnn_cell cell, int64_t B, int6
                                               const float* h0, int K, float* H_out, float* resid_hist,
                                               int wait_status, void* stream);
 
+/* ---- head-wise GRU: block-diagonal recurrent weights --------------------
+ * ParaGRU(mix='head', n_heads) of the pararnn-torch page (Models / Usage,
+ * "Dreamer-style block GRU": block-diagonal A).  The page prints no
+ * equations; the cell here is the GRU of torch.nn.GRUCell with its recurrent
+ * weight restricted to n_heads dense d x d blocks (D = n_heads * d), in this
+ * library's gate convention.  For one head, state s (d values):
+ *     z = sig(p_z + U_z s),  r = sig(p_r + U_r s),  n = U_c s,
+ *     c = tanh(p_c + r * n), s' = (1 - z) * s + z * c       (* elementwise)
+ * -- the diagonal GRU above when every U_g is diagonal.  Its Jacobian is a
+ * dense d x d block per head, so each Newton iteration's scan multiplies d x d
+ * matrices (d^3 work per step, against d^2 for the sequential unroll).
+ * Newton iterations, warm start and K have the meaning of
+ * pararnn_newton_forward; each linear solve is done in the update form
+ * delta_t = A_t delta_{t-1} - F_t, h^(k+1) = h^(k) + delta.
+ *
+ * Layouts (row-major, device memory owned by the caller):
+ *   preacts  (B, T, 3, D)         float32 or bfloat16 (px_dtype), gates z, r, c
+ *   U        (3, n_heads, d, d)   float32: U[g][h][i][j] is the weight of state
+ *                                 j of head h in gate g's pre-activation i
+ *   h0       (B, D)               float32, or NULL for a zero initial state
+ *   H_out    (B, T, D)            float32
+ * d = D / n_heads must be 16, 32 or 64.
+ *
+ * Returns the workspace size for these sizes, or 0 when they are invalid
+ * (d not in {16, 32, 64}, D not a multiple of n_heads, K outside 1..64, B*T
+ * at or above 2^31).  It holds a second iterate buffer (K >= 2) and each
+ * chunk's d x d Jacobian product: about B*T*D*4 + B*T*n_heads*(d+2)*d*4/32
+ * bytes. */
+size_t pararnn_head_gru_workspace_bytes(int64_t B, int64_t T, int64_t D, int n_heads, int K);
+
+/* K Newton iterations of the head-wise GRU; H_out = h^(K).
+ *   workspace  >= pararnn_head_gru_workspace_bytes(B, T, D, n_heads, K)
+ *              bytes, 256-byte aligned device memory; no zero-filling needed
+ *              (only its 256-byte header is reset, on `stream`).
+ *   resid_hist NULL, or K+1 floats: max |F(h^(k))| for k = 0..K.
+ * Errors: PARARNN_EINVAL, with nothing launched, for invalid sizes or dtype,
+ * a missing or small workspace, and null, host or misaligned pointers;
+ * PARARNN_ECUDA if a launch fails.  A non-finite value in H_out is recorded in
+ * the workspace and returned by pararnn_status_sync(workspace, stream).  No
+ * thread block waits on another, so PARARNN_ETIMEOUT does not occur. */
+pararnn_status pararnn_head_gru_forward(int64_t B, int64_t T, int64_t D, int n_heads, pararnn_dtype px_dtype,
+                                        const void* preacts, const float* U, const float* h0, int K, float* H_out,
+                                        void* workspace, size_t ws_bytes, float* resid_hist, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

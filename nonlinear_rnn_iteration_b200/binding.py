@@ -37,6 +37,8 @@ SIGNATURES = {
     "pararnn_last_error": (ctypes.c_char_p, []),
     "pararnn_probe_wait_timeout": (_I, [_P, _SZ, _U64, _P]),
     "pararnn_newton_forward_noalloc": (_I, [_I, _I64, _I64, _I64, _I, _P, _P, _P, _I, _P, _P, _I, _P]),
+    "pararnn_head_gru_workspace_bytes": (_SZ, [_I64, _I64, _I64, _I, _I]),
+    "pararnn_head_gru_forward": (_I, [_I64, _I64, _I64, _I, _I, _P, _P, _P, _I, _P, _P, _SZ, _P, _P]),
 }
 
 _lib = None
@@ -134,6 +136,17 @@ def pararnn_newton_forward_noalloc(cell, B, T, D, px_dtype, preacts, diag_w, h0,
                                                  _ptr(H_out), _ptr(resid_hist), int(wait_status), _stream(stream))
 
 
+def pararnn_head_gru_workspace_bytes(B, T, D, n_heads, K):
+    return load().pararnn_head_gru_workspace_bytes(B, T, D, n_heads, K)
+
+
+def pararnn_head_gru_forward(B, T, D, n_heads, px_dtype, preacts, U, h0, K, H_out, workspace, ws_bytes, resid_hist,
+                             stream):
+    return load().pararnn_head_gru_forward(B, T, D, n_heads, px_dtype, _ptr(preacts), _ptr(U), _ptr(h0), K,
+                                           _ptr(H_out), _ptr(workspace), ws_bytes, _ptr(resid_hist),
+                                           _stream(stream))
+
+
 # ---- tensor-level helpers (allocation through torch, compute in the library) ----
 
 def _check(status, where):
@@ -208,3 +221,28 @@ def newton_backward(cell, px, H, dL_dH, diag_w=None, h0=None, workspace=None, wa
     if sync_status:
         _check(pararnn_status_sync(workspace, st), "pararnn_newton_backward (device status)")
     return dpx, da, dh0
+
+
+def head_gru_forward(px, U, h0=None, K=1, out=None, workspace=None, resid_hist=None, stream=None, sync_status=True):
+    """Head-wise GRU: px (B,T,3,D), U (3, n_heads, d, d) -> H = h^(K) (B,T,D), float32."""
+    import torch
+
+    if px.dim() != 4 or px.shape[2] != 3 or not px.is_contiguous():
+        raise ValueError("preacts must be contiguous (B, T, 3, D), got %s" % (tuple(px.shape),))
+    if U.dim() != 4 or U.shape[0] != 3 or U.shape[2] != U.shape[3] or not U.is_contiguous():
+        raise ValueError("U must be contiguous (3, n_heads, d, d), got %s" % (tuple(U.shape),))
+    B, T, _, D = px.shape
+    nh = U.shape[1]
+    if out is None:
+        out = torch.empty((B, T, D), dtype=torch.float32, device=px.device)
+    if workspace is None:
+        n = pararnn_head_gru_workspace_bytes(B, T, D, nh, K)
+        if n == 0:
+            raise PararnnError(EINVAL, "pararnn_head_gru_workspace_bytes", "invalid sizes")
+        workspace = torch.empty(n, dtype=torch.uint8, device=px.device)
+    st = stream if stream is not None else torch.cuda.current_stream(px.device)
+    _check(pararnn_head_gru_forward(B, T, D, nh, _dtype_code(px), px, U, h0, K, out, workspace, workspace.numel(),
+                                    resid_hist, st), "pararnn_head_gru_forward")
+    if sync_status:
+        _check(pararnn_status_sync(workspace, st), "pararnn_head_gru_forward (device status)")
+    return out

@@ -304,8 +304,10 @@ __global__ void probe_wait_kernel(unsigned* status, const word_t* word, uint32_t
 }  // namespace
 
 namespace pararnn {
-// lets the other translation unit of the library (noalloc.cu) report through pararnn_last_error()
+// let the library's other translation units (noalloc.cu, head_gru.cu) report
+// through pararnn_last_error() and check pointers the same way
 void set_last_error(const char* msg) { fail(PARARNN_OK, "%s", msg); }
+bool pointer_on_device(const void* p) { return device_reachable(p); }
 }  // namespace pararnn
 
 extern "C" {

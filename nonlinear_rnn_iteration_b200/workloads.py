@@ -17,6 +17,17 @@ lstm_4x32768x1024_k4      LSTM    4     32768    1024   4    f32
 gru_1x131072x4096_k2_bf16 GRU     1     131072   4096   2    bf16, + backward
 ========================  ======  ====  =======  =====  ===  ===============
 
+Head-wise GRU (block-diagonal recurrent weights, ParaGRU(mix='head')):
+
+===========================  ====  ====  ===  =======  ===  ===  ====
+name                         B     T     D    n_heads  d    K    px
+===========================  ====  ====  ===  =======  ===  ===  ====
+headgru_8x4096x512_h8_k3     8     4096  512  8        64   3    f32
+===========================  ====  ====  ===  =======  ===  ===  ====
+
+with px ~ N(0,1), recurrent blocks U_g ~ U(-1, 1) / sqrt(d) entrywise (so
+that U_g s stays O(1)), h0 = 0; draw order px, U; seed 5.
+
 Distributions: GRU / LSTM pre-activations px ~ N(0,1), diagonal recurrent
 weights a ~ U(-0.5, 0.5) per gate and channel, initial state h0 = 0.  Linear:
 decay a_t = sigmoid(N(0,1)) in gate slot 0 and input b_t ~ N(0,1) in slot 1.
@@ -160,3 +171,57 @@ def sample_channels(w: Workload, n: int, seed: int = 12345):
     n = min(n, w.B * w.D)
     flat = np.sort(rng.choice(w.B * w.D, size=n, replace=False))
     return [(int(c // w.D), int(c % w.D)) for c in flat]
+
+
+# --------------------------------------------------------------------------
+# head-wise GRU (block-diagonal recurrent weights)
+# --------------------------------------------------------------------------
+
+@dataclass(frozen=True)
+class HeadWorkload:
+    name: str
+    B: int
+    T: int
+    D: int
+    n_heads: int
+    K: int
+    px_dtype: str
+    seed: int
+
+    @property
+    def d(self) -> int:
+        return self.D // self.n_heads
+
+    @property
+    def elements(self) -> int:
+        return self.B * self.T * self.D
+
+
+HEAD_WORKLOADS = {
+    w.name: w
+    for w in [
+        HeadWorkload("headgru_8x4096x512_h8_k3", 8, 4096, 512, 8, 3, "f32", 5),
+    ]
+}
+
+
+def head_host_inputs(B: int, T: int, D: int, n_heads: int, seed: int) -> dict:
+    """px (B,T,3,D) ~ N(0,1) and U (3, n_heads, d, d) ~ U(-1,1)/sqrt(d), float32."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    d = D // n_heads
+    px = rng.standard_normal((B, T, 3, D), dtype=np.float32)
+    U = (rng.uniform(-1.0, 1.0, size=(3, n_heads, d, d)) / np.sqrt(d)).astype(np.float32)
+    return {"px": px, "U": U, "h0": None}
+
+
+def head_device_inputs(w: HeadWorkload, device, seed: int | None = None) -> dict:
+    """The same distributions drawn in device memory (torch generator)."""
+    import torch
+
+    g = torch.Generator(device=device)
+    g.manual_seed(w.seed if seed is None else seed)
+    px32 = torch.randn((w.B, w.T, 3, w.D), generator=g, device=device, dtype=torch.float32)
+    U = (torch.rand((3, w.n_heads, w.d, w.d), generator=g, device=device, dtype=torch.float32) * 2.0 - 1.0) / float(
+        np.sqrt(w.d))
+    px = px32.to(torch.bfloat16) if w.px_dtype == "bf16" else px32
+    return {"px32": px32, "px": px, "U": U, "h0": None}

@@ -1,0 +1,123 @@
+"""GPU parity of the head-wise GRU forward (block-diagonal recurrent weights)
+against the fp64 oracle, through the C ABI.
+
+Tolerances as for the diagonal cells (gpu_util.rel_err): H <= 1e-4; the
+residual history within 1e-4 of the largest residual; bf16 pre-activations
+against the oracle on the same bf16 values <= 1e-4.  Cases cover every
+supported head width (16, 32, 64), one and several heads, sequences that end
+inside a chunk, an initial state, K = 1..3 and K = T.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_util import rel_err, to_np
+from nonlinear_rnn_iteration_b200 import binding, workloads
+
+pytestmark = pytest.mark.gpu
+TOL_H = 1e-4
+DEV = "cuda:0"
+
+
+def _case(B, T, D, nh, seed, h0=False):
+    x = workloads.head_host_inputs(B, T, D, nh, seed)
+    hz = (0.5 * np.random.default_rng(seed + 1).standard_normal((B, D))).astype(np.float32) if h0 else None
+    t = lambda a: None if a is None else torch.from_numpy(np.ascontiguousarray(a)).to(DEV)
+    return x["px"], x["U"], hz, t(x["px"]), t(x["U"]), t(hz)
+
+
+CASES = [  # (B, T, D, n_heads, K)
+    (2, 100, 64, 1, 3),
+    (1, 77, 96, 3, 2),
+    (2, 40, 48, 3, 1),
+    (1, 130, 128, 2, 3),
+    (2, 64, 256, 4, 2),
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: "B%dT%dD%dh%dK%d" % c)
+@pytest.mark.parametrize("h0", [False, True])
+def test_head_forward_small(case, h0, cuda_device):
+    B, T, D, nh, K = case
+    px, U, hz, pxt, Ut, h0t = _case(B, T, D, nh, seed=D + T, h0=h0)
+    resid = torch.zeros(K + 1, device=DEV)
+    H = binding.head_gru_forward(pxt, Ut, h0t, K=K, resid_hist=resid)
+    ref, rref = oracle.head_gru_newton(px, U, hz, K=K)
+    assert rel_err(to_np(H), ref) <= TOL_H
+    r = resid.cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(r - rref) <= 1e-4 * max(1.0, rref.max()) + 1e-6 * np.abs(rref))
+
+
+def test_head_forward_bf16(cuda_device):
+    B, T, D, nh, K = 2, 90, 128, 2, 3
+    px, U, _, _, Ut, _ = _case(B, T, D, nh, seed=7)
+    pxb = workloads.round_bf16(px)
+    H = binding.head_gru_forward(torch.from_numpy(px).to(DEV).to(torch.bfloat16), Ut, None, K=K)
+    ref, _ = oracle.head_gru_newton(pxb, U, None, K=K)
+    assert rel_err(to_np(H), ref) <= TOL_H
+
+
+def test_head_k_equal_t_is_the_unroll(cuda_device):
+    B, T, D, nh = 1, 10, 64, 2
+    px, U, hz, pxt, Ut, h0t = _case(B, T, D, nh, seed=9, h0=True)
+    H = binding.head_gru_forward(pxt, Ut, h0t, K=T)
+    assert rel_err(to_np(H), oracle.head_gru_unroll(px, U, hz)) <= 5e-5
+
+
+def test_head_deterministic(cuda_device):
+    B, T, D, nh = 2, 200, 128, 2
+    _, _, _, pxt, Ut, _ = _case(B, T, D, nh, seed=11)
+    a = binding.head_gru_forward(pxt, Ut, None, K=3)
+    b = binding.head_gru_forward(pxt, Ut, None, K=3)
+    assert torch.equal(a, b)
+
+
+def test_head_full_size_sampled(cuda_device):
+    w = workloads.HEAD_WORKLOADS["headgru_8x4096x512_h8_k3"]
+    x = workloads.head_device_inputs(w, DEV)
+    resid = torch.zeros(w.K + 1, device=DEV)
+    H = binding.head_gru_forward(x["px"], x["U"], None, K=w.K, resid_hist=resid)
+    U = x["U"].cpu().numpy()
+    rng = np.random.default_rng(5)
+    for b, h in [(int(rng.integers(w.B)), int(rng.integers(w.n_heads))) for _ in range(3)]:
+        sl = slice(h * w.d, (h + 1) * w.d)
+        px = x["px"][b:b + 1, :, :, sl].cpu().numpy()
+        ref, _ = oracle.head_gru_newton(px, U[:, h:h + 1], None, K=w.K)
+        assert rel_err(to_np(H[b:b + 1, :, sl]), ref) <= TOL_H, (b, h)
+    r = resid.cpu().numpy()
+    assert np.isfinite(r).all() and r[-1] < 1e-2 * r[0]
+
+
+def test_head_rejects_bad_arguments(cuda_device):
+    px = torch.zeros((1, 4, 3, 16), device=DEV)
+    U = torch.zeros((3, 2, 8, 8), device=DEV)
+    H = torch.zeros((1, 4, 16), device=DEV)
+    ws = torch.zeros(1 << 20, dtype=torch.uint8, device=DEV)
+    # head width 8 is not supported; D not a multiple of n_heads; K out of range
+    assert binding.pararnn_head_gru_workspace_bytes(1, 4, 16, 2, 1) == 0
+    assert binding.pararnn_head_gru_workspace_bytes(1, 4, 50, 3, 1) == 0
+    assert binding.pararnn_head_gru_workspace_bytes(1, 4, 64, 1, 0) == 0
+    assert binding.pararnn_head_gru_forward(1, 4, 16, 2, binding.F32, px, U, None, 1, H, ws, ws.numel(), None,
+                                            None) == binding.EINVAL
+    # a workspace that is too small
+    n = binding.pararnn_head_gru_workspace_bytes(1, 4, 64, 1, 2)
+    px = torch.zeros((1, 4, 3, 64), device=DEV)
+    U = torch.zeros((3, 1, 64, 64), device=DEV)
+    H = torch.zeros((1, 4, 64), device=DEV)
+    assert binding.pararnn_head_gru_forward(1, 4, 64, 1, binding.F32, px, U, None, 2, H, ws, n - 1, None,
+                                            None) == binding.EINVAL
+    # host memory
+    assert binding.pararnn_head_gru_forward(1, 4, 64, 1, binding.F32, px.cpu().data_ptr(), U, None, 2, H, ws,
+                                            ws.numel(), None, None) == binding.EINVAL
+
+
+def test_head_empty_and_nonfinite(cuda_device):
+    px = torch.zeros((0, 5, 3, 64), device=DEV)
+    U = torch.zeros((3, 1, 64, 64), device=DEV)
+    assert binding.head_gru_forward(px, U, None, K=2).shape == (0, 5, 64)
+    px = torch.randn((1, 40, 3, 64), device=DEV)
+    px[0, 17, 2, 5] = float("nan")
+    with pytest.raises(binding.PararnnError) as e:
+        binding.head_gru_forward(px, U, None, K=2)
+    assert e.value.status == binding.ENONFINITE
