@@ -57,90 +57,91 @@ struct Params {
 template <typename PxT>
 __device__ __forceinline__ float ldp(const PxT* p) { return PxTraits<PxT>::cvt(*p); }
 
-// Shared state of one chunk walk: the head's weights transposed,
-// UT[g][j][i] = U_g[i][j] (so that thread i reads consecutive words), and the
-// per-step vectors.
+// Thread layout of a chunk walk: row i of the head is handled by TPR
+// consecutive threads (qt = 0..TPR-1); thread qt owns the SEG columns
+// m = qt + TPR*s of row i of U_z, U_r, U_c, kept in registers for the whole
+// chunk.  A row's dot products are summed over its TPR threads with
+// shuffles, and every thread of the row then evaluates the row's gates (the
+// redundancy is cheaper than another round through shared memory).  Vectors
+// over the head's state live in shared memory in the permuted order
+// vpos(m) = (m % TPR) * SEG + m / TPR, so a thread's SEG elements are
+// contiguous.
 template <int DH>
-struct Walk {
-    float UT[3][DH][DH];
-    float px[3][DH];      // p_z, p_r, p_c of the step
-    float sprev[DH];      // h^(k)_{t-1}
-    float scur[DH];       // h^(k)_t
-    float u[3][DH];       // U_g s_prev
-    float v[3][DH];       // U_g delta_{t-1} (re-walk)
-    float dz[DH], al[DH], be[DH], ga[DH], F[DH];
-    float del[2][DH];     // delta_{t-1}, delta_t
+struct Geo {
+    static constexpr int TPR = kThreads / DH;
+    static constexpr int SEG = DH / TPR;
+    static_assert(TPR * SEG == DH && TPR <= 32, "one row's threads share a warp");
+    static __device__ __forceinline__ int vpos(int m) { return (m % TPR) * SEG + m / TPR; }
 };
 
 template <int DH>
-__device__ void load_weights(Walk<DH>& w, const float* U, int nh, int h) {
-    for (int idx = threadIdx.x; idx < 3 * DH * DH; idx += kThreads) {
-        const int g = idx / (DH * DH), rem = idx - g * DH * DH, i = rem / DH, j = rem - i * DH;
-        w.UT[g][j][i] = U[((int64_t)(g * nh + h) * DH + i) * DH + j];
-    }
+__device__ __forceinline__ float row_sum(float v) {
+#pragma unroll
+    for (int o = Geo<DH>::TPR / 2; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
 }
 
-// h^(k) of row t of this head into dst (all d values): the iterate buffer, or
-// the warm start f(0, x_t) = sig(p_z) tanh(p_c) at k = 0; h0 (or 0) at t = -1.
-template <int DH, typename PxT>
-__device__ __forceinline__ void iterate_row(const Params& pr, int64_t b, int h, int64_t t, float* dst) {
-    const int i = threadIdx.x;
-    if (i >= DH) return;
-    const int64_t c = (int64_t)h * DH + i;
-    if (t < 0) {
-        dst[i] = pr.h0 ? pr.h0[b * pr.D + c] : 0.0f;
-    } else if (pr.Hold) {
-        dst[i] = pr.Hold[(b * pr.T + t) * pr.D + c];
-    } else {
-        const PxT* x = static_cast<const PxT*>(pr.px) + (b * pr.T + t) * 3 * pr.D + c;
-        dst[i] = sigmoid_f(ldp(x)) * tanh_f(ldp(x + 2 * pr.D));
-    }
-}
-
-// The cell at (s_prev, x_t) for row t: gates, f, F = h^(k)_t - f, and the
-// Jacobian's row factors.  Returns |F| of this thread's row (0 for others).
-template <int DH, typename PxT>
-__device__ __forceinline__ float linearise(Walk<DH>& w, const Params& pr, int64_t b, int h, int64_t t, bool with_v) {
-    const int tid = threadIdx.x;
-    // pre-activations and the iterate at row t
-    if (tid < 3 * DH) {
-        const int g = tid / DH, i = tid - g * DH;
-        w.px[g][i] = ldp(static_cast<const PxT*>(pr.px) + ((b * pr.T + t) * 3 + g) * pr.D + (int64_t)h * DH + i);
-    }
-    iterate_row<DH, PxT>(pr, b, h, t, w.scur);
-    // U_g s_prev (and U_g delta_{t-1} for the re-walk)
-    if (tid < 3 * DH) {
-        const int g = tid / DH, i = tid - g * DH;
-        float acc = 0.0f, acc2 = 0.0f;
-#pragma unroll 8
-        for (int j = 0; j < DH; ++j) {
-            const float uw = w.UT[g][j][i];
-            acc = __fmaf_rn(uw, w.sprev[j], acc);
-            if (with_v) acc2 = __fmaf_rn(uw, w.del[0][j], acc2);
+// The head's recurrent weights owned by this thread.
+template <int DH>
+struct RowU {
+    float z[Geo<DH>::SEG], r[Geo<DH>::SEG], c[Geo<DH>::SEG];
+    __device__ __forceinline__ void load(const float* U, int nh, int h, int i, int qt) {
+        constexpr int SEG = Geo<DH>::SEG, TPR = Geo<DH>::TPR;
+        const int64_t hs = (int64_t)DH * DH;
+#pragma unroll
+        for (int s = 0; s < SEG; ++s) {
+            const int m = qt + TPR * s;
+            z[s] = __ldg(U + (0 * nh + h) * hs + (int64_t)i * DH + m);
+            r[s] = __ldg(U + ((int64_t)1 * nh + h) * hs + (int64_t)i * DH + m);
+            c[s] = __ldg(U + ((int64_t)2 * nh + h) * hs + (int64_t)i * DH + m);
         }
-        w.u[g][i] = acc;
-        if (with_v) w.v[g][i] = acc2;
     }
-    __syncthreads();
-    float aF = 0.0f;
-    if (tid < DH) {
-        const int i = tid;
-        const float s = w.sprev[i];
-        const float z = sigmoid_f(w.px[0][i] + w.u[0][i]);
-        const float r = sigmoid_f(w.px[1][i] + w.u[1][i]);
-        const float n = w.u[2][i];
-        const float c = tanh_f(__fmaf_rn(r, n, w.px[2][i]));
-        const float f = __fmaf_rn(z, c - s, s);
-        const float zc = z * __fmaf_rn(-c, c, 1.0f);  // z (1 - c^2)
-        w.dz[i] = 1.0f - z;
-        w.al[i] = (c - s) * (z - z * z);
-        w.be[i] = zc * n * (r - r * r);
-        w.ga[i] = zc * r;
-        w.F[i] = w.scur[i] - f;
-        aF = fabsf(w.F[i]);
-    }
-    __syncthreads();
-    return aF;
+};
+
+// The inputs of one step for row i: pre-activations and h^(k)_t.
+struct StepIn {
+    float pz, pr, pc, s;
+};
+
+template <int DH, typename PxT>
+__device__ __forceinline__ StepIn load_step(const Params& pr, int64_t b, int h, int i, int64_t t) {
+    StepIn in;
+    const int64_t c = (int64_t)h * DH + i;
+    const PxT* x = static_cast<const PxT*>(pr.px) + (b * pr.T + t) * 3 * pr.D + c;
+    in.pz = ldp(x);
+    in.pr = ldp(x + pr.D);
+    in.pc = ldp(x + 2 * pr.D);
+    // h^(k)_t: the iterate buffer, or the warm start f(0, x_t) = sig(p_z) tanh(p_c)
+    in.s = pr.Hold ? pr.Hold[(b * pr.T + t) * pr.D + c] : sigmoid_f(in.pz) * tanh_f(in.pc);
+    return in;
+}
+
+// h^(k)_{t0-1} of row i: h0 (or 0) before the sequence, else as load_step
+template <int DH, typename PxT>
+__device__ __forceinline__ float iterate_before(const Params& pr, int64_t b, int h, int i, int64_t t0) {
+    if (t0 == 0) return pr.h0 ? pr.h0[b * pr.D + (int64_t)h * DH + i] : 0.0f;
+    return load_step<DH, PxT>(pr, b, h, i, t0 - 1).s;
+}
+
+// The cell's row i at (s_prev, x_t), given the row's pre-activation sums
+// u_g = (U_g s_prev)_i: F = h^(k)_t - f and the Jacobian's row factors.
+struct RowLin {
+    float F, dz, al, be, ga;
+};
+
+__device__ __forceinline__ RowLin row_linearise(const StepIn& in, float sp, float uz, float ur, float uc) {
+    RowLin o;
+    const float z = sigmoid_f(in.pz + uz);
+    const float r = sigmoid_f(in.pr + ur);
+    const float c = tanh_f(__fmaf_rn(r, uc, in.pc));
+    const float f = __fmaf_rn(z, c - sp, sp);
+    const float zc = z * __fmaf_rn(-c, c, 1.0f);  // z (1 - c^2)
+    o.F = in.s - f;
+    o.dz = 1.0f - z;
+    o.al = (c - sp) * (z - z * z);
+    o.be = zc * uc * (r - r * r);
+    o.ga = zc * r;
+    return o;
 }
 
 // max over the block into *resid: a warp max, then one atomic per warp
@@ -152,19 +153,98 @@ __device__ __forceinline__ void block_max_resid(float v, float* resid) {
 
 // ---- A: the chunk's Jacobian product and its delta from a zero carry -----
 // (or, with kResidOnly, just max |F(h^(k))| over the chunk)
-template <int DH, typename PxT, bool kResidOnly>
+//
+// The product P <- A_t P (d x d x d per step) runs on the tensor cores with
+// mma.sync m16n8k8 in TF32.  TF32 keeps 10 mantissa bits, so each operand is
+// kept as a TF32 head and a TF32 remainder, x = x_hi + x_lo, and the product
+// accumulates a_lo b_hi + a_hi b_lo + a_hi b_hi in float32 (the lo * lo term
+// is below float32 rounding): float32 accuracy from three TF32 products.
+// Every element is split once, by the thread that produces it, and stored as
+// a {hi, lo} pair; rows of pairs are padded to d + 4 pairs, which puts each
+// half-warp's 64-bit fragment loads on distinct banks.
+constexpr int kPad = 4;
+
+template <int DH>
 struct SmemA {
-    Walk<DH> w;
-    float AT[DH][DH];     // A_t transposed: AT[m][i] = A_t[i][m]
-    float Pm[2][DH][DH];  // running product, row-major
+    uint2 AT[DH][DH + kPad];     // A_t transposed (AT[m][i] = A_t[i][m]) as {hi, lo} TF32 pairs
+    uint2 Pm[2][DH][DH + kPad];  // running product, row-major, {hi, lo} pairs
+    float sv[2][DH];             // h^(k)_{t-1}, permuted (vpos)
+    float dv[2][DH];             // delta_{t-1}, permuted
 };
 
+__device__ __forceinline__ uint2 split_tf32(float x) {
+    uint32_t h, l;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(h) : "f"(x));
+    const float r = x - __uint_as_float(h);
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(l) : "f"(r));
+    return make_uint2(h, l);
+}
+
+__device__ __forceinline__ void mma_tf32(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Pout = A Pin, with A given transposed (AT[m][i] = A[i][m]); all three d x d
+// {hi, lo} arrays with row stride d + kPad.  The 16 x 8 output tiles are
+// spread over the 8 warps, the tiles of one warp sharing their rows (and so
+// their A fragments).  Fragment layout of m16n8k8 (lane = 4 g + t): A rows g
+// and g+8, columns t and t+4; B rows t and t+4, column g; C rows g and g+8,
+// columns 2t and 2t+1.
+template <int DH>
+__device__ __forceinline__ void matmul_tf32x3(const uint2 (*AT)[DH + kPad], const uint2 (*Pin)[DH + kPad],
+                                              uint2 (*Pout)[DH + kPad]) {
+    constexpr int MT = DH / 16, NT = DH / 8;             // 16-row and 8-column tiles
+    constexpr int WPM = (kThreads / 32) / MT;            // warps per row of tiles
+    constexpr int NPW = NT / WPM > 0 ? NT / WPM : 1;     // column tiles per warp
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    const int mt = warp % MT, nt0 = (warp / MT) * NPW;
+    if (nt0 >= NT) return;
+    const int r0 = mt * 16 + g;
+    float c[NPW][4];
+#pragma unroll
+    for (int n = 0; n < NPW; ++n)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) c[n][e] = 0.0f;
+#pragma unroll 2
+    for (int ks = 0; ks < DH / 8; ++ks) {
+        const int k0 = ks * 8 + t;
+        const uint2 a0 = AT[k0][r0], a1 = AT[k0][r0 + 8], a2 = AT[k0 + 4][r0], a3 = AT[k0 + 4][r0 + 8];
+        const uint32_t ahi[4] = {a0.x, a1.x, a2.x, a3.x}, alo[4] = {a0.y, a1.y, a2.y, a3.y};
+#pragma unroll
+        for (int n = 0; n < NPW; ++n) {
+            const int col = (nt0 + n) * 8 + g;
+            const uint2 b0 = Pin[k0][col], b1 = Pin[k0 + 4][col];
+            mma_tf32(c[n], alo, b0.x, b1.x);
+            mma_tf32(c[n], ahi, b0.y, b1.y);
+            mma_tf32(c[n], ahi, b0.x, b1.x);
+        }
+    }
+#pragma unroll
+    for (int n = 0; n < NPW; ++n) {
+        const int col = (nt0 + n) * 8 + 2 * t;
+        Pout[r0][col] = split_tf32(c[n][0]);
+        Pout[r0][col + 1] = split_tf32(c[n][1]);
+        Pout[r0 + 8][col] = split_tf32(c[n][2]);
+        Pout[r0 + 8][col + 1] = split_tf32(c[n][3]);
+    }
+}
+
+// Two block barriers per step: step t writes AT and the step-parity halves of
+// sv / dv (reading the other halves); after the first barrier the product
+// reads AT and Pm[cur] and writes Pm[cur ^ 1]; the second barrier frees AT
+// for the next step.  A buffer is rewritten only after a barrier that every
+// reader of its previous contents has passed.
 template <int DH, typename PxT, bool kResidOnly>
-__global__ void __launch_bounds__(kThreads) head_chunk_kernel(const Params pr) {
+__global__ void __launch_bounds__(kThreads, 2) head_chunk_kernel(const Params pr) {
+    using Gm = Geo<DH>;
+    constexpr int TPR = Gm::TPR, SEG = Gm::SEG;
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    auto& sm = *reinterpret_cast<SmemA<DH, PxT, kResidOnly>*>(smem_raw);
-    Walk<DH>& w = sm.w;
-    const int tid = threadIdx.x;
+    auto& sm = *reinterpret_cast<SmemA<DH>*>(smem_raw);
+    const int tid = threadIdx.x, i = tid / TPR, qt = tid % TPR;
     const int64_t task = blockIdx.x;
     const int64_t seq = task / pr.nChunks;
     const int chunk = (int)(task - seq * pr.nChunks);
@@ -173,100 +253,114 @@ __global__ void __launch_bounds__(kThreads) head_chunk_kernel(const Params pr) {
     const int64_t t0 = (int64_t)chunk * kChunk;
     const int64_t t1 = t0 + kChunk < pr.T ? t0 + kChunk : pr.T;
 
-    load_weights<DH>(w, pr.U, pr.nh, h);
-    iterate_row<DH, PxT>(pr, b, h, t0 - 1, w.sprev);
-    if (tid < DH) w.del[0][tid] = 0.0f;
+    RowU<DH> U;
+    U.load(pr.U, pr.nh, h, i, qt);
+    const float s_before = iterate_before<DH, PxT>(pr, b, h, i, t0);
+    if (qt == 0) {
+        sm.sv[0][Gm::vpos(i)] = s_before;
+        sm.dv[0][Gm::vpos(i)] = 0.0f;
+    }
+    if constexpr (!kResidOnly)
+        for (int idx = tid; idx < DH * DH; idx += kThreads)
+            sm.Pm[0][idx / DH][idx % DH] = make_uint2(idx / DH == idx % DH ? __float_as_uint(1.0f) : 0u, 0u);
+    StepIn nxt = load_step<DH, PxT>(pr, b, h, i, t0);
     __syncthreads();
 
-    // thread tile of the product: TM x TM entries of P
-    constexpr int TM = DH / 16;
-    const int i0 = (tid / 16) * TM, j0 = (tid % 16) * TM;
-    int cur = 0;
+    int par = 0, cur = 0;
     float rmax = 0.0f;
     for (int64_t t = t0; t < t1; ++t) {
-        rmax = nanmax_f(rmax, linearise<DH, PxT>(w, pr, b, h, t, false));
+        const StepIn in = nxt;
+        if (t + 1 < t1) nxt = load_step<DH, PxT>(pr, b, h, i, t + 1);
+        // (U_g s_prev)_i
+        float uz = 0.0f, ur = 0.0f, uc = 0.0f;
+#pragma unroll
+        for (int s = 0; s < SEG; ++s) {
+            const float x = sm.sv[par][qt * SEG + s];
+            uz = __fmaf_rn(U.z[s], x, uz);
+            ur = __fmaf_rn(U.r[s], x, ur);
+            uc = __fmaf_rn(U.c[s], x, uc);
+        }
+        uz = row_sum<DH>(uz);
+        ur = row_sum<DH>(ur);
+        uc = row_sum<DH>(uc);
+        const float sp = sm.sv[par][Gm::vpos(i)];
+        const RowLin L = row_linearise(in, sp, uz, ur, uc);
+        if (qt == 0) rmax = nanmax_f(rmax, fabsf(L.F));
         if constexpr (!kResidOnly) {
-            // A_t, transposed
-            for (int idx = tid; idx < DH * DH; idx += kThreads) {
-                const int m = idx / DH, i = idx - m * DH;  // AT[m][i] = A[i][m]
-                float a = (i == m) ? w.dz[i] : 0.0f;
-                a = __fmaf_rn(w.al[i], w.UT[0][m][i], a);
-                a = __fmaf_rn(w.be[i], w.UT[1][m][i], a);
-                a = __fmaf_rn(w.ga[i], w.UT[2][m][i], a);
-                sm.AT[m][i] = a;
+            // row i of A_t into AT, and delta_t = A_t delta_{t-1} - F_t
+            float dp = 0.0f;
+#pragma unroll
+            for (int s = 0; s < SEG; ++s) {
+                const int m = qt + TPR * s;
+                float a = __fmaf_rn(L.al, U.z[s], (m == i) ? L.dz : 0.0f);
+                a = __fmaf_rn(L.be, U.r[s], a);
+                a = __fmaf_rn(L.ga, U.c[s], a);
+                sm.AT[m][i] = split_tf32(a);
+                dp = __fmaf_rn(a, sm.dv[par][qt * SEG + s], dp);
             }
+            dp = row_sum<DH>(dp);
+            if (qt == 0) sm.dv[par ^ 1][Gm::vpos(i)] = dp - L.F;
+        }
+        if (qt == 0) sm.sv[par ^ 1][Gm::vpos(i)] = in.s;
+        __syncthreads();
+        if constexpr (!kResidOnly) {
+            matmul_tf32x3<DH>(sm.AT, sm.Pm[cur], sm.Pm[cur ^ 1]);
+            cur ^= 1;
             __syncthreads();
-            // delta_t = A_t delta_{t-1} - F_t
-            if (tid < DH) {
-                float acc = -w.F[tid];
-#pragma unroll 8
-                for (int m = 0; m < DH; ++m) acc = __fmaf_rn(sm.AT[m][tid], w.del[0][m], acc);
-                w.del[1][tid] = acc;
-            }
-            // P <- A_t P (P = A_t at the chunk's first step)
-            if (t == t0) {
-#pragma unroll
-                for (int a = 0; a < TM; ++a)
-#pragma unroll
-                    for (int c = 0; c < TM; ++c) sm.Pm[cur][i0 + a][j0 + c] = sm.AT[j0 + c][i0 + a];
-            } else {
-                float acc[TM][TM];
-#pragma unroll
-                for (int a = 0; a < TM; ++a)
-#pragma unroll
-                    for (int c = 0; c < TM; ++c) acc[a][c] = 0.0f;
-#pragma unroll 4
-                for (int m = 0; m < DH; ++m) {
-                    float av[TM], pv[TM];
-#pragma unroll
-                    for (int a = 0; a < TM; ++a) av[a] = sm.AT[m][i0 + a];
-#pragma unroll
-                    for (int c = 0; c < TM; ++c) pv[c] = sm.Pm[cur][m][j0 + c];
-#pragma unroll
-                    for (int a = 0; a < TM; ++a)
-#pragma unroll
-                        for (int c = 0; c < TM; ++c) acc[a][c] = __fmaf_rn(av[a], pv[c], acc[a][c]);
-                }
-#pragma unroll
-                for (int a = 0; a < TM; ++a)
-#pragma unroll
-                    for (int c = 0; c < TM; ++c) sm.Pm[cur ^ 1][i0 + a][j0 + c] = acc[a][c];
-                cur ^= 1;
-            }
         }
-        __syncthreads();
-        if (tid < DH) {
-            w.sprev[tid] = w.scur[tid];
-            if constexpr (!kResidOnly) w.del[0][tid] = w.del[1][tid];
-        }
-        __syncthreads();
+        par ^= 1;
     }
     if (pr.resid) block_max_resid(rmax, pr.resid + pr.k);
     if constexpr (!kResidOnly) {
         float* Pout = pr.P + task * DH * DH;
-        for (int idx = tid; idx < DH * DH; idx += kThreads) Pout[idx] = (&sm.Pm[cur][0][0])[idx];
-        if (tid < DH) pr.q[task * DH + tid] = w.del[0][tid];
+        for (int idx = tid; idx < DH * DH; idx += kThreads) {
+            const uint2 v = sm.Pm[cur][idx / DH][idx % DH];
+            Pout[idx] = __uint_as_float(v.x) + __uint_as_float(v.y);
+        }
+        if (qt == 0) pr.q[task * DH + i] = sm.dv[par][Gm::vpos(i)];
     }
 }
 
 // ---- B: the carries of one (batch row, head), chunk after chunk ----------
+// Thread i keeps row i of the next chunk's P in registers while it applies
+// the current one, so each chunk costs one dependent step, not a load's
+// latency.
 template <int DH>
 __global__ void __launch_bounds__(64) head_carry_kernel(const Params pr) {
     __shared__ float x[2][DH];
     const int64_t seq = blockIdx.x;
     const int i = threadIdx.x;
-    if (i < DH) x[0][i] = 0.0f;  // delta_{-1} = 0: h0 is given, not solved for
+    const bool act = i < DH;
+    if (act) x[0][i] = 0.0f;  // delta_{-1} = 0: h0 is given, not solved for
+    float4 row[DH / 4];
+    float qv = 0.0f;
+    auto fetch = [&](int c) {
+        const int64_t task = seq * pr.nChunks + c;
+        const float4* Prow = reinterpret_cast<const float4*>(pr.P + (task * DH + i) * DH);
+#pragma unroll
+        for (int m = 0; m < DH / 4; ++m) row[m] = Prow[m];
+        qv = pr.q[task * DH + i];
+    };
+    if (act) fetch(0);
     __syncthreads();
     int cur = 0;
     for (int c = 0; c < pr.nChunks; ++c) {
-        const int64_t task = seq * pr.nChunks + c;
-        if (i < DH) {
-            pr.carry[task * DH + i] = x[cur][i];
-            const float* Prow = pr.P + (task * DH + i) * DH;
-            float acc = pr.q[task * DH + i];
-#pragma unroll 8
-            for (int m = 0; m < DH; ++m) acc = __fmaf_rn(Prow[m], x[cur][m], acc);
-            x[cur ^ 1][i] = acc;
+        float4 r[DH / 4];
+        float qc = qv;
+#pragma unroll
+        for (int m = 0; m < DH / 4; ++m) r[m] = row[m];
+        if (act && c + 1 < pr.nChunks) fetch(c + 1);
+        if (act) {
+            pr.carry[(seq * pr.nChunks + c) * DH + i] = x[cur][i];
+            float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+            for (int m = 0; m < DH / 4; ++m) {
+                acc[0] = __fmaf_rn(r[m].x, x[cur][4 * m], acc[0]);
+                acc[1] = __fmaf_rn(r[m].y, x[cur][4 * m + 1], acc[1]);
+                acc[2] = __fmaf_rn(r[m].z, x[cur][4 * m + 2], acc[2]);
+                acc[3] = __fmaf_rn(r[m].w, x[cur][4 * m + 3], acc[3]);
+            }
+            x[cur ^ 1][i] = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + qc;
         }
         __syncthreads();
         cur ^= 1;
@@ -274,11 +368,21 @@ __global__ void __launch_bounds__(64) head_carry_kernel(const Params pr) {
 }
 
 // ---- C: re-walk each chunk from its carry and write h^(k+1) --------------
+// delta_t = A_t delta_{t-1} - F_t with A_t applied as
+// diag(1-z) + diag(alpha) U_z + diag(beta) U_r + diag(gamma) U_c; one block
+// barrier per step, the vectors double-buffered as in the chunk kernel.
+template <int DH>
+struct SmemC {
+    float sv[2][DH];
+    float dv[2][DH];
+};
+
 template <int DH, typename PxT>
-__global__ void __launch_bounds__(kThreads) head_walk_kernel(const Params pr) {
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    Walk<DH>& w = *reinterpret_cast<Walk<DH>*>(smem_raw);
-    const int tid = threadIdx.x;
+__global__ void __launch_bounds__(kThreads, 2) head_walk_kernel(const Params pr) {
+    using Gm = Geo<DH>;
+    constexpr int TPR = Gm::TPR, SEG = Gm::SEG;
+    __shared__ SmemC<DH> sm;
+    const int tid = threadIdx.x, i = tid / TPR, qt = tid % TPR;
     const int64_t task = blockIdx.x;
     const int64_t seq = task / pr.nChunks;
     const int chunk = (int)(task - seq * pr.nChunks);
@@ -287,30 +391,52 @@ __global__ void __launch_bounds__(kThreads) head_walk_kernel(const Params pr) {
     const int64_t t0 = (int64_t)chunk * kChunk;
     const int64_t t1 = t0 + kChunk < pr.T ? t0 + kChunk : pr.T;
 
-    load_weights<DH>(w, pr.U, pr.nh, h);
-    iterate_row<DH, PxT>(pr, b, h, t0 - 1, w.sprev);
-    if (tid < DH) w.del[0][tid] = pr.carry[task * DH + tid];
+    RowU<DH> U;
+    U.load(pr.U, pr.nh, h, i, qt);
+    const float s_before = iterate_before<DH, PxT>(pr, b, h, i, t0);
+    if (qt == 0) {
+        sm.sv[0][Gm::vpos(i)] = s_before;
+        sm.dv[0][Gm::vpos(i)] = pr.carry[task * DH + i];
+    }
+    StepIn nxt = load_step<DH, PxT>(pr, b, h, i, t0);
     __syncthreads();
+    int par = 0;
     bool bad = false;
     for (int64_t t = t0; t < t1; ++t) {
-        linearise<DH, PxT>(w, pr, b, h, t, true);
-        if (tid < DH) {
-            const int i = tid;
-            float d = __fmaf_rn(w.dz[i], w.del[0][i], -w.F[i]);
-            d = __fmaf_rn(w.al[i], w.v[0][i], d);
-            d = __fmaf_rn(w.be[i], w.v[1][i], d);
-            d = __fmaf_rn(w.ga[i], w.v[2][i], d);
-            const float hn = w.scur[i] + d;
+        const StepIn in = nxt;
+        if (t + 1 < t1) nxt = load_step<DH, PxT>(pr, b, h, i, t + 1);
+        float uz = 0.0f, ur = 0.0f, uc = 0.0f, vz = 0.0f, vr = 0.0f, vc = 0.0f;
+#pragma unroll
+        for (int s = 0; s < SEG; ++s) {
+            const float x = sm.sv[par][qt * SEG + s], y = sm.dv[par][qt * SEG + s];
+            uz = __fmaf_rn(U.z[s], x, uz);
+            ur = __fmaf_rn(U.r[s], x, ur);
+            uc = __fmaf_rn(U.c[s], x, uc);
+            vz = __fmaf_rn(U.z[s], y, vz);
+            vr = __fmaf_rn(U.r[s], y, vr);
+            vc = __fmaf_rn(U.c[s], y, vc);
+        }
+        uz = row_sum<DH>(uz);
+        ur = row_sum<DH>(ur);
+        uc = row_sum<DH>(uc);
+        vz = row_sum<DH>(vz);
+        vr = row_sum<DH>(vr);
+        vc = row_sum<DH>(vc);
+        const float sp = sm.sv[par][Gm::vpos(i)], dprev = sm.dv[par][Gm::vpos(i)];
+        const RowLin L = row_linearise(in, sp, uz, ur, uc);
+        float d = __fmaf_rn(L.dz, dprev, -L.F);
+        d = __fmaf_rn(L.al, vz, d);
+        d = __fmaf_rn(L.be, vr, d);
+        d = __fmaf_rn(L.ga, vc, d);
+        if (qt == 0) {
+            const float hn = in.s + d;
             pr.Hnew[(b * pr.T + t) * pr.D + (int64_t)h * DH + i] = hn;
             bad |= !isfinite(hn);
-            w.del[1][i] = d;
+            sm.sv[par ^ 1][Gm::vpos(i)] = in.s;
+            sm.dv[par ^ 1][Gm::vpos(i)] = d;
         }
         __syncthreads();
-        if (tid < DH) {
-            w.sprev[tid] = w.scur[tid];
-            w.del[0][tid] = w.del[1][tid];
-        }
-        __syncthreads();
+        par ^= 1;
     }
     if (__any_sync(0xffffffffu, bad) && (tid & 31) == 0) atomicOr(pr.status, kStatusNonFinite);
 }
@@ -351,11 +477,9 @@ cudaError_t set_smem(Kern k, size_t bytes) {
 
 template <int DH, typename PxT>
 cudaError_t launch_all(const Plan& pl, Params pr, float* H_out, float* Hbuf, int K, cudaStream_t st) {
-    const size_t smemA = sizeof(SmemA<DH, PxT, false>), smemR = sizeof(SmemA<DH, PxT, true>);
-    const size_t smemC = sizeof(Walk<DH>);
+    const size_t smemA = sizeof(SmemA<DH>), smemR = sizeof(SmemA<DH>);
     cudaError_t e = set_smem(head_chunk_kernel<DH, PxT, false>, smemA);
     if (e == cudaSuccess) e = set_smem(head_chunk_kernel<DH, PxT, true>, smemR);
-    if (e == cudaSuccess) e = set_smem(head_walk_kernel<DH, PxT>, smemC);
     if (e != cudaSuccess) return e;
     const unsigned ntask = (unsigned)(pl.nSeq * pl.nChunks);
     for (int k = 0; k < K; ++k) {
@@ -366,7 +490,7 @@ cudaError_t launch_all(const Plan& pl, Params pr, float* H_out, float* Hbuf, int
         pr.Hnew = ((K - (k + 1)) % 2 == 0) ? H_out : Hbuf;
         head_chunk_kernel<DH, PxT, false><<<ntask, kThreads, smemA, st>>>(pr);
         head_carry_kernel<DH><<<(unsigned)pl.nSeq, 64, 0, st>>>(pr);
-        head_walk_kernel<DH, PxT><<<ntask, kThreads, smemC, st>>>(pr);
+        head_walk_kernel<DH, PxT><<<ntask, kThreads, 0, st>>>(pr);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     if (pr.resid) {
