@@ -127,7 +127,7 @@ TF32_PER_BF16 = 1.1 / 2.25
 
 
 def time_head(w, device, steps, warmup):
-    """Device time of one head-wise forward call (CUDA events on the
+    """Device time of one head-wise GRU forward call (CUDA events on the
     launching stream); returns (ms, status name)."""
     import torch
 
@@ -160,6 +160,9 @@ def time_head(w, device, steps, warmup):
 
 
 def head_line(w, ms, status):
+    """A head-wise forward's line: time, elements/s, and the FLOP rate of its
+    Jacobian products -- 2 d^3 useful FLOP per step and (batch row, head),
+    issued as three TF32 products -- against the TF32 tensor peak."""
     peaks = measured_peaks()
     useful = 2.0 * w.d ** 3 * w.B * w.T * w.n_heads * w.K
     tf32_peak = peaks["bf16_tflops"] * TF32_PER_BF16
@@ -172,33 +175,8 @@ def head_line(w, ms, status):
                          "unit": "TFLOP/s", "frac_issued": round(3 * useful / (ms / 1e3) / 1e12 / tf32_peak, 4)}}
 
 
-def run_head(args):
-    """--workload <head-wise>: time that forward alone and print its line
-    (a profiling and inspection mode, not the bench contract's line)."""
-    import torch
-
-    from nonlinear_rnn_iteration_b200 import workloads
-
-    w = workloads.HEAD_WORKLOADS[args.workload]
-    if args.B or args.T:
-        w = workloads.HeadWorkload("%s@B%dT%d" % (w.name, args.B or w.B, args.T or w.T), args.B or w.B,
-                                   args.T or w.T, w.D, w.n_heads, w.K, w.px_dtype, w.seed)
-    device = torch.device("cuda", 0)
-    torch.cuda.set_device(device)
-    ms, status = time_head(w, device, args.steps, args.warmup)
-    line = {"workload": w.name, "metric": METRIC, "unit": UNIT, "data": "synthetic", **head_line(w, ms, status)}
-    print(json.dumps(line), flush=True)
-
-
 def head_workloads(device):
-    """Device-time lines for the head-wise GRU (block-diagonal weights).
-
-    Per step the forward multiplies two d x d Jacobian-block matrices per
-    (batch row, head): 2 d^3 useful FLOP, issued as three TF32 products
-    (head/remainder splitting) on the tensor cores.  The line reports the
-    call's time, elements/s and those products' FLOP rate over the whole call
-    against the TF32 peak (measured bf16 x nominal TF32/bf16 ratio).
-    """
+    """Device-time lines for the head-wise GRU workloads."""
     from nonlinear_rnn_iteration_b200 import workloads
 
     out = {}
@@ -206,6 +184,246 @@ def head_workloads(device):
         ms, status = time_head(w, device, steps=5, warmup=3)
         out[name] = head_line(w, ms, status)
     return out
+
+
+def recorded_traffic(kernel, workload):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel sources; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    e = rec.get("%s/%s" % (kernel, workload))
+    if not e or e.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.QUERY,
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        if self.path and os.path.exists(self.path):
+            for line in open(self.path):
+                f = [x.strip() for x in line.split(",")]
+                if len(f) >= 9:
+                    try:
+                        rows.append((float(f[1]), float(f[2]), float(f[3]), f[4], f[5], f[6], f[7], f[8]))
+                    except ValueError:
+                        pass
+            os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        loaded = [r for r in rows if r[2] > 200.0] or rows
+        sm = sorted(r[0] for r in loaded)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in loaded for i in range(4) if r[4 + i].lower() == "active"})
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
+                "samples": len(rows)}
+
+
+# --------------------------------------------------------------------------
+# the native arm
+# --------------------------------------------------------------------------
+
+class Problem:
+    """One workload's device buffers and its C-ABI step."""
+
+    def __init__(self, w, device, seed):
+        import torch
+
+        from nonlinear_rnn_iteration_b200 import binding, workloads
+
+        self.w, self.dev, self.b = w, device, binding
+        x = workloads.device_inputs(w, device, seed=seed, with_grad=w.backward)
+        self.px, self.a = x["px"], x["a"]
+        self.g = x.get("dLdH")
+        del x
+        self.H = torch.empty((w.B, w.T, w.S, w.D), dtype=torch.float32, device=device)
+        self.ws = binding.workspace_for(w.cell_id, w.B, w.T, w.D, w.K, device)
+        if w.backward:
+            self.dpx = torch.empty((w.B, w.T, w.G, w.D), dtype=torch.float32, device=device)
+            self.da = torch.empty((w.G, w.D), dtype=torch.float32, device=device)
+        self.code = binding.BF16 if w.px_dtype == "bf16" else binding.F32
+        self.stream = torch.cuda.current_stream(device)
+
+    def forward(self, px=None, H=None):
+        w = self.w
+        st = self.b.pararnn_newton_forward(w.cell_id, w.B, w.T, w.D, self.code, self.px if px is None else px,
+                                           self.a, None, w.K, self.H if H is None else H, self.ws,
+                                           self.ws.numel(), None, self.stream)
+        if st != 0:
+            raise RuntimeError("forward: %s %s" % (self.b.STATUS[st], self.b.pararnn_last_error()))
+
+    def backward(self):
+        w = self.w
+        st = self.b.pararnn_newton_backward(w.cell_id, w.B, w.T, w.D, self.code, self.px, self.a, None, self.H,
+                                            self.g, self.dpx, self.da, None, self.ws, self.ws.numel(), self.stream)
+        if st != 0:
+            raise RuntimeError("backward: %s %s" % (self.b.STATUS[st], self.b.pararnn_last_error()))
+
+    def step(self):
+        self.forward()
+        if self.w.backward:
+            self.backward()
+
+    def launches_per_step(self):
+        return 1 + (2 if self.w.backward else 0)
+
+    def check_status(self):
+        st = self.b.pararnn_status_sync(self.ws, self.stream)
+        if st != 0:
+            raise RuntimeError("device status %s" % self.b.STATUS[st])
+
+
+def time_device(prob, steps, warmup, dist, device, per_call=True):
+    """Returns (ms_per_step max over ranks, fwd_ms, bwd_ms) with CUDA events."""
+    import torch
+
+    for _ in range(warmup):
+        prob.step()
+    prob.check_status()
+    barrier(dist, device)
+    torch.cuda.synchronize(device)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(prob.stream)
+    for i in range(steps):
+        ev[i][0].record(prob.stream)
+        prob.forward()
+        ev[i][1].record(prob.stream)
+        if prob.w.backward:
+            prob.backward()
+        ev[i][2].record(prob.stream)
+    t1.record(prob.stream)
+    torch.cuda.synchronize(device)
+    barrier(dist, device)
+    total = t0.elapsed_time(t1)
+    fwd = sum(a.elapsed_time(b) for a, b, _ in ev) / steps
+    bwd = sum(b.elapsed_time(c) for _, b, c in ev) / steps
+    prob.check_status()
+    return reduce_max(dist, total, device) / steps, fwd, bwd
+
+
+def time_e2e(prob, steps):
+    """Same step through the public API with host buffers: pinned host ->
+    device copy of the pre-activations, the forward (and backward) call, device
+    -> host copy of the result, all inside the timed region."""
+    import torch
+
+    w = prob.w
+    px_host = torch.empty(prob.px.shape, dtype=prob.px.dtype, pin_memory=True)
+    px_host.copy_(prob.px)
+    H_host = torch.empty(prob.H.shape, dtype=torch.float32, pin_memory=True)
+    outs = [H_host]
+    if w.backward:
+        g_host = torch.empty(prob.g.shape, dtype=torch.float32, pin_memory=True)
+        g_host.copy_(prob.g)
+        dpx_host = torch.empty(prob.dpx.shape, dtype=torch.float32, pin_memory=True)
+        outs.append(dpx_host)
+    px_dev = torch.empty_like(prob.px)
+    s = prob.stream
+
+    def one():
+        px_dev.copy_(px_host, non_blocking=True)
+        if w.backward:
+            prob.g.copy_(g_host, non_blocking=True)
+        prob.forward(px=px_dev)
+        if w.backward:
+            prob.backward()
+        H_host.copy_(prob.H, non_blocking=True)
+        if w.backward:
+            dpx_host.copy_(prob.dpx, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(s)
+    for _ in range(steps):
+        one()
+    t1.record(s)
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1) / steps
+    h2d = px_host.numel() * px_host.element_size() + (g_host.numel() * 4 if w.backward else 0)
+    d2h = sum(o.numel() * o.element_size() for o in outs)
+    return ms, h2d, d2h
+
+
+def cpu_baseline(w, device, seed, target_s=12.0):
+    """The oracle as it stands, on a bounded sample of the workload's channels
+    (full length T each), on this host's cores."""
+    import numpy as np
+
+    import oracle
+    from nonlinear_rnn_iteration_b200 import workloads
+
+    threads = os.cpu_count() or 1
+    x = workloads.device_inputs(w, device, seed=seed)
+
+    def run(n):
+        chans = workloads.sample_channels(w, n, seed=5)
+        bs = [b for b, _ in chans]
+        ds = [d for _, d in chans]
+        import torch
+
+        bi, di = torch.tensor(bs, device=device), torch.tensor(ds, device=device)
+        # (1, T, G, n) contiguous fp64, prepared outside the timed region
+        px = np.ascontiguousarray(x["px"][bi, :, :, di].float().cpu().numpy().transpose(1, 2, 0)[None],
+                                  dtype=np.float64)
+        a = None if x["a"] is None else np.ascontiguousarray(x["a"][:, di].cpu().numpy(), dtype=np.float64)
+        t = time.perf_counter()
+        if w.cell == "linear":
+            oracle.unroll(w.cell_id, px, a, None, nthreads=threads)
+        else:
+            oracle.newton(w.cell_id, px, a, None, K=w.K, nthreads=threads)
+        return time.perf_counter() - t, n * w.T
+
+    n = max(threads, 8)
+    dt, el = run(n)
+    while dt < 1.0 and n < w.B * w.D:
+        n = min(w.B * w.D, n * 4)
+        dt, el = run(n)
+    n_final = int(min(w.B * w.D, max(n, n * target_s / max(dt, 1e-3))))
+    if n_final > n:
+        dt, el = run(n_final)
+        n = n_final
+    del x
+    kind = "sequential unroll" if w.cell == "linear" else "Newton K=%d with sequential solves" % w.K
+    return {"value": el / dt, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": "%d of %d channels at full T=%d (%s, fp64), %.1f s" % (n, w.B * w.D, w.T, kind, dt)}
 
 
 def extra_workloads(names, device, seed_base):
@@ -289,6 +507,24 @@ def run_native(args):
         print(json.dumps(line), flush=True)
     if dist is not None:
         dist.destroy_process_group()
+
+
+def run_head(args):
+    """--workload <head-wise>: time that forward alone and print its line
+    (a profiling and inspection mode, not the bench contract's line)."""
+    import torch
+
+    from nonlinear_rnn_iteration_b200 import workloads
+
+    w = workloads.HEAD_WORKLOADS[args.workload]
+    if args.B or args.T:
+        w = workloads.HeadWorkload("%s@B%dT%d" % (w.name, args.B or w.B, args.T or w.T), args.B or w.B,
+                                   args.T or w.T, w.D, w.n_heads, w.K, w.px_dtype, w.seed)
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    ms, status = time_head(w, device, args.steps, args.warmup)
+    line = {"workload": w.name, "metric": METRIC, "unit": UNIT, "data": "synthetic", **head_line(w, ms, status)}
+    print(json.dumps(line), flush=True)
 
 
 def run_reference(args):

@@ -1,0 +1,42 @@
+"""bench.py on the CPU: its pieces exist and its host-side arithmetic and
+argument handling behave (the timed paths themselves need a GPU)."""
+import json
+import os
+import subprocess
+import sys
+
+import bench
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def test_entry_points_exist():
+    for name in ("Problem", "ClockSampler", "time_device", "time_e2e", "cpu_baseline", "extra_workloads",
+                 "head_workloads", "time_head", "head_line", "run_native", "run_head", "run_reference", "main",
+                 "measured_peaks", "recorded_traffic", "kernel_source_hash"):
+        assert callable(getattr(bench, name, None)), name
+
+
+def test_aggregate_throughput_and_peaks():
+    assert bench.aggregate_throughput(1000, 2, 4, 8.0) == 1000 * 2 * 4 / 8e-3
+    p = bench.measured_peaks()
+    assert p["hbm_gbs"] > 1000 and p["bf16_tflops"] > 100
+    assert len(bench.kernel_source_hash()) == 16
+
+
+def test_head_line_arithmetic():
+    from nonlinear_rnn_iteration_b200 import workloads
+
+    w = workloads.HEAD_WORKLOADS["headgru_8x4096x512_h8_k3"]
+    line = bench.head_line(w, 10.0, "PARARNN_OK")
+    useful = 2.0 * 64 ** 3 * 8 * 4096 * 8 * 3 / 1e-2 / 1e12
+    assert abs(line["roofline"]["achieved_useful"] - round(useful, 2)) < 1e-9
+    assert line["elem_per_s"] == w.elements / 1e-2
+    json.dumps(line)
+
+
+def test_help_lists_every_workload():
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--help"], capture_output=True, text=True,
+                         cwd=ROOT, check=True).stdout
+    for name in ("linear_8x16384x1024", "gru_1x131072x4096_k2_bf16", "headgru_8x4096x512_h8_k3"):
+        assert name in out
