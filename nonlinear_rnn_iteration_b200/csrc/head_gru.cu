@@ -159,17 +159,20 @@ __device__ __forceinline__ void block_max_resid(float v, float* resid) {
 // kept as a TF32 head and a TF32 remainder, x = x_hi + x_lo, and the product
 // accumulates a_lo b_hi + a_hi b_lo + a_hi b_hi in float32 (the lo * lo term
 // is below float32 rounding): float32 accuracy from three TF32 products.
-// Every element is split once, by the thread that produces it, and stored as
-// a {hi, lo} pair; rows of pairs are padded to d + 4 pairs, which puts each
-// half-warp's 64-bit fragment loads on distinct banks.
+// The running product is split once, by the thread that produces it, and
+// stored as {hi, lo} pairs (each of its elements is read by several warps);
+// the Jacobian is stored as float and split when its fragment is loaded.
+// Rows are padded (d + 4 pairs, d + 8 floats), which puts each warp's (or
+// half-warp's, for 64-bit pairs) fragment loads on distinct banks.
 constexpr int kPad = 4;
+constexpr int kPadA = 8;
 
 template <int DH>
 struct SmemA {
-    uint2 AT[DH][DH + kPad];     // A_t transposed (AT[m][i] = A_t[i][m]) as {hi, lo} TF32 pairs
-    uint2 Pm[2][DH][DH + kPad];  // running product, row-major, {hi, lo} pairs
-    float sv[2][DH];             // h^(k)_{t-1}, permuted (vpos)
-    float dv[2][DH];             // delta_{t-1}, permuted
+    float AT[2][DH][DH + kPadA];  // A_t transposed (AT[m][i] = A_t[i][m]), two steps in turn
+    uint2 Pm[2][DH][DH + kPad];   // running product, row-major, {hi, lo} TF32 pairs
+    float sv[2][DH];              // h^(k) rows, permuted (vpos), two steps in turn
+    float dv[2][DH];              // delta rows, permuted, two steps in turn
 };
 
 __device__ __forceinline__ uint2 split_tf32(float x) {
@@ -195,7 +198,7 @@ __device__ __forceinline__ void mma_tf32(float (&c)[4], const uint32_t (&a)[4], 
 // and g+8, columns t and t+4; B rows t and t+4, column g; C rows g and g+8,
 // columns 2t and 2t+1.
 template <int DH>
-__device__ __forceinline__ void matmul_tf32x3(const uint2 (*AT)[DH + kPad], const uint2 (*Pin)[DH + kPad],
+__device__ __forceinline__ void matmul_tf32x3(const float (*AT)[DH + kPadA], const uint2 (*Pin)[DH + kPad],
                                               uint2 (*Pout)[DH + kPad]) {
     constexpr int MT = DH / 16, NT = DH / 8;             // 16-row and 8-column tiles
     constexpr int WPM = (kThreads / 32) / MT;            // warps per row of tiles
@@ -212,7 +215,8 @@ __device__ __forceinline__ void matmul_tf32x3(const uint2 (*AT)[DH + kPad], cons
 #pragma unroll 2
     for (int ks = 0; ks < DH / 8; ++ks) {
         const int k0 = ks * 8 + t;
-        const uint2 a0 = AT[k0][r0], a1 = AT[k0][r0 + 8], a2 = AT[k0 + 4][r0], a3 = AT[k0 + 4][r0 + 8];
+        const uint2 a0 = split_tf32(AT[k0][r0]), a1 = split_tf32(AT[k0][r0 + 8]);
+        const uint2 a2 = split_tf32(AT[k0 + 4][r0]), a3 = split_tf32(AT[k0 + 4][r0 + 8]);
         const uint32_t ahi[4] = {a0.x, a1.x, a2.x, a3.x}, alo[4] = {a0.y, a1.y, a2.y, a3.y};
 #pragma unroll
         for (int n = 0; n < NPW; ++n) {
@@ -233,11 +237,14 @@ __device__ __forceinline__ void matmul_tf32x3(const uint2 (*AT)[DH + kPad], cons
     }
 }
 
-// Two block barriers per step: step t writes AT and the step-parity halves of
-// sv / dv (reading the other halves); after the first barrier the product
-// reads AT and Pm[cur] and writes Pm[cur ^ 1]; the second barrier frees AT
-// for the next step.  A buffer is rewritten only after a barrier that every
-// reader of its previous contents has passed.
+// One block barrier per step, and the product of step t shares its barrier
+// interval with the row work of step t+1 (A_{t+1} depends on the known
+// iterate only, not on the product), so the tensor and FMA/ALU pipes work
+// side by side.  Step t's row work reads sv/dv[p] (h^(k)_{t-1}, delta_{t-1})
+// and writes AT[p] = A_t and sv/dv[p ^ 1], p = (t - t0) & 1; the product of
+// step t reads AT[p] and Pm[cur] and writes Pm[cur ^ 1].  Every buffer is
+// rewritten only after a barrier that all readers of its previous contents
+// have passed.
 template <int DH, typename PxT, bool kResidOnly>
 __global__ void __launch_bounds__(kThreads, 2) head_chunk_kernel(const Params pr) {
     using Gm = Geo<DH>;
@@ -263,19 +270,15 @@ __global__ void __launch_bounds__(kThreads, 2) head_chunk_kernel(const Params pr
     if constexpr (!kResidOnly)
         for (int idx = tid; idx < DH * DH; idx += kThreads)
             sm.Pm[0][idx / DH][idx % DH] = make_uint2(idx / DH == idx % DH ? __float_as_uint(1.0f) : 0u, 0u);
-    StepIn nxt = load_step<DH, PxT>(pr, b, h, i, t0);
-    __syncthreads();
-
-    int par = 0, cur = 0;
     float rmax = 0.0f;
-    for (int64_t t = t0; t < t1; ++t) {
-        const StepIn in = nxt;
-        if (t + 1 < t1) nxt = load_step<DH, PxT>(pr, b, h, i, t + 1);
-        // (U_g s_prev)_i
+
+    // the row work of one step: row i of A_t into AT[p], and the next rows
+    // of the iterate and of delta (delta_t = A_t delta_{t-1} - F_t)
+    auto row_step = [&](const StepIn& in, int p) {
         float uz = 0.0f, ur = 0.0f, uc = 0.0f;
 #pragma unroll
         for (int s = 0; s < SEG; ++s) {
-            const float x = sm.sv[par][qt * SEG + s];
+            const float x = sm.sv[p][qt * SEG + s];
             uz = __fmaf_rn(U.z[s], x, uz);
             ur = __fmaf_rn(U.r[s], x, ur);
             uc = __fmaf_rn(U.c[s], x, uc);
@@ -283,11 +286,10 @@ __global__ void __launch_bounds__(kThreads, 2) head_chunk_kernel(const Params pr
         uz = row_sum<DH>(uz);
         ur = row_sum<DH>(ur);
         uc = row_sum<DH>(uc);
-        const float sp = sm.sv[par][Gm::vpos(i)];
+        const float sp = sm.sv[p][Gm::vpos(i)];
         const RowLin L = row_linearise(in, sp, uz, ur, uc);
         if (qt == 0) rmax = nanmax_f(rmax, fabsf(L.F));
         if constexpr (!kResidOnly) {
-            // row i of A_t into AT, and delta_t = A_t delta_{t-1} - F_t
             float dp = 0.0f;
 #pragma unroll
             for (int s = 0; s < SEG; ++s) {
@@ -295,20 +297,34 @@ __global__ void __launch_bounds__(kThreads, 2) head_chunk_kernel(const Params pr
                 float a = __fmaf_rn(L.al, U.z[s], (m == i) ? L.dz : 0.0f);
                 a = __fmaf_rn(L.be, U.r[s], a);
                 a = __fmaf_rn(L.ga, U.c[s], a);
-                sm.AT[m][i] = split_tf32(a);
-                dp = __fmaf_rn(a, sm.dv[par][qt * SEG + s], dp);
+                sm.AT[p][m][i] = a;
+                dp = __fmaf_rn(a, sm.dv[p][qt * SEG + s], dp);
             }
             dp = row_sum<DH>(dp);
-            if (qt == 0) sm.dv[par ^ 1][Gm::vpos(i)] = dp - L.F;
+            if (qt == 0) sm.dv[p ^ 1][Gm::vpos(i)] = dp - L.F;
         }
-        if (qt == 0) sm.sv[par ^ 1][Gm::vpos(i)] = in.s;
+        if (qt == 0) sm.sv[p ^ 1][Gm::vpos(i)] = in.s;
+    };
+
+    StepIn nxt = load_step<DH, PxT>(pr, b, h, i, t0);
+    __syncthreads();
+    {
+        const StepIn in = nxt;
+        if (t0 + 1 < t1) nxt = load_step<DH, PxT>(pr, b, h, i, t0 + 1);
+        row_step(in, 0);
+    }
+    __syncthreads();
+    int p = 0, cur = 0;
+    for (int64_t t = t0; t < t1; ++t) {
+        if constexpr (!kResidOnly) matmul_tf32x3<DH>(sm.AT[p], sm.Pm[cur], sm.Pm[cur ^ 1]);
+        if (t + 1 < t1) {
+            const StepIn in = nxt;
+            if (t + 2 < t1) nxt = load_step<DH, PxT>(pr, b, h, i, t + 2);
+            row_step(in, p ^ 1);
+        }
         __syncthreads();
-        if constexpr (!kResidOnly) {
-            matmul_tf32x3<DH>(sm.AT, sm.Pm[cur], sm.Pm[cur ^ 1]);
-            cur ^= 1;
-            __syncthreads();
-        }
-        par ^= 1;
+        cur ^= 1;
+        p ^= 1;
     }
     if (pr.resid) block_max_resid(rmax, pr.resid + pr.k);
     if constexpr (!kResidOnly) {
@@ -317,7 +333,8 @@ __global__ void __launch_bounds__(kThreads, 2) head_chunk_kernel(const Params pr
             const uint2 v = sm.Pm[cur][idx / DH][idx % DH];
             Pout[idx] = __uint_as_float(v.x) + __uint_as_float(v.y);
         }
-        if (qt == 0) pr.q[task * DH + i] = sm.dv[par][Gm::vpos(i)];
+        // delta at the chunk's last step: written to dv[(t1 - t0) & 1]
+        if (qt == 0) pr.q[task * DH + i] = sm.dv[p][Gm::vpos(i)];
     }
 }
 
