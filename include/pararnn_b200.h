@@ -219,7 +219,8 @@ pararnn_status pararnn_newton_forward_noalloc(pararnn_cell cell, int64_t B, int6
  * Returns the workspace size for these sizes, or 0 when they are invalid
  * (d not in {16, 32, 64}, D not a multiple of n_heads, K outside 1..64, B*T
  * at or above 2^31).  It holds a second iterate buffer (K >= 2) and each
- * chunk's d x d Jacobian product: about B*T*D*4 + B*T*n_heads*(d+2)*d*4/32
+ * chunk's d x d Jacobian product (chunks of 64 steps): about
+ * B*T*D*4 + B*T*n_heads*(d+2)*d*4/64
  * bytes. */
 size_t pararnn_head_gru_workspace_bytes(int64_t B, int64_t T, int64_t D, int n_heads, int K);
 

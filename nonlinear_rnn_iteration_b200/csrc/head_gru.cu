@@ -36,7 +36,7 @@ bool pointer_on_device(const void* p);      // pararnn_abi.cu
 namespace hg {
 
 constexpr int kThreads = 256;
-constexpr int kChunk = 32;  // steps per chunk
+constexpr int kChunk = 64;  // steps per chunk
 constexpr int kMaxK = 64;
 
 struct Params {

@@ -19,8 +19,8 @@ Functions and what they follow:
   weights and the initial state (Method section, backward pass).
 * :func:`cell_step`, :func:`cell_jacobian`, :func:`cell_param_grads` -- one
   cell application and its closed-form derivatives, exposed for the pins.
-* :func:`head_gru_unroll`, :func:`head_gru_newton`, :func:`head_gru_step`,
-  :func:`head_gru_jacobian` -- the same for the head-wise GRU
+* :func:`head_gru_unroll`, :func:`head_gru_newton`, :func:`head_gru_adjoint`,
+  :func:`head_gru_step`, :func:`head_gru_jacobian` -- the same for the head-wise GRU
   (``ParaGRU(mix='head', n_heads)`` on the pararnn-torch page: block-diagonal
   recurrent weights, one dense d x d block per head, d = D / n_heads).
 
@@ -113,6 +113,8 @@ def _bind(so_path):
     lib.oracle_head_gru_unroll.restype = ci
     lib.oracle_head_gru_newton.argtypes = [i64, i64, i64, ci, P, P, P, ci, P, P, ci]
     lib.oracle_head_gru_newton.restype = ci
+    lib.oracle_head_gru_adjoint.argtypes = [i64, i64, i64, ci, P, P, P, P, P, P, P, P, ci]
+    lib.oracle_head_gru_adjoint.restype = ci
     return lib
 
 
@@ -268,3 +270,18 @@ def head_gru_newton(px, U, h0=None, K=1, nthreads=None):
     if rc:
         raise ValueError("oracle_head_gru_newton: bad arguments")
     return H, resid
+
+
+def head_gru_adjoint(px, U, H, dLdH, h0=None, nthreads=None):
+    """Adjoint at trajectory H: returns (dL/dpx (B,T,3,D), dL/dU (3,n_heads,d,d), dL/dh0 (B,D))."""
+    lib = _load()
+    px, U, h0, H, g = _f64(px), _f64(U), _f64(h0), _f64(H), _f64(dLdH)
+    B, T, D, nh = _head_shape(px, U)
+    dpx = np.zeros((B, T, 3, D))
+    dU = np.zeros(U.shape)
+    dh0 = np.zeros((B, D))
+    rc = lib.oracle_head_gru_adjoint(B, T, D, nh, _ptr(px), _ptr(U), _ptr(h0), _ptr(H), _ptr(g), _ptr(dpx), _ptr(dU),
+                                     _ptr(dh0), _threads(nthreads))
+    if rc:
+        raise ValueError("oracle_head_gru_adjoint: bad arguments")
+    return dpx, dU, dh0

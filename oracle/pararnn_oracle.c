@@ -645,3 +645,147 @@ int oracle_head_gru_newton(int64_t B, int64_t T, int64_t D, int nh, const double
         for (int k = 0; k <= K; ++k) resid[k] = j.resid[k];
     return rc;
 }
+
+/* ---- head-wise GRU: the adjoint ------------------------------------------
+ * At a trajectory H (the forward's output), g_t = dL/dH_t, per head:
+ *     lambda_t = g_t + A_{t+1}^T lambda_{t+1},  lambda_{T-1} = g_{T-1},
+ * with A_{t+1} the Jacobian at (h_t, x_{t+1}); then, with the gate factors
+ * at (h_{t-1}, x_t) (h_{-1} = h0):
+ *     dL/dp_z = lambda * alpha,  dL/dp_r = lambda * beta,
+ *     dL/dp_c = lambda * z (1 - c^2),
+ *     dL/dU_z[i][j] = sum_{b,t} lambda_i alpha_i h_{t-1,j}   (likewise U_r with
+ *     beta, U_c with gamma), summed over b then t in natural order,
+ *     dL/dh0 = A_0^T lambda_0.
+ * Layouts: dL_dH (B,T,D), dL_dpx (B,T,3,D), dL_dU (3, n_heads, d, d),
+ * dL_dh0 (B,D). */
+
+typedef struct {
+    int64_t B, T, D;
+    int nh, d, nthreads, tid;
+    const double *px, *U, *h0, *H, *g;
+    double *dpx, *dU_b, *dh0;  /* dU_b: per batch row partials [B][3][nh][d][d] */
+} ajob_t;
+
+/* the gate factors of head h at (s, x_t): alpha, beta, z (1 - c^2), gamma */
+static void head_factors(int d, const double* p, const double* U, const double* s, double* al, double* be, double* zc,
+                         double* ga) {
+    const double* Uz = U;
+    const double* Ur = U + (size_t)d * d;
+    const double* Uc = U + 2 * (size_t)d * d;
+    for (int i = 0; i < d; ++i) {
+        double az = p[i], ar = p[d + i], n = 0.0;
+        for (int j = 0; j < d; ++j) {
+            az += Uz[(size_t)i * d + j] * s[j];
+            ar += Ur[(size_t)i * d + j] * s[j];
+            n += Uc[(size_t)i * d + j] * s[j];
+        }
+        double z = sig(az), r = sig(ar), c = tanh(p[2 * d + i] + r * n);
+        al[i] = (c - s[i]) * z * (1.0 - z);
+        be[i] = z * (1.0 - c * c) * n * r * (1.0 - r);
+        zc[i] = z * (1.0 - c * c);
+        ga[i] = z * (1.0 - c * c) * r;
+    }
+}
+
+static void head_adjoint_seq(ajob_t* j, int64_t b, int h) {
+    const int d = j->d;
+    const int64_t T = j->T;
+    size_t dd = (size_t)d * d;
+    hjob_t hj;  /* only for the gather helpers */
+    memset(&hj, 0, sizeof hj);
+    hj.B = j->B; hj.T = j->T; hj.D = j->D; hj.nh = j->nh; hj.d = d; hj.px = j->px; hj.U = j->U; hj.h0 = j->h0;
+    double* Ubuf = (double*)malloc(3 * dd * sizeof(double));
+    double* lam = (double*)malloc((size_t)d * sizeof(double));
+    double* nl = (double*)malloc((size_t)d * sizeof(double));
+    double* A = (double*)malloc(dd * sizeof(double));
+    double* p = (double*)malloc(3 * (size_t)d * sizeof(double));
+    double* prev = (double*)malloc((size_t)d * sizeof(double));
+    double* cur = (double*)malloc((size_t)d * sizeof(double));
+    double* al = (double*)malloc((size_t)d * sizeof(double));
+    double* be = (double*)malloc((size_t)d * sizeof(double));
+    double* zc = (double*)malloc((size_t)d * sizeof(double));
+    double* ga = (double*)malloc((size_t)d * sizeof(double));
+    const double* U = head_U(&hj, h, Ubuf);
+    double* dU = j->dU_b + (size_t)b * 3 * j->nh * dd;
+    for (int64_t t = T - 1; t >= 0; --t) {
+        /* lambda_t = g_t + A_{t+1}^T lambda_{t+1} */
+        for (int i = 0; i < d; ++i) lam[i] = j->g[(b * T + t) * j->D + (int64_t)h * d + i] + (t + 1 < T ? nl[i] : 0.0);
+        /* state before row t */
+        if (t == 0) head_h0(&hj, b, h, prev);
+        else
+            for (int i = 0; i < d; ++i) prev[i] = j->H[(b * T + t - 1) * j->D + (int64_t)h * d + i];
+        head_p(&hj, b, t, h, p);
+        head_factors(d, p, U, prev, al, be, zc, ga);
+        for (int i = 0; i < d; ++i) {
+            const int64_t o = ((b * T + t) * 3) * j->D + (int64_t)h * d + i;
+            j->dpx[o] = lam[i] * al[i];
+            j->dpx[o + j->D] = lam[i] * be[i];
+            j->dpx[o + 2 * j->D] = lam[i] * zc[i];
+            for (int m = 0; m < d; ++m) {
+                dU[((size_t)0 * j->nh + h) * dd + (size_t)i * d + m] += lam[i] * al[i] * prev[m];
+                dU[((size_t)1 * j->nh + h) * dd + (size_t)i * d + m] += lam[i] * be[i] * prev[m];
+                dU[((size_t)2 * j->nh + h) * dd + (size_t)i * d + m] += lam[i] * ga[i] * prev[m];
+            }
+        }
+        /* A_t^T lambda_t: the next (earlier) row's propagated term, and dL/dh0 at t = 0 */
+        oracle_head_gru_jacobian(d, p, U, prev, A);
+        for (int m = 0; m < d; ++m) {
+            double acc = 0.0;
+            for (int i = 0; i < d; ++i) acc += A[(size_t)i * d + m] * lam[i];
+            cur[m] = acc;
+        }
+        memcpy(nl, cur, d * sizeof(double));
+        if (t == 0 && j->dh0)
+            for (int m = 0; m < d; ++m) j->dh0[b * j->D + (int64_t)h * d + m] = cur[m];
+    }
+    free(Ubuf); free(lam); free(nl); free(A); free(p); free(prev); free(cur); free(al); free(be); free(zc); free(ga);
+}
+
+static void* head_adjoint_worker(void* arg) {
+    ajob_t* j = (ajob_t*)arg;
+    int64_t nseq = j->B * j->nh;
+    int64_t per = (nseq + j->nthreads - 1) / j->nthreads;
+    int64_t lo = (int64_t)j->tid * per, hi = lo + per < nseq ? lo + per : nseq;
+    for (int64_t q = lo; q < hi; ++q) head_adjoint_seq(j, q / j->nh, (int)(q % j->nh));
+    return NULL;
+}
+
+/* The head-wise GRU adjoint at trajectory H.  dL_dU (may be NULL) is summed
+ * over b in natural order (each b's sum over t is in reverse time order, as
+ * the recursion runs); dL_dh0 may be NULL. */
+int oracle_head_gru_adjoint(int64_t B, int64_t T, int64_t D, int nh, const double* px, const double* U,
+                            const double* h0, const double* H, const double* dLdH, double* dLdpx, double* dLdU,
+                            double* dLdh0, int nthreads) {
+    if (head_check(B, T, D, nh, px, U) || !H || !dLdH || !dLdpx) return -1;
+    const int d = (int)(D / nh);
+    const size_t per_b = (size_t)3 * nh * d * d;
+    double* part = (double*)calloc(B * per_b > 0 ? B * per_b : 1, sizeof(double));
+    if (!part) return -2;
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > 256) nthreads = 256;
+    ajob_t proto;
+    memset(&proto, 0, sizeof proto);
+    proto.B = B; proto.T = T; proto.D = D; proto.nh = nh; proto.d = d; proto.px = px; proto.U = U; proto.h0 = h0;
+    proto.H = H; proto.g = dLdH; proto.dpx = dLdpx; proto.dU_b = part; proto.dh0 = dLdh0;
+    ajob_t* jobs = (ajob_t*)calloc((size_t)nthreads, sizeof(ajob_t));
+    pthread_t* th = (pthread_t*)calloc((size_t)nthreads, sizeof(pthread_t));
+    if (!jobs || !th) { free(jobs); free(th); free(part); return -2; }
+    for (int i = 0; i < nthreads; ++i) {
+        jobs[i] = proto;
+        jobs[i].nthreads = nthreads;
+        jobs[i].tid = i;
+    }
+    for (int i = 1; i < nthreads; ++i) pthread_create(&th[i], NULL, head_adjoint_worker, &jobs[i]);
+    head_adjoint_worker(&jobs[0]);
+    for (int i = 1; i < nthreads; ++i) pthread_join(th[i], NULL);
+    if (dLdU)
+        for (size_t k = 0; k < per_b; ++k) {
+            double acc = 0.0;
+            for (int64_t b = 0; b < B; ++b) acc += part[(size_t)b * per_b + k];
+            dLdU[k] = acc;
+        }
+    free(jobs);
+    free(th);
+    free(part);
+    return 0;
+}

@@ -435,7 +435,92 @@ def pin_head_prefix_exact_and_diagonal():
     _close(rh, rd, 1e-13, "head vs diagonal residual history")
 
 
+def _torch_head_unroll_t(px_t, U_t, h0_t, d):
+    """The head-wise unroll on torch tensors (differentiable in px, U, h0)."""
+    B, T, _, D = px_t.shape
+    nh = U_t.shape[1]
+    outs = []
+    for h in range(nh):
+        sl = slice(h * d, (h + 1) * d)
+        I, Z = torch.eye(d, dtype=torch.float64), torch.zeros((d, d), dtype=torch.float64)
+        w_ih = torch.cat([torch.cat([Z, I, Z], 1), torch.cat([-I, Z, Z], 1), torch.cat([Z, Z, I], 1)], 0)
+        w_hh = torch.cat([U_t[1, h], -U_t[0, h], U_t[2, h]], 0)
+        zb = torch.zeros(3 * d, dtype=torch.float64)
+        s = h0_t[:, sl]
+        seq = []
+        for t in range(T):
+            s = torch._VF.gru_cell(px_t[:, t, :, sl].reshape(B, 3 * d), s, w_ih, w_hh, zb, zb)
+            seq.append(s)
+        outs.append(torch.stack(seq, 1))
+    return torch.cat(outs, 2)
+
+
+def pin_head_adjoint_bptt():
+    # at the unroll the adjoint is back-propagation through time
+    B, T, nh, d = 2, 7, 2, 3
+    px, U, hz = _head_inputs(B, T, nh, d, seed=36, h0=True)
+    g = _rng(37).standard_normal((B, T, nh * d))
+    px_t, U_t, h0_t = (torch.tensor(a, requires_grad=True) for a in (px, U, hz))
+    Ht = _torch_head_unroll_t(px_t, U_t, h0_t, d)
+    (Ht * torch.tensor(g)).sum().backward()
+    dpx, dU, dh0 = oracle.head_gru_adjoint(px, U, Ht.detach().numpy(), g, hz)
+    _close(dpx, px_t.grad.numpy(), 1e-12, "head adjoint dL/dpx vs BPTT")
+    _close(dU, U_t.grad.numpy(), 1e-12, "head adjoint dL/dU vs BPTT")
+    _close(dh0, h0_t.grad.numpy(), 1e-12, "head adjoint dL/dh0 vs BPTT")
+
+
+def pin_head_adjoint_dense():
+    # at an unconverged iterate: the implicit gradient of F(H) = 0, solved
+    # densely -- lambda = J^T \ g, dL/dtheta = -(dF/dtheta)^T lambda
+    B, T, nh, d = 1, 5, 2, 2
+    D = nh * d
+    px, U, hz = _head_inputs(B, T, nh, d, seed=38, h0=True)
+    H, _ = oracle.head_gru_newton(px, U, hz, K=1)
+    g = _rng(39).standard_normal((B, T, D))
+
+    def F(Hf, pxf, Uf, h0f):
+        Hm = Hf.reshape(B, T, D)
+        prev = torch.cat([h0f.reshape(B, 1, D), Hm[:, :-1]], 1)
+        rows = []
+        for t in range(T):
+            f_t = _torch_head_unroll_t(pxf[:, t:t + 1], Uf, prev[:, t], d)[:, 0]
+            rows.append(Hm[:, t] - f_t)
+        return torch.stack(rows, 1).reshape(-1)
+
+    args = tuple(torch.tensor(a) for a in (H, px, U, hz))
+    J = torch.autograd.functional.jacobian(F, args)
+    lam = torch.linalg.solve(J[0].reshape(B * T * D, B * T * D).T, torch.tensor(g).reshape(-1))
+    grads = [-(Jk.reshape(B * T * D, -1).T @ lam).reshape(a.shape) for Jk, a in zip(J[1:], args[1:])]
+    dpx, dU, dh0 = oracle.head_gru_adjoint(px, U, H, g, hz)
+    _close(dpx, grads[0].numpy(), 1e-11, "head adjoint dL/dpx vs implicit gradient")
+    _close(dU, grads[1].numpy(), 1e-11, "head adjoint dL/dU vs implicit gradient")
+    _close(dh0, grads[2].numpy(), 1e-11, "head adjoint dL/dh0 vs implicit gradient")
+
+
+def pin_head_adjoint_diagonal():
+    # diagonal blocks: the diagonal GRU's adjoint (its own code path); dL/dU's
+    # diagonal is the diagonal cell's dL/da
+    rng = _rng(40)
+    B, T, nh, d = 2, 15, 2, 3
+    D = nh * d
+    px = rng.standard_normal((B, T, 3, D))
+    a = rng.uniform(-0.5, 0.5, (3, D))
+    U = np.zeros((3, nh, d, d))
+    for gi in range(3):
+        for h in range(nh):
+            U[gi, h] = np.diag(a[gi, h * d:(h + 1) * d])
+    H, _ = oracle.newton(oracle.DIAG_GRU, px, a, K=2)
+    g = rng.standard_normal((B, T, 1, D))
+    dpx_d, da_d, dh0_d = oracle.adjoint(oracle.DIAG_GRU, px, a, None, H, g)
+    dpx, dU, dh0 = oracle.head_gru_adjoint(px, U, H[:, :, 0, :], g[:, :, 0, :])
+    _close(dpx, dpx_d, 1e-13, "head adjoint vs diagonal dL/dpx")
+    diag = np.stack([np.concatenate([np.diag(dU[gi, h]) for h in range(nh)]) for gi in range(3)])
+    _close(diag, da_d, 1e-13, "head adjoint dL/dU diagonal vs diagonal dL/da")
+    _close(dh0, dh0_d[:, 0, :], 1e-13, "head adjoint vs diagonal dL/dh0")
+
+
 ALL_PINS = [pin_cell_step, pin_jacobian, pin_param_grads, pin_unroll, pin_newton_dense, pin_affine_one_step,
             pin_prefix_exact, pin_lstm_zero_weights, pin_adjoint_dense, pin_adjoint_bptt, pin_adjoint_fd,
             pin_residual_monotone, pin_head_step_and_jacobian, pin_head_unroll, pin_head_newton_dense,
-            pin_head_prefix_exact_and_diagonal]
+            pin_head_prefix_exact_and_diagonal, pin_head_adjoint_bptt, pin_head_adjoint_dense,
+            pin_head_adjoint_diagonal]

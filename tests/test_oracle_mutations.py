@@ -56,6 +56,12 @@ MUTATIONS = {
         "                memcpy(prev, s + t * d, d * sizeof(double));"),
     "head_no_warm_start": ("oracle_head_gru_step(d, p, U, tmp, s + t * d);",
                            "for (int i = 0; i < d; ++i) s[t * d + i] = 0.0;"),
+    "head_adjoint_transposed": ("for (int i = 0; i < d; ++i) acc += A[(size_t)i * d + m] * lam[i];",
+                                "for (int i = 0; i < d; ++i) acc += A[(size_t)m * d + i] * lam[i];"),
+    "head_adjoint_dUc_factor": ("+= lam[i] * ga[i] * prev[m];", "+= lam[i] * be[i] * prev[m];"),
+    "head_adjoint_state_index": ("prev[i] = j->H[(b * T + t - 1) * j->D + (int64_t)h * d + i];",
+                                 "prev[i] = j->H[(b * T + t) * j->D + (int64_t)h * d + i];"),
+    "head_adjoint_dpc_factor": ("j->dpx[o + 2 * j->D] = lam[i] * zc[i];", "j->dpx[o + 2 * j->D] = lam[i] * ga[i];"),
 }
 
 
