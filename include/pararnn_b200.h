@@ -238,6 +238,32 @@ pararnn_status pararnn_head_gru_forward(int64_t B, int64_t T, int64_t D, int n_h
                                         const void* preacts, const float* U, const float* h0, int K, float* H_out,
                                         void* workspace, size_t ws_bytes, float* resid_hist, void* stream);
 
+/* The adjoint of the head-wise GRU at a trajectory H (normally H_out of
+ * pararnn_head_gru_forward), the head-wise counterpart of
+ * pararnn_newton_backward: with g_t = dL/dH_t,
+ *     lambda_t = g_t + A_{t+1}^T lambda_{t+1},   lambda_{T-1} = g_{T-1},
+ * A_{t+1} the head's Jacobian block at (h_t, x_{t+1}); then
+ *     dL/dp_z = lambda * alpha, dL/dp_r = lambda * beta,
+ *     dL/dp_c = lambda * z (1 - c^2)                     (at (h_{t-1}, x_t)),
+ *     dL/dU_g[i][j] = sum over b, t of lambda_i f_{g,i} h_{t-1,j}
+ *                     (f = alpha, beta, gamma for g = z, r, c),
+ *     dL/dh0 = A_0^T lambda_0,
+ * alpha, beta, gamma as in the Jacobian above.  Layouts: H, dL_dH (B, T, D);
+ * dL_dpx (B, T, 3, D); dL_dU (3, n_heads, d, d) or NULL; dL_dh0 (B, D) or
+ * NULL; all float32 device memory owned by the caller.  dL_dU is summed in a
+ * fixed order (no floating-point atomics): repeated calls give identical
+ * bits.  Returns the workspace size, or 0 for invalid sizes (as for the
+ * forward): about B*T*D*4 + B*T*n_heads*(d+2)*d*4/64 bytes plus 12 n_heads
+ * d^2 * min(64, B*T/256) * 4 bytes of split partials. */
+size_t pararnn_head_gru_backward_workspace_bytes(int64_t B, int64_t T, int64_t D, int n_heads);
+
+/* Errors as for pararnn_head_gru_forward; a non-finite value in dL_dpx is
+ * recorded in the workspace for pararnn_status_sync(). */
+pararnn_status pararnn_head_gru_backward(int64_t B, int64_t T, int64_t D, int n_heads, pararnn_dtype px_dtype,
+                                         const void* preacts, const float* U, const float* h0, const float* H,
+                                         const float* dL_dH, float* dL_dpx, float* dL_dU, float* dL_dh0,
+                                         void* workspace, size_t ws_bytes, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

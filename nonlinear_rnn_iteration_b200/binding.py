@@ -39,6 +39,8 @@ SIGNATURES = {
     "pararnn_newton_forward_noalloc": (_I, [_I, _I64, _I64, _I64, _I, _P, _P, _P, _I, _P, _P, _I, _P]),
     "pararnn_head_gru_workspace_bytes": (_SZ, [_I64, _I64, _I64, _I, _I]),
     "pararnn_head_gru_forward": (_I, [_I64, _I64, _I64, _I, _I, _P, _P, _P, _I, _P, _P, _SZ, _P, _P]),
+    "pararnn_head_gru_backward_workspace_bytes": (_SZ, [_I64, _I64, _I64, _I]),
+    "pararnn_head_gru_backward": (_I, [_I64, _I64, _I64, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
 }
 
 _lib = None
@@ -147,6 +149,17 @@ def pararnn_head_gru_forward(B, T, D, n_heads, px_dtype, preacts, U, h0, K, H_ou
                                            _stream(stream))
 
 
+def pararnn_head_gru_backward_workspace_bytes(B, T, D, n_heads):
+    return load().pararnn_head_gru_backward_workspace_bytes(B, T, D, n_heads)
+
+
+def pararnn_head_gru_backward(B, T, D, n_heads, px_dtype, preacts, U, h0, H, dL_dH, dL_dpx, dL_dU, dL_dh0, workspace,
+                              ws_bytes, stream):
+    return load().pararnn_head_gru_backward(B, T, D, n_heads, px_dtype, _ptr(preacts), _ptr(U), _ptr(h0), _ptr(H),
+                                            _ptr(dL_dH), _ptr(dL_dpx), _ptr(dL_dU), _ptr(dL_dh0), _ptr(workspace),
+                                            ws_bytes, _stream(stream))
+
+
 # ---- tensor-level helpers (allocation through torch, compute in the library) ----
 
 def _check(status, where):
@@ -246,3 +259,26 @@ def head_gru_forward(px, U, h0=None, K=1, out=None, workspace=None, resid_hist=N
     if sync_status:
         _check(pararnn_status_sync(workspace, st), "pararnn_head_gru_forward (device status)")
     return out
+
+
+def head_gru_backward(px, U, H, dL_dH, h0=None, want_dU=True, want_dh0=False, workspace=None, stream=None,
+                      sync_status=True):
+    """Head-wise GRU adjoint: returns (dL/dpx (B,T,3,D), dL/dU (3,n_heads,d,d) or None, dL/dh0 (B,D) or None)."""
+    import torch
+
+    B, T, _, D = px.shape
+    nh = U.shape[1]
+    dpx = torch.empty((B, T, 3, D), dtype=torch.float32, device=px.device)
+    dU = torch.empty(tuple(U.shape), dtype=torch.float32, device=px.device) if want_dU else None
+    dh0 = torch.empty((B, D), dtype=torch.float32, device=px.device) if want_dh0 else None
+    if workspace is None:
+        n = pararnn_head_gru_backward_workspace_bytes(B, T, D, nh)
+        if n == 0:
+            raise PararnnError(EINVAL, "pararnn_head_gru_backward_workspace_bytes", "invalid sizes")
+        workspace = torch.empty(n, dtype=torch.uint8, device=px.device)
+    st = stream if stream is not None else torch.cuda.current_stream(px.device)
+    _check(pararnn_head_gru_backward(B, T, D, nh, _dtype_code(px), px, U, h0, H, dL_dH, dpx, dU, dh0, workspace,
+                                     workspace.numel(), st), "pararnn_head_gru_backward")
+    if sync_status:
+        _check(pararnn_status_sync(workspace, st), "pararnn_head_gru_backward (device status)")
+    return dpx, dU, dh0

@@ -25,6 +25,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <cstring>
 
 #include "common.cuh"
 #include "pararnn_b200.h"
@@ -50,6 +51,11 @@ struct Params {
     float* carry;       // [nSeq][nChunks][d]: delta just before each chunk
     float* resid;       // K+1 floats or null
     unsigned* status;   // workspace header word 0
+    // backward only
+    const float* G;     // dL/dH (B,T,D)
+    float* dpx;         // dL/dpx (B,T,3,D)
+    float* ec;          // lambda * gamma (B,T,D): the factor of dL/dU_c
+    float* dh0;         // dL/dh0 (B,D) or null
     int64_t B, T, D;
     int nh, k, nChunks;
 };
@@ -191,13 +197,14 @@ __device__ __forceinline__ void mma_tf32(float (&c)[4], const uint32_t (&a)[4], 
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// Pout = A Pin, with A given transposed (AT[m][i] = A[i][m]); all three d x d
+// Pout = A Pin, with A given transposed (AT[m][i] = A[i][m]) -- or, with
+// kLeftT = false, Pout = AT Pin; all three d x d
 // {hi, lo} arrays with row stride d + kPad.  The 16 x 8 output tiles are
 // spread over the 8 warps, the tiles of one warp sharing their rows (and so
 // their A fragments).  Fragment layout of m16n8k8 (lane = 4 g + t): A rows g
 // and g+8, columns t and t+4; B rows t and t+4, column g; C rows g and g+8,
 // columns 2t and 2t+1.
-template <int DH>
+template <int DH, bool kLeftT = true>
 __device__ __forceinline__ void matmul_tf32x3(const float (*AT)[DH + kPadA], const uint2 (*Pin)[DH + kPad],
                                               uint2 (*Pout)[DH + kPad]) {
     constexpr int MT = DH / 16, NT = DH / 8;             // 16-row and 8-column tiles
@@ -215,8 +222,12 @@ __device__ __forceinline__ void matmul_tf32x3(const float (*AT)[DH + kPadA], con
 #pragma unroll 2
     for (int ks = 0; ks < DH / 8; ++ks) {
         const int k0 = ks * 8 + t;
-        const uint2 a0 = split_tf32(AT[k0][r0]), a1 = split_tf32(AT[k0][r0 + 8]);
-        const uint2 a2 = split_tf32(AT[k0 + 4][r0]), a3 = split_tf32(AT[k0 + 4][r0 + 8]);
+        // kLeftT: the left factor is the transpose of AT (A[r][k] = AT[k][r]);
+        // otherwise AT itself, row-major (the backward's A^T)
+        const uint2 a0 = split_tf32(kLeftT ? AT[k0][r0] : AT[r0][k0]);
+        const uint2 a1 = split_tf32(kLeftT ? AT[k0][r0 + 8] : AT[r0 + 8][k0]);
+        const uint2 a2 = split_tf32(kLeftT ? AT[k0 + 4][r0] : AT[r0][k0 + 4]);
+        const uint2 a3 = split_tf32(kLeftT ? AT[k0 + 4][r0 + 8] : AT[r0 + 8][k0 + 4]);
         const uint32_t ahi[4] = {a0.x, a1.x, a2.x, a3.x}, alo[4] = {a0.y, a1.y, a2.y, a3.y};
 #pragma unroll
         for (int n = 0; n < NPW; ++n) {
@@ -341,17 +352,20 @@ __global__ void __launch_bounds__(kThreads, 2) head_chunk_kernel(const Params pr
 // ---- B: the carries of one (batch row, head), chunk after chunk ----------
 // Thread i keeps row i of the next chunk's P in registers while it applies
 // the current one, so each chunk costs one dependent step, not a load's
-// latency.
-template <int DH>
+// latency.  The forward runs the chunks in time order from delta_{-1} = 0
+// (h0 is given, not solved for); the backward (kReverse) runs them from the
+// end, from mu_T = 0.
+template <int DH, bool kReverse = false>
 __global__ void __launch_bounds__(64) head_carry_kernel(const Params pr) {
     __shared__ float x[2][DH];
     const int64_t seq = blockIdx.x;
     const int i = threadIdx.x;
     const bool act = i < DH;
-    if (act) x[0][i] = 0.0f;  // delta_{-1} = 0: h0 is given, not solved for
+    if (act) x[0][i] = 0.0f;
     float4 row[DH / 4];
     float qv = 0.0f;
-    auto fetch = [&](int c) {
+    auto fetch = [&](int k) {
+        const int c = kReverse ? pr.nChunks - 1 - k : k;
         const int64_t task = seq * pr.nChunks + c;
         const float4* Prow = reinterpret_cast<const float4*>(pr.P + (task * DH + i) * DH);
 #pragma unroll
@@ -368,7 +382,8 @@ __global__ void __launch_bounds__(64) head_carry_kernel(const Params pr) {
         for (int m = 0; m < DH / 4; ++m) r[m] = row[m];
         if (act && c + 1 < pr.nChunks) fetch(c + 1);
         if (act) {
-            pr.carry[(seq * pr.nChunks + c) * DH + i] = x[cur][i];
+            const int cc = kReverse ? pr.nChunks - 1 - c : c;
+            pr.carry[(seq * pr.nChunks + cc) * DH + i] = x[cur][i];
             float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
             for (int m = 0; m < DH / 4; ++m) {
@@ -458,6 +473,259 @@ __global__ void __launch_bounds__(kThreads, 2) head_walk_kernel(const Params pr)
     if (__any_sync(0xffffffffu, bad) && (tid & 31) == 0) atomicOr(pr.status, kStatusNonFinite);
 }
 
+// ==== the adjoint ===========================================================
+// At the trajectory H, with g_t = dL/dH_t, the kernels scan the propagated
+// adjoint mu_t = A_t^T lambda_t in reverse time:
+//     mu_t = A_t^T (g_t + mu_{t+1}),  mu_T = 0,  lambda_t = g_t + mu_{t+1},
+// so that each element needs only its own row's Jacobian (the same reading
+// as the diagonal cells' backward), and dL/dh0 = mu_0.  Then
+//     dL/dp_z = lambda * alpha, dL/dp_r = lambda * beta, dL/dp_c = lambda * z (1 - c^2),
+//     dL/dU_g = sum_{b,t} (lambda * f_g) h_{t-1}^T,  f = alpha, beta, gamma.
+// Launches: the chunk kernel (Q = A_{t0}^T ... A_{t1-1}^T on the tensor cores
+// and the chunk's mu from a zero carry), the carry kernel in reverse chunk
+// order, the walk kernel (lambda, dL/dpx, lambda * gamma, mu, dL/dh0) and a
+// fixed-order reduction of the outer products for dL/dU.
+
+// Per-step inputs of the backward row work for row i: pre-activations,
+// g_t[i], and the state two rows back (the one the next row work needs).
+struct BStepIn {
+    float pz, pr, pc, g, s2;
+};
+
+template <int DH, typename PxT>
+__device__ __forceinline__ BStepIn load_bstep(const Params& pr, int64_t b, int h, int i, int64_t t) {
+    BStepIn in;
+    const int64_t c = (int64_t)h * DH + i;
+    const PxT* x = static_cast<const PxT*>(pr.px) + (b * pr.T + t) * 3 * pr.D + c;
+    in.pz = ldp(x);
+    in.pr = ldp(x + pr.D);
+    in.pc = ldp(x + 2 * pr.D);
+    in.g = pr.G[(b * pr.T + t) * pr.D + c];
+    const int64_t t2 = t - 2;
+    in.s2 = t2 >= 0 ? pr.Hold[(b * pr.T + t2) * pr.D + c] : (t2 == -1 && pr.h0 ? pr.h0[b * pr.D + c] : 0.0f);
+    return in;
+}
+
+// the state just before row t (h_{t-1}, h0 at t = 0)
+template <int DH>
+__device__ __forceinline__ float state_before(const Params& pr, int64_t b, int h, int i, int64_t t) {
+    const int64_t c = (int64_t)h * DH + i;
+    if (t >= 1) return pr.Hold[(b * pr.T + t - 1) * pr.D + c];
+    return pr.h0 ? pr.h0[b * pr.D + c] : 0.0f;
+}
+
+template <int DH>
+struct SmemB {
+    float AT[2][DH][DH + kPadA];  // AT[m][i] = A_t[i][m] = (A_t^T)[m][i], two steps in turn
+    uint2 Pm[2][DH][DH + kPad];   // the running product of transposed Jacobians ({hi, lo} pairs)
+    float sv[2][DH];              // h_{t-1} rows for the row work (permuted)
+    float gv[2][DH];              // g_t rows (permuted)
+    float mv[2][DH];              // mu rows (permuted)
+    float fv[2][4][DH];           // alpha, beta, z (1 - c^2), gamma of the step (walk only)
+};
+
+// The backward's row work for step t, parity p: the gates at (h_{t-1}, x_t),
+// row i of A_t into AT[p], g_t and (walk) the row factors into gv / fv, and
+// h_{t-2} into sv[p ^ 1] for the next (earlier) step's row work.
+template <int DH, bool kWalk>
+__device__ __forceinline__ void bwd_row_work(SmemB<DH>& sm, const RowU<DH>& U, const BStepIn& in, int p, int i,
+                                             int qt) {
+    constexpr int TPR = Geo<DH>::TPR, SEG = Geo<DH>::SEG;
+    float uz = 0.0f, ur = 0.0f, uc = 0.0f;
+#pragma unroll
+    for (int s = 0; s < SEG; ++s) {
+        const float x = sm.sv[p][qt * SEG + s];
+        uz = __fmaf_rn(U.z[s], x, uz);
+        ur = __fmaf_rn(U.r[s], x, ur);
+        uc = __fmaf_rn(U.c[s], x, uc);
+    }
+    uz = row_sum<DH>(uz);
+    ur = row_sum<DH>(ur);
+    uc = row_sum<DH>(uc);
+    const float sp = sm.sv[p][Geo<DH>::vpos(i)];
+    const float z = sigmoid_f(in.pz + uz);
+    const float r = sigmoid_f(in.pr + ur);
+    const float c = tanh_f(__fmaf_rn(r, uc, in.pc));
+    const float zc = z * __fmaf_rn(-c, c, 1.0f);
+    const float dz = 1.0f - z, al = (c - sp) * (z - z * z), be = zc * uc * (r - r * r), ga = zc * r;
+#pragma unroll
+    for (int s = 0; s < SEG; ++s) {
+        const int m = qt + TPR * s;
+        float a = __fmaf_rn(al, U.z[s], (m == i) ? dz : 0.0f);
+        a = __fmaf_rn(be, U.r[s], a);
+        a = __fmaf_rn(ga, U.c[s], a);
+        sm.AT[p][m][i] = a;
+    }
+    if (qt == 0) {
+        const int vi = Geo<DH>::vpos(i);
+        sm.gv[p][vi] = in.g;
+        sm.sv[p ^ 1][vi] = in.s2;
+        if constexpr (kWalk) {
+            sm.fv[p][0][vi] = al;
+            sm.fv[p][1][vi] = be;
+            sm.fv[p][2][vi] = zc;
+            sm.fv[p][3][vi] = ga;
+        }
+    }
+}
+
+// mu_t[m] = sum_i AT[p][m][i] (g_t[i] + mu_{t+1}[i]) for thread (m, qt)
+template <int DH>
+__device__ __forceinline__ float bwd_mu(const SmemB<DH>& sm, int p, int m, int qt) {
+    constexpr int TPR = Geo<DH>::TPR, SEG = Geo<DH>::SEG;
+    float acc = 0.0f;
+#pragma unroll
+    for (int s = 0; s < SEG; ++s) {
+        const int i = qt + TPR * s;
+        const float lam = sm.gv[p][qt * SEG + s] + sm.mv[p ^ 1][qt * SEG + s];
+        acc = __fmaf_rn(sm.AT[p][m][i], lam, acc);
+    }
+    return row_sum<DH>(acc);
+}
+
+// ---- backward A: the chunk's product of transposed Jacobians -------------
+// Steps run from t1-1 down to t0 (r = t1-1-t, p = r & 1); as in the forward
+// chunk kernel the product of step t and mu_t share a barrier interval with
+// the row work of step t-1.
+template <int DH, typename PxT, bool kWalk>
+__global__ void __launch_bounds__(kThreads, 2) head_bwd_kernel(const Params pr) {
+    using Gm = Geo<DH>;
+    constexpr int TPR = Gm::TPR;
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    auto& sm = *reinterpret_cast<SmemB<DH>*>(smem_raw);
+    const int tid = threadIdx.x, i = tid / TPR, qt = tid % TPR;
+    const int64_t task = blockIdx.x;
+    const int64_t seq = task / pr.nChunks;
+    const int chunk = (int)(task - seq * pr.nChunks);
+    const int64_t b = seq / pr.nh;
+    const int h = (int)(seq - b * pr.nh);
+    const int64_t t0 = (int64_t)chunk * kChunk;
+    const int64_t t1 = t0 + kChunk < pr.T ? t0 + kChunk : pr.T;
+
+    RowU<DH> U;
+    U.load(pr.U, pr.nh, h, i, qt);
+    if (qt == 0) {
+        sm.sv[0][Gm::vpos(i)] = state_before<DH>(pr, b, h, i, t1 - 1);
+        // mu_{t1}: zero for the chunk's own product, the carry for the walk
+        sm.mv[1][Gm::vpos(i)] = kWalk ? pr.carry[task * DH + i] : 0.0f;
+    }
+    if constexpr (!kWalk)
+        for (int idx = tid; idx < DH * DH; idx += kThreads)
+            sm.Pm[0][idx / DH][idx % DH] = make_uint2(idx / DH == idx % DH ? __float_as_uint(1.0f) : 0u, 0u);
+    BStepIn nxt = load_bstep<DH, PxT>(pr, b, h, i, t1 - 1);
+    __syncthreads();
+    {
+        const BStepIn in = nxt;
+        if (t1 - 2 >= t0) nxt = load_bstep<DH, PxT>(pr, b, h, i, t1 - 2);
+        bwd_row_work<DH, kWalk>(sm, U, in, 0, i, qt);
+    }
+    __syncthreads();
+    int p = 0, cur = 0;
+    bool bad = false;
+    for (int64_t t = t1 - 1; t >= t0; --t) {
+        if constexpr (!kWalk) matmul_tf32x3<DH, false>(sm.AT[p], sm.Pm[cur], sm.Pm[cur ^ 1]);
+        const float mu = bwd_mu<DH>(sm, p, i, qt);  // thread (m = i, qt)
+        if (qt == 0) {
+            sm.mv[p][Gm::vpos(i)] = mu;
+            if constexpr (kWalk) {
+                // the epilogue of row i at step t
+                const int vi = Gm::vpos(i);
+                const float lam = sm.gv[p][vi] + sm.mv[p ^ 1][vi];
+                const int64_t o = ((b * pr.T + t) * 3) * pr.D + (int64_t)h * DH + i;
+                const float d0 = lam * sm.fv[p][0][vi], d1 = lam * sm.fv[p][1][vi], d2 = lam * sm.fv[p][2][vi];
+                pr.dpx[o] = d0;
+                pr.dpx[o + pr.D] = d1;
+                pr.dpx[o + 2 * pr.D] = d2;
+                pr.ec[(b * pr.T + t) * pr.D + (int64_t)h * DH + i] = lam * sm.fv[p][3][vi];
+                bad |= !(isfinite(d0) && isfinite(d1) && isfinite(d2));
+                if (t == 0 && pr.dh0) pr.dh0[b * pr.D + (int64_t)h * DH + i] = mu;
+            }
+        }
+        if (t - 1 >= t0) {
+            const BStepIn in = nxt;
+            if (t - 2 >= t0) nxt = load_bstep<DH, PxT>(pr, b, h, i, t - 2);
+            bwd_row_work<DH, kWalk>(sm, U, in, p ^ 1, i, qt);
+        }
+        __syncthreads();
+        cur ^= 1;
+        p ^= 1;
+    }
+    if constexpr (!kWalk) {
+        float* Pout = pr.P + task * DH * DH;
+        for (int idx = tid; idx < DH * DH; idx += kThreads) {
+            const uint2 v = sm.Pm[cur][idx / DH][idx % DH];
+            Pout[idx] = __uint_as_float(v.x) + __uint_as_float(v.y);
+        }
+        // mu at the chunk's first step: written to mv[p ^ 1] by the last iteration
+        if (qt == 0) pr.q[task * DH + i] = sm.mv[p ^ 1][Gm::vpos(i)];
+    } else {
+        if (__any_sync(0xffffffffu, bad) && (tid & 31) == 0) atomicOr(pr.status, kStatusNonFinite);
+    }
+}
+
+// ---- dL/dU: outer products summed in a fixed order -------------------------
+// part[split][g][h] = sum over the split's rows (b, t) of e_g[b,t] h_{t-1}^T
+// (e_z = dL/dp_z, e_r = dL/dp_r, e_c = lambda * gamma), rows in increasing
+// (b, t) order; the reduce kernel sums the splits in order.
+constexpr int kURows = 32;
+
+template <int DH>
+__global__ void __launch_bounds__(kThreads) head_dU_kernel(const Params pr, int64_t rows_per_split, float* part) {
+    __shared__ float Es[kURows][DH], Ss[kURows][DH];
+    constexpr int TM = DH / 16;
+    const int tid = threadIdx.x, i0 = (tid / 16) * TM, j0 = (tid % 16) * TM;
+    const int split = blockIdx.x, gh = blockIdx.y, g = gh / pr.nh, h = gh % pr.nh;
+    const int64_t nrows = pr.B * pr.T;
+    const int64_t r0 = split * rows_per_split;
+    const int64_t r1 = r0 + rows_per_split < nrows ? r0 + rows_per_split : nrows;
+    float acc[TM][TM];
+#pragma unroll
+    for (int a = 0; a < TM; ++a)
+#pragma unroll
+        for (int c = 0; c < TM; ++c) acc[a][c] = 0.0f;
+    for (int64_t rb = r0; rb < r1; rb += kURows) {
+        for (int idx = tid; idx < kURows * DH; idx += kThreads) {
+            const int rr = idx / DH, k = idx - rr * DH;
+            const int64_t row = rb + rr;
+            float e = 0.0f, sv = 0.0f;
+            if (row < r1) {
+                const int64_t bb = row / pr.T, t = row - bb * pr.T, c = (int64_t)h * DH + k;
+                e = g < 2 ? pr.dpx[((bb * pr.T + t) * 3 + g) * pr.D + c] : pr.ec[(bb * pr.T + t) * pr.D + c];
+                sv = t >= 1 ? pr.Hold[(bb * pr.T + t - 1) * pr.D + c] : (pr.h0 ? pr.h0[bb * pr.D + c] : 0.0f);
+            }
+            Es[rr][k] = e;
+            Ss[rr][k] = sv;
+        }
+        __syncthreads();
+#pragma unroll 4
+        for (int rr = 0; rr < kURows; ++rr) {
+            float ev[TM], sw[TM];
+#pragma unroll
+            for (int a = 0; a < TM; ++a) ev[a] = Es[rr][i0 + a];
+#pragma unroll
+            for (int c = 0; c < TM; ++c) sw[c] = Ss[rr][j0 + c];
+#pragma unroll
+            for (int a = 0; a < TM; ++a)
+#pragma unroll
+                for (int c = 0; c < TM; ++c) acc[a][c] = __fmaf_rn(ev[a], sw[c], acc[a][c]);
+        }
+        __syncthreads();
+    }
+    float* out = part + ((int64_t)split * gridDim.y + gh) * DH * DH;
+#pragma unroll
+    for (int a = 0; a < TM; ++a)
+#pragma unroll
+        for (int c = 0; c < TM; ++c) out[(i0 + a) * DH + j0 + c] = acc[a][c];
+}
+
+__global__ void head_dU_reduce_kernel(const float* part, int nsplit, int64_t n, float* dU) {
+    const int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (k >= n) return;
+    float acc = 0.0f;
+    for (int sp = 0; sp < nsplit; ++sp) acc += part[sp * n + k];
+    dU[k] = acc;
+}
+
 // ---- host side --------------------------------------------------------------
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -515,6 +783,56 @@ cudaError_t launch_all(const Plan& pl, Params pr, float* H_out, float* Hbuf, int
         pr.k = K;
         pr.Hold = H_out;
         head_chunk_kernel<DH, PxT, true><<<ntask, kThreads, smemR, st>>>(pr);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+struct BPlan {
+    int d = 0, nChunks = 0, nsplit = 0;
+    int64_t nSeq = 0, rows_per_split = 0;
+    size_t off_P = 0, off_q = 0, off_c = 0, off_ec = 0, off_part = 0, total = 0;
+};
+
+// backward workspace: 256-byte header (status word) | chunk products Q |
+// chunk mus q | chunk carries | lambda * gamma (B,T,D) | dL/dU split partials
+bool make_bplan(int64_t B, int64_t T, int64_t D, int nh, BPlan& pl) {
+    Plan fp;
+    if (!make_plan(B, T, D, nh, 1, fp)) return false;
+    pl.d = fp.d;
+    pl.nChunks = fp.nChunks;
+    pl.nSeq = fp.nSeq;
+    const size_t ntask = (size_t)pl.nSeq * pl.nChunks, d = pl.d;
+    const int64_t rows = B * T;
+    pl.nsplit = (int)(rows > 0 ? (rows + 255) / 256 : 1);
+    if (pl.nsplit > 64) pl.nsplit = 64;
+    pl.rows_per_split = rows > 0 ? (rows + pl.nsplit - 1) / pl.nsplit : 1;
+    pl.off_P = 256;
+    pl.off_q = align256(pl.off_P + ntask * d * d * sizeof(float));
+    pl.off_c = align256(pl.off_q + ntask * d * sizeof(float));
+    pl.off_ec = align256(pl.off_c + ntask * d * sizeof(float));
+    pl.off_part = align256(pl.off_ec + (size_t)B * T * D * sizeof(float));
+    pl.total = align256(pl.off_part + (size_t)pl.nsplit * 3 * nh * d * d * sizeof(float));
+    return true;
+}
+
+template <int DH, typename PxT>
+cudaError_t launch_bwd(const BPlan& pl, const Params& pr, float* dU, cudaStream_t st) {
+    const size_t smem = sizeof(SmemB<DH>);
+    cudaError_t e = set_smem(head_bwd_kernel<DH, PxT, false>, smem);
+    if (e == cudaSuccess) e = set_smem(head_bwd_kernel<DH, PxT, true>, smem);
+    if (e != cudaSuccess) return e;
+    const unsigned ntask = (unsigned)(pl.nSeq * pl.nChunks);
+    head_bwd_kernel<DH, PxT, false><<<ntask, kThreads, smem, st>>>(pr);
+    head_carry_kernel<DH, true><<<(unsigned)pl.nSeq, 64, 0, st>>>(pr);
+    head_bwd_kernel<DH, PxT, true><<<ntask, kThreads, smem, st>>>(pr);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (dU) {
+        float* part = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(pr.status) + pl.off_part);
+        head_dU_kernel<DH><<<dim3((unsigned)pl.nsplit, (unsigned)(3 * pr.nh)), kThreads, 0, st>>>(
+            pr, pl.rows_per_split, part);
+        const int64_t n = (int64_t)3 * pr.nh * DH * DH;
+        head_dU_reduce_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(part, pl.nsplit, n, dU);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     return cudaSuccess;
@@ -604,6 +922,85 @@ extern "C" pararnn_status pararnn_head_gru_forward(int64_t B, int64_t T, int64_t
     if (e != cudaSuccess) {
         cudaGetLastError();
         return hg::fail(PARARNN_ECUDA, "pararnn_head_gru_forward: kernel launch failed");
+    }
+    return PARARNN_OK;
+}
+
+extern "C" size_t pararnn_head_gru_backward_workspace_bytes(int64_t B, int64_t T, int64_t D, int n_heads) {
+    hg::BPlan pl;
+    if (!hg::make_bplan(B, T, D, n_heads, pl)) return 0;
+    return pl.total;
+}
+
+extern "C" pararnn_status pararnn_head_gru_backward(int64_t B, int64_t T, int64_t D, int n_heads,
+                                                    pararnn_dtype px_dtype, const void* preacts, const float* U,
+                                                    const float* h0, const float* H, const float* dL_dH,
+                                                    float* dL_dpx, float* dL_dU, float* dL_dh0, void* workspace,
+                                                    size_t ws_bytes, void* stream) {
+    hg::BPlan pl;
+    if (!hg::make_bplan(B, T, D, n_heads, pl))
+        return hg::fail(PARARNN_EINVAL,
+                        "pararnn_head_gru_backward: need B, T, D >= 0, D = n_heads * d with d in {16, 32, 64}, "
+                        "and B*T below 2^31");
+    if (px_dtype != PARARNN_F32 && px_dtype != PARARNN_BF16)
+        return hg::fail(PARARNN_EINVAL, "pararnn_head_gru_backward: unknown pre-activation dtype");
+    if (!workspace || ws_bytes < pl.total)
+        return hg::fail(PARARNN_EINVAL, "pararnn_head_gru_backward: workspace missing or smaller than "
+                                        "pararnn_head_gru_backward_workspace_bytes()");
+    if (!pointer_on_device(workspace) || (reinterpret_cast<uintptr_t>(workspace) & 255))
+        return hg::fail(PARARNN_EINVAL, "pararnn_head_gru_backward: workspace must be 256-byte aligned device memory");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    unsigned char* ws = static_cast<unsigned char*>(workspace);
+    cudaError_t e = cudaMemsetAsync(ws, 0, 256, st);
+    if (e != cudaSuccess) return hg::fail(PARARNN_ECUDA, "pararnn_head_gru_backward: header reset failed");
+    const int d = pl.d;
+    if (B == 0 || T == 0 || D == 0) {
+        // nothing flows back: dL/dU (and dL/dh0) are zero
+        if (dL_dU && pointer_on_device(dL_dU)) cudaMemsetAsync(dL_dU, 0, sizeof(float) * 3 * n_heads * d * d, st);
+        if (dL_dh0 && pointer_on_device(dL_dh0)) cudaMemsetAsync(dL_dh0, 0, sizeof(float) * B * D, st);
+        return PARARNN_OK;
+    }
+    const size_t esz = px_dtype == PARARNN_BF16 ? 2 : 4;
+    const void* need[] = {preacts, U, H, dL_dH, dL_dpx};
+    for (const void* q : need)
+        if (!q || !pointer_on_device(q))
+            return hg::fail(PARARNN_EINVAL, "pararnn_head_gru_backward: a required pointer is null or not device memory");
+    const void* opt[] = {h0, dL_dU, dL_dh0};
+    for (const void* q : opt)
+        if (q && (!pointer_on_device(q) || (reinterpret_cast<uintptr_t>(q) & 3)))
+            return hg::fail(PARARNN_EINVAL, "pararnn_head_gru_backward: h0, dL_dU or dL_dh0 is not aligned device memory");
+    if ((reinterpret_cast<uintptr_t>(preacts) % esz) || (reinterpret_cast<uintptr_t>(U) & 3) ||
+        (reinterpret_cast<uintptr_t>(H) & 3) || (reinterpret_cast<uintptr_t>(dL_dH) & 3) ||
+        (reinterpret_cast<uintptr_t>(dL_dpx) & 3))
+        return hg::fail(PARARNN_EINVAL, "pararnn_head_gru_backward: misaligned pointer");
+    hg::Params pr;
+    memset(&pr, 0, sizeof pr);
+    pr.px = preacts;
+    pr.U = U;
+    pr.h0 = h0;
+    pr.Hold = H;
+    pr.G = dL_dH;
+    pr.dpx = dL_dpx;
+    pr.dh0 = dL_dh0;
+    pr.P = reinterpret_cast<float*>(ws + pl.off_P);
+    pr.q = reinterpret_cast<float*>(ws + pl.off_q);
+    pr.carry = reinterpret_cast<float*>(ws + pl.off_c);
+    pr.ec = reinterpret_cast<float*>(ws + pl.off_ec);
+    pr.status = reinterpret_cast<unsigned*>(ws);
+    pr.B = B;
+    pr.T = T;
+    pr.D = D;
+    pr.nh = n_heads;
+    pr.nChunks = pl.nChunks;
+    const bool bf = px_dtype == PARARNN_BF16;
+    switch (d) {
+        case 16: e = bf ? hg::launch_bwd<16, __nv_bfloat16>(pl, pr, dL_dU, st) : hg::launch_bwd<16, float>(pl, pr, dL_dU, st); break;
+        case 32: e = bf ? hg::launch_bwd<32, __nv_bfloat16>(pl, pr, dL_dU, st) : hg::launch_bwd<32, float>(pl, pr, dL_dU, st); break;
+        default: e = bf ? hg::launch_bwd<64, __nv_bfloat16>(pl, pr, dL_dU, st) : hg::launch_bwd<64, float>(pl, pr, dL_dU, st); break;
+    }
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return hg::fail(PARARNN_ECUDA, "pararnn_head_gru_backward: kernel launch failed");
     }
     return PARARNN_OK;
 }

@@ -121,3 +121,61 @@ def test_head_empty_and_nonfinite(cuda_device):
     with pytest.raises(binding.PararnnError) as e:
         binding.head_gru_forward(px, U, None, K=2)
     assert e.value.status == binding.ENONFINITE
+
+
+# ---- the adjoint ---------------------------------------------------------
+TOL_G = 1e-3
+
+BWD_CASES = [  # (B, T, D, n_heads, K)
+    (2, 100, 64, 1, 3),
+    (1, 150, 96, 3, 2),
+    (2, 40, 64, 2, 1),
+    (1, 200, 128, 2, 3),
+]
+
+
+@pytest.mark.parametrize("case", BWD_CASES, ids=lambda c: "B%dT%dD%dh%dK%d" % c)
+@pytest.mark.parametrize("h0", [False, True])
+def test_head_backward_small(case, h0, cuda_device):
+    B, T, D, nh, K = case
+    px, U, hz, pxt, Ut, h0t = _case(B, T, D, nh, seed=3 * D + T, h0=h0)
+    g = np.random.default_rng(T + D).standard_normal((B, T, D)).astype(np.float32)
+    H = binding.head_gru_forward(pxt, Ut, h0t, K=K)
+    dpx, dU, dh0 = binding.head_gru_backward(pxt, Ut, H, torch.from_numpy(g).to(DEV), h0=h0t, want_dh0=True)
+    r_dpx, r_dU, r_dh0 = oracle.head_gru_adjoint(px, U, to_np(H), g, hz)
+    assert rel_err(to_np(dpx), r_dpx) <= TOL_G
+    assert rel_err(to_np(dU), r_dU) <= TOL_G
+    assert rel_err(to_np(dh0), r_dh0) <= TOL_G
+
+
+def test_head_backward_deterministic_and_optional_outputs(cuda_device):
+    B, T, D, nh = 2, 300, 128, 2
+    _, _, _, pxt, Ut, _ = _case(B, T, D, nh, seed=21)
+    H = binding.head_gru_forward(pxt, Ut, None, K=3)
+    g = torch.randn((B, T, D), device=DEV)
+    a = binding.head_gru_backward(pxt, Ut, H, g, want_dh0=True)
+    b = binding.head_gru_backward(pxt, Ut, H, g, want_dh0=True)
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1]) and torch.equal(a[2], b[2])
+    c = binding.head_gru_backward(pxt, Ut, H, g, want_dU=False)
+    assert c[1] is None and c[2] is None and torch.equal(c[0], a[0])
+
+
+def test_head_backward_full_size_sampled(cuda_device):
+    w = workloads.HEAD_WORKLOADS["headgru_8x4096x512_h8_k3"]
+    x = workloads.head_device_inputs(w, DEV)
+    H = binding.head_gru_forward(x["px"], x["U"], None, K=w.K)
+    g = torch.randn((w.B, w.T, w.D), device=DEV, generator=torch.Generator(device=DEV).manual_seed(77))
+    dpx, dU, _ = binding.head_gru_backward(x["px"], x["U"], H, g)
+    # dL/dpx per sampled (b, head) sequence; dL/dU of one head summed over all b
+    U = x["U"].cpu().numpy()
+    h = 5
+    sl = slice(h * w.d, (h + 1) * w.d)
+    dU_ref = np.zeros((3, 1, w.d, w.d))
+    for b in range(w.B):
+        px = x["px"][b:b + 1, :, :, sl].cpu().numpy()
+        r_dpx, r_dU, _ = oracle.head_gru_adjoint(px, U[:, h:h + 1], to_np(H[b:b + 1, :, sl]),
+                                                 to_np(g[b:b + 1, :, sl]))
+        dU_ref += r_dU
+        if b in (0, 5):
+            assert rel_err(to_np(dpx[b:b + 1, :, :, sl]), r_dpx) <= TOL_G, b
+    assert rel_err(to_np(dU[:, h:h + 1]), dU_ref) <= TOL_G
