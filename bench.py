@@ -127,8 +127,9 @@ TF32_PER_BF16 = 1.1 / 2.25
 
 
 def time_head(w, device, steps, warmup):
-    """Device time of one head-wise GRU forward call (CUDA events on the
-    launching stream); returns (ms, status name)."""
+    """Device times of one head-wise GRU forward call and one adjoint call at
+    its output (CUDA events on the launching stream); returns
+    (forward ms, backward ms, status name)."""
     import torch
 
     from nonlinear_rnn_iteration_b200 import binding, workloads
@@ -137,29 +138,39 @@ def time_head(w, device, steps, warmup):
     H = torch.empty((w.B, w.T, w.D), device=device)
     n = binding.pararnn_head_gru_workspace_bytes(w.B, w.T, w.D, w.n_heads, w.K)
     ws = torch.empty(n, dtype=torch.uint8, device=device)
+    nb = binding.pararnn_head_gru_backward_workspace_bytes(w.B, w.T, w.D, w.n_heads)
+    wsb = torch.empty(nb, dtype=torch.uint8, device=device)
+    g = torch.randn((w.B, w.T, w.D), device=device, generator=torch.Generator(device=device).manual_seed(w.seed + 100))
     stream = torch.cuda.current_stream(device)
 
-    def call():
+    def fwd():
         binding.head_gru_forward(x["px"], x["U"], None, K=w.K, out=H, workspace=ws, stream=stream,
                                  sync_status=False)
 
-    for _ in range(warmup):
-        call()
-    torch.cuda.synchronize(device)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(steps):
-        call()
-    e1.record(stream)
-    torch.cuda.synchronize(device)
-    ms = e0.elapsed_time(e1) / steps
+    def bwd():
+        binding.head_gru_backward(x["px"], x["U"], H, g, workspace=wsb, stream=stream, sync_status=False)
+
+    times = []
+    for f in (fwd, bwd):
+        for _ in range(warmup):
+            f()
+        torch.cuda.synchronize(device)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            f()
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        times.append(e0.elapsed_time(e1) / steps)
     st = binding.pararnn_status_sync(ws, stream)
-    del x, H, ws
+    if st == binding.OK:
+        st = binding.pararnn_status_sync(wsb, stream)
+    del x, H, ws, wsb, g
     torch.cuda.empty_cache()
-    return ms, binding.STATUS.get(st, st)
+    return times[0], times[1], binding.STATUS.get(st, st)
 
 
-def head_line(w, ms, status):
+def head_line(w, ms, bwd_ms, status):
     """A head-wise forward's line: time, elements/s, and the FLOP rate of its
     Jacobian products -- 2 d^3 useful FLOP per step and (batch row, head),
     issued as three TF32 products -- against the TF32 tensor peak."""
@@ -167,7 +178,8 @@ def head_line(w, ms, status):
     useful = 2.0 * w.d ** 3 * w.B * w.T * w.n_heads * w.K
     tf32_peak = peaks["bf16_tflops"] * TF32_PER_BF16
     return {"ms_per_step": round(ms, 4), "elem_per_s": w.elements / (ms / 1e3), "K": w.K,
-            "n_heads": w.n_heads, "d": w.d, "status": status,
+            "n_heads": w.n_heads, "d": w.d, "status": status, "bwd_ms": round(bwd_ms, 4),
+            "bwd_elem_per_s": w.elements / (bwd_ms / 1e3),
             "roofline": {"bound": "tensor", "kernel": "head_chunk_kernel (Jacobian products)",
                          "achieved_useful": round(useful / (ms / 1e3) / 1e12, 2),
                          "achieved_issued": round(3 * useful / (ms / 1e3) / 1e12, 2),
@@ -181,8 +193,8 @@ def head_workloads(device):
 
     out = {}
     for name, w in workloads.HEAD_WORKLOADS.items():
-        ms, status = time_head(w, device, steps=5, warmup=3)
-        out[name] = head_line(w, ms, status)
+        ms, bms, status = time_head(w, device, steps=5, warmup=3)
+        out[name] = head_line(w, ms, bms, status)
     return out
 
 
@@ -522,8 +534,9 @@ def run_head(args):
                                    args.T or w.T, w.D, w.n_heads, w.K, w.px_dtype, w.seed)
     device = torch.device("cuda", 0)
     torch.cuda.set_device(device)
-    ms, status = time_head(w, device, args.steps, args.warmup)
-    line = {"workload": w.name, "metric": METRIC, "unit": UNIT, "data": "synthetic", **head_line(w, ms, status)}
+    ms, bms, status = time_head(w, device, args.steps, args.warmup)
+    line = {"workload": w.name, "metric": METRIC, "unit": UNIT, "data": "synthetic",
+            **head_line(w, ms, bms, status)}
     print(json.dumps(line), flush=True)
 
 

@@ -1,4 +1,4 @@
-// head_gru.cu -- Newton forward of the head-wise GRU (block-diagonal
+// head_gru.cu -- Newton forward and adjoint of the head-wise GRU (block-diagonal
 // recurrent weights: ParaGRU(mix='head', n_heads) on the pararnn-torch page,
 // Models / Usage, "block-diagonal A").
 //
@@ -20,7 +20,10 @@
 //   C. per chunk: re-walk from its carry, delta_t = A_t delta_{t-1} - F_t
 //      (A_t applied as the sum above, never formed), and write h^(k+1).
 // No block waits on another, so there is no look-back and nothing to time
-// out.  All arithmetic is float32; pre-activations f32 or bf16.
+// out.  All arithmetic is float32; pre-activations f32 or bf16.  The adjoint
+// (pararnn_head_gru_backward) runs the same three launches in reverse time
+// on the propagated adjoint, plus a fixed-order reduction for dL/dU (see
+// "the adjoint" below).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 

@@ -28,10 +28,11 @@ def test_head_line_arithmetic():
     from nonlinear_rnn_iteration_b200 import workloads
 
     w = workloads.HEAD_WORKLOADS["headgru_8x4096x512_h8_k3"]
-    line = bench.head_line(w, 10.0, "PARARNN_OK")
+    line = bench.head_line(w, 10.0, 5.0, "PARARNN_OK")
     useful = 2.0 * 64 ** 3 * 8 * 4096 * 8 * 3 / 1e-2 / 1e12
     assert abs(line["roofline"]["achieved_useful"] - round(useful, 2)) < 1e-9
     assert line["elem_per_s"] == w.elements / 1e-2
+    assert line["bwd_elem_per_s"] == w.elements / 5e-3
     json.dumps(line)
 
 
