@@ -13,7 +13,7 @@ gru_1x1024x64_k3          GRU     1     1024     64     3    f32
 linear_8x16384x1024       linear  8     16384    1024   1    f32
 gru_8x4096x2048_k3        GRU     8     4096     2048   3    f32
 gru_8x4096x2048_k3_bf16   GRU     8     4096     2048   3    bf16 (f32 state)
-lstm_4x32768x1024_k4      LSTM    4     32768    1024   4    f32
+lstm_4x32768x1024_k4      LSTM    4     32768    1024   4    f32, + backward
 gru_1x131072x4096_k2_bf16 GRU     1     131072   4096   2    bf16, + backward
 ========================  ======  ====  =======  =====  ===  ===============
 
@@ -86,7 +86,7 @@ WORKLOADS = {
         Workload("linear_8x16384x1024", "linear", 8, 16384, 1024, 1, "f32", 1),
         Workload("gru_8x4096x2048_k3", "diag_gru", 8, 4096, 2048, 3, "f32", 2),
         Workload("gru_8x4096x2048_k3_bf16", "diag_gru", 8, 4096, 2048, 3, "bf16", 2),
-        Workload("lstm_4x32768x1024_k4", "diag_lstm", 4, 32768, 1024, 4, "f32", 3),
+        Workload("lstm_4x32768x1024_k4", "diag_lstm", 4, 32768, 1024, 4, "f32", 3, backward=True),
         Workload("gru_1x131072x4096_k2_bf16", "diag_gru", 1, 131072, 4096, 2, "bf16", 4, backward=True),
     ]
 }
