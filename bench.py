@@ -351,9 +351,11 @@ def time_device(prob, steps, warmup, dist, device, per_call=True):
 
 
 def time_e2e(prob, steps):
-    """Same step through the public API with host buffers: pinned host ->
-    device copy of the pre-activations, the forward (and backward) call, device
-    -> host copy of the result, all inside the timed region."""
+    """Same step through the public API with host buffers, all copies inside
+    the timed region: a forward-only step goes through the host-buffer entry
+    point (pinned host in, pinned host out, copies overlapped with the solve);
+    a step with a backward copies the pre-activations and dL/dH in, runs both
+    calls and copies H and dL/dpx out."""
     import torch
 
     w = prob.w
@@ -368,6 +370,31 @@ def time_e2e(prob, steps):
         outs.append(dpx_host)
     px_dev = torch.empty_like(prob.px)
     s = prob.stream
+    if not w.backward:
+        # the public host-buffer entry point: slices of batch rows whose copies
+        # in and out overlap the solve
+        from nonlinear_rnn_iteration_b200 import binding
+
+        code = binding.BF16 if prob.px.dtype == torch.bfloat16 else binding.F32
+        n = binding.pararnn_newton_forward_host_workspace_bytes(w.cell_id, w.B, w.T, w.D, w.K, code, 1)
+        ws_host = torch.zeros(n, dtype=torch.uint8, device=prob.px.device)
+
+        def one():
+            st = binding.pararnn_newton_forward_host(w.cell_id, w.B, w.T, w.D, code, px_host, prob.a, None, w.K,
+                                                     H_host, ws_host, n, 1, s)
+            if st != binding.OK:
+                raise RuntimeError("pararnn_newton_forward_host: %s" % binding.pararnn_last_error())
+
+        one()
+        torch.cuda.synchronize()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(s)
+        for _ in range(steps):
+            one()
+        t1.record(s)
+        torch.cuda.synchronize()
+        ms = t0.elapsed_time(t1) / steps
+        return ms, px_host.numel() * px_host.element_size(), H_host.numel() * 4
 
     def one():
         px_dev.copy_(px_host, non_blocking=True)

@@ -193,6 +193,34 @@ pararnn_status pararnn_newton_forward_noalloc(pararnn_cell cell, int64_t B, int6
                                               const float* h0, int K, float* H_out, float* resid_hist,
                                               int wait_status, void* stream);
 
+/* ---- the forward on host buffers (serving) --------------------------------
+ * pararnn_newton_forward for pre-activations and H in host memory (pinned
+ * memory lets the copies overlap; pageable memory works, with the copies
+ * serialised).  The batch is cut into slices of rows_per_slice rows that
+ * pass through three device slots on three internal streams -- copy in,
+ * solve, copy out -- so that both PCIe directions and the solver work at
+ * once.  Batch rows are independent recurrences, so every row of H is
+ * bit-identical to pararnn_newton_forward's on the whole batch.
+ *   preacts_host  (B, T, G, D) px_dtype, host (or device) memory
+ *   diag_w, h0    device memory, as for pararnn_newton_forward
+ *   H_host        (B, T, S, D) float32, host (or device) memory
+ *   workspace     >= pararnn_newton_forward_host_workspace_bytes(...) bytes,
+ *                 256-byte aligned device memory, zero-filled once at
+ *                 allocation like the ordinary workspace
+ * The work is ordered after what is already queued on `stream`, and work
+ * queued on `stream` afterwards runs after it; the call returns once
+ * everything is queued.  No residual history is kept.  A non-finite value in
+ * any slice's output is reported by pararnn_status_sync(workspace, stream).
+ * Errors as for pararnn_newton_forward, plus PARARNN_EINVAL for
+ * rows_per_slice < 1 and PARARNN_ECUDA if the internal streams cannot be
+ * created. */
+size_t pararnn_newton_forward_host_workspace_bytes(pararnn_cell cell, int64_t B, int64_t T, int64_t D, int K,
+                                                   pararnn_dtype px_dtype, int64_t rows_per_slice);
+pararnn_status pararnn_newton_forward_host(pararnn_cell cell, int64_t B, int64_t T, int64_t D,
+                                           pararnn_dtype px_dtype, const void* preacts_host, const float* diag_w,
+                                           const float* h0, int K, float* H_host, void* workspace, size_t ws_bytes,
+                                           int64_t rows_per_slice, void* stream);
+
 /* ---- head-wise GRU: block-diagonal recurrent weights --------------------
  * ParaGRU(mix='head', n_heads) of the pararnn-torch page (Models / Usage,
  * "Dreamer-style block GRU": block-diagonal A).  The page prints no

@@ -1,0 +1,181 @@
+// host_path.cu -- the Newton forward on host buffers, copies overlapped with
+// the solve.
+//
+// A serving caller usually holds the pre-activations in host memory and
+// wants H back there.  Copying everything in, solving, and copying
+// everything out leaves the PCIe link idle in one direction at a time and
+// the GPU idle during both copies.  Batch rows are independent recurrences
+// (the tiles of the solver never span two rows), so this entry point cuts
+// the batch into slices of rows and pipelines them through kSlots device
+// slots on three streams -- copy in, solve, copy out -- so that slice i+1
+// comes in while slice i is solved and slice i-1 goes out.  Every row's
+// result is bit-identical to what pararnn_newton_forward returns for the
+// whole batch.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "common.cuh"
+#include "pararnn_b200.h"
+
+namespace pararnn {
+void set_last_error(const char* msg);   // pararnn_abi.cu
+bool pointer_on_device(const void* p);  // pararnn_abi.cu
+
+namespace hp {
+
+constexpr int kSlots = 3;
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct Layout {
+    int64_t rows = 0;  // batch rows per slice
+    size_t px_bytes = 0, h_bytes = 0, fw_bytes = 0, slot_bytes = 0, total = 0;
+};
+
+bool layout(pararnn_cell cell, int64_t B, int64_t T, int64_t D, int K, int64_t rows_per_slice, size_t esz,
+            Layout& l) {
+    const int G = pararnn_num_gates(cell), S = pararnn_state_width(cell);
+    if (G < 0 || B < 0 || T < 0 || D < 0 || rows_per_slice < 1) return false;
+    l.rows = rows_per_slice < B ? rows_per_slice : (B > 0 ? B : 1);
+    l.fw_bytes = pararnn_workspace_bytes(cell, l.rows, T, D, K);
+    if (l.fw_bytes == 0) return false;
+    l.px_bytes = align256((size_t)l.rows * T * G * D * esz);
+    l.h_bytes = align256((size_t)l.rows * T * S * D * sizeof(float));
+    l.slot_bytes = align256(l.fw_bytes) + l.px_bytes + l.h_bytes;
+    l.total = 256 + kSlots * l.slot_bytes;
+    return true;
+}
+
+// fold one slot's device status into the call's header
+__global__ void fold_status(unsigned* dst, const unsigned* src) {
+    if (threadIdx.x == 0 && *src) atomicOr(dst, *src);
+}
+
+pararnn_status fail(pararnn_status st, const char* msg) {
+    set_last_error(msg);
+    return st;
+}
+
+}  // namespace hp
+}  // namespace pararnn
+
+using namespace pararnn;
+
+extern "C" size_t pararnn_newton_forward_host_workspace_bytes(pararnn_cell cell, int64_t B, int64_t T, int64_t D,
+                                                              int K, pararnn_dtype px_dtype,
+                                                              int64_t rows_per_slice) {
+    hp::Layout l;
+    const size_t esz = px_dtype == PARARNN_BF16 ? 2 : 4;
+    if (px_dtype != PARARNN_F32 && px_dtype != PARARNN_BF16) return 0;
+    if (!hp::layout(cell, B, T, D, K, rows_per_slice, esz, l)) return 0;
+    return l.total;
+}
+
+extern "C" pararnn_status pararnn_newton_forward_host(pararnn_cell cell, int64_t B, int64_t T, int64_t D,
+                                                      pararnn_dtype px_dtype, const void* preacts_host,
+                                                      const float* diag_w, const float* h0, int K, float* H_host,
+                                                      void* workspace, size_t ws_bytes, int64_t rows_per_slice,
+                                                      void* stream) {
+    if (px_dtype != PARARNN_F32 && px_dtype != PARARNN_BF16)
+        return hp::fail(PARARNN_EINVAL, "pararnn_newton_forward_host: unknown pre-activation dtype");
+    const size_t esz = px_dtype == PARARNN_BF16 ? 2 : 4;
+    hp::Layout l;
+    if (!hp::layout(cell, B, T, D, K, rows_per_slice, esz, l))
+        return hp::fail(PARARNN_EINVAL, "pararnn_newton_forward_host: bad cell, sizes, K or rows_per_slice");
+    if (!workspace || ws_bytes < l.total || !pointer_on_device(workspace) ||
+        (reinterpret_cast<uintptr_t>(workspace) & 255))
+        return hp::fail(PARARNN_EINVAL, "pararnn_newton_forward_host: workspace missing, small or not 256-byte "
+                                        "aligned device memory (see pararnn_newton_forward_host_workspace_bytes)");
+    cudaStream_t user = static_cast<cudaStream_t>(stream);
+    unsigned char* ws = static_cast<unsigned char*>(workspace);
+    cudaError_t e = cudaMemsetAsync(ws, 0, 256, user);
+    if (e != cudaSuccess) return hp::fail(PARARNN_ECUDA, "pararnn_newton_forward_host: header reset failed");
+    if (B == 0 || T == 0 || D == 0) return PARARNN_OK;
+    if (!preacts_host || !H_host)
+        return hp::fail(PARARNN_EINVAL, "pararnn_newton_forward_host: preacts_host and H_host are required");
+    const int G = pararnn_num_gates(cell), S = pararnn_state_width(cell);
+    const int64_t nslices = (B + l.rows - 1) / l.rows;
+
+    // three streams (in, solve, out) ordered after the work already on `stream`
+    cudaStream_t sin = nullptr, scomp = nullptr, sout = nullptr;
+    cudaEvent_t start = nullptr, ev_in[hp::kSlots] = {}, ev_comp[hp::kSlots] = {}, ev_out[hp::kSlots] = {};
+    auto cleanup = [&]() {
+        for (int k = 0; k < hp::kSlots; ++k) {
+            if (ev_in[k]) cudaEventDestroy(ev_in[k]);
+            if (ev_comp[k]) cudaEventDestroy(ev_comp[k]);
+            if (ev_out[k]) cudaEventDestroy(ev_out[k]);
+        }
+        if (start) cudaEventDestroy(start);
+        if (sin) cudaStreamDestroy(sin);
+        if (scomp) cudaStreamDestroy(scomp);
+        if (sout) cudaStreamDestroy(sout);
+    };
+    e = cudaStreamCreateWithFlags(&sin, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&scomp, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&sout, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&start, cudaEventDisableTiming);
+    for (int k = 0; k < hp::kSlots && e == cudaSuccess; ++k) {
+        e = cudaEventCreateWithFlags(&ev_in[k], cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev_comp[k], cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev_out[k], cudaEventDisableTiming);
+    }
+    if (e == cudaSuccess) e = cudaEventRecord(start, user);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(sin, start, 0);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(scomp, start, 0);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(sout, start, 0);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        cleanup();
+        return hp::fail(PARARNN_ECUDA, "pararnn_newton_forward_host: stream or event setup failed");
+    }
+
+    const size_t row_px = (size_t)T * G * D * esz, row_h = (size_t)T * S * D * sizeof(float);
+    pararnn_status st = PARARNN_OK;
+    for (int64_t i = 0; i < nslices && st == PARARNN_OK; ++i) {
+        const int k = (int)(i % hp::kSlots);
+        const int64_t b0 = i * l.rows, nb = (b0 + l.rows <= B) ? l.rows : B - b0;
+        unsigned char* slot = ws + 256 + (size_t)k * l.slot_bytes;
+        void* fw = slot;
+        void* px_dev = slot + hp::align256(l.fw_bytes);
+        float* h_dev = reinterpret_cast<float*>(slot + hp::align256(l.fw_bytes) + l.px_bytes);
+        // in: the slot's pre-activations are free once the solve of slice i - kSlots is done
+        if (i >= hp::kSlots) e = cudaStreamWaitEvent(sin, ev_comp[k], 0);
+        if (e == cudaSuccess)
+            e = cudaMemcpyAsync(px_dev, static_cast<const unsigned char*>(preacts_host) + (size_t)b0 * row_px,
+                                (size_t)nb * row_px, cudaMemcpyDefault, sin);
+        if (e == cudaSuccess) e = cudaEventRecord(ev_in[k], sin);
+        // solve: after the copy in, and after slice i - kSlots has left the slot's H
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(scomp, ev_in[k], 0);
+        if (e == cudaSuccess && i >= hp::kSlots) e = cudaStreamWaitEvent(scomp, ev_out[k], 0);
+        if (e != cudaSuccess) break;
+        st = pararnn_newton_forward(cell, nb, T, D, px_dtype, px_dev, diag_w,
+                                    h0 ? h0 + (size_t)b0 * S * D : nullptr, K, h_dev, fw, l.fw_bytes, nullptr,
+                                    scomp);
+        if (st != PARARNN_OK) break;
+        hp::fold_status<<<1, 32, 0, scomp>>>(reinterpret_cast<unsigned*>(ws), reinterpret_cast<unsigned*>(fw));
+        e = cudaGetLastError();
+        if (e == cudaSuccess) e = cudaEventRecord(ev_comp[k], scomp);
+        // out
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(sout, ev_comp[k], 0);
+        if (e == cudaSuccess)
+            e = cudaMemcpyAsync(reinterpret_cast<unsigned char*>(H_host) + (size_t)b0 * row_h, h_dev,
+                                (size_t)nb * row_h, cudaMemcpyDefault, sout);
+        if (e == cudaSuccess) e = cudaEventRecord(ev_out[k], sout);
+        if (e != cudaSuccess) break;
+    }
+    // `stream` continues after all three
+    cudaEvent_t done[3] = {ev_in[0], ev_comp[0], ev_out[0]};
+    cudaStream_t ss[3] = {sin, scomp, sout};
+    for (int j = 0; j < 3 && e == cudaSuccess; ++j) {
+        e = cudaEventRecord(done[j], ss[j]);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(user, done[j], 0);
+    }
+    cleanup();
+    if (st != PARARNN_OK) return st;  // pararnn_newton_forward set the message
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return hp::fail(PARARNN_ECUDA, "pararnn_newton_forward_host: copy or launch failed");
+    }
+    return PARARNN_OK;
+}
