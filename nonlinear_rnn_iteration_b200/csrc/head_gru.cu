@@ -355,17 +355,16 @@ __global__ void __launch_bounds__(kThreads, 2) head_chunk_kernel(const Params pr
 
 // ---- A on the fifth-generation tensor cores (head width 64) -------------
 // The chunk work of head_chunk_kernel, with the product P <- A_t P issued as
-// tcgen05.mma (kind::tf32, M = N = 64, K = 8 per instruction) by one thread
-// per chain: operands in shared memory, the accumulator in tensor memory.
-// A block runs two chains, the same chunk of two (batch row, head)
-// sequences, 256 threads each for the Jacobian rows; a second sequence
-// that does not exist (odd B * n_heads) repeats the first and writes
-// nothing.  The head/remainder split is kept (x = x_hi + x_lo, a_lo b_hi +
-// a_hi b_lo + a_hi b_hi accumulated in float32 in tensor memory): the head
-// is rounded to TF32 with cvt.rna, the remainder stored as float (its low
-// bits are below float32 rounding of the product).
+// tcgen05.mma (kind::tf32, M = N = 64, K = 8 per instruction) by one thread:
+// operands in shared memory, the accumulator in tensor memory.  One chunk
+// per block, two blocks per SM: the blocks run unsynchronised, so one's
+// tensor-core work overlaps the other's tensor-memory epilogue and barrier.
+// The head/remainder split is kept (x = x_hi + x_lo, a_lo b_hi + a_hi b_lo +
+// a_hi b_hi accumulated in float32 in tensor memory): the head is rounded to
+// TF32 with cvt.rna, the remainder stored as float (its low bits are below
+// float32 rounding of the product).
 //
-// Operand layouts (no swizzle; 16-byte "core matrices" of 8 rows):
+// Operand layouts (no swizzle; "core matrices" of 8 rows of 16 bytes):
 //   A_t, K-major: element (i, m) at float (m / 4) * 256 + (i / 8) * 32 +
 //     (i % 8) * 4 + m % 4, i.e. 8-row groups 128 bytes apart (stride byte
 //     offset) and 4-column K chunks 1024 bytes apart (leading byte offset);
@@ -376,37 +375,32 @@ __global__ void __launch_bounds__(kThreads, 2) head_chunk_kernel(const Params pr
 // stores: a warp's Jacobian rows fill whole 128-byte lines, and each eight
 // threads of the epilogue write eight consecutive 16-byte core rows.
 //
-// The accumulator of chain e sits in tensor-memory columns 64e .. 64e+63;
-// with M = 64, row r of the product is lane 32 (r / 16) + r % 16.  Warp w
-// reads lanes 32 (w % 4) .. +15 of columns 16 (w / 4) .. +15 of both chains
-// with one 16x32bx2 load: threads 0-15 get chain 0, threads 16-31 chain 1.
+// With M = 64, row r of the accumulator is tensor-memory lane
+// 32 (r / 16) + r % 16.  Warp w reads lanes 32 (w % 4) .. +15 of columns
+// 32 (w / 4) .. +31 with one 16x32bx2 load: threads 0-15 get the first 16
+// columns, threads 16-31 the next 16.
 //
 // One block barrier per step, as in head_chunk_kernel: after it the issuing
-// threads start the product of step t; all threads form the Jacobian rows of
+// thread starts the product of step t; all threads form the Jacobian rows of
 // step t+1 meanwhile, then wait for the product (mbarrier signalled by
 // tcgen05.commit), move it from tensor memory into the P operand, fence the
 // generic-proxy writes for the tensor cores, and meet at the next barrier.
 namespace tc {
 
 constexpr int kD = 64;
-constexpr int kBlock = 2 * kThreads;
-constexpr uint32_t kTmemCols = 128;
+constexpr uint32_t kTmemCols = 64;
 constexpr uint64_t kWaitNs = 1000000000ull;  // 1 s: far beyond a 64-step product chain
 
-struct Chain {
+struct Smem {
     float Ahi[2][kD * kD];  // A_t, K-major, two steps in turn
     float Alo[2][kD * kD];
     float Phi[kD * kD];     // running product, MN-major
     float Plo[kD * kD];
-};
-
-struct Smem {
-    Chain ch[2];
-    float sv[2][2][kD];  // [chain][step parity] h^(k) rows, permuted (vpos)
-    float dv[2][2][kD];  // [chain][step parity] delta rows, permuted
-    uint64_t bar[2];     // product of chain e done
-    uint32_t tmem;       // tensor-memory base address from tcgen05.alloc
-    int abort;           // a wait ran out: stop issuing, keep the barrier count
+    float sv[2][kD];        // h^(k) rows, permuted (vpos), two steps in turn
+    float dv[2][kD];        // delta rows, permuted, two steps in turn
+    uint64_t bar;           // the product of this step is done
+    uint32_t tmem;          // tensor-memory base address from tcgen05.alloc
+    int abort;              // a wait ran out: stop issuing, keep the barrier count
 };
 
 __device__ __forceinline__ int a_idx(int i, int m) { return (m >> 2) * 256 + (i >> 3) * 32 + (i & 7) * 4 + (m & 3); }
@@ -447,12 +441,12 @@ __device__ __forceinline__ void sync_block() {
     fence_after();
 }
 
-// 16 lanes x 16 columns twice (the second half 64 columns on), and the
+// 16 lanes x 16 columns twice (the second half 16 columns on), and the
 // wait for the load in the same statement so no use can move above it
 __device__ __forceinline__ void load_acc(uint32_t taddr, float (&v)[16]) {
     uint32_t r[16];
     asm volatile(
-        "tcgen05.ld.sync.aligned.16x32bx2.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16], 64;\n\t"
+        "tcgen05.ld.sync.aligned.16x32bx2.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16], 16;\n\t"
         "tcgen05.wait::ld.sync.aligned;"
         : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
           "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
@@ -471,19 +465,16 @@ __device__ __forceinline__ float tf32_head(float x) {
 }  // namespace tc
 
 template <typename PxT>
-__global__ void __launch_bounds__(tc::kBlock, 1) head_chunk_tc_kernel(const Params pr) {
+__global__ void __launch_bounds__(kThreads, 2) head_chunk_tc_kernel(const Params pr) {
     using Gm = Geo<tc::kD>;
     constexpr int TPR = Gm::TPR, SEG = Gm::SEG, DH = tc::kD;
     extern __shared__ __align__(16) unsigned char smem_raw[];
     auto& sm = *reinterpret_cast<tc::Smem*>(smem_raw);
     volatile int& abort_flag = sm.abort;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int c = tid / kThreads, ct = tid % kThreads, i = ct / TPR, qt = ct % TPR;
-    const int64_t nSeq = pr.B * pr.nh;
-    const int64_t pair = blockIdx.x / pr.nChunks;
-    const int chunk = (int)(blockIdx.x - pair * pr.nChunks);
-    // the sequence of this thread's chain; a missing second one repeats the first
-    const int64_t seq = 2 * pair + c < nSeq ? 2 * pair + c : 2 * pair;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, i = tid / TPR, qt = tid % TPR;
+    const int64_t task = blockIdx.x;
+    const int64_t seq = task / pr.nChunks;
+    const int chunk = (int)(task - seq * pr.nChunks);
     const int64_t b = seq / pr.nh;
     const int h = (int)(seq - b * pr.nh);
     const int64_t t0 = (int64_t)chunk * kChunk;
@@ -496,8 +487,7 @@ __global__ void __launch_bounds__(tc::kBlock, 1) head_chunk_tc_kernel(const Para
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
     if (tid == 0) {
-        mbar_init(&sm.bar[0], 1);
-        mbar_init(&sm.bar[1], 1);
+        mbar_init(&sm.bar, 1);
         abort_flag = 0;
         mbar_fence_init();
     }
@@ -505,14 +495,14 @@ __global__ void __launch_bounds__(tc::kBlock, 1) head_chunk_tc_kernel(const Para
     U.load(pr.U, pr.nh, h, i, qt);
     const float s_before = iterate_before<DH, PxT>(pr, b, h, i, t0);
     if (qt == 0) {
-        sm.sv[c][0][Gm::vpos(i)] = s_before;
-        sm.dv[c][0][Gm::vpos(i)] = 0.0f;
+        sm.sv[0][Gm::vpos(i)] = s_before;
+        sm.dv[0][Gm::vpos(i)] = 0.0f;
     }
     // P = I
-    for (int idx = ct; idx < DH * DH; idx += kThreads) {
+    for (int idx = tid; idx < DH * DH; idx += kThreads) {
         const int k = idx / DH, n = idx % DH;
-        sm.ch[c].Phi[tc::p_idx(k, n)] = k == n ? 1.0f : 0.0f;
-        sm.ch[c].Plo[tc::p_idx(k, n)] = 0.0f;
+        sm.Phi[tc::p_idx(k, n)] = k == n ? 1.0f : 0.0f;
+        sm.Plo[tc::p_idx(k, n)] = 0.0f;
     }
     float rmax = 0.0f;
 
@@ -522,7 +512,7 @@ __global__ void __launch_bounds__(tc::kBlock, 1) head_chunk_tc_kernel(const Para
         float uz = 0.0f, ur = 0.0f, uc = 0.0f;
 #pragma unroll
         for (int s = 0; s < SEG; ++s) {
-            const float x = sm.sv[c][p][qt * SEG + s];
+            const float x = sm.sv[p][qt * SEG + s];
             uz = __fmaf_rn(U.z[s], x, uz);
             ur = __fmaf_rn(U.r[s], x, ur);
             uc = __fmaf_rn(U.c[s], x, uc);
@@ -530,11 +520,11 @@ __global__ void __launch_bounds__(tc::kBlock, 1) head_chunk_tc_kernel(const Para
         uz = row_sum<DH>(uz);
         ur = row_sum<DH>(ur);
         uc = row_sum<DH>(uc);
-        const float sp = sm.sv[c][p][Gm::vpos(i)];
+        const float sp = sm.sv[p][Gm::vpos(i)];
         const RowLin L = row_linearise(in, sp, uz, ur, uc);
         if (qt == 0) rmax = nanmax_f(rmax, fabsf(L.F));
-        float* ahi = sm.ch[c].Ahi[p];
-        float* alo = sm.ch[c].Alo[p];
+        float* ahi = sm.Ahi[p];
+        float* alo = sm.Alo[p];
         float dp = 0.0f;
 #pragma unroll
         for (int s = 0; s < SEG; ++s) {
@@ -545,12 +535,12 @@ __global__ void __launch_bounds__(tc::kBlock, 1) head_chunk_tc_kernel(const Para
             const float hi = tc::tf32_head(a);
             ahi[tc::a_idx(i, m)] = hi;
             alo[tc::a_idx(i, m)] = a - hi;
-            dp = __fmaf_rn(a, sm.dv[c][p][qt * SEG + s], dp);
+            dp = __fmaf_rn(a, sm.dv[p][qt * SEG + s], dp);
         }
         dp = row_sum<DH>(dp);
         if (qt == 0) {
-            sm.dv[c][p ^ 1][Gm::vpos(i)] = dp - L.F;
-            sm.sv[c][p ^ 1][Gm::vpos(i)] = in.s;
+            sm.dv[p ^ 1][Gm::vpos(i)] = dp - L.F;
+            sm.sv[p ^ 1][Gm::vpos(i)] = in.s;
         }
     };
 
@@ -566,51 +556,46 @@ __global__ void __launch_bounds__(tc::kBlock, 1) head_chunk_tc_kernel(const Para
     }
     tc::sync_block();
 
-    // epilogue geometry: this warp's lanes and columns of both accumulators
-    const int eq = warp & 3, ej = warp >> 2, ee = lane >> 4;
-    const int ek = 16 * eq + (lane & 15);  // product row held by this thread
-    const uint32_t taddr = tmem + ((uint32_t)(32 * eq) << 16) + (uint32_t)(16 * ej);
-    const int64_t eseq = 2 * pair + ee;
-    const bool evalid = eseq < nSeq;
-    const int64_t etask = (evalid ? eseq : 0) * pr.nChunks + chunk;
+    // epilogue geometry: this thread's row and columns of the accumulator
+    const int eq = warp & 3;
+    const int ek = 16 * eq + (lane & 15);              // product row
+    const int en = 32 * (warp >> 2) + 16 * (lane >> 4);  // first of 16 columns
+    const uint32_t taddr = tmem + ((uint32_t)(32 * eq) << 16) + (uint32_t)(32 * (warp >> 2));
 
     int p = 0;
     for (int64_t t = t0; t < t1; ++t) {
         const uint32_t par = (uint32_t)((t - t0) & 1);
-        if (ct == 0 && !abort_flag) {
-            // P_t = A_t P_{t-1} into columns 64c .. 64c+63
-            const uint32_t ah = smem_u32(sm.ch[c].Ahi[p]), al = smem_u32(sm.ch[c].Alo[p]);
-            const uint32_t ph = smem_u32(sm.ch[c].Phi), pl = smem_u32(sm.ch[c].Plo);
-            const uint32_t d = tmem + (uint32_t)(64 * c);
+        if (tid == 0 && !abort_flag) {
+            // P_t = A_t P_{t-1}
+            const uint32_t ah = smem_u32(sm.Ahi[p]), al = smem_u32(sm.Alo[p]);
+            const uint32_t ph = smem_u32(sm.Phi), pl = smem_u32(sm.Plo);
 #pragma unroll
             for (int ks = 0; ks < DH / 8; ++ks) {
                 const uint32_t ko = (uint32_t)ks * 2048u;
                 const uint64_t dah = tc::sdesc(ah + ko, 1024, 128), dal = tc::sdesc(al + ko, 1024, 128);
                 const uint64_t dph = tc::sdesc(ph + ko, 2048, 128), dpl = tc::sdesc(pl + ko, 2048, 128);
-                tc::mma(d, dal, dph, ks > 0 ? 1u : 0u);
-                tc::mma(d, dah, dpl, 1u);
-                tc::mma(d, dah, dph, 1u);
+                tc::mma(tmem, dal, dph, ks > 0 ? 1u : 0u);
+                tc::mma(tmem, dah, dpl, 1u);
+                tc::mma(tmem, dah, dph, 1u);
             }
-            tc::commit(&sm.bar[c]);
+            tc::commit(&sm.bar);
         }
         if (t + 1 < t1) {
             const StepIn in = nxt;
             if (t + 2 < t1) nxt = load_step<DH, PxT>(pr, b, h, i, t + 2);
             row_step(in, p ^ 1);
         }
-        // wait for both products (bounded), then move them out of tensor memory
+        // wait for the product (bounded), then move it out of tensor memory
         if (!abort_flag) {
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                uint64_t start = 0;
-                while (!mbar_try_wait(&sm.bar[e], par)) {
-                    const uint64_t now = globaltimer_ns();
-                    if (start == 0) start = now | 1;
-                    else if (now - start > tc::kWaitNs) {
-                        if (lane == 0) atomicOr(pr.status, kStatusTimeout);
-                        abort_flag = 1;
-                        break;
-                    }
+            uint64_t start = 0;
+            while (!mbar_try_wait(&sm.bar, par)) {
+                const uint64_t now = globaltimer_ns();
+                if (start == 0) {
+                    start = now | 1;
+                } else if (now - start > tc::kWaitNs) {
+                    if (lane == 0) atomicOr(pr.status, kStatusTimeout);
+                    abort_flag = 1;
+                    break;
                 }
             }
         }
@@ -618,8 +603,6 @@ __global__ void __launch_bounds__(tc::kBlock, 1) head_chunk_tc_kernel(const Para
         float v[16];
         tc::load_acc(taddr, v);
         if (t + 1 < t1) {
-            float* phi = sm.ch[ee].Phi;
-            float* plo = sm.ch[ee].Plo;
 #pragma unroll
             for (int g = 0; g < 4; ++g) {
                 float4 hv, lv;
@@ -631,12 +614,12 @@ __global__ void __launch_bounds__(tc::kBlock, 1) head_chunk_tc_kernel(const Para
                 lv.y = v[4 * g + 1] - hv.y;
                 lv.z = v[4 * g + 2] - hv.z;
                 lv.w = v[4 * g + 3] - hv.w;
-                const int o = tc::p_idx(ek, 16 * ej + 4 * g);
-                *reinterpret_cast<float4*>(phi + o) = hv;
-                *reinterpret_cast<float4*>(plo + o) = lv;
+                const int o = tc::p_idx(ek, en + 4 * g);
+                *reinterpret_cast<float4*>(sm.Phi + o) = hv;
+                *reinterpret_cast<float4*>(sm.Plo + o) = lv;
             }
-        } else if (evalid) {
-            float* Pout = pr.P + etask * DH * DH + (int64_t)ek * DH + 16 * ej;
+        } else {
+            float* Pout = pr.P + task * DH * DH + (int64_t)ek * DH + en;
 #pragma unroll
             for (int g = 0; g < 4; ++g)
                 *reinterpret_cast<float4*>(Pout + 4 * g) = make_float4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
@@ -646,7 +629,7 @@ __global__ void __launch_bounds__(tc::kBlock, 1) head_chunk_tc_kernel(const Para
     }
     if (pr.resid) block_max_resid(rmax, pr.resid + pr.k);
     // delta at the chunk's last step: written to dv[(t1 - t0) & 1]
-    if (qt == 0 && 2 * pair + c < nSeq) pr.q[(seq * pr.nChunks + chunk) * DH + i] = sm.dv[c][p][Gm::vpos(i)];
+    if (qt == 0) pr.q[task * DH + i] = sm.dv[p][Gm::vpos(i)];
     if (warp == 0)
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(tc::kTmemCols)
                      : "memory");
@@ -1065,15 +1048,14 @@ cudaError_t set_smem(Kern k, size_t bytes) {
 
 template <int DH, typename PxT>
 cudaError_t launch_all(const Plan& pl, Params pr, float* H_out, float* Hbuf, int K, cudaStream_t st) {
-    // head width 64: the products on tcgen05, two sequences per block;
-    // narrower heads (M < 64 does not exist for tcgen05.mma) on mma.sync
+    // head width 64: the products on tcgen05; narrower heads (tcgen05.mma
+    // has no M below 64) on mma.sync
     constexpr bool kTc = DH == tc::kD;
     const size_t smemA = kTc ? sizeof(tc::Smem) : sizeof(SmemA<DH>), smemR = sizeof(SmemA<DH>);
     cudaError_t e = kTc ? set_smem(head_chunk_tc_kernel<PxT>, smemA) : set_smem(head_chunk_kernel<DH, PxT, false>, smemA);
     if (e == cudaSuccess) e = set_smem(head_chunk_kernel<DH, PxT, true>, smemR);
     if (e != cudaSuccess) return e;
     const unsigned ntask = (unsigned)(pl.nSeq * pl.nChunks);
-    const unsigned npair_blocks = (unsigned)((pl.nSeq + 1) / 2 * pl.nChunks);
     for (int k = 0; k < K; ++k) {
         // iterate k lives in X_k, X_j = H_out when K - j is even, else the
         // workspace buffer, so that h^(K) lands in H_out
@@ -1081,7 +1063,7 @@ cudaError_t launch_all(const Plan& pl, Params pr, float* H_out, float* Hbuf, int
         pr.Hold = k == 0 ? nullptr : (((K - k) % 2 == 0) ? H_out : Hbuf);
         pr.Hnew = ((K - (k + 1)) % 2 == 0) ? H_out : Hbuf;
         if constexpr (kTc)
-            head_chunk_tc_kernel<PxT><<<npair_blocks, tc::kBlock, smemA, st>>>(pr);
+            head_chunk_tc_kernel<PxT><<<ntask, kThreads, smemA, st>>>(pr);
         else
             head_chunk_kernel<DH, PxT, false><<<ntask, kThreads, smemA, st>>>(pr);
         head_carry_kernel<DH><<<(unsigned)pl.nSeq, 64, 0, st>>>(pr);
