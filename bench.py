@@ -180,7 +180,7 @@ def head_line(w, ms, bwd_ms, status):
     return {"ms_per_step": round(ms, 4), "elem_per_s": w.elements / (ms / 1e3), "K": w.K,
             "n_heads": w.n_heads, "d": w.d, "status": status, "bwd_ms": round(bwd_ms, 4),
             "bwd_elem_per_s": w.elements / (bwd_ms / 1e3),
-            "roofline": {"bound": "tensor", "kernel": "head_chunk_kernel (Jacobian products)",
+            "roofline": {"bound": "tensor", "kernel": "head_chunk_tc_kernel (Jacobian products, tcgen05 TF32)",
                          "achieved_useful": round(useful / (ms / 1e3) / 1e12, 2),
                          "achieved_issued": round(3 * useful / (ms / 1e3) / 1e12, 2),
                          "peak": round(tf32_peak, 1), "peak_source": peaks["source"] + " (bf16 x TF32 ratio)",

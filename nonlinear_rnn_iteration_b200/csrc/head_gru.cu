@@ -949,6 +949,221 @@ __global__ void __launch_bounds__(kThreads, 2) head_bwd_kernel(const Params pr) 
     }
 }
 
+// ---- backward A on the fifth-generation tensor cores (head width 64) ------
+// head_bwd_kernel's product Q <- A_t^T Q (t from t1-1 down to t0) as
+// tcgen05.mma, organised as head_chunk_tc_kernel.  The left operand A_t^T
+// is stored MN-major (element (m, i) of A_t^T = A_t[i][m] at float
+// (i / 8) * 512 + (m / 4) * 32 + (i % 8) * 4 + m % 4, the running product's
+// layout), so each warp's Jacobian rows again fill whole 128-byte lines;
+// mu_t = A_t^T lambda is read back from the same operand as head + remainder
+// (their sum is A_t[i][m] exactly).
+namespace tc {
+
+struct SmemB {
+    float Ahi[2][kD * kD];  // A_t^T, MN-major, two steps in turn
+    float Alo[2][kD * kD];
+    float Phi[kD * kD];     // running product, MN-major
+    float Plo[kD * kD];
+    float sv[2][kD];        // h_{t-1} rows for the row work (permuted)
+    float gv[2][kD];        // g_t rows (permuted)
+    float mv[2][kD];        // mu rows (permuted)
+    uint64_t bar;
+    uint32_t tmem;
+    int abort;
+};
+
+// instruction descriptor of the backward: as kIdesc, with A MN-major too
+constexpr uint32_t kIdescT = kIdesc | (1u << 15);
+
+__device__ __forceinline__ void mma_t(uint32_t d, uint64_t a, uint64_t b, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d), "l"(a), "l"(b), "r"(kIdescT), "r"(accumulate));
+}
+
+}  // namespace tc
+
+template <typename PxT>
+__global__ void __launch_bounds__(kThreads, 2) head_bwd_tc_kernel(const Params pr) {
+    using Gm = Geo<tc::kD>;
+    constexpr int TPR = Gm::TPR, SEG = Gm::SEG, DH = tc::kD;
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    auto& sm = *reinterpret_cast<tc::SmemB*>(smem_raw);
+    volatile int& abort_flag = sm.abort;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, i = tid / TPR, qt = tid % TPR;
+    const int64_t task = blockIdx.x;
+    const int64_t seq = task / pr.nChunks;
+    const int chunk = (int)(task - seq * pr.nChunks);
+    const int64_t b = seq / pr.nh;
+    const int h = (int)(seq - b * pr.nh);
+    const int64_t t0 = (int64_t)chunk * kChunk;
+    const int64_t t1 = t0 + kChunk < pr.T ? t0 + kChunk : pr.T;
+
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&sm.tmem)),
+                     "r"(tc::kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    if (tid == 0) {
+        mbar_init(&sm.bar, 1);
+        abort_flag = 0;
+        mbar_fence_init();
+    }
+    RowU<DH> U;
+    U.load(pr.U, pr.nh, h, i, qt);
+    if (qt == 0) {
+        sm.sv[0][Gm::vpos(i)] = state_before<DH>(pr, b, h, i, t1 - 1);
+        sm.mv[1][Gm::vpos(i)] = 0.0f;  // mu_{t1} for the chunk's own product
+    }
+    for (int idx = tid; idx < DH * DH; idx += kThreads) {
+        const int k = idx / DH, n = idx % DH;
+        sm.Phi[tc::p_idx(k, n)] = k == n ? 1.0f : 0.0f;
+        sm.Plo[tc::p_idx(k, n)] = 0.0f;
+    }
+
+    // the row work of step t, parity p: the gates at (h_{t-1}, x_t), row i of
+    // A_t as column i of A_t^T (split) into A[p], g_t into gv[p], and h_{t-2}
+    // into sv[p ^ 1] for the next (earlier) step
+    auto row_step = [&](const BStepIn& in, int p) {
+        float uz = 0.0f, ur = 0.0f, uc = 0.0f;
+#pragma unroll
+        for (int s = 0; s < SEG; ++s) {
+            const float x = sm.sv[p][qt * SEG + s];
+            uz = __fmaf_rn(U.z[s], x, uz);
+            ur = __fmaf_rn(U.r[s], x, ur);
+            uc = __fmaf_rn(U.c[s], x, uc);
+        }
+        uz = row_sum<DH>(uz);
+        ur = row_sum<DH>(ur);
+        uc = row_sum<DH>(uc);
+        const float sp = sm.sv[p][Gm::vpos(i)];
+        const float z = sigmoid_f(in.pz + uz);
+        const float r = sigmoid_f(in.pr + ur);
+        const float c = tanh_f(__fmaf_rn(r, uc, in.pc));
+        const float zc = z * __fmaf_rn(-c, c, 1.0f);
+        const float dz = 1.0f - z, al = (c - sp) * (z - z * z), be = zc * uc * (r - r * r), ga = zc * r;
+        float* ahi = sm.Ahi[p];
+        float* alo = sm.Alo[p];
+#pragma unroll
+        for (int s = 0; s < SEG; ++s) {
+            const int m = qt + TPR * s;
+            float a = __fmaf_rn(al, U.z[s], (m == i) ? dz : 0.0f);
+            a = __fmaf_rn(be, U.r[s], a);
+            a = __fmaf_rn(ga, U.c[s], a);
+            const float hi = tc::tf32_head(a);
+            ahi[tc::p_idx(i, m)] = hi;  // (A_t^T)[m][i]: K index i, M index m
+            alo[tc::p_idx(i, m)] = a - hi;
+        }
+        if (qt == 0) {
+            const int vi = Gm::vpos(i);
+            sm.gv[p][vi] = in.g;
+            sm.sv[p ^ 1][vi] = in.s2;
+        }
+    };
+
+    BStepIn nxt = load_bstep<DH, PxT>(pr, b, h, i, t1 - 1);
+    tc::fence_before();
+    __syncthreads();
+    tc::fence_after();
+    const uint32_t tmem = sm.tmem;
+    {
+        const BStepIn in = nxt;
+        if (t1 - 2 >= t0) nxt = load_bstep<DH, PxT>(pr, b, h, i, t1 - 2);
+        row_step(in, 0);
+    }
+    tc::sync_block();
+
+    const int eq = warp & 3;
+    const int ek = 16 * eq + (lane & 15);
+    const int en = 32 * (warp >> 2) + 16 * (lane >> 4);
+    const uint32_t taddr = tmem + ((uint32_t)(32 * eq) << 16) + (uint32_t)(32 * (warp >> 2));
+
+    int p = 0;
+    for (int64_t t = t1 - 1; t >= t0; --t) {
+        const uint32_t par = (uint32_t)((t1 - 1 - t) & 1);
+        if (tid == 0 && !abort_flag) {
+            // Q_t = A_t^T Q_{t+1}
+            const uint32_t ah = smem_u32(sm.Ahi[p]), al = smem_u32(sm.Alo[p]);
+            const uint32_t ph = smem_u32(sm.Phi), pl = smem_u32(sm.Plo);
+#pragma unroll
+            for (int ks = 0; ks < DH / 8; ++ks) {
+                const uint32_t ko = (uint32_t)ks * 2048u;
+                const uint64_t dah = tc::sdesc(ah + ko, 2048, 128), dal = tc::sdesc(al + ko, 2048, 128);
+                const uint64_t dph = tc::sdesc(ph + ko, 2048, 128), dpl = tc::sdesc(pl + ko, 2048, 128);
+                tc::mma_t(tmem, dal, dph, ks > 0 ? 1u : 0u);
+                tc::mma_t(tmem, dah, dpl, 1u);
+                tc::mma_t(tmem, dah, dph, 1u);
+            }
+            tc::commit(&sm.bar);
+        }
+        {
+            // mu_t[m] = sum_i A_t[i][m] (g_t[i] + mu_{t+1}[i]) for thread (m = i, qt)
+            float acc = 0.0f;
+#pragma unroll
+            for (int s = 0; s < SEG; ++s) {
+                const int k = qt + TPR * s;
+                const float lam = sm.gv[p][qt * SEG + s] + sm.mv[p ^ 1][qt * SEG + s];
+                const int o = tc::p_idx(k, i);
+                acc = __fmaf_rn(sm.Ahi[p][o] + sm.Alo[p][o], lam, acc);
+            }
+            acc = row_sum<DH>(acc);
+            if (qt == 0) sm.mv[p][Gm::vpos(i)] = acc;
+        }
+        if (t - 1 >= t0) {
+            const BStepIn in = nxt;
+            if (t - 2 >= t0) nxt = load_bstep<DH, PxT>(pr, b, h, i, t - 2);
+            row_step(in, p ^ 1);
+        }
+        if (!abort_flag) {
+            uint64_t start = 0;
+            while (!mbar_try_wait(&sm.bar, par)) {
+                const uint64_t now = globaltimer_ns();
+                if (start == 0) {
+                    start = now | 1;
+                } else if (now - start > tc::kWaitNs) {
+                    if (lane == 0) atomicOr(pr.status, kStatusTimeout);
+                    abort_flag = 1;
+                    break;
+                }
+            }
+        }
+        tc::fence_after();
+        float v[16];
+        tc::load_acc(taddr, v);
+        if (t - 1 >= t0) {
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+                float4 hv, lv;
+                hv.x = tc::tf32_head(v[4 * g + 0]);
+                hv.y = tc::tf32_head(v[4 * g + 1]);
+                hv.z = tc::tf32_head(v[4 * g + 2]);
+                hv.w = tc::tf32_head(v[4 * g + 3]);
+                lv.x = v[4 * g + 0] - hv.x;
+                lv.y = v[4 * g + 1] - hv.y;
+                lv.z = v[4 * g + 2] - hv.z;
+                lv.w = v[4 * g + 3] - hv.w;
+                const int o = tc::p_idx(ek, en + 4 * g);
+                *reinterpret_cast<float4*>(sm.Phi + o) = hv;
+                *reinterpret_cast<float4*>(sm.Plo + o) = lv;
+            }
+        } else {
+            float* Pout = pr.P + task * DH * DH + (int64_t)ek * DH + en;
+#pragma unroll
+            for (int g = 0; g < 4; ++g)
+                *reinterpret_cast<float4*>(Pout + 4 * g) = make_float4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
+        }
+        tc::sync_block();
+        p ^= 1;
+    }
+    // mu at the chunk's first step: written to mv[p ^ 1] by the last iteration
+    if (qt == 0) pr.q[task * DH + i] = sm.mv[p ^ 1][Gm::vpos(i)];
+    if (warp == 0)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(tc::kTmemCols)
+                     : "memory");
+}
+
 // ---- dL/dU: outer products summed in a fixed order -------------------------
 // part[split][g][h] = sum over the split's rows (b, t) of e_g[b,t] h_{t-1}^T
 // (e_z = dL/dp_z, e_r = dL/dp_r, e_c = lambda * gamma), rows in increasing
@@ -1110,12 +1325,17 @@ bool make_bplan(int64_t B, int64_t T, int64_t D, int nh, BPlan& pl) {
 
 template <int DH, typename PxT>
 cudaError_t launch_bwd(const BPlan& pl, const Params& pr, float* dU, cudaStream_t st) {
-    const size_t smem = sizeof(SmemB<DH>);
-    cudaError_t e = set_smem(head_bwd_kernel<DH, PxT, false>, smem);
+    // head width 64: the products on tcgen05, as in the forward
+    constexpr bool kTc = DH == tc::kD;
+    const size_t smem = sizeof(SmemB<DH>), smemP = kTc ? sizeof(tc::SmemB) : smem;
+    cudaError_t e = kTc ? set_smem(head_bwd_tc_kernel<PxT>, smemP) : set_smem(head_bwd_kernel<DH, PxT, false>, smemP);
     if (e == cudaSuccess) e = set_smem(head_bwd_kernel<DH, PxT, true>, smem);
     if (e != cudaSuccess) return e;
     const unsigned ntask = (unsigned)(pl.nSeq * pl.nChunks);
-    head_bwd_kernel<DH, PxT, false><<<ntask, kThreads, smem, st>>>(pr);
+    if constexpr (kTc)
+        head_bwd_tc_kernel<PxT><<<ntask, kThreads, smemP, st>>>(pr);
+    else
+        head_bwd_kernel<DH, PxT, false><<<ntask, kThreads, smemP, st>>>(pr);
     head_carry_kernel<DH, true><<<(unsigned)pl.nSeq, 64, 0, st>>>(pr);
     head_bwd_kernel<DH, PxT, true><<<ntask, kThreads, smem, st>>>(pr);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
