@@ -689,6 +689,8 @@ __global__ void __launch_bounds__(64) head_carry_kernel(const Params pr) {
 // delta_t = A_t delta_{t-1} - F_t with A_t applied as
 // diag(1-z) + diag(alpha) U_z + diag(beta) U_r + diag(gamma) U_c; one block
 // barrier per step, the vectors double-buffered as in the chunk kernel.
+constexpr int kWalkAhead = 2;
+
 template <int DH>
 struct SmemC {
     float sv[2][DH];
@@ -716,13 +718,20 @@ __global__ void __launch_bounds__(kThreads, 2) head_walk_kernel(const Params pr)
         sm.sv[0][Gm::vpos(i)] = s_before;
         sm.dv[0][Gm::vpos(i)] = pr.carry[task * DH + i];
     }
-    StepIn nxt = load_step<DH, PxT>(pr, b, h, i, t0);
+    // inputs prefetched kWalkAhead steps ahead (measured: two steps ahead
+    // beats one by about 1 %; deeper gains nothing)
+    StepIn ahead[kWalkAhead];
+#pragma unroll
+    for (int j = 0; j < kWalkAhead; ++j)
+        if (t0 + j < t1) ahead[j] = load_step<DH, PxT>(pr, b, h, i, t0 + j);
     __syncthreads();
     int par = 0;
     bool bad = false;
     for (int64_t t = t0; t < t1; ++t) {
-        const StepIn in = nxt;
-        if (t + 1 < t1) nxt = load_step<DH, PxT>(pr, b, h, i, t + 1);
+        const StepIn in = ahead[0];
+#pragma unroll
+        for (int j = 0; j + 1 < kWalkAhead; ++j) ahead[j] = ahead[j + 1];
+        if (t + kWalkAhead < t1) ahead[kWalkAhead - 1] = load_step<DH, PxT>(pr, b, h, i, t + kWalkAhead);
         float uz = 0.0f, ur = 0.0f, uc = 0.0f, vz = 0.0f, vr = 0.0f, vc = 0.0f;
 #pragma unroll
         for (int s = 0; s < SEG; ++s) {
