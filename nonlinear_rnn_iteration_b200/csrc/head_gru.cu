@@ -567,16 +567,17 @@ __global__ void __launch_bounds__(kThreads, 2) head_chunk_tc_kernel(const Params
         const uint32_t par = (uint32_t)((t - t0) & 1);
         if (tid == 0 && !abort_flag) {
             // P_t = A_t P_{t-1}
-            const uint32_t ah = smem_u32(sm.Ahi[p]), al = smem_u32(sm.Alo[p]);
-            const uint32_t ph = smem_u32(sm.Phi), pl = smem_u32(sm.Plo);
+            // K step ks starts 2048 bytes further on in every operand: 128
+            // in the descriptors' start-address field (no carry out of it)
+            const uint64_t dah = tc::sdesc(smem_u32(sm.Ahi[p]), 1024, 128);
+            const uint64_t dal = tc::sdesc(smem_u32(sm.Alo[p]), 1024, 128);
+            const uint64_t dph = tc::sdesc(smem_u32(sm.Phi), 2048, 128), dpl = tc::sdesc(smem_u32(sm.Plo), 2048, 128);
 #pragma unroll
             for (int ks = 0; ks < DH / 8; ++ks) {
-                const uint32_t ko = (uint32_t)ks * 2048u;
-                const uint64_t dah = tc::sdesc(ah + ko, 1024, 128), dal = tc::sdesc(al + ko, 1024, 128);
-                const uint64_t dph = tc::sdesc(ph + ko, 2048, 128), dpl = tc::sdesc(pl + ko, 2048, 128);
-                tc::mma(tmem, dal, dph, ks > 0 ? 1u : 0u);
-                tc::mma(tmem, dah, dpl, 1u);
-                tc::mma(tmem, dah, dph, 1u);
+                const uint64_t ko = (uint64_t)ks * 128u;
+                tc::mma(tmem, dal + ko, dph + ko, ks > 0 ? 1u : 0u);
+                tc::mma(tmem, dah + ko, dpl + ko, 1u);
+                tc::mma(tmem, dah + ko, dph + ko, 1u);
             }
             tc::commit(&sm.bar);
         }
@@ -1094,16 +1095,15 @@ __global__ void __launch_bounds__(kThreads, 2) head_bwd_tc_kernel(const Params p
         const uint32_t par = (uint32_t)((t1 - 1 - t) & 1);
         if (tid == 0 && !abort_flag) {
             // Q_t = A_t^T Q_{t+1}
-            const uint32_t ah = smem_u32(sm.Ahi[p]), al = smem_u32(sm.Alo[p]);
-            const uint32_t ph = smem_u32(sm.Phi), pl = smem_u32(sm.Plo);
+            const uint64_t dah = tc::sdesc(smem_u32(sm.Ahi[p]), 2048, 128);
+            const uint64_t dal = tc::sdesc(smem_u32(sm.Alo[p]), 2048, 128);
+            const uint64_t dph = tc::sdesc(smem_u32(sm.Phi), 2048, 128), dpl = tc::sdesc(smem_u32(sm.Plo), 2048, 128);
 #pragma unroll
             for (int ks = 0; ks < DH / 8; ++ks) {
-                const uint32_t ko = (uint32_t)ks * 2048u;
-                const uint64_t dah = tc::sdesc(ah + ko, 2048, 128), dal = tc::sdesc(al + ko, 2048, 128);
-                const uint64_t dph = tc::sdesc(ph + ko, 2048, 128), dpl = tc::sdesc(pl + ko, 2048, 128);
-                tc::mma_t(tmem, dal, dph, ks > 0 ? 1u : 0u);
-                tc::mma_t(tmem, dah, dpl, 1u);
-                tc::mma_t(tmem, dah, dph, 1u);
+                const uint64_t ko = (uint64_t)ks * 128u;  // 2048 bytes on
+                tc::mma_t(tmem, dal + ko, dph + ko, ks > 0 ? 1u : 0u);
+                tc::mma_t(tmem, dah + ko, dpl + ko, 1u);
+                tc::mma_t(tmem, dah + ko, dph + ko, 1u);
             }
             tc::commit(&sm.bar);
         }
