@@ -4,8 +4,10 @@ against the fp64 oracle, through the C ABI.
 Tolerances as for the diagonal cells (gpu_util.rel_err): H <= 1e-4; the
 residual history within 1e-4 of the largest residual; bf16 pre-activations
 against the oracle on the same bf16 values <= 1e-4.  Cases cover every
-supported head width (16, 32, 64), one and several heads, sequences that end
-inside a chunk, an initial state, K = 1..3 and K = T.
+supported head width (16, 32, 64; 64 runs the chunk products on tcgen05,
+the narrower widths on mma.sync), one and several heads, a single step,
+sequences that end inside a chunk or one step into a new one, an initial
+state, K = 1..3 and K = T.
 """
 import numpy as np
 import pytest
@@ -33,6 +35,9 @@ CASES = [  # (B, T, D, n_heads, K)
     (2, 40, 48, 3, 1),
     (1, 130, 128, 2, 3),
     (2, 64, 256, 4, 2),
+    # head width 64 (the tcgen05 products): one step, a last chunk of one step
+    (1, 1, 64, 1, 1),
+    (3, 65, 64, 1, 2),
 ]
 
 
@@ -131,6 +136,8 @@ BWD_CASES = [  # (B, T, D, n_heads, K)
     (1, 150, 96, 3, 2),
     (2, 40, 64, 2, 1),
     (1, 200, 128, 2, 3),
+    (1, 1, 64, 1, 1),
+    (3, 65, 64, 1, 2),
 ]
 
 
