@@ -83,3 +83,26 @@ def test_residual_history_falls(cell, cuda_device):
     assert r[0] > 1e-2 and r[-1] < 1e-5 * r[0]
     for k in range(1, K + 1):
         assert r[k] <= r[k - 1] * 1.01 + 1e-6
+
+
+def test_kstar_head_wise(cuda_device):
+    """The same measurement for the head-wise GRU (dense 64 x 64 Jacobian
+    blocks, the chunk products on tcgen05), with the workload's draw:
+    pre-activations ~ N(0,1), U ~ U(-1,1)/sqrt(d), h0 = 0, two heads."""
+    from nonlinear_rnn_iteration_b200 import workloads
+
+    rows = []
+    for T in (16, 64, 256, 1024):
+        x = workloads.head_host_inputs(1, T, 128, 2, 200 + T)
+        ref = oracle.head_gru_unroll(x["px"], x["U"], None)
+        pxt, Ut = torch.from_numpy(x["px"]).to(DEV), torch.from_numpy(x["U"]).to(DEV)
+        err = {k: rel_err(to_np(binding.head_gru_forward(pxt, Ut, None, K=k)), ref) for k in range(1, K_MAX + 1)}
+        kstar = next((k for k in range(1, K_MAX + 1) if err[k] <= TAU), None)
+        rows.append((T, kstar, err))
+        assert kstar is not None, "no K <= %d reaches %g at T=%d: %s" % (K_MAX, TAU, T, err)
+        assert kstar < T or T <= 16
+        if kstar < K_MAX:
+            assert err[kstar + 1] <= TAU
+    print("\nK* (rel. error vs the fp64 unroll <= %g), head-wise GRU, B=1, D=128, 2 heads of 64" % TAU)
+    for T, kstar, err in rows:
+        print("  T=%5d  K*=%2d   error at K=1,2,3,4: %s" % (T, kstar, ", ".join("%.1e" % err[k] for k in (1, 2, 3, 4))))
