@@ -43,6 +43,10 @@ namespace hg {
 constexpr int kThreads = 256;
 constexpr int kChunk = 64;  // steps per chunk
 constexpr int kMaxK = 64;
+// row factors stored per step: forward h^(k)_t, F_t, 1 - z, alpha, beta,
+// gamma; backward 1 - z, alpha, beta, z (1 - c^2), gamma
+constexpr int kNF = 6;
+constexpr int kNB = 5;
 
 struct Params {
     const void* px;     // (B,T,3,D)
@@ -53,6 +57,8 @@ struct Params {
     float* P;           // [nSeq][nChunks][d][d]
     float* q;           // [nSeq][nChunks][d]
     float* carry;       // [nSeq][nChunks][d]: delta just before each chunk
+    float* L;           // [nSeq][T][kNF or kNB][d]: each step's row factors, formed by the chunk
+                        // kernel for the Jacobian rows and read back by the walk
     float* resid;       // K+1 floats or null
     unsigned* status;   // workspace header word 0
     // backward only
@@ -152,6 +158,19 @@ __device__ __forceinline__ RowLin row_linearise(const StepIn& in, float sp, floa
     o.be = zc * uc * (r - r * r);
     o.ga = zc * r;
     return o;
+}
+
+// step t's forward row factors of row i, for the walk
+template <int DH>
+__device__ __forceinline__ void store_row_factors(const Params& pr, int64_t seq, int64_t t, int i, float s,
+                                                  const RowLin& L) {
+    float* o = pr.L + ((seq * pr.T + t) * kNF) * DH + i;
+    o[0] = s;
+    o[DH] = L.F;
+    o[2 * DH] = L.dz;
+    o[3 * DH] = L.al;
+    o[4 * DH] = L.be;
+    o[5 * DH] = L.ga;
 }
 
 // max over the block into *resid: a warp max, then one atomic per warp
@@ -287,9 +306,10 @@ __global__ void __launch_bounds__(kThreads, 2) head_chunk_kernel(const Params pr
             sm.Pm[0][idx / DH][idx % DH] = make_uint2(idx / DH == idx % DH ? __float_as_uint(1.0f) : 0u, 0u);
     float rmax = 0.0f;
 
-    // the row work of one step: row i of A_t into AT[p], and the next rows
-    // of the iterate and of delta (delta_t = A_t delta_{t-1} - F_t)
-    auto row_step = [&](const StepIn& in, int p) {
+    // the row work of step t: row i of A_t into AT[p], the row factors for
+    // the walk, and the next rows of the iterate and of delta
+    // (delta_t = A_t delta_{t-1} - F_t)
+    auto row_step = [&](const StepIn& in, int p, int64_t t) {
         float uz = 0.0f, ur = 0.0f, uc = 0.0f;
 #pragma unroll
         for (int s = 0; s < SEG; ++s) {
@@ -305,6 +325,7 @@ __global__ void __launch_bounds__(kThreads, 2) head_chunk_kernel(const Params pr
         const RowLin L = row_linearise(in, sp, uz, ur, uc);
         if (qt == 0) rmax = nanmax_f(rmax, fabsf(L.F));
         if constexpr (!kResidOnly) {
+            if (qt == 0) store_row_factors<DH>(pr, seq, t, i, in.s, L);
             float dp = 0.0f;
 #pragma unroll
             for (int s = 0; s < SEG; ++s) {
@@ -326,7 +347,7 @@ __global__ void __launch_bounds__(kThreads, 2) head_chunk_kernel(const Params pr
     {
         const StepIn in = nxt;
         if (t0 + 1 < t1) nxt = load_step<DH, PxT>(pr, b, h, i, t0 + 1);
-        row_step(in, 0);
+        row_step(in, 0, t0);
     }
     __syncthreads();
     int p = 0, cur = 0;
@@ -335,7 +356,7 @@ __global__ void __launch_bounds__(kThreads, 2) head_chunk_kernel(const Params pr
         if (t + 1 < t1) {
             const StepIn in = nxt;
             if (t + 2 < t1) nxt = load_step<DH, PxT>(pr, b, h, i, t + 2);
-            row_step(in, p ^ 1);
+            row_step(in, p ^ 1, t + 1);
         }
         __syncthreads();
         cur ^= 1;
@@ -506,9 +527,10 @@ __global__ void __launch_bounds__(kThreads, 2) head_chunk_tc_kernel(const Params
     }
     float rmax = 0.0f;
 
-    // the row work of one step: row i of A_t (split) into A[p], and the next
-    // rows of the iterate and of delta (delta_t = A_t delta_{t-1} - F_t)
-    auto row_step = [&](const StepIn& in, int p) {
+    // the row work of step t: row i of A_t (split) into A[p], the row factors
+    // for the walk, and the next rows of the iterate and of delta
+    // (delta_t = A_t delta_{t-1} - F_t)
+    auto row_step = [&](const StepIn& in, int p, int64_t t) {
         float uz = 0.0f, ur = 0.0f, uc = 0.0f;
 #pragma unroll
         for (int s = 0; s < SEG; ++s) {
@@ -522,7 +544,10 @@ __global__ void __launch_bounds__(kThreads, 2) head_chunk_tc_kernel(const Params
         uc = row_sum<DH>(uc);
         const float sp = sm.sv[p][Gm::vpos(i)];
         const RowLin L = row_linearise(in, sp, uz, ur, uc);
-        if (qt == 0) rmax = nanmax_f(rmax, fabsf(L.F));
+        if (qt == 0) {
+            rmax = nanmax_f(rmax, fabsf(L.F));
+            store_row_factors<DH>(pr, seq, t, i, in.s, L);
+        }
         float* ahi = sm.Ahi[p];
         float* alo = sm.Alo[p];
         float dp = 0.0f;
@@ -552,7 +577,7 @@ __global__ void __launch_bounds__(kThreads, 2) head_chunk_tc_kernel(const Params
     {
         const StepIn in = nxt;
         if (t0 + 1 < t1) nxt = load_step<DH, PxT>(pr, b, h, i, t0 + 1);
-        row_step(in, 0);
+        row_step(in, 0, t0);
     }
     tc::sync_block();
 
@@ -584,7 +609,7 @@ __global__ void __launch_bounds__(kThreads, 2) head_chunk_tc_kernel(const Params
         if (t + 1 < t1) {
             const StepIn in = nxt;
             if (t + 2 < t1) nxt = load_step<DH, PxT>(pr, b, h, i, t + 2);
-            row_step(in, p ^ 1);
+            row_step(in, p ^ 1, t + 1);
         }
         // wait for the product (bounded), then move it out of tensor memory
         if (!abort_flag) {
@@ -688,21 +713,20 @@ __global__ void __launch_bounds__(64) head_carry_kernel(const Params pr) {
 
 // ---- C: re-walk each chunk from its carry and write h^(k+1) --------------
 // delta_t = A_t delta_{t-1} - F_t with A_t applied as
-// diag(1-z) + diag(alpha) U_z + diag(beta) U_r + diag(gamma) U_c; one block
-// barrier per step, the vectors double-buffered as in the chunk kernel.
+// diag(1-z) + diag(alpha) U_z + diag(beta) U_r + diag(gamma) U_c.  The row
+// factors (h^(k)_t, F_t, 1 - z, alpha, beta, gamma) are the ones the chunk
+// kernel formed for the Jacobian rows, so per step the walk does only the
+// dependent chain: three dot products with delta_{t-1} and the update.  One
+// block barrier per step, delta double-buffered; the factors are prefetched
+// kWalkAhead steps ahead by the row's first thread, the only one that
+// combines them.
 constexpr int kWalkAhead = 2;
 
 template <int DH>
-struct SmemC {
-    float sv[2][DH];
-    float dv[2][DH];
-};
-
-template <int DH, typename PxT>
 __global__ void __launch_bounds__(kThreads, 2) head_walk_kernel(const Params pr) {
     using Gm = Geo<DH>;
     constexpr int TPR = Gm::TPR, SEG = Gm::SEG;
-    __shared__ SmemC<DH> sm;
+    __shared__ float dv[2][DH];  // delta rows, permuted, two steps in turn
     const int tid = threadIdx.x, i = tid / TPR, qt = tid % TPR;
     const int64_t task = blockIdx.x;
     const int64_t seq = task / pr.nChunks;
@@ -714,54 +738,51 @@ __global__ void __launch_bounds__(kThreads, 2) head_walk_kernel(const Params pr)
 
     RowU<DH> U;
     U.load(pr.U, pr.nh, h, i, qt);
-    const float s_before = iterate_before<DH, PxT>(pr, b, h, i, t0);
-    if (qt == 0) {
-        sm.sv[0][Gm::vpos(i)] = s_before;
-        sm.dv[0][Gm::vpos(i)] = pr.carry[task * DH + i];
-    }
-    // inputs prefetched kWalkAhead steps ahead (measured: two steps ahead
-    // beats one by about 1 %; deeper gains nothing)
-    StepIn ahead[kWalkAhead];
+    auto load_f = [&](int64_t t, float (&f)[kNF]) {
+        const float* src = pr.L + ((seq * pr.T + t) * kNF) * DH + i;
 #pragma unroll
-    for (int j = 0; j < kWalkAhead; ++j)
-        if (t0 + j < t1) ahead[j] = load_step<DH, PxT>(pr, b, h, i, t0 + j);
+        for (int j = 0; j < kNF; ++j) f[j] = src[j * DH];
+    };
+    float ahead[kWalkAhead][kNF];
+    if (qt == 0) {
+        dv[0][Gm::vpos(i)] = pr.carry[task * DH + i];
+#pragma unroll
+        for (int j = 0; j < kWalkAhead; ++j)
+            if (t0 + j < t1) load_f(t0 + j, ahead[j]);
+    }
     __syncthreads();
     int par = 0;
     bool bad = false;
     for (int64_t t = t0; t < t1; ++t) {
-        const StepIn in = ahead[0];
-#pragma unroll
-        for (int j = 0; j + 1 < kWalkAhead; ++j) ahead[j] = ahead[j + 1];
-        if (t + kWalkAhead < t1) ahead[kWalkAhead - 1] = load_step<DH, PxT>(pr, b, h, i, t + kWalkAhead);
-        float uz = 0.0f, ur = 0.0f, uc = 0.0f, vz = 0.0f, vr = 0.0f, vc = 0.0f;
+        float vz = 0.0f, vr = 0.0f, vc = 0.0f;
 #pragma unroll
         for (int s = 0; s < SEG; ++s) {
-            const float x = sm.sv[par][qt * SEG + s], y = sm.dv[par][qt * SEG + s];
-            uz = __fmaf_rn(U.z[s], x, uz);
-            ur = __fmaf_rn(U.r[s], x, ur);
-            uc = __fmaf_rn(U.c[s], x, uc);
+            const float y = dv[par][qt * SEG + s];
             vz = __fmaf_rn(U.z[s], y, vz);
             vr = __fmaf_rn(U.r[s], y, vr);
             vc = __fmaf_rn(U.c[s], y, vc);
         }
-        uz = row_sum<DH>(uz);
-        ur = row_sum<DH>(ur);
-        uc = row_sum<DH>(uc);
         vz = row_sum<DH>(vz);
         vr = row_sum<DH>(vr);
         vc = row_sum<DH>(vc);
-        const float sp = sm.sv[par][Gm::vpos(i)], dprev = sm.dv[par][Gm::vpos(i)];
-        const RowLin L = row_linearise(in, sp, uz, ur, uc);
-        float d = __fmaf_rn(L.dz, dprev, -L.F);
-        d = __fmaf_rn(L.al, vz, d);
-        d = __fmaf_rn(L.be, vr, d);
-        d = __fmaf_rn(L.ga, vc, d);
         if (qt == 0) {
-            const float hn = in.s + d;
+            float f[kNF];
+#pragma unroll
+            for (int j = 0; j < kNF; ++j) f[j] = ahead[0][j];
+#pragma unroll
+            for (int a = 0; a + 1 < kWalkAhead; ++a)
+#pragma unroll
+                for (int j = 0; j < kNF; ++j) ahead[a][j] = ahead[a + 1][j];
+            if (t + kWalkAhead < t1) load_f(t + kWalkAhead, ahead[kWalkAhead - 1]);
+            const float dprev = dv[par][Gm::vpos(i)];
+            float d = __fmaf_rn(f[2], dprev, -f[1]);  // (1 - z) delta_{t-1} - F_t
+            d = __fmaf_rn(f[3], vz, d);
+            d = __fmaf_rn(f[4], vr, d);
+            d = __fmaf_rn(f[5], vc, d);
+            const float hn = f[0] + d;
             pr.Hnew[(b * pr.T + t) * pr.D + (int64_t)h * DH + i] = hn;
             bad |= !isfinite(hn);
-            sm.sv[par ^ 1][Gm::vpos(i)] = in.s;
-            sm.dv[par ^ 1][Gm::vpos(i)] = d;
+            dv[par ^ 1][Gm::vpos(i)] = d;
         }
         __syncthreads();
         par ^= 1;
@@ -817,15 +838,26 @@ struct SmemB {
     float sv[2][DH];              // h_{t-1} rows for the row work (permuted)
     float gv[2][DH];              // g_t rows (permuted)
     float mv[2][DH];              // mu rows (permuted)
-    float fv[2][4][DH];           // alpha, beta, z (1 - c^2), gamma of the step (walk only)
 };
 
+// step t's backward row factors of row i, for the walk
+template <int DH>
+__device__ __forceinline__ void store_brow_factors(const Params& pr, int64_t seq, int64_t t, int i, float dz, float al,
+                                                   float be, float zc, float ga) {
+    float* o = pr.L + ((seq * pr.T + t) * kNB) * DH + i;
+    o[0] = dz;
+    o[DH] = al;
+    o[2 * DH] = be;
+    o[3 * DH] = zc;
+    o[4 * DH] = ga;
+}
+
 // The backward's row work for step t, parity p: the gates at (h_{t-1}, x_t),
-// row i of A_t into AT[p], g_t and (walk) the row factors into gv / fv, and
+// row i of A_t into AT[p], the row factors for the walk, g_t into gv, and
 // h_{t-2} into sv[p ^ 1] for the next (earlier) step's row work.
-template <int DH, bool kWalk>
+template <int DH>
 __device__ __forceinline__ void bwd_row_work(SmemB<DH>& sm, const RowU<DH>& U, const BStepIn& in, int p, int i,
-                                             int qt) {
+                                             int qt, const Params& pr, int64_t seq, int64_t t) {
     constexpr int TPR = Geo<DH>::TPR, SEG = Geo<DH>::SEG;
     float uz = 0.0f, ur = 0.0f, uc = 0.0f;
 #pragma unroll
@@ -856,12 +888,7 @@ __device__ __forceinline__ void bwd_row_work(SmemB<DH>& sm, const RowU<DH>& U, c
         const int vi = Geo<DH>::vpos(i);
         sm.gv[p][vi] = in.g;
         sm.sv[p ^ 1][vi] = in.s2;
-        if constexpr (kWalk) {
-            sm.fv[p][0][vi] = al;
-            sm.fv[p][1][vi] = be;
-            sm.fv[p][2][vi] = zc;
-            sm.fv[p][3][vi] = ga;
-        }
+        store_brow_factors<DH>(pr, seq, t, i, dz, al, be, zc, ga);
     }
 }
 
@@ -882,8 +909,9 @@ __device__ __forceinline__ float bwd_mu(const SmemB<DH>& sm, int p, int m, int q
 // ---- backward A: the chunk's product of transposed Jacobians -------------
 // Steps run from t1-1 down to t0 (r = t1-1-t, p = r & 1); as in the forward
 // chunk kernel the product of step t and mu_t share a barrier interval with
-// the row work of step t-1.
-template <int DH, typename PxT, bool kWalk>
+// the row work of step t-1.  (Head widths 16 and 32; 64 runs
+// head_bwd_tc_kernel.)
+template <int DH, typename PxT>
 __global__ void __launch_bounds__(kThreads, 2) head_bwd_kernel(const Params pr) {
     using Gm = Geo<DH>;
     constexpr int TPR = Gm::TPR;
@@ -902,61 +930,144 @@ __global__ void __launch_bounds__(kThreads, 2) head_bwd_kernel(const Params pr) 
     U.load(pr.U, pr.nh, h, i, qt);
     if (qt == 0) {
         sm.sv[0][Gm::vpos(i)] = state_before<DH>(pr, b, h, i, t1 - 1);
-        // mu_{t1}: zero for the chunk's own product, the carry for the walk
-        sm.mv[1][Gm::vpos(i)] = kWalk ? pr.carry[task * DH + i] : 0.0f;
+        sm.mv[1][Gm::vpos(i)] = 0.0f;  // mu_{t1} for the chunk's own product
     }
-    if constexpr (!kWalk)
-        for (int idx = tid; idx < DH * DH; idx += kThreads)
-            sm.Pm[0][idx / DH][idx % DH] = make_uint2(idx / DH == idx % DH ? __float_as_uint(1.0f) : 0u, 0u);
+    for (int idx = tid; idx < DH * DH; idx += kThreads)
+        sm.Pm[0][idx / DH][idx % DH] = make_uint2(idx / DH == idx % DH ? __float_as_uint(1.0f) : 0u, 0u);
     BStepIn nxt = load_bstep<DH, PxT>(pr, b, h, i, t1 - 1);
     __syncthreads();
     {
         const BStepIn in = nxt;
         if (t1 - 2 >= t0) nxt = load_bstep<DH, PxT>(pr, b, h, i, t1 - 2);
-        bwd_row_work<DH, kWalk>(sm, U, in, 0, i, qt);
+        bwd_row_work<DH>(sm, U, in, 0, i, qt, pr, seq, t1 - 1);
     }
     __syncthreads();
     int p = 0, cur = 0;
-    bool bad = false;
     for (int64_t t = t1 - 1; t >= t0; --t) {
-        if constexpr (!kWalk) matmul_tf32x3<DH, false>(sm.AT[p], sm.Pm[cur], sm.Pm[cur ^ 1]);
+        matmul_tf32x3<DH, false>(sm.AT[p], sm.Pm[cur], sm.Pm[cur ^ 1]);
         const float mu = bwd_mu<DH>(sm, p, i, qt);  // thread (m = i, qt)
-        if (qt == 0) {
-            sm.mv[p][Gm::vpos(i)] = mu;
-            if constexpr (kWalk) {
-                // the epilogue of row i at step t
-                const int vi = Gm::vpos(i);
-                const float lam = sm.gv[p][vi] + sm.mv[p ^ 1][vi];
-                const int64_t o = ((b * pr.T + t) * 3) * pr.D + (int64_t)h * DH + i;
-                const float d0 = lam * sm.fv[p][0][vi], d1 = lam * sm.fv[p][1][vi], d2 = lam * sm.fv[p][2][vi];
-                pr.dpx[o] = d0;
-                pr.dpx[o + pr.D] = d1;
-                pr.dpx[o + 2 * pr.D] = d2;
-                pr.ec[(b * pr.T + t) * pr.D + (int64_t)h * DH + i] = lam * sm.fv[p][3][vi];
-                bad |= !(isfinite(d0) && isfinite(d1) && isfinite(d2));
-                if (t == 0 && pr.dh0) pr.dh0[b * pr.D + (int64_t)h * DH + i] = mu;
-            }
-        }
+        if (qt == 0) sm.mv[p][Gm::vpos(i)] = mu;
         if (t - 1 >= t0) {
             const BStepIn in = nxt;
             if (t - 2 >= t0) nxt = load_bstep<DH, PxT>(pr, b, h, i, t - 2);
-            bwd_row_work<DH, kWalk>(sm, U, in, p ^ 1, i, qt);
+            bwd_row_work<DH>(sm, U, in, p ^ 1, i, qt, pr, seq, t - 1);
         }
         __syncthreads();
         cur ^= 1;
         p ^= 1;
     }
-    if constexpr (!kWalk) {
-        float* Pout = pr.P + task * DH * DH;
-        for (int idx = tid; idx < DH * DH; idx += kThreads) {
-            const uint2 v = sm.Pm[cur][idx / DH][idx % DH];
-            Pout[idx] = __uint_as_float(v.x) + __uint_as_float(v.y);
-        }
-        // mu at the chunk's first step: written to mv[p ^ 1] by the last iteration
-        if (qt == 0) pr.q[task * DH + i] = sm.mv[p ^ 1][Gm::vpos(i)];
-    } else {
-        if (__any_sync(0xffffffffu, bad) && (tid & 31) == 0) atomicOr(pr.status, kStatusNonFinite);
+    float* Pout = pr.P + task * DH * DH;
+    for (int idx = tid; idx < DH * DH; idx += kThreads) {
+        const uint2 v = sm.Pm[cur][idx / DH][idx % DH];
+        Pout[idx] = __uint_as_float(v.x) + __uint_as_float(v.y);
     }
+    // mu at the chunk's first step: written to mv[p ^ 1] by the last iteration
+    if (qt == 0) pr.q[task * DH + i] = sm.mv[p ^ 1][Gm::vpos(i)];
+}
+
+// ---- backward C: re-walk each chunk from its carry -----------------------
+// From mu_{t1} (the carry) down to t0: lambda_t = g_t + mu_{t+1},
+// dL/dpx_t = lambda_t (alpha, beta, z (1 - c^2)), lambda_t gamma (the factor
+// of dL/dU_c), and mu_t = A_t^T lambda_t applied without forming A_t:
+//     mu_t = (1 - z) lambda + U_z^T (alpha lambda) + U_r^T (beta lambda)
+//            + U_c^T (gamma lambda),
+// with the row factors the product kernel stored.  Thread (m, qt) keeps
+// column m of U_z, U_r, U_c (rows k = qt + TPR s) in registers; the row's
+// first thread owns lambda_m and mu_m.  One block barrier per step, the
+// scaled vectors double-buffered.
+template <int DH>
+struct ColU {
+    float z[Geo<DH>::SEG], r[Geo<DH>::SEG], c[Geo<DH>::SEG];
+    __device__ __forceinline__ void load(const float* U, int nh, int h, int m, int qt) {
+        constexpr int SEG = Geo<DH>::SEG, TPR = Geo<DH>::TPR;
+        const int64_t hs = (int64_t)DH * DH;
+#pragma unroll
+        for (int s = 0; s < SEG; ++s) {
+            const int k = qt + TPR * s;
+            z[s] = __ldg(U + (0 * nh + h) * hs + (int64_t)k * DH + m);
+            r[s] = __ldg(U + ((int64_t)1 * nh + h) * hs + (int64_t)k * DH + m);
+            c[s] = __ldg(U + ((int64_t)2 * nh + h) * hs + (int64_t)k * DH + m);
+        }
+    }
+};
+
+template <int DH>
+__global__ void __launch_bounds__(kThreads, 2) head_bwd_walk_kernel(const Params pr) {
+    using Gm = Geo<DH>;
+    constexpr int TPR = Gm::TPR, SEG = Gm::SEG;
+    __shared__ float wv[2][3][DH];  // alpha lambda, beta lambda, gamma lambda (permuted), two steps in turn
+    const int tid = threadIdx.x, i = tid / TPR, qt = tid % TPR;
+    const int64_t task = blockIdx.x;
+    const int64_t seq = task / pr.nChunks;
+    const int chunk = (int)(task - seq * pr.nChunks);
+    const int64_t b = seq / pr.nh;
+    const int h = (int)(seq - b * pr.nh);
+    const int64_t t0 = (int64_t)chunk * kChunk;
+    const int64_t t1 = t0 + kChunk < pr.T ? t0 + kChunk : pr.T;
+    const int64_t col = (int64_t)h * DH + i;
+
+    ColU<DH> UT;
+    UT.load(pr.U, pr.nh, h, i, qt);
+    // the row factors and g of step t (read by the row's first thread only)
+    auto load_f = [&](int64_t t, float (&f)[kNB + 1]) {
+        const float* src = pr.L + ((seq * pr.T + t) * kNB) * DH + i;
+#pragma unroll
+        for (int j = 0; j < kNB; ++j) f[j] = src[j * DH];
+        f[kNB] = pr.G[(b * pr.T + t) * pr.D + col];
+    };
+    float ahead[kWalkAhead][kNB + 1];
+    float mu = 0.0f;  // mu_{t+1} of row i (first thread of the row)
+    if (qt == 0) {
+        mu = pr.carry[task * DH + i];
+#pragma unroll
+        for (int j = 0; j < kWalkAhead; ++j)
+            if (t1 - 1 - j >= t0) load_f(t1 - 1 - j, ahead[j]);
+    }
+    int par = 0;
+    bool bad = false;
+    for (int64_t t = t1 - 1; t >= t0; --t) {
+        float dzl = 0.0f;
+        if (qt == 0) {
+            float f[kNB + 1];
+#pragma unroll
+            for (int j = 0; j <= kNB; ++j) f[j] = ahead[0][j];
+#pragma unroll
+            for (int a = 0; a + 1 < kWalkAhead; ++a)
+#pragma unroll
+                for (int j = 0; j <= kNB; ++j) ahead[a][j] = ahead[a + 1][j];
+            if (t - kWalkAhead >= t0) load_f(t - kWalkAhead, ahead[kWalkAhead - 1]);
+            const float lam = f[kNB] + mu;
+            const int64_t o = ((b * pr.T + t) * 3) * pr.D + col;
+            const float d0 = lam * f[1], d1 = lam * f[2], d2 = lam * f[3];
+            pr.dpx[o] = d0;
+            pr.dpx[o + pr.D] = d1;
+            pr.dpx[o + 2 * pr.D] = d2;
+            pr.ec[(b * pr.T + t) * pr.D + col] = lam * f[4];
+            bad |= !(isfinite(d0) && isfinite(d1) && isfinite(d2));
+            const int vi = Gm::vpos(i);
+            wv[par][0][vi] = f[1] * lam;
+            wv[par][1][vi] = f[2] * lam;
+            wv[par][2][vi] = f[4] * lam;
+            dzl = f[0] * lam;
+        }
+        __syncthreads();
+        float sz = 0.0f, sr = 0.0f, sc = 0.0f;
+#pragma unroll
+        for (int s = 0; s < SEG; ++s) {
+            sz = __fmaf_rn(UT.z[s], wv[par][0][qt * SEG + s], sz);
+            sr = __fmaf_rn(UT.r[s], wv[par][1][qt * SEG + s], sr);
+            sc = __fmaf_rn(UT.c[s], wv[par][2][qt * SEG + s], sc);
+        }
+        sz = row_sum<DH>(sz);
+        sr = row_sum<DH>(sr);
+        sc = row_sum<DH>(sc);
+        if (qt == 0) {
+            mu = ((dzl + sz) + sr) + sc;  // mu_t
+            if (t == 0 && pr.dh0) pr.dh0[b * pr.D + col] = mu;
+        }
+        par ^= 1;
+    }
+    if (__any_sync(0xffffffffu, bad) && (tid & 31) == 0) atomicOr(pr.status, kStatusNonFinite);
 }
 
 // ---- backward A on the fifth-generation tensor cores (head width 64) ------
@@ -1034,9 +1145,10 @@ __global__ void __launch_bounds__(kThreads, 2) head_bwd_tc_kernel(const Params p
     }
 
     // the row work of step t, parity p: the gates at (h_{t-1}, x_t), row i of
-    // A_t as column i of A_t^T (split) into A[p], g_t into gv[p], and h_{t-2}
-    // into sv[p ^ 1] for the next (earlier) step
-    auto row_step = [&](const BStepIn& in, int p) {
+    // A_t as column i of A_t^T (split) into A[p], the row factors for the
+    // walk, g_t into gv[p], and h_{t-2} into sv[p ^ 1] for the next (earlier)
+    // step
+    auto row_step = [&](const BStepIn& in, int p, int64_t t) {
         float uz = 0.0f, ur = 0.0f, uc = 0.0f;
 #pragma unroll
         for (int s = 0; s < SEG; ++s) {
@@ -1070,6 +1182,7 @@ __global__ void __launch_bounds__(kThreads, 2) head_bwd_tc_kernel(const Params p
             const int vi = Gm::vpos(i);
             sm.gv[p][vi] = in.g;
             sm.sv[p ^ 1][vi] = in.s2;
+            store_brow_factors<DH>(pr, seq, t, i, dz, al, be, zc, ga);
         }
     };
 
@@ -1081,7 +1194,7 @@ __global__ void __launch_bounds__(kThreads, 2) head_bwd_tc_kernel(const Params p
     {
         const BStepIn in = nxt;
         if (t1 - 2 >= t0) nxt = load_bstep<DH, PxT>(pr, b, h, i, t1 - 2);
-        row_step(in, 0);
+        row_step(in, 0, t1 - 1);
     }
     tc::sync_block();
 
@@ -1123,7 +1236,7 @@ __global__ void __launch_bounds__(kThreads, 2) head_bwd_tc_kernel(const Params p
         if (t - 1 >= t0) {
             const BStepIn in = nxt;
             if (t - 2 >= t0) nxt = load_bstep<DH, PxT>(pr, b, h, i, t - 2);
-            row_step(in, p ^ 1);
+            row_step(in, p ^ 1, t - 1);
         }
         if (!abort_flag) {
             uint64_t start = 0;
@@ -1243,11 +1356,12 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 struct Plan {
     int d = 0, nChunks = 0;
     int64_t nSeq = 0;
-    size_t off_h = 0, off_P = 0, off_q = 0, off_c = 0, total = 0;
+    size_t off_h = 0, off_P = 0, off_q = 0, off_c = 0, off_L = 0, total = 0;
 };
 
 // workspace: 256-byte header (status word) | second iterate buffer (K >= 2)
-// | chunk products P | chunk deltas q | chunk carries
+// | chunk products P | chunk deltas q | chunk carries | row factors
+// (kNF per element; the backward's plan sizes kNB)
 bool make_plan(int64_t B, int64_t T, int64_t D, int nh, int K, Plan& pl) {
     if (B < 0 || T < 0 || D < 0 || nh < 1 || D % nh != 0) return false;
     const int64_t d = D / nh;
@@ -1261,7 +1375,8 @@ bool make_plan(int64_t B, int64_t T, int64_t D, int nh, int K, Plan& pl) {
     pl.off_P = align256(pl.off_h + (K >= 2 ? (size_t)B * T * D * sizeof(float) : 0));
     pl.off_q = align256(pl.off_P + ntask * d * d * sizeof(float));
     pl.off_c = align256(pl.off_q + ntask * d * sizeof(float));
-    pl.total = align256(pl.off_c + ntask * d * sizeof(float));
+    pl.off_L = align256(pl.off_c + ntask * d * sizeof(float));
+    pl.total = align256(pl.off_L + (size_t)B * T * D * kNF * sizeof(float));
     return true;
 }
 
@@ -1291,7 +1406,7 @@ cudaError_t launch_all(const Plan& pl, Params pr, float* H_out, float* Hbuf, int
         else
             head_chunk_kernel<DH, PxT, false><<<ntask, kThreads, smemA, st>>>(pr);
         head_carry_kernel<DH><<<(unsigned)pl.nSeq, 64, 0, st>>>(pr);
-        head_walk_kernel<DH, PxT><<<ntask, kThreads, 0, st>>>(pr);
+        head_walk_kernel<DH><<<ntask, kThreads, 0, st>>>(pr);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     if (pr.resid) {
@@ -1307,11 +1422,12 @@ cudaError_t launch_all(const Plan& pl, Params pr, float* H_out, float* Hbuf, int
 struct BPlan {
     int d = 0, nChunks = 0, nsplit = 0;
     int64_t nSeq = 0, rows_per_split = 0;
-    size_t off_P = 0, off_q = 0, off_c = 0, off_ec = 0, off_part = 0, total = 0;
+    size_t off_P = 0, off_q = 0, off_c = 0, off_ec = 0, off_L = 0, off_part = 0, total = 0;
 };
 
 // backward workspace: 256-byte header (status word) | chunk products Q |
-// chunk mus q | chunk carries | lambda * gamma (B,T,D) | dL/dU split partials
+// chunk mus q | chunk carries | lambda * gamma (B,T,D) | row factors (kNB
+// per element) | dL/dU split partials
 bool make_bplan(int64_t B, int64_t T, int64_t D, int nh, BPlan& pl) {
     Plan fp;
     if (!make_plan(B, T, D, nh, 1, fp)) return false;
@@ -1327,7 +1443,8 @@ bool make_bplan(int64_t B, int64_t T, int64_t D, int nh, BPlan& pl) {
     pl.off_q = align256(pl.off_P + ntask * d * d * sizeof(float));
     pl.off_c = align256(pl.off_q + ntask * d * sizeof(float));
     pl.off_ec = align256(pl.off_c + ntask * d * sizeof(float));
-    pl.off_part = align256(pl.off_ec + (size_t)B * T * D * sizeof(float));
+    pl.off_L = align256(pl.off_ec + (size_t)B * T * D * sizeof(float));
+    pl.off_part = align256(pl.off_L + (size_t)B * T * D * kNB * sizeof(float));
     pl.total = align256(pl.off_part + (size_t)pl.nsplit * 3 * nh * d * d * sizeof(float));
     return true;
 }
@@ -1336,17 +1453,16 @@ template <int DH, typename PxT>
 cudaError_t launch_bwd(const BPlan& pl, const Params& pr, float* dU, cudaStream_t st) {
     // head width 64: the products on tcgen05, as in the forward
     constexpr bool kTc = DH == tc::kD;
-    const size_t smem = sizeof(SmemB<DH>), smemP = kTc ? sizeof(tc::SmemB) : smem;
-    cudaError_t e = kTc ? set_smem(head_bwd_tc_kernel<PxT>, smemP) : set_smem(head_bwd_kernel<DH, PxT, false>, smemP);
-    if (e == cudaSuccess) e = set_smem(head_bwd_kernel<DH, PxT, true>, smem);
+    const size_t smemP = kTc ? sizeof(tc::SmemB) : sizeof(SmemB<DH>);
+    cudaError_t e = kTc ? set_smem(head_bwd_tc_kernel<PxT>, smemP) : set_smem(head_bwd_kernel<DH, PxT>, smemP);
     if (e != cudaSuccess) return e;
     const unsigned ntask = (unsigned)(pl.nSeq * pl.nChunks);
     if constexpr (kTc)
         head_bwd_tc_kernel<PxT><<<ntask, kThreads, smemP, st>>>(pr);
     else
-        head_bwd_kernel<DH, PxT, false><<<ntask, kThreads, smemP, st>>>(pr);
+        head_bwd_kernel<DH, PxT><<<ntask, kThreads, smemP, st>>>(pr);
     head_carry_kernel<DH, true><<<(unsigned)pl.nSeq, 64, 0, st>>>(pr);
-    head_bwd_kernel<DH, PxT, true><<<ntask, kThreads, smem, st>>>(pr);
+    head_bwd_walk_kernel<DH><<<ntask, kThreads, 0, st>>>(pr);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (dU) {
         float* part = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(pr.status) + pl.off_part);
@@ -1414,6 +1530,7 @@ extern "C" pararnn_status pararnn_head_gru_forward(int64_t B, int64_t T, int64_t
         if (e != cudaSuccess) return hg::fail(PARARNN_ECUDA, "pararnn_head_gru_forward: resid_hist reset failed");
     }
     hg::Params pr;
+    memset(&pr, 0, sizeof pr);
     pr.px = preacts;
     pr.U = U;
     pr.h0 = h0;
@@ -1422,6 +1539,7 @@ extern "C" pararnn_status pararnn_head_gru_forward(int64_t B, int64_t T, int64_t
     pr.P = reinterpret_cast<float*>(ws + pl.off_P);
     pr.q = reinterpret_cast<float*>(ws + pl.off_q);
     pr.carry = reinterpret_cast<float*>(ws + pl.off_c);
+    pr.L = reinterpret_cast<float*>(ws + pl.off_L);
     pr.resid = resid_hist;
     pr.status = reinterpret_cast<unsigned*>(ws);
     pr.B = B;
@@ -1507,6 +1625,7 @@ extern "C" pararnn_status pararnn_head_gru_backward(int64_t B, int64_t T, int64_
     pr.q = reinterpret_cast<float*>(ws + pl.off_q);
     pr.carry = reinterpret_cast<float*>(ws + pl.off_c);
     pr.ec = reinterpret_cast<float*>(ws + pl.off_ec);
+    pr.L = reinterpret_cast<float*>(ws + pl.off_L);
     pr.status = reinterpret_cast<unsigned*>(ws);
     pr.B = B;
     pr.T = T;
