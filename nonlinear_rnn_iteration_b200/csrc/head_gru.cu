@@ -717,10 +717,11 @@ __global__ void __launch_bounds__(64) head_carry_kernel(const Params pr) {
 // factors (h^(k)_t, F_t, 1 - z, alpha, beta, gamma) are the ones the chunk
 // kernel formed for the Jacobian rows, so per step the walk does only the
 // dependent chain: three dot products with delta_{t-1} and the update.  One
-// block barrier per step, delta double-buffered; the factors are prefetched
-// kWalkAhead steps ahead by the row's first thread, the only one that
-// combines them.
-constexpr int kWalkAhead = 2;
+// block barrier per step, delta double-buffered.  The row's first thread,
+// the only one that combines the factors, loads them two steps ahead into
+// one of two register sets that alternate with the steps (the loop body is
+// unrolled twice so that a set is consumed before it is reloaded and no
+// register copy waits on a load in flight).
 
 template <int DH>
 __global__ void __launch_bounds__(kThreads, 2) head_walk_kernel(const Params pr) {
@@ -743,17 +744,16 @@ __global__ void __launch_bounds__(kThreads, 2) head_walk_kernel(const Params pr)
 #pragma unroll
         for (int j = 0; j < kNF; ++j) f[j] = src[j * DH];
     };
-    float ahead[kWalkAhead][kNF];
+    float fa[kNF], fb[kNF];
     if (qt == 0) {
         dv[0][Gm::vpos(i)] = pr.carry[task * DH + i];
-#pragma unroll
-        for (int j = 0; j < kWalkAhead; ++j)
-            if (t0 + j < t1) load_f(t0 + j, ahead[j]);
+        load_f(t0, fa);
+        if (t0 + 1 < t1) load_f(t0 + 1, fb);
     }
     __syncthreads();
     int par = 0;
     bool bad = false;
-    for (int64_t t = t0; t < t1; ++t) {
+    auto step = [&](int64_t t, float (&f)[kNF]) {
         float vz = 0.0f, vr = 0.0f, vc = 0.0f;
 #pragma unroll
         for (int s = 0; s < SEG; ++s) {
@@ -766,14 +766,6 @@ __global__ void __launch_bounds__(kThreads, 2) head_walk_kernel(const Params pr)
         vr = row_sum<DH>(vr);
         vc = row_sum<DH>(vc);
         if (qt == 0) {
-            float f[kNF];
-#pragma unroll
-            for (int j = 0; j < kNF; ++j) f[j] = ahead[0][j];
-#pragma unroll
-            for (int a = 0; a + 1 < kWalkAhead; ++a)
-#pragma unroll
-                for (int j = 0; j < kNF; ++j) ahead[a][j] = ahead[a + 1][j];
-            if (t + kWalkAhead < t1) load_f(t + kWalkAhead, ahead[kWalkAhead - 1]);
             const float dprev = dv[par][Gm::vpos(i)];
             float d = __fmaf_rn(f[2], dprev, -f[1]);  // (1 - z) delta_{t-1} - F_t
             d = __fmaf_rn(f[3], vz, d);
@@ -783,9 +775,14 @@ __global__ void __launch_bounds__(kThreads, 2) head_walk_kernel(const Params pr)
             pr.Hnew[(b * pr.T + t) * pr.D + (int64_t)h * DH + i] = hn;
             bad |= !isfinite(hn);
             dv[par ^ 1][Gm::vpos(i)] = d;
+            if (t + 2 < t1) load_f(t + 2, f);
         }
         __syncthreads();
         par ^= 1;
+    };
+    for (int64_t t = t0; t < t1; t += 2) {
+        step(t, fa);
+        if (t + 1 < t1) step(t + 1, fb);
     }
     if (__any_sync(0xffffffffu, bad) && (tid & 31) == 0) atomicOr(pr.status, kStatusNonFinite);
 }
@@ -1015,27 +1012,20 @@ __global__ void __launch_bounds__(kThreads, 2) head_bwd_walk_kernel(const Params
         for (int j = 0; j < kNB; ++j) f[j] = src[j * DH];
         f[kNB] = pr.G[(b * pr.T + t) * pr.D + col];
     };
-    float ahead[kWalkAhead][kNB + 1];
+    // two register sets of factors, alternating with the steps (as in the
+    // forward walk)
+    float fa[kNB + 1], fb[kNB + 1];
     float mu = 0.0f;  // mu_{t+1} of row i (first thread of the row)
     if (qt == 0) {
         mu = pr.carry[task * DH + i];
-#pragma unroll
-        for (int j = 0; j < kWalkAhead; ++j)
-            if (t1 - 1 - j >= t0) load_f(t1 - 1 - j, ahead[j]);
+        load_f(t1 - 1, fa);
+        if (t1 - 2 >= t0) load_f(t1 - 2, fb);
     }
     int par = 0;
     bool bad = false;
-    for (int64_t t = t1 - 1; t >= t0; --t) {
+    auto step = [&](int64_t t, float (&f)[kNB + 1]) {
         float dzl = 0.0f;
         if (qt == 0) {
-            float f[kNB + 1];
-#pragma unroll
-            for (int j = 0; j <= kNB; ++j) f[j] = ahead[0][j];
-#pragma unroll
-            for (int a = 0; a + 1 < kWalkAhead; ++a)
-#pragma unroll
-                for (int j = 0; j <= kNB; ++j) ahead[a][j] = ahead[a + 1][j];
-            if (t - kWalkAhead >= t0) load_f(t - kWalkAhead, ahead[kWalkAhead - 1]);
             const float lam = f[kNB] + mu;
             const int64_t o = ((b * pr.T + t) * 3) * pr.D + col;
             const float d0 = lam * f[1], d1 = lam * f[2], d2 = lam * f[3];
@@ -1049,6 +1039,7 @@ __global__ void __launch_bounds__(kThreads, 2) head_bwd_walk_kernel(const Params
             wv[par][1][vi] = f[2] * lam;
             wv[par][2][vi] = f[4] * lam;
             dzl = f[0] * lam;
+            if (t - 2 >= t0) load_f(t - 2, f);
         }
         __syncthreads();
         float sz = 0.0f, sr = 0.0f, sc = 0.0f;
@@ -1066,6 +1057,10 @@ __global__ void __launch_bounds__(kThreads, 2) head_bwd_walk_kernel(const Params
             if (t == 0 && pr.dh0) pr.dh0[b * pr.D + col] = mu;
         }
         par ^= 1;
+    };
+    for (int64_t t = t1 - 1; t >= t0; t -= 2) {
+        step(t, fa);
+        if (t - 1 >= t0) step(t - 1, fb);
     }
     if (__any_sync(0xffffffffu, bad) && (tid & 31) == 0) atomicOr(pr.status, kStatusNonFinite);
 }
