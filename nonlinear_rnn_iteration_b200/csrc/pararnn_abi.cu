@@ -38,13 +38,16 @@ pararnn_status cuda_fail(cudaError_t e, const char* what) {
 // Element-wise path otherwise: 32 channels per tile.  Blocks of 8 warps
 // (7 compute + the scan warp) or 6 warps let two blocks share an SM with
 // 128 or 168 registers per thread; a 9-warp block puts 5 warps of two blocks
-// on one of the SM's four schedulers and caps registers at 96.
+// on one of the SM's four schedulers and caps registers at 96.  The LSTM
+// backward runs one block of 11 warps per SM (10 compute warps, 80-step
+// tiles): half as many tiles to look back across as 5 compute warps give,
+// at 168 registers.
 template <typename PxT> using FwdLinT = FwdShape<CellLinear, PxT, 4, 8, 4, 8, 2, 3, true>;
 template <typename PxT> using FwdGruT = FwdShape<CellGRU, PxT, 4, 8, 8, 4, 2, 2, true>;
 template <typename PxT> using FwdLstmT = FwdShape<CellLSTM, PxT, 2, 16, 7, 5, 2, 2, true>;
 template <typename PxT> using BwdLinT = FwdShape<CellLinear, PxT, 2, 16, 5, 8, 2, 2, true>;
 template <typename PxT> using BwdGruT = FwdShape<CellGRU, PxT, 2, 16, 5, 8, 2, 2, true>;
-template <typename PxT> using BwdLstmT = FwdShape<CellLSTM, PxT, 2, 16, 5, 4, 2, 2, true>;
+template <typename PxT> using BwdLstmT = FwdShape<CellLSTM, PxT, 2, 16, 10, 4, 1, 2, true>;
 template <typename PxT> using FwdLinS = FwdShape<CellLinear, PxT, 1, 32, 7, 4, 2, 2, false>;
 template <typename PxT> using FwdGruS = FwdShape<CellGRU, PxT, 1, 32, 7, 4, 2, 2, false>;
 template <typename PxT> using FwdLstmS = FwdShape<CellLSTM, PxT, 1, 32, 7, 4, 2, 2, false>;
