@@ -1284,56 +1284,109 @@ __global__ void __launch_bounds__(kThreads, 2) head_bwd_tc_kernel(const Params p
 // ---- dL/dU: outer products summed in a fixed order -------------------------
 // part[split][g][h] = sum over the split's rows (b, t) of e_g[b,t] h_{t-1}^T
 // (e_z = dL/dp_z, e_r = dL/dp_r, e_c = lambda * gamma), rows in increasing
-// (b, t) order; the reduce kernel sums the splits in order.
+// (b, t) order; the reduce kernel sums the splits in order.  A block takes
+// one split of the rows for one head and all three gates, so each row of
+// h_{t-1} is loaded once for the three products; batches of kURows rows are
+// double-buffered in shared memory with cp.async (16-byte copies when every
+// source row is 16-byte aligned, else 4-byte ones), the next batch in flight
+// while the current one is multiplied.
 constexpr int kURows = 32;
 
 template <int DH>
-__global__ void __launch_bounds__(kThreads) head_dU_kernel(const Params pr, int64_t rows_per_split, float* part) {
-    __shared__ float Es[kURows][DH], Ss[kURows][DH];
+struct SmemU {
+    float E[2][3][kURows][DH];  // e_z, e_r, e_c rows, two batches in turn
+    float S[2][kURows][DH];     // h_{t-1} rows
+};
+
+template <int kBytes>
+__device__ __forceinline__ void cp_async(void* dst, const void* src) {
+    if constexpr (kBytes == 16)
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+    else
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+
+template <int DH, int kVec>
+__global__ void __launch_bounds__(kThreads, 2) head_dU_kernel(const Params pr, int64_t rows_per_split, float* part) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    auto& sm = *reinterpret_cast<SmemU<DH>*>(smem_raw);
     constexpr int TM = DH / 16;
+    constexpr int QPR = DH / kVec;  // copies per row and array
     const int tid = threadIdx.x, i0 = (tid / 16) * TM, j0 = (tid % 16) * TM;
-    const int split = blockIdx.x, gh = blockIdx.y, g = gh / pr.nh, h = gh % pr.nh;
+    const int split = blockIdx.x, h = blockIdx.y;
     const int64_t nrows = pr.B * pr.T;
     const int64_t r0 = split * rows_per_split;
     const int64_t r1 = r0 + rows_per_split < nrows ? r0 + rows_per_split : nrows;
-    float acc[TM][TM];
+    float acc[3][TM][TM];
 #pragma unroll
-    for (int a = 0; a < TM; ++a)
+    for (int g = 0; g < 3; ++g)
 #pragma unroll
-        for (int c = 0; c < TM; ++c) acc[a][c] = 0.0f;
-    for (int64_t rb = r0; rb < r1; rb += kURows) {
-        for (int idx = tid; idx < kURows * DH; idx += kThreads) {
-            const int rr = idx / DH, k = idx - rr * DH;
+        for (int a = 0; a < TM; ++a)
+#pragma unroll
+            for (int c = 0; c < TM; ++c) acc[g][a][c] = 0.0f;
+
+    // start the copies of rows rb .. rb + kURows - 1 into buffer `buf`
+    auto issue = [&](int64_t rb, int buf) {
+        for (int idx = tid; idx < kURows * 4 * QPR; idx += kThreads) {
+            const int rr = idx / (4 * QPR), rem = idx - rr * (4 * QPR), arr = rem / QPR, q = rem - arr * QPR;
             const int64_t row = rb + rr;
-            float e = 0.0f, sv = 0.0f;
+            float* dst = arr < 3 ? &sm.E[buf][arr][rr][q * kVec] : &sm.S[buf][rr][q * kVec];
+            const float* src = nullptr;
             if (row < r1) {
-                const int64_t bb = row / pr.T, t = row - bb * pr.T, c = (int64_t)h * DH + k;
-                e = g < 2 ? pr.dpx[((bb * pr.T + t) * 3 + g) * pr.D + c] : pr.ec[(bb * pr.T + t) * pr.D + c];
-                sv = t >= 1 ? pr.Hold[(bb * pr.T + t - 1) * pr.D + c] : (pr.h0 ? pr.h0[bb * pr.D + c] : 0.0f);
+                const int64_t bb = row / pr.T, t = row - bb * pr.T, c = (int64_t)h * DH + q * kVec;
+                if (arr < 2)
+                    src = pr.dpx + ((bb * pr.T + t) * 3 + arr) * pr.D + c;
+                else if (arr == 2)
+                    src = pr.ec + (bb * pr.T + t) * pr.D + c;
+                else
+                    src = t >= 1 ? pr.Hold + (bb * pr.T + t - 1) * pr.D + c : (pr.h0 ? pr.h0 + bb * pr.D + c : nullptr);
             }
-            Es[rr][k] = e;
-            Ss[rr][k] = sv;
+            if (src) {
+                cp_async<kVec * 4>(dst, src);
+            } else {
+#pragma unroll
+                for (int v = 0; v < kVec; ++v) dst[v] = 0.0f;
+            }
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+
+    int buf = 0;
+    if (r0 < r1) issue(r0, 0);
+    for (int64_t rb = r0; rb < r1; rb += kURows, buf ^= 1) {
+        if (rb + kURows < r1) {
+            issue(rb + kURows, buf ^ 1);
+            asm volatile("cp.async.wait_group 1;" ::: "memory");
+        } else {
+            asm volatile("cp.async.wait_group 0;" ::: "memory");
         }
         __syncthreads();
 #pragma unroll 4
         for (int rr = 0; rr < kURows; ++rr) {
-            float ev[TM], sw[TM];
+            float sw[TM];
 #pragma unroll
-            for (int a = 0; a < TM; ++a) ev[a] = Es[rr][i0 + a];
+            for (int c = 0; c < TM; ++c) sw[c] = sm.S[buf][rr][j0 + c];
 #pragma unroll
-            for (int c = 0; c < TM; ++c) sw[c] = Ss[rr][j0 + c];
+            for (int g = 0; g < 3; ++g) {
+                float ev[TM];
 #pragma unroll
-            for (int a = 0; a < TM; ++a)
+                for (int a = 0; a < TM; ++a) ev[a] = sm.E[buf][g][rr][i0 + a];
 #pragma unroll
-                for (int c = 0; c < TM; ++c) acc[a][c] = __fmaf_rn(ev[a], sw[c], acc[a][c]);
+                for (int a = 0; a < TM; ++a)
+#pragma unroll
+                    for (int c = 0; c < TM; ++c) acc[g][a][c] = __fmaf_rn(ev[a], sw[c], acc[g][a][c]);
+            }
         }
-        __syncthreads();
+        __syncthreads();  // the buffer is refilled by the next batch's copies
     }
-    float* out = part + ((int64_t)split * gridDim.y + gh) * DH * DH;
 #pragma unroll
-    for (int a = 0; a < TM; ++a)
+    for (int g = 0; g < 3; ++g) {
+        float* out = part + ((int64_t)split * 3 * gridDim.y + (int64_t)g * gridDim.y + h) * DH * DH;
 #pragma unroll
-        for (int c = 0; c < TM; ++c) out[(i0 + a) * DH + j0 + c] = acc[a][c];
+        for (int a = 0; a < TM; ++a)
+#pragma unroll
+            for (int c = 0; c < TM; ++c) out[(i0 + a) * DH + j0 + c] = acc[g][a][c];
+    }
 }
 
 __global__ void head_dU_reduce_kernel(const float* part, int nsplit, int64_t n, float* dU) {
@@ -1386,7 +1439,11 @@ cudaError_t launch_all(const Plan& pl, Params pr, float* H_out, float* Hbuf, int
     // has no M below 64) on mma.sync
     constexpr bool kTc = DH == tc::kD;
     const size_t smemA = kTc ? sizeof(tc::Smem) : sizeof(SmemA<DH>), smemR = sizeof(SmemA<DH>);
-    cudaError_t e = kTc ? set_smem(head_chunk_tc_kernel<PxT>, smemA) : set_smem(head_chunk_kernel<DH, PxT, false>, smemA);
+    cudaError_t e;
+    if constexpr (kTc)
+        e = set_smem(head_chunk_tc_kernel<PxT>, smemA);
+    else
+        e = set_smem(head_chunk_kernel<DH, PxT, false>, smemA);
     if (e == cudaSuccess) e = set_smem(head_chunk_kernel<DH, PxT, true>, smemR);
     if (e != cudaSuccess) return e;
     const unsigned ntask = (unsigned)(pl.nSeq * pl.nChunks);
@@ -1431,8 +1488,12 @@ bool make_bplan(int64_t B, int64_t T, int64_t D, int nh, BPlan& pl) {
     pl.nSeq = fp.nSeq;
     const size_t ntask = (size_t)pl.nSeq * pl.nChunks, d = pl.d;
     const int64_t rows = B * T;
+    // splits of at least 256 rows, at most 64, and about one wave of
+    // blocks (two per SM on the 148 SMs) over the heads
     pl.nsplit = (int)(rows > 0 ? (rows + 255) / 256 : 1);
     if (pl.nsplit > 64) pl.nsplit = 64;
+    const int wave = nh < 296 ? 296 / nh : 1;
+    if (pl.nsplit > wave) pl.nsplit = wave;
     pl.rows_per_split = rows > 0 ? (rows + pl.nsplit - 1) / pl.nsplit : 1;
     pl.off_P = 256;
     pl.off_q = align256(pl.off_P + ntask * d * d * sizeof(float));
@@ -1449,7 +1510,11 @@ cudaError_t launch_bwd(const BPlan& pl, const Params& pr, float* dU, cudaStream_
     // head width 64: the products on tcgen05, as in the forward
     constexpr bool kTc = DH == tc::kD;
     const size_t smemP = kTc ? sizeof(tc::SmemB) : sizeof(SmemB<DH>);
-    cudaError_t e = kTc ? set_smem(head_bwd_tc_kernel<PxT>, smemP) : set_smem(head_bwd_kernel<DH, PxT>, smemP);
+    cudaError_t e;
+    if constexpr (kTc)
+        e = set_smem(head_bwd_tc_kernel<PxT>, smemP);
+    else
+        e = set_smem(head_bwd_kernel<DH, PxT>, smemP);
     if (e != cudaSuccess) return e;
     const unsigned ntask = (unsigned)(pl.nSeq * pl.nChunks);
     if constexpr (kTc)
@@ -1461,8 +1526,19 @@ cudaError_t launch_bwd(const BPlan& pl, const Params& pr, float* dU, cudaStream_
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (dU) {
         float* part = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(pr.status) + pl.off_part);
-        head_dU_kernel<DH><<<dim3((unsigned)pl.nsplit, (unsigned)(3 * pr.nh)), kThreads, 0, st>>>(
-            pr, pl.rows_per_split, part);
+        // 16-byte copies need every source row 16-byte aligned: the
+        // workspace's lambda * gamma always is, dL/dpx, H and h0 are checked
+        const bool vec = ((reinterpret_cast<uintptr_t>(pr.dpx) | reinterpret_cast<uintptr_t>(pr.Hold) |
+                           reinterpret_cast<uintptr_t>(pr.h0)) & 15) == 0;
+        const size_t smemU = sizeof(SmemU<DH>);
+        const dim3 grid((unsigned)pl.nsplit, (unsigned)pr.nh);
+        if (vec) {
+            if ((e = set_smem(head_dU_kernel<DH, 4>, smemU)) != cudaSuccess) return e;
+            head_dU_kernel<DH, 4><<<grid, kThreads, smemU, st>>>(pr, pl.rows_per_split, part);
+        } else {
+            if ((e = set_smem(head_dU_kernel<DH, 1>, smemU)) != cudaSuccess) return e;
+            head_dU_kernel<DH, 1><<<grid, kThreads, smemU, st>>>(pr, pl.rows_per_split, part);
+        }
         const int64_t n = (int64_t)3 * pr.nh * DH * DH;
         head_dU_reduce_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(part, pl.nsplit, n, dU);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
