@@ -363,12 +363,14 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
 #pragma unroll
                             for (int s = 0; s < S; ++s) spv[s] = sp[s][v];
                             Cell::elem(pg, wr[v], spv, f, A, be);
-                            if (!rvalid) {
-#pragma unroll
-                                for (int a = 0; a < S * S; ++a) A[a] = (a % (S + 1) == 0) ? 1.0f : 0.0f;
-#pragma unroll
-                                for (int s = 0; s < S; ++s) be[s] = 0.0f;
-                            } else if (want_resid) {
+                            // rows past the end of the sequence (and channels
+                            // past D) keep their elements: in time order they
+                            // come after every valid row of their channel, so
+                            // they reach only scan values nobody reads (the
+                            // sequence's last inclusive state and h rows that
+                            // are never stored); their pre-activations are
+                            // zero-filled, so the values stay finite
+                            if (rvalid && want_resid) {
 #pragma unroll
                                 for (int s = 0; s < S; ++s) res = nanmax_f(res, fabsf(h[r][s][v] - f[s]));
                             }
