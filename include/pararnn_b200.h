@@ -247,9 +247,9 @@ pararnn_status pararnn_newton_forward_host(pararnn_cell cell, int64_t B, int64_t
  * Returns the workspace size for these sizes, or 0 when they are invalid
  * (d not in {16, 32, 64}, D not a multiple of n_heads, K outside 1..64, B*T
  * at or above 2^31).  It holds a second iterate buffer (K >= 2), each
- * chunk's d x d Jacobian product (chunks of 64 steps) and six float row
+ * chunk's d x d Jacobian product (chunks of 128 steps) and six float row
  * factors per element, which the chunk pass forms and the re-walk reads:
- * about B*T*D*4*7 + B*T*n_heads*(d+2)*d*4/64 bytes. */
+ * about B*T*D*4*7 + B*T*n_heads*(d+2)*d*4/128 bytes. */
 size_t pararnn_head_gru_workspace_bytes(int64_t B, int64_t T, int64_t D, int n_heads, int K);
 
 /* K Newton iterations of the head-wise GRU; H_out = h^(K).
@@ -281,7 +281,7 @@ pararnn_status pararnn_head_gru_forward(int64_t B, int64_t T, int64_t D, int n_h
  * NULL; all float32 device memory owned by the caller.  dL_dU is summed in a
  * fixed order (no floating-point atomics): repeated calls give identical
  * bits.  Returns the workspace size, or 0 for invalid sizes (as for the
- * forward): about B*T*D*4*6 + B*T*n_heads*(d+2)*d*4/64 bytes (lambda * gamma
+ * forward): about B*T*D*4*6 + B*T*n_heads*(d+2)*d*4/128 bytes (lambda * gamma
  * and five float row factors per element, and the chunk products) plus
  * 12 n_heads d^2 * min(64, B*T/256) * 4 bytes of split partials. */
 size_t pararnn_head_gru_backward_workspace_bytes(int64_t B, int64_t T, int64_t D, int n_heads);

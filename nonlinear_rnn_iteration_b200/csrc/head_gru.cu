@@ -41,7 +41,7 @@ bool pointer_on_device(const void* p);      // pararnn_abi.cu
 namespace hg {
 
 constexpr int kThreads = 256;
-constexpr int kChunk = 64;  // steps per chunk
+constexpr int kChunk = 128;  // steps per chunk
 constexpr int kMaxK = 64;
 // row factors stored per step: forward h^(k)_t, F_t, 1 - z, alpha, beta,
 // gamma; backward 1 - z, alpha, beta, z (1 - c^2), gamma
@@ -410,7 +410,7 @@ namespace tc {
 
 constexpr int kD = 64;
 constexpr uint32_t kTmemCols = 64;
-constexpr uint64_t kWaitNs = 1000000000ull;  // 1 s: far beyond a 64-step product chain
+constexpr uint64_t kWaitNs = 1000000000ull;  // 1 s: far beyond one step's product
 
 struct Smem {
     float Ahi[2][kD * kD];  // A_t, K-major, two steps in turn

@@ -35,9 +35,11 @@ CASES = [  # (B, T, D, n_heads, K)
     (2, 40, 48, 3, 1),
     (1, 130, 128, 2, 3),
     (2, 64, 256, 4, 2),
-    # head width 64 (the tcgen05 products): one step, a last chunk of one step
+    # head width 64 (the tcgen05 products): one step, a last chunk of one
+    # step, two whole chunks of 128 steps
     (1, 1, 64, 1, 1),
-    (3, 65, 64, 1, 2),
+    (3, 129, 64, 1, 2),
+    (1, 256, 128, 2, 2),
 ]
 
 
@@ -137,7 +139,7 @@ BWD_CASES = [  # (B, T, D, n_heads, K)
     (2, 40, 64, 2, 1),
     (1, 200, 128, 2, 3),
     (1, 1, 64, 1, 1),
-    (3, 65, 64, 1, 2),
+    (3, 129, 64, 1, 2),
 ]
 
 
