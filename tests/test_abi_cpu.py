@@ -112,3 +112,55 @@ def test_probe_rejects_bad_arguments():
     assert binding.pararnn_probe_wait_timeout(None, 1024, 1000, None) == binding.EINVAL
     assert binding.pararnn_probe_wait_timeout(1 << 40, 16, 1000, None) == binding.EINVAL
     assert binding.pararnn_probe_wait_timeout(1 << 40, 1024, 0, None) == binding.EINVAL
+
+
+def test_head_gru_workspace_bytes():
+    f, fb = binding.pararnn_head_gru_workspace_bytes, binding.pararnn_head_gru_backward_workspace_bytes
+    # invalid: head width 8, D not a multiple of n_heads, K outside 1..64
+    assert f(1, 16, 64, 8, 2) == 0
+    assert f(1, 16, 100, 3, 2) == 0
+    assert f(1, 16, 128, 2, 0) == 0 and f(1, 16, 128, 2, 65) == 0
+    assert fb(1, 16, 64, 8) == 0 and fb(1, 16, 100, 3) == 0
+    B, T, D, nh = 2, 300, 128, 2
+    n = B * T * D * 4
+    one, two = f(B, T, D, nh, 1), f(B, T, D, nh, 2)
+    # six float row factors per element; K >= 2 adds the second iterate buffer
+    assert one >= 6 * n and two - one >= n
+    assert f(B, T, D, nh, 3) == two
+    assert f(B, 2 * T, D, nh, 2) > two
+    # lambda * gamma and five float row factors per element, plus the products
+    assert fb(B, T, D, nh) >= 6 * n
+    assert f(0, T, D, nh, 2) >= 256 and fb(0, T, D, nh) >= 256
+
+
+def test_head_gru_rejects_bad_arguments():
+    fake = 1 << 40  # never dereferenced: the checks fail first
+    ws = binding.pararnn_head_gru_workspace_bytes(1, 8, 64, 1, 2)
+    fwd = binding.pararnn_head_gru_forward
+    assert fwd(1, 8, 64, 1, binding.F32, fake, fake, None, 0, fake, fake, ws, None, None) == binding.EINVAL  # K
+    assert fwd(1, 8, 48, 2, binding.F32, fake, fake, None, 2, fake, fake, ws, None, None) == binding.EINVAL  # d = 24
+    assert fwd(1, 8, 64, 1, 7, fake, fake, None, 2, fake, fake, ws, None, None) == binding.EINVAL  # dtype
+    assert fwd(1, 8, 64, 1, binding.F32, fake, fake, None, 2, fake, None, ws, None, None) == binding.EINVAL
+    assert fwd(1, 8, 64, 1, binding.F32, fake, fake, None, 2, fake, fake, ws - 1, None, None) == binding.EINVAL
+    assert binding.pararnn_last_error() != ""
+    wsb = binding.pararnn_head_gru_backward_workspace_bytes(1, 8, 64, 1)
+    bwd = binding.pararnn_head_gru_backward
+    assert bwd(1, 8, 64, 1, binding.F32, fake, fake, None, fake, fake, fake, None, None, fake, wsb - 1,
+               None) == binding.EINVAL
+    assert bwd(1, 8, 60, 1, binding.F32, fake, fake, None, fake, fake, fake, None, None, fake, 1 << 30,
+               None) == binding.EINVAL  # d = 60
+
+
+def test_host_path_workspace_bytes():
+    f = binding.pararnn_newton_forward_host_workspace_bytes
+    gru = 1
+    assert f(gru, 8, 1024, 256, 3, 7, 1) == 0  # dtype
+    assert f(gru, 8, 1024, 256, 3, binding.F32, 0) == 0  # rows per slice
+    assert f(9, 8, 1024, 256, 3, binding.F32, 1) == 0  # cell
+    one, two = f(gru, 8, 1024, 256, 3, binding.F32, 1), f(gru, 8, 1024, 256, 3, binding.F32, 2)
+    # three device slots, each holding one slice's pre-activations, H and solver workspace
+    row_px, row_h = 1024 * 3 * 256 * 4, 1024 * 256 * 4
+    assert one >= 3 * (row_px + row_h) and two - one >= 3 * (row_px + row_h)
+    assert f(gru, 8, 1024, 256, 3, binding.BF16, 1) < one  # bf16 slices are smaller
+    # a slice never exceeds the batch
+    assert f(gru, 2, 1024, 256, 3, binding.F32, 5) == f(gru, 2, 1024, 256, 3, binding.F32, 2)
