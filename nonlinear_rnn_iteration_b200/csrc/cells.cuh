@@ -69,14 +69,19 @@ struct CellGRU {
     static __device__ __forceinline__ void elem(const float (&p)[G], const float (&w)[G], const float (&sp)[S],
                                                 float (&f)[S], float (&A)[S * S], float (&beta)[S]) {
         const float h = sp[0];
-        float z, r, c, Gz, Gr, Gc;
-        gates(p, w, h, z, r, c, Gz, Gr, Gc);
-        f[0] = __fmaf_rn(z, c - h, h);  // (1 - z) h + z c
-        // df/dh: the direct (1 - z) plus each gate's pre-activation term
-        float a = 1.0f - z;
-        a = __fmaf_rn(w[0], Gz, a);
-        a = __fmaf_rn(w[1], Gr, a);
-        a = __fmaf_rn(w[2] * r, Gc, a);
+        const float z = sigmoid_f(__fmaf_rn(w[0], h, p[0]));
+        const float r = sigmoid_f(__fmaf_rn(w[1], h, p[1]));
+        const float wr = w[2] * r;
+        const float c = tanh_f(__fmaf_rn(wr, h, p[2]));
+        const float ch = c - h;
+        f[0] = __fmaf_rn(z, ch, h);  // (1 - z) h + z c
+        // df/dh = (1 - z) + a_z G_z + a_r G_r + a_c r G_c with G_z = (c - h) z (1 - z),
+        // G_c = z (1 - c^2), G_r = G_c a_c h r (1 - r); the last two share G_c a_c:
+        //   a_r G_r + a_c r G_c = G_c a_c (a_r h r (1 - r) + r)
+        const float gcw = z * __fmaf_rn(-c, c, 1.0f) * w[2];
+        const float tr = __fmaf_rn(w[1] * h, __fmaf_rn(-r, r, r), r);
+        float a = __fmaf_rn(w[0], ch * __fmaf_rn(-z, z, z), 1.0f - z);
+        a = __fmaf_rn(gcw, tr, a);
         A[0] = a;
         beta[0] = __fmaf_rn(-a, h, f[0]);
     }
