@@ -126,7 +126,7 @@ struct CellLSTM {
         f[1] = o * tanh_f(cn);
     }
     struct Terms {
-        float i, fg, o, g, cn, tn, dcn_dh;
+        float i, fg, o, g, ig, cn, tn, dcn_dh;
     };
     static __device__ __forceinline__ Terms terms(const float (&p)[G], const float (&w)[G], float c, float h) {
         Terms q;
@@ -134,7 +134,8 @@ struct CellLSTM {
         q.fg = sigmoid_f(__fmaf_rn(w[1], h, p[1]) + 1.0f);
         q.o = sigmoid_f(__fmaf_rn(w[2], h, p[2]));
         q.g = tanh_f(__fmaf_rn(w[3], h, p[3]));
-        q.cn = __fmaf_rn(q.fg, c, q.i * q.g);
+        q.ig = q.i * q.g;
+        q.cn = __fmaf_rn(q.fg, c, q.ig);
         q.tn = tanh_f(q.cn);
         // dc'/dh through the f, i and c gates' pre-activations
         float d = c * (q.fg - q.fg * q.fg) * w[1];
@@ -154,7 +155,9 @@ struct CellLSTM {
         A[1] = q.dcn_dh;                                        // dc'/dh
         A[2] = k * q.fg;                                        // dh'/dc
         A[3] = __fmaf_rn((q.o - q.o * q.o) * w[2], q.tn, k * q.dcn_dh);  // dh'/dh
-        beta[0] = f[0] - __fmaf_rn(A[0], c, A[1] * h);
+        // beta = f - A (c, h): for the c row, c' - f c = i g exactly in real
+        // arithmetic, so beta_c = i g - (dc'/dh) h
+        beta[0] = __fmaf_rn(-A[1], h, q.ig);
         beta[1] = f[1] - __fmaf_rn(A[2], c, A[3] * h);
     }
     static __device__ __forceinline__ void bwd(const float (&p)[G], const float (&w)[G], const float (&sp)[S],
