@@ -80,14 +80,19 @@ __device__ __forceinline__ float ldp(const PxT* p) { return PxTraits<PxT>::cvt(*
 // shuffles, and every thread of the row then evaluates the row's gates (the
 // redundancy is cheaper than another round through shared memory).  Vectors
 // over the head's state live in shared memory in the permuted order
-// vpos(m) = (m % TPR) * SEG + m / TPR, so a thread's SEG elements are
-// contiguous.
+// vpos(m) = (m % TPR) * SEGP + m / TPR, so a thread's SEG elements are
+// contiguous.  With 4 threads per row (d = 64) each thread's segment is
+// padded by 4 floats (SEGP = 20), so that the four 16-byte loads of a
+// row's threads fall on four different bank groups; the narrower heads'
+// segments already do.
 template <int DH>
 struct Geo {
     static constexpr int TPR = kThreads / DH;
     static constexpr int SEG = DH / TPR;
+    static constexpr int SEGP = SEG + (SEG == 16 ? 4 : 0);  // padded segment
+    static constexpr int VLEN = TPR * SEGP;                 // floats of a permuted vector
     static_assert(TPR * SEG == DH && TPR <= 32, "one row's threads share a warp");
-    static __device__ __forceinline__ int vpos(int m) { return (m % TPR) * SEG + m / TPR; }
+    static __device__ __forceinline__ int vpos(int m) { return (m % TPR) * SEGP + m / TPR; }
 };
 
 template <int DH>
@@ -200,8 +205,8 @@ template <int DH>
 struct SmemA {
     float AT[2][DH][DH + kPadA];  // A_t transposed (AT[m][i] = A_t[i][m]), two steps in turn
     uint2 Pm[2][DH][DH + kPad];   // running product, row-major, {hi, lo} TF32 pairs
-    float sv[2][DH];              // h^(k) rows, permuted (vpos), two steps in turn
-    float dv[2][DH];              // delta rows, permuted, two steps in turn
+    float sv[2][Geo<DH>::VLEN];   // h^(k) rows, permuted (vpos), two steps in turn
+    float dv[2][Geo<DH>::VLEN];   // delta rows, permuted, two steps in turn
 };
 
 __device__ __forceinline__ uint2 split_tf32(float x) {
@@ -282,7 +287,7 @@ __device__ __forceinline__ void matmul_tf32x3(const float (*AT)[DH + kPadA], con
 template <int DH, typename PxT, bool kResidOnly>
 __global__ void __launch_bounds__(kThreads, 2) head_chunk_kernel(const Params pr) {
     using Gm = Geo<DH>;
-    constexpr int TPR = Gm::TPR, SEG = Gm::SEG;
+    constexpr int TPR = Gm::TPR, SEG = Gm::SEG, SEGP = Gm::SEGP;
     extern __shared__ __align__(16) unsigned char smem_raw[];
     auto& sm = *reinterpret_cast<SmemA<DH>*>(smem_raw);
     const int tid = threadIdx.x, i = tid / TPR, qt = tid % TPR;
@@ -313,7 +318,7 @@ __global__ void __launch_bounds__(kThreads, 2) head_chunk_kernel(const Params pr
         float uz = 0.0f, ur = 0.0f, uc = 0.0f;
 #pragma unroll
         for (int s = 0; s < SEG; ++s) {
-            const float x = sm.sv[p][qt * SEG + s];
+            const float x = sm.sv[p][qt * SEGP + s];
             uz = __fmaf_rn(U.z[s], x, uz);
             ur = __fmaf_rn(U.r[s], x, ur);
             uc = __fmaf_rn(U.c[s], x, uc);
@@ -334,7 +339,7 @@ __global__ void __launch_bounds__(kThreads, 2) head_chunk_kernel(const Params pr
                 a = __fmaf_rn(L.be, U.r[s], a);
                 a = __fmaf_rn(L.ga, U.c[s], a);
                 sm.AT[p][m][i] = a;
-                dp = __fmaf_rn(a, sm.dv[p][qt * SEG + s], dp);
+                dp = __fmaf_rn(a, sm.dv[p][qt * SEGP + s], dp);
             }
             dp = row_sum<DH>(dp);
             if (qt == 0) sm.dv[p ^ 1][Gm::vpos(i)] = dp - L.F;
@@ -417,8 +422,8 @@ struct Smem {
     float Alo[2][kD * kD];
     float Phi[kD * kD];     // running product, MN-major
     float Plo[kD * kD];
-    float sv[2][kD];        // h^(k) rows, permuted (vpos), two steps in turn
-    float dv[2][kD];        // delta rows, permuted, two steps in turn
+    float sv[2][Geo<kD>::VLEN];  // h^(k) rows, permuted (vpos), two steps in turn
+    float dv[2][Geo<kD>::VLEN];  // delta rows, permuted, two steps in turn
     uint64_t bar;           // the product of this step is done
     uint32_t tmem;          // tensor-memory base address from tcgen05.alloc
     int abort;              // a wait ran out: stop issuing, keep the barrier count
@@ -488,7 +493,7 @@ __device__ __forceinline__ float tf32_head(float x) {
 template <typename PxT>
 __global__ void __launch_bounds__(kThreads, 2) head_chunk_tc_kernel(const Params pr) {
     using Gm = Geo<tc::kD>;
-    constexpr int TPR = Gm::TPR, SEG = Gm::SEG, DH = tc::kD;
+    constexpr int TPR = Gm::TPR, SEG = Gm::SEG, SEGP = Gm::SEGP, DH = tc::kD;
     extern __shared__ __align__(16) unsigned char smem_raw[];
     auto& sm = *reinterpret_cast<tc::Smem*>(smem_raw);
     volatile int& abort_flag = sm.abort;
@@ -534,7 +539,7 @@ __global__ void __launch_bounds__(kThreads, 2) head_chunk_tc_kernel(const Params
         float uz = 0.0f, ur = 0.0f, uc = 0.0f;
 #pragma unroll
         for (int s = 0; s < SEG; ++s) {
-            const float x = sm.sv[p][qt * SEG + s];
+            const float x = sm.sv[p][qt * SEGP + s];
             uz = __fmaf_rn(U.z[s], x, uz);
             ur = __fmaf_rn(U.r[s], x, ur);
             uc = __fmaf_rn(U.c[s], x, uc);
@@ -560,7 +565,7 @@ __global__ void __launch_bounds__(kThreads, 2) head_chunk_tc_kernel(const Params
             const float hi = tc::tf32_head(a);
             ahi[tc::a_idx(i, m)] = hi;
             alo[tc::a_idx(i, m)] = a - hi;
-            dp = __fmaf_rn(a, sm.dv[p][qt * SEG + s], dp);
+            dp = __fmaf_rn(a, sm.dv[p][qt * SEGP + s], dp);
         }
         dp = row_sum<DH>(dp);
         if (qt == 0) {
@@ -726,8 +731,8 @@ __global__ void __launch_bounds__(64) head_carry_kernel(const Params pr) {
 template <int DH>
 __global__ void __launch_bounds__(kThreads, 2) head_walk_kernel(const Params pr) {
     using Gm = Geo<DH>;
-    constexpr int TPR = Gm::TPR, SEG = Gm::SEG;
-    __shared__ float dv[2][DH];  // delta rows, permuted, two steps in turn
+    constexpr int TPR = Gm::TPR, SEG = Gm::SEG, SEGP = Gm::SEGP;
+    __shared__ float dv[2][Gm::VLEN];  // delta rows, permuted, two steps in turn
     const int tid = threadIdx.x, i = tid / TPR, qt = tid % TPR;
     const int64_t task = blockIdx.x;
     const int64_t seq = task / pr.nChunks;
@@ -757,7 +762,7 @@ __global__ void __launch_bounds__(kThreads, 2) head_walk_kernel(const Params pr)
         float vz = 0.0f, vr = 0.0f, vc = 0.0f;
 #pragma unroll
         for (int s = 0; s < SEG; ++s) {
-            const float y = dv[par][qt * SEG + s];
+            const float y = dv[par][qt * SEGP + s];
             vz = __fmaf_rn(U.z[s], y, vz);
             vr = __fmaf_rn(U.r[s], y, vr);
             vc = __fmaf_rn(U.c[s], y, vc);
@@ -832,9 +837,9 @@ template <int DH>
 struct SmemB {
     float AT[2][DH][DH + kPadA];  // AT[m][i] = A_t[i][m] = (A_t^T)[m][i], two steps in turn
     uint2 Pm[2][DH][DH + kPad];   // the running product of transposed Jacobians ({hi, lo} pairs)
-    float sv[2][DH];              // h_{t-1} rows for the row work (permuted)
-    float gv[2][DH];              // g_t rows (permuted)
-    float mv[2][DH];              // mu rows (permuted)
+    float sv[2][Geo<DH>::VLEN];   // h_{t-1} rows for the row work (permuted)
+    float gv[2][Geo<DH>::VLEN];   // g_t rows (permuted)
+    float mv[2][Geo<DH>::VLEN];   // mu rows (permuted)
 };
 
 // step t's backward row factors of row i, for the walk
@@ -855,11 +860,11 @@ __device__ __forceinline__ void store_brow_factors(const Params& pr, int64_t seq
 template <int DH>
 __device__ __forceinline__ void bwd_row_work(SmemB<DH>& sm, const RowU<DH>& U, const BStepIn& in, int p, int i,
                                              int qt, const Params& pr, int64_t seq, int64_t t) {
-    constexpr int TPR = Geo<DH>::TPR, SEG = Geo<DH>::SEG;
+    constexpr int TPR = Geo<DH>::TPR, SEG = Geo<DH>::SEG, SEGP = Geo<DH>::SEGP;
     float uz = 0.0f, ur = 0.0f, uc = 0.0f;
 #pragma unroll
     for (int s = 0; s < SEG; ++s) {
-        const float x = sm.sv[p][qt * SEG + s];
+        const float x = sm.sv[p][qt * SEGP + s];
         uz = __fmaf_rn(U.z[s], x, uz);
         ur = __fmaf_rn(U.r[s], x, ur);
         uc = __fmaf_rn(U.c[s], x, uc);
@@ -892,12 +897,12 @@ __device__ __forceinline__ void bwd_row_work(SmemB<DH>& sm, const RowU<DH>& U, c
 // mu_t[m] = sum_i AT[p][m][i] (g_t[i] + mu_{t+1}[i]) for thread (m, qt)
 template <int DH>
 __device__ __forceinline__ float bwd_mu(const SmemB<DH>& sm, int p, int m, int qt) {
-    constexpr int TPR = Geo<DH>::TPR, SEG = Geo<DH>::SEG;
+    constexpr int TPR = Geo<DH>::TPR, SEG = Geo<DH>::SEG, SEGP = Geo<DH>::SEGP;
     float acc = 0.0f;
 #pragma unroll
     for (int s = 0; s < SEG; ++s) {
         const int i = qt + TPR * s;
-        const float lam = sm.gv[p][qt * SEG + s] + sm.mv[p ^ 1][qt * SEG + s];
+        const float lam = sm.gv[p][qt * SEGP + s] + sm.mv[p ^ 1][qt * SEGP + s];
         acc = __fmaf_rn(sm.AT[p][m][i], lam, acc);
     }
     return row_sum<DH>(acc);
@@ -991,8 +996,8 @@ struct ColU {
 template <int DH>
 __global__ void __launch_bounds__(kThreads, 2) head_bwd_walk_kernel(const Params pr) {
     using Gm = Geo<DH>;
-    constexpr int TPR = Gm::TPR, SEG = Gm::SEG;
-    __shared__ float wv[2][3][DH];  // alpha lambda, beta lambda, gamma lambda (permuted), two steps in turn
+    constexpr int TPR = Gm::TPR, SEG = Gm::SEG, SEGP = Gm::SEGP;
+    __shared__ float wv[2][3][Gm::VLEN];  // alpha lambda, beta lambda, gamma lambda (permuted), two steps in turn
     const int tid = threadIdx.x, i = tid / TPR, qt = tid % TPR;
     const int64_t task = blockIdx.x;
     const int64_t seq = task / pr.nChunks;
@@ -1045,9 +1050,9 @@ __global__ void __launch_bounds__(kThreads, 2) head_bwd_walk_kernel(const Params
         float sz = 0.0f, sr = 0.0f, sc = 0.0f;
 #pragma unroll
         for (int s = 0; s < SEG; ++s) {
-            sz = __fmaf_rn(UT.z[s], wv[par][0][qt * SEG + s], sz);
-            sr = __fmaf_rn(UT.r[s], wv[par][1][qt * SEG + s], sr);
-            sc = __fmaf_rn(UT.c[s], wv[par][2][qt * SEG + s], sc);
+            sz = __fmaf_rn(UT.z[s], wv[par][0][qt * SEGP + s], sz);
+            sr = __fmaf_rn(UT.r[s], wv[par][1][qt * SEGP + s], sr);
+            sc = __fmaf_rn(UT.c[s], wv[par][2][qt * SEGP + s], sc);
         }
         sz = row_sum<DH>(sz);
         sr = row_sum<DH>(sr);
@@ -1080,9 +1085,9 @@ struct SmemB {
     float Alo[2][kD * kD];
     float Phi[kD * kD];     // running product, MN-major
     float Plo[kD * kD];
-    float sv[2][kD];        // h_{t-1} rows for the row work (permuted)
-    float gv[2][kD];        // g_t rows (permuted)
-    float mv[2][kD];        // mu rows (permuted)
+    float sv[2][Geo<kD>::VLEN];  // h_{t-1} rows for the row work (permuted)
+    float gv[2][Geo<kD>::VLEN];  // g_t rows (permuted)
+    float mv[2][Geo<kD>::VLEN];  // mu rows (permuted)
     uint64_t bar;
     uint32_t tmem;
     int abort;
@@ -1103,7 +1108,7 @@ __device__ __forceinline__ void mma_t(uint32_t d, uint64_t a, uint64_t b, uint32
 template <typename PxT>
 __global__ void __launch_bounds__(kThreads, 2) head_bwd_tc_kernel(const Params pr) {
     using Gm = Geo<tc::kD>;
-    constexpr int TPR = Gm::TPR, SEG = Gm::SEG, DH = tc::kD;
+    constexpr int TPR = Gm::TPR, SEG = Gm::SEG, SEGP = Gm::SEGP, DH = tc::kD;
     extern __shared__ __align__(16) unsigned char smem_raw[];
     auto& sm = *reinterpret_cast<tc::SmemB*>(smem_raw);
     volatile int& abort_flag = sm.abort;
@@ -1147,7 +1152,7 @@ __global__ void __launch_bounds__(kThreads, 2) head_bwd_tc_kernel(const Params p
         float uz = 0.0f, ur = 0.0f, uc = 0.0f;
 #pragma unroll
         for (int s = 0; s < SEG; ++s) {
-            const float x = sm.sv[p][qt * SEG + s];
+            const float x = sm.sv[p][qt * SEGP + s];
             uz = __fmaf_rn(U.z[s], x, uz);
             ur = __fmaf_rn(U.r[s], x, ur);
             uc = __fmaf_rn(U.c[s], x, uc);
@@ -1221,7 +1226,7 @@ __global__ void __launch_bounds__(kThreads, 2) head_bwd_tc_kernel(const Params p
 #pragma unroll
             for (int s = 0; s < SEG; ++s) {
                 const int k = qt + TPR * s;
-                const float lam = sm.gv[p][qt * SEG + s] + sm.mv[p ^ 1][qt * SEG + s];
+                const float lam = sm.gv[p][qt * SEGP + s] + sm.mv[p ^ 1][qt * SEGP + s];
                 const int o = tc::p_idx(k, i);
                 acc = __fmaf_rn(sm.Ahi[p][o] + sm.Alo[p][o], lam, acc);
             }
