@@ -36,10 +36,12 @@ CASES = [  # (B, T, D, n_heads, K)
     (1, 130, 128, 2, 3),
     (2, 64, 256, 4, 2),
     # head width 64 (the tcgen05 products): one step, a last chunk of one
-    # step, two whole chunks of 128 steps
+    # step, two whole chunks of 128 steps, three chunks (the first chunk's
+    # product then carries into the last)
     (1, 1, 64, 1, 1),
     (3, 129, 64, 1, 2),
     (1, 256, 128, 2, 2),
+    (1, 300, 64, 1, 3),
 ]
 
 
@@ -140,6 +142,7 @@ BWD_CASES = [  # (B, T, D, n_heads, K)
     (1, 200, 128, 2, 3),
     (1, 1, 64, 1, 1),
     (3, 129, 64, 1, 2),
+    (1, 300, 64, 1, 3),
 ]
 
 
