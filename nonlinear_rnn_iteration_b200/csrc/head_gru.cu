@@ -723,10 +723,10 @@ __global__ void __launch_bounds__(64) head_carry_kernel(const Params pr) {
 // kernel formed for the Jacobian rows, so per step the walk does only the
 // dependent chain: three dot products with delta_{t-1} and the update.  One
 // block barrier per step, delta double-buffered.  The row's first thread,
-// the only one that combines the factors, loads them two steps ahead into
-// one of two register sets that alternate with the steps (the loop body is
-// unrolled twice so that a set is consumed before it is reloaded and no
-// register copy waits on a load in flight).
+// the only one that combines the factors, loads them four steps ahead into
+// one of four register sets that take turns with the steps (the loop body
+// is unrolled four times so that a set is consumed before it is reloaded
+// and no register copy waits on a load in flight).
 
 template <int DH>
 __global__ void __launch_bounds__(kThreads, 2) head_walk_kernel(const Params pr) {
@@ -749,11 +749,13 @@ __global__ void __launch_bounds__(kThreads, 2) head_walk_kernel(const Params pr)
 #pragma unroll
         for (int j = 0; j < kNF; ++j) f[j] = src[j * DH];
     };
-    float fa[kNF], fb[kNF];
+    float fa[kNF], fb[kNF], fc[kNF], fd[kNF];
     if (qt == 0) {
         dv[0][Gm::vpos(i)] = pr.carry[task * DH + i];
         load_f(t0, fa);
         if (t0 + 1 < t1) load_f(t0 + 1, fb);
+        if (t0 + 2 < t1) load_f(t0 + 2, fc);
+        if (t0 + 3 < t1) load_f(t0 + 3, fd);
     }
     __syncthreads();
     int par = 0;
@@ -780,14 +782,16 @@ __global__ void __launch_bounds__(kThreads, 2) head_walk_kernel(const Params pr)
             pr.Hnew[(b * pr.T + t) * pr.D + (int64_t)h * DH + i] = hn;
             bad |= !isfinite(hn);
             dv[par ^ 1][Gm::vpos(i)] = d;
-            if (t + 2 < t1) load_f(t + 2, f);
+            if (t + 4 < t1) load_f(t + 4, f);
         }
         __syncthreads();
         par ^= 1;
     };
-    for (int64_t t = t0; t < t1; t += 2) {
+    for (int64_t t = t0; t < t1; t += 4) {
         step(t, fa);
         if (t + 1 < t1) step(t + 1, fb);
+        if (t + 2 < t1) step(t + 2, fc);
+        if (t + 3 < t1) step(t + 3, fd);
     }
     if (__any_sync(0xffffffffu, bad) && (tid & 31) == 0) atomicOr(pr.status, kStatusNonFinite);
 }
@@ -1017,14 +1021,16 @@ __global__ void __launch_bounds__(kThreads, 2) head_bwd_walk_kernel(const Params
         for (int j = 0; j < kNB; ++j) f[j] = src[j * DH];
         f[kNB] = pr.G[(b * pr.T + t) * pr.D + col];
     };
-    // two register sets of factors, alternating with the steps (as in the
+    // four register sets of factors, taking turns with the steps (as in the
     // forward walk)
-    float fa[kNB + 1], fb[kNB + 1];
+    float fa[kNB + 1], fb[kNB + 1], fc[kNB + 1], fd[kNB + 1];
     float mu = 0.0f;  // mu_{t+1} of row i (first thread of the row)
     if (qt == 0) {
         mu = pr.carry[task * DH + i];
         load_f(t1 - 1, fa);
         if (t1 - 2 >= t0) load_f(t1 - 2, fb);
+        if (t1 - 3 >= t0) load_f(t1 - 3, fc);
+        if (t1 - 4 >= t0) load_f(t1 - 4, fd);
     }
     int par = 0;
     bool bad = false;
@@ -1044,7 +1050,7 @@ __global__ void __launch_bounds__(kThreads, 2) head_bwd_walk_kernel(const Params
             wv[par][1][vi] = f[2] * lam;
             wv[par][2][vi] = f[4] * lam;
             dzl = f[0] * lam;
-            if (t - 2 >= t0) load_f(t - 2, f);
+            if (t - 4 >= t0) load_f(t - 4, f);
         }
         __syncthreads();
         float sz = 0.0f, sr = 0.0f, sc = 0.0f;
@@ -1063,9 +1069,11 @@ __global__ void __launch_bounds__(kThreads, 2) head_bwd_walk_kernel(const Params
         }
         par ^= 1;
     };
-    for (int64_t t = t1 - 1; t >= t0; t -= 2) {
+    for (int64_t t = t1 - 1; t >= t0; t -= 4) {
         step(t, fa);
         if (t - 1 >= t0) step(t - 1, fb);
+        if (t - 2 >= t0) step(t - 2, fc);
+        if (t - 3 >= t0) step(t - 3, fd);
     }
     if (__any_sync(0xffffffffu, bad) && (tid & 31) == 0) atomicOr(pr.status, kStatusNonFinite);
 }
