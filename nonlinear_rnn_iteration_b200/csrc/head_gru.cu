@@ -15,10 +15,13 @@
 // elements are (A_t, -F_t) with dense d x d blocks, done in three launches
 // per iteration over chunks of kChunk steps of one (batch row, head):
 //   A. per chunk: the product P = A_{t1-1} ... A_{t0} (one d x d x d product
-//      per step) and the chunk's delta from a zero carry, q;
+//      per step; on the fifth-generation tensor cores for d = 64, with
+//      mma.sync for d = 16 and 32), the chunk's delta from a zero carry, q,
+//      and each step's row factors for C;
 //   B. per (batch row, head): the carries, carry_{c+1} = P_c carry_c + q_c;
 //   C. per chunk: re-walk from its carry, delta_t = A_t delta_{t-1} - F_t
-//      (A_t applied as the sum above, never formed), and write h^(k+1).
+//      (A_t applied as the sum above from the stored factors, never
+//      formed), and write h^(k+1).
 // No block waits on another, so there is no look-back and nothing to time
 // out.  All arithmetic is float32; pre-activations f32 or bf16.  The adjoint
 // (pararnn_head_gru_backward) runs the same three launches in reverse time
@@ -186,7 +189,9 @@ __device__ __forceinline__ void block_max_resid(float v, float* resid) {
 }
 
 // ---- A: the chunk's Jacobian product and its delta from a zero carry -----
-// (or, with kResidOnly, just max |F(h^(k))| over the chunk)
+// (or, with kResidOnly, just max |F(h^(k))| over the chunk).  This is the
+// kernel for head widths 16 and 32 (and the residual-only pass of every
+// width); width 64 runs head_chunk_tc_kernel below.
 //
 // The product P <- A_t P (d x d x d per step) runs on the tensor cores with
 // mma.sync m16n8k8 in TF32.  TF32 keeps 10 mantissa bits, so each operand is
