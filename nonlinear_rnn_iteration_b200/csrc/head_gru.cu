@@ -386,7 +386,8 @@ __global__ void __launch_bounds__(kThreads, 2) head_chunk_kernel(const Params pr
 
 // ---- A on the fifth-generation tensor cores (head width 64) -------------
 // The chunk work of head_chunk_kernel, with the product P <- A_t P issued as
-// tcgen05.mma (kind::tf32, M = N = 64, K = 8 per instruction) by one thread:
+// tcgen05.mma (kind::tf32, M = N = 64, K = 8 per instruction) by one thread
+// and formed transposed, P^T <- P^T A_t^T, so that both operands are K-major:
 // operands in shared memory, the accumulator in tensor memory.  One chunk
 // per block, two blocks per SM: the blocks run unsynchronised, so one's
 // tensor-core work overlaps the other's tensor-memory epilogue and barrier.
@@ -395,16 +396,16 @@ __global__ void __launch_bounds__(kThreads, 2) head_chunk_kernel(const Params pr
 // TF32 with cvt.rna, the remainder stored as float (its low bits are below
 // float32 rounding of the product).
 //
-// Operand layouts (no swizzle; "core matrices" of 8 rows of 16 bytes):
-//   A_t, K-major: element (i, m) at float (m / 4) * 256 + (i / 8) * 32 +
-//     (i % 8) * 4 + m % 4, i.e. 8-row groups 128 bytes apart (stride byte
-//     offset) and 4-column K chunks 1024 bytes apart (leading byte offset);
-//   P, MN-major: element (k, n) at float (k / 8) * 512 + (n / 4) * 32 +
-//     (k % 8) * 4 + n % 4, i.e. 4-column N groups 128 bytes apart, 8-row K
-//     groups 2048 bytes apart.
-// Both are written by the threads that produce them with conflict-free
-// stores: a warp's Jacobian rows fill whole 128-byte lines, and each eight
-// threads of the epilogue write eight consecutive 16-byte core rows.
+// Operand layout (no swizzle; "core matrices" of 8 rows of 16 bytes), one
+// for both: row i, K index m of a 64 x 64 operand at float (m / 4) * 256 +
+// (i / 8) * 32 + (i % 8) * 4 + m % 4, i.e. 8-row groups 128 bytes apart
+// (stride byte offset) and 4-column K chunks 1024 bytes apart (leading byte
+// offset).  The right operand A_t^T (K x N) is stored as its N rows, which
+// are the rows of A_t: row i of A_t is row i of the operand.  The left
+// operand P^T has row n = column n of P.  Both are written by the threads
+// that produce them with conflict-free stores: a warp's Jacobian rows fill
+// whole 128-byte lines, and each eight threads of the epilogue write eight
+// consecutive 16-byte core rows.
 //
 // With M = 64, row r of the accumulator is tensor-memory lane
 // 32 (r / 16) + r % 16.  Warp w reads lanes 32 (w % 4) .. +15 of columns
@@ -435,7 +436,6 @@ struct Smem {
 };
 
 __device__ __forceinline__ int a_idx(int i, int m) { return (m >> 2) * 256 + (i >> 3) * 32 + (i & 7) * 4 + (m & 3); }
-__device__ __forceinline__ int p_idx(int k, int n) { return (k >> 3) * 512 + (n >> 2) * 32 + (k & 7) * 4 + (n & 3); }
 
 // shared-memory matrix descriptor: start, leading and stride byte offsets
 // (each >> 4), descriptor version 1, no swizzle
@@ -444,9 +444,11 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t
            ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46);
 }
 
-// instruction descriptor: f32 accumulator, A and B TF32, A K-major, B
-// MN-major, N = 64, M = 64
-constexpr uint32_t kIdesc = (1u << 4) | (2u << 7) | (2u << 10) | (1u << 16) | ((64u >> 3) << 17) | ((64u >> 4) << 24);
+// instruction descriptor: f32 accumulator, A and B TF32, both K-major,
+// N = 64, M = 64.  (With B MN-major and no swizzle the TF32 product came out
+// zero on sm_100a, so every operand here is K-major: the products are formed
+// transposed, the running product as the left operand.)
+constexpr uint32_t kIdesc = (1u << 4) | (2u << 7) | (2u << 10) | ((64u >> 3) << 17) | ((64u >> 4) << 24);
 
 __device__ __forceinline__ void mma(uint32_t d, uint64_t a, uint64_t b, uint32_t accumulate) {
     asm volatile(
@@ -529,11 +531,11 @@ __global__ void __launch_bounds__(kThreads, 2) head_chunk_tc_kernel(const Params
         sm.sv[0][Gm::vpos(i)] = s_before;
         sm.dv[0][Gm::vpos(i)] = 0.0f;
     }
-    // P = I
+    // P^T = I
     for (int idx = tid; idx < DH * DH; idx += kThreads) {
         const int k = idx / DH, n = idx % DH;
-        sm.Phi[tc::p_idx(k, n)] = k == n ? 1.0f : 0.0f;
-        sm.Plo[tc::p_idx(k, n)] = 0.0f;
+        sm.Phi[tc::a_idx(n, k)] = k == n ? 1.0f : 0.0f;
+        sm.Plo[tc::a_idx(n, k)] = 0.0f;
     }
     float rmax = 0.0f;
 
@@ -601,18 +603,19 @@ __global__ void __launch_bounds__(kThreads, 2) head_chunk_tc_kernel(const Params
     for (int64_t t = t0; t < t1; ++t) {
         const uint32_t par = (uint32_t)((t - t0) & 1);
         if (tid == 0 && !abort_flag) {
-            // P_t = A_t P_{t-1}
-            // K step ks starts 2048 bytes further on in every operand: 128
-            // in the descriptors' start-address field (no carry out of it)
+            // P_t^T = P_{t-1}^T A_t^T: the left operand is P^T (rows n, K
+            // index k), the right one A_t with its rows as the N index.  K
+            // step ks starts 2048 bytes further on in both operands: 128 in
+            // the descriptors' start-address field (no carry out of it)
             const uint64_t dah = tc::sdesc(smem_u32(sm.Ahi[p]), 1024, 128);
             const uint64_t dal = tc::sdesc(smem_u32(sm.Alo[p]), 1024, 128);
-            const uint64_t dph = tc::sdesc(smem_u32(sm.Phi), 2048, 128), dpl = tc::sdesc(smem_u32(sm.Plo), 2048, 128);
+            const uint64_t dph = tc::sdesc(smem_u32(sm.Phi), 1024, 128), dpl = tc::sdesc(smem_u32(sm.Plo), 1024, 128);
 #pragma unroll
             for (int ks = 0; ks < DH / 8; ++ks) {
                 const uint64_t ko = (uint64_t)ks * 128u;
-                tc::mma(tmem, dal + ko, dph + ko, ks > 0 ? 1u : 0u);
-                tc::mma(tmem, dah + ko, dpl + ko, 1u);
-                tc::mma(tmem, dah + ko, dph + ko, 1u);
+                tc::mma(tmem, dph + ko, dal + ko, ks > 0 ? 1u : 0u);
+                tc::mma(tmem, dpl + ko, dah + ko, 1u);
+                tc::mma(tmem, dph + ko, dah + ko, 1u);
             }
             tc::commit(&sm.bar);
         }
@@ -650,15 +653,15 @@ __global__ void __launch_bounds__(kThreads, 2) head_chunk_tc_kernel(const Params
                 lv.y = v[4 * g + 1] - hv.y;
                 lv.z = v[4 * g + 2] - hv.z;
                 lv.w = v[4 * g + 3] - hv.w;
-                const int o = tc::p_idx(ek, en + 4 * g);
+                const int o = tc::a_idx(ek, en + 4 * g);
                 *reinterpret_cast<float4*>(sm.Phi + o) = hv;
                 *reinterpret_cast<float4*>(sm.Plo + o) = lv;
             }
         } else {
-            float* Pout = pr.P + task * DH * DH + (int64_t)ek * DH + en;
+            // row ek of P^T is column ek of P (row-major in the workspace)
+            float* Pout = pr.P + task * DH * DH + (int64_t)en * DH + ek;
 #pragma unroll
-            for (int g = 0; g < 4; ++g)
-                *reinterpret_cast<float4*>(Pout + 4 * g) = make_float4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
+            for (int j = 0; j < 16; ++j) Pout[(int64_t)j * DH] = v[j];
         }
         tc::sync_block();
         p ^= 1;
@@ -1085,18 +1088,18 @@ __global__ void __launch_bounds__(kThreads, 2) head_bwd_walk_kernel(const Params
 
 // ---- backward A on the fifth-generation tensor cores (head width 64) ------
 // head_bwd_kernel's product Q <- A_t^T Q (t from t1-1 down to t0) as
-// tcgen05.mma, organised as head_chunk_tc_kernel.  The left operand A_t^T
-// is stored MN-major (element (m, i) of A_t^T = A_t[i][m] at float
-// (i / 8) * 512 + (m / 4) * 32 + (i % 8) * 4 + m % 4, the running product's
-// layout), so each warp's Jacobian rows again fill whole 128-byte lines;
-// mu_t = A_t^T lambda is read back from the same operand as head + remainder
-// (their sum is A_t[i][m] exactly).
+// tcgen05.mma, organised as head_chunk_tc_kernel and likewise transposed:
+// Q^T <- Q^T A_t, the left operand Q^T, the right one A_t (K x N) stored as
+// its N rows, the columns of A_t: element A_t[i][m] at float (i / 4) * 256 +
+// (m / 8) * 32 + (m % 8) * 4 + i % 4 (two-way bank conflicts in the row
+// work's stores).  mu_t = A_t^T lambda is read back from the same operand
+// as head + remainder (their sum is A_t[i][m] exactly).
 namespace tc {
 
 struct SmemB {
-    float Ahi[2][kD * kD];  // A_t^T, MN-major, two steps in turn
+    float Ahi[2][kD * kD];  // A_t, K-major with its columns as the N index, two steps in turn
     float Alo[2][kD * kD];
-    float Phi[kD * kD];     // running product, MN-major
+    float Phi[kD * kD];     // running product, transposed, K-major
     float Plo[kD * kD];
     float sv[2][Geo<kD>::VLEN];  // h_{t-1} rows for the row work (permuted)
     float gv[2][Geo<kD>::VLEN];  // g_t rows (permuted)
@@ -1105,16 +1108,6 @@ struct SmemB {
     uint32_t tmem;
     int abort;
 };
-
-// instruction descriptor of the backward: as kIdesc, with A MN-major too
-constexpr uint32_t kIdescT = kIdesc | (1u << 15);
-
-__device__ __forceinline__ void mma_t(uint32_t d, uint64_t a, uint64_t b, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}"
-        ::"r"(d), "l"(a), "l"(b), "r"(kIdescT), "r"(accumulate));
-}
 
 }  // namespace tc
 
@@ -1153,8 +1146,8 @@ __global__ void __launch_bounds__(kThreads, 2) head_bwd_tc_kernel(const Params p
     }
     for (int idx = tid; idx < DH * DH; idx += kThreads) {
         const int k = idx / DH, n = idx % DH;
-        sm.Phi[tc::p_idx(k, n)] = k == n ? 1.0f : 0.0f;
-        sm.Plo[tc::p_idx(k, n)] = 0.0f;
+        sm.Phi[tc::a_idx(n, k)] = k == n ? 1.0f : 0.0f;
+        sm.Plo[tc::a_idx(n, k)] = 0.0f;
     }
 
     // the row work of step t, parity p: the gates at (h_{t-1}, x_t), row i of
@@ -1188,8 +1181,8 @@ __global__ void __launch_bounds__(kThreads, 2) head_bwd_tc_kernel(const Params p
             a = __fmaf_rn(be, U.r[s], a);
             a = __fmaf_rn(ga, U.c[s], a);
             const float hi = tc::tf32_head(a);
-            ahi[tc::p_idx(i, m)] = hi;  // (A_t^T)[m][i]: K index i, M index m
-            alo[tc::p_idx(i, m)] = a - hi;
+            ahi[tc::a_idx(m, i)] = hi;  // A_t[i][m]: K index i, N index m
+            alo[tc::a_idx(m, i)] = a - hi;
         }
         if (qt == 0) {
             const int vi = Gm::vpos(i);
@@ -1220,16 +1213,16 @@ __global__ void __launch_bounds__(kThreads, 2) head_bwd_tc_kernel(const Params p
     for (int64_t t = t1 - 1; t >= t0; --t) {
         const uint32_t par = (uint32_t)((t1 - 1 - t) & 1);
         if (tid == 0 && !abort_flag) {
-            // Q_t = A_t^T Q_{t+1}
-            const uint64_t dah = tc::sdesc(smem_u32(sm.Ahi[p]), 2048, 128);
-            const uint64_t dal = tc::sdesc(smem_u32(sm.Alo[p]), 2048, 128);
-            const uint64_t dph = tc::sdesc(smem_u32(sm.Phi), 2048, 128), dpl = tc::sdesc(smem_u32(sm.Plo), 2048, 128);
+            // Q_t^T = Q_{t+1}^T A_t (Q_t = A_t^T Q_{t+1})
+            const uint64_t dah = tc::sdesc(smem_u32(sm.Ahi[p]), 1024, 128);
+            const uint64_t dal = tc::sdesc(smem_u32(sm.Alo[p]), 1024, 128);
+            const uint64_t dph = tc::sdesc(smem_u32(sm.Phi), 1024, 128), dpl = tc::sdesc(smem_u32(sm.Plo), 1024, 128);
 #pragma unroll
             for (int ks = 0; ks < DH / 8; ++ks) {
                 const uint64_t ko = (uint64_t)ks * 128u;  // 2048 bytes on
-                tc::mma_t(tmem, dal + ko, dph + ko, ks > 0 ? 1u : 0u);
-                tc::mma_t(tmem, dah + ko, dpl + ko, 1u);
-                tc::mma_t(tmem, dah + ko, dph + ko, 1u);
+                tc::mma(tmem, dph + ko, dal + ko, ks > 0 ? 1u : 0u);
+                tc::mma(tmem, dpl + ko, dah + ko, 1u);
+                tc::mma(tmem, dph + ko, dah + ko, 1u);
             }
             tc::commit(&sm.bar);
         }
@@ -1240,7 +1233,7 @@ __global__ void __launch_bounds__(kThreads, 2) head_bwd_tc_kernel(const Params p
             for (int s = 0; s < SEG; ++s) {
                 const int k = qt + TPR * s;
                 const float lam = sm.gv[p][qt * SEGP + s] + sm.mv[p ^ 1][qt * SEGP + s];
-                const int o = tc::p_idx(k, i);
+                const int o = tc::a_idx(i, k);  // A_t[k][i]
                 acc = __fmaf_rn(sm.Ahi[p][o] + sm.Alo[p][o], lam, acc);
             }
             acc = row_sum<DH>(acc);
@@ -1279,15 +1272,15 @@ __global__ void __launch_bounds__(kThreads, 2) head_bwd_tc_kernel(const Params p
                 lv.y = v[4 * g + 1] - hv.y;
                 lv.z = v[4 * g + 2] - hv.z;
                 lv.w = v[4 * g + 3] - hv.w;
-                const int o = tc::p_idx(ek, en + 4 * g);
+                const int o = tc::a_idx(ek, en + 4 * g);
                 *reinterpret_cast<float4*>(sm.Phi + o) = hv;
                 *reinterpret_cast<float4*>(sm.Plo + o) = lv;
             }
         } else {
-            float* Pout = pr.P + task * DH * DH + (int64_t)ek * DH + en;
+            // row ek of P^T is column ek of P (row-major in the workspace)
+            float* Pout = pr.P + task * DH * DH + (int64_t)en * DH + ek;
 #pragma unroll
-            for (int g = 0; g < 4; ++g)
-                *reinterpret_cast<float4*>(Pout + 4 * g) = make_float4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
+            for (int j = 0; j < 16; ++j) Pout[(int64_t)j * DH] = v[j];
         }
         tc::sync_block();
         p ^= 1;

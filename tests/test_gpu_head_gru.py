@@ -58,6 +58,45 @@ def test_head_forward_small(case, h0, cuda_device):
     assert np.all(np.abs(r - rref) <= 1e-4 * max(1.0, rref.max()) + 1e-6 * np.abs(rref))
 
 
+# Slow memory: p_z shifted down by 5 keeps the update gate almost closed,
+# so h_t stays close to h_{t-1} and the product of a chunk's 128 Jacobians
+# keeps a norm of about 0.4 (with unshifted inputs it is below 1e-27 and a
+# wrong chunk product would go unseen).  Every head width, several chunks.
+SLOW_CASES = [  # (B, T, D, n_heads, K)
+    (1, 300, 64, 1, 3),
+    (2, 260, 128, 2, 2),
+    (1, 300, 32, 1, 3),
+    (1, 280, 48, 3, 2),
+]
+SLOW_SHIFT = -5.0
+
+
+def _slow_case(B, T, D, nh, seed, h0=False):
+    px, U, hz, _, Ut, h0t = _case(B, T, D, nh, seed, h0=h0)
+    px = px.copy()
+    px[:, :, 0, :] += SLOW_SHIFT
+    return px, U, hz, torch.from_numpy(px).to(DEV), Ut, h0t
+
+
+def test_slow_memory_chunk_product_is_not_negligible():
+    # the inputs of the slow-memory cases make the chunk products matter
+    px, U, _, _, _, _ = _slow_case(1, 300, 64, 1, seed=364)
+    H = oracle.head_gru_unroll(px, U)
+    Q = np.eye(64)
+    for t in range(128, 256):
+        Q = oracle.head_gru_jacobian(px[0, t], U[:, 0], H[0, t - 1]) @ Q
+    assert np.linalg.norm(Q, 2) > 0.1
+
+
+@pytest.mark.parametrize("case", SLOW_CASES, ids=lambda c: "B%dT%dD%dh%dK%d" % c)
+def test_head_forward_slow_memory(case, cuda_device):
+    B, T, D, nh, K = case
+    px, U, hz, pxt, Ut, h0t = _slow_case(B, T, D, nh, seed=D + T + 1, h0=True)
+    H = binding.head_gru_forward(pxt, Ut, h0t, K=K)
+    ref, _ = oracle.head_gru_newton(px, U, hz, K=K)
+    assert rel_err(to_np(H), ref) <= TOL_H
+
+
 def test_head_forward_bf16(cuda_device):
     B, T, D, nh, K = 2, 90, 128, 2, 3
     px, U, _, _, Ut, _ = _case(B, T, D, nh, seed=7)
@@ -152,6 +191,19 @@ def test_head_backward_small(case, h0, cuda_device):
     B, T, D, nh, K = case
     px, U, hz, pxt, Ut, h0t = _case(B, T, D, nh, seed=3 * D + T, h0=h0)
     g = np.random.default_rng(T + D).standard_normal((B, T, D)).astype(np.float32)
+    H = binding.head_gru_forward(pxt, Ut, h0t, K=K)
+    dpx, dU, dh0 = binding.head_gru_backward(pxt, Ut, H, torch.from_numpy(g).to(DEV), h0=h0t, want_dh0=True)
+    r_dpx, r_dU, r_dh0 = oracle.head_gru_adjoint(px, U, to_np(H), g, hz)
+    assert rel_err(to_np(dpx), r_dpx) <= TOL_G
+    assert rel_err(to_np(dU), r_dU) <= TOL_G
+    assert rel_err(to_np(dh0), r_dh0) <= TOL_G
+
+
+@pytest.mark.parametrize("case", SLOW_CASES, ids=lambda c: "B%dT%dD%dh%dK%d" % c)
+def test_head_backward_slow_memory(case, cuda_device):
+    B, T, D, nh, K = case
+    px, U, hz, pxt, Ut, h0t = _slow_case(B, T, D, nh, seed=3 * D + T + 1, h0=True)
+    g = np.random.default_rng(T + D + 1).standard_normal((B, T, D)).astype(np.float32)
     H = binding.head_gru_forward(pxt, Ut, h0t, K=K)
     dpx, dU, dh0 = binding.head_gru_backward(pxt, Ut, H, torch.from_numpy(g).to(DEV), h0=h0t, want_dh0=True)
     r_dpx, r_dU, r_dh0 = oracle.head_gru_adjoint(px, U, to_np(H), g, hz)
