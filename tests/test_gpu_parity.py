@@ -100,6 +100,89 @@ def test_backward_small(case, bf16, cuda_device):
         assert da is None
 
 
+# Slow memory: gates shifted so the per-step Jacobian stays near 1 (linear
+# lambda = sig(N(0,1) + 5), GRU p_z - 5, LSTM p_f + 2).  A tile's product of
+# Jacobians then keeps a size of order 1e-2 .. 1 (with the unshifted inputs
+# it is below 1e-10), so the multiplicative half of every carry between
+# tiles is checked, not only the additive one.  (A larger LSTM shift makes
+# the first Newton iterates from the zero guess overflow-sized, residual
+# 1e5 .. 1e20, which tests nothing but conditioning.)
+SLOW_SHIFT = {oracle.LINEAR: (0, 5.0), oracle.DIAG_GRU: (0, -5.0), oracle.DIAG_LSTM: (1, 2.0)}
+SLOW = [
+    (oracle.LINEAR, 2, 700, 136, 1),
+    (oracle.DIAG_GRU, 2, 700, 100, 3),
+    (oracle.DIAG_GRU, 1, 2000, 37, 2),
+    (oracle.DIAG_LSTM, 2, 700, 72, 4),
+    (oracle.DIAG_LSTM, 1, 1500, 13, 3),
+]
+
+
+def _slow_host(cell, B, T, D, seed):
+    rng = np.random.default_rng(seed)
+    G, S = oracle.NUM_GATES[cell], oracle.STATE_WIDTH[cell]
+    px = rng.standard_normal((B, T, G, D)).astype(np.float32)
+    gate, shift = SLOW_SHIFT[cell]
+    px[:, :, gate, :] += shift
+    if cell == oracle.LINEAR:
+        px[:, :, 0, :] = 1.0 / (1.0 + np.exp(-px[:, :, 0, :]))
+        w = None
+    else:
+        w = rng.uniform(-0.5, 0.5, (G, D)).astype(np.float32)
+    hz = (0.5 * rng.standard_normal((B, S, D))).astype(np.float32)
+    g = rng.standard_normal((B, T, S, D)).astype(np.float32)
+    return px, w, hz, g
+
+
+def _slow_inputs(cell, B, T, D, seed, bf16=False):
+    px, w, hz, g = _slow_host(cell, B, T, D, seed)
+    px_used = workloads.round_bf16(px) if bf16 else px
+    t = lambda a: None if a is None else torch.from_numpy(np.ascontiguousarray(a)).to(DEV)
+    pxt = t(px).to(torch.bfloat16) if bf16 else t(px)
+    return dict(px=px, px_used=px_used, w=w, h0=hz, g=g, pxt=pxt, wt=t(w), h0t=t(hz), gt=t(g))
+
+
+def test_slow_memory_tile_product_is_not_negligible():
+    # dL/dpx 80 steps (the longest tile) before a unit gradient at the last
+    # step stays above 1e-3 for the slow-memory inputs of every cell (with
+    # the unshifted inputs it is 1e-13 .. 1e-26)
+    for cell in (oracle.LINEAR, oracle.DIAG_GRU, oracle.DIAG_LSTM):
+        px, w, hz, _ = _slow_host(cell, 1, 400, 8, seed=5)
+        H = oracle.unroll(cell, px, w, hz)
+        g = np.zeros((1, 400, oracle.STATE_WIDTH[cell], 8))
+        g[0, -1, -1, :] = 1.0  # dL/dh at the last step only
+        dpx, _, _ = oracle.adjoint(cell, px, w, hz, H, g)
+        # lambda 80 steps before the end, read off dL/dpx of the additive
+        # (linear) or candidate (GRU, LSTM) gate through its local factor
+        lam = np.abs(dpx[0, 400 - 81]).max()
+        assert lam > 1e-3, (cell, lam)
+
+
+@pytest.mark.parametrize("case", SLOW, ids=lambda c: "cell%d_B%dT%dD%dK%d" % c)
+def test_slow_memory_forward_backward(case, cuda_device):
+    cell, B, T, D, K = case
+    x = _slow_inputs(cell, B, T, D, seed=T + D + cell)
+    H = binding.newton_forward(cell, x["pxt"], x["wt"], x["h0t"], K=K)
+    Ho, _ = oracle.newton(cell, x["px"], x["w"], x["h0"], K=K)
+    assert rel_err(to_np(H), Ho) <= TOL_H
+    # the adjoint at the trajectory the GPU returned: with slow memory the
+    # adjoint is sensitive to the trajectory, and this checks the backward
+    # kernels themselves
+    dpx, da, dh0 = binding.newton_backward(cell, x["pxt"], H, x["gt"], x["wt"], x["h0t"], want_dh0=True)
+    dpxo, dao, dh0o = oracle.adjoint(cell, x["px"], x["w"], x["h0"], to_np(H), x["g"])
+    assert rel_err(to_np(dpx), dpxo) <= TOL_G
+    assert rel_err(to_np(dh0), dh0o) <= TOL_G
+    if da is not None:
+        assert rel_err(to_np(da), dao) <= TOL_G
+
+
+@pytest.mark.parametrize("cell", [oracle.LINEAR, oracle.DIAG_GRU, oracle.DIAG_LSTM])
+def test_slow_memory_bf16(cell, cuda_device):
+    x = _slow_inputs(cell, 2, 600, 64, seed=40 + cell, bf16=True)
+    H = binding.newton_forward(cell, x["pxt"], x["wt"], x["h0t"], K=3)
+    Ho, _ = oracle.newton(cell, x["px_used"], x["w"], x["h0"], K=3)
+    assert rel_err(to_np(H), Ho) <= TOL_H
+
+
 def test_linear_any_k_is_one_scan(cuda_device):
     x = _inputs(oracle.LINEAR, 1, 100, 64, seed=3)
     r1 = torch.zeros(2, device=DEV)
