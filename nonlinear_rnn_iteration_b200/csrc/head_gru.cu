@@ -1091,8 +1091,7 @@ __global__ void __launch_bounds__(kThreads, 2) head_bwd_walk_kernel(const Params
 // tcgen05.mma, organised as head_chunk_tc_kernel and likewise transposed:
 // Q^T <- Q^T A_t, the left operand Q^T, the right one A_t (K x N) stored as
 // its N rows, the columns of A_t: element A_t[i][m] at float (i / 4) * 256 +
-// (m / 8) * 32 + (m % 8) * 4 + i % 4 (two-way bank conflicts in the row
-// work's stores).  mu_t = A_t^T lambda is read back from the same operand
+// (m / 8) * 32 + (m % 8) * 4 + i % 4.  mu_t = A_t^T lambda is read back from the same operand
 // as head + remainder (their sum is A_t[i][m] exactly).
 namespace tc {
 
@@ -1174,15 +1173,28 @@ __global__ void __launch_bounds__(kThreads, 2) head_bwd_tc_kernel(const Params p
         const float dz = 1.0f - z, al = (c - sp) * (z - z * z), be = zc * uc * (r - r * r), ga = zc * r;
         float* ahi = sm.Ahi[p];
         float* alo = sm.Alo[p];
+        // A_t[i][m] goes to element (N index m, K index i).  A warp holds rows
+        // i .. i+7: rows i and i+4 share a bank for the same m, so the second
+        // quad of rows stores each pair of columns in the other order, and one
+        // store instruction covers eight values of m % 8 (no bank conflicts).
+        static_assert(TPR == 4 && SEG % 2 == 0, "eight rows per warp, columns in pairs");
+        const bool swap = (i >> 2) & 1;
 #pragma unroll
-        for (int s = 0; s < SEG; ++s) {
-            const int m = qt + TPR * s;
-            float a = __fmaf_rn(al, U.z[s], (m == i) ? dz : 0.0f);
-            a = __fmaf_rn(be, U.r[s], a);
-            a = __fmaf_rn(ga, U.c[s], a);
-            const float hi = tc::tf32_head(a);
-            ahi[tc::a_idx(m, i)] = hi;  // A_t[i][m]: K index i, N index m
-            alo[tc::a_idx(m, i)] = a - hi;
+        for (int s = 0; s < SEG; s += 2) {
+            const int m0 = qt + TPR * s, m1 = m0 + TPR;
+            float a0 = __fmaf_rn(al, U.z[s], (m0 == i) ? dz : 0.0f);
+            a0 = __fmaf_rn(be, U.r[s], a0);
+            a0 = __fmaf_rn(ga, U.c[s], a0);
+            float a1 = __fmaf_rn(al, U.z[s + 1], (m1 == i) ? dz : 0.0f);
+            a1 = __fmaf_rn(be, U.r[s + 1], a1);
+            a1 = __fmaf_rn(ga, U.c[s + 1], a1);
+            const float x = swap ? a1 : a0, y = swap ? a0 : a1;
+            const int mx = swap ? m1 : m0, my = swap ? m0 : m1;
+            const float xh = tc::tf32_head(x), yh = tc::tf32_head(y);
+            ahi[tc::a_idx(mx, i)] = xh;
+            alo[tc::a_idx(mx, i)] = x - xh;
+            ahi[tc::a_idx(my, i)] = yh;
+            alo[tc::a_idx(my, i)] = y - yh;
         }
         if (qt == 0) {
             const int vi = Gm::vpos(i);
