@@ -386,13 +386,14 @@ __global__ void __launch_bounds__(kThreads, 2) head_chunk_kernel(const Params pr
 
 // ---- A on the fifth-generation tensor cores (head width 64) -------------
 // The chunk work of head_chunk_kernel, with the product P <- A_t P issued as
-// tcgen05.mma (kind::tf32, M = N = 64, K = 8 per instruction) by one thread
-// and formed transposed, P^T <- P^T A_t^T, so that both operands are K-major:
-// operands in shared memory, the accumulator in tensor memory.  One chunk
+// tcgen05.mma (kind::tf32, M = N = 64, K = 8 per instruction) and formed
+// transposed, P^T <- P^T A_t^T, so that both operands are K-major: operands
+// in shared memory, the accumulators in tensor memory.  One chunk
 // per block, two blocks per SM: the blocks run unsynchronised, so one's
 // tensor-core work overlaps the other's tensor-memory epilogue and barrier.
-// The head/remainder split is kept (x = x_hi + x_lo, a_lo b_hi + a_hi b_lo +
-// a_hi b_hi accumulated in float32 in tensor memory): the head is rounded to
+// The head/remainder split is kept (x = x_hi + x_lo; a_lo b_hi, a_hi b_lo and
+// a_hi b_hi, each accumulated over K in float32 in tensor memory by its own
+// issuing thread, summed in the epilogue): the head is rounded to
 // TF32 with cvt.rna, the remainder stored as float (its low bits are below
 // float32 rounding of the product).
 //
@@ -413,14 +414,16 @@ __global__ void __launch_bounds__(kThreads, 2) head_chunk_kernel(const Params pr
 // columns, threads 16-31 the next 16.
 //
 // One block barrier per step, as in head_chunk_kernel: after it the issuing
-// thread starts the product of step t; all threads form the Jacobian rows of
-// step t+1 meanwhile, then wait for the product (mbarrier signalled by
-// tcgen05.commit), move it from tensor memory into the P operand, fence the
-// generic-proxy writes for the tensor cores, and meet at the next barrier.
+// threads start the product of step t; all threads form the Jacobian rows of
+// step t+1 meanwhile, then wait for the product (mbarrier signalled by each
+// issuer's tcgen05.commit), move it from tensor memory into the P operand,
+// fence the generic-proxy writes for the tensor cores, and meet at the next
+// barrier.
 namespace tc {
 
 constexpr int kD = 64;
-constexpr uint32_t kTmemCols = 64;
+constexpr uint32_t kTmemCols = 256;  // forward: three 64-column accumulators, one per split term
+constexpr uint32_t kTmemColsB = 64;  // backward: one accumulator
 constexpr uint64_t kWaitNs = 1000000000ull;  // 1 s: far beyond one step's product
 
 struct Smem {
@@ -489,6 +492,19 @@ __device__ __forceinline__ void load_acc(uint32_t taddr, float (&v)[16]) {
     for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(r[j]);
 }
 
+// the three accumulators (64 columns apart) of a thread's 16 columns,
+// summed as (lo.hi + hi.lo) + hi.hi
+__device__ __forceinline__ void load_acc3(uint32_t taddr, float (&v)[16]) {
+    float w[16];
+    load_acc(taddr, v);
+    load_acc(taddr + 64u, w);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) v[j] += w[j];
+    load_acc(taddr + 128u, w);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) v[j] += w[j];
+}
+
 __device__ __forceinline__ float tf32_head(float x) {
     uint32_t h;
     asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(h) : "f"(x));
@@ -520,7 +536,7 @@ __global__ void __launch_bounds__(kThreads, 2) head_chunk_tc_kernel(const Params
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
     if (tid == 0) {
-        mbar_init(&sm.bar, 1);
+        mbar_init(&sm.bar, 3);  // one arrival per issuing thread
         abort_flag = 0;
         mbar_fence_init();
     }
@@ -602,20 +618,22 @@ __global__ void __launch_bounds__(kThreads, 2) head_chunk_tc_kernel(const Params
     int p = 0;
     for (int64_t t = t0; t < t1; ++t) {
         const uint32_t par = (uint32_t)((t - t0) & 1);
-        if (tid == 0 && !abort_flag) {
+        if ((tid == 0 || tid == 96 || tid == 192) && !abort_flag) {
             // P_t^T = P_{t-1}^T A_t^T: the left operand is P^T (rows n, K
-            // index k), the right one A_t with its rows as the N index.  K
-            // step ks starts 2048 bytes further on in both operands: 128 in
+            // index k), the right one A_t with its rows as the N index.  One
+            // split term per issuing thread (threads of warps 0, 3 and 6),
+            // each into its own accumulator: one thread issuing all 24 MMAs
+            // delayed its warp's row work, and the block's barrier with it.
+            // K step ks starts 2048 bytes further on in both operands: 128 in
             // the descriptors' start-address field (no carry out of it)
-            const uint64_t dah = tc::sdesc(smem_u32(sm.Ahi[p]), 1024, 128);
-            const uint64_t dal = tc::sdesc(smem_u32(sm.Alo[p]), 1024, 128);
-            const uint64_t dph = tc::sdesc(smem_u32(sm.Phi), 1024, 128), dpl = tc::sdesc(smem_u32(sm.Plo), 1024, 128);
+            const int term = tid / 96;  // 0: P_hi A_lo, 1: P_lo A_hi, 2: P_hi A_hi
+            const uint64_t da = tc::sdesc(smem_u32(term == 1 ? sm.Plo : sm.Phi), 1024, 128);
+            const uint64_t db = tc::sdesc(smem_u32(term == 0 ? sm.Alo[p] : sm.Ahi[p]), 1024, 128);
+            const uint32_t d = tmem + 64u * (uint32_t)term;
 #pragma unroll
             for (int ks = 0; ks < DH / 8; ++ks) {
                 const uint64_t ko = (uint64_t)ks * 128u;
-                tc::mma(tmem, dph + ko, dal + ko, ks > 0 ? 1u : 0u);
-                tc::mma(tmem, dpl + ko, dah + ko, 1u);
-                tc::mma(tmem, dph + ko, dah + ko, 1u);
+                tc::mma(d, da + ko, db + ko, ks > 0 ? 1u : 0u);
             }
             tc::commit(&sm.bar);
         }
@@ -640,7 +658,7 @@ __global__ void __launch_bounds__(kThreads, 2) head_chunk_tc_kernel(const Params
         }
         tc::fence_after();
         float v[16];
-        tc::load_acc(taddr, v);
+        tc::load_acc3(taddr, v);
         if (t + 1 < t1) {
 #pragma unroll
             for (int g = 0; g < 4; ++g) {
@@ -1087,28 +1105,70 @@ __global__ void __launch_bounds__(kThreads, 2) head_bwd_walk_kernel(const Params
 }
 
 // ---- backward A on the fifth-generation tensor cores (head width 64) ------
-// head_bwd_kernel's product Q <- A_t^T Q (t from t1-1 down to t0) as
-// tcgen05.mma, organised as head_chunk_tc_kernel and likewise transposed:
-// Q^T <- Q^T A_t, the left operand Q^T, the right one A_t (K x N) stored as
-// its N rows, the columns of A_t: element A_t[i][m] at float (i / 4) * 256 +
-// (m / 8) * 32 + (m % 8) * 4 + i % 4.  mu_t = A_t^T lambda is read back from the same operand
-// as head + remainder (their sum is A_t[i][m] exactly).
+// The chunk work of head_bwd_kernel for head width 64, run forward in time
+// over the chunk.  The prefix products R_t = A_{t0}^T ... A_t^T
+// (R_t = R_{t-1} A_t^T, R_{t0-1} = I) are formed on tcgen05 with the operand
+// layout of head_chunk_tc_kernel: R is the left operand, A_t^T the right one
+// stored as the rows of A_t, so the Jacobian rows are formed and stored as in
+// the forward.  The chunk's product is R_{t1-1} = A_{t0}^T ... A_{t1-1}^T,
+// and its adjoint from a zero carry is mu_{t0} = sum_t R_t g_t.  The
+// epilogue threads hold R_t after step t's product: each adds its 16
+// columns' share R_t[ek][n] g_t[n] to a float32 register, and the four
+// shares of a row are summed after the last step.  No thread forms
+// A_t^T lambda from shared memory.
 namespace tc {
 
+
 struct SmemB {
-    float Ahi[2][kD * kD];  // A_t, K-major with its columns as the N index, two steps in turn
+    float Ahi[2][kD * kD];  // A_t, K-major (rows of A_t as the N index), two steps in turn
     float Alo[2][kD * kD];
-    float Phi[kD * kD];     // running product, transposed, K-major
+    float Phi[kD * kD];     // R_{t-1}, K-major
     float Plo[kD * kD];
+    float gv[2][kD];        // g_t, two steps in turn
+    float red[kD];          // the second half of each row's mu shares
     float sv[2][Geo<kD>::VLEN];  // h_{t-1} rows for the row work (permuted)
-    float gv[2][Geo<kD>::VLEN];  // g_t rows (permuted)
-    float mv[2][Geo<kD>::VLEN];  // mu rows (permuted)
     uint64_t bar;
     uint32_t tmem;
     int abort;
 };
 
+// the bounded wait for a commit (1 s, then the timeout bit and no further MMA)
+__device__ __forceinline__ void wait_bar(const Params& pr, uint64_t* bar, uint32_t par, volatile int& abort_flag,
+                                         int lane) {
+    if (abort_flag) return;
+    uint64_t start = 0;
+    while (!mbar_try_wait(bar, par)) {
+        const uint64_t now = globaltimer_ns();
+        if (start == 0) {
+            start = now | 1;
+        } else if (now - start > kWaitNs) {
+            if (lane == 0) atomicOr(pr.status, kStatusTimeout);
+            abort_flag = 1;
+            return;
+        }
+    }
+}
+
 }  // namespace tc
+
+// Per-step inputs of the forward-in-time backward row work for row i:
+// pre-activations, g_t[i] and h_t[i] (the state the next step needs).
+struct BStepF {
+    float pz, pr, pc, g, s;
+};
+
+template <int DH, typename PxT>
+__device__ __forceinline__ BStepF load_bstepf(const Params& pr, int64_t b, int h, int i, int64_t t) {
+    BStepF in;
+    const int64_t c = (int64_t)h * DH + i;
+    const PxT* x = static_cast<const PxT*>(pr.px) + (b * pr.T + t) * 3 * pr.D + c;
+    in.pz = ldp(x);
+    in.pr = ldp(x + pr.D);
+    in.pc = ldp(x + 2 * pr.D);
+    in.g = pr.G[(b * pr.T + t) * pr.D + c];
+    in.s = pr.Hold[(b * pr.T + t) * pr.D + c];
+    return in;
+}
 
 template <typename PxT>
 __global__ void __launch_bounds__(kThreads, 2) head_bwd_tc_kernel(const Params pr) {
@@ -1128,7 +1188,7 @@ __global__ void __launch_bounds__(kThreads, 2) head_bwd_tc_kernel(const Params p
 
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&sm.tmem)),
-                     "r"(tc::kTmemCols)
+                     "r"(tc::kTmemColsB)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
@@ -1139,10 +1199,8 @@ __global__ void __launch_bounds__(kThreads, 2) head_bwd_tc_kernel(const Params p
     }
     RowU<DH> U;
     U.load(pr.U, pr.nh, h, i, qt);
-    if (qt == 0) {
-        sm.sv[0][Gm::vpos(i)] = state_before<DH>(pr, b, h, i, t1 - 1);
-        sm.mv[1][Gm::vpos(i)] = 0.0f;  // mu_{t1} for the chunk's own product
-    }
+    if (qt == 0) sm.sv[0][Gm::vpos(i)] = state_before<DH>(pr, b, h, i, t0);
+    // R = I
     for (int idx = tid; idx < DH * DH; idx += kThreads) {
         const int k = idx / DH, n = idx % DH;
         sm.Phi[tc::a_idx(n, k)] = k == n ? 1.0f : 0.0f;
@@ -1150,10 +1208,9 @@ __global__ void __launch_bounds__(kThreads, 2) head_bwd_tc_kernel(const Params p
     }
 
     // the row work of step t, parity p: the gates at (h_{t-1}, x_t), row i of
-    // A_t as column i of A_t^T (split) into A[p], the row factors for the
-    // walk, g_t into gv[p], and h_{t-2} into sv[p ^ 1] for the next (earlier)
-    // step
-    auto row_step = [&](const BStepIn& in, int p, int64_t t) {
+    // A_t (split) into A[p], g_t into gv[p], the row factors for the walk,
+    // and h_t into sv[p ^ 1] for the next step
+    auto row_step = [&](const BStepF& in, int p, int64_t t) {
         float uz = 0.0f, ur = 0.0f, uc = 0.0f;
 #pragma unroll
         for (int s = 0; s < SEG; ++s) {
@@ -1173,134 +1230,116 @@ __global__ void __launch_bounds__(kThreads, 2) head_bwd_tc_kernel(const Params p
         const float dz = 1.0f - z, al = (c - sp) * (z - z * z), be = zc * uc * (r - r * r), ga = zc * r;
         float* ahi = sm.Ahi[p];
         float* alo = sm.Alo[p];
-        // A_t[i][m] goes to element (N index m, K index i).  A warp holds rows
-        // i .. i+7: rows i and i+4 share a bank for the same m, so the second
-        // quad of rows stores each pair of columns in the other order, and one
-        // store instruction covers eight values of m % 8 (no bank conflicts).
-        static_assert(TPR == 4 && SEG % 2 == 0, "eight rows per warp, columns in pairs");
-        const bool swap = (i >> 2) & 1;
 #pragma unroll
-        for (int s = 0; s < SEG; s += 2) {
-            const int m0 = qt + TPR * s, m1 = m0 + TPR;
-            float a0 = __fmaf_rn(al, U.z[s], (m0 == i) ? dz : 0.0f);
-            a0 = __fmaf_rn(be, U.r[s], a0);
-            a0 = __fmaf_rn(ga, U.c[s], a0);
-            float a1 = __fmaf_rn(al, U.z[s + 1], (m1 == i) ? dz : 0.0f);
-            a1 = __fmaf_rn(be, U.r[s + 1], a1);
-            a1 = __fmaf_rn(ga, U.c[s + 1], a1);
-            const float x = swap ? a1 : a0, y = swap ? a0 : a1;
-            const int mx = swap ? m1 : m0, my = swap ? m0 : m1;
-            const float xh = tc::tf32_head(x), yh = tc::tf32_head(y);
-            ahi[tc::a_idx(mx, i)] = xh;
-            alo[tc::a_idx(mx, i)] = x - xh;
-            ahi[tc::a_idx(my, i)] = yh;
-            alo[tc::a_idx(my, i)] = y - yh;
+        for (int s = 0; s < SEG; ++s) {
+            const int m = qt + TPR * s;
+            float a = __fmaf_rn(al, U.z[s], (m == i) ? dz : 0.0f);
+            a = __fmaf_rn(be, U.r[s], a);
+            a = __fmaf_rn(ga, U.c[s], a);
+            const float hi = tc::tf32_head(a);
+            ahi[tc::a_idx(i, m)] = hi;
+            alo[tc::a_idx(i, m)] = a - hi;
         }
         if (qt == 0) {
-            const int vi = Gm::vpos(i);
-            sm.gv[p][vi] = in.g;
-            sm.sv[p ^ 1][vi] = in.s2;
+            sm.gv[p][i] = in.g;
+            sm.sv[p ^ 1][Gm::vpos(i)] = in.s;
             store_brow_factors<DH>(pr, seq, t, i, dz, al, be, zc, ga);
         }
     };
 
-    BStepIn nxt = load_bstep<DH, PxT>(pr, b, h, i, t1 - 1);
+    BStepF nxt = load_bstepf<DH, PxT>(pr, b, h, i, t0);
     tc::fence_before();
     __syncthreads();
     tc::fence_after();
     const uint32_t tmem = sm.tmem;
     {
-        const BStepIn in = nxt;
-        if (t1 - 2 >= t0) nxt = load_bstep<DH, PxT>(pr, b, h, i, t1 - 2);
-        row_step(in, 0, t1 - 1);
+        const BStepF in = nxt;
+        if (t0 + 1 < t1) nxt = load_bstepf<DH, PxT>(pr, b, h, i, t0 + 1);
+        row_step(in, 0, t0);
     }
     tc::sync_block();
 
+    // epilogue geometry, as in the forward
     const int eq = warp & 3;
     const int ek = 16 * eq + (lane & 15);
     const int en = 32 * (warp >> 2) + 16 * (lane >> 4);
     const uint32_t taddr = tmem + ((uint32_t)(32 * eq) << 16) + (uint32_t)(32 * (warp >> 2));
 
+    // descriptors: K step ks starts 2048 bytes further on in each operand
+    // (128 in the start-address field)
+    const uint64_t dph = tc::sdesc(smem_u32(sm.Phi), 1024, 128), dpl = tc::sdesc(smem_u32(sm.Plo), 1024, 128);
+    float mu = 0.0f;  // this thread's share of mu_{t0}[ek]: columns en .. en+15
     int p = 0;
-    for (int64_t t = t1 - 1; t >= t0; --t) {
-        const uint32_t par = (uint32_t)((t1 - 1 - t) & 1);
+    for (int64_t t = t0; t < t1; ++t) {
+        const uint32_t par = (uint32_t)((t - t0) & 1);
         if (tid == 0 && !abort_flag) {
-            // Q_t^T = Q_{t+1}^T A_t (Q_t = A_t^T Q_{t+1})
+            // R_t = R_{t-1} A_t^T
             const uint64_t dah = tc::sdesc(smem_u32(sm.Ahi[p]), 1024, 128);
             const uint64_t dal = tc::sdesc(smem_u32(sm.Alo[p]), 1024, 128);
-            const uint64_t dph = tc::sdesc(smem_u32(sm.Phi), 1024, 128), dpl = tc::sdesc(smem_u32(sm.Plo), 1024, 128);
 #pragma unroll
             for (int ks = 0; ks < DH / 8; ++ks) {
-                const uint64_t ko = (uint64_t)ks * 128u;  // 2048 bytes on
+                const uint64_t ko = (uint64_t)ks * 128u;
                 tc::mma(tmem, dph + ko, dal + ko, ks > 0 ? 1u : 0u);
                 tc::mma(tmem, dpl + ko, dah + ko, 1u);
                 tc::mma(tmem, dph + ko, dah + ko, 1u);
             }
             tc::commit(&sm.bar);
         }
-        {
-            // mu_t[m] = sum_i A_t[i][m] (g_t[i] + mu_{t+1}[i]) for thread (m = i, qt)
-            float acc = 0.0f;
-#pragma unroll
-            for (int s = 0; s < SEG; ++s) {
-                const int k = qt + TPR * s;
-                const float lam = sm.gv[p][qt * SEGP + s] + sm.mv[p ^ 1][qt * SEGP + s];
-                const int o = tc::a_idx(i, k);  // A_t[k][i]
-                acc = __fmaf_rn(sm.Ahi[p][o] + sm.Alo[p][o], lam, acc);
-            }
-            acc = row_sum<DH>(acc);
-            if (qt == 0) sm.mv[p][Gm::vpos(i)] = acc;
+        if (t + 1 < t1) {
+            const BStepF in = nxt;
+            if (t + 2 < t1) nxt = load_bstepf<DH, PxT>(pr, b, h, i, t + 2);
+            row_step(in, p ^ 1, t + 1);
         }
-        if (t - 1 >= t0) {
-            const BStepIn in = nxt;
-            if (t - 2 >= t0) nxt = load_bstep<DH, PxT>(pr, b, h, i, t - 2);
-            row_step(in, p ^ 1, t - 1);
-        }
-        if (!abort_flag) {
-            uint64_t start = 0;
-            while (!mbar_try_wait(&sm.bar, par)) {
-                const uint64_t now = globaltimer_ns();
-                if (start == 0) {
-                    start = now | 1;
-                } else if (now - start > tc::kWaitNs) {
-                    if (lane == 0) atomicOr(pr.status, kStatusTimeout);
-                    abort_flag = 1;
-                    break;
-                }
-            }
-        }
+        tc::wait_bar(pr, &sm.bar, par, abort_flag, lane);
         tc::fence_after();
         float v[16];
         tc::load_acc(taddr, v);
-        if (t - 1 >= t0) {
+        {
+            // this thread's share of R_t g_t
+            const float4* gq = reinterpret_cast<const float4*>(sm.gv[p] + en);
 #pragma unroll
             for (int g = 0; g < 4; ++g) {
-                float4 hv, lv;
-                hv.x = tc::tf32_head(v[4 * g + 0]);
-                hv.y = tc::tf32_head(v[4 * g + 1]);
-                hv.z = tc::tf32_head(v[4 * g + 2]);
-                hv.w = tc::tf32_head(v[4 * g + 3]);
-                lv.x = v[4 * g + 0] - hv.x;
-                lv.y = v[4 * g + 1] - hv.y;
-                lv.z = v[4 * g + 2] - hv.z;
-                lv.w = v[4 * g + 3] - hv.w;
-                const int o = tc::a_idx(ek, en + 4 * g);
-                *reinterpret_cast<float4*>(sm.Phi + o) = hv;
-                *reinterpret_cast<float4*>(sm.Plo + o) = lv;
+                const float4 gg = gq[g];
+                mu = __fmaf_rn(v[4 * g + 0], gg.x, mu);
+                mu = __fmaf_rn(v[4 * g + 1], gg.y, mu);
+                mu = __fmaf_rn(v[4 * g + 2], gg.z, mu);
+                mu = __fmaf_rn(v[4 * g + 3], gg.w, mu);
             }
-        } else {
-            // row ek of P^T is column ek of P (row-major in the workspace)
-            float* Pout = pr.P + task * DH * DH + (int64_t)en * DH + ek;
+        }
+        // R_t into the left operand for the next step's products
 #pragma unroll
-            for (int j = 0; j < 16; ++j) Pout[(int64_t)j * DH] = v[j];
+        for (int g = 0; g < 4; ++g) {
+            float4 hv, lv;
+            hv.x = tc::tf32_head(v[4 * g + 0]);
+            hv.y = tc::tf32_head(v[4 * g + 1]);
+            hv.z = tc::tf32_head(v[4 * g + 2]);
+            hv.w = tc::tf32_head(v[4 * g + 3]);
+            lv.x = v[4 * g + 0] - hv.x;
+            lv.y = v[4 * g + 1] - hv.y;
+            lv.z = v[4 * g + 2] - hv.z;
+            lv.w = v[4 * g + 3] - hv.w;
+            const int o = tc::a_idx(ek, en + 4 * g);
+            *reinterpret_cast<float4*>(sm.Phi + o) = hv;
+            *reinterpret_cast<float4*>(sm.Plo + o) = lv;
+        }
+        if (t + 1 == t1) {
+            // R_{t1-1}: the chunk's product A_{t0}^T ... A_{t1-1}^T, row-major
+            float* Pout = pr.P + task * DH * DH + (int64_t)ek * DH + en;
+#pragma unroll
+            for (int g = 0; g < 4; ++g)
+                *reinterpret_cast<float4*>(Pout + 4 * g) = make_float4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
         }
         tc::sync_block();
         p ^= 1;
     }
-    // mu at the chunk's first step: written to mv[p ^ 1] by the last iteration
-    if (qt == 0) pr.q[task * DH + i] = sm.mv[p ^ 1][Gm::vpos(i)];
+    // the four shares of row ek: lanes l and l + 16, then warps w and w + 4
+    mu += __shfl_xor_sync(0xffffffffu, mu, 16);
+    if (warp >= 4 && lane < 16) sm.red[ek] = mu;
+    tc::fence_before();
+    __syncthreads();
+    if (warp < 4 && lane < 16) pr.q[task * DH + ek] = mu + sm.red[ek];
     if (warp == 0)
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(tc::kTmemCols)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(tc::kTmemColsB)
                      : "memory");
 }
 
