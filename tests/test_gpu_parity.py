@@ -15,6 +15,7 @@ import pytest
 import torch
 
 import oracle
+import slow_inputs
 from gpu_util import gather_channels, norm_err, rel_err, to_np
 from nonlinear_rnn_iteration_b200 import binding, workloads
 
@@ -100,14 +101,9 @@ def test_backward_small(case, bf16, cuda_device):
         assert da is None
 
 
-# Slow memory: gates shifted so the per-step Jacobian stays near 1 (linear
-# lambda = sig(N(0,1) + 5), GRU p_z - 5, LSTM p_f + 2).  A tile's product of
-# Jacobians then keeps a size of order 1e-2 .. 1 (with the unshifted inputs
-# it is below 1e-10), so the multiplicative half of every carry between
-# tiles is checked, not only the additive one.  (A larger LSTM shift makes
-# the first Newton iterates from the zero guess overflow-sized, residual
-# 1e5 .. 1e20, which tests nothing but conditioning.)
-SLOW_SHIFT = {oracle.LINEAR: (0, 5.0), oracle.DIAG_GRU: (0, -5.0), oracle.DIAG_LSTM: (1, 2.0)}
+# Slow memory (slow_inputs.py): one gate shifted so each step's Jacobian
+# stays near 1 and a tile's product keeps a size of 1e-2 .. 1, so the
+# multiplicative half of every carry between tiles is checked too.
 SLOW = [
     (oracle.LINEAR, 2, 700, 136, 1),
     (oracle.DIAG_GRU, 2, 700, 100, 3),
@@ -117,44 +113,12 @@ SLOW = [
 ]
 
 
-def _slow_host(cell, B, T, D, seed):
-    rng = np.random.default_rng(seed)
-    G, S = oracle.NUM_GATES[cell], oracle.STATE_WIDTH[cell]
-    px = rng.standard_normal((B, T, G, D)).astype(np.float32)
-    gate, shift = SLOW_SHIFT[cell]
-    px[:, :, gate, :] += shift
-    if cell == oracle.LINEAR:
-        px[:, :, 0, :] = 1.0 / (1.0 + np.exp(-px[:, :, 0, :]))
-        w = None
-    else:
-        w = rng.uniform(-0.5, 0.5, (G, D)).astype(np.float32)
-    hz = (0.5 * rng.standard_normal((B, S, D))).astype(np.float32)
-    g = rng.standard_normal((B, T, S, D)).astype(np.float32)
-    return px, w, hz, g
-
-
 def _slow_inputs(cell, B, T, D, seed, bf16=False):
-    px, w, hz, g = _slow_host(cell, B, T, D, seed)
+    px, w, hz, g = slow_inputs.diag_host(cell, B, T, D, seed)
     px_used = workloads.round_bf16(px) if bf16 else px
     t = lambda a: None if a is None else torch.from_numpy(np.ascontiguousarray(a)).to(DEV)
     pxt = t(px).to(torch.bfloat16) if bf16 else t(px)
     return dict(px=px, px_used=px_used, w=w, h0=hz, g=g, pxt=pxt, wt=t(w), h0t=t(hz), gt=t(g))
-
-
-def test_slow_memory_tile_product_is_not_negligible():
-    # dL/dpx 80 steps (the longest tile) before a unit gradient at the last
-    # step stays above 1e-3 for the slow-memory inputs of every cell (with
-    # the unshifted inputs it is 1e-13 .. 1e-26)
-    for cell in (oracle.LINEAR, oracle.DIAG_GRU, oracle.DIAG_LSTM):
-        px, w, hz, _ = _slow_host(cell, 1, 400, 8, seed=5)
-        H = oracle.unroll(cell, px, w, hz)
-        g = np.zeros((1, 400, oracle.STATE_WIDTH[cell], 8))
-        g[0, -1, -1, :] = 1.0  # dL/dh at the last step only
-        dpx, _, _ = oracle.adjoint(cell, px, w, hz, H, g)
-        # lambda 80 steps before the end, read off dL/dpx of the additive
-        # (linear) or candidate (GRU, LSTM) gate through its local factor
-        lam = np.abs(dpx[0, 400 - 81]).max()
-        assert lam > 1e-3, (cell, lam)
 
 
 @pytest.mark.parametrize("case", SLOW, ids=lambda c: "cell%d_B%dT%dD%dK%d" % c)
