@@ -202,6 +202,25 @@ def test_head_backward_slow_memory(case, cuda_device):
     assert rel_err(to_np(dh0), r_dh0) <= TOL_G
 
 
+@pytest.mark.parametrize("D,nh", [(128, 2), (64, 2)], ids=["d64", "d32"])
+def test_head_backward_bf16(D, nh, cuda_device):
+    # bf16 pre-activations (widened on load) against the oracle on the same
+    # bf16 values, slow memory, three chunks
+    B, T, K = 2, 300, 3
+    px, U = slow_inputs.head_host(B, T, D, nh, seed=D + 5)
+    pxb = workloads.round_bf16(px)
+    pxt = torch.from_numpy(px).to(DEV).to(torch.bfloat16)
+    Ut = torch.from_numpy(U).to(DEV)
+    g = np.random.default_rng(D + 6).standard_normal((B, T, D)).astype(np.float32)
+    H = binding.head_gru_forward(pxt, Ut, None, K=K)
+    ref, _ = oracle.head_gru_newton(pxb, U, None, K=K)
+    assert rel_err(to_np(H), ref) <= TOL_H
+    dpx, dU, _ = binding.head_gru_backward(pxt, Ut, H, torch.from_numpy(g).to(DEV))
+    r_dpx, r_dU, _ = oracle.head_gru_adjoint(pxb, U, to_np(H), g, None)
+    assert rel_err(to_np(dpx), r_dpx) <= TOL_G
+    assert rel_err(to_np(dU), r_dU) <= TOL_G
+
+
 def test_head_backward_deterministic_and_optional_outputs(cuda_device):
     B, T, D, nh = 2, 300, 128, 2
     _, _, _, pxt, Ut, _ = _case(B, T, D, nh, seed=21)
