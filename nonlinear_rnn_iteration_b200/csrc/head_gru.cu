@@ -429,7 +429,7 @@ constexpr uint64_t kWaitNs = 1000000000ull;  // 1 s: far beyond one step's produ
 struct Smem {
     float Ahi[2][kD * kD];  // A_t, K-major, two steps in turn
     float Alo[2][kD * kD];
-    float Phi[kD * kD];     // running product, MN-major
+    float Phi[kD * kD];     // running product P^T, K-major
     float Plo[kD * kD];
     float sv[2][Geo<kD>::VLEN];  // h^(k) rows, permuted (vpos), two steps in turn
     float dv[2][Geo<kD>::VLEN];  // delta rows, permuted, two steps in turn
