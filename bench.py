@@ -50,6 +50,11 @@ ALGO_BYTES = {
     ("linear", "f32", "bwd"): 24, ("diag_gru", "f32", "bwd"): 32, ("diag_gru", "bf16", "bwd"): 26,
     ("diag_lstm", "f32", "bwd"): 48, ("diag_lstm", "bf16", "bwd"): 40,
 }
+# channels per slice of the host-buffer pipeline in the e2e measurement:
+# 8 x 1024 channels in slices of 256 make 32 slices, whose shorter fill and
+# drain beat whole rows (8 slices)
+E2E_CHANNELS = 256
+
 KERNEL_SOURCES = ["newton_fwd.cuh", "adjoint_bwd.cuh", "lookback.cuh", "cells.cuh", "common.cuh", "tma.cuh", "pararnn_abi.cu"]
 
 
@@ -371,17 +376,18 @@ def time_e2e(prob, steps):
     px_dev = torch.empty_like(prob.px)
     s = prob.stream
     if not w.backward:
-        # the public host-buffer entry point: slices of batch rows whose copies
-        # in and out overlap the solve
+        # the public host-buffer entry point: slices of one batch row and
+        # E2E_CHANNELS channels whose copies in and out overlap the solve
         from nonlinear_rnn_iteration_b200 import binding
 
         code = binding.BF16 if prob.px.dtype == torch.bfloat16 else binding.F32
-        n = binding.pararnn_newton_forward_host_workspace_bytes(w.cell_id, w.B, w.T, w.D, w.K, code, 1)
+        chans = E2E_CHANNELS if (w.D % 8 == 0 and w.D > E2E_CHANNELS) else 0
+        n = binding.pararnn_newton_forward_host_workspace_bytes(w.cell_id, w.B, w.T, w.D, w.K, code, 1, chans)
         ws_host = torch.zeros(n, dtype=torch.uint8, device=prob.px.device)
 
         def one():
             st = binding.pararnn_newton_forward_host(w.cell_id, w.B, w.T, w.D, code, px_host, prob.a, None, w.K,
-                                                     H_host, ws_host, n, 1, s)
+                                                     H_host, ws_host, n, 1, chans, s)
             if st != binding.OK:
                 raise RuntimeError("pararnn_newton_forward_host: %s" % binding.pararnn_last_error())
 

@@ -196,11 +196,17 @@ pararnn_status pararnn_newton_forward_noalloc(pararnn_cell cell, int64_t B, int6
 /* ---- the forward on host buffers (serving) --------------------------------
  * pararnn_newton_forward for pre-activations and H in host memory (pinned
  * memory lets the copies overlap; pageable memory works, with the copies
- * serialised).  The batch is cut into slices of rows_per_slice rows that
- * pass through three device slots on three internal streams -- copy in,
- * solve, copy out -- so that both PCIe directions and the solver work at
- * once.  Batch rows are independent recurrences, so every row of H is
- * bit-identical to pararnn_newton_forward's on the whole batch.
+ * serialised).  The batch is cut into slices of rows_per_slice rows and,
+ * when channels_per_slice is not 0, of channels_per_slice channels each
+ * (copied with strided 2-D copies); the slices pass through three device
+ * slots on three internal streams -- copy in, solve, copy out -- so that
+ * both PCIe directions and the solver work at once.  More, smaller slices
+ * shorten the pipeline's fill and drain.  Batch rows and channels are
+ * independent recurrences, so every value of H is bit-identical to
+ * pararnn_newton_forward's on the whole batch.
+ *   channels_per_slice  0 (or >= D): whole rows; otherwise a multiple of 8,
+ *                 and D must be a multiple of 8 too (every slice then keeps
+ *                 the whole batch's 16-byte row alignment and solver path)
  *   preacts_host  (B, T, G, D) px_dtype, host (or device) memory
  *   diag_w, h0    device memory, as for pararnn_newton_forward
  *   H_host        (B, T, S, D) float32, host (or device) memory
@@ -212,14 +218,16 @@ pararnn_status pararnn_newton_forward_noalloc(pararnn_cell cell, int64_t B, int6
  * everything is queued.  No residual history is kept.  A non-finite value in
  * any slice's output is reported by pararnn_status_sync(workspace, stream).
  * Errors as for pararnn_newton_forward, plus PARARNN_EINVAL for
- * rows_per_slice < 1 and PARARNN_ECUDA if the internal streams cannot be
- * created. */
+ * rows_per_slice < 1 or a channels_per_slice outside the rule above, and
+ * PARARNN_ECUDA if the internal streams cannot be created.  The workspace
+ * size function returns 0 for the same invalid arguments. */
 size_t pararnn_newton_forward_host_workspace_bytes(pararnn_cell cell, int64_t B, int64_t T, int64_t D, int K,
-                                                   pararnn_dtype px_dtype, int64_t rows_per_slice);
+                                                   pararnn_dtype px_dtype, int64_t rows_per_slice,
+                                                   int64_t channels_per_slice);
 pararnn_status pararnn_newton_forward_host(pararnn_cell cell, int64_t B, int64_t T, int64_t D,
                                            pararnn_dtype px_dtype, const void* preacts_host, const float* diag_w,
                                            const float* h0, int K, float* H_host, void* workspace, size_t ws_bytes,
-                                           int64_t rows_per_slice, void* stream);
+                                           int64_t rows_per_slice, int64_t channels_per_slice, void* stream);
 
 /* ---- head-wise GRU: block-diagonal recurrent weights --------------------
  * ParaGRU(mix='head', n_heads) of the pararnn-torch page (Models / Usage,

@@ -37,8 +37,8 @@ SIGNATURES = {
     "pararnn_last_error": (ctypes.c_char_p, []),
     "pararnn_probe_wait_timeout": (_I, [_P, _SZ, _U64, _P]),
     "pararnn_newton_forward_noalloc": (_I, [_I, _I64, _I64, _I64, _I, _P, _P, _P, _I, _P, _P, _I, _P]),
-    "pararnn_newton_forward_host_workspace_bytes": (_SZ, [_I, _I64, _I64, _I64, _I, _I, _I64]),
-    "pararnn_newton_forward_host": (_I, [_I, _I64, _I64, _I64, _I, _P, _P, _P, _I, _P, _P, _SZ, _I64, _P]),
+    "pararnn_newton_forward_host_workspace_bytes": (_SZ, [_I, _I64, _I64, _I64, _I, _I, _I64, _I64]),
+    "pararnn_newton_forward_host": (_I, [_I, _I64, _I64, _I64, _I, _P, _P, _P, _I, _P, _P, _SZ, _I64, _I64, _P]),
     "pararnn_head_gru_workspace_bytes": (_SZ, [_I64, _I64, _I64, _I, _I]),
     "pararnn_head_gru_forward": (_I, [_I64, _I64, _I64, _I, _I, _P, _P, _P, _I, _P, _P, _SZ, _P, _P]),
     "pararnn_head_gru_backward_workspace_bytes": (_SZ, [_I64, _I64, _I64, _I]),
@@ -140,15 +140,16 @@ def pararnn_newton_forward_noalloc(cell, B, T, D, px_dtype, preacts, diag_w, h0,
                                                  _ptr(H_out), _ptr(resid_hist), int(wait_status), _stream(stream))
 
 
-def pararnn_newton_forward_host_workspace_bytes(cell, B, T, D, K, px_dtype, rows_per_slice):
-    return load().pararnn_newton_forward_host_workspace_bytes(cell, B, T, D, K, px_dtype, rows_per_slice)
+def pararnn_newton_forward_host_workspace_bytes(cell, B, T, D, K, px_dtype, rows_per_slice, channels_per_slice=0):
+    return load().pararnn_newton_forward_host_workspace_bytes(cell, B, T, D, K, px_dtype, rows_per_slice,
+                                                              channels_per_slice)
 
 
 def pararnn_newton_forward_host(cell, B, T, D, px_dtype, preacts_host, diag_w, h0, K, H_host, workspace, ws_bytes,
-                                rows_per_slice, stream):
+                                rows_per_slice, channels_per_slice, stream):
     return load().pararnn_newton_forward_host(cell, B, T, D, px_dtype, _ptr(preacts_host), _ptr(diag_w), _ptr(h0), K,
                                               _ptr(H_host), _ptr(workspace), ws_bytes, rows_per_slice,
-                                              _stream(stream))
+                                              channels_per_slice, _stream(stream))
 
 
 def pararnn_head_gru_workspace_bytes(B, T, D, n_heads, K):
@@ -297,8 +298,8 @@ def head_gru_backward(px, U, H, dL_dH, h0=None, want_dU=True, want_dh0=False, wo
     return dpx, dU, dh0
 
 
-def newton_forward_host(cell, px_host, diag_w=None, h0=None, K=1, out_host=None, rows_per_slice=1, workspace=None,
-                        stream=None, sync_status=True):
+def newton_forward_host(cell, px_host, diag_w=None, h0=None, K=1, out_host=None, rows_per_slice=1,
+                        channels_per_slice=0, workspace=None, stream=None, sync_status=True):
     """The forward on host tensors (pinned for overlap): H (B,T,S,D) float32 on the host."""
     import torch
 
@@ -310,13 +311,14 @@ def newton_forward_host(cell, px_host, diag_w=None, h0=None, K=1, out_host=None,
         out_host = torch.empty((B, T, S, D), dtype=torch.float32, pin_memory=px_host.is_pinned())
     dev = diag_w.device if diag_w is not None else torch.device("cuda", torch.cuda.current_device())
     if workspace is None:
-        n = pararnn_newton_forward_host_workspace_bytes(cell, B, T, D, K, code, rows_per_slice)
+        n = pararnn_newton_forward_host_workspace_bytes(cell, B, T, D, K, code, rows_per_slice, channels_per_slice)
         if n == 0:
             raise PararnnError(EINVAL, "pararnn_newton_forward_host_workspace_bytes", "invalid arguments")
         workspace = torch.zeros(n, dtype=torch.uint8, device=dev)
     st = stream if stream is not None else torch.cuda.current_stream(dev)
     _check(pararnn_newton_forward_host(cell, B, T, D, code, px_host, diag_w, h0, K, out_host, workspace,
-                                       workspace.numel(), rows_per_slice, st), "pararnn_newton_forward_host")
+                                       workspace.numel(), rows_per_slice, channels_per_slice, st),
+           "pararnn_newton_forward_host")
     if sync_status:
         _check(pararnn_status_sync(workspace, st), "pararnn_newton_forward_host (device status)")
     return out_host

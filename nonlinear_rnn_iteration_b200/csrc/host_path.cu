@@ -10,7 +10,10 @@
 // slots on three streams -- copy in, solve, copy out -- so that slice i+1
 // comes in while slice i is solved and slice i-1 goes out.  Every row's
 // result is bit-identical to what pararnn_newton_forward returns for the
-// whole batch.
+// whole batch.  The channels are independent recurrences too, so a slice
+// may also take only a range of channels (copied with strided 2-D copies):
+// more, smaller slices shorten the pipeline's fill and drain, when only the
+// first slice's copy in and the last one's solve and copy out run alone.
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -29,20 +32,31 @@ constexpr int kSlots = 3;
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct Layout {
-    int64_t rows = 0;  // batch rows per slice
-    size_t px_bytes = 0, h_bytes = 0, fw_bytes = 0, slot_bytes = 0, total = 0;
+    int64_t rows = 0;   // batch rows per slice
+    int64_t chans = 0;  // channels per slice
+    size_t px_bytes = 0, h_bytes = 0, w_bytes = 0, h0_bytes = 0, fw_bytes = 0, slot_bytes = 0, total = 0;
 };
 
-bool layout(pararnn_cell cell, int64_t B, int64_t T, int64_t D, int K, int64_t rows_per_slice, size_t esz,
-            Layout& l) {
+// channels_per_slice: 0 (or >= D) for whole rows, else a multiple of 8 with
+// D a multiple of 8, so that every slice's rows keep the 16-byte alignment
+// the whole batch has and the solver takes the same path (bit-identical
+// results)
+bool layout(pararnn_cell cell, int64_t B, int64_t T, int64_t D, int K, int64_t rows_per_slice,
+            int64_t channels_per_slice, size_t esz, Layout& l) {
     const int G = pararnn_num_gates(cell), S = pararnn_state_width(cell);
-    if (G < 0 || B < 0 || T < 0 || D < 0 || rows_per_slice < 1) return false;
+    if (G < 0 || B < 0 || T < 0 || D < 0 || rows_per_slice < 1 || channels_per_slice < 0) return false;
+    const bool split = channels_per_slice > 0 && channels_per_slice < D;
+    if (split && (channels_per_slice % 8 != 0 || D % 8 != 0)) return false;
     l.rows = rows_per_slice < B ? rows_per_slice : (B > 0 ? B : 1);
-    l.fw_bytes = pararnn_workspace_bytes(cell, l.rows, T, D, K);
+    l.chans = split ? channels_per_slice : (D > 0 ? D : 1);
+    l.fw_bytes = pararnn_workspace_bytes(cell, l.rows, T, l.chans, K);
     if (l.fw_bytes == 0) return false;
-    l.px_bytes = align256((size_t)l.rows * T * G * D * esz);
-    l.h_bytes = align256((size_t)l.rows * T * S * D * sizeof(float));
-    l.slot_bytes = align256(l.fw_bytes) + l.px_bytes + l.h_bytes;
+    l.px_bytes = align256((size_t)l.rows * T * G * l.chans * esz);
+    l.h_bytes = align256((size_t)l.rows * T * S * l.chans * sizeof(float));
+    // a channel slice's own copies of the weights and of h0 (contiguous)
+    l.w_bytes = split ? align256((size_t)G * l.chans * sizeof(float)) : 0;
+    l.h0_bytes = split ? align256((size_t)l.rows * S * l.chans * sizeof(float)) : 0;
+    l.slot_bytes = align256(l.fw_bytes) + l.px_bytes + l.h_bytes + l.w_bytes + l.h0_bytes;
     l.total = 256 + kSlots * l.slot_bytes;
     return true;
 }
@@ -63,12 +77,12 @@ pararnn_status fail(pararnn_status st, const char* msg) {
 using namespace pararnn;
 
 extern "C" size_t pararnn_newton_forward_host_workspace_bytes(pararnn_cell cell, int64_t B, int64_t T, int64_t D,
-                                                              int K, pararnn_dtype px_dtype,
-                                                              int64_t rows_per_slice) {
+                                                              int K, pararnn_dtype px_dtype, int64_t rows_per_slice,
+                                                              int64_t channels_per_slice) {
     hp::Layout l;
     const size_t esz = px_dtype == PARARNN_BF16 ? 2 : 4;
     if (px_dtype != PARARNN_F32 && px_dtype != PARARNN_BF16) return 0;
-    if (!hp::layout(cell, B, T, D, K, rows_per_slice, esz, l)) return 0;
+    if (!hp::layout(cell, B, T, D, K, rows_per_slice, channels_per_slice, esz, l)) return 0;
     return l.total;
 }
 
@@ -76,13 +90,14 @@ extern "C" pararnn_status pararnn_newton_forward_host(pararnn_cell cell, int64_t
                                                       pararnn_dtype px_dtype, const void* preacts_host,
                                                       const float* diag_w, const float* h0, int K, float* H_host,
                                                       void* workspace, size_t ws_bytes, int64_t rows_per_slice,
-                                                      void* stream) {
+                                                      int64_t channels_per_slice, void* stream) {
     if (px_dtype != PARARNN_F32 && px_dtype != PARARNN_BF16)
         return hp::fail(PARARNN_EINVAL, "pararnn_newton_forward_host: unknown pre-activation dtype");
     const size_t esz = px_dtype == PARARNN_BF16 ? 2 : 4;
     hp::Layout l;
-    if (!hp::layout(cell, B, T, D, K, rows_per_slice, esz, l))
-        return hp::fail(PARARNN_EINVAL, "pararnn_newton_forward_host: bad cell, sizes, K or rows_per_slice");
+    if (!hp::layout(cell, B, T, D, K, rows_per_slice, channels_per_slice, esz, l))
+        return hp::fail(PARARNN_EINVAL, "pararnn_newton_forward_host: bad cell, sizes, K, rows_per_slice or "
+                                        "channels_per_slice");
     if (!workspace || ws_bytes < l.total || !pointer_on_device(workspace) ||
         (reinterpret_cast<uintptr_t>(workspace) & 255))
         return hp::fail(PARARNN_EINVAL, "pararnn_newton_forward_host: workspace missing, small or not 256-byte "
@@ -95,7 +110,9 @@ extern "C" pararnn_status pararnn_newton_forward_host(pararnn_cell cell, int64_t
     if (!preacts_host || !H_host)
         return hp::fail(PARARNN_EINVAL, "pararnn_newton_forward_host: preacts_host and H_host are required");
     const int G = pararnn_num_gates(cell), S = pararnn_state_width(cell);
-    const int64_t nslices = (B + l.rows - 1) / l.rows;
+    const int64_t nrs = (B + l.rows - 1) / l.rows, ncs = (D + l.chans - 1) / l.chans;
+    const int64_t nslices = nrs * ncs;  // channel slices of a row slice are consecutive
+    const bool split = ncs > 1;
 
     // three streams (in, solve, out) ordered after the work already on `stream`
     cudaStream_t sin = nullptr, scomp = nullptr, sout = nullptr;
@@ -134,33 +151,52 @@ extern "C" pararnn_status pararnn_newton_forward_host(pararnn_cell cell, int64_t
     pararnn_status st = PARARNN_OK;
     for (int64_t i = 0; i < nslices && st == PARARNN_OK; ++i) {
         const int k = (int)(i % hp::kSlots);
-        const int64_t b0 = i * l.rows, nb = (b0 + l.rows <= B) ? l.rows : B - b0;
+        const int64_t ir = i / ncs, ic = i - ir * ncs;
+        const int64_t b0 = ir * l.rows, nb = (b0 + l.rows <= B) ? l.rows : B - b0;
+        const int64_t d0 = ic * l.chans, dn = (d0 + l.chans <= D) ? l.chans : D - d0;
         unsigned char* slot = ws + 256 + (size_t)k * l.slot_bytes;
         void* fw = slot;
         void* px_dev = slot + hp::align256(l.fw_bytes);
         float* h_dev = reinterpret_cast<float*>(slot + hp::align256(l.fw_bytes) + l.px_bytes);
+        float* w_dev = reinterpret_cast<float*>(slot + hp::align256(l.fw_bytes) + l.px_bytes + l.h_bytes);
+        float* h0_dev = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(w_dev) + l.w_bytes);
         // in: the slot's pre-activations are free once the solve of slice i - kSlots is done
         if (i >= hp::kSlots) e = cudaStreamWaitEvent(sin, ev_comp[k], 0);
-        if (e == cudaSuccess)
-            e = cudaMemcpyAsync(px_dev, static_cast<const unsigned char*>(preacts_host) + (size_t)b0 * row_px,
-                                (size_t)nb * row_px, cudaMemcpyDefault, sin);
+        const unsigned char* src = static_cast<const unsigned char*>(preacts_host) + (size_t)b0 * row_px;
+        if (e == cudaSuccess && !split)
+            e = cudaMemcpyAsync(px_dev, src, (size_t)nb * row_px, cudaMemcpyDefault, sin);
+        if (e == cudaSuccess && split)  // nb * T * G rows of dn channels, D apart in host memory
+            e = cudaMemcpy2DAsync(px_dev, (size_t)dn * esz, src + (size_t)d0 * esz, (size_t)D * esz,
+                                  (size_t)dn * esz, (size_t)nb * T * G, cudaMemcpyDefault, sin);
+        if (e == cudaSuccess && split && diag_w)  // (G, dn) from (G, D)
+            e = cudaMemcpy2DAsync(w_dev, (size_t)dn * sizeof(float), diag_w + d0, (size_t)D * sizeof(float),
+                                  (size_t)dn * sizeof(float), (size_t)G, cudaMemcpyDefault, sin);
+        if (e == cudaSuccess && split && h0)  // (nb, S, dn) from (B, S, D)
+            e = cudaMemcpy2DAsync(h0_dev, (size_t)dn * sizeof(float), h0 + (size_t)b0 * S * D + d0,
+                                  (size_t)D * sizeof(float), (size_t)dn * sizeof(float), (size_t)nb * S,
+                                  cudaMemcpyDefault, sin);
         if (e == cudaSuccess) e = cudaEventRecord(ev_in[k], sin);
         // solve: after the copy in, and after slice i - kSlots has left the slot's H
         if (e == cudaSuccess) e = cudaStreamWaitEvent(scomp, ev_in[k], 0);
         if (e == cudaSuccess && i >= hp::kSlots) e = cudaStreamWaitEvent(scomp, ev_out[k], 0);
         if (e != cudaSuccess) break;
-        st = pararnn_newton_forward(cell, nb, T, D, px_dtype, px_dev, diag_w,
-                                    h0 ? h0 + (size_t)b0 * S * D : nullptr, K, h_dev, fw, l.fw_bytes, nullptr,
-                                    scomp);
+        const float* w_use = split ? (diag_w ? w_dev : nullptr) : diag_w;
+        const float* h0_use = split ? (h0 ? h0_dev : nullptr) : (h0 ? h0 + (size_t)b0 * S * D : nullptr);
+        st = pararnn_newton_forward(cell, nb, T, dn, px_dtype, px_dev, w_use, h0_use, K, h_dev, fw, l.fw_bytes,
+                                    nullptr, scomp);
         if (st != PARARNN_OK) break;
         hp::fold_status<<<1, 32, 0, scomp>>>(reinterpret_cast<unsigned*>(ws), reinterpret_cast<unsigned*>(fw));
         e = cudaGetLastError();
         if (e == cudaSuccess) e = cudaEventRecord(ev_comp[k], scomp);
         // out
         if (e == cudaSuccess) e = cudaStreamWaitEvent(sout, ev_comp[k], 0);
-        if (e == cudaSuccess)
-            e = cudaMemcpyAsync(reinterpret_cast<unsigned char*>(H_host) + (size_t)b0 * row_h, h_dev,
-                                (size_t)nb * row_h, cudaMemcpyDefault, sout);
+        unsigned char* dst = reinterpret_cast<unsigned char*>(H_host) + (size_t)b0 * row_h;
+        if (e == cudaSuccess && !split)
+            e = cudaMemcpyAsync(dst, h_dev, (size_t)nb * row_h, cudaMemcpyDefault, sout);
+        if (e == cudaSuccess && split)  // nb * T * S rows of dn channels, D apart in host memory
+            e = cudaMemcpy2DAsync(dst + (size_t)d0 * sizeof(float), (size_t)D * sizeof(float), h_dev,
+                                  (size_t)dn * sizeof(float), (size_t)dn * sizeof(float), (size_t)nb * T * S,
+                                  cudaMemcpyDefault, sout);
         if (e == cudaSuccess) e = cudaEventRecord(ev_out[k], sout);
         if (e != cudaSuccess) break;
     }

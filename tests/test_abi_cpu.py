@@ -162,5 +162,12 @@ def test_host_path_workspace_bytes():
     row_px, row_h = 1024 * 3 * 256 * 4, 1024 * 256 * 4
     assert one >= 3 * (row_px + row_h) and two - one >= 3 * (row_px + row_h)
     assert f(gru, 8, 1024, 256, 3, binding.BF16, 1) < one  # bf16 slices are smaller
+    # channel slices: a multiple of 8 of a D that is a multiple of 8; 0 or
+    # >= D means whole rows
+    assert f(gru, 8, 1024, 256, 3, binding.F32, 1, 12) == 0
+    assert f(gru, 8, 1024, 100, 3, binding.F32, 1, 8) == 0
+    assert f(gru, 8, 1024, 256, 3, binding.F32, 1, -8) == 0
+    assert f(gru, 8, 1024, 256, 3, binding.F32, 1, 256) == one == f(gru, 8, 1024, 256, 3, binding.F32, 1, 512)
+    assert 0 < f(gru, 8, 1024, 256, 3, binding.F32, 1, 64) < one
     # a slice never exceeds the batch
     assert f(gru, 2, 1024, 256, 3, binding.F32, 5) == f(gru, 2, 1024, 256, 3, binding.F32, 2)

@@ -1,6 +1,7 @@
 """The forward on host buffers (pararnn_newton_forward_host): slices of batch
-rows pipelined through three device slots must give, row for row, exactly
-the bits pararnn_newton_forward gives for the whole batch on the device."""
+rows (and of channels) pipelined through three device slots must give,
+value for value, exactly the bits pararnn_newton_forward gives for the whole
+batch on the device."""
 import numpy as np
 import pytest
 import torch
@@ -57,4 +58,22 @@ def test_host_path_reports_nonfinite_and_bad_arguments(cuda_device):
     ws = torch.zeros(n, dtype=torch.uint8, device=DEV)
     H = torch.empty((B, T, 1, D))
     assert binding.pararnn_newton_forward_host(binding.DIAG_GRU, B, T, D, binding.F32, px, w, None, 2, H, ws, n - 256,
-                                               2, None) == binding.EINVAL
+                                               2, 0, None) == binding.EINVAL
+    # channel slices: a multiple of 8, of a D that is a multiple of 8
+    assert binding.pararnn_newton_forward_host(binding.DIAG_GRU, B, T, D, binding.F32, px, w, None, 2, H, ws, n,
+                                               2, 12, None) == binding.EINVAL
+
+
+@pytest.mark.parametrize("cell,K,bf16", [(binding.LINEAR, 1, False), (binding.DIAG_GRU, 3, False),
+                                         (binding.DIAG_GRU, 2, True), (binding.DIAG_LSTM, 3, False)])
+@pytest.mark.parametrize("rows,chans", [(1, 8), (2, 64), (5, 128), (1, 136), (3, 400)])
+def test_host_path_channel_slices(cell, K, bf16, rows, chans, cuda_device):
+    # slices of rows x channels (strided 2-D copies, the weights and h0 cut
+    # to the slice): the same bits as the device path on the whole batch
+    B, T, D = 5, 300, 136
+    px, w = _inputs(cell, B, T, D, seed=cell * 10 + rows + chans, bf16=bf16)
+    S = binding.pararnn_state_width(cell)
+    h0 = torch.randn((B, S, D), device=DEV, generator=torch.Generator(device=DEV).manual_seed(chans))
+    ref = binding.newton_forward(cell, px.to(DEV), w, h0, K=K).cpu()
+    H = binding.newton_forward_host(cell, px.pin_memory(), w, h0, K=K, rows_per_slice=rows, channels_per_slice=chans)
+    assert torch.equal(H, ref)
