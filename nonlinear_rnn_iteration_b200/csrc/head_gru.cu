@@ -24,9 +24,10 @@
 //      formed), and write h^(k+1).
 // No block waits on another, so there is no look-back and nothing to time
 // out.  All arithmetic is float32; pre-activations f32 or bf16.  The adjoint
-// (pararnn_head_gru_backward) runs the same three launches in reverse time
-// on the propagated adjoint, plus a fixed-order reduction for dL/dU (see
-// "the adjoint" below).
+// (pararnn_head_gru_backward) runs the same three launches on the propagated
+// adjoint, its carries and re-walk in reverse time (its d = 64 chunk pass
+// forms prefix products forward in time within the chunk), plus a
+// fixed-order reduction for dL/dU (see "the adjoint" below).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
