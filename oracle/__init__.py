@@ -102,7 +102,7 @@ def _bind(so_path):
     lib.oracle_unroll.restype = ci
     lib.oracle_newton.argtypes = [ci, i64, i64, i64, P, P, P, ci, P, P, ci]
     lib.oracle_newton.restype = ci
-    lib.oracle_residual.argtypes = [ci, i64, i64, i64, P, P, P, P]
+    lib.oracle_residual.argtypes = [ci, i64, i64, i64, P, P, P, P, ci]
     lib.oracle_residual.restype = ctypes.c_double
     lib.oracle_adjoint.argtypes = [ci, i64, i64, i64, P, P, P, P, P, P, P, P, ci]
     lib.oracle_adjoint.restype = ci
@@ -191,11 +191,18 @@ def newton(cell, px, w=None, h0=None, K=1, nthreads=None):
     return H, resid
 
 
-def residual(cell, px, w, h0, H):
+def residual(cell, px, w, h0, H, nthreads=None):
+    """max |F(H)|_t = max |H_t - f(H_{t-1}, x_t)| over the whole batch, for a
+    given trajectory H (B,T,S,D); H_{-1} = h0."""
     lib = _load()
     px, w, h0, H = _f64(px), _f64(w), _f64(h0), _f64(H)
     B, T, D = _shape(cell, px)
-    return float(lib.oracle_residual(cell, B, T, D, _ptr(px), _ptr(w), _ptr(h0), _ptr(H)))
+    if H.shape != (B, T, STATE_WIDTH[cell], D):
+        raise ValueError("H must be (B,T,S,D) = %s, got %s" % ((B, T, STATE_WIDTH[cell], D), H.shape))
+    r = float(lib.oracle_residual(cell, B, T, D, _ptr(px), _ptr(w), _ptr(h0), _ptr(H), _threads(nthreads)))
+    if r < 0:
+        raise ValueError("oracle_residual rejected its arguments (%g)" % r)
+    return r
 
 
 def adjoint(cell, px, w, h0, H, dLdH, nthreads=None):

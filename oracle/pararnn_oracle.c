@@ -181,7 +181,7 @@ typedef struct {
     double* dLdpx;
     double* dLda_b;       /* adjoint: per-batch partial (B,G,D) */
     double* dLdh0;
-    int mode;             /* 0 unroll, 1 newton, 2 adjoint */
+    int mode;             /* 0 unroll, 1 newton, 2 adjoint, 3 residual */
     int nthreads;
     int tid;
     double resid[64];     /* per-thread residual history (K+1 <= 64) */
@@ -333,7 +333,8 @@ static void* worker(void* arg) {
         int64_t b = c / j->D, d = c % j->D;
         if (j->mode == 0) channel_unroll(j, b, d);
         else if (j->mode == 1) channel_newton(j, b, d);
-        else channel_adjoint(j, b, d);
+        else if (j->mode == 2) channel_adjoint(j, b, d);
+        else j->resid[0] = nanmax(j->resid[0], channel_residual(j, b, d));
     }
     return NULL;
 }
@@ -394,16 +395,18 @@ int oracle_newton(int cell, int64_t B, int64_t T, int64_t D, const double* px, c
     return rc;
 }
 
-/* max |F(H)| of a given trajectory H */
+/* max |F(H)| = max_{b,t,s,d} |H_t - f(H_{t-1}, x_t)| (H_{-1} = h0) of a given
+ * trajectory H, the quantity the residual history records; channels are
+ * shared among nthreads threads.  Returns a negative value on bad arguments. */
 double oracle_residual(int cell, int64_t B, int64_t T, int64_t D, const double* px, const double* w,
-                       const double* h0, const double* H) {
+                       const double* h0, const double* H, int nthreads) {
+    if (check(cell, B, T, D, px) || (cell != 0 && !w) || (B * T * D > 0 && !H)) return -1.0;
     job_t j;
     memset(&j, 0, sizeof j);
     j.cell = cell; j.S = ncell_state(cell); j.G = ncell_gates(cell);
-    j.B = B; j.T = T; j.D = D; j.px = px; j.w = w; j.h0 = h0; j.H = (double*)H;
-    double r = 0.0;
-    for (int64_t c = 0; c < B * D; ++c) r = nanmax(r, channel_residual(&j, c / D, c % D));
-    return r;
+    j.B = B; j.T = T; j.D = D; j.px = px; j.w = w; j.h0 = h0; j.H = (double*)H; j.mode = 3;
+    if (run(&j, nthreads)) return -2.0;
+    return j.resid[0];
 }
 
 /* Adjoint at trajectory H: dL_dpx (B,T,G,D), dL_da (G,D) summed over b then

@@ -26,7 +26,9 @@ What pins what:
                     finite differences of <g, unroll(theta)>.
 * residual       -- strictly decreasing over Newton steps on seeded cells of
                     every workload's cell (an empirical property, not a
-                    theorem).
+                    theorem); max |F(H)| of an arbitrary trajectory against
+                    the torch residual of the dense Newton pin, and zero at
+                    the unroll.
 """
 import numpy as np
 import torch
@@ -174,6 +176,29 @@ def pin_newton_dense():
                 _close(Ho[0, :, :, 0], H.detach().numpy().reshape(T, S), 1e-12,
                        "cell %d Newton k=%d vs dense" % (cell, k))
                 _close(ro, res, 1e-12, "cell %d residual history k=%d" % (cell, k))
+
+
+def pin_residual_function():
+    # max |F(H)| of an arbitrary trajectory (not a Newton iterate) against the
+    # torch residual F(H)_t = H_t - f(H_{t-1}, x_t) built from torch's cells;
+    # several channels and batch rows, so a max over the wrong axis fails too
+    for cell in CELLS:
+        B, T, D, G, S = 2, 9, 3, oracle.NUM_GATES[cell], oracle.STATE_WIDTH[cell]
+        for h0flag in (False, True):
+            px, w, h0 = _rand_inputs(cell, B, T, D, seed=60 + cell + 3 * h0flag, h0=h0flag)
+            H = _rng(70 + cell).standard_normal((B, T, S, D)) * 0.7
+            ref = 0.0
+            for b in range(B):
+                for d in range(D):
+                    p = torch.tensor(px[b, :, :, d])
+                    a = torch.tensor(_wcol(w, d, G))
+                    hh0 = torch.tensor(_h0col(h0, b, d, S))
+                    F = _dense_F(cell, p, a, hh0)
+                    ref = max(ref, float(F(torch.tensor(H[b, :, :, d]).reshape(-1), p, a, hh0).abs().max()))
+            _close(oracle.residual(cell, px, w, h0, H, nthreads=2), ref, 1e-13, "cell %d residual of H" % cell)
+        # the unroll solves F(H) = 0
+        U = oracle.unroll(cell, px, w, h0)
+        assert oracle.residual(cell, px, w, h0, U) < 1e-14, "cell %d residual of the unroll" % cell
 
 
 def pin_affine_one_step():
@@ -521,6 +546,6 @@ def pin_head_adjoint_diagonal():
 
 ALL_PINS = [pin_cell_step, pin_jacobian, pin_param_grads, pin_unroll, pin_newton_dense, pin_affine_one_step,
             pin_prefix_exact, pin_lstm_zero_weights, pin_adjoint_dense, pin_adjoint_bptt, pin_adjoint_fd,
-            pin_residual_monotone, pin_head_step_and_jacobian, pin_head_unroll, pin_head_newton_dense,
+            pin_residual_monotone, pin_residual_function, pin_head_step_and_jacobian, pin_head_unroll, pin_head_newton_dense,
             pin_head_prefix_exact_and_diagonal, pin_head_adjoint_bptt, pin_head_adjoint_dense,
             pin_head_adjoint_diagonal]
