@@ -14,6 +14,10 @@ Functions and what they follow:
   from the warm start h^(0)_t = f(0, x_t) (pararnn-torch PyPI page, Method
   section; ParaRNN thread, tweet [3/8]); each step's linear system is solved
   by plain forward substitution.
+* :func:`newton_picard` -- the same after P Picard (fixed-point) sweeps
+  h^(p+1)_t = f(h^(p)_{t-1}, x_t) from the warm start (API overview,
+  "Solver": ``picard_iters``; Method section: zero-hidden start + Picard).
+* :func:`residual` -- max |F(H)| of a given trajectory.
 * :func:`adjoint` -- reverse recursion lambda_t = g_t + A_{t+1}^T lambda_{t+1}
   at a given trajectory and the gradients w.r.t. pre-activations, diagonal
   weights and the initial state (Method section, backward pass).
@@ -102,6 +106,8 @@ def _bind(so_path):
     lib.oracle_unroll.restype = ci
     lib.oracle_newton.argtypes = [ci, i64, i64, i64, P, P, P, ci, P, P, ci]
     lib.oracle_newton.restype = ci
+    lib.oracle_newton_picard.argtypes = [ci, i64, i64, i64, P, P, P, ci, ci, P, P, ci]
+    lib.oracle_newton_picard.restype = ci
     lib.oracle_residual.argtypes = [ci, i64, i64, i64, P, P, P, P, ci]
     lib.oracle_residual.restype = ctypes.c_double
     lib.oracle_adjoint.argtypes = [ci, i64, i64, i64, P, P, P, P, P, P, P, P, ci]
@@ -188,6 +194,22 @@ def newton(cell, px, w=None, h0=None, K=1, nthreads=None):
                            _threads(nthreads))
     if rc:
         raise ValueError("oracle_newton rejected its arguments (%d)" % rc)
+    return H, resid
+
+
+def newton_picard(cell, px, w=None, h0=None, P=0, K=1, nthreads=None):
+    """P Picard sweeps h^(p+1)_t = f(h^(p)_{t-1}, x_t) from the warm start,
+    then K Newton iterations; returns (H^(K), resid) with resid[k] = max
+    |F(H^(k))| for k = 0..K, H^(0) being the guess after the sweeps."""
+    lib = _load()
+    px, w, h0 = _f64(px), _f64(w), _f64(h0)
+    B, T, D = _shape(cell, px)
+    H = np.zeros((B, T, STATE_WIDTH[cell], D))
+    resid = np.zeros(K + 1)
+    rc = lib.oracle_newton_picard(cell, B, T, D, _ptr(px), _ptr(w), _ptr(h0), int(P), int(K), _ptr(H), _ptr(resid),
+                                  _threads(nthreads))
+    if rc:
+        raise ValueError("oracle_newton_picard rejected its arguments (%d)" % rc)
     return H, resid
 
 

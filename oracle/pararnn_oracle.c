@@ -16,6 +16,10 @@
  *     section; ParaRNN thread, tweet [3/8]), starting from the warm start
  *     h_t^(0) = f(0, x_t) (Method section, "paper App. A"), each linear
  *     system J delta = -F solved by a plain forward substitution in time;
+ *   - optionally P Picard (fixed-point) sweeps before the Newton iterations,
+ *     h_t^(p+1) = f(h_{t-1}^(p), x_t) with h_{-1}^(p) = h0, which warm the
+ *     first guess further (API overview, "Solver": picard_iters; Method
+ *     section: zero-hidden start plus Picard);
  *   - the adjoint of the recurrence at a given trajectory H: the reverse
  *     recursion lambda_t = g_t + A_{t+1}^T lambda_{t+1} and the parameter
  *     gradients it implies (Method section, "Backward follows paper eq. 2.6";
@@ -172,6 +176,7 @@ typedef struct {
     int cell, S, G;
     int64_t B, T, D;
     int K;
+    int P;                /* Picard sweeps before the Newton iterations */
     const double* px;
     const double* w;
     const double* h0;
@@ -244,6 +249,21 @@ static void channel_newton(job_t* j, int64_t b, int64_t d) {
         load_p(j, b, t, d, p);
         oracle_cell_step(j->cell, p, w, zero, fv);
         for (int i = 0; i < S; ++i) *Hat(j->H, j, b, t, i, d) = fv[i];
+    }
+    /* Picard sweeps: h_t^(p+1) = f(h_{t-1}^(p), x_t), h_{-1}^(p) = h0.  The
+     * rows are rewritten from the last one back, so that row t-1 still holds
+     * sweep p's value when row t is formed. */
+    for (int sweep = 0; sweep < j->P; ++sweep) {
+        double prev[MAXS];
+        for (int64_t t = j->T - 1; t >= 0; --t) {
+            load_p(j, b, t, d, p);
+            if (t > 0)
+                for (int i = 0; i < S; ++i) prev[i] = Hget(j->H, j, b, t - 1, i, d);
+            else
+                load_h0(j, b, d, prev);
+            oracle_cell_step(j->cell, p, w, prev, fv);
+            for (int i = 0; i < S; ++i) *Hat(j->H, j, b, t, i, d) = fv[i];
+        }
     }
     for (int k = 0; k < j->K; ++k) {
         /* Newton step: J(H) delta = -F(H).  J is lower block-bidiagonal with
@@ -380,19 +400,26 @@ int oracle_unroll(int cell, int64_t B, int64_t T, int64_t D, const double* px, c
     return run(&j, nthreads);
 }
 
-/* K Newton iterations from the warm start.  resid (K+1 doubles, may be NULL)
- * receives max |F(H^(k))| over the whole batch for k = 0..K. */
-int oracle_newton(int cell, int64_t B, int64_t T, int64_t D, const double* px, const double* w,
-                  const double* h0, int K, double* H, double* resid, int nthreads) {
-    if (check(cell, B, T, D, px) || (cell != 0 && !w) || K < 0 || K > 62) return -1;
+/* P Picard sweeps from the warm start, then K Newton iterations.  resid
+ * (K+1 doubles, may be NULL) receives max |F(H^(k))| over the whole batch for
+ * k = 0..K, H^(0) being the guess after the sweeps. */
+int oracle_newton_picard(int cell, int64_t B, int64_t T, int64_t D, const double* px, const double* w,
+                         const double* h0, int P, int K, double* H, double* resid, int nthreads) {
+    if (check(cell, B, T, D, px) || (cell != 0 && !w) || K < 0 || K > 62 || P < 0) return -1;
     job_t j;
     memset(&j, 0, sizeof j);
     j.cell = cell; j.S = ncell_state(cell); j.G = ncell_gates(cell);
-    j.B = B; j.T = T; j.D = D; j.K = K; j.px = px; j.w = w; j.h0 = h0; j.H = H; j.mode = 1;
+    j.B = B; j.T = T; j.D = D; j.K = K; j.P = P; j.px = px; j.w = w; j.h0 = h0; j.H = H; j.mode = 1;
     int rc = run(&j, nthreads);
     if (rc == 0 && resid)
         for (int k = 0; k <= K; ++k) resid[k] = j.resid[k];
     return rc;
+}
+
+/* K Newton iterations from the warm start (no Picard sweep). */
+int oracle_newton(int cell, int64_t B, int64_t T, int64_t D, const double* px, const double* w,
+                  const double* h0, int K, double* H, double* resid, int nthreads) {
+    return oracle_newton_picard(cell, B, T, D, px, w, h0, 0, K, H, resid, nthreads);
 }
 
 /* max |F(H)| = max_{b,t,s,d} |H_t - f(H_{t-1}, x_t)| (H_{-1} = h0) of a given

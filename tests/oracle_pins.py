@@ -24,6 +24,10 @@ What pins what:
                     then -lambda^T dF/dtheta by autograd) at an unconverged
                     iterate; BPTT by torch autograd at the unroll; central
                     finite differences of <g, unroll(theta)>.
+* Picard sweeps -- a plain loop over torch's cells from the warm start, a
+                    dense Newton step from the swept guess, and the prefix
+                    theorem (each sweep fixes one more leading row; T sweeps
+                    give the unroll).
 * residual       -- strictly decreasing over Newton steps on seeded cells of
                     every workload's cell (an empirical property, not a
                     theorem); max |F(H)| of an arbitrary trajectory against
@@ -230,6 +234,58 @@ def pin_prefix_exact():
                     _close(Hn[:, :n], U[:, :n], 1e-12, "cell %d prefix after %d steps" % (cell, k))
                 if k >= T:
                     _close(Hn, U, 1e-12, "cell %d after T steps" % cell)
+
+
+def pin_picard_torch_loop():
+    # P Picard sweeps from the warm start written as a plain loop over torch's
+    # cells, then one dense Newton step (autograd Jacobian, linear solve) from
+    # there: the oracle's sweeps and its Newton step from the swept guess
+    for cell in CELLS:
+        T, G, S = 10, oracle.NUM_GATES[cell], oracle.STATE_WIDTH[cell]
+        for h0flag in (False, True):
+            px, w, h0 = _rand_inputs(cell, 2, T, 2, seed=80 + cell + 5 * h0flag, h0=h0flag)
+            for P in (1, 2, 3):
+                Hp, _ = oracle.newton_picard(cell, px, w, h0, P=P, K=0)
+                H1, r1 = oracle.newton_picard(cell, px, w, h0, P=P, K=1)
+                for b in range(2):
+                    for d in range(2):
+                        p = torch.tensor(px[b, :, :, d])
+                        a = torch.tensor(_wcol(w, d, G))
+                        hh0 = torch.tensor(_h0col(h0, b, d, S))
+                        f = step_fn_weights(cell)
+                        X = [f(torch.zeros(S, dtype=torch.float64), p[t], a) for t in range(T)]
+                        for _ in range(P):
+                            X = [f(hh0 if t == 0 else X[t - 1], p[t], a) for t in range(T)]
+                        Xs = torch.stack(X)
+                        _close(Hp[b, :, :, d], Xs.numpy(), 1e-13, "cell %d Picard P=%d" % (cell, P))
+                        F = _dense_F(cell, p, a, hh0)
+                        Hf = Xs.reshape(-1)
+                        J = torch.autograd.functional.jacobian(lambda x: F(x, p, a, hh0), Hf)
+                        Hn = Hf + torch.linalg.solve(J, -F(Hf, p, a, hh0))
+                        _close(H1[b, :, :, d], Hn.detach().numpy().reshape(T, S), 1e-12,
+                               "cell %d Picard P=%d + Newton" % (cell, P))
+
+
+def pin_picard_prefix_exact():
+    # sweep p makes one more leading row exact: with h0 = 0 the warm start is
+    # already exact at t = 0, so P sweeps fix rows 0..P, and K Newton steps
+    # after them rows 0..P+K; P >= T sweeps alone give the unroll
+    for cell in CELLS:
+        T = 8
+        for h0flag in (False, True):
+            px, w, h0 = _rand_inputs(cell, 1, T, 2, seed=90 + cell + 7 * h0flag, h0=h0flag)
+            U = oracle.unroll(cell, px, w, h0)
+            for P in range(0, T + 1):
+                for K in (0, 1, 2):
+                    Hn, _ = oracle.newton_picard(cell, px, w, h0, P=P, K=K)
+                    n = min(T, P + K + (0 if h0flag else 1))
+                    if n:
+                        _close(Hn[:, :n], U[:, :n], 1e-12, "cell %d P=%d K=%d prefix" % (cell, P, K))
+                    if cell != oracle.LINEAR and n < T and K == 0:
+                        # the next row is not exact yet (a missing sweep would pass the check above)
+                        assert np.max(np.abs(Hn[:, n] - U[:, n])) > 1e-9, "cell %d P=%d row %d" % (cell, P, n)
+                if P >= T:
+                    _close(oracle.newton_picard(cell, px, w, h0, P=P, K=0)[0], U, 1e-12, "cell %d P=T" % cell)
 
 
 def pin_lstm_zero_weights():
@@ -545,7 +601,7 @@ def pin_head_adjoint_diagonal():
 
 
 ALL_PINS = [pin_cell_step, pin_jacobian, pin_param_grads, pin_unroll, pin_newton_dense, pin_affine_one_step,
-            pin_prefix_exact, pin_lstm_zero_weights, pin_adjoint_dense, pin_adjoint_bptt, pin_adjoint_fd,
+            pin_prefix_exact, pin_picard_torch_loop, pin_picard_prefix_exact, pin_lstm_zero_weights, pin_adjoint_dense, pin_adjoint_bptt, pin_adjoint_fd,
             pin_residual_monotone, pin_residual_function, pin_head_step_and_jacobian, pin_head_unroll, pin_head_newton_dense,
             pin_head_prefix_exact_and_diagonal, pin_head_adjoint_bptt, pin_head_adjoint_dense,
             pin_head_adjoint_diagonal]

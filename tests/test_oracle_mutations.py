@@ -38,6 +38,12 @@ MUTATIONS = {
                            "for (int m = 0; m < S; ++m) nl[i] += A[i * S + m] * lam[m];"),
     "adjoint_wrong_time_index": ("load_p(j, b, t + 1, d, pn);", "load_p(j, b, t, d, pn);"),
     "adjoint_da_uses_dp": ("ga += lam[i] * da[i * G + g];", "ga += lam[i] * dp[i * G + g];"),
+    "picard_forward_order": ("for (int64_t t = j->T - 1; t >= 0; --t) {\n            load_p(j, b, t, d, p);\n            if (t > 0)",
+                             "for (int64_t t = 0; t < j->T; ++t) {\n            load_p(j, b, t, d, p);\n            if (t > 0)"),
+    "picard_sweep_skipped": ("for (int sweep = 0; sweep < j->P; ++sweep) {", "for (int sweep = 1; sweep < j->P; ++sweep) {"),
+    "picard_zero_initial_state": ("            else\n                load_h0(j, b, d, prev);\n            oracle_cell_step(j->cell, p, w, prev, fv);",
+                                  "            else\n                prev[0] = prev[1] = 0.0;\n            oracle_cell_step(j->cell, p, w, prev, fv);"),
+    "residual_wrong_row": ("cur[i] = Hget(j->H, j, b, t, i, d);", "cur[i] = Hget(j->H, j, b, t > 0 ? t - 1 : 0, i, d);"),
     # head-wise GRU
     "head_step_weight_transposed": ("            az += Uz[(size_t)i * d + j] * s[j];\n            ar += Ur[(size_t)i * d + j] * s[j];\n"
                                     "            n += Uc[(size_t)i * d + j] * s[j];\n        }\n"
