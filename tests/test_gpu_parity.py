@@ -217,26 +217,24 @@ def test_deterministic(cuda_device):
 # float32 rounding errors of f (activations within 4e-6 relative), far below
 # this bound times the largest state
 RESID_ABS, RESID_REL = 2e-5, 1e-4
-# below this (times the largest state) a residual is float32 rounding noise
-RESID_FLOOR = 1e-5
 
 
-def _full_residuals(w, x, H, chunk=256):
-    """(max |F(h^(0))|, max |F(H)|) over every channel of a full-size
-    workload, by the oracle: the warm start's residual is the K = 0 entry of
-    its Newton history; H's is its residual function.  The device tensors are
-    copied to the host a slice of channels at a time."""
-    r0 = rK = 0.0
+def _full_residuals(w, x, Hs, chunk=256):
+    """[max |F(h^(0))|] + [max |F(H)| for H in Hs] over every channel of a
+    full-size workload, by the oracle: the warm start's residual is the K = 0
+    entry of its Newton history, each H's is its residual function.  The
+    device tensors are copied to the host a slice of channels at a time."""
+    r = [0.0] * (1 + len(Hs))
     for d0 in range(0, w.D, chunk):
         d1 = min(w.D, d0 + chunk)
         px = x["px"][:, :, :, d0:d1].float().cpu().numpy()
         a = None if x["a"] is None else x["a"][:, d0:d1].cpu().numpy()
-        Hc = H[:, :, :, d0:d1].cpu().numpy()
         _, ro = oracle.newton(w.cell_id, px, a, None, K=0)
-        r0 = max(r0, float(ro[0]))
-        rK = max(rK, oracle.residual(w.cell_id, px, a, None, Hc))
-        del px, Hc
-    return r0, rK
+        r[0] = max(r[0], float(ro[0]))
+        for i, H in enumerate(Hs):
+            r[i + 1] = max(r[i + 1], oracle.residual(w.cell_id, px, a, None, H[:, :, :, d0:d1].cpu().numpy()))
+        del px
+    return r
 
 
 @pytest.mark.parametrize("name", [n for n in workloads.WORKLOADS])
@@ -256,29 +254,30 @@ def test_workload_full_size_sampled(name, cuda_device):
     # oracle on the sampled channels: a (1,T,G,n) problem from the gathered values
     px1 = pxs_dev[None]
     w1 = None if a_np is None else a_np[:, [d for _, d in chans]]
-    Ho, ro = oracle.newton(w.cell_id, px1, w1, None, K=w.K)
+    Ho, _ = oracle.newton(w.cell_id, px1, w1, None, K=w.K)
     assert rel_err(Hs, Ho[0]) <= TOL_H, name
     if w.px_dtype == "bf16":
         px32s = gather_channels(x["px32"], chans)[None]
         Hf, _ = oracle.newton(w.cell_id, px32s, w1, None, K=w.K)
         assert norm_err(Hs, Hf[0]) <= TOL_BF16_F32, name
-    # the residual history is a max over the whole batch
+    # the residual history is a max over the whole batch.  Every entry is
+    # pinned over every channel by the oracle's fp64 max |F|: r[0] at the warm
+    # start, r[K] at the returned H, and r[k] at the output of a k-iteration
+    # call, whose iterates are bit-identical to the first k of this call's
+    # (the same arithmetic in the same order; results do not depend on
+    # timing).  Over millions of channels the maximum need not fall at every
+    # step -- Newton converges only locally, and the LSTM workload's first
+    # step raises it -- so the history is pinned entry by entry, not by a
+    # trend.
     r = to_np(resid)
-    print("%s: GPU residual history %s" % (name, r))
-    # its two ends are pinned over every channel: r[0] is max |F| of the warm
-    # start and r[K] max |F| of the returned H, both by the oracle in fp64;
-    # the kernel evaluates f in float32, so they agree to float32 rounding
-    r0, rK = _full_residuals(w, x, H)
+    Hk = [binding.newton_forward(w.cell_id, x["px"], x["a"], None, K=k) for k in range(1, w.K)]
+    ref = _full_residuals(w, x, Hk + [H])
+    print("%s: GPU residual history %s, oracle %s" % (name, r, np.array(ref)))
     scale = max(1.0, float(H.abs().max()))  # float32 rounding scales with the state's size
-    assert abs(r[0] - r0) <= RESID_ABS * scale + RESID_REL * r0, (r, r0)
-    assert abs(r[-1] - rK) <= RESID_ABS * scale + RESID_REL * rK, (r, rK)
-    # the iterates in between are not kept; the sample's history is a lower bound
-    assert np.all(r[:-1] + 1e-5 >= ro[:-1] * (1 - 1e-3)), (r, ro)
-    # and every Newton step lowers the residual until it reaches the float32
-    # rounding floor (the seeded cells' property the oracle's pins check in
-    # fp64)
-    for k in range(w.K):
-        assert r[k + 1] < r[k] or r[k + 1] <= RESID_FLOOR * scale, (k, r)
+    for k in range(w.K + 1):
+        assert abs(r[k] - ref[k]) <= RESID_ABS * scale + RESID_REL * ref[k], (k, r, ref)
+    del Hk
+    assert r[-1] < r[0], r
     if w.backward:
         g = x["dLdH"]
         dpx, da, _ = binding.newton_backward(w.cell_id, x["px"], H, g, x["a"])
