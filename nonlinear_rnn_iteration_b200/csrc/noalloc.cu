@@ -26,23 +26,27 @@ constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char g_scratch[kScratchBytes];
 
-// Per device: the array's device address, looked up once with that device
+// Per device: the array's device address, looked up with that device
 // current (in host code the array's name is only a stand-in, not an address
-// a kernel may use), and the outcome of that set-up.
-std::once_flag g_once[kMaxDevices];
+// a kernel may use).  A failed look-up is not remembered, so a later call
+// retries it.  The array needs no clearing: every forward call clears the
+// part of its workspace that it reads.
+std::mutex g_mutex;
 void* g_scratch_ptr[kMaxDevices];
-cudaError_t g_setup_err[kMaxDevices];
 
-void setup_device(int dev) {
-    void* p = nullptr;
-    cudaError_t e = cudaGetSymbolAddress(&p, g_scratch);
-    // the carries in the workspace must start out zero-filled; later calls
-    // keep it consistent themselves
-    if (e == cudaSuccess) e = cudaMemset(p, 0, kScratchBytes);
-    if (e == cudaSuccess) e = cudaDeviceSynchronize();
-    if (e != cudaSuccess) cudaGetLastError();
-    g_setup_err[dev] = e;
-    g_scratch_ptr[dev] = e == cudaSuccess ? p : nullptr;
+cudaError_t scratch_for(int dev, void** out) {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (!g_scratch_ptr[dev]) {
+        void* p = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&p, g_scratch);
+        if (e != cudaSuccess) {
+            cudaGetLastError();
+            return e;
+        }
+        g_scratch_ptr[dev] = p;
+    }
+    *out = g_scratch_ptr[dev];
+    return cudaSuccess;
 }
 
 }  // namespace
@@ -61,24 +65,27 @@ extern "C" pararnn_status pararnn_newton_forward_noalloc(pararnn_cell cell, int6
         pararnn::set_last_error("pararnn_newton_forward_noalloc: device ordinal out of range");
         return PARARNN_EINVAL;
     }
-    const size_t need = pararnn_workspace_bytes(cell, B, T, D, K);
-    if (need == 0 || K < 1) {
-        pararnn::set_last_error("pararnn_newton_forward_noalloc: bad cell, size or K");
+    if (K < 0) {
+        pararnn::set_last_error("pararnn_newton_forward_noalloc: K must be 0 (the measured K*) or at least 1");
         return PARARNN_EINVAL;
     }
+    // 0 means invalid sizes or cell; pararnn_workspace_bytes has then already
+    // stored the specific reason for pararnn_last_error()
+    const size_t need = pararnn_workspace_bytes(cell, B, T, D, K);
+    if (need == 0) return PARARNN_EINVAL;
     if (need > kScratchBytes) {
         pararnn::set_last_error(
             "pararnn_newton_forward_noalloc: this problem needs more scratch memory than the fixed 32 MiB array "
             "holds; use pararnn_newton_forward with a workspace of pararnn_workspace_bytes() bytes");
         return PARARNN_EINVAL;
     }
-    std::call_once(g_once[dev], setup_device, dev);
-    if (g_setup_err[dev] != cudaSuccess) {
-        pararnn::set_last_error("pararnn_newton_forward_noalloc: could not set up the scratch array on this device");
+    void* scratch = nullptr;
+    if (scratch_for(dev, &scratch) != cudaSuccess) {
+        pararnn::set_last_error("pararnn_newton_forward_noalloc: could not look up the scratch array on this device");
         return PARARNN_ECUDA;
     }
-    pararnn_status st = pararnn_newton_forward(cell, B, T, D, px_dtype, preacts, diag_w, h0, K, H_out,
-                                               g_scratch_ptr[dev], kScratchBytes, resid_hist, stream);
+    pararnn_status st = pararnn_newton_forward(cell, B, T, D, px_dtype, preacts, diag_w, h0, K, H_out, scratch,
+                                               kScratchBytes, resid_hist, stream);
     if (st != PARARNN_OK || !wait_status) return st;
-    return pararnn_status_sync(g_scratch_ptr[dev], stream);
+    return pararnn_status_sync(scratch, stream);
 }

@@ -44,6 +44,31 @@ def test_noalloc_forward_matches_forward_on_two_calls_in_a_row(cuda_device):
         assert torch.isfinite(resid).all() and resid[-1] < resid[0]
 
 
+def test_noalloc_forward_allocates_no_device_memory(cuda_device):
+    # after a first call (which looks up the array on this device), further
+    # calls leave both torch's allocator counters and the driver's free
+    # device memory exactly where they were
+    stream = torch.cuda.current_stream()
+    cell, B, T, D, K = binding.DIAG_GRU, 1, 500, 128, 3
+    px, w = _problem(cell, B, T, D, 21)
+    H = torch.empty((B, T, 1, D), device=DEV)
+    resid = torch.empty(K + 1, device=DEV)
+    st = binding.pararnn_newton_forward_noalloc(cell, B, T, D, binding.F32, px, w, None, K, H, resid, 1, stream)
+    assert st == binding.OK, binding.pararnn_last_error()
+    torch.cuda.synchronize()
+    stats0 = torch.cuda.memory_stats()
+    free0, _ = torch.cuda.mem_get_info()
+    for _ in range(3):
+        st = binding.pararnn_newton_forward_noalloc(cell, B, T, D, binding.F32, px, w, None, K, H, resid, 1, stream)
+        assert st == binding.OK, binding.pararnn_last_error()
+    torch.cuda.synchronize()
+    stats1 = torch.cuda.memory_stats()
+    free1, _ = torch.cuda.mem_get_info()
+    for key in ("allocation.all.allocated", "segment.all.allocated", "reserved_bytes.all.current"):
+        assert stats1.get(key, 0) == stats0.get(key, 0), key
+    assert free1 == free0
+
+
 def test_noalloc_forward_rejects_problems_beyond_its_array(cuda_device):
     px = torch.empty(1, device=DEV)
     H = torch.empty(1, device=DEV)
