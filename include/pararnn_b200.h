@@ -100,33 +100,68 @@ int pararnn_state_width(pararnn_cell cell);
  * pararnn_newton_backward need for a (B, T, D) problem; the same buffer
  * serves both.  0 for an unknown cell or a negative size.  Pure host
  * function.  The workspace holds a status word, a tile counter, the
- * inter-block scan carries and per-block gradient partials.  Zero-fill it
- * once after allocating it (cudaMemset); after that the library keeps it
- * consistent from call to call: carries are tagged with a per-call number
- * and words left by earlier calls never read as valid.  Calls that share a
- * workspace must be ordered (the same stream, or synchronised); calls that
+ * inter-block scan carries and per-block gradient partials.  It needs no
+ * initialisation: every call clears, on its stream and before its kernels
+ * run, every word of it that the call reads before writing (the status word,
+ * the tile counter and all scan carries), so whatever an earlier call -- or
+ * any other use of the memory -- left there is never read.  Calls that share
+ * a workspace must be ordered (the same stream, or synchronised); calls that
  * overlap on the GPU with one workspace race. */
 size_t pararnn_workspace_bytes(pararnn_cell cell, int64_t B, int64_t T, int64_t D, int K);
 
-/* Newton forward: K >= 1 iterations from the warm start, output H = h^(K).
+/* The measured Newton budget K*(cell, T) that K = 0 selects (pararnn-torch
+ * page, Method section: K*(T) is the smallest iteration count that matches
+ * the sequential unroll within about 1e-4, measured per cell on a T grid,
+ * and NewtonConfig(max_iters=None) reads those tables).  Here the table was
+ * measured on this library's forward against an fp64 sequential unroll, on
+ * synthetic cells (pre-activations ~ N(0,1), diagonal recurrent weights
+ * ~ U(-0.5, 0.5), h0 = 0) at T = 16, 64, ..., 262144; a T between grid
+ * points takes the entry of the next grid point up, a T past the grid the
+ * last entry.  Inputs drawn otherwise (trained weights, saturated gates) can
+ * need another K.  Returns 1 for the linear cell (one scan is exact) and -1
+ * for an unknown cell or a negative T.  Pure host function. */
+int pararnn_kstar(pararnn_cell cell, int64_t T);
+
+/* Newton forward: K iterations from the warm start, output H = h^(K).
  * (Method section; NewtonConfig(max_iters=K), API overview section.)
  *   preacts    (B,T,G,D) in px_dtype, read only
  *   diag_w     (G,D) f32 or NULL (zeros)
  *   h0         (B,S,D) f32 or NULL (zeros)
- *   K          1..64 Newton iterations; the linear cell is exact after one,
- *              and performs exactly one scan for any K
+ *   K          1..64 Newton iterations, or 0 for K = pararnn_kstar(cell, T)
+ *              (max_iters=None); the linear cell is exact after one, and
+ *              performs exactly one scan for any K
  *   H_out      (B,T,S,D) f32, written
  *   workspace  >= pararnn_workspace_bytes(cell,B,T,D,K) bytes, 16-byte
- *              aligned, zero-filled once after allocation
+ *              aligned device memory, any contents (cleared on `stream`)
  *   resid_hist NULL, or K+1 floats of device memory that receive
  *              max_{b,t,s,d} |F(H^(k))| for k = 0..K (the residual history a
- *              NewtonDivergenceError carries, Evaluation section)
+ *              NewtonDivergenceError carries, Evaluation section); with
+ *              K = 0, pararnn_kstar(cell, T) + 1 floats
  * B, T or D equal to 0 is an empty problem: nothing is launched except the
  * zeroing of resid_hist. */
 pararnn_status pararnn_newton_forward(pararnn_cell cell, int64_t B, int64_t T, int64_t D,
                                       pararnn_dtype px_dtype, const void* preacts, const float* diag_w,
                                       const float* h0, int K, float* H_out, void* workspace,
                                       size_t ws_bytes, float* resid_hist, void* stream);
+
+/* The Newton forward with picard_iters Picard sweeps before the Newton
+ * iterations (API overview, "Solver": picard_iters warms the first guess;
+ * Method section: a zero-hidden start plus Picard).  From the warm start
+ * h^(0)_t = f(0, x_t), each sweep forms h^(p+1)_t = f(h^(p)_{t-1}, x_t) for
+ * every t at once, with h^(p)_{-1} = h0; sweep p makes the first p rows
+ * (p + 1 when h0 is zero) equal to the sequential unroll.  The K Newton
+ * iterations then start from h^(P), and resid_hist[0] is the residual of
+ * h^(P).  picard_iters is 0..4 (0: exactly pararnn_newton_forward); the
+ * linear cell ignores it.  Every other argument, the workspace size and the
+ * errors are those of pararnn_newton_forward; a picard_iters outside 0..4
+ * returns PARARNN_EINVAL.  The sweeps run inside the same kernel as the
+ * Newton iterations: each thread evaluates its rows and the picard_iters + 1
+ * rows before them, so no further HBM traffic or look-back is needed. */
+pararnn_status pararnn_newton_forward_picard(pararnn_cell cell, int64_t B, int64_t T, int64_t D,
+                                             pararnn_dtype px_dtype, const void* preacts, const float* diag_w,
+                                             const float* h0, int picard_iters, int K, float* H_out,
+                                             void* workspace, size_t ws_bytes, float* resid_hist,
+                                             void* stream);
 
 /* Adjoint (backward) at the trajectory H (normally the forward's output):
  *   lambda_t = dL/dH_t + A_{t+1}^T lambda_{t+1},  lambda_{T-1} = dL/dH_{T-1},
@@ -160,6 +195,40 @@ const char* pararnn_status_string(pararnn_status status);
  * the calling thread ("" if none). */
 const char* pararnn_last_error(void);
 
+/* Test hooks for the bounded waits between thread blocks and for the choice
+ * of path (no counterpart on the pages).  They apply to the
+ * pararnn_newton_forward and pararnn_newton_backward calls made afterwards on
+ * the calling thread:
+ *   wait_limit_ns  the limit of every wait of one thread block on another
+ *                  (a look-back for a predecessor's carry, a staged tile);
+ *                  0 restores the default of 2 s; at most 10 s
+ *   flags          PARARNN_HOOK_STALL_FIRST_TILE: the first tile of the scan
+ *                  computes as usual but never publishes its carry, so the
+ *                  look-back of the tile after it runs out of time.  The
+ *                  waiting block then records PARARNN_ETIMEOUT in the
+ *                  workspace, takes a zero carry and finishes; the kernel ends
+ *                  after about K * wait_limit_ns and pararnn_status_sync()
+ *                  reports PARARNN_ETIMEOUT.  Outputs of such a call are
+ *                  invalid.  Forwards take the look-back path while it is set.
+ *                  PARARNN_HOOK_NO_CLUSTER: forwards never take the
+ *                  small-problem path (below), so that both paths can be
+ *                  compared on the same small inputs.
+ *                  0 clears both.
+ * Returns PARARNN_EINVAL (nothing changed) for a limit above 10 s or an
+ * unknown flag.  Pure host function.
+ *
+ * The small-problem path: when every channel group's tiles along T fit in
+ * one thread-block cluster (T up to 8 tiles: 1024 steps for the GRU, 560 for
+ * the LSTM, 1024 for the linear cell), pararnn_newton_forward runs as one
+ * kernel whose thread blocks pass their carries through distributed shared
+ * memory; it launches nothing else (no clearing of the workspace) and
+ * records its status in a word tagged with its call number, which
+ * pararnn_status_sync() reads.  Its results are bit-identical to the
+ * look-back path's. */
+#define PARARNN_HOOK_STALL_FIRST_TILE 1
+#define PARARNN_HOOK_NO_CLUSTER 2
+pararnn_status pararnn_debug_hooks(uint64_t wait_limit_ns, int flags);
+
 /* Runs the library's bounded inter-block wait on a flag that nothing sets,
  * with a limit of timeout_ns nanoseconds, so that a test can see the time-out
  * path end cleanly: the kernel records PARARNN_ETIMEOUT in the workspace and
@@ -183,11 +252,14 @@ pararnn_status pararnn_probe_wait_timeout(void* workspace, size_t ws_bytes, uint
  *                device status as pararnn_status_sync would.
  * Problems whose pararnn_workspace_bytes(cell, B, T, D, K) exceeds 32 MiB
  * return PARARNN_EINVAL with an explanation in pararnn_last_error().  The
- * first call on a device sets that device up (it looks up the array's device
- * address and clears the array once, synchronising the device): make that
- * first call before any stream capture.  All calls share the one array, which
- * keeps the last call's contents: calls that overlap on the GPU race, so
- * order them (one stream, or synchronise between them). */
+ * first call on a device sets that device up: it looks up the array's device
+ * address with cudaGetSymbolAddress (which may load the library's device code
+ * onto that device), so make that first call before any stream capture.  A
+ * failed look-up returns PARARNN_ECUDA and is tried again on the next call.
+ * All calls share the one array, which keeps the last call's contents; each
+ * call clears, on `stream`, the part it reads before writing, as
+ * pararnn_newton_forward does with its workspace.  Calls that overlap on the
+ * GPU race, so order them (one stream, or synchronise between them). */
 pararnn_status pararnn_newton_forward_noalloc(pararnn_cell cell, int64_t B, int64_t T, int64_t D,
                                               pararnn_dtype px_dtype, const void* preacts, const float* diag_w,
                                               const float* h0, int K, float* H_out, float* resid_hist,
@@ -211,8 +283,7 @@ pararnn_status pararnn_newton_forward_noalloc(pararnn_cell cell, int64_t B, int6
  *   diag_w, h0    device memory, as for pararnn_newton_forward
  *   H_host        (B, T, S, D) float32, host (or device) memory
  *   workspace     >= pararnn_newton_forward_host_workspace_bytes(...) bytes,
- *                 256-byte aligned device memory, zero-filled once at
- *                 allocation like the ordinary workspace
+ *                 256-byte aligned device memory, any contents
  * The work is ordered after what is already queued on `stream`, and work
  * queued on `stream` afterwards runs after it; the call returns once
  * everything is queued.  No residual history is kept.  A non-finite value in
@@ -269,7 +340,9 @@ size_t pararnn_head_gru_workspace_bytes(int64_t B, int64_t T, int64_t D, int n_h
  * a missing or small workspace, and null, host or misaligned pointers;
  * PARARNN_ECUDA if a launch fails.  A non-finite value in H_out is recorded in
  * the workspace and returned by pararnn_status_sync(workspace, stream).  No
- * thread block waits on another, so PARARNN_ETIMEOUT does not occur. */
+ * thread block waits on another, but a block waits on its own tensor-core
+ * products; if such a wait runs past 1 s the block stops issuing products and
+ * records PARARNN_ETIMEOUT, which pararnn_status_sync() then returns. */
 pararnn_status pararnn_head_gru_forward(int64_t B, int64_t T, int64_t D, int n_heads, pararnn_dtype px_dtype,
                                         const void* preacts, const float* U, const float* h0, int K, float* H_out,
                                         void* workspace, size_t ws_bytes, float* resid_hist, void* stream);
@@ -300,6 +373,25 @@ pararnn_status pararnn_head_gru_backward(int64_t B, int64_t T, int64_t D, int n_
                                          const void* preacts, const float* U, const float* h0, const float* H,
                                          const float* dL_dH, float* dL_dpx, float* dL_dU, float* dL_dh0,
                                          void* workspace, size_t ws_bytes, void* stream);
+
+/* The sequential unroll of the head-wise GRU, s_t = f(s_{t-1}, x_t) for
+ * t = 0..T-1 with s_{-1} = h0: the one-step recurrence that the Newton
+ * forward reproduces at convergence (pararnn-torch page, API overview /
+ * Quickstart: sequential_apply beside newton_apply).  One thread block per
+ * (batch row, head) walks the sequence with the head's d x d blocks in
+ * registers (3 d^2 multiply-adds per step, against the Newton scan's d x d x d
+ * products), so it suits problems with many sequences; the Newton forward
+ * suits few long ones.  Same layouts and head widths (16, 32, 64) as
+ * pararnn_head_gru_forward; preacts must be 16-byte aligned.
+ *   workspace  >= 256 bytes of device memory (only its status word is used;
+ *              cleared on `stream`)
+ * Errors: PARARNN_EINVAL (nothing launched) for bad sizes, dtype, pointers or
+ * workspace; PARARNN_ECUDA if the launch fails.  A non-finite value in H_out
+ * is recorded for pararnn_status_sync(workspace, stream).  No block waits on
+ * another. */
+pararnn_status pararnn_head_gru_unroll(int64_t B, int64_t T, int64_t D, int n_heads, pararnn_dtype px_dtype,
+                                       const void* preacts, const float* U, const float* h0, float* H_out,
+                                       void* workspace, size_t ws_bytes, void* stream);
 
 #ifdef __cplusplus
 }

@@ -30,12 +30,15 @@ SIGNATURES = {
     "pararnn_num_gates": (_I, [_I]),
     "pararnn_state_width": (_I, [_I]),
     "pararnn_workspace_bytes": (_SZ, [_I, _I64, _I64, _I64, _I]),
+    "pararnn_kstar": (_I, [_I, _I64]),
     "pararnn_newton_forward": (_I, [_I, _I64, _I64, _I64, _I, _P, _P, _P, _I, _P, _P, _SZ, _P, _P]),
+    "pararnn_newton_forward_picard": (_I, [_I, _I64, _I64, _I64, _I, _P, _P, _P, _I, _I, _P, _P, _SZ, _P, _P]),
     "pararnn_newton_backward": (_I, [_I, _I64, _I64, _I64, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "pararnn_status_sync": (_I, [_P, _P]),
     "pararnn_status_string": (ctypes.c_char_p, [_I]),
     "pararnn_last_error": (ctypes.c_char_p, []),
     "pararnn_probe_wait_timeout": (_I, [_P, _SZ, _U64, _P]),
+    "pararnn_debug_hooks": (_I, [_U64, _I]),
     "pararnn_newton_forward_noalloc": (_I, [_I, _I64, _I64, _I64, _I, _P, _P, _P, _I, _P, _P, _I, _P]),
     "pararnn_newton_forward_host_workspace_bytes": (_SZ, [_I, _I64, _I64, _I64, _I, _I, _I64, _I64]),
     "pararnn_newton_forward_host": (_I, [_I, _I64, _I64, _I64, _I, _P, _P, _P, _I, _P, _P, _SZ, _I64, _I64, _P]),
@@ -43,6 +46,7 @@ SIGNATURES = {
     "pararnn_head_gru_forward": (_I, [_I64, _I64, _I64, _I, _I, _P, _P, _P, _I, _P, _P, _SZ, _P, _P]),
     "pararnn_head_gru_backward_workspace_bytes": (_SZ, [_I64, _I64, _I64, _I]),
     "pararnn_head_gru_backward": (_I, [_I64, _I64, _I64, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "pararnn_head_gru_unroll": (_I, [_I64, _I64, _I64, _I, _I, _P, _P, _P, _P, _P, _SZ, _P]),
 }
 
 _lib = None
@@ -111,6 +115,17 @@ def pararnn_newton_forward(cell, B, T, D, px_dtype, preacts, diag_w, h0, K, H_ou
                                          _ptr(H_out), _ptr(workspace), ws_bytes, _ptr(resid_hist), _stream(stream))
 
 
+def pararnn_kstar(cell, T):
+    return load().pararnn_kstar(cell, T)
+
+
+def pararnn_newton_forward_picard(cell, B, T, D, px_dtype, preacts, diag_w, h0, picard_iters, K, H_out, workspace,
+                                  ws_bytes, resid_hist, stream):
+    return load().pararnn_newton_forward_picard(cell, B, T, D, px_dtype, _ptr(preacts), _ptr(diag_w), _ptr(h0),
+                                                picard_iters, K, _ptr(H_out), _ptr(workspace), ws_bytes,
+                                                _ptr(resid_hist), _stream(stream))
+
+
 def pararnn_newton_backward(cell, B, T, D, px_dtype, preacts, diag_w, h0, H, dL_dH, dL_dpx, dL_da, dL_dh0,
                             workspace, ws_bytes, stream):
     return load().pararnn_newton_backward(cell, B, T, D, px_dtype, _ptr(preacts), _ptr(diag_w), _ptr(h0), _ptr(H),
@@ -132,6 +147,10 @@ def pararnn_last_error():
 
 def pararnn_probe_wait_timeout(workspace, ws_bytes, timeout_ns, stream):
     return load().pararnn_probe_wait_timeout(_ptr(workspace), ws_bytes, timeout_ns, _stream(stream))
+
+
+def pararnn_debug_hooks(wait_limit_ns, stall_first_tile):
+    return load().pararnn_debug_hooks(wait_limit_ns, int(stall_first_tile))
 
 
 def pararnn_newton_forward_noalloc(cell, B, T, D, px_dtype, preacts, diag_w, h0, K, H_out, resid_hist, wait_status,
@@ -174,6 +193,11 @@ def pararnn_head_gru_backward(B, T, D, n_heads, px_dtype, preacts, U, h0, H, dL_
                                             ws_bytes, _stream(stream))
 
 
+def pararnn_head_gru_unroll(B, T, D, n_heads, px_dtype, preacts, U, h0, H_out, workspace, ws_bytes, stream):
+    return load().pararnn_head_gru_unroll(B, T, D, n_heads, px_dtype, _ptr(preacts), _ptr(U), _ptr(h0), _ptr(H_out),
+                                          _ptr(workspace), ws_bytes, _stream(stream))
+
+
 # ---- tensor-level helpers (allocation through torch, compute in the library) ----
 
 def _check(status, where):
@@ -202,19 +226,22 @@ def _shape(cell, px):
 
 
 def workspace_for(cell, B, T, D, K, device):
-    """A zero-filled workspace (the one initialisation the C ABI asks for)."""
+    """An uninitialised workspace: every call clears what it reads."""
     import torch
 
     n = pararnn_workspace_bytes(cell, B, T, D, K)
-    return torch.zeros(n, dtype=torch.uint8, device=device)
+    return torch.empty(n, dtype=torch.uint8, device=device)
 
 
 def newton_forward(cell, px, diag_w=None, h0=None, K=1, out=None, workspace=None, resid_hist=None, stream=None,
-                   sync_status=True):
-    """H = h^(K) of shape (B,T,S,D), float32, on px's device."""
+                   sync_status=True, picard_iters=0):
+    """H = h^(K) of shape (B,T,S,D), float32, on px's device.  K=0 (or None)
+    takes the measured K*(cell, T); picard_iters > 0 runs that many Picard
+    sweeps before the Newton iterations."""
     import torch
 
     cell = CELLS.get(cell, cell)
+    K = 0 if K is None else K
     B, T, D = _shape(cell, px)
     S = pararnn_state_width(cell)
     if out is None:
@@ -222,8 +249,13 @@ def newton_forward(cell, px, diag_w=None, h0=None, K=1, out=None, workspace=None
     if workspace is None:
         workspace = workspace_for(cell, B, T, D, K, px.device)
     st = stream if stream is not None else torch.cuda.current_stream(px.device)
-    _check(pararnn_newton_forward(cell, B, T, D, _dtype_code(px), px, diag_w, h0, K, out, workspace,
-                                  workspace.numel(), resid_hist, st), "pararnn_newton_forward")
+    if picard_iters:
+        _check(pararnn_newton_forward_picard(cell, B, T, D, _dtype_code(px), px, diag_w, h0, picard_iters, K, out,
+                                             workspace, workspace.numel(), resid_hist, st),
+               "pararnn_newton_forward_picard")
+    else:
+        _check(pararnn_newton_forward(cell, B, T, D, _dtype_code(px), px, diag_w, h0, K, out, workspace,
+                                      workspace.numel(), resid_hist, st), "pararnn_newton_forward")
     if sync_status:
         _check(pararnn_status_sync(workspace, st), "pararnn_newton_forward (device status)")
     return out
@@ -296,6 +328,26 @@ def head_gru_backward(px, U, H, dL_dH, h0=None, want_dU=True, want_dh0=False, wo
     if sync_status:
         _check(pararnn_status_sync(workspace, st), "pararnn_head_gru_backward (device status)")
     return dpx, dU, dh0
+
+
+def head_gru_unroll(px, U, h0=None, out=None, workspace=None, stream=None, sync_status=True):
+    """Head-wise GRU, sequential unroll on the GPU: px (B,T,3,D), U (3,n_heads,d,d) -> H (B,T,D), float32."""
+    import torch
+
+    if px.dim() != 4 or px.shape[2] != 3 or not px.is_contiguous():
+        raise ValueError("preacts must be contiguous (B, T, 3, D), got %s" % (tuple(px.shape),))
+    B, T, _, D = px.shape
+    nh = U.shape[1]
+    if out is None:
+        out = torch.empty((B, T, D), dtype=torch.float32, device=px.device)
+    if workspace is None:
+        workspace = torch.empty(256, dtype=torch.uint8, device=px.device)
+    st = stream if stream is not None else torch.cuda.current_stream(px.device)
+    _check(pararnn_head_gru_unroll(B, T, D, nh, _dtype_code(px), px, U, h0, out, workspace, workspace.numel(), st),
+           "pararnn_head_gru_unroll")
+    if sync_status:
+        _check(pararnn_status_sync(workspace, st), "pararnn_head_gru_unroll (device status)")
+    return out
 
 
 def newton_forward_host(cell, px_host, diag_w=None, h0=None, K=1, out_host=None, rows_per_slice=1,

@@ -138,6 +138,17 @@ __device__ __forceinline__ void issue_bwd_load(const BwdMaps<Sh>* maps, BwdSmem<
     tile_load<kStream>(&sm.stg[stage].g[0][0][0], &maps->g, &sm.bar[stage], (int)d0, 0, row);
 }
 
+// y = A^T v on a pair of channels
+template <int S>
+__device__ __forceinline__ void mat_t_vec2(const f2 (&A)[S * S], const f2 (&v)[S], f2 (&y)[S]) {
+    if constexpr (S == 1) {
+        y[0] = mul2(A[0], v[0]);
+    } else {
+        y[0] = fma2(A[0], v[0], mul2(A[2], v[1]));
+        y[1] = fma2(A[1], v[0], mul2(A[3], v[1]));
+    }
+}
+
 // y = A^T v
 template <int S>
 __device__ __forceinline__ void mat_t_vec(const float (&A)[S * S], const float (&v)[S], float (&y)[S]) {
@@ -288,6 +299,16 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
 #pragma unroll
                 for (int g = 0; g < G; ++g) wr[v][g] = sm.w[g][cc + v];
 
+            // two channels per instruction where the thread holds an even
+            // number of them (packed f32x2; same rounding as one by one)
+            constexpr bool kPack = (V % 2 == 0) && Cell::kNonlinear;
+            constexpr int VP = kPack ? V / 2 : 1;
+            typename Cell::W2 wp[VP];
+            if constexpr (kPack) {
+#pragma unroll
+                for (int q = 0; q < VP; ++q) wp[q] = Cell::weights2(wr[2 * q], wr[2 * q + 1]);
+            }
+
             // ---- linearisation at (h_{t-1}, x_t) and the sub-chunk's element,
             //      composed in scan order (latest row first) ----
             float jA[R][S * S][V], sens[R][NS][V], gr[R][S][V];
@@ -305,34 +326,90 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
                 for (int s = 0; s < S; ++s) lds_row<V>((t0 == 0 && row == 0) ? &sm.hprev[s][cc] : &sm.stg[st].H[row][s][cc], hv[s]);
 #pragma unroll
                 for (int s = 0; s < S; ++s) lds_row<V>(&sm.stg[st].g[row][s][cc], gr[r][s]);
+                if constexpr (kPack) {
 #pragma unroll
-                for (int v = 0; v < V; ++v) {
-                    float pg[G], spv[S], A[S * S], se[NS];
+                    for (int q = 0; q < VP; ++q) {
+                        const int v0 = 2 * q, v1 = 2 * q + 1;
+                        f2 pg[G], spv[S], A[S * S], se[NS], gv[S];
 #pragma unroll
-                    for (int g = 0; g < G; ++g) pg[g] = pv[g][v];
+                        for (int g = 0; g < G; ++g) pg[g] = f2{pv[g][v0], pv[g][v1]};
 #pragma unroll
-                    for (int s = 0; s < S; ++s) spv[s] = hv[s][v];
-                    Cell::bwd(pg, wr[v], spv, A, se);
-                    if (!rvalid) {
-                        // past the end of the sequence: the identity element
+                        for (int s = 0; s < S; ++s) spv[s] = f2{hv[s][v0], hv[s][v1]};
+                        Cell::bwd2(pg, wp[q], spv, A, se);
+                        if (!rvalid) {
+                            // past the end of the sequence: the identity element
 #pragma unroll
-                        for (int a = 0; a < S * S; ++a) A[a] = (a % (S + 1) == 0) ? 1.0f : 0.0f;
+                            for (int a = 0; a < S * S; ++a) A[a] = splat2((a % (S + 1) == 0) ? 1.0f : 0.0f);
 #pragma unroll
-                        for (int s = 0; s < S; ++s) gr[r][s][v] = 0.0f;
+                            for (int s = 0; s < S; ++s) {
+                                gr[r][s][v0] = 0.0f;
+                                gr[r][s][v1] = 0.0f;
+                            }
+                        }
+#pragma unroll
+                        for (int a = 0; a < S * S; ++a) {
+                            jA[r][a][v0] = A[a].x;
+                            jA[r][a][v1] = A[a].y;
+                        }
+#pragma unroll
+                        for (int n = 0; n < NS; ++n) {
+                            sens[r][n][v0] = se[n].x;
+                            sens[r][n][v1] = se[n].y;
+                        }
+                        f2 M[S * S], bv[S], accA[S * S], accb[S];
+#pragma unroll
+                        for (int i = 0; i < S; ++i)
+#pragma unroll
+                            for (int m = 0; m < S; ++m) M[i * S + m] = A[m * S + i];  // A^T
+#pragma unroll
+                        for (int s = 0; s < S; ++s) gv[s] = f2{gr[r][s][v0], gr[r][s][v1]};
+                        mat_t_vec2<S>(A, gv, bv);
+#pragma unroll
+                        for (int a = 0; a < S * S; ++a) accA[a] = f2{mine.e[v0].A[a], mine.e[v1].A[a]};
+#pragma unroll
+                        for (int s = 0; s < S; ++s) accb[s] = f2{mine.e[v0].b[s], mine.e[v1].b[s]};
+                        compose_after2<S>(M, bv, accA, accb);
+#pragma unroll
+                        for (int a = 0; a < S * S; ++a) {
+                            mine.e[v0].A[a] = accA[a].x;
+                            mine.e[v1].A[a] = accA[a].y;
+                        }
+#pragma unroll
+                        for (int s = 0; s < S; ++s) {
+                            mine.e[v0].b[s] = accb[s].x;
+                            mine.e[v1].b[s] = accb[s].y;
+                        }
                     }
+                } else {
 #pragma unroll
-                    for (int a = 0; a < S * S; ++a) jA[r][a][v] = A[a];
+                    for (int v = 0; v < V; ++v) {
+                        float pg[G], spv[S], A[S * S], se[NS];
 #pragma unroll
-                    for (int n = 0; n < NS; ++n) sens[r][n][v] = se[n];
-                    float M[S * S], gv[S], bv[S];
+                        for (int g = 0; g < G; ++g) pg[g] = pv[g][v];
 #pragma unroll
-                    for (int i = 0; i < S; ++i)
+                        for (int s = 0; s < S; ++s) spv[s] = hv[s][v];
+                        Cell::bwd(pg, wr[v], spv, A, se);
+                        if (!rvalid) {
+                            // past the end of the sequence: the identity element
 #pragma unroll
-                        for (int m = 0; m < S; ++m) M[i * S + m] = A[m * S + i];  // A^T
+                            for (int a = 0; a < S * S; ++a) A[a] = (a % (S + 1) == 0) ? 1.0f : 0.0f;
 #pragma unroll
-                    for (int s = 0; s < S; ++s) gv[s] = gr[r][s][v];
-                    mat_t_vec<S>(A, gv, bv);
-                    compose_after<S>(M, bv, mine.e[v]);
+                            for (int s = 0; s < S; ++s) gr[r][s][v] = 0.0f;
+                        }
+#pragma unroll
+                        for (int a = 0; a < S * S; ++a) jA[r][a][v] = A[a];
+#pragma unroll
+                        for (int n = 0; n < NS; ++n) sens[r][n][v] = se[n];
+                        float M[S * S], gv[S], bv[S];
+#pragma unroll
+                        for (int i = 0; i < S; ++i)
+#pragma unroll
+                            for (int m = 0; m < S; ++m) M[i * S + m] = A[m * S + i];  // A^T
+#pragma unroll
+                        for (int s = 0; s < S; ++s) gv[s] = gr[r][s][v];
+                        mat_t_vec<S>(A, gv, bv);
+                        compose_after<S>(M, bv, mine.e[v]);
+                    }
                 }
             }
             warp_prefix<S, V, LC, W, NW, true>(mine, excl, warp, lane, sm.wagg);
@@ -348,37 +425,92 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
                 for (int v = 0; v < V; ++v) da_acc[g][v] = 0.0f;
             float outp[R][G][V];
             bool bad = false;
+            if constexpr (kPack) {
 #pragma unroll
-            for (int v = 0; v < V; ++v) {
-                float x[S], cv[S];  // x = mu_{t+1}, the propagated adjoint after row t
+                for (int q = 0; q < VP; ++q) {
+                    const int v0 = 2 * q, v1 = 2 * q + 1;
+                    f2 x[S], cv[S], PA[S * S], Pb[S], dacc[G];  // x = mu_{t+1}
 #pragma unroll
-                for (int s = 0; s < S; ++s) cv[s] = sm.cin[s][cc + v];
-                apply<S>(pre.e[v].A, pre.e[v].b, cv, x);
+                    for (int s = 0; s < S; ++s) cv[s] = f2{sm.cin[s][cc + v0], sm.cin[s][cc + v1]};
 #pragma unroll
-                for (int r = R - 1; r >= 0; --r) {
-                    const bool rvalid = (tb + r < T) && cvalid;
-                    float lam[S], A[S * S];
+                    for (int a = 0; a < S * S; ++a) PA[a] = f2{pre.e[v0].A[a], pre.e[v1].A[a]};
 #pragma unroll
-                    for (int s = 0; s < S; ++s) lam[s] = gr[r][s][v] + x[s];
+                    for (int s = 0; s < S; ++s) Pb[s] = f2{pre.e[v0].b[s], pre.e[v1].b[s]};
+                    apply2<S>(PA, Pb, cv, x);
 #pragma unroll
-                    for (int a = 0; a < S * S; ++a) A[a] = jA[r][a][v];
-                    mat_t_vec<S>(A, lam, x);  // mu_t
-                    float se[NS], dp[G], da[G];
+                    for (int g = 0; g < G; ++g) dacc[g] = splat2(0.0f);
 #pragma unroll
-                    for (int n = 0; n < NS; ++n) se[n] = sens[r][n][v];
-                    Cell::grads(se, lam, dp, da);
+                    for (int r = R - 1; r >= 0; --r) {
+                        const bool rvalid = (tb + r < T) && cvalid;
+                        f2 lam[S], A[S * S], se[NS], dp[G], da[G];
 #pragma unroll
-                    for (int g2 = 0; g2 < G; ++g2) {
-                        outp[r][g2][v] = dp[g2];
+                        for (int s = 0; s < S; ++s) lam[s] = add2(f2{gr[r][s][v0], gr[r][s][v1]}, x[s]);
+#pragma unroll
+                        for (int a = 0; a < S * S; ++a) A[a] = f2{jA[r][a][v0], jA[r][a][v1]};
+                        mat_t_vec2<S>(A, lam, x);  // mu_t
+#pragma unroll
+                        for (int n = 0; n < NS; ++n) se[n] = f2{sens[r][n][v0], sens[r][n][v1]};
+                        Cell::grads2(se, lam, dp, da);
+#pragma unroll
+                        for (int g2 = 0; g2 < G; ++g2) {
+                            outp[r][g2][v0] = dp[g2].x;
+                            outp[r][g2][v1] = dp[g2].y;
+                        }
                         if (rvalid) {
-                            da_acc[g2][v] += da[g2];
-                            bad |= !isfinite(dp[g2]);
+#pragma unroll
+                            for (int g2 = 0; g2 < G; ++g2) {
+                                dacc[g2] = add2(dacc[g2], da[g2]);
+                                bad |= !isfinite(dp[g2].x) || !isfinite(dp[g2].y);
+                            }
+                        }
+                        if (r == 0 && tb == 0 && rvalid && prm.dLdh0) {
+                            // dL/dh0 = A_0^T lambda_0 = mu_0
+#pragma unroll
+                            for (int s = 0; s < S; ++s) {
+                                prm.dLdh0[(b * S + s) * D + d0 + cc + v0] = x[s].x;
+                                prm.dLdh0[(b * S + s) * D + d0 + cc + v1] = x[s].y;
+                            }
                         }
                     }
-                    if (r == 0 && tb == 0 && rvalid && prm.dLdh0) {
-                        // dL/dh0 = A_0^T lambda_0 = mu_0
 #pragma unroll
-                        for (int s = 0; s < S; ++s) prm.dLdh0[(b * S + s) * D + d0 + cc + v] = x[s];
+                    for (int g = 0; g < G; ++g) {
+                        da_acc[g][v0] = dacc[g].x;
+                        da_acc[g][v1] = dacc[g].y;
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int v = 0; v < V; ++v) {
+                    float x[S], cv[S];  // x = mu_{t+1}, the propagated adjoint after row t
+#pragma unroll
+                    for (int s = 0; s < S; ++s) cv[s] = sm.cin[s][cc + v];
+                    apply<S>(pre.e[v].A, pre.e[v].b, cv, x);
+#pragma unroll
+                    for (int r = R - 1; r >= 0; --r) {
+                        const bool rvalid = (tb + r < T) && cvalid;
+                        float lam[S], A[S * S];
+#pragma unroll
+                        for (int s = 0; s < S; ++s) lam[s] = gr[r][s][v] + x[s];
+#pragma unroll
+                        for (int a = 0; a < S * S; ++a) A[a] = jA[r][a][v];
+                        mat_t_vec<S>(A, lam, x);  // mu_t
+                        float se[NS], dp[G], da[G];
+#pragma unroll
+                        for (int n = 0; n < NS; ++n) se[n] = sens[r][n][v];
+                        Cell::grads(se, lam, dp, da);
+#pragma unroll
+                        for (int g2 = 0; g2 < G; ++g2) {
+                            outp[r][g2][v] = dp[g2];
+                            if (rvalid) {
+                                da_acc[g2][v] += da[g2];
+                                bad |= !isfinite(dp[g2]);
+                            }
+                        }
+                        if (r == 0 && tb == 0 && rvalid && prm.dLdh0) {
+                            // dL/dh0 = A_0^T lambda_0 = mu_0
+#pragma unroll
+                            for (int s = 0; s < S; ++s) prm.dLdh0[(b * S + s) * D + d0 + cc + v] = x[s];
+                        }
                     }
                 }
             }

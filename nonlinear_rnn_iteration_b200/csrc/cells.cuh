@@ -24,6 +24,7 @@ namespace pararnn {
 struct CellLinear {
     static constexpr int G = 2, S = 1, NSENS = 1;
     static constexpr bool kNonlinear = false;  // one scan is exact
+    struct W2 {};  // no packed form: the linear cell's arithmetic is one FMA per row
 
     static __device__ __forceinline__ void warm(const float (&p)[G], const float (&)[G], float (&f)[S]) {
         f[0] = p[1];
@@ -84,6 +85,80 @@ struct CellGRU {
         a = __fmaf_rn(gcw, tr, a);
         A[0] = a;
         beta[0] = __fmaf_rn(-a, h, f[0]);
+    }
+    // ---- two channels per instruction (packed f32x2) ----
+    // the recurrent weights of a channel pair, with the negated copy the
+    // sign-free algebra below needs
+    struct W2 {
+        f2 w0, w1, w2, nw2;
+    };
+    static __device__ __forceinline__ W2 weights2(const float (&wa)[G], const float (&wb)[G]) {
+        return W2{f2{wa[0], wb[0]}, f2{wa[1], wb[1]}, f2{wa[2], wb[2]}, f2{-wa[2], -wb[2]}};
+    }
+    // elem() on a pair of channels.  No packed negation exists, so the gates
+    // are formed negated, nz = -z and nr = -r (neg_sigmoid2), and every sign
+    // is carried by the algebra:
+    //   f      = z (c - h) + h            = nz (h - c) + h
+    //   a_c r  = (-a_c) nr
+    //   G_z a_z= a_z (c - h)(z - z^2)     = a_z (h - c)(nz^2 + nz)
+    //   1 - z  = 1 + nz
+    //   the shared reset/candidate term  G_c a_c (a_r h r (1 - r) + r)
+    //          = (nz (c^2 - 1) (-a_c)) * (a_r h (nr^2 + nr) + nr)
+    // Each product or sum is the same floating-point operation as in elem()
+    // up to the sign of its operands, so each result is elem()'s, negated
+    // where the algebra says so.
+    static __device__ __forceinline__ void elem2(const f2 (&p)[G], const W2& w, const f2 (&sp)[S], f2 (&f)[S],
+                                                 f2 (&A)[S * S], f2 (&beta)[S]) {
+        elem2(p, w, sp[0], f[0], A[0], beta[0]);
+    }
+    static __device__ __forceinline__ void elem2(const f2 (&p)[G], const W2& w, f2 h, f2& f, f2& A, f2& beta) {
+        const f2 nz = neg_sigmoid2(fma2(w.w0, h, p[0]));
+        const f2 nr = neg_sigmoid2(fma2(w.w1, h, p[1]));
+        const f2 wr = mul2(w.nw2, nr);
+        const f2 c = tanh2(fma2(wr, h, p[2]));
+        const f2 hc = sub2(h, c);
+        f = fma2(nz, hc, h);
+        const f2 ngcw = mul2(mul2(nz, fma2(c, c, splat2(-1.0f))), w.nw2);
+        const f2 ntr = fma2(mul2(w.w1, h), fma2(nr, nr, nr), nr);
+        f2 a = fma2(w.w0, mul2(hc, fma2(nz, nz, nz)), add2(splat2(1.0f), nz));
+        a = fma2(ngcw, ntr, a);
+        A = a;
+        beta = fma2(a, mul2(h, splat2(-1.0f)), f);
+    }
+    // bwd() on a pair of channels, with the negated gates of elem2():
+    //   G_z = (c - h)(z - z^2)      = (h - c)(nz^2 + nz)
+    //   G_c = z (1 - c^2)           = nz (c^2 - 1)
+    //   G_r = G_c a_c h (r - r^2)   = ((G_c (-a_c)) h)(nr^2 + nr)
+    //   r h = -(nr h)
+    static __device__ __forceinline__ void bwd2(const f2 (&p)[G], const W2& w, const f2 (&sp)[S], f2 (&A)[S * S],
+                                                f2 (&sens)[NSENS]) {
+        const f2 h = sp[0], mone = splat2(-1.0f);
+        const f2 nz = neg_sigmoid2(fma2(w.w0, h, p[0]));
+        const f2 nr = neg_sigmoid2(fma2(w.w1, h, p[1]));
+        const f2 wr = mul2(w.nw2, nr);
+        const f2 c = tanh2(fma2(wr, h, p[2]));
+        const f2 Gz = mul2(sub2(h, c), fma2(nz, nz, nz));
+        const f2 Gc = mul2(nz, fma2(c, c, mone));
+        const f2 Gr = mul2(mul2(mul2(Gc, w.nw2), h), fma2(nr, nr, nr));
+        f2 a = add2(splat2(1.0f), nz);
+        a = fma2(w.w0, Gz, a);
+        a = fma2(w.w1, Gr, a);
+        a = fma2(wr, Gc, a);
+        A[0] = a;
+        sens[0] = Gz;
+        sens[1] = Gr;
+        sens[2] = Gc;
+        sens[3] = mul2(mul2(nr, h), mone);
+        sens[4] = h;
+    }
+    static __device__ __forceinline__ void grads2(const f2 (&sens)[NSENS], const f2 (&lam)[S], f2 (&dp)[G],
+                                                  f2 (&da)[G]) {
+        dp[0] = mul2(lam[0], sens[0]);
+        dp[1] = mul2(lam[0], sens[1]);
+        dp[2] = mul2(lam[0], sens[2]);
+        da[0] = mul2(dp[0], sens[4]);
+        da[1] = mul2(dp[1], sens[4]);
+        da[2] = mul2(dp[2], sens[3]);
     }
     static __device__ __forceinline__ void bwd(const float (&p)[G], const float (&w)[G], const float (&sp)[S],
                                                float (&A)[S * S], float (&sens)[NSENS]) {
@@ -160,6 +235,78 @@ struct CellLSTM {
         beta[0] = __fmaf_rn(-A[1], h, q.ig);
         beta[1] = f[1] - __fmaf_rn(A[2], c, A[3] * h);
     }
+    // ---- two channels per instruction (packed f32x2) ----
+    struct W2 {
+        f2 w0, w1, w2, w3, nw3;
+    };
+    static __device__ __forceinline__ W2 weights2(const float (&wa)[G], const float (&wb)[G]) {
+        return W2{f2{wa[0], wb[0]}, f2{wa[1], wb[1]}, f2{wa[2], wb[2]}, f2{wa[3], wb[3]}, f2{-wa[3], -wb[3]}};
+    }
+    // elem() on a pair of channels; sp = (c, h), A row-major (2 x 2)
+    static __device__ __forceinline__ void elem2(const f2 (&p)[G], const W2& w, const f2 (&sp)[S], f2 (&f)[S],
+                                                 f2 (&A)[S * S], f2 (&beta)[S]) {
+        const f2 one = splat2(1.0f), mone = splat2(-1.0f);
+        const f2 c = sp[0], h = sp[1];
+        const f2 i = sigmoid2(fma2(w.w0, h, p[0]));
+        const f2 fg = sigmoid2(add2(fma2(w.w1, h, p[1]), one));
+        const f2 o = sigmoid2(fma2(w.w2, h, p[2]));
+        const f2 g = tanh2(fma2(w.w3, h, p[3]));
+        const f2 ig = mul2(i, g);
+        const f2 cn = fma2(fg, c, ig);
+        const f2 tn = tanh2(cn);
+        // dc'/dh through the f, i and c gates' pre-activations
+        f2 d = mul2(mul2(c, fma2(fg, mul2(fg, mone), fg)), w.w1);
+        d = fma2(mul2(g, fma2(i, mul2(i, mone), i)), w.w0, d);
+        d = fma2(mul2(i, fma2(g, g, mone)), w.nw3, d);  // i (1 - g^2) a_c, both signs flipped
+        const f2 k = mul2(mul2(o, fma2(tn, tn, mone)), mone);  // dh'/dc' = o (1 - tn^2)
+        f[0] = cn;
+        f[1] = mul2(o, tn);
+        A[0] = fg;
+        A[1] = d;
+        A[2] = mul2(k, fg);
+        A[3] = fma2(mul2(fma2(o, mul2(o, mone), o), w.w2), tn, mul2(k, d));
+        beta[0] = fma2(d, mul2(h, mone), ig);
+        beta[1] = sub2(f[1], fma2(A[2], c, mul2(A[3], h)));
+    }
+    // bwd() on a pair of channels
+    static __device__ __forceinline__ void bwd2(const f2 (&p)[G], const W2& w, const f2 (&sp)[S], f2 (&A)[S * S],
+                                                f2 (&sens)[NSENS]) {
+        const f2 one = splat2(1.0f), mone = splat2(-1.0f);
+        const f2 c = sp[0], h = sp[1];
+        const f2 i = sigmoid2(fma2(w.w0, h, p[0]));
+        const f2 fg = sigmoid2(add2(fma2(w.w1, h, p[1]), one));
+        const f2 o = sigmoid2(fma2(w.w2, h, p[2]));
+        const f2 g = tanh2(fma2(w.w3, h, p[3]));
+        const f2 tn = tanh2(fma2(fg, c, mul2(i, g)));
+        const f2 si = mul2(g, fma2(i, mul2(i, mone), i));     // dc'/dp_i = g i (1 - i)
+        const f2 sf = mul2(c, fma2(fg, mul2(fg, mone), fg));  // dc'/dp_f = c f (1 - f)
+        const f2 nsc = mul2(i, fma2(g, g, mone));             // -(dc'/dp_c) = -i (1 - g^2)
+        f2 d = mul2(sf, w.w1);
+        d = fma2(si, w.w0, d);
+        d = fma2(nsc, w.nw3, d);
+        const f2 k = mul2(mul2(o, fma2(tn, tn, mone)), mone);  // dh'/dc' = o (1 - tn^2)
+        const f2 dho = mul2(fma2(o, mul2(o, mone), o), tn);    // dh'/dp_o = o (1 - o) tn
+        A[0] = fg;
+        A[1] = d;
+        A[2] = mul2(k, fg);
+        A[3] = fma2(dho, w.w2, mul2(k, d));
+        sens[0] = si;
+        sens[1] = sf;
+        sens[2] = mul2(nsc, mone);
+        sens[3] = k;
+        sens[4] = dho;
+        sens[5] = h;
+    }
+    static __device__ __forceinline__ void grads2(const f2 (&sens)[NSENS], const f2 (&lam)[S], f2 (&dp)[G],
+                                                  f2 (&da)[G]) {
+        const f2 m = fma2(lam[1], sens[3], lam[0]);
+        dp[0] = mul2(m, sens[0]);
+        dp[1] = mul2(m, sens[1]);
+        dp[2] = mul2(lam[1], sens[4]);
+        dp[3] = mul2(m, sens[2]);
+#pragma unroll
+        for (int g = 0; g < G; ++g) da[g] = mul2(dp[g], sens[5]);
+    }
     static __device__ __forceinline__ void bwd(const float (&p)[G], const float (&w)[G], const float (&sp)[S],
                                                float (&A)[S * S], float (&sens)[NSENS]) {
         const float c = sp[0], h = sp[1];
@@ -208,6 +355,43 @@ __device__ __forceinline__ void elem_identity(Elem<S>& e) {
     for (int i = 0; i < S * S; ++i) e.A[i] = (i % (S + 1) == 0) ? 1.0f : 0.0f;
 #pragma unroll
     for (int i = 0; i < S; ++i) e.b[i] = 0.0f;
+}
+
+// ---- the same algebra on a pair of channels (packed f32x2) -----------------
+// Each operation rounds like its scalar counterpart above, so a pair gives
+// the bits two scalar calls would.
+
+// y = A x + b
+template <int S>
+__device__ __forceinline__ void apply2(const f2 (&A)[S * S], const f2 (&b)[S], const f2 (&x)[S], f2 (&y)[S]) {
+    if constexpr (S == 1) {
+        y[0] = fma2(A[0], x[0], b[0]);
+    } else {
+        y[0] = fma2(A[0], x[0], fma2(A[1], x[1], b[0]));
+        y[1] = fma2(A[2], x[0], fma2(A[3], x[1], b[1]));
+    }
+}
+
+// (accA, accb) <- (A, b) o (accA, accb), on pairs
+template <int S>
+__device__ __forceinline__ void compose_after2(const f2 (&A)[S * S], const f2 (&b)[S], f2 (&accA)[S * S],
+                                               f2 (&accb)[S]) {
+    if constexpr (S == 1) {
+        accb[0] = fma2(A[0], accb[0], b[0]);
+        accA[0] = mul2(A[0], accA[0]);
+    } else {
+        f2 nb[2];
+        apply2<2>(A, b, accb, nb);
+        f2 nA[4];
+        nA[0] = fma2(A[0], accA[0], mul2(A[1], accA[2]));
+        nA[1] = fma2(A[0], accA[1], mul2(A[1], accA[3]));
+        nA[2] = fma2(A[2], accA[0], mul2(A[3], accA[2]));
+        nA[3] = fma2(A[2], accA[1], mul2(A[3], accA[3]));
+#pragma unroll
+        for (int i = 0; i < 4; ++i) accA[i] = nA[i];
+        accb[0] = nb[0];
+        accb[1] = nb[1];
+    }
 }
 
 // y = A x + b

@@ -158,6 +158,75 @@ __device__ __forceinline__ float tanh_f(float x) {
     return fabsf(x) < 0.0625f ? poly : big;
 }
 
+// ---- packed pairs: two channels per instruction ----------------------------
+// sm_100a's fma / add / sub / mul .rn.f32x2 operate on two floats held in a
+// register pair and round each half exactly like the scalar instruction, so a
+// computation written on pairs gives the same bits as the same computation on
+// each channel alone.  There is no packed negation or min/max: signs are
+// folded into constants instead.
+struct f2 {
+    float x, y;
+};
+
+__device__ __forceinline__ f2 splat2(float a) { return f2{a, a}; }
+
+__device__ __forceinline__ f2 fma2(f2 a, f2 b, f2 c) {
+    f2 d;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+__device__ __forceinline__ f2 mul2(f2 a, f2 b) {
+    f2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+__device__ __forceinline__ f2 add2(f2 a, f2 b) {
+    f2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+__device__ __forceinline__ f2 sub2(f2 a, f2 b) {
+    f2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "sub.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+__device__ __forceinline__ f2 ex2_2(f2 a) { return f2{exp2_approx(a.x), exp2_approx(a.y)}; }
+__device__ __forceinline__ f2 rcp_2(f2 a) { return f2{rcp_approx(a.x), rcp_approx(a.y)}; }
+
+// -sigma(x) = 1 / (-1 - e^{-x}): the same rounding as sigmoid_f, negated
+// (a reciprocal of a negated value is the exact negation), which saves the
+// packed negation the callers would otherwise need
+__device__ __forceinline__ f2 neg_sigmoid2(f2 x) {
+    return rcp_2(sub2(splat2(-1.0f), ex2_2(mul2(x, splat2(-kLog2e)))));
+}
+__device__ __forceinline__ f2 sigmoid2(f2 x) {
+    return rcp_2(add2(ex2_2(mul2(x, splat2(-kLog2e))), splat2(1.0f)));
+}
+// tanh_f on a pair, the same operations in the same order
+__device__ __forceinline__ f2 tanh2(f2 x) {
+    const f2 big = fma2(splat2(-2.0f), rcp_2(add2(ex2_2(mul2(x, splat2(2.0f * kLog2e))), splat2(1.0f))),
+                        splat2(1.0f));
+    const f2 x2 = mul2(x, x);
+    const f2 poly = mul2(x, fma2(x2, fma2(x2, splat2(2.0f / 15.0f), splat2(-1.0f / 3.0f)), splat2(1.0f)));
+    return f2{fabsf(x.x) < 0.0625f ? poly.x : big.x, fabsf(x.y) < 0.0625f ? poly.y : big.y};
+}
+
 // max that keeps a NaN (so a non-finite residual is reported, not hidden)
 __device__ __forceinline__ float nanmax_f(float a, float b) { return (a != a || a > b) ? a : b; }
 

@@ -61,9 +61,19 @@ bool layout(pararnn_cell cell, int64_t B, int64_t T, int64_t D, int K, int64_t r
     return true;
 }
 
-// fold one slot's device status into the call's header
+// fold one slot's device status into the call's header.  A forward on the
+// small-problem path leaves its flags in the tagged word (header bytes 8..15,
+// valid when their tag equals the call number at bytes 16..19); every other
+// forward clears those bytes and uses word 0.
 __global__ void fold_status(unsigned* dst, const unsigned* src) {
-    if (threadIdx.x == 0 && *src) atomicOr(dst, *src);
+    if (threadIdx.x != 0) return;
+    unsigned f = src[0];
+    const unsigned ep = src[4];
+    if (ep) {
+        const unsigned long long tw = *reinterpret_cast<const unsigned long long*>(src + 2);
+        f = (static_cast<unsigned>(tw >> 32) == ep) ? static_cast<unsigned>(tw) : 0u;
+    }
+    if (f) atomicOr(dst, f);
 }
 
 pararnn_status fail(pararnn_status st, const char* msg) {

@@ -14,8 +14,8 @@
 //   inclusive  per channel, the state after the tile's last row      S words
 // A word is valid when its tag equals this call's epoch, so a value and its
 // "ready" flag travel in one single-copy-atomic store: no fence is needed.
-// Words left by earlier calls carry other tags and read as not ready; a
-// zero-filled workspace never matches (epochs start at 1).  The status word
+// The host clears every look-back word on the stream before the kernel runs,
+// and a cleared word never matches (epochs start at 1).  The status word
 // lets one warp read 32 predecessors' states in one round trip; payload
 // words are checked again when they are read, so a status seen before its
 // payload costs a retry, never a wrong value.
@@ -43,6 +43,7 @@ struct LookbackCtx {
     int nSlots;
     uint32_t epoch;
     uint64_t timeout_ns;
+    int stall_first;   // test hook: the tile with ticket 0 never publishes its state
 };
 
 __device__ __forceinline__ void st_word(word_t* p, float v, uint32_t epoch) {
@@ -425,6 +426,9 @@ __device__ __forceinline__ void tile_lookback(const LookbackCtx& cx, int64_t til
 template <int S, int W>
 __device__ __forceinline__ void publish_inclusive(const LookbackCtx& cx, int64_t tile, int slot, int lane,
                                                   const Inclusive<S, W>& out) {
+    // the stall hook: the first tile of the scan withholds its state, so its
+    // successor's bounded look-back runs out (the time-out path under test)
+    if (cx.stall_first && tile == 0) return;
     publish_words<S, W>(cx.inc + (tile * cx.nSlots + slot) * S * W, out.v, cx.epoch, lane);
     __syncwarp();
     if (lane == 0) st_status(cx.tstat + tile * cx.nSlots + slot, kTileInclusive, cx.epoch);

@@ -36,6 +36,7 @@
 #pragma once
 
 #include "cells.cuh"
+#include "cluster.cuh"
 #include "common.cuh"
 #include "lookback.cuh"
 #include "tma.cuh"
@@ -51,11 +52,21 @@ struct FwdParams {
     unsigned* ticket;    // workspace header word 1
     int64_t B, T, D;
     int K;
+    int picard;          // Picard sweeps before the Newton iterations (0..kPicardMax)
     int64_t nCG;         // channel groups per batch row
     int64_t nChunks;     // tiles along T
     int64_t nTiles;
     LookbackCtx lb;      // nGroups = B * nCG, nSlots = K
+    // the small-problem (cluster) path: status flags tagged with the call
+    // number, and the word that names the call the flags belong to
+    unsigned long long* tagged_status;  // workspace header bytes 8..15
+    unsigned* status_epoch;             // workspace header bytes 16..19
 };
+
+// Picard sweeps a forward call may ask for: each sweep reaches one row
+// further back, so a thread evaluates up to kPicardMax + 1 rows before its
+// own sub-chunk.
+constexpr int kPicardMax = 4;
 
 // V channels per thread, LC lanes across channels, NW compute warps, R rows
 // per thread, MINB blocks per SM the register budget is sized for, NSTAGE
@@ -96,9 +107,65 @@ struct FwdSmem {
     float wagg[Sh::NWARPS][Sh::NA][Sh::W];  // each compute warp's composed element
     float cin[Sh::S][Sh::W];                // the state just before the tile (current iterate)
     float w[Sh::G][Sh::W];                  // the tile's recurrent weights
+    float cagg[2][Sh::NA][Sh::W];           // cluster path: this tile's element, iterations in turn
     uint64_t bar[Sh::NSTAGE];
     unsigned ticket[Sh::NSTAGE];
 };
+
+// The cluster path's carry for one Newton iteration (scan warp, between the
+// "warp totals" and "carry" block barriers; the compute warps take the same
+// cluster barrier meanwhile).  The tiles of one channel group along T are the
+// CTAs of one cluster, rank = position along T.  Each composes its warp
+// totals into its tile's element, and after the cluster barrier reads the
+// elements of the tiles before it from their shared memory and applies them,
+// in order, to the first carry: the same sequence of operations as the
+// look-back's inclusive states, so the carry has the same bits.
+template <class Sh>
+__device__ __forceinline__ void cluster_carry(const float (&wagg)[Sh::NWARPS][Sh::NA][Sh::W],
+                                              float (&cagg)[Sh::NA][Sh::W],
+                                              const float (&first_carry)[Sh::W / 32][Sh::S], uint32_t rank,
+                                              int lane, float (&cin)[Sh::S][Sh::W]) {
+    constexpr int S = Sh::S, NA = Sh::NA, W = Sh::W, CPL = W / 32;
+#pragma unroll
+    for (int j = 0; j < CPL; ++j) {
+        Elem<S> tot;
+        elem_identity<S>(tot);
+#pragma unroll
+        for (int k = 0; k < Sh::NWARPS; ++k) {
+            float A[S * S], b[S];
+#pragma unroll
+            for (int a = 0; a < S * S; ++a) A[a] = wagg[k][a][lane + 32 * j];
+#pragma unroll
+            for (int s = 0; s < S; ++s) b[s] = wagg[k][S * S + s][lane + 32 * j];
+            compose_after<S>(A, b, tot);
+        }
+#pragma unroll
+        for (int a = 0; a < S * S; ++a) cagg[a][lane + 32 * j] = tot.A[a];
+#pragma unroll
+        for (int s = 0; s < S; ++s) cagg[S * S + s][lane + 32 * j] = tot.b[s];
+    }
+    __syncwarp();
+    cluster_arrive_release();
+    cluster_wait_acquire();
+#pragma unroll
+    for (int j = 0; j < CPL; ++j) {
+        float x[S];
+#pragma unroll
+        for (int s = 0; s < S; ++s) x[s] = first_carry[j][s];
+        for (uint32_t i = 0; i < rank; ++i) {
+            float A[S * S], b[S], y[S];
+#pragma unroll
+            for (int a = 0; a < S * S; ++a) A[a] = ld_dsmem(&cagg[a][lane + 32 * j], i);
+#pragma unroll
+            for (int s = 0; s < S; ++s) b[s] = ld_dsmem(&cagg[S * S + s][lane + 32 * j], i);
+            apply<S>(A, b, x, y);
+#pragma unroll
+            for (int s = 0; s < S; ++s) x[s] = y[s];
+        }
+#pragma unroll
+        for (int s = 0; s < S; ++s) cin[s][lane + 32 * j] = x[s];
+    }
+}
 
 template <class Cell, typename PxT, class Sh>
 __device__ __forceinline__ void issue_tile_load(const CUtensorMap* map, FwdSmem<Sh, PxT>& sm, const FwdParams& prm,
@@ -113,7 +180,12 @@ __device__ __forceinline__ void issue_tile_load(const CUtensorMap* map, FwdSmem<
                 (int)(b * prm.T + chunk * Sh::L) - Sh::ROW0);
 }
 
-template <class Cell, typename PxT, class Sh, bool kLean>
+// kCluster: the small-problem path.  Every tile is its own CTA, launched in
+// clusters of nChunks CTAs (one channel group of one batch row, all along T);
+// the carries pass through distributed shared memory (cluster_carry), so
+// there is no ticket counter, no look-back and nothing in the workspace but
+// the tagged status word.
+template <class Cell, typename PxT, class Sh, bool kLean, bool kPicard = false, bool kCluster = false>
 __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
     newton_fwd_kernel(const __grid_constant__ CUtensorMap tmap, const FwdParams prm) {
     constexpr int G = Sh::G, S = Sh::S, V = Sh::V, R = Sh::R, NW = Sh::NWARPS, NSTAGE = Sh::NSTAGE;
@@ -128,6 +200,12 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
     const int64_t T = prm.T, D = prm.D;
     const PxT* pxg = static_cast<const PxT*>(prm.px);
     const bool need_prev = Cell::kNonlinear || prm.resid != nullptr;
+    auto report = [&](unsigned bit) {
+        if constexpr (kCluster)
+            set_tagged_status(prm.tagged_status, prm.lb.epoch, bit);
+        else
+            atomicOr(prm.lb.status, bit);
+    };
 
     // prologue (scan warp): claim the first NSTAGE-1 tiles and start streaming them in
     if (is_scan && lane == 0) {
@@ -136,12 +214,23 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
             for (int s = 0; s < NSTAGE; ++s) mbar_init(&sm.bar[s], 1);
             mbar_fence_init();
         }
+        if constexpr (kCluster) {
+            // one tile per CTA: blockIdx.x = group * nChunks + position along T
+            const int64_t gid = blockIdx.x / prm.nChunks;
+            const unsigned t = (unsigned)((int64_t)cluster_ctarank() * prm.lb.nGroups + gid);
+            sm.ticket[0] = t;
 #pragma unroll
-        for (int s = 0; s < NSTAGE - 1; ++s) {
-            const unsigned t = atomicAdd(prm.ticket, 1u);
-            sm.ticket[s] = t;
-            if constexpr (Sh::kTma)
-                if (t < prm.nTiles) issue_tile_load<Cell, PxT, Sh>(&tmap, sm, prm, t, s);
+            for (int s = 1; s < NSTAGE; ++s) sm.ticket[s] = (unsigned)prm.nTiles;
+            if constexpr (Sh::kTma) issue_tile_load<Cell, PxT, Sh>(&tmap, sm, prm, t, 0);
+            if (blockIdx.x == 0) *prm.status_epoch = prm.lb.epoch;  // the flags of this call are the valid ones
+        } else {
+#pragma unroll
+            for (int s = 0; s < NSTAGE - 1; ++s) {
+                const unsigned t = atomicAdd(prm.ticket, 1u);
+                sm.ticket[s] = t;
+                if constexpr (Sh::kTma)
+                    if (t < prm.nTiles) issue_tile_load<Cell, PxT, Sh>(&tmap, sm, prm, t, s);
+            }
         }
     }
     block_sync();
@@ -173,9 +262,11 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
             // it saves
             Probe<S, W> pr;
             pr.st = 0;
-            if constexpr (!kLean) probe_issue<S, W>(prm.lb, tile, chunk, 0, lane, pr);
+            if constexpr (!kLean && !kCluster) probe_issue<S, W>(prm.lb, tile, chunk, 0, lane, pr);
             block_sync();  // tile set up
-            if (lane == 0) {
+            if constexpr (kCluster) {
+                if (lane == 0) sm.ticket[(it + NSTAGE - 1) % NSTAGE] = (unsigned)prm.nTiles;  // no further tile
+            } else if (lane == 0) {
                 // claim the tile NSTAGE-1 ahead and start streaming it in; its
                 // stage was last read by the previous tile, whose readers have
                 // all passed this tile's set-up barrier
@@ -188,7 +279,14 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
                     if (t2 < prm.nTiles && prev_t < prm.nTiles) issue_tile_load<Cell, PxT, Sh>(&tmap, sm, prm, t2, sn);
             }
             Inclusive<S, W> inc;
-            if constexpr (kLean) {
+            if constexpr (kCluster) {
+                const int K = kLean ? 1 : prm.K;
+                for (int k = 0; k < K; ++k) {
+                    block_sync();  // warp totals ready
+                    cluster_carry<Sh>(sm.wagg, sm.cagg[k & 1], first_carry, (uint32_t)chunk, lane, sm.cin);
+                    block_sync();  // carry ready
+                }
+            } else if constexpr (kLean) {
                 block_sync();  // warp totals ready
                 tile_lookback<S, W, NW, false>(prm.lb, tile, chunk, 0, lane, sm.wagg, first_carry, pr, sm.cin, inc);
                 block_sync();  // carry ready
@@ -219,7 +317,7 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
                 Deadline dl;
                 while (!mbar_try_wait(&sm.bar[st], (it / NSTAGE) & 1)) {
                     if (dl.expired(prm.lb.timeout_ns)) {
-                        if (tid == 0) atomicOr(prm.lb.status, kStatusTimeout);
+                        if (tid == 0) report(kStatusTimeout);
                         break;
                     }
                 }
@@ -256,7 +354,9 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
                 }
                 warp_prefix<S, V, LC, W, NW, false>(mine, excl, warp, lane, sm.wagg);
                 block_sync();  // warp totals ready
+                if constexpr (kCluster) cluster_arrive_release();
                 sub_prefix<S, V, LC, W, NW, false>(excl, warp, lane, sm.wagg, pre);
+                if constexpr (kCluster) cluster_wait_acquire();
                 block_sync();  // carry ready
                 float x[V];
 #pragma unroll
@@ -278,7 +378,7 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
                         store_row<V>(prm.H + (b * T + t) * D + d0 + cc, out);
                     }
                 }
-                if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(prm.lb.status, kStatusNonFinite);
+                if (__any_sync(0xffffffffu, bad) && lane == 0) report(kStatusNonFinite);
             } else {
                 // ---- general path: warm start, K Newton iterations ----
                 const bool want_resid = prm.resid != nullptr;
@@ -288,18 +388,20 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
 #pragma unroll
                     for (int g = 0; g < G; ++g) wr[v][g] = sm.w[g][cc + v];
                 float h[R][S][V];
+                if constexpr (!kPicard) {
 #pragma unroll
-                for (int r = 0; r < R; ++r) {
-                    float pv[G][V];
-                    load_p(r, pv);
+                    for (int r = 0; r < R; ++r) {
+                        float pv[G][V];
+                        load_p(r, pv);
 #pragma unroll
-                    for (int v = 0; v < V; ++v) {
-                        float pg[G], f[S];
+                        for (int v = 0; v < V; ++v) {
+                            float pg[G], f[S];
 #pragma unroll
-                        for (int g = 0; g < G; ++g) pg[g] = pv[g][v];
-                        Cell::warm(pg, wr[v], f);
+                            for (int g = 0; g < G; ++g) pg[g] = pv[g][v];
+                            Cell::warm(pg, wr[v], f);
 #pragma unroll
-                        for (int s = 0; s < S; ++s) h[r][s][v] = f[s];
+                            for (int s = 0; s < S; ++s) h[r][s][v] = f[s];
+                        }
                     }
                 }
                 // h^(0) just before the sub-chunk: h0 at the start of a row,
@@ -310,7 +412,90 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
                 for (int s = 0; s < S; ++s)
 #pragma unroll
                     for (int v = 0; v < V; ++v) hin[s][v] = 0.0f;
-                if (need_prev && cvalid) {
+                if constexpr (kPicard) {
+                    // Picard sweeps h^(p+1)_t = f(h^(p)_{t-1}, x_t) from the
+                    // warm start, on this thread's rows and the P + 1 rows
+                    // before them (row j of the window is time tb + j); sweep p
+                    // is valid from row -(P+1) + p on, so after P sweeps rows
+                    // -1 .. R-1 hold h^(P).  Every thread forms the rows it
+                    // shares with its neighbours by the same arithmetic from
+                    // the same inputs, so the copies agree bit for bit.
+                    constexpr int NWIN = R + kPicardMax + 1;  // window rows j = -(kPicardMax+1) .. R-1
+                    constexpr int J0 = kPicardMax + 1;        // window index of row j is j + J0
+                    const int P = prm.picard;
+                    float win[NWIN][S][V];
+                    float h0v[S][V];
+#pragma unroll
+                    for (int s = 0; s < S; ++s)
+#pragma unroll
+                        for (int v = 0; v < V; ++v)
+                            h0v[s][v] = (prm.h0 && cvalid) ? prm.h0[(b * S + s) * D + d0 + cc + v] : 0.0f;
+                    // pre-activations of window row j: the stage holds rows from
+                    // t0 - ROW0 on; rows before it come from global memory
+                    auto load_pw = [&](int j, float (&pv)[G][V]) {
+                        const int srow = Sh::ROW0 + sub * R + j;
+                        const int64_t t = tb + j;
+                        if (srow >= 0) {
+#pragma unroll
+                            for (int g = 0; g < G; ++g) lds_row<V>(&sm.px[st].v[srow][g][cc], pv[g]);
+                        } else {
+#pragma unroll
+                            for (int g = 0; g < G; ++g)
+#pragma unroll
+                                for (int v = 0; v < V; ++v)
+                                    pv[g][v] = (t >= 0 && cvalid)
+                                                   ? PxTraits<PxT>::cvt(pxg[((b * T + t) * G + g) * D + d0 + cc + v])
+                                                   : 0.0f;
+                        }
+                    };
+#pragma unroll
+                    for (int jj = 0; jj < NWIN; ++jj) {
+                        const int j = jj - J0;
+                        if (j < -(P + 1)) continue;
+                        float pv[G][V];
+                        load_pw(j, pv);
+#pragma unroll
+                        for (int v = 0; v < V; ++v) {
+                            float pg[G], f[S];
+#pragma unroll
+                            for (int g = 0; g < G; ++g) pg[g] = pv[g][v];
+                            Cell::warm(pg, wr[v], f);
+#pragma unroll
+                            for (int s = 0; s < S; ++s) win[jj][s][v] = (tb + j >= 0) ? f[s] : h0v[s][v];
+                        }
+                    }
+                    for (int p = 1; p <= P; ++p) {
+                        // rows from the last back, so row j-1 still holds sweep p-1
+#pragma unroll
+                        for (int jj = NWIN - 1; jj >= 1; --jj) {
+                            const int j = jj - J0;
+                            if (j < -(P + 1) + p || tb + j < 0) continue;
+                            float pv[G][V];
+                            load_pw(j, pv);
+#pragma unroll
+                            for (int v = 0; v < V; ++v) {
+                                float pg[G], spv[S], f[S], A[S * S], be[S];
+#pragma unroll
+                                for (int g = 0; g < G; ++g) pg[g] = pv[g][v];
+#pragma unroll
+                                for (int s = 0; s < S; ++s) spv[s] = (tb + j - 1 >= 0) ? win[jj - 1][s][v] : h0v[s][v];
+                                Cell::elem(pg, wr[v], spv, f, A, be);
+#pragma unroll
+                                for (int s = 0; s < S; ++s) win[jj][s][v] = f[s];
+                            }
+                        }
+                    }
+#pragma unroll
+                    for (int r = 0; r < R; ++r)
+#pragma unroll
+                        for (int s = 0; s < S; ++s)
+#pragma unroll
+                            for (int v = 0; v < V; ++v) h[r][s][v] = win[J0 + r][s][v];
+#pragma unroll
+                    for (int s = 0; s < S; ++s)
+#pragma unroll
+                        for (int v = 0; v < V; ++v) hin[s][v] = cvalid ? win[J0 - 1][s][v] : 0.0f;
+                } else if (need_prev && cvalid) {
                     if (tb == 0) {
                         if (prm.h0)
 #pragma unroll
@@ -341,6 +526,15 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
                     }
                 }
                 const int K = prm.K;
+                // two channels per instruction where the thread holds an even
+                // number of them (packed f32x2; same rounding as one by one)
+                constexpr bool kPack = (V % 2 == 0) && Cell::kNonlinear;
+                constexpr int VP = kPack ? V / 2 : 1;
+                typename Cell::W2 wp[VP];
+                if constexpr (kPack) {
+#pragma unroll
+                    for (int q = 0; q < VP; ++q) wp[q] = Cell::weights2(wr[2 * q], wr[2 * q + 1]);
+                }
                 for (int k = 0; k <= K; ++k) {
                     // ---- 1. elements of iteration k+1 and the residual of iterate k ----
                     float sp[S][V];
@@ -355,31 +549,63 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
                         const bool rvalid = (tb + r < T) && cvalid;
                         float pv[G][V];
                         load_p(r, pv);
+                        // rows past the end of the sequence (and channels
+                        // past D) keep their elements: in time order they
+                        // come after every valid row of their channel, so
+                        // they reach only scan values nobody reads (the
+                        // sequence's last inclusive state and h rows that
+                        // are never stored); their pre-activations are
+                        // zero-filled, so the values stay finite
+                        if constexpr (kPack) {
 #pragma unroll
-                        for (int v = 0; v < V; ++v) {
-                            float pg[G], spv[S], f[S], A[S * S], be[S];
+                            for (int q = 0; q < VP; ++q) {
+                                const int v0 = 2 * q, v1 = 2 * q + 1;
+                                f2 pg[G], spv[S], f[S], A[S * S], be[S];
 #pragma unroll
-                            for (int g = 0; g < G; ++g) pg[g] = pv[g][v];
+                                for (int g = 0; g < G; ++g) pg[g] = f2{pv[g][v0], pv[g][v1]};
 #pragma unroll
-                            for (int s = 0; s < S; ++s) spv[s] = sp[s][v];
-                            Cell::elem(pg, wr[v], spv, f, A, be);
-                            // rows past the end of the sequence (and channels
-                            // past D) keep their elements: in time order they
-                            // come after every valid row of their channel, so
-                            // they reach only scan values nobody reads (the
-                            // sequence's last inclusive state and h rows that
-                            // are never stored); their pre-activations are
-                            // zero-filled, so the values stay finite
-                            if (rvalid && want_resid) {
+                                for (int s = 0; s < S; ++s) spv[s] = f2{sp[s][v0], sp[s][v1]};
+                                Cell::elem2(pg, wp[q], spv, f, A, be);
+                                if (rvalid && want_resid) {
 #pragma unroll
-                                for (int s = 0; s < S; ++s) res = nanmax_f(res, fabsf(h[r][s][v] - f[s]));
+                                    for (int s = 0; s < S; ++s) {
+                                        res = nanmax_f(res, fabsf(h[r][s][v0] - f[s].x));
+                                        res = nanmax_f(res, fabsf(h[r][s][v1] - f[s].y));
+                                    }
+                                }
+#pragma unroll
+                                for (int a = 0; a < S * S; ++a) {
+                                    eA[r][a][v0] = A[a].x;
+                                    eA[r][a][v1] = A[a].y;
+                                }
+#pragma unroll
+                                for (int s = 0; s < S; ++s) {
+                                    eb[r][s][v0] = be[s].x;
+                                    eb[r][s][v1] = be[s].y;
+                                    sp[s][v0] = h[r][s][v0];
+                                    sp[s][v1] = h[r][s][v1];
+                                }
                             }
+                        } else {
 #pragma unroll
-                            for (int a = 0; a < S * S; ++a) eA[r][a][v] = A[a];
+                            for (int v = 0; v < V; ++v) {
+                                float pg[G], spv[S], f[S], A[S * S], be[S];
 #pragma unroll
-                            for (int s = 0; s < S; ++s) {
-                                eb[r][s][v] = be[s];
-                                sp[s][v] = h[r][s][v];
+                                for (int g = 0; g < G; ++g) pg[g] = pv[g][v];
+#pragma unroll
+                                for (int s = 0; s < S; ++s) spv[s] = sp[s][v];
+                                Cell::elem(pg, wr[v], spv, f, A, be);
+                                if (rvalid && want_resid) {
+#pragma unroll
+                                    for (int s = 0; s < S; ++s) res = nanmax_f(res, fabsf(h[r][s][v] - f[s]));
+                                }
+#pragma unroll
+                                for (int a = 0; a < S * S; ++a) eA[r][a][v] = A[a];
+#pragma unroll
+                                for (int s = 0; s < S; ++s) {
+                                    eb[r][s][v] = be[s];
+                                    sp[s][v] = h[r][s][v];
+                                }
                             }
                         }
                     }
@@ -390,45 +616,113 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
                     }
                     if (k == K) break;  // the last pass only measured the residual of h^(K)
                     ElemV<S, V> mine, excl, pre;
+                    if constexpr (kPack) {
 #pragma unroll
-                    for (int v = 0; v < V; ++v) {
-                        elem_identity<S>(mine.e[v]);
+                        for (int q = 0; q < VP; ++q) {
+                            const int v0 = 2 * q, v1 = 2 * q + 1;
+                            f2 accA[S * S], accb[S];
 #pragma unroll
-                        for (int r = 0; r < R; ++r) {
-                            float A[S * S], be[S];
+                            for (int a = 0; a < S * S; ++a) accA[a] = splat2((a % (S + 1) == 0) ? 1.0f : 0.0f);
 #pragma unroll
-                            for (int a = 0; a < S * S; ++a) A[a] = eA[r][a][v];
+                            for (int s = 0; s < S; ++s) accb[s] = splat2(0.0f);
 #pragma unroll
-                            for (int s = 0; s < S; ++s) be[s] = eb[r][s][v];
-                            compose_after<S>(A, be, mine.e[v]);
+                            for (int r = 0; r < R; ++r) {
+                                f2 A[S * S], be[S];
+#pragma unroll
+                                for (int a = 0; a < S * S; ++a) A[a] = f2{eA[r][a][v0], eA[r][a][v1]};
+#pragma unroll
+                                for (int s = 0; s < S; ++s) be[s] = f2{eb[r][s][v0], eb[r][s][v1]};
+                                compose_after2<S>(A, be, accA, accb);
+                            }
+#pragma unroll
+                            for (int a = 0; a < S * S; ++a) {
+                                mine.e[v0].A[a] = accA[a].x;
+                                mine.e[v1].A[a] = accA[a].y;
+                            }
+#pragma unroll
+                            for (int s = 0; s < S; ++s) {
+                                mine.e[v0].b[s] = accb[s].x;
+                                mine.e[v1].b[s] = accb[s].y;
+                            }
+                        }
+                    } else {
+#pragma unroll
+                        for (int v = 0; v < V; ++v) {
+                            elem_identity<S>(mine.e[v]);
+#pragma unroll
+                            for (int r = 0; r < R; ++r) {
+                                float A[S * S], be[S];
+#pragma unroll
+                                for (int a = 0; a < S * S; ++a) A[a] = eA[r][a][v];
+#pragma unroll
+                                for (int s = 0; s < S; ++s) be[s] = eb[r][s][v];
+                                compose_after<S>(A, be, mine.e[v]);
+                            }
                         }
                     }
                     warp_prefix<S, V, LC, W, NW, false>(mine, excl, warp, lane, sm.wagg);
                     block_sync();  // warp totals ready
+                    if constexpr (kCluster) cluster_arrive_release();
                     // ---- 2. prefix of the earlier warps (the scan warp finds the carry meanwhile) ----
                     sub_prefix<S, V, LC, W, NW, false>(excl, warp, lane, sm.wagg, pre);
+                    if constexpr (kCluster) cluster_wait_acquire();
                     block_sync();  // carry ready
                     // ---- 3. re-walk the rows from the carry-in: h^(k+1) ----
+                    if constexpr (kPack) {
 #pragma unroll
-                    for (int v = 0; v < V; ++v) {
-                        float x[S], cv[S];
+                        for (int q = 0; q < VP; ++q) {
+                            const int v0 = 2 * q, v1 = 2 * q + 1;
+                            f2 x[S], cv[S], PA[S * S], Pb[S];
 #pragma unroll
-                        for (int s = 0; s < S; ++s) cv[s] = sm.cin[s][cc + v];
-                        apply<S>(pre.e[v].A, pre.e[v].b, cv, x);
+                            for (int s = 0; s < S; ++s) cv[s] = f2{sm.cin[s][cc + v0], sm.cin[s][cc + v1]};
 #pragma unroll
-                        for (int s = 0; s < S; ++s) hin[s][v] = x[s];  // h^(k+1) just before the sub-chunk
+                            for (int a = 0; a < S * S; ++a) PA[a] = f2{pre.e[v0].A[a], pre.e[v1].A[a]};
 #pragma unroll
-                        for (int r = 0; r < R; ++r) {
-                            float A[S * S], be[S], y[S];
-#pragma unroll
-                            for (int a = 0; a < S * S; ++a) A[a] = eA[r][a][v];
-#pragma unroll
-                            for (int s = 0; s < S; ++s) be[s] = eb[r][s][v];
-                            apply<S>(A, be, x, y);
+                            for (int s = 0; s < S; ++s) Pb[s] = f2{pre.e[v0].b[s], pre.e[v1].b[s]};
+                            apply2<S>(PA, Pb, cv, x);
 #pragma unroll
                             for (int s = 0; s < S; ++s) {
-                                x[s] = y[s];
-                                h[r][s][v] = y[s];
+                                hin[s][v0] = x[s].x;  // h^(k+1) just before the sub-chunk
+                                hin[s][v1] = x[s].y;
+                            }
+#pragma unroll
+                            for (int r = 0; r < R; ++r) {
+                                f2 A[S * S], be[S], y[S];
+#pragma unroll
+                                for (int a = 0; a < S * S; ++a) A[a] = f2{eA[r][a][v0], eA[r][a][v1]};
+#pragma unroll
+                                for (int s = 0; s < S; ++s) be[s] = f2{eb[r][s][v0], eb[r][s][v1]};
+                                apply2<S>(A, be, x, y);
+#pragma unroll
+                                for (int s = 0; s < S; ++s) {
+                                    x[s] = y[s];
+                                    h[r][s][v0] = y[s].x;
+                                    h[r][s][v1] = y[s].y;
+                                }
+                            }
+                        }
+                    } else {
+#pragma unroll
+                        for (int v = 0; v < V; ++v) {
+                            float x[S], cv[S];
+#pragma unroll
+                            for (int s = 0; s < S; ++s) cv[s] = sm.cin[s][cc + v];
+                            apply<S>(pre.e[v].A, pre.e[v].b, cv, x);
+#pragma unroll
+                            for (int s = 0; s < S; ++s) hin[s][v] = x[s];  // h^(k+1) just before the sub-chunk
+#pragma unroll
+                            for (int r = 0; r < R; ++r) {
+                                float A[S * S], be[S], y[S];
+#pragma unroll
+                                for (int a = 0; a < S * S; ++a) A[a] = eA[r][a][v];
+#pragma unroll
+                                for (int s = 0; s < S; ++s) be[s] = eb[r][s][v];
+                                apply<S>(A, be, x, y);
+#pragma unroll
+                                for (int s = 0; s < S; ++s) {
+                                    x[s] = y[s];
+                                    h[r][s][v] = y[s];
+                                }
                             }
                         }
                     }
@@ -448,13 +742,18 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
                         }
                     }
                 }
-                if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(prm.lb.status, kStatusNonFinite);
+                if (__any_sync(0xffffffffu, bad) && lane == 0) report(kStatusNonFinite);
             }
         }
         // No barrier here: the next tile's barrier (tile set up) comes before
         // its scan warp refills a stage or rewrites a ticket slot, and every
         // other shared array is rewritten only after a barrier that all of
         // this tile's readers have passed.
+    }
+    if constexpr (kCluster) {
+        // no CTA leaves while another may still read its shared memory
+        cluster_arrive_release();
+        cluster_wait_acquire();
     }
 }
 

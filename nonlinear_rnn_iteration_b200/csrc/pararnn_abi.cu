@@ -6,6 +6,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <unordered_map>
 
 #include "pararnn_b200.h"
 
@@ -56,11 +57,45 @@ template <typename PxT> using BwdGruS = FwdShape<CellGRU, PxT, 1, 32, 7, 4, 2, 2
 template <typename PxT> using BwdLstmS = FwdShape<CellLSTM, PxT, 1, 32, 7, 2, 2, 2, false>;
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far beyond any legitimate wait
+constexpr uint64_t kMaxWaitLimitNs = 10000000000ull;
 constexpr int kMaxK = 64;
 
+// K*(cell, T): the smallest Newton budget whose forward matches the
+// sequential unroll within 1e-4 (the relative error with a 1e-2 * max floor)
+// on the synthetic cells -- pre-activations ~ N(0,1), recurrent weights
+// ~ U(-0.5, 0.5), h0 = 0, 256 channels, two seeds -- measured on a T grid
+// (pararnn-torch page, Method section: K*(T) tables that max_iters=None
+// reads).  Between grid points a length takes the entry of the next grid
+// point up: K* does not fall as T grows on the grid, so that envelope never
+// gives fewer iterations than a measured neighbour needs.  Past the last
+// grid point the last entry holds.
+struct KStarRow {
+    int64_t T;
+    int gru, lstm;
+};
+constexpr KStarRow kKStar[] = {
+    {16, 3, 3},    {64, 3, 4},    {256, 3, 4},    {1024, 3, 4},   {4096, 3, 4},
+    {16384, 3, 4}, {65536, 3, 4}, {131072, 4, 4}, {262144, 4, 4},
+};
+
+int kstar_of(pararnn_cell cell, int64_t T) {
+    if (cell == PARARNN_CELL_LINEAR) return 1;
+    const int n = (int)(sizeof kKStar / sizeof kKStar[0]);
+    int i = 0;
+    while (i < n - 1 && kKStar[i].T < T) ++i;
+    return cell == PARARNN_CELL_DIAG_GRU ? kKStar[i].gru : kKStar[i].lstm;
+}
+
+// Test hooks (pararnn_debug_hooks), per calling thread: the limit of every
+// bounded wait between thread blocks, and the stall of the first tile.
+thread_local uint64_t t_wait_limit_ns = kWaitLimitNs;
+thread_local int t_stall_first = 0;
+thread_local int t_no_cluster = 0;
+
 // Epoch tags of the look-back words: unique per call within this process and
-// never 0, so that words left by other calls (or a zero-filled workspace)
-// never read as ready.
+// never 0.  Every call clears its look-back words on the stream before its
+// kernel runs, so a word from another call cannot be met; the tag still lets a
+// value and its "ready" mark travel in one 64-bit store (no fences).
 std::atomic<uint32_t> g_epoch{0};
 uint32_t next_epoch() {
     uint32_t e;
@@ -199,15 +234,62 @@ bool log_enabled() {
     return on;
 }
 
+// Launch facts that do not change between calls -- a kernel's resident
+// blocks per SM, whether a cluster shape fits, the SM count -- are looked up
+// once per (kernel, device, shape) and kept, so that a call on a small
+// problem spends its time on the GPU, not in driver queries.
+struct LaunchKey {
+    const void* kern;
+    int dev, a, b;
+    bool operator==(const LaunchKey& o) const { return kern == o.kern && dev == o.dev && a == o.a && b == o.b; }
+};
+struct LaunchKeyHash {
+    size_t operator()(const LaunchKey& k) const {
+        return std::hash<const void*>()(k.kern) ^ (size_t(k.dev) * 0x9e3779b97f4a7c15ull) ^ (size_t(k.a) << 20) ^
+               (size_t(k.b) << 40);
+    }
+};
+std::mutex g_launch_mutex;
+std::unordered_map<LaunchKey, int, LaunchKeyHash> g_launch_facts;
+
+// value cached under key, or computed by f() (which returns an int, or -1 on
+// a CUDA error, which is not cached)
+template <class F>
+int launch_fact(const LaunchKey& key, F f) {
+    {
+        std::lock_guard<std::mutex> lock(g_launch_mutex);
+        auto it = g_launch_facts.find(key);
+        if (it != g_launch_facts.end()) return it->second;
+    }
+    const int v = f();
+    if (v >= 0) {
+        std::lock_guard<std::mutex> lock(g_launch_mutex);
+        g_launch_facts[key] = v;
+    }
+    return v;
+}
+
 template <class Kern>
 pararnn_status persistent_grid(Kern kern, int threads, size_t smem, int64_t nTiles, unsigned& grid,
                                const char* what) {
-    int dev = 0, sms = 0, per_sm = 0;
+    int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
-    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (e == cudaSuccess) e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem);
-    if (e != cudaSuccess) return cuda_fail(e, "occupancy query");
+    if (e != cudaSuccess) return cuda_fail(e, "device query");
+    const int sms = launch_fact(LaunchKey{nullptr, dev, 0, 0}, [&] {
+        int n = 0;
+        return cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess ? n : -1;
+    });
+    const int per_sm = launch_fact(LaunchKey{reinterpret_cast<const void*>(kern), dev, threads, (int)smem}, [&] {
+        int n = 0;
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess ||
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, threads, smem) != cudaSuccess)
+            return -1;
+        return n;
+    });
+    if (sms < 0 || per_sm < 0) {
+        e = cudaGetLastError();
+        return cuda_fail(e == cudaSuccess ? cudaErrorUnknown : e, "occupancy query");
+    }
     if (per_sm < 1) return fail(PARARNN_ECUDA, "kernel does not fit on an SM");
     const int64_t want = (int64_t)sms * per_sm;
     grid = (unsigned)(nTiles < want ? nTiles : want);
@@ -217,8 +299,87 @@ pararnn_status persistent_grid(Kern kern, int threads, size_t smem, int64_t nTil
     return PARARNN_OK;
 }
 
+// The small-problem path: every channel group's tiles fit in one cluster
+// (at most kMaxClusterTiles along T), so the forward runs as clusters whose
+// CTAs pass carries through distributed shared memory -- one kernel launch,
+// no workspace clearing, no look-back (newton_fwd_kernel's kCluster mode).
+constexpr int kMaxClusterTiles = 8;
+
+template <class Kern>
+bool cluster_fits_query(Kern kern, int threads, size_t smem, int csize) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof cfg);
+    cfg.gridDim = dim3(csize, 1, 1);
+    cfg.blockDim = dim3(threads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = csize;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    return n >= 1;
+}
+
+template <class Kern>
+bool cluster_fits(Kern kern, int threads, size_t smem, int csize) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    // keyed apart from the persistent-grid facts by a negative thread count
+    return launch_fact(LaunchKey{reinterpret_cast<const void*>(kern), dev, -threads, csize},
+                       [&] { return cluster_fits_query(kern, threads, smem, csize) ? 1 : 0; }) == 1;
+}
+
+template <class Cell, typename PxT, class Sh, bool kLean, bool kPicard>
+pararnn_status launch_fwd_cluster(const Plan& pl, FwdParams prm, const CUtensorMap& map, cudaStream_t st,
+                                  bool& done) {
+    done = false;
+    auto kern = newton_fwd_kernel<Cell, PxT, Sh, kLean, kPicard, true>;
+    const size_t smem = sizeof(FwdSmem<Sh, PxT>);
+    const int csize = (int)pl.nChunks;
+    if (!cluster_fits(kern, Sh::NT, smem, csize)) return PARARNN_OK;  // the caller takes the look-back path
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof cfg);
+    cfg.gridDim = dim3((unsigned)pl.nTiles, 1, 1);
+    cfg.blockDim = dim3(Sh::NT, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = csize;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    if (log_enabled())
+        fprintf(stderr, "pararnn: newton_fwd(cluster) grid=%lld cluster=%d threads=%d smem=%zu\n",
+                (long long)pl.nTiles, csize, Sh::NT, smem);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, map, prm);
+    if (e != cudaSuccess) return cuda_fail(e, "forward cluster kernel launch");
+    done = true;
+    return PARARNN_OK;
+}
+
+// Launches the forward.  The small-problem cluster path runs when the
+// tiles of a channel group fit in one cluster (and the hooks allow it);
+// otherwise the workspace's first `clear_bytes` bytes (header and look-back
+// words) are cleared on the stream and the persistent look-back kernel runs.
 template <class Cell, typename PxT, class Sh>
-pararnn_status launch_fwd(const Plan& pl, FwdParams prm, cudaStream_t st) {
+pararnn_status launch_fwd(const Plan& pl, FwdParams prm, cudaStream_t st, void* ws, size_t clear_bytes,
+                          bool allow_cluster) {
     prm.nCG = pl.nCG;
     prm.nChunks = pl.nChunks;
     prm.nTiles = pl.nTiles;
@@ -228,6 +389,20 @@ pararnn_status launch_fwd(const Plan& pl, FwdParams prm, cudaStream_t st) {
         pararnn_status s = make_map(&map, prm.px, sizeof(PxT) == 2, prm.D, Sh::G, prm.B * prm.T, Sh::W, Sh::LF);
         if (s != PARARNN_OK) return s;
     }
+    if (allow_cluster && pl.nChunks <= kMaxClusterTiles) {
+        bool done = false;
+        pararnn_status s = PARARNN_OK;
+        if constexpr (!Cell::kNonlinear) {
+            s = prm.resid == nullptr ? launch_fwd_cluster<Cell, PxT, Sh, true, false>(pl, prm, map, st, done)
+                                     : launch_fwd_cluster<Cell, PxT, Sh, false, false>(pl, prm, map, st, done);
+        } else {
+            s = prm.picard > 0 ? launch_fwd_cluster<Cell, PxT, Sh, false, true>(pl, prm, map, st, done)
+                               : launch_fwd_cluster<Cell, PxT, Sh, false, false>(pl, prm, map, st, done);
+        }
+        if (s != PARARNN_OK || done) return s;
+    }
+    cudaError_t e = cudaMemsetAsync(ws, 0, clear_bytes, st);
+    if (e != cudaSuccess) return cuda_fail(e, "workspace reset");
     const size_t smem = sizeof(FwdSmem<Sh, PxT>);
     unsigned grid = 0;
     pararnn_status s;
@@ -241,13 +416,22 @@ pararnn_status launch_fwd(const Plan& pl, FwdParams prm, cudaStream_t st) {
             launched = true;
         }
     }
+    if constexpr (Cell::kNonlinear) {
+        if (prm.picard > 0) {  // Picard sweeps before the Newton iterations
+            auto kern = newton_fwd_kernel<Cell, PxT, Sh, false, true>;
+            s = persistent_grid(kern, Sh::NT, smem, pl.nTiles, grid, "newton_fwd(picard)");
+            if (s != PARARNN_OK) return s;
+            kern<<<grid, Sh::NT, smem, st>>>(map, prm);
+            launched = true;
+        }
+    }
     if (!launched) {
         auto kern = newton_fwd_kernel<Cell, PxT, Sh, false>;
         s = persistent_grid(kern, Sh::NT, smem, pl.nTiles, grid, "newton_fwd");
         if (s != PARARNN_OK) return s;
         kern<<<grid, Sh::NT, smem, st>>>(map, prm);
     }
-    cudaError_t e = cudaGetLastError();
+    e = cudaGetLastError();
     return e == cudaSuccess ? PARARNN_OK : cuda_fail(e, "forward kernel launch");
 }
 
@@ -323,8 +507,14 @@ int pararnn_state_width(pararnn_cell cell) {
     return cell == PARARNN_CELL_LINEAR ? 1 : cell == PARARNN_CELL_DIAG_GRU ? 1 : cell == PARARNN_CELL_DIAG_LSTM ? 2 : -1;
 }
 
+int pararnn_kstar(pararnn_cell cell, int64_t T) {
+    if (!cell_ok(cell) || T < 0) return -1;
+    return kstar_of(cell, T);
+}
+
 size_t pararnn_workspace_bytes(pararnn_cell cell, int64_t B, int64_t T, int64_t D, int K) {
     if (check_sizes(cell, B, T, D) != PARARNN_OK) return 0;
+    if (K == 0) K = kstar_of(cell, T);
     if (K < 1) K = 1;
     if (K > kMaxK) K = kMaxK;
     size_t m = kHeaderBytes + 256;
@@ -336,16 +526,23 @@ size_t pararnn_workspace_bytes(pararnn_cell cell, int64_t B, int64_t T, int64_t 
     return m;
 }
 
-pararnn_status pararnn_newton_forward(pararnn_cell cell, int64_t B, int64_t T, int64_t D, pararnn_dtype px_dtype,
-                                      const void* preacts, const float* diag_w, const float* h0, int K,
-                                      float* H_out, void* workspace, size_t ws_bytes, float* resid_hist,
-                                      void* stream) {
+}  // extern "C"
+
+namespace {
+
+pararnn_status forward_impl(pararnn_cell cell, int64_t B, int64_t T, int64_t D, pararnn_dtype px_dtype,
+                            const void* preacts, const float* diag_w, const float* h0, int picard, int K,
+                            float* H_out, void* workspace, size_t ws_bytes, float* resid_hist, void* stream) {
     g_last_error[0] = 0;
     pararnn_status st = check_sizes(cell, B, T, D);
     if (st != PARARNN_OK) return st;
     if (px_dtype != PARARNN_F32 && px_dtype != PARARNN_BF16)
         return fail(PARARNN_EINVAL, "unknown pre-activation dtype %d", (int)px_dtype);
-    if (K < 1 || K > kMaxK) return fail(PARARNN_EINVAL, "K=%d outside 1..%d", K, kMaxK);
+    if (K == 0) K = kstar_of(cell, T);  // max_iters=None: the measured K*(cell, T)
+    if (K < 1 || K > kMaxK) return fail(PARARNN_EINVAL, "K=%d outside 0..%d", K, kMaxK);
+    if (picard < 0 || picard > kPicardMax)
+        return fail(PARARNN_EINVAL, "picard_iters=%d outside 0..%d", picard, kPicardMax);
+    if (cell == PARARNN_CELL_LINEAR) picard = 0;  // one scan is exact: no guess to warm
     if (!workspace) return fail(PARARNN_EINVAL, "workspace is NULL");
     if (!aligned(workspace, 16)) return fail(PARARNN_EINVAL, "workspace not 16-byte aligned");
     const size_t need = pararnn_workspace_bytes(cell, B, T, D, K);
@@ -371,13 +568,21 @@ pararnn_status pararnn_newton_forward(pararnn_cell cell, int64_t B, int64_t T, i
     if (pl.nTiles >= (int64_t(1) << 31)) return fail(PARARNN_EINVAL, "too many tiles");
 
     char* ws = static_cast<char*>(workspace);
-    cudaError_t e = cudaMemsetAsync(ws, 0, kHeaderBytes, s);
-    if (e != cudaSuccess) return cuda_fail(e, "workspace reset");
+    cudaError_t e = cudaSuccess;
     if (resid_hist) {
         e = cudaMemsetAsync(resid_hist, 0, sizeof(float) * (K + 1), s);
         if (e != cudaSuccess) return cuda_fail(e, "resid_hist reset");
     }
-    if (empty) return PARARNN_OK;
+    if (empty) {
+        e = cudaMemsetAsync(ws, 0, kHeaderBytes, s);
+        return e == cudaSuccess ? PARARNN_OK : cuda_fail(e, "workspace reset");
+    }
+    // the look-back path clears, on the stream, everything of the workspace
+    // it reads before writing it: the header (status word, tile counter) and
+    // every look-back word (tile status, aggregates, inclusive states); the
+    // small-problem cluster path reads none of it and tags its status instead
+    const size_t clear_bytes = pl.off_part;
+    const bool allow_cluster = !t_no_cluster && !t_stall_first;
 
     FwdParams prm;
     memset(&prm, 0, sizeof prm);
@@ -390,6 +595,7 @@ pararnn_status pararnn_newton_forward(pararnn_cell cell, int64_t B, int64_t T, i
     prm.T = T;
     prm.D = D;
     prm.K = Keff;
+    prm.picard = picard;
     prm.ticket = reinterpret_cast<unsigned*>(ws) + 1;
     prm.lb.status = reinterpret_cast<unsigned*>(ws);
     prm.lb.tstat = reinterpret_cast<word_t*>(ws + pl.off_tstat);
@@ -398,20 +604,20 @@ pararnn_status pararnn_newton_forward(pararnn_cell cell, int64_t B, int64_t T, i
     prm.lb.nGroups = pl.nGroups;
     prm.lb.nSlots = pl.g.nSlots;
     prm.lb.epoch = next_epoch();
-    prm.lb.timeout_ns = kWaitLimitNs;
+    prm.lb.timeout_ns = t_wait_limit_ns;
+    prm.lb.stall_first = t_stall_first;
+    prm.tagged_status = reinterpret_cast<unsigned long long*>(ws + 8);
+    prm.status_epoch = reinterpret_cast<unsigned*>(ws + 16);
 
     typedef __nv_bfloat16 bf16;
     const bool bf = px_dtype == PARARNN_BF16;
-    if (cell == PARARNN_CELL_LINEAR) {
-        if (tma) st = bf ? launch_fwd<CellLinear, bf16, FwdLinT<bf16>>(pl, prm, s) : launch_fwd<CellLinear, float, FwdLinT<float>>(pl, prm, s);
-        else st = bf ? launch_fwd<CellLinear, bf16, FwdLinS<bf16>>(pl, prm, s) : launch_fwd<CellLinear, float, FwdLinS<float>>(pl, prm, s);
-    } else if (cell == PARARNN_CELL_DIAG_GRU) {
-        if (tma) st = bf ? launch_fwd<CellGRU, bf16, FwdGruT<bf16>>(pl, prm, s) : launch_fwd<CellGRU, float, FwdGruT<float>>(pl, prm, s);
-        else st = bf ? launch_fwd<CellGRU, bf16, FwdGruS<bf16>>(pl, prm, s) : launch_fwd<CellGRU, float, FwdGruS<float>>(pl, prm, s);
-    } else {
-        if (tma) st = bf ? launch_fwd<CellLSTM, bf16, FwdLstmT<bf16>>(pl, prm, s) : launch_fwd<CellLSTM, float, FwdLstmT<float>>(pl, prm, s);
-        else st = bf ? launch_fwd<CellLSTM, bf16, FwdLstmS<bf16>>(pl, prm, s) : launch_fwd<CellLSTM, float, FwdLstmS<float>>(pl, prm, s);
-    }
+#define PARARNN_FWD(C, SH) \
+    (bf ? launch_fwd<C, bf16, SH<bf16>>(pl, prm, s, ws, clear_bytes, allow_cluster) \
+        : launch_fwd<C, float, SH<float>>(pl, prm, s, ws, clear_bytes, allow_cluster))
+    if (cell == PARARNN_CELL_LINEAR) st = tma ? PARARNN_FWD(CellLinear, FwdLinT) : PARARNN_FWD(CellLinear, FwdLinS);
+    else if (cell == PARARNN_CELL_DIAG_GRU) st = tma ? PARARNN_FWD(CellGRU, FwdGruT) : PARARNN_FWD(CellGRU, FwdGruS);
+    else st = tma ? PARARNN_FWD(CellLSTM, FwdLstmT) : PARARNN_FWD(CellLSTM, FwdLstmS);
+#undef PARARNN_FWD
     if (st != PARARNN_OK) return st;
     if (resid_hist && Keff < K) {
         // the linear cell is exact after its one scan: later iterates equal it
@@ -421,6 +627,26 @@ pararnn_status pararnn_newton_forward(pararnn_cell cell, int64_t B, int64_t T, i
         }
     }
     return PARARNN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+pararnn_status pararnn_newton_forward(pararnn_cell cell, int64_t B, int64_t T, int64_t D, pararnn_dtype px_dtype,
+                                      const void* preacts, const float* diag_w, const float* h0, int K,
+                                      float* H_out, void* workspace, size_t ws_bytes, float* resid_hist,
+                                      void* stream) {
+    return forward_impl(cell, B, T, D, px_dtype, preacts, diag_w, h0, 0, K, H_out, workspace, ws_bytes, resid_hist,
+                        stream);
+}
+
+pararnn_status pararnn_newton_forward_picard(pararnn_cell cell, int64_t B, int64_t T, int64_t D,
+                                             pararnn_dtype px_dtype, const void* preacts, const float* diag_w,
+                                             const float* h0, int picard_iters, int K, float* H_out,
+                                             void* workspace, size_t ws_bytes, float* resid_hist, void* stream) {
+    return forward_impl(cell, B, T, D, px_dtype, preacts, diag_w, h0, picard_iters, K, H_out, workspace, ws_bytes,
+                        resid_hist, stream);
 }
 
 pararnn_status pararnn_newton_backward(pararnn_cell cell, int64_t B, int64_t T, int64_t D, pararnn_dtype px_dtype,
@@ -459,8 +685,10 @@ pararnn_status pararnn_newton_backward(pararnn_cell cell, int64_t B, int64_t T, 
     const Plan pl = make_plan(cell, B, T, D, 1, false, tma);
     if (pl.nTiles >= (int64_t(1) << 31)) return fail(PARARNN_EINVAL, "too many tiles");
 
+    // clear the status word, the tile counter and every look-back word (the
+    // per-tile dL/da partials after them are written before they are read)
     char* ws = static_cast<char*>(workspace);
-    cudaError_t e = cudaMemsetAsync(ws, 0, kHeaderBytes, s);
+    cudaError_t e = cudaMemsetAsync(ws, 0, empty ? kHeaderBytes : pl.off_part, s);
     if (e != cudaSuccess) return cuda_fail(e, "workspace reset");
     if (empty) {
         const int G = pararnn_num_gates(cell);
@@ -496,7 +724,8 @@ pararnn_status pararnn_newton_backward(pararnn_cell cell, int64_t B, int64_t T, 
     prm.lb.nGroups = pl.nGroups;
     prm.lb.nSlots = 1;
     prm.lb.epoch = next_epoch();
-    prm.lb.timeout_ns = kWaitLimitNs;
+    prm.lb.timeout_ns = t_wait_limit_ns;
+    prm.lb.stall_first = t_stall_first;
 
     typedef __nv_bfloat16 bf16;
     const bool bf = px_dtype == PARARNN_BF16;
@@ -515,12 +744,17 @@ pararnn_status pararnn_newton_backward(pararnn_cell cell, int64_t B, int64_t T, 
 
 pararnn_status pararnn_status_sync(const void* workspace, void* stream) {
     if (!workspace) return fail(PARARNN_EINVAL, "workspace is NULL");
-    unsigned word = 0;
+    // header words: 0 the status flags of a look-back call (cleared at its
+    // start); 2..3 the tagged flags of a small-problem cluster call and 4 that
+    // call's number (0 after any look-back call, which clears them)
+    unsigned hdr[5] = {0, 0, 0, 0, 0};
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    cudaError_t e = cudaMemcpyAsync(&word, workspace, sizeof word, cudaMemcpyDeviceToHost, s);
+    cudaError_t e = cudaMemcpyAsync(hdr, workspace, sizeof hdr, cudaMemcpyDeviceToHost, s);
     if (e != cudaSuccess) return cuda_fail(e, "status copy");
     e = cudaStreamSynchronize(s);
     if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+    unsigned word = hdr[0];
+    if (hdr[4] != 0) word = (hdr[3] == hdr[4]) ? hdr[2] : 0u;
     if (word & kStatusTimeout) return PARARNN_ETIMEOUT;
     if (word & kStatusNonFinite) return PARARNN_ENONFINITE;
     return PARARNN_OK;
@@ -538,6 +772,17 @@ const char* pararnn_status_string(pararnn_status status) {
 }
 
 const char* pararnn_last_error(void) { return g_last_error; }
+
+pararnn_status pararnn_debug_hooks(uint64_t wait_limit_ns, int flags) {
+    g_last_error[0] = 0;
+    if (wait_limit_ns > kMaxWaitLimitNs) return fail(PARARNN_EINVAL, "wait limit above 10 s");
+    if (flags & ~(PARARNN_HOOK_STALL_FIRST_TILE | PARARNN_HOOK_NO_CLUSTER))
+        return fail(PARARNN_EINVAL, "unknown hook flags 0x%x", flags);
+    t_wait_limit_ns = wait_limit_ns ? wait_limit_ns : kWaitLimitNs;
+    t_stall_first = (flags & PARARNN_HOOK_STALL_FIRST_TILE) != 0;
+    t_no_cluster = (flags & PARARNN_HOOK_NO_CLUSTER) != 0;
+    return PARARNN_OK;
+}
 
 pararnn_status pararnn_probe_wait_timeout(void* workspace, size_t ws_bytes, uint64_t timeout_ns, void* stream) {
     g_last_error[0] = 0;

@@ -171,3 +171,39 @@ def test_host_path_workspace_bytes():
     assert 0 < f(gru, 8, 1024, 256, 3, binding.F32, 1, 64) < one
     # a slice never exceeds the batch
     assert f(gru, 2, 1024, 256, 3, binding.F32, 5) == f(gru, 2, 1024, 256, 3, binding.F32, 2)
+
+
+def test_debug_hooks_reject_long_limits():
+    # pure host function: it only records the limits for later calls on this thread
+    assert binding.pararnn_debug_hooks(20_000_000_000, 0) == binding.EINVAL
+    assert "10 s" in binding.pararnn_last_error()
+    assert binding.pararnn_debug_hooks(20_000_000, 1) == binding.OK
+    assert binding.pararnn_debug_hooks(0, 0) == binding.OK
+
+
+def test_kstar_table_lookup():
+    # K = 0 selects K*(cell, T): the linear cell needs its one scan; a length
+    # between grid points takes the next grid point's entry, past the grid the
+    # last entry
+    assert binding.pararnn_kstar(binding.LINEAR, 1000) == 1
+    assert binding.pararnn_kstar(7, 1000) == -1
+    assert binding.pararnn_kstar(binding.DIAG_GRU, -1) == -1
+    for cell in (binding.DIAG_GRU, binding.DIAG_LSTM):
+        ks = [binding.pararnn_kstar(cell, T) for T in (1, 16, 17, 64, 1000, 1024, 4096, 131072, 262144, 10 ** 7)]
+        assert all(1 <= k <= 8 for k in ks)
+        assert ks == sorted(ks)  # an envelope: never fewer iterations for a longer sequence
+        assert binding.pararnn_kstar(cell, 17) == binding.pararnn_kstar(cell, 64)
+        assert binding.pararnn_kstar(cell, 10 ** 7) == binding.pararnn_kstar(cell, 262144)
+    # the workspace for K = 0 is the one for K = K*
+    for cell in (binding.DIAG_GRU, binding.DIAG_LSTM):
+        assert binding.pararnn_workspace_bytes(cell, 2, 5000, 64, 0) == binding.pararnn_workspace_bytes(
+            cell, 2, 5000, 64, binding.pararnn_kstar(cell, 5000))
+
+
+def test_picard_iters_outside_range_is_rejected():
+    # checked before any pointer: nothing is launched
+    for p in (-1, 5):
+        st = binding.pararnn_newton_forward_picard(binding.DIAG_GRU, 1, 10, 8, binding.F32, None, None, None, p, 2,
+                                                   None, None, 0, None, None)
+        assert st == binding.EINVAL
+        assert "picard_iters" in binding.pararnn_last_error()

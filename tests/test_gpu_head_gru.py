@@ -252,3 +252,50 @@ def test_head_backward_full_size_sampled(cuda_device):
         if b in (0, 5):
             assert rel_err(to_np(dpx[b:b + 1, :, :, sl]), r_dpx) <= TOL_G, b
     assert rel_err(to_np(dU[:, h:h + 1]), dU_ref) <= TOL_G
+
+
+# ---- the sequential unroll on the GPU (pararnn_head_gru_unroll) -------------
+
+@pytest.mark.parametrize("case", [(2, 100, 64, 1), (1, 77, 96, 3), (2, 40, 48, 3), (1, 130, 128, 2),
+                                  (3, 33, 256, 4), (1, 1, 64, 1)], ids=lambda c: "B%dT%dD%dh%d" % c)
+@pytest.mark.parametrize("h0", [False, True])
+def test_head_unroll_matches_oracle(case, h0, cuda_device):
+    B, T, D, nh = case
+    px, U, hz, pxt, Ut, hzt = _case(B, T, D, nh, seed=T + D, h0=h0)
+    H = binding.head_gru_unroll(pxt, Ut, hzt)
+    ref = oracle.head_gru_unroll(px, U, hz)
+    assert rel_err(to_np(H), ref) <= TOL_H
+
+
+def test_head_unroll_bf16_slow_memory_and_newton(cuda_device):
+    # bf16 pre-activations against the oracle on the same values
+    x = workloads.head_host_inputs(2, 300, 128, 2, 31)
+    pxb = torch.from_numpy(x["px"]).to(DEV).to(torch.bfloat16)
+    H = binding.head_gru_unroll(pxb, torch.from_numpy(x["U"]).to(DEV))
+    ref = oracle.head_gru_unroll(pxb.float().cpu().numpy(), x["U"], None)
+    assert rel_err(to_np(H), ref) <= TOL_H
+    # slow memory, several chunks of pre-activations
+    px, U = slow_inputs.head_host(1, 400, 128, 2, 32)
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(DEV)
+    H = binding.head_gru_unroll(t(px), t(U))
+    assert rel_err(to_np(H), oracle.head_gru_unroll(px, U, None)) <= TOL_H
+    # the Newton forward at K = T reaches the same sequence
+    px, U, hz, pxt, Ut, hzt = _case(1, 20, 64, 1, seed=33, h0=True)
+    Hn = binding.head_gru_forward(pxt, Ut, hzt, K=20)
+    Hu = binding.head_gru_unroll(pxt, Ut, hzt)
+    assert rel_err(to_np(Hn), to_np(Hu)) <= TOL_H
+
+
+def test_head_unroll_rejects_bad_arguments(cuda_device):
+    px = torch.zeros((1, 8, 3, 64), device=DEV)
+    U = torch.zeros((3, 1, 64, 64), device=DEV)
+    H = torch.empty((1, 8, 64), device=DEV)
+    ws = torch.empty(256, dtype=torch.uint8, device=DEV)
+    s = torch.cuda.current_stream()
+    assert binding.pararnn_head_gru_unroll(1, 8, 64, 3, binding.F32, px, U, None, H, ws, 256, s) == binding.EINVAL
+    assert binding.pararnn_head_gru_unroll(1, 8, 64, 8, binding.F32, px, U, None, H, ws, 256, s) == binding.EINVAL
+    assert binding.pararnn_head_gru_unroll(1, 8, 64, 1, binding.F32, px, U, None, H, ws, 16, s) == binding.EINVAL
+    assert binding.pararnn_head_gru_unroll(1, 8, 64, 1, binding.F32, px.cpu(), U, None, H, ws, 256, s) == binding.EINVAL
+    bad = torch.full((1, 8, 3, 64), float("nan"), device=DEV)
+    assert binding.pararnn_head_gru_unroll(1, 8, 64, 1, binding.F32, bad, U, None, H, ws, 256, s) == binding.OK
+    assert binding.pararnn_status_sync(ws, s) == binding.ENONFINITE

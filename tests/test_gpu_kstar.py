@@ -60,6 +60,31 @@ def test_kstar_against_unroll(cell, cuda_device):
     assert ks == sorted(ks) or max(ks) - min(ks) <= 4
 
 
+KSTAR_GRID = (16, 64, 256, 1024, 4096, 16384, 65536, 131072, 262144)
+
+
+@pytest.mark.parametrize("cell", [oracle.DIAG_GRU, oracle.DIAG_LSTM], ids=["gru", "lstm"])
+def test_library_kstar_table_reaches_the_unroll(cell, cuda_device):
+    """The table K = 0 reads (pararnn_kstar): on its own grid, with the draws
+    it was measured on (256 channels, two seeds per length), the forward at
+    K*(cell, T) matches the fp64 unroll within 1e-4, and K = 0 gives exactly
+    that forward."""
+    name = "GRU" if cell == oracle.DIAG_GRU else "LSTM"
+    print("\nlibrary K*, %s, B=1, D=256: error at K*-1 and K*" % name)
+    for T in KSTAR_GRID:
+        ks = binding.pararnn_kstar(cell, T)
+        for seed in (100 + T, 7 + T):
+            px, w = _draw(cell, T, 256, seed)
+            ref = oracle.unroll(cell, px, w)
+            pxt, wt = torch.from_numpy(px).to(DEV), torch.from_numpy(w).to(DEV)
+            H = binding.newton_forward(cell, pxt, wt, None, K=ks)
+            assert torch.equal(H, binding.newton_forward(cell, pxt, wt, None, K=0))
+            err = rel_err(to_np(H), ref)
+            below = rel_err(to_np(binding.newton_forward(cell, pxt, wt, None, K=ks - 1)), ref)
+            print("  T=%6d seed=%6d K*=%d  error %.1e at K*-1, %.1e at K*" % (T, seed, ks, below, err))
+            assert err <= TAU, (T, seed, ks, err)
+
+
 @pytest.mark.parametrize("cell", [oracle.DIAG_GRU, oracle.DIAG_LSTM], ids=["gru", "lstm"])
 def test_k_equal_t_is_the_unroll(cell, cuda_device):
     T = 12
