@@ -6,7 +6,9 @@
 A step is one pass of the hot path over one batch of the workload: one
 ``pararnn_newton_forward`` call (all K Newton iterations; the linear workload
 is one exact scan), plus ``pararnn_newton_backward`` for workloads that carry
-a backward pass.  Inputs are resident in HBM before timing and are larger
+a backward pass.  The default workload is the largest: the long-sequence
+diagonal GRU (B=1, T=131072, D=4096, K=2, bf16 pre-activations with float32
+state), forward and adjoint in every step.  Inputs are resident in HBM before timing and are larger
 than L2, so no flush is needed between steps.  The device time of the K
 timed steps is measured with CUDA events on the launching stream between a
 barrier and a synchronize on both sides; with N > 1 processes (one per GPU,
@@ -36,20 +38,39 @@ sys.path.insert(0, ROOT)
 METRIC = "Newton-solve B·T·D elements/sec at K iters; achieved HBM GB/s vs B200 peak"
 UNIT = "elem/s"
 
-# Algorithmic HBM bytes per (b,t,d) element for one call, by what the fused
-# kernels must move at minimum: every pre-activation read once, every output
-# written once (the Newton iterate never leaves the chip between iterations).
+# HBM bytes per (b,t,d) element for one call, two ways.
+#
+# Fused minimum (what these kernels move): every pre-activation read once,
+# every output written once; the Newton iterate never leaves the chip between
+# iterations.
 #   linear f32 fwd: a, b read (8) + h written (4)                         = 12
 #   GRU fwd: px read (3 x 4 f32 | 3 x 2 bf16) + h written (4)            = 16 | 10
 #   LSTM fwd f32: px read (4 x 4) + (c, h) written (8)                    = 24
 #   GRU bwd: px (3 x 4 | 3 x 2) + H (4) + dL/dH (4) read, dL/dpx (3 x 4) written
 #                                                                        = 32 | 26
+# Streaming design (one HBM pass per Newton iteration, the method's plain
+# form): the first iteration reads px and writes the state, each later one
+# reads px and the state and writes the state; the backward moves the same
+# bytes in both designs.  This is the figure the HBM roofline fraction is
+# taken on.
 ALGO_BYTES = {
     ("linear", "f32", "fwd"): 12, ("diag_gru", "f32", "fwd"): 16, ("diag_gru", "bf16", "fwd"): 10,
     ("diag_lstm", "f32", "fwd"): 24, ("diag_lstm", "bf16", "fwd"): 16,
     ("linear", "f32", "bwd"): 24, ("diag_gru", "f32", "bwd"): 32, ("diag_gru", "bf16", "bwd"): 26,
     ("diag_lstm", "f32", "bwd"): 48, ("diag_lstm", "bf16", "bwd"): 40,
 }
+PX_BYTES = {"f32": 4, "bf16": 2}
+# nominal B200 HBM3e bandwidth, reported beside the measured copy bandwidth
+NOMINAL_HBM_GBS = 8000.0
+
+
+def streaming_bytes_per_elem(w, direction):
+    """Bytes per element of the streaming design (see above)."""
+    if direction == "bwd" or w.cell == "linear":
+        return ALGO_BYTES[(w.cell, w.px_dtype, direction)]
+    px = w.G * PX_BYTES[w.px_dtype]
+    state = 4 * w.S
+    return (px + state) + (px + 2 * state) * (w.K - 1)
 # channels per slice of the host-buffer pipeline in the e2e measurement:
 # 8 x 1024 channels in slices of 256 make 32 slices, whose shorter fill and
 # drain beat whole rows (8 slices)
@@ -155,8 +176,14 @@ def time_head(w, device, steps, warmup):
     def bwd():
         binding.head_gru_backward(x["px"], x["U"], H, g, workspace=wsb, stream=stream, sync_status=False)
 
+    Hu = torch.empty_like(H)
+    wsu = torch.empty(256, dtype=torch.uint8, device=device)
+
+    def unroll():
+        binding.head_gru_unroll(x["px"], x["U"], None, out=Hu, workspace=wsu, stream=stream, sync_status=False)
+
     times = []
-    for f in (fwd, bwd):
+    for f in (fwd, bwd, unroll):
         for _ in range(warmup):
             f()
         torch.cuda.synchronize(device)
@@ -170,21 +197,28 @@ def time_head(w, device, steps, warmup):
     st = binding.pararnn_status_sync(ws, stream)
     if st == binding.OK:
         st = binding.pararnn_status_sync(wsb, stream)
-    del x, H, ws, wsb, g
+    if st == binding.OK:
+        st = binding.pararnn_status_sync(wsu, stream)
+    del x, H, Hu, ws, wsb, wsu, g
     torch.cuda.empty_cache()
-    return times[0], times[1], binding.STATUS.get(st, st)
+    return times[0], times[1], binding.STATUS.get(st, st), times[2]
 
 
-def head_line(w, ms, bwd_ms, status):
+def head_line(w, ms, bwd_ms, status, unroll_ms=None):
     """A head-wise forward's line: time, elements/s, and the FLOP rate of its
     Jacobian products -- 2 d^3 useful FLOP per step and (batch row, head),
-    issued as three TF32 products -- against the TF32 tensor peak."""
+    issued as three TF32 products -- against the TF32 tensor peak; beside it
+    the sequential unroll on the GPU (pararnn_head_gru_unroll) of the same
+    problem."""
     peaks = measured_peaks()
     useful = 2.0 * w.d ** 3 * w.B * w.T * w.n_heads * w.K
     tf32_peak = peaks["bf16_tflops"] * TF32_PER_BF16
+    extra = {}
+    if unroll_ms is not None:
+        extra = {"unroll_ms": round(unroll_ms, 4), "unroll_elem_per_s": w.elements / (unroll_ms / 1e3)}
     return {"ms_per_step": round(ms, 4), "elem_per_s": w.elements / (ms / 1e3), "K": w.K,
             "n_heads": w.n_heads, "d": w.d, "status": status, "bwd_ms": round(bwd_ms, 4),
-            "bwd_elem_per_s": w.elements / (bwd_ms / 1e3),
+            "bwd_elem_per_s": w.elements / (bwd_ms / 1e3), **extra,
             "roofline": {"bound": "tensor", "kernel": "head_chunk_tc_kernel (Jacobian products, tcgen05 TF32)",
                          "achieved_useful": round(useful / (ms / 1e3) / 1e12, 2),
                          "achieved_issued": round(3 * useful / (ms / 1e3) / 1e12, 2),
@@ -198,23 +232,49 @@ def head_workloads(device):
 
     out = {}
     for name, w in workloads.HEAD_WORKLOADS.items():
-        ms, bms, status = time_head(w, device, steps=5, warmup=3)
-        out[name] = head_line(w, ms, bms, status)
+        ms, bms, status, ums = time_head(w, device, steps=5, warmup=3)
+        out[name] = head_line(w, ms, bms, status, ums)
     return out
 
 
-def recorded_traffic(kernel, workload):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken
-    on the current kernel sources; else None."""
+def recorded_traffic(kernel, w):
+    """DRAM bytes per launch of `kernel` on workload `w` from the committed
+    ncu records (profiles/traffic.json), if they were taken on the current
+    kernel sources; else None.  A record taken on a shorter sequence of the
+    same workload (every tile moves the same bytes) is scaled to the full
+    launch by the ratio of elements."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
         rec = json.load(f)
-    e = rec.get("%s/%s" % (kernel, workload))
-    if not e or e.get("kernel_source_hash") != kernel_source_hash():
-        return None
-    return e.get("dram_bytes_per_launch")
+    for key, e in rec.items():
+        if key != "%s/%s" % (kernel, w.name) and not key.startswith("%s/%s@" % (kernel, w.name)):
+            continue
+        if e.get("kernel_source_hash") != kernel_source_hash():
+            continue
+        n = e.get("elements", w.elements)
+        return {"dram_bytes_per_launch": int(round(e["dram_bytes_per_launch"] * w.elements / n)),
+                "captured_on": key, "scaled_by": round(w.elements / n, 3)}
+    return None
+
+
+def kernel_roofline(w, direction, ms, peaks):
+    """The HBM roofline record of one kernel launch on workload `w`."""
+    kernel = "newton_fwd_kernel" if direction == "fwd" else "adjoint_bwd_kernel"
+    sb = streaming_bytes_per_elem(w, direction) * w.elements
+    fb = ALGO_BYTES[(w.cell, w.px_dtype, direction)] * w.elements
+    achieved = sb / (ms / 1e3) / 1e9
+    tr = recorded_traffic(kernel, w)
+    return {"bound": "hbm", "kernel": kernel, "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
+            "peak_source": peaks["source"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+            "frac_of_nominal_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),
+            "traffic": None if tr is None else tr["dram_bytes_per_launch"],
+            "traffic_record": tr,
+            "bytes_per_elem": sb // w.elements, "bytes_model": "streaming design (one HBM pass per iteration)",
+            "fused_bytes_per_elem": fb // w.elements,
+            "fused_achieved": round(fb / (ms / 1e3) / 1e9, 1),
+            "algorithmic_bytes_per_launch": sb, "launch_ms": round(ms, 4)}
 
 
 class ClockSampler:
@@ -427,48 +487,64 @@ def time_e2e(prob, steps):
     return ms, h2d, d2h
 
 
-def cpu_baseline(w, device, seed, target_s=12.0):
-    """The oracle as it stands, on a bounded sample of the workload's channels
-    (full length T each), on this host's cores."""
+def cpu_baseline(w, device, seed, target_s=12.0, max_bytes=2.0e9):
+    """The oracle as it stands -- Newton with sequential solves, plus the
+    sequential adjoint for a workload with a backward -- on a bounded sample
+    of the workload's channels (full length T each), on this host's cores and
+    on one core."""
     import numpy as np
+    import torch
 
     import oracle
     from nonlinear_rnn_iteration_b200 import workloads
 
     threads = os.cpu_count() or 1
-    x = workloads.device_inputs(w, device, seed=seed)
+    x = workloads.device_inputs(w, device, seed=seed, with_grad=w.backward)
 
-    def run(n):
+    def sample(n):
         chans = workloads.sample_channels(w, n, seed=5)
-        bs = [b for b, _ in chans]
-        ds = [d for _, d in chans]
-        import torch
-
-        bi, di = torch.tensor(bs, device=device), torch.tensor(ds, device=device)
-        # (1, T, G, n) contiguous fp64, prepared outside the timed region
-        px = np.ascontiguousarray(x["px"][bi, :, :, di].float().cpu().numpy().transpose(1, 2, 0)[None],
-                                  dtype=np.float64)
+        bi = torch.tensor([b for b, _ in chans], device=device)
+        di = torch.tensor([d for _, d in chans], device=device)
+        # (1, T, X, n) contiguous fp64, prepared outside the timed region
+        prep = lambda t: np.ascontiguousarray(t[bi, :, :, di].float().cpu().numpy().transpose(1, 2, 0)[None],
+                                              dtype=np.float64)
         a = None if x["a"] is None else np.ascontiguousarray(x["a"][:, di].cpu().numpy(), dtype=np.float64)
+        return prep(x["px"]), a, (prep(x["dLdH"]) if w.backward else None)
+
+    def run(inp, nthreads):
+        px, a, g = inp
         t = time.perf_counter()
         if w.cell == "linear":
-            oracle.unroll(w.cell_id, px, a, None, nthreads=threads)
+            H = oracle.unroll(w.cell_id, px, a, None, nthreads=nthreads)
         else:
-            oracle.newton(w.cell_id, px, a, None, K=w.K, nthreads=threads)
-        return time.perf_counter() - t, n * w.T
+            H, _ = oracle.newton(w.cell_id, px, a, None, K=w.K, nthreads=nthreads)
+        if w.backward:
+            oracle.adjoint(w.cell_id, px, a, None, H, g, nthreads=nthreads)
+        return time.perf_counter() - t
 
-    n = max(threads, 8)
-    dt, el = run(n)
-    while dt < 1.0 and n < w.B * w.D:
-        n = min(w.B * w.D, n * 4)
-        dt, el = run(n)
-    n_final = int(min(w.B * w.D, max(n, n * target_s / max(dt, 1e-3))))
+    # bytes of fp64 host arrays per sampled channel (inputs, H, gradients)
+    per_chan = 8 * w.T * (w.G + w.S + (w.S + w.G if w.backward else 0))
+    n_cap = max(1, min(w.B * w.D, int(max_bytes // per_chan)))
+    n = min(n_cap, max(threads, 8))
+    dt = run(sample(n), threads)
+    while dt < 1.0 and n < n_cap:
+        n = min(n_cap, n * 4)
+        dt = run(sample(n), threads)
+    n_final = int(min(n_cap, max(n, n * target_s / max(dt, 1e-3))))
     if n_final > n:
-        dt, el = run(n_final)
         n = n_final
+        dt = run(sample(n), threads)
+    # one core, on a sample sized for a few seconds
+    n1 = max(1, min(n, int(n * 3.0 / max(dt * threads, 1e-3))))
+    dt1 = run(sample(n1), 1)
     del x
     kind = "sequential unroll" if w.cell == "linear" else "Newton K=%d with sequential solves" % w.K
-    return {"value": el / dt, "unit": UNIT, "cores": threads, "kind": "oracle",
-            "sample": "%d of %d channels at full T=%d (%s, fp64), %.1f s" % (n, w.B * w.D, w.T, kind, dt)}
+    if w.backward:
+        kind += " + sequential adjoint"
+    return {"value": n * w.T / dt, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": "%d of %d channels at full T=%d (%s, fp64), %.1f s" % (n, w.B * w.D, w.T, kind, dt),
+            "value_1_core": n1 * w.T / dt1, "cores_1_core": 1,
+            "sample_1_core": "%d channels at full T=%d, %.1f s" % (n1, w.T, dt1)}
 
 
 def extra_workloads(names, device, seed_base):
@@ -477,20 +553,16 @@ def extra_workloads(names, device, seed_base):
 
     from nonlinear_rnn_iteration_b200 import workloads
 
-    peak = measured_peaks()["hbm_gbs"]
+    peaks = measured_peaks()
     out = {}
     for name in names:
         w = workloads.WORKLOADS[name]
         prob = Problem(w, device, seed_base + w.seed)
         ms, fwd, bwd = time_device(prob, steps=5, warmup=3, dist=None, device=device)
-        fb = ALGO_BYTES[(w.cell, w.px_dtype, "fwd")] * w.elements
-        rec = {"ms_per_step": round(ms, 4), "elem_per_s": w.elements / (ms / 1e3),
-               "fwd_ms": round(fwd, 4), "fwd_algo_gbs": round(fb / (fwd / 1e3) / 1e9, 1),
-               "fwd_frac_hbm": round(fb / (fwd / 1e3) / 1e9 / peak, 3), "fwd_bytes_per_elem": fb // w.elements}
+        rec = {"ms_per_step": round(ms, 4), "elem_per_s": w.elements / (ms / 1e3), "fwd_ms": round(fwd, 4),
+               "fwd": kernel_roofline(w, "fwd", fwd, peaks)}
         if w.backward:
-            bb = ALGO_BYTES[(w.cell, w.px_dtype, "bwd")] * w.elements
-            rec.update(bwd_ms=round(bwd, 4), bwd_algo_gbs=round(bb / (bwd / 1e3) / 1e9, 1),
-                       bwd_frac_hbm=round(bb / (bwd / 1e3) / 1e9 / peak, 3), bwd_bytes_per_elem=bb // w.elements)
+            rec.update(bwd_ms=round(bwd, 4), bwd=kernel_roofline(w, "bwd", bwd, peaks))
         out[name] = rec
         del prob
         torch.cuda.empty_cache()
@@ -516,26 +588,29 @@ def run_native(args):
     clocks = clk.summary()
     value = aggregate_throughput(w.elements, world, 1, ms)
     peaks = measured_peaks()
-    dir_ = "fwd"
-    algo = ALGO_BYTES[(w.cell, w.px_dtype, dir_)] * w.elements
-    achieved = algo / (fwd_ms / 1e3) / 1e9
-    roof = {"bound": "hbm", "kernel": "newton_fwd_kernel", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
-            "peak_source": peaks["source"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
-            "traffic": recorded_traffic("newton_fwd_kernel", w.name),
-            "algorithmic_bytes_per_launch": algo, "bytes_per_elem": algo // w.elements,
-            "launch_ms": round(fwd_ms, 4)}
+    kernels = {"fwd": kernel_roofline(w, "fwd", fwd_ms, peaks)}
+    if w.backward:
+        kernels["bwd"] = kernel_roofline(w, "bwd", bwd_ms, peaks)
+    # the dominant kernel: the one that takes longer per step
+    dominant = "bwd" if (w.backward and bwd_ms > fwd_ms) else "fwd"
+    roof = dict(kernels[dominant])
+    roof["all_kernels"] = kernels
     if args.quick:
         e2e = None
     else:
         e2e_ms, h2d, d2h = time_e2e(prob, steps=3)
         e2e = {"value": w.elements / (e2e_ms / 1e3) * world, "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 3)}
+    step = "forward (K=%d Newton iterations)" % w.K if w.cell != "linear" else "forward (one exact scan)"
+    if w.backward:
+        step += " + adjoint backward"
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32" if w.px_dtype == "f32" else "bf16 px / f32 state", "data": "synthetic",
         "config": {"workload": w.name, "cell": w.cell, "B": w.B, "T": w.T, "D": w.D, "K": w.K,
-                   "px_dtype": w.px_dtype, "backward": w.backward,
+                   "px_dtype": w.px_dtype, "backward": w.backward, "step": step,
+                   "fwd_ms": round(fwd_ms, 4), "bwd_ms": round(bwd_ms, 4) if w.backward else None,
                    "l2": "inputs larger than L2 (%.2f GB pre-activations per rank), no flush"
                          % (prob.px.numel() * prob.px.element_size() / 1e9),
                    "parallelism": "replicas%d" % world},
@@ -567,9 +642,9 @@ def run_head(args):
                                    args.T or w.T, w.D, w.n_heads, w.K, w.px_dtype, w.seed)
     device = torch.device("cuda", 0)
     torch.cuda.set_device(device)
-    ms, bms, status = time_head(w, device, args.steps, args.warmup)
+    ms, bms, status, ums = time_head(w, device, args.steps, args.warmup)
     line = {"workload": w.name, "metric": METRIC, "unit": UNIT, "data": "synthetic",
-            **head_line(w, ms, bms, status)}
+            **head_line(w, ms, bms, status, ums)}
     print(json.dumps(line), flush=True)
 
 
@@ -589,33 +664,40 @@ def run_reference(args):
     # takes a few seconds on this host
     n = max(threads, 8)
     per_step = []
-    x = workloads.host_inputs(w.with_shape(B=1, D=n), seed=w.seed)
+    # fp64 host arrays per channel (inputs, H, gradients): the sample stays
+    # within about 2 GB of host memory
+    per_chan = 8 * w.T * (w.G + w.S + (w.S + w.G if w.backward else 0))
+    n_cap = max(1, min(w.B * w.D, int(2.0e9 // per_chan)))
+    n = min(n, n_cap)
 
     def prepare(xx):
         # fp64 contiguous inputs, converted outside the timed region
         return {k: (None if v is None else np.ascontiguousarray(v, dtype=np.float64)) for k, v in xx.items()}
 
-    x = prepare(x)
+    x = prepare(workloads.host_inputs(w.with_shape(B=1, D=n), seed=w.seed, with_grad=w.backward))
 
     def one():
         t = time.perf_counter()
         if w.cell == "linear":
-            oracle.unroll(w.cell_id, x["px"], x["a"], None, nthreads=threads)
+            H = oracle.unroll(w.cell_id, x["px"], x["a"], None, nthreads=threads)
         else:
-            oracle.newton(w.cell_id, x["px"], x["a"], None, K=w.K, nthreads=threads)
+            H, _ = oracle.newton(w.cell_id, x["px"], x["a"], None, K=w.K, nthreads=threads)
+        if w.backward:
+            oracle.adjoint(w.cell_id, x["px"], x["a"], None, H, x["dLdH"], nthreads=threads)
         return time.perf_counter() - t
 
     probe = one()
     scale = max(1, int(2.0 / max(probe, 1e-3)))
-    n = min(w.B * w.D, n * scale)
-    x = prepare(workloads.host_inputs(w.with_shape(B=1, D=n), seed=w.seed))
+    n = min(n_cap, n * scale)
+    x = prepare(workloads.host_inputs(w.with_shape(B=1, D=n), seed=w.seed, with_grad=w.backward))
     for _ in range(args.warmup):
         one()
     for _ in range(args.steps):
         per_step.append(one())
     ms = 1e3 * sum(per_step) / len(per_step)
     value = n * w.T / (ms / 1e3)
-    sample = "%d of %d channels at full T=%d per step (fp64 oracle)" % (n, w.B * w.D, w.T)
+    sample = "%d of %d channels at full T=%d per step (fp64 oracle: %s)" % (
+        n, w.B * w.D, w.T, "Newton K=%d + adjoint" % w.K if w.backward else "Newton K=%d" % w.K)
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",

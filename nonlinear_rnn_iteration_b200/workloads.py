@@ -91,7 +91,7 @@ WORKLOADS = {
     ]
 }
 
-HEADLINE = "linear_8x16384x1024"
+HEADLINE = "gru_1x131072x4096_k2_bf16"
 
 
 # --------------------------------------------------------------------------

@@ -41,3 +41,24 @@ def test_help_lists_every_workload():
                          cwd=ROOT, check=True).stdout
     for name in ("linear_8x16384x1024", "gru_1x131072x4096_k2_bf16", "headgru_8x4096x512_h8_k3"):
         assert name in out
+
+
+def test_streaming_bytes_per_element():
+    # one HBM pass per Newton iteration: the first reads px and writes the
+    # state, each later one also reads the state back
+    from nonlinear_rnn_iteration_b200 import workloads
+
+    W = workloads.WORKLOADS
+    assert bench.streaming_bytes_per_elem(W["linear_8x16384x1024"], "fwd") == 12
+    assert bench.streaming_bytes_per_elem(W["gru_8x4096x2048_k3"], "fwd") == 16 + 20 + 20
+    assert bench.streaming_bytes_per_elem(W["gru_8x4096x2048_k3_bf16"], "fwd") == 10 + 14 + 14
+    assert bench.streaming_bytes_per_elem(W["lstm_4x32768x1024_k4"], "fwd") == 24 + 3 * 32
+    assert bench.streaming_bytes_per_elem(W["gru_1x131072x4096_k2_bf16"], "fwd") == 10 + 14
+    assert bench.streaming_bytes_per_elem(W["gru_1x131072x4096_k2_bf16"], "bwd") == 26
+    w = W["gru_1x131072x4096_k2_bf16"]
+    r = bench.kernel_roofline(w, "fwd", 2.0, {"hbm_gbs": 6000.0, "source": "of test"})
+    assert r["algorithmic_bytes_per_launch"] == 24 * w.elements
+    assert abs(r["achieved"] - round(24 * w.elements / 2e-3 / 1e9, 1)) < 1e-9
+    assert r["frac"] == round(r["achieved"] / 6000.0, 4)
+    assert r["fused_bytes_per_elem"] == 10
+    json.dumps(r)
