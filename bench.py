@@ -371,6 +371,19 @@ class Problem:
         if st != 0:
             raise RuntimeError("backward: %s %s" % (self.b.STATUS[st], self.b.pararnn_last_error()))
 
+    def unroll(self):
+        """The sequential recurrence on the GPU (pararnn_unroll) over the same
+        inputs, for the Newton-vs-sequential comparison."""
+        import torch
+
+        w = self.w
+        if not hasattr(self, "ws_unroll"):
+            self.ws_unroll = torch.empty(256, dtype=torch.uint8, device=self.dev)
+        st = self.b.pararnn_unroll(w.cell_id, w.B, w.T, w.D, self.code, self.px, self.a, None, self.H,
+                                   self.ws_unroll, 256, self.stream)
+        if st != 0:
+            raise RuntimeError("unroll: %s %s" % (self.b.STATUS[st], self.b.pararnn_last_error()))
+
     def step(self):
         self.forward()
         if self.w.backward:
@@ -385,8 +398,15 @@ class Problem:
             raise RuntimeError("device status %s" % self.b.STATUS[st])
 
 
-def time_device(prob, steps, warmup, dist, device, per_call=True):
-    """Returns (ms_per_step max over ranks, fwd_ms, bwd_ms) with CUDA events."""
+def time_device(prob, steps, warmup, dist, device):
+    """Returns (ms_per_step max over ranks, fwd_ms, bwd_ms) with CUDA events.
+
+    The step time is the contract's: `steps` whole steps back to back between
+    two events, bracketed by a barrier and a synchronize.  The per-kernel
+    times come from separate passes of `steps` forward calls, then `steps`
+    backward calls, back to back between two events each (no event between
+    calls, so that on a small problem the host's enqueueing of the next call
+    overlaps the device's work on the last)."""
     import torch
 
     for _ in range(warmup):
@@ -394,25 +414,43 @@ def time_device(prob, steps, warmup, dist, device, per_call=True):
     prob.check_status()
     barrier(dist, device)
     torch.cuda.synchronize(device)
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-           torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    t0.record(prob.stream)
-    for i in range(steps):
-        ev[i][0].record(prob.stream)
-        prob.forward()
-        ev[i][1].record(prob.stream)
-        if prob.w.backward:
-            prob.backward()
-        ev[i][2].record(prob.stream)
-    t1.record(prob.stream)
-    torch.cuda.synchronize(device)
+
+    def timed(fn):
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(prob.stream)
+        for _ in range(steps):
+            fn()
+        t1.record(prob.stream)
+        torch.cuda.synchronize(device)
+        return t0.elapsed_time(t1)
+
+    total = timed(prob.step)
     barrier(dist, device)
-    total = t0.elapsed_time(t1)
-    fwd = sum(a.elapsed_time(b) for a, b, _ in ev) / steps
-    bwd = sum(b.elapsed_time(c) for _, b, c in ev) / steps
+    prob.check_status()
+    fwd = timed(prob.forward) / steps
+    bwd = timed(prob.backward) / steps if prob.w.backward else 0.0
+    torch.cuda.synchronize(device)
     prob.check_status()
     return reduce_max(dist, total, device) / steps, fwd, bwd
+
+
+def time_unroll(prob, steps=3):
+    """Device time of the sequential recurrence on the GPU (CUDA events, calls
+    back to back); the forward's H buffer is reused as its output."""
+    import torch
+
+    prob.unroll()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(prob.stream)
+    for _ in range(steps):
+        prob.unroll()
+    t1.record(prob.stream)
+    torch.cuda.synchronize()
+    st = prob.b.pararnn_status_sync(prob.ws_unroll, prob.stream)
+    if st != 0:
+        raise RuntimeError("unroll device status %s" % prob.b.STATUS[st])
+    return t0.elapsed_time(t1) / steps
 
 
 def time_e2e(prob, steps):
@@ -558,11 +596,16 @@ def extra_workloads(names, device, seed_base):
     for name in names:
         w = workloads.WORKLOADS[name]
         prob = Problem(w, device, seed_base + w.seed)
-        ms, fwd, bwd = time_device(prob, steps=5, warmup=3, dist=None, device=device)
+        ms, fwd, bwd = time_device(prob, steps=20, warmup=3, dist=None, device=device)
+        in_bytes = prob.px.numel() * prob.px.element_size()
         rec = {"ms_per_step": round(ms, 4), "elem_per_s": w.elements / (ms / 1e3), "fwd_ms": round(fwd, 4),
-               "fwd": kernel_roofline(w, "fwd", fwd, peaks)}
+               "fwd": kernel_roofline(w, "fwd", fwd, peaks),
+               "l2": ("inputs larger than L2 (%.2f GB)" % (in_bytes / 1e9)) if in_bytes > 126e6 else
+                     ("inputs L2-resident (%.2f MB): a latency measurement" % (in_bytes / 1e6))}
         if w.backward:
             rec.update(bwd_ms=round(bwd, 4), bwd=kernel_roofline(w, "bwd", bwd, peaks))
+        ums = time_unroll(prob)
+        rec.update(unroll_ms=round(ums, 4), newton_fwd_speedup_vs_gpu_unroll=round(ums / fwd, 2))
         out[name] = rec
         del prob
         torch.cuda.empty_cache()
@@ -619,6 +662,12 @@ def run_native(args):
     del prob
     torch.cuda.empty_cache()
     if rank == 0 and world == 1 and not args.quick:
+        prob = Problem(w, device, rank_seed(w.seed, rank))
+        ums = time_unroll(prob)
+        line["config"]["sequential_unroll_on_gpu_ms"] = round(ums, 4)
+        line["config"]["newton_fwd_speedup_vs_gpu_unroll"] = round(ums / fwd_ms, 2)
+        del prob
+        torch.cuda.empty_cache()
         line["cpu_baseline"] = cpu_baseline(w, device, rank_seed(w.seed, rank))
         if not args.no_extra:
             line["workloads"] = extra_workloads([n for n in workloads.WORKLOADS if n != w.name], device, 0)

@@ -144,6 +144,23 @@ pararnn_status pararnn_newton_forward(pararnn_cell cell, int64_t B, int64_t T, i
                                       const float* h0, int K, float* H_out, void* workspace,
                                       size_t ws_bytes, float* resid_hist, void* stream);
 
+/* The sequential unroll of a diagonal cell on the GPU: h_t = f(h_{t-1}, x_t)
+ * for t = 0..T-1, h_{-1} = h0 -- the one-step recurrence the Newton forward
+ * reproduces at convergence (pararnn-torch page, API overview / Quickstart:
+ * sequential_apply beside newton_apply), for timing the Newton forward
+ * against the sequential recurrence on the same device.  One thread per
+ * (batch row, channel) walks the sequence; arguments and layouts as for
+ * pararnn_newton_forward (diag_w ignored by the linear cell).
+ *   workspace  >= 256 bytes of device memory (only its status word is used;
+ *              cleared on `stream`)
+ * Errors: PARARNN_EINVAL (nothing launched) for an unknown cell or dtype, bad
+ * sizes (B * D at or above 2^37), null, host or misaligned pointers, or a
+ * missing workspace; PARARNN_ECUDA if the launch fails.  A non-finite value
+ * in H_out is recorded for pararnn_status_sync(workspace, stream). */
+pararnn_status pararnn_unroll(pararnn_cell cell, int64_t B, int64_t T, int64_t D, pararnn_dtype px_dtype,
+                              const void* preacts, const float* diag_w, const float* h0, float* H_out,
+                              void* workspace, size_t ws_bytes, void* stream);
+
 /* The Newton forward with picard_iters Picard sweeps before the Newton
  * iterations (API overview, "Solver": picard_iters warms the first guess;
  * Method section: a zero-hidden start plus Picard).  From the warm start
@@ -218,13 +235,14 @@ const char* pararnn_last_error(void);
  * unknown flag.  Pure host function.
  *
  * The small-problem path: when every channel group's tiles along T fit in
- * one thread-block cluster (T up to 8 tiles: 1024 steps for the GRU, 560 for
- * the LSTM, 1024 for the linear cell), pararnn_newton_forward runs as one
- * kernel whose thread blocks pass their carries through distributed shared
- * memory; it launches nothing else (no clearing of the workspace) and
- * records its status in a word tagged with its call number, which
- * pararnn_status_sync() reads.  Its results are bit-identical to the
- * look-back path's. */
+ * one thread-block cluster (up to 16 tiles where the device allows clusters
+ * of 16, else 8) and K <= 8, pararnn_newton_forward runs as one kernel whose
+ * thread blocks pass their carries through distributed shared memory; it
+ * launches nothing else (no clearing of the workspace) and records its
+ * status in a word tagged with its call number, which pararnn_status_sync()
+ * reads.  Problems with few channel groups (B * ceil(D/32) <= 18) and
+ * T <= 1024 use tiles of 64 steps on both paths.  The small-problem path's
+ * results are bit-identical to the look-back path's. */
 #define PARARNN_HOOK_STALL_FIRST_TILE 1
 #define PARARNN_HOOK_NO_CLUSTER 2
 pararnn_status pararnn_debug_hooks(uint64_t wait_limit_ns, int flags);

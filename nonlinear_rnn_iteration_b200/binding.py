@@ -33,6 +33,7 @@ SIGNATURES = {
     "pararnn_kstar": (_I, [_I, _I64]),
     "pararnn_newton_forward": (_I, [_I, _I64, _I64, _I64, _I, _P, _P, _P, _I, _P, _P, _SZ, _P, _P]),
     "pararnn_newton_forward_picard": (_I, [_I, _I64, _I64, _I64, _I, _P, _P, _P, _I, _I, _P, _P, _SZ, _P, _P]),
+    "pararnn_unroll": (_I, [_I, _I64, _I64, _I64, _I, _P, _P, _P, _P, _P, _SZ, _P]),
     "pararnn_newton_backward": (_I, [_I, _I64, _I64, _I64, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "pararnn_status_sync": (_I, [_P, _P]),
     "pararnn_status_string": (ctypes.c_char_p, [_I]),
@@ -124,6 +125,11 @@ def pararnn_newton_forward_picard(cell, B, T, D, px_dtype, preacts, diag_w, h0, 
     return load().pararnn_newton_forward_picard(cell, B, T, D, px_dtype, _ptr(preacts), _ptr(diag_w), _ptr(h0),
                                                 picard_iters, K, _ptr(H_out), _ptr(workspace), ws_bytes,
                                                 _ptr(resid_hist), _stream(stream))
+
+
+def pararnn_unroll(cell, B, T, D, px_dtype, preacts, diag_w, h0, H_out, workspace, ws_bytes, stream):
+    return load().pararnn_unroll(cell, B, T, D, px_dtype, _ptr(preacts), _ptr(diag_w), _ptr(h0), _ptr(H_out),
+                                 _ptr(workspace), ws_bytes, _stream(stream))
 
 
 def pararnn_newton_backward(cell, B, T, D, px_dtype, preacts, diag_w, h0, H, dL_dH, dL_dpx, dL_da, dL_dh0,
@@ -258,6 +264,25 @@ def newton_forward(cell, px, diag_w=None, h0=None, K=1, out=None, workspace=None
                                       workspace.numel(), resid_hist, st), "pararnn_newton_forward")
     if sync_status:
         _check(pararnn_status_sync(workspace, st), "pararnn_newton_forward (device status)")
+    return out
+
+
+def unroll(cell, px, diag_w=None, h0=None, out=None, workspace=None, stream=None, sync_status=True):
+    """The sequential recurrence on the GPU: H (B,T,S,D) float32."""
+    import torch
+
+    cell = CELLS.get(cell, cell)
+    B, T, D = _shape(cell, px)
+    S = pararnn_state_width(cell)
+    if out is None:
+        out = torch.empty((B, T, S, D), dtype=torch.float32, device=px.device)
+    if workspace is None:
+        workspace = torch.empty(256, dtype=torch.uint8, device=px.device)
+    st = stream if stream is not None else torch.cuda.current_stream(px.device)
+    _check(pararnn_unroll(cell, B, T, D, _dtype_code(px), px, diag_w, h0, out, workspace, workspace.numel(), st),
+           "pararnn_unroll")
+    if sync_status:
+        _check(pararnn_status_sync(workspace, st), "pararnn_unroll (device status)")
     return out
 
 

@@ -175,7 +175,11 @@ __device__ __forceinline__ void store_tile_partial(const BwdSmem<Sh, PxT>& sm, i
     }
 }
 
-template <class Cell, typename PxT, class Sh>
+// kRecompute (packed path only): keep no per-row state in registers across
+// the carry barriers -- the epilogue evaluates each row's Jacobian and
+// sensitivities again from the tile still staged in shared memory -- so that
+// a thread needs far fewer registers and more warps share an SM.
+template <class Cell, typename PxT, class Sh, bool kRecompute = false>
 __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
     adjoint_bwd_kernel(const __grid_constant__ BwdMaps<Sh> maps, const BwdParams prm) {
     constexpr int G = Sh::G, S = Sh::S, V = Sh::V, R = Sh::R, NS = Cell::NSENS, NW = Sh::NWARPS;
@@ -309,6 +313,38 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
                 for (int q = 0; q < VP; ++q) wp[q] = Cell::weights2(wr[2 * q], wr[2 * q + 1]);
             }
 
+            // the linearisation of row r at (h_{t-1}, x_t) for channel pair q,
+            // from the staged tile: A, the sensitivities and g_t (the identity
+            // element and g = 0 past the end of the sequence)
+            auto lin2 = [&](int r, int q, f2 (&A)[S * S], f2 (&se)[NS], f2 (&gv)[S]) {
+              if constexpr (kPack) {
+                const int row = sub * R + r;
+                const bool rvalid = (tb + r < T) && cvalid;
+                const int c0 = cc + 2 * q;
+                f2 pg[G], spv[S];
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    float pv2[2];
+                    lds_row<2>(&sm.stg[st].px[row][g][c0], pv2);
+                    pg[g] = f2{pv2[0], pv2[1]};
+                }
+#pragma unroll
+                for (int s = 0; s < S; ++s) {
+                    float hv2[2], gv2[2];
+                    lds_row<2>((t0 == 0 && row == 0) ? &sm.hprev[s][c0] : &sm.stg[st].H[row][s][c0], hv2);
+                    lds_row<2>(&sm.stg[st].g[row][s][c0], gv2);
+                    spv[s] = f2{hv2[0], hv2[1]};
+                    gv[s] = rvalid ? f2{gv2[0], gv2[1]} : splat2(0.0f);
+                }
+                Cell::bwd2(pg, wp[q], spv, A, se);
+                if (!rvalid) {
+#pragma unroll
+                    for (int a = 0; a < S * S; ++a) A[a] = splat2((a % (S + 1) == 0) ? 1.0f : 0.0f);
+                }
+              }
+            };
+            (void)lin2;
+
             // ---- linearisation at (h_{t-1}, x_t) and the sub-chunk's element,
             //      composed in scan order (latest row first) ----
             float jA[R][S * S][V], sens[R][NS][V], gr[R][S][V];
@@ -320,13 +356,43 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
                 const int row = sub * R + r;
                 const bool rvalid = (tb + r < T) && cvalid;
                 float pv[G][V], hv[S][V];
+                if constexpr (!(kPack && kRecompute)) {
 #pragma unroll
-                for (int g = 0; g < G; ++g) lds_row<V>(&sm.stg[st].px[row][g][cc], pv[g]);
+                    for (int g = 0; g < G; ++g) lds_row<V>(&sm.stg[st].px[row][g][cc], pv[g]);
 #pragma unroll
-                for (int s = 0; s < S; ++s) lds_row<V>((t0 == 0 && row == 0) ? &sm.hprev[s][cc] : &sm.stg[st].H[row][s][cc], hv[s]);
+                    for (int s = 0; s < S; ++s)
+                        lds_row<V>((t0 == 0 && row == 0) ? &sm.hprev[s][cc] : &sm.stg[st].H[row][s][cc], hv[s]);
 #pragma unroll
-                for (int s = 0; s < S; ++s) lds_row<V>(&sm.stg[st].g[row][s][cc], gr[r][s]);
-                if constexpr (kPack) {
+                    for (int s = 0; s < S; ++s) lds_row<V>(&sm.stg[st].g[row][s][cc], gr[r][s]);
+                }
+                if constexpr (kPack && kRecompute) {
+#pragma unroll
+                    for (int q = 0; q < VP; ++q) {
+                        const int v0 = 2 * q, v1 = 2 * q + 1;
+                        f2 A[S * S], se[NS], gv[S], M[S * S], bv[S], accA[S * S], accb[S];
+                        lin2(r, q, A, se, gv);
+#pragma unroll
+                        for (int i = 0; i < S; ++i)
+#pragma unroll
+                            for (int m = 0; m < S; ++m) M[i * S + m] = A[m * S + i];  // A^T
+                        mat_t_vec2<S>(A, gv, bv);
+#pragma unroll
+                        for (int a = 0; a < S * S; ++a) accA[a] = f2{mine.e[v0].A[a], mine.e[v1].A[a]};
+#pragma unroll
+                        for (int s = 0; s < S; ++s) accb[s] = f2{mine.e[v0].b[s], mine.e[v1].b[s]};
+                        compose_after2<S>(M, bv, accA, accb);
+#pragma unroll
+                        for (int a = 0; a < S * S; ++a) {
+                            mine.e[v0].A[a] = accA[a].x;
+                            mine.e[v1].A[a] = accA[a].y;
+                        }
+#pragma unroll
+                        for (int s = 0; s < S; ++s) {
+                            mine.e[v0].b[s] = accb[s].x;
+                            mine.e[v1].b[s] = accb[s].y;
+                        }
+                    }
+                } else if constexpr (kPack) {
 #pragma unroll
                     for (int q = 0; q < VP; ++q) {
                         const int v0 = 2 * q, v1 = 2 * q + 1;
@@ -425,7 +491,62 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
                 for (int v = 0; v < V; ++v) da_acc[g][v] = 0.0f;
             float outp[R][G][V];
             bool bad = false;
-            if constexpr (kPack) {
+            if constexpr (kPack && kRecompute) {
+#pragma unroll
+                for (int q = 0; q < VP; ++q) {
+                    const int v0 = 2 * q, v1 = 2 * q + 1;
+                    f2 x[S], cv[S], PA[S * S], Pb[S], dacc[G];  // x = mu_{t+1}
+#pragma unroll
+                    for (int s = 0; s < S; ++s) cv[s] = f2{sm.cin[s][cc + v0], sm.cin[s][cc + v1]};
+#pragma unroll
+                    for (int a = 0; a < S * S; ++a) PA[a] = f2{pre.e[v0].A[a], pre.e[v1].A[a]};
+#pragma unroll
+                    for (int s = 0; s < S; ++s) Pb[s] = f2{pre.e[v0].b[s], pre.e[v1].b[s]};
+                    apply2<S>(PA, Pb, cv, x);
+#pragma unroll
+                    for (int g = 0; g < G; ++g) dacc[g] = splat2(0.0f);
+#pragma unroll
+                    for (int r = R - 1; r >= 0; --r) {
+                        const int64_t t = tb + r;
+                        const bool rvalid = (t < T) && cvalid;
+                        f2 lam[S], A[S * S], se[NS], gv[S], dp[G], da[G];
+                        lin2(r, q, A, se, gv);
+#pragma unroll
+                        for (int s = 0; s < S; ++s) lam[s] = add2(gv[s], x[s]);
+                        mat_t_vec2<S>(A, lam, x);  // mu_t
+                        Cell::grads2(se, lam, dp, da);
+                        if (rvalid) {
+                            float o0[G], o1[G];
+#pragma unroll
+                            for (int g2 = 0; g2 < G; ++g2) {
+                                dacc[g2] = add2(dacc[g2], da[g2]);
+                                bad |= !isfinite(dp[g2].x) || !isfinite(dp[g2].y);
+                                o0[g2] = dp[g2].x;
+                                o1[g2] = dp[g2].y;
+                            }
+#pragma unroll
+                            for (int g2 = 0; g2 < G; ++g2) {
+                                float o2[2] = {o0[g2], o1[g2]};
+                                store_out_row<2, BwdStreamHints<Cell>::value>(
+                                    prm.dLdpx + ((b * T + t) * G + g2) * D + d0 + cc + v0, o2);
+                            }
+                        }
+                        if (r == 0 && tb == 0 && rvalid && prm.dLdh0) {
+                            // dL/dh0 = A_0^T lambda_0 = mu_0
+#pragma unroll
+                            for (int s = 0; s < S; ++s) {
+                                prm.dLdh0[(b * S + s) * D + d0 + cc + v0] = x[s].x;
+                                prm.dLdh0[(b * S + s) * D + d0 + cc + v1] = x[s].y;
+                            }
+                        }
+                    }
+#pragma unroll
+                    for (int g = 0; g < G; ++g) {
+                        da_acc[g][v0] = dacc[g].x;
+                        da_acc[g][v1] = dacc[g].y;
+                    }
+                }
+            } else if constexpr (kPack) {
 #pragma unroll
                 for (int q = 0; q < VP; ++q) {
                     const int v0 = 2 * q, v1 = 2 * q + 1;
@@ -514,14 +635,16 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
                     }
                 }
             }
+            if constexpr (!(kPack && kRecompute)) {
 #pragma unroll
-            for (int r = 0; r < R; ++r) {
-                const int64_t t = tb + r;
-                if (t < T && cvalid) {
+                for (int r = 0; r < R; ++r) {
+                    const int64_t t = tb + r;
+                    if (t < T && cvalid) {
 #pragma unroll
-                    for (int g = 0; g < G; ++g)
-                        store_out_row<V, BwdStreamHints<Cell>::value>(prm.dLdpx + ((b * T + t) * G + g) * D + d0 + cc,
-                                                                      outp[r][g]);
+                        for (int g = 0; g < G; ++g)
+                            store_out_row<V, BwdStreamHints<Cell>::value>(
+                                prm.dLdpx + ((b * T + t) * G + g) * D + d0 + cc, outp[r][g]);
+                    }
                 }
             }
             if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(prm.lb.status, kStatusNonFinite);

@@ -95,6 +95,10 @@ struct CellGRU {
     static __device__ __forceinline__ W2 weights2(const float (&wa)[G], const float (&wb)[G]) {
         return W2{f2{wa[0], wb[0]}, f2{wa[1], wb[1]}, f2{wa[2], wb[2]}, f2{-wa[2], -wb[2]}};
     }
+    // warm() on a pair of channels
+    static __device__ __forceinline__ void warm2(const f2 (&p)[G], f2 (&f)[S]) {
+        f[0] = mul2(sigmoid2(p[0]), tanh2(p[2]));
+    }
     // elem() on a pair of channels.  No packed negation exists, so the gates
     // are formed negated, nz = -z and nr = -r (neg_sigmoid2), and every sign
     // is carried by the algebra:
@@ -241,6 +245,14 @@ struct CellLSTM {
     };
     static __device__ __forceinline__ W2 weights2(const float (&wa)[G], const float (&wb)[G]) {
         return W2{f2{wa[0], wb[0]}, f2{wa[1], wb[1]}, f2{wa[2], wb[2]}, f2{wa[3], wb[3]}, f2{-wa[3], -wb[3]}};
+    }
+    // warm() on a pair of channels
+    static __device__ __forceinline__ void warm2(const f2 (&p)[G], f2 (&f)[S]) {
+        const f2 i = sigmoid2(p[0]);
+        const f2 o = sigmoid2(p[2]);
+        const f2 cn = mul2(i, tanh2(p[3]));
+        f[0] = cn;
+        f[1] = mul2(o, tanh2(cn));
     }
     // elem() on a pair of channels; sp = (c, h), A row-major (2 x 2)
     static __device__ __forceinline__ void elem2(const f2 (&p)[G], const W2& w, const f2 (&sp)[S], f2 (&f)[S],

@@ -22,6 +22,10 @@
 #include "pararnn_b200.h"
 
 namespace pararnn {
+pararnn_status newton_forward_slice(int64_t B_whole, int64_t D_whole, pararnn_cell cell, int64_t B, int64_t T,
+                                    int64_t D, pararnn_dtype px_dtype, const void* preacts, const float* diag_w,
+                                    const float* h0, int K, float* H_out, void* workspace, size_t ws_bytes,
+                                    void* stream);  // pararnn_abi.cu
 void set_last_error(const char* msg);   // pararnn_abi.cu
 bool pointer_on_device(const void* p);  // pararnn_abi.cu
 
@@ -192,8 +196,8 @@ extern "C" pararnn_status pararnn_newton_forward_host(pararnn_cell cell, int64_t
         if (e != cudaSuccess) break;
         const float* w_use = split ? (diag_w ? w_dev : nullptr) : diag_w;
         const float* h0_use = split ? (h0 ? h0_dev : nullptr) : (h0 ? h0 + (size_t)b0 * S * D : nullptr);
-        st = pararnn_newton_forward(cell, nb, T, dn, px_dtype, px_dev, w_use, h0_use, K, h_dev, fw, l.fw_bytes,
-                                    nullptr, scomp);
+        st = newton_forward_slice(B, D, cell, nb, T, dn, px_dtype, px_dev, w_use, h0_use, K, h_dev, fw, l.fw_bytes,
+                                  scomp);
         if (st != PARARNN_OK) break;
         hp::fold_status<<<1, 32, 0, scomp>>>(reinterpret_cast<unsigned*>(ws), reinterpret_cast<unsigned*>(fw));
         e = cudaGetLastError();

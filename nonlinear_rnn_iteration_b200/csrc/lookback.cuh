@@ -329,14 +329,35 @@ __device__ __forceinline__ void sub_prefix(const ElemV<S, V>& excl, int warp, in
     for (int v = 0; v < V; ++v) {
         Elem<S> acc;
         elem_identity<S>(acc);
-        for (int k = 0; k < ws; ++k) {
-            const int wk = kReverse ? (NW - 1 - k) : k;
-            float A[S * S], b[S];
+        // the same compositions in the same order either way.  A scalar state
+        // unrolls over the block's warps with the position test inside, so
+        // that the shared-memory loads can all be issued before the chain of
+        // compositions (measured 2-5 % faster); a 2 x 2 state keeps the loop,
+        // whose six words per warp would otherwise cost registers (measured
+        // 3-4 % slower unrolled)
+        if constexpr (S == 1) {
 #pragma unroll
-            for (int a = 0; a < S * S; ++a) A[a] = wagg[wk][a][cc + v];
+            for (int k = 0; k < NW; ++k) {
+                if (k < ws) {
+                    const int wk = kReverse ? (NW - 1 - k) : k;
+                    float A[S * S], b[S];
 #pragma unroll
-            for (int s = 0; s < S; ++s) b[s] = wagg[wk][S * S + s][cc + v];
-            compose_after<S>(A, b, acc);
+                    for (int a = 0; a < S * S; ++a) A[a] = wagg[wk][a][cc + v];
+#pragma unroll
+                    for (int s = 0; s < S; ++s) b[s] = wagg[wk][S * S + s][cc + v];
+                    compose_after<S>(A, b, acc);
+                }
+            }
+        } else {
+            for (int k = 0; k < ws; ++k) {
+                const int wk = kReverse ? (NW - 1 - k) : k;
+                float A[S * S], b[S];
+#pragma unroll
+                for (int a = 0; a < S * S; ++a) A[a] = wagg[wk][a][cc + v];
+#pragma unroll
+                for (int s = 0; s < S; ++s) b[s] = wagg[wk][S * S + s][cc + v];
+                compose_after<S>(A, b, acc);
+            }
         }
         compose_elem<S>(excl.e[v], acc);
         pre.e[v] = acc;

@@ -93,6 +93,12 @@ struct FwdShape {
     static_assert(W <= 256 && L + 1 <= 256 && G <= 256, "TMA box dimensions are at most 256");
 };
 
+// the largest cluster the small-problem path launches (16 needs the
+// non-portable cluster-size attribute), and the most Newton iterations it
+// runs (each iteration has its own element buffer and mbarrier)
+constexpr int kMaxClusterRanks = 16;
+constexpr int kMaxClusterK = 8;
+
 // One TMA destination: a tensor copy writes to a 128-byte aligned shared
 // address, so every stage is padded to a multiple of 128 bytes.
 template <class Sh, typename PxT>
@@ -107,24 +113,30 @@ struct FwdSmem {
     float wagg[Sh::NWARPS][Sh::NA][Sh::W];  // each compute warp's composed element
     float cin[Sh::S][Sh::W];                // the state just before the tile (current iterate)
     float w[Sh::G][Sh::W];                  // the tile's recurrent weights
-    float cagg[2][Sh::NA][Sh::W];           // cluster path: this tile's element, iterations in turn
+    float cagg[kMaxClusterK][Sh::NA][Sh::W];  // cluster path: this tile's element, per iteration
+    uint64_t cbar[kMaxClusterK];              // cluster path: the predecessors' elements are ready
     uint64_t bar[Sh::NSTAGE];
     unsigned ticket[Sh::NSTAGE];
 };
 
 // The cluster path's carry for one Newton iteration (scan warp, between the
-// "warp totals" and "carry" block barriers; the compute warps take the same
-// cluster barrier meanwhile).  The tiles of one channel group along T are the
-// CTAs of one cluster, rank = position along T.  Each composes its warp
-// totals into its tile's element, and after the cluster barrier reads the
-// elements of the tiles before it from their shared memory and applies them,
-// in order, to the first carry: the same sequence of operations as the
-// look-back's inclusive states, so the carry has the same bits.
+// "warp totals" and "carry" block barriers).  The tiles of one channel group
+// along T are the CTAs of one cluster, rank = position along T.  Each
+// composes its warp totals into its tile's element (this iteration's own
+// buffer), makes it visible at cluster scope and arrives on this
+// iteration's mbarrier in every later tile's CTA; it then waits (bounded)
+// until the tiles before it have all arrived on its own, reads their
+// elements from their shared memory and applies them, in order, to the
+// first carry: the same operations, in the same order, as the look-back's
+// chain of inclusive states, so the carry has the same bits.  Only scan
+// warps take part: the compute warps never wait on another CTA.  Returns
+// false if the wait ran out of time (the carry is then not valid).
 template <class Sh>
-__device__ __forceinline__ void cluster_carry(const float (&wagg)[Sh::NWARPS][Sh::NA][Sh::W],
-                                              float (&cagg)[Sh::NA][Sh::W],
+__device__ __forceinline__ bool cluster_carry(const float (&wagg)[Sh::NWARPS][Sh::NA][Sh::W],
+                                              float (&cagg)[Sh::NA][Sh::W], uint64_t* cbar,
                                               const float (&first_carry)[Sh::W / 32][Sh::S], uint32_t rank,
-                                              int lane, float (&cin)[Sh::S][Sh::W]) {
+                                              uint32_t nranks, int lane, float (&cin)[Sh::S][Sh::W],
+                                              uint64_t timeout_ns) {
     constexpr int S = Sh::S, NA = Sh::NA, W = Sh::W, CPL = W / 32;
 #pragma unroll
     for (int j = 0; j < CPL; ++j) {
@@ -144,27 +156,57 @@ __device__ __forceinline__ void cluster_carry(const float (&wagg)[Sh::NWARPS][Sh
 #pragma unroll
         for (int s = 0; s < S; ++s) cagg[S * S + s][lane + 32 * j] = tot.b[s];
     }
+    // every lane's element words ordered before any lane's arrive
+    fence_acq_rel_cluster();
     __syncwarp();
-    cluster_arrive_release();
-    cluster_wait_acquire();
+    for (uint32_t r = rank + 1 + lane; r < nranks; r += 32) mbar_arrive_remote(cbar, r);
+    bool ok = true;
+    if (rank > 0) {
+        Deadline dl;
+        while (!mbar_try_wait_cluster(cbar, 0)) {
+            if (dl.expired(timeout_ns)) {
+                ok = false;
+                break;
+            }
+        }
+    }
+    // the predecessors' elements are loaded in batches (every remote load of
+    // a batch in flight at once: all of them for a scalar state, whose
+    // elements are two words), then applied in order
+    constexpr int NB = S == 1 ? kMaxClusterRanks : 4;
+    static_assert(kMaxClusterRanks % NB == 0, "whole batches of cluster ranks");
 #pragma unroll
     for (int j = 0; j < CPL; ++j) {
         float x[S];
 #pragma unroll
         for (int s = 0; s < S; ++s) x[s] = first_carry[j][s];
-        for (uint32_t i = 0; i < rank; ++i) {
-            float A[S * S], b[S], y[S];
 #pragma unroll
-            for (int a = 0; a < S * S; ++a) A[a] = ld_dsmem(&cagg[a][lane + 32 * j], i);
+        for (uint32_t i0 = 0; i0 < (uint32_t)kMaxClusterRanks; i0 += NB) {
+            if (i0 >= rank) break;
+            float e[NB][NA];
 #pragma unroll
-            for (int s = 0; s < S; ++s) b[s] = ld_dsmem(&cagg[S * S + s][lane + 32 * j], i);
-            apply<S>(A, b, x, y);
+            for (int m = 0; m < NB; ++m)
+                if (i0 + m < rank) {
 #pragma unroll
-            for (int s = 0; s < S; ++s) x[s] = y[s];
+                    for (int a = 0; a < NA; ++a) e[m][a] = ld_dsmem(&cagg[a][lane + 32 * j], i0 + m);
+                }
+#pragma unroll
+            for (int m = 0; m < NB; ++m)
+                if (i0 + m < rank) {
+                    float A[S * S], b[S], y[S];
+#pragma unroll
+                    for (int a = 0; a < S * S; ++a) A[a] = e[m][a];
+#pragma unroll
+                    for (int s = 0; s < S; ++s) b[s] = e[m][S * S + s];
+                    apply<S>(A, b, x, y);
+#pragma unroll
+                    for (int s = 0; s < S; ++s) x[s] = y[s];
+                }
         }
 #pragma unroll
         for (int s = 0; s < S; ++s) cin[s][lane + 32 * j] = x[s];
     }
+    return ok;
 }
 
 template <class Cell, typename PxT, class Sh>
@@ -223,6 +265,14 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
             for (int s = 1; s < NSTAGE; ++s) sm.ticket[s] = (unsigned)prm.nTiles;
             if constexpr (Sh::kTma) issue_tile_load<Cell, PxT, Sh>(&tmap, sm, prm, t, 0);
             if (blockIdx.x == 0) *prm.status_epoch = prm.lb.epoch;  // the flags of this call are the valid ones
+            // one mbarrier per Newton iteration, completed by the arrivals of
+            // every tile before this one (none for the first)
+            const uint32_t rank = cluster_ctarank();
+            if (rank > 0) {
+                const int nk = kLean ? 1 : prm.K;
+                for (int k = 0; k < nk; ++k) mbar_init(&sm.cbar[k], rank);
+            }
+            asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         } else {
 #pragma unroll
             for (int s = 0; s < NSTAGE - 1; ++s) {
@@ -234,6 +284,11 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
         }
     }
     block_sync();
+    if constexpr (kCluster) {
+        // every CTA's mbarriers are initialised before any CTA arrives on them
+        cluster_arrive_release();
+        cluster_wait_acquire();
+    }
 
     for (int it = 0;; ++it) {
         const int st = it % NSTAGE;
@@ -283,7 +338,9 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
                 const int K = kLean ? 1 : prm.K;
                 for (int k = 0; k < K; ++k) {
                     block_sync();  // warp totals ready
-                    cluster_carry<Sh>(sm.wagg, sm.cagg[k & 1], first_carry, (uint32_t)chunk, lane, sm.cin);
+                    const bool ok = cluster_carry<Sh>(sm.wagg, sm.cagg[k], &sm.cbar[k], first_carry, (uint32_t)chunk,
+                                                      (uint32_t)prm.nChunks, lane, sm.cin, prm.lb.timeout_ns);
+                    if (!__all_sync(0xffffffffu, ok) && lane == 0) report(kStatusTimeout);
                     block_sync();  // carry ready
                 }
             } else if constexpr (kLean) {
@@ -354,9 +411,7 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
                 }
                 warp_prefix<S, V, LC, W, NW, false>(mine, excl, warp, lane, sm.wagg);
                 block_sync();  // warp totals ready
-                if constexpr (kCluster) cluster_arrive_release();
                 sub_prefix<S, V, LC, W, NW, false>(excl, warp, lane, sm.wagg, pre);
-                if constexpr (kCluster) cluster_wait_acquire();
                 block_sync();  // carry ready
                 float x[V];
 #pragma unroll
@@ -387,12 +442,26 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
                 for (int v = 0; v < V; ++v)
 #pragma unroll
                     for (int g = 0; g < G; ++g) wr[v][g] = sm.w[g][cc + v];
-                float h[R][S][V];
-                if constexpr (!kPicard) {
+                // two channels per instruction where the thread holds an even
+                // number of them (packed f32x2; same rounding as one by one)
+                constexpr bool kPack = (V % 2 == 0) && Cell::kNonlinear;
+                constexpr int VP = kPack ? V / 2 : 1;
+                // f(0, x) for V channels of one row, pairwise where packed
+                auto warm_row = [&](const float (&pv)[G][V], float (&out)[S][V]) {
+                    if constexpr (kPack) {
 #pragma unroll
-                    for (int r = 0; r < R; ++r) {
-                        float pv[G][V];
-                        load_p(r, pv);
+                        for (int q = 0; q < VP; ++q) {
+                            f2 pg[G], f[S];
+#pragma unroll
+                            for (int g = 0; g < G; ++g) pg[g] = f2{pv[g][2 * q], pv[g][2 * q + 1]};
+                            Cell::warm2(pg, f);
+#pragma unroll
+                            for (int s = 0; s < S; ++s) {
+                                out[s][2 * q] = f[s].x;
+                                out[s][2 * q + 1] = f[s].y;
+                            }
+                        }
+                    } else {
 #pragma unroll
                         for (int v = 0; v < V; ++v) {
                             float pg[G], f[S];
@@ -400,8 +469,17 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
                             for (int g = 0; g < G; ++g) pg[g] = pv[g][v];
                             Cell::warm(pg, wr[v], f);
 #pragma unroll
-                            for (int s = 0; s < S; ++s) h[r][s][v] = f[s];
+                            for (int s = 0; s < S; ++s) out[s][v] = f[s];
                         }
+                    }
+                };
+                float h[R][S][V];
+                if constexpr (!kPicard) {
+#pragma unroll
+                    for (int r = 0; r < R; ++r) {
+                        float pv[G][V];
+                        load_p(r, pv);
+                        warm_row(pv, h[r]);
                     }
                 }
                 // h^(0) just before the sub-chunk: h0 at the start of a row,
@@ -514,22 +592,10 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
                                 for (int v = 0; v < V; ++v)
                                     pv[g][v] = PxTraits<PxT>::cvt(pxg[((b * T + tb - 1) * G + g) * D + d0 + cc + v]);
                         }
-#pragma unroll
-                        for (int v = 0; v < V; ++v) {
-                            float pg[G], f[S];
-#pragma unroll
-                            for (int g = 0; g < G; ++g) pg[g] = pv[g][v];
-                            Cell::warm(pg, wr[v], f);
-#pragma unroll
-                            for (int s = 0; s < S; ++s) hin[s][v] = f[s];
-                        }
+                        warm_row(pv, hin);
                     }
                 }
                 const int K = prm.K;
-                // two channels per instruction where the thread holds an even
-                // number of them (packed f32x2; same rounding as one by one)
-                constexpr bool kPack = (V % 2 == 0) && Cell::kNonlinear;
-                constexpr int VP = kPack ? V / 2 : 1;
                 typename Cell::W2 wp[VP];
                 if constexpr (kPack) {
 #pragma unroll
@@ -662,11 +728,9 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
                     }
                     warp_prefix<S, V, LC, W, NW, false>(mine, excl, warp, lane, sm.wagg);
                     block_sync();  // warp totals ready
-                    if constexpr (kCluster) cluster_arrive_release();
-                    // ---- 2. prefix of the earlier warps (the scan warp finds the carry meanwhile) ----
+                        // ---- 2. prefix of the earlier warps (the scan warp finds the carry meanwhile) ----
                     sub_prefix<S, V, LC, W, NW, false>(excl, warp, lane, sm.wagg, pre);
-                    if constexpr (kCluster) cluster_wait_acquire();
-                    block_sync();  // carry ready
+                        block_sync();  // carry ready
                     // ---- 3. re-walk the rows from the carry-in: h^(k+1) ----
                     if constexpr (kPack) {
 #pragma unroll

@@ -55,6 +55,23 @@ template <typename PxT> using FwdLstmS = FwdShape<CellLSTM, PxT, 1, 32, 7, 4, 2,
 template <typename PxT> using BwdLinS = FwdShape<CellLinear, PxT, 1, 32, 7, 4, 2, 2, false>;
 template <typename PxT> using BwdGruS = FwdShape<CellGRU, PxT, 1, 32, 7, 4, 2, 2, false>;
 template <typename PxT> using BwdLstmS = FwdShape<CellLSTM, PxT, 1, 32, 7, 2, 2, 2, false>;
+// Small problems (few channel groups, T of at most 16 tiles of 64 steps):
+// tiles of 64 steps, so that twice as many thread blocks share the work of
+// each Newton iteration and a channel group's tiles still fit one cluster.
+// The choice depends on the sizes only (small_problem), so the cluster path
+// and the look-back path of the same call use the same tiles.
+template <typename PxT> using FwdLinQ = FwdShape<CellLinear, PxT, 4, 8, 4, 4, 1, 2, true>;
+template <typename PxT> using FwdGruQ = FwdShape<CellGRU, PxT, 4, 8, 8, 2, 1, 2, true>;
+template <typename PxT> using FwdLstmQ = FwdShape<CellLSTM, PxT, 2, 16, 8, 4, 1, 2, true>;
+constexpr int kSmallL = 64;        // steps per tile of the small-problem shapes
+constexpr int kSmallMaxTiles = 16;  // along T
+constexpr int64_t kSmallMaxGroups = 18;
+
+// the adjoint's epilogue-recompute mode (adjoint_bwd_kernel), by cell
+template <class Cell>
+struct BwdRecompute {
+    static constexpr bool value = false;
+};
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far beyond any legitimate wait
 constexpr uint64_t kMaxWaitLimitNs = 10000000000ull;
@@ -121,9 +138,20 @@ Geometry geom_of(int nSlots) {
     return g;
 }
 
+// A forward of few channel groups (B * ceil(D/32)) over at most 16 tiles of
+// 64 steps takes the small-problem tiles.
+bool small_problem(int64_t B, int64_t T, int64_t D) {
+    return T > 0 && (T + kSmallL - 1) / kSmallL <= kSmallMaxTiles && B * ((D + 31) / 32) <= kSmallMaxGroups;
+}
+
 // The tile geometry does not depend on the pre-activation dtype.
-Geometry geometry(pararnn_cell cell, bool fwd, bool tma, int K) {
+Geometry geometry(pararnn_cell cell, bool fwd, bool tma, int K, bool small = false) {
     const int ns = fwd ? (cell == PARARNN_CELL_LINEAR ? 1 : K) : 1;
+    if (fwd && tma && small) {
+        if (cell == PARARNN_CELL_LINEAR) return geom_of<FwdLinQ<float>>(ns);
+        if (cell == PARARNN_CELL_DIAG_GRU) return geom_of<FwdGruQ<float>>(ns);
+        return geom_of<FwdLstmQ<float>>(ns);
+    }
     if (cell == PARARNN_CELL_LINEAR) {
         if (fwd) return tma ? geom_of<FwdLinT<float>>(ns) : geom_of<FwdLinS<float>>(ns);
         return tma ? geom_of<BwdLinT<float>>(ns) : geom_of<BwdLinS<float>>(ns);
@@ -144,9 +172,9 @@ struct Plan {
     Geometry g;
 };
 
-Plan make_plan(pararnn_cell cell, int64_t B, int64_t T, int64_t D, int K, bool fwd, bool tma) {
+Plan make_plan(pararnn_cell cell, int64_t B, int64_t T, int64_t D, int K, bool fwd, bool tma, bool small = false) {
     Plan p;
-    p.g = geometry(cell, fwd, tma, K);
+    p.g = geometry(cell, fwd, tma, K, small);
     p.nCG = (D + p.g.W - 1) / p.g.W;
     p.nChunks = (T + p.g.L - 1) / p.g.L;
     p.nGroups = B * p.nCG;
@@ -303,11 +331,15 @@ pararnn_status persistent_grid(Kern kern, int threads, size_t smem, int64_t nTil
 // (at most kMaxClusterTiles along T), so the forward runs as clusters whose
 // CTAs pass carries through distributed shared memory -- one kernel launch,
 // no workspace clearing, no look-back (newton_fwd_kernel's kCluster mode).
-constexpr int kMaxClusterTiles = 8;
+constexpr int kMaxClusterTiles = kMaxClusterRanks;  // above 8 where the device allows a non-portable size
 
 template <class Kern>
 bool cluster_fits_query(Kern kern, int threads, size_t smem, int csize) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    if (csize > 8 && cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
         cudaGetLastError();
         return false;
     }
@@ -389,7 +421,7 @@ pararnn_status launch_fwd(const Plan& pl, FwdParams prm, cudaStream_t st, void* 
         pararnn_status s = make_map(&map, prm.px, sizeof(PxT) == 2, prm.D, Sh::G, prm.B * prm.T, Sh::W, Sh::LF);
         if (s != PARARNN_OK) return s;
     }
-    if (allow_cluster && pl.nChunks <= kMaxClusterTiles) {
+    if (allow_cluster && pl.nChunks <= kMaxClusterTiles && prm.K <= kMaxClusterK) {
         bool done = false;
         pararnn_status s = PARARNN_OK;
         if constexpr (!Cell::kNonlinear) {
@@ -450,7 +482,7 @@ pararnn_status launch_bwd(const Plan& pl, BwdParams prm, float* dLda, cudaStream
         if (s != PARARNN_OK) return s;
     }
     const size_t smem = sizeof(BwdSmem<Sh, PxT>);
-    auto kern = adjoint_bwd_kernel<Cell, PxT, Sh>;
+    auto kern = adjoint_bwd_kernel<Cell, PxT, Sh, BwdRecompute<Cell>::value>;
     unsigned grid = 0;
     pararnn_status s = persistent_grid(kern, Sh::NT, smem, pl.nTiles, grid, "adjoint_bwd");
     if (s != PARARNN_OK) return s;
@@ -497,6 +529,26 @@ void set_last_error(const char* msg) { fail(PARARNN_OK, "%s", msg); }
 bool pointer_on_device(const void* p) { return device_reachable(p); }
 }  // namespace pararnn
 
+namespace {
+pararnn_status forward_impl(pararnn_cell cell, int64_t B, int64_t T, int64_t D, pararnn_dtype px_dtype,
+                            const void* preacts, const float* diag_w, const float* h0, int picard, int K,
+                            float* H_out, void* workspace, size_t ws_bytes, float* resid_hist, void* stream,
+                            int small_hint);
+}  // namespace
+
+namespace pararnn {
+// pararnn_newton_forward on a slice (rows and/or channels) of a B_whole x T x
+// D_whole problem, tiled as the whole problem would be, so that the slice's
+// values are bit-identical to the whole problem's (host_path.cu)
+pararnn_status newton_forward_slice(int64_t B_whole, int64_t D_whole, pararnn_cell cell, int64_t B, int64_t T,
+                                    int64_t D, pararnn_dtype px_dtype, const void* preacts, const float* diag_w,
+                                    const float* h0, int K, float* H_out, void* workspace, size_t ws_bytes,
+                                    void* stream) {
+    return forward_impl(cell, B, T, D, px_dtype, preacts, diag_w, h0, 0, K, H_out, workspace, ws_bytes, nullptr,
+                        stream, small_problem(B_whole, T, D_whole) ? 1 : 0);
+}
+}  // namespace pararnn
+
 extern "C" {
 
 int pararnn_num_gates(pararnn_cell cell) {
@@ -523,6 +575,10 @@ size_t pararnn_workspace_bytes(pararnn_cell cell, int64_t B, int64_t T, int64_t 
             const Plan p = make_plan(cell, B, T, D, K, fwd != 0, tma != 0);
             if (p.total > m) m = p.total;
         }
+    if (small_problem(B, T, D)) {
+        const Plan p = make_plan(cell, B, T, D, K, true, true, true);
+        if (p.total > m) m = p.total;
+    }
     return m;
 }
 
@@ -530,9 +586,13 @@ size_t pararnn_workspace_bytes(pararnn_cell cell, int64_t B, int64_t T, int64_t 
 
 namespace {
 
+// small_hint: -1 chooses the tiles from (B, T, D); 0 or 1 is the choice made
+// for a larger problem this call is a slice of (the host-buffer path), so
+// that every slice is tiled as the whole problem would be
 pararnn_status forward_impl(pararnn_cell cell, int64_t B, int64_t T, int64_t D, pararnn_dtype px_dtype,
                             const void* preacts, const float* diag_w, const float* h0, int picard, int K,
-                            float* H_out, void* workspace, size_t ws_bytes, float* resid_hist, void* stream) {
+                            float* H_out, void* workspace, size_t ws_bytes, float* resid_hist, void* stream,
+                            int small_hint = -1) {
     g_last_error[0] = 0;
     pararnn_status st = check_sizes(cell, B, T, D);
     if (st != PARARNN_OK) return st;
@@ -564,7 +624,8 @@ pararnn_status forward_impl(pararnn_cell cell, int64_t B, int64_t T, int64_t D, 
     // TMA staging needs 16-byte rows of pre-activations and 16-byte stores of H
     const bool tma = ((D * (int64_t)esz) % 16 == 0) && aligned(preacts, 16) && aligned(H_out, 16);
     const int Keff = cell == PARARNN_CELL_LINEAR ? 1 : K;
-    const Plan pl = make_plan(cell, B, T, D, Keff, true, tma);
+    const bool small = tma && (small_hint < 0 ? small_problem(B, T, D) : small_hint != 0);
+    const Plan pl = make_plan(cell, B, T, D, Keff, true, tma, small);
     if (pl.nTiles >= (int64_t(1) << 31)) return fail(PARARNN_EINVAL, "too many tiles");
 
     char* ws = static_cast<char*>(workspace);
@@ -614,9 +675,14 @@ pararnn_status forward_impl(pararnn_cell cell, int64_t B, int64_t T, int64_t D, 
 #define PARARNN_FWD(C, SH) \
     (bf ? launch_fwd<C, bf16, SH<bf16>>(pl, prm, s, ws, clear_bytes, allow_cluster) \
         : launch_fwd<C, float, SH<float>>(pl, prm, s, ws, clear_bytes, allow_cluster))
-    if (cell == PARARNN_CELL_LINEAR) st = tma ? PARARNN_FWD(CellLinear, FwdLinT) : PARARNN_FWD(CellLinear, FwdLinS);
-    else if (cell == PARARNN_CELL_DIAG_GRU) st = tma ? PARARNN_FWD(CellGRU, FwdGruT) : PARARNN_FWD(CellGRU, FwdGruS);
-    else st = tma ? PARARNN_FWD(CellLSTM, FwdLstmT) : PARARNN_FWD(CellLSTM, FwdLstmS);
+    if (cell == PARARNN_CELL_LINEAR)
+        st = small ? PARARNN_FWD(CellLinear, FwdLinQ)
+                   : tma ? PARARNN_FWD(CellLinear, FwdLinT) : PARARNN_FWD(CellLinear, FwdLinS);
+    else if (cell == PARARNN_CELL_DIAG_GRU)
+        st = small ? PARARNN_FWD(CellGRU, FwdGruQ) : tma ? PARARNN_FWD(CellGRU, FwdGruT) : PARARNN_FWD(CellGRU, FwdGruS);
+    else
+        st = small ? PARARNN_FWD(CellLSTM, FwdLstmQ)
+                   : tma ? PARARNN_FWD(CellLSTM, FwdLstmT) : PARARNN_FWD(CellLSTM, FwdLstmS);
 #undef PARARNN_FWD
     if (st != PARARNN_OK) return st;
     if (resid_hist && Keff < K) {

@@ -22,6 +22,7 @@ pytestmark = pytest.mark.gpu
 TOL_H, TOL_G = 1e-4, 1e-3
 DEV = "cuda:0"
 HEADER_WORDS = 256 // 8  # the first tile's status word follows the 256-byte header
+NO_CLUSTER = 2           # PARARNN_HOOK_NO_CLUSTER
 
 
 def _inputs(cell, B, T, D, seed):
@@ -52,8 +53,17 @@ def _retag(ws, old, new):
     return int(hit.sum().item())
 
 
+@pytest.fixture
+def lookback_path():
+    # these tests plant look-back words, so the forward must take the
+    # look-back path even where the problem would fit the cluster path
+    assert binding.pararnn_debug_hooks(0, NO_CLUSTER) == binding.OK
+    yield
+    binding.pararnn_debug_hooks(0, 0)
+
+
 @pytest.mark.parametrize("cell", [oracle.LINEAR, oracle.DIAG_GRU, oracle.DIAG_LSTM])
-def test_stale_lookback_words_with_live_tags(cell, cuda_device):
+def test_stale_lookback_words_with_live_tags(cell, cuda_device, lookback_path):
     # one workspace, large enough for both shapes, never zero-filled
     shapes = [(2, 1500, 160, 3), (1, 2300, 96, 2)]
     n = max(binding.pararnn_workspace_bytes(cell, B, T, D, K) for B, T, D, K in shapes)
@@ -85,7 +95,7 @@ def test_stale_lookback_words_with_live_tags(cell, cuda_device):
         assert rel_err(to_np(da), dao) <= TOL_G
 
 
-def test_uniform_fill_that_reads_as_published_carries(cuda_device):
+def test_uniform_fill_that_reads_as_published_carries(cuda_device, lookback_path):
     # every word of the workspace says "inclusive state published" under the
     # tag the next call will use, with a payload of float bits 2 (a carry of
     # about 3e-45): a call that trusted it would start each tile from zero
@@ -114,6 +124,7 @@ def test_lookback_timeout_then_recovery(cell, cuda_device):
     dpx = torch.empty((B, T, G, D), device=DEV)
     assert binding.pararnn_debug_hooks(20_000_000, 1) == binding.OK  # 20 ms, stall the first tile
     try:
+        # (the stall hook also keeps the forward on the look-back path)
         for direction in ("forward", "backward"):
             torch.cuda.synchronize()
             t0 = time.perf_counter()
