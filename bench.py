@@ -355,19 +355,33 @@ class Problem:
             self.da = torch.empty((w.G, w.D), dtype=torch.float32, device=device)
         self.code = binding.BF16 if w.px_dtype == "bf16" else binding.F32
         self.stream = torch.cuda.current_stream(device)
+        # the C entry points with their arguments resolved once (device
+        # addresses and the stream handle), called as a C caller would call
+        # them: the per-call cost is the library's, not Python's
+        lib = binding.load()
+        ptr = lambda t: None if t is None else t.data_ptr()
+        self._fwd = lib.pararnn_newton_forward
+        self._fwd_args = (w.cell_id, w.B, w.T, w.D, self.code, ptr(self.px), ptr(self.a), None, w.K, ptr(self.H),
+                          ptr(self.ws), self.ws.numel(), None, self.stream.cuda_stream)
+        if w.backward:
+            self._bwd = lib.pararnn_newton_backward
+            self._bwd_args = (w.cell_id, w.B, w.T, w.D, self.code, ptr(self.px), ptr(self.a), None, ptr(self.H),
+                              ptr(self.g), ptr(self.dpx), ptr(self.da), None, ptr(self.ws), self.ws.numel(),
+                              self.stream.cuda_stream)
 
     def forward(self, px=None, H=None):
         w = self.w
-        st = self.b.pararnn_newton_forward(w.cell_id, w.B, w.T, w.D, self.code, self.px if px is None else px,
-                                           self.a, None, w.K, self.H if H is None else H, self.ws,
-                                           self.ws.numel(), None, self.stream)
+        if px is None and H is None:
+            st = self._fwd(*self._fwd_args)
+        else:
+            st = self.b.pararnn_newton_forward(w.cell_id, w.B, w.T, w.D, self.code, self.px if px is None else px,
+                                               self.a, None, w.K, self.H if H is None else H, self.ws,
+                                               self.ws.numel(), None, self.stream)
         if st != 0:
             raise RuntimeError("forward: %s %s" % (self.b.STATUS[st], self.b.pararnn_last_error()))
 
     def backward(self):
-        w = self.w
-        st = self.b.pararnn_newton_backward(w.cell_id, w.B, w.T, w.D, self.code, self.px, self.a, None, self.H,
-                                            self.g, self.dpx, self.da, None, self.ws, self.ws.numel(), self.stream)
+        st = self._bwd(*self._bwd_args)
         if st != 0:
             raise RuntimeError("backward: %s %s" % (self.b.STATUS[st], self.b.pararnn_last_error()))
 
@@ -432,6 +446,37 @@ def time_device(prob, steps, warmup, dist, device):
     torch.cuda.synchronize(device)
     prob.check_status()
     return reduce_max(dist, total, device) / steps, fwd, bwd
+
+
+def time_graph(prob, steps=50, replays=4):
+    """Device time per forward call with the calls replayed from a CUDA graph
+    (captured once on a side stream): the kernel's own time without the
+    per-launch overhead, for launch-bound (small) problems."""
+    import torch
+
+    side = torch.cuda.Stream(prob.dev)
+    args = list(prob._fwd_args)
+    args[-1] = side.cuda_stream
+    side.wait_stream(prob.stream)
+    with torch.cuda.stream(side):
+        for _ in range(3):
+            prob._fwd(*args)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side):
+        for _ in range(steps):
+            prob._fwd(*args)
+    g.replay()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(side)
+    for _ in range(replays):
+        g.replay()
+    t1.record(side)
+    torch.cuda.synchronize()
+    del g
+    prob.check_status()
+    return t0.elapsed_time(t1) / (steps * replays)
 
 
 def time_unroll(prob, steps=3):
@@ -606,6 +651,9 @@ def extra_workloads(names, device, seed_base):
             rec.update(bwd_ms=round(bwd, 4), bwd=kernel_roofline(w, "bwd", bwd, peaks))
         ums = time_unroll(prob)
         rec.update(unroll_ms=round(ums, 4), newton_fwd_speedup_vs_gpu_unroll=round(ums / fwd, 2))
+        if fwd < 0.1:
+            # launch-bound: the forward's device time without launch overhead
+            rec["fwd_ms_graph_replay"] = round(time_graph(prob), 4)
         out[name] = rec
         del prob
         torch.cuda.empty_cache()

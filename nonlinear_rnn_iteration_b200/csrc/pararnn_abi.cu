@@ -236,8 +236,52 @@ EncodeTiledFn encode_fn() {
 
 // 3-D map over a (rows, inner, D) row-major tensor: dims (D, inner, rows),
 // box (W, inner, L), zero fill outside.
+// The last few tensor maps this thread encoded, by their arguments: a
+// descriptor is plain data made from the arguments alone, so repeated calls
+// on the same buffers (a training loop) reuse it instead of asking the
+// driver again.
+struct MapCacheEntry {
+    const void* base;
+    int64_t D, rows;
+    int inner, W, L;
+    bool bf16, valid;
+    CUtensorMap map;
+};
+constexpr int kMapCache = 4;
+thread_local MapCacheEntry t_maps[kMapCache];
+thread_local int t_map_next = 0;
+
+pararnn_status encode_map(CUtensorMap* map, const void* base, bool bf16, int64_t D, int inner, int64_t rows, int W,
+                          int L);
+
 pararnn_status make_map(CUtensorMap* map, const void* base, bool bf16, int64_t D, int inner, int64_t rows, int W,
                         int L) {
+    for (int i = 0; i < kMapCache; ++i) {
+        const MapCacheEntry& e = t_maps[i];
+        if (e.valid && e.base == base && e.bf16 == bf16 && e.D == D && e.inner == inner && e.rows == rows &&
+            e.W == W && e.L == L) {
+            *map = e.map;
+            return PARARNN_OK;
+        }
+    }
+    pararnn_status st = encode_map(map, base, bf16, D, inner, rows, W, L);
+    if (st != PARARNN_OK) return st;
+    MapCacheEntry& e = t_maps[t_map_next];
+    t_map_next = (t_map_next + 1) % kMapCache;
+    e.base = base;
+    e.bf16 = bf16;
+    e.D = D;
+    e.inner = inner;
+    e.rows = rows;
+    e.W = W;
+    e.L = L;
+    e.map = *map;
+    e.valid = true;
+    return PARARNN_OK;
+}
+
+pararnn_status encode_map(CUtensorMap* map, const void* base, bool bf16, int64_t D, int inner, int64_t rows, int W,
+                          int L) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return fail(PARARNN_ECUDA, "cuTensorMapEncodeTiled is unavailable");
     const size_t esz = bf16 ? 2 : 4;
