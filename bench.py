@@ -75,6 +75,9 @@ def streaming_bytes_per_elem(w, direction):
 # 8 x 1024 channels in slices of 256 make 32 slices, whose shorter fill and
 # drain beat whole rows (8 slices)
 E2E_CHANNELS = 256
+# channels per slice of the forward + adjoint host-buffer pipeline: each
+# slice holds all B rows, so 4096 channels in slices of 128 make 32 slices
+E2E_STEP_CHANNELS = 128
 
 KERNEL_SOURCES = ["newton_fwd.cuh", "adjoint_bwd.cuh", "lookback.cuh", "cells.cuh", "common.cuh", "tma.cuh", "pararnn_abi.cu"]
 
@@ -500,33 +503,43 @@ def time_unroll(prob, steps=3):
 
 def time_e2e(prob, steps):
     """Same step through the public API with host buffers, all copies inside
-    the timed region: a forward-only step goes through the host-buffer entry
-    point (pinned host in, pinned host out, copies overlapped with the solve);
-    a step with a backward copies the pre-activations and dL/dH in, runs both
-    calls and copies H and dL/dpx out."""
+    the timed region: the host-buffer entry points take pinned host inputs
+    and write pinned host outputs, their copies overlapped with the solve --
+    pararnn_newton_forward_host for a forward-only step,
+    pararnn_newton_step_host (pre-activations and dL/dH in, H and dL/dpx out)
+    for a step with the adjoint backward."""
     import torch
 
+    from nonlinear_rnn_iteration_b200 import binding
+
     w = prob.w
+    s = prob.stream
     px_host = torch.empty(prob.px.shape, dtype=prob.px.dtype, pin_memory=True)
     px_host.copy_(prob.px)
     H_host = torch.empty(prob.H.shape, dtype=torch.float32, pin_memory=True)
-    outs = [H_host]
+    code = binding.BF16 if prob.px.dtype == torch.bfloat16 else binding.F32
     if w.backward:
         g_host = torch.empty(prob.g.shape, dtype=torch.float32, pin_memory=True)
         g_host.copy_(prob.g)
         dpx_host = torch.empty(prob.dpx.shape, dtype=torch.float32, pin_memory=True)
-        outs.append(dpx_host)
-    px_dev = torch.empty_like(prob.px)
-    s = prob.stream
-    if not w.backward:
-        # the public host-buffer entry point: slices of one batch row and
-        # E2E_CHANNELS channels whose copies in and out overlap the solve
-        from nonlinear_rnn_iteration_b200 import binding
+        chans = E2E_STEP_CHANNELS if (w.D % 8 == 0 and w.D > E2E_STEP_CHANNELS) else 0
+        n = binding.pararnn_newton_step_host_workspace_bytes(w.cell_id, w.B, w.T, w.D, w.K, code, chans)
+        ws_host = torch.empty(n, dtype=torch.uint8, device=prob.px.device)
+        da = prob.da
 
-        code = binding.BF16 if prob.px.dtype == torch.bfloat16 else binding.F32
+        def one():
+            st = binding.pararnn_newton_step_host(w.cell_id, w.B, w.T, w.D, code, px_host, prob.a, None, w.K,
+                                                  g_host, H_host, dpx_host, da, ws_host, n, chans, s)
+            if st != binding.OK:
+                raise RuntimeError("pararnn_newton_step_host: %s" % binding.pararnn_last_error())
+
+        h2d = px_host.numel() * px_host.element_size() + g_host.numel() * 4
+        d2h = H_host.numel() * 4 + dpx_host.numel() * 4
+    else:
+        # slices of one batch row and E2E_CHANNELS channels
         chans = E2E_CHANNELS if (w.D % 8 == 0 and w.D > E2E_CHANNELS) else 0
         n = binding.pararnn_newton_forward_host_workspace_bytes(w.cell_id, w.B, w.T, w.D, w.K, code, 1, chans)
-        ws_host = torch.zeros(n, dtype=torch.uint8, device=prob.px.device)
+        ws_host = torch.empty(n, dtype=torch.uint8, device=prob.px.device)
 
         def one():
             st = binding.pararnn_newton_forward_host(w.cell_id, w.B, w.T, w.D, code, px_host, prob.a, None, w.K,
@@ -534,28 +547,8 @@ def time_e2e(prob, steps):
             if st != binding.OK:
                 raise RuntimeError("pararnn_newton_forward_host: %s" % binding.pararnn_last_error())
 
-        one()
-        torch.cuda.synchronize()
-        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        t0.record(s)
-        for _ in range(steps):
-            one()
-        t1.record(s)
-        torch.cuda.synchronize()
-        ms = t0.elapsed_time(t1) / steps
-        return ms, px_host.numel() * px_host.element_size(), H_host.numel() * 4
-
-    def one():
-        px_dev.copy_(px_host, non_blocking=True)
-        if w.backward:
-            prob.g.copy_(g_host, non_blocking=True)
-        prob.forward(px=px_dev)
-        if w.backward:
-            prob.backward()
-        H_host.copy_(prob.H, non_blocking=True)
-        if w.backward:
-            dpx_host.copy_(prob.dpx, non_blocking=True)
-
+        h2d = px_host.numel() * px_host.element_size()
+        d2h = H_host.numel() * 4
     one()
     torch.cuda.synchronize()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -564,10 +557,10 @@ def time_e2e(prob, steps):
         one()
     t1.record(s)
     torch.cuda.synchronize()
-    ms = t0.elapsed_time(t1) / steps
-    h2d = px_host.numel() * px_host.element_size() + (g_host.numel() * 4 if w.backward else 0)
-    d2h = sum(o.numel() * o.element_size() for o in outs)
-    return ms, h2d, d2h
+    st = binding.pararnn_status_sync(ws_host, s)
+    if st != binding.OK:
+        raise RuntimeError("host-buffer step device status %s" % binding.STATUS[st])
+    return t0.elapsed_time(t1) / steps, h2d, d2h
 
 
 def cpu_baseline(w, device, seed, target_s=12.0, max_bytes=2.0e9):

@@ -318,6 +318,41 @@ pararnn_status pararnn_newton_forward_host(pararnn_cell cell, int64_t B, int64_t
                                            const float* h0, int K, float* H_host, void* workspace, size_t ws_bytes,
                                            int64_t rows_per_slice, int64_t channels_per_slice, void* stream);
 
+/* ---- a training step on host buffers --------------------------------------
+ * pararnn_newton_forward followed by pararnn_newton_backward, with the
+ * pre-activations and dL/dH read from host memory and H and dL/dpx written
+ * back to it (pinned memory lets the copies overlap).  The channels are cut
+ * into slices of channels_per_slice channels, each holding every batch row,
+ * that pass through three device slots on three internal streams -- copy in,
+ * forward + adjoint, copy out -- so that both PCIe directions and the solver
+ * work at once.  A slice's dL/da columns are complete sums over (b, t) and
+ * are written straight into dL_da.  Channels are independent recurrences and
+ * the tiling along T does not depend on the slice, so every output is
+ * bit-identical to pararnn_newton_forward + pararnn_newton_backward on the
+ * whole batch (Method section: forward by Newton, backward by one linear
+ * adjoint scan; the API overview's training use of ParaGRU / ParaLSTM).
+ *   channels_per_slice  0 (or >= D): one slice; otherwise a multiple of 8,
+ *                 and D must be a multiple of 8 too
+ *   preacts_host  (B, T, G, D) px_dtype, host (or device) memory
+ *   dL_dH_host    (B, T, S, D) float32, host (or device) memory
+ *   diag_w, h0    device memory or NULL, as for pararnn_newton_forward
+ *   H_host        (B, T, S, D) float32, host (or device) memory, written
+ *   dL_dpx_host   (B, T, G, D) float32, host (or device) memory, written
+ *   dL_da         (G, D) float32 device memory or NULL, written (NULL, and
+ *                 nothing written, for the linear cell)
+ *   workspace     >= pararnn_newton_step_host_workspace_bytes(...) bytes,
+ *                 256-byte aligned device memory, any contents
+ * K as for pararnn_newton_forward (0 takes pararnn_kstar).  Ordering with
+ * `stream`, status reporting and errors as for pararnn_newton_forward_host;
+ * dL/dh0 is not computed.  The workspace size function returns 0 for invalid
+ * arguments. */
+size_t pararnn_newton_step_host_workspace_bytes(pararnn_cell cell, int64_t B, int64_t T, int64_t D, int K,
+                                                pararnn_dtype px_dtype, int64_t channels_per_slice);
+pararnn_status pararnn_newton_step_host(pararnn_cell cell, int64_t B, int64_t T, int64_t D, pararnn_dtype px_dtype,
+                                        const void* preacts_host, const float* diag_w, const float* h0, int K,
+                                        const float* dL_dH_host, float* H_host, float* dL_dpx_host, float* dL_da,
+                                        void* workspace, size_t ws_bytes, int64_t channels_per_slice, void* stream);
+
 /* ---- head-wise GRU: block-diagonal recurrent weights --------------------
  * ParaGRU(mix='head', n_heads) of the pararnn-torch page (Models / Usage,
  * "Dreamer-style block GRU": block-diagonal A).  The page prints no

@@ -43,6 +43,8 @@ SIGNATURES = {
     "pararnn_newton_forward_noalloc": (_I, [_I, _I64, _I64, _I64, _I, _P, _P, _P, _I, _P, _P, _I, _P]),
     "pararnn_newton_forward_host_workspace_bytes": (_SZ, [_I, _I64, _I64, _I64, _I, _I, _I64, _I64]),
     "pararnn_newton_forward_host": (_I, [_I, _I64, _I64, _I64, _I, _P, _P, _P, _I, _P, _P, _SZ, _I64, _I64, _P]),
+    "pararnn_newton_step_host_workspace_bytes": (_SZ, [_I, _I64, _I64, _I64, _I, _I, _I64]),
+    "pararnn_newton_step_host": (_I, [_I, _I64, _I64, _I64, _I, _P, _P, _P, _I, _P, _P, _P, _P, _P, _SZ, _I64, _P]),
     "pararnn_head_gru_workspace_bytes": (_SZ, [_I64, _I64, _I64, _I, _I]),
     "pararnn_head_gru_forward": (_I, [_I64, _I64, _I64, _I, _I, _P, _P, _P, _I, _P, _P, _SZ, _P, _P]),
     "pararnn_head_gru_backward_workspace_bytes": (_SZ, [_I64, _I64, _I64, _I]),
@@ -175,6 +177,17 @@ def pararnn_newton_forward_host(cell, B, T, D, px_dtype, preacts_host, diag_w, h
     return load().pararnn_newton_forward_host(cell, B, T, D, px_dtype, _ptr(preacts_host), _ptr(diag_w), _ptr(h0), K,
                                               _ptr(H_host), _ptr(workspace), ws_bytes, rows_per_slice,
                                               channels_per_slice, _stream(stream))
+
+
+def pararnn_newton_step_host_workspace_bytes(cell, B, T, D, K, px_dtype, channels_per_slice=0):
+    return load().pararnn_newton_step_host_workspace_bytes(cell, B, T, D, K, px_dtype, channels_per_slice)
+
+
+def pararnn_newton_step_host(cell, B, T, D, px_dtype, preacts_host, diag_w, h0, K, dL_dH_host, H_host, dL_dpx_host,
+                             dL_da, workspace, ws_bytes, channels_per_slice, stream):
+    return load().pararnn_newton_step_host(cell, B, T, D, px_dtype, _ptr(preacts_host), _ptr(diag_w), _ptr(h0), K,
+                                           _ptr(dL_dH_host), _ptr(H_host), _ptr(dL_dpx_host), _ptr(dL_da),
+                                           _ptr(workspace), ws_bytes, channels_per_slice, _stream(stream))
 
 
 def pararnn_head_gru_workspace_bytes(B, T, D, n_heads, K):
@@ -399,3 +412,35 @@ def newton_forward_host(cell, px_host, diag_w=None, h0=None, K=1, out_host=None,
     if sync_status:
         _check(pararnn_status_sync(workspace, st), "pararnn_newton_forward_host (device status)")
     return out_host
+
+
+def newton_step_host(cell, px_host, dL_dH_host, diag_w=None, h0=None, K=1, channels_per_slice=0, outs=None,
+                     workspace=None, stream=None, sync_status=True):
+    """Forward + adjoint on host tensors (pinned for overlap): returns
+    (H, dL/dpx) on the host and dL/da (G, D) on the device (None for the
+    linear cell)."""
+    import torch
+
+    cell = CELLS.get(cell, cell)
+    B, T, D = _shape(cell, px_host)
+    S, G = pararnn_state_width(cell), pararnn_num_gates(cell)
+    code = _dtype_code(px_host)
+    dev = diag_w.device if diag_w is not None else torch.device("cuda", torch.cuda.current_device())
+    if outs is None:
+        pin = px_host.is_pinned()
+        outs = (torch.empty((B, T, S, D), dtype=torch.float32, pin_memory=pin),
+                torch.empty((B, T, G, D), dtype=torch.float32, pin_memory=pin),
+                None if cell == LINEAR else torch.empty((G, D), dtype=torch.float32, device=dev))
+    H_host, dpx_host, da = outs
+    if workspace is None:
+        n = pararnn_newton_step_host_workspace_bytes(cell, B, T, D, K, code, channels_per_slice)
+        if n == 0:
+            raise PararnnError(EINVAL, "pararnn_newton_step_host_workspace_bytes", "invalid arguments")
+        workspace = torch.empty(n, dtype=torch.uint8, device=dev)
+    st = stream if stream is not None else torch.cuda.current_stream(dev)
+    _check(pararnn_newton_step_host(cell, B, T, D, code, px_host, diag_w, h0, K, dL_dH_host, H_host, dpx_host, da,
+                                    workspace, workspace.numel(), channels_per_slice, st),
+           "pararnn_newton_step_host")
+    if sync_status:
+        _check(pararnn_status_sync(workspace, st), "pararnn_newton_step_host (device status)")
+    return H_host, dpx_host, da

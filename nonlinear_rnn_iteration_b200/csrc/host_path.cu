@@ -229,3 +229,204 @@ extern "C" pararnn_status pararnn_newton_forward_host(pararnn_cell cell, int64_t
     }
     return PARARNN_OK;
 }
+
+// ---- a whole training step on host buffers ----------------------------------
+// The forward and the adjoint of one batch, with the pre-activations and
+// dL/dH coming from host memory and H and dL/dpx going back to it, pipelined
+// like the forward above but by slices of channels only: a slice holds every
+// batch row of its channels, so its dL/da columns are complete sums and go
+// straight to their place in dL_da.  Channels are independent recurrences and
+// the tiling along T does not depend on the slice, so every value is
+// bit-identical to pararnn_newton_forward + pararnn_newton_backward on the
+// whole batch.
+
+namespace pararnn {
+namespace hp {
+
+struct StepLayout {
+    int64_t chans = 0;
+    size_t ws_bytes = 0, px_bytes = 0, g_bytes = 0, h_bytes = 0, dpx_bytes = 0, w_bytes = 0, h0_bytes = 0,
+           da_bytes = 0, slot_bytes = 0, total = 0;
+};
+
+bool step_layout(pararnn_cell cell, int64_t B, int64_t T, int64_t D, int K, int64_t channels_per_slice, size_t esz,
+                 StepLayout& l) {
+    const int G = pararnn_num_gates(cell), S = pararnn_state_width(cell);
+    if (G < 0 || B < 0 || T < 0 || D < 0 || channels_per_slice < 0) return false;
+    const bool split = channels_per_slice > 0 && channels_per_slice < D;
+    if (split && (channels_per_slice % 8 != 0 || D % 8 != 0)) return false;
+    l.chans = split ? channels_per_slice : (D > 0 ? D : 1);
+    const int64_t Bq = B > 0 ? B : 1;
+    l.ws_bytes = pararnn_workspace_bytes(cell, Bq, T, l.chans, K);
+    if (l.ws_bytes == 0) return false;
+    l.px_bytes = align256((size_t)Bq * T * G * l.chans * esz);
+    l.g_bytes = align256((size_t)Bq * T * S * l.chans * sizeof(float));
+    l.h_bytes = l.g_bytes;
+    l.dpx_bytes = align256((size_t)Bq * T * G * l.chans * sizeof(float));
+    l.w_bytes = align256((size_t)G * l.chans * sizeof(float));
+    l.h0_bytes = align256((size_t)Bq * S * l.chans * sizeof(float));
+    l.da_bytes = align256((size_t)G * l.chans * sizeof(float));
+    l.slot_bytes = align256(l.ws_bytes) + l.px_bytes + l.g_bytes + l.h_bytes + l.dpx_bytes + l.w_bytes + l.h0_bytes +
+                   l.da_bytes;
+    l.total = 256 + kSlots * l.slot_bytes;
+    return true;
+}
+
+}  // namespace hp
+}  // namespace pararnn
+
+extern "C" size_t pararnn_newton_step_host_workspace_bytes(pararnn_cell cell, int64_t B, int64_t T, int64_t D, int K,
+                                                          pararnn_dtype px_dtype, int64_t channels_per_slice) {
+    if (px_dtype != PARARNN_F32 && px_dtype != PARARNN_BF16) return 0;
+    hp::StepLayout l;
+    if (!hp::step_layout(cell, B, T, D, K, channels_per_slice, px_dtype == PARARNN_BF16 ? 2 : 4, l)) return 0;
+    return l.total;
+}
+
+extern "C" pararnn_status pararnn_newton_step_host(pararnn_cell cell, int64_t B, int64_t T, int64_t D,
+                                                   pararnn_dtype px_dtype, const void* preacts_host,
+                                                   const float* diag_w, const float* h0, int K,
+                                                   const float* dL_dH_host, float* H_host, float* dL_dpx_host,
+                                                   float* dL_da, void* workspace, size_t ws_bytes,
+                                                   int64_t channels_per_slice, void* stream) {
+    if (px_dtype != PARARNN_F32 && px_dtype != PARARNN_BF16)
+        return hp::fail(PARARNN_EINVAL, "pararnn_newton_step_host: unknown pre-activation dtype");
+    const size_t esz = px_dtype == PARARNN_BF16 ? 2 : 4;
+    hp::StepLayout l;
+    if (!hp::step_layout(cell, B, T, D, K, channels_per_slice, esz, l))
+        return hp::fail(PARARNN_EINVAL, "pararnn_newton_step_host: bad cell, sizes, K or channels_per_slice");
+    if (!workspace || ws_bytes < l.total || !pointer_on_device(workspace) ||
+        (reinterpret_cast<uintptr_t>(workspace) & 255))
+        return hp::fail(PARARNN_EINVAL, "pararnn_newton_step_host: workspace missing, small or not 256-byte aligned "
+                                        "device memory (see pararnn_newton_step_host_workspace_bytes)");
+    if ((diag_w && !pointer_on_device(diag_w)) || (h0 && !pointer_on_device(h0)) ||
+        (dL_da && !pointer_on_device(dL_da)))
+        return hp::fail(PARARNN_EINVAL, "pararnn_newton_step_host: diag_w, h0 and dL_da must be device memory");
+    cudaStream_t user = static_cast<cudaStream_t>(stream);
+    unsigned char* ws = static_cast<unsigned char*>(workspace);
+    cudaError_t e = cudaMemsetAsync(ws, 0, 256, user);
+    if (e != cudaSuccess) return hp::fail(PARARNN_ECUDA, "pararnn_newton_step_host: header reset failed");
+    const int G = pararnn_num_gates(cell), S = pararnn_state_width(cell);
+    if (cell == PARARNN_CELL_LINEAR) dL_da = nullptr;  // no recurrent weights
+    if (B == 0 || T == 0 || D == 0) {
+        if (dL_da && D > 0) e = cudaMemsetAsync(dL_da, 0, sizeof(float) * G * D, user);
+        return e == cudaSuccess ? PARARNN_OK : hp::fail(PARARNN_ECUDA, "pararnn_newton_step_host: dL_da reset failed");
+    }
+    if (!preacts_host || !dL_dH_host || !H_host || !dL_dpx_host)
+        return hp::fail(PARARNN_EINVAL, "pararnn_newton_step_host: preacts, dL_dH, H and dL_dpx are required");
+    const int64_t ncs = (D + l.chans - 1) / l.chans;
+
+    cudaStream_t sin = nullptr, scomp = nullptr, sout = nullptr;
+    cudaEvent_t start = nullptr, ev_in[hp::kSlots] = {}, ev_comp[hp::kSlots] = {}, ev_out[hp::kSlots] = {};
+    auto cleanup = [&]() {
+        for (int k = 0; k < hp::kSlots; ++k) {
+            if (ev_in[k]) cudaEventDestroy(ev_in[k]);
+            if (ev_comp[k]) cudaEventDestroy(ev_comp[k]);
+            if (ev_out[k]) cudaEventDestroy(ev_out[k]);
+        }
+        if (start) cudaEventDestroy(start);
+        if (sin) cudaStreamDestroy(sin);
+        if (scomp) cudaStreamDestroy(scomp);
+        if (sout) cudaStreamDestroy(sout);
+    };
+    e = cudaStreamCreateWithFlags(&sin, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&scomp, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&sout, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&start, cudaEventDisableTiming);
+    for (int k = 0; k < hp::kSlots && e == cudaSuccess; ++k) {
+        e = cudaEventCreateWithFlags(&ev_in[k], cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev_comp[k], cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev_out[k], cudaEventDisableTiming);
+    }
+    if (e == cudaSuccess) e = cudaEventRecord(start, user);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(sin, start, 0);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(scomp, start, 0);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(sout, start, 0);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        cleanup();
+        return hp::fail(PARARNN_ECUDA, "pararnn_newton_step_host: stream or event setup failed");
+    }
+
+    pararnn_status st = PARARNN_OK;
+    for (int64_t ic = 0; ic < ncs && st == PARARNN_OK; ++ic) {
+        const int k = (int)(ic % hp::kSlots);
+        const int64_t d0 = ic * l.chans, dn = (d0 + l.chans <= D) ? l.chans : D - d0;
+        unsigned char* p = ws + 256 + (size_t)k * l.slot_bytes;
+        void* sws = p;
+        p += hp::align256(l.ws_bytes);
+        void* px_dev = p;
+        p += l.px_bytes;
+        float* g_dev = reinterpret_cast<float*>(p);
+        p += l.g_bytes;
+        float* h_dev = reinterpret_cast<float*>(p);
+        p += l.h_bytes;
+        float* dpx_dev = reinterpret_cast<float*>(p);
+        p += l.dpx_bytes;
+        float* w_dev = reinterpret_cast<float*>(p);
+        p += l.w_bytes;
+        float* h0_dev = reinterpret_cast<float*>(p);
+        p += l.h0_bytes;
+        float* da_dev = reinterpret_cast<float*>(p);
+        // in: after the slot's previous slice has been solved
+        if (ic >= hp::kSlots) e = cudaStreamWaitEvent(sin, ev_comp[k], 0);
+        // (B*T*G rows of dn channels, D apart in host memory) and the same for dL/dH
+        if (e == cudaSuccess)
+            e = cudaMemcpy2DAsync(px_dev, (size_t)dn * esz, static_cast<const unsigned char*>(preacts_host) + d0 * esz,
+                                  (size_t)D * esz, (size_t)dn * esz, (size_t)B * T * G, cudaMemcpyDefault, sin);
+        if (e == cudaSuccess)
+            e = cudaMemcpy2DAsync(g_dev, (size_t)dn * sizeof(float), dL_dH_host + d0, (size_t)D * sizeof(float),
+                                  (size_t)dn * sizeof(float), (size_t)B * T * S, cudaMemcpyDefault, sin);
+        if (e == cudaSuccess && diag_w)
+            e = cudaMemcpy2DAsync(w_dev, (size_t)dn * sizeof(float), diag_w + d0, (size_t)D * sizeof(float),
+                                  (size_t)dn * sizeof(float), (size_t)G, cudaMemcpyDefault, sin);
+        if (e == cudaSuccess && h0)
+            e = cudaMemcpy2DAsync(h0_dev, (size_t)dn * sizeof(float), h0 + d0, (size_t)D * sizeof(float),
+                                  (size_t)dn * sizeof(float), (size_t)B * S, cudaMemcpyDefault, sin);
+        if (e == cudaSuccess) e = cudaEventRecord(ev_in[k], sin);
+        // solve: after the copy in, and after the slot's previous outputs have left
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(scomp, ev_in[k], 0);
+        if (e == cudaSuccess && ic >= hp::kSlots) e = cudaStreamWaitEvent(scomp, ev_out[k], 0);
+        if (e != cudaSuccess) break;
+        const float* w_use = diag_w ? w_dev : nullptr;
+        const float* h0_use = h0 ? h0_dev : nullptr;
+        st = newton_forward_slice(B, D, cell, B, T, dn, px_dtype, px_dev, w_use, h0_use, K, h_dev, sws, l.ws_bytes,
+                                  scomp);
+        if (st != PARARNN_OK) break;
+        hp::fold_status<<<1, 32, 0, scomp>>>(reinterpret_cast<unsigned*>(ws), reinterpret_cast<unsigned*>(sws));
+        e = cudaGetLastError();
+        if (e != cudaSuccess) break;
+        st = pararnn_newton_backward(cell, B, T, dn, px_dtype, px_dev, w_use, h0_use, h_dev, g_dev, dpx_dev,
+                                     dL_da ? da_dev : nullptr, nullptr, sws, l.ws_bytes, scomp);
+        if (st != PARARNN_OK) break;
+        hp::fold_status<<<1, 32, 0, scomp>>>(reinterpret_cast<unsigned*>(ws), reinterpret_cast<unsigned*>(sws));
+        e = cudaGetLastError();
+        if (e == cudaSuccess && dL_da)  // (G, dn) into (G, D) at column d0
+            e = cudaMemcpy2DAsync(dL_da + d0, (size_t)D * sizeof(float), da_dev, (size_t)dn * sizeof(float),
+                                  (size_t)dn * sizeof(float), (size_t)G, cudaMemcpyDeviceToDevice, scomp);
+        if (e == cudaSuccess) e = cudaEventRecord(ev_comp[k], scomp);
+        // out
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(sout, ev_comp[k], 0);
+        if (e == cudaSuccess)
+            e = cudaMemcpy2DAsync(H_host + d0, (size_t)D * sizeof(float), h_dev, (size_t)dn * sizeof(float),
+                                  (size_t)dn * sizeof(float), (size_t)B * T * S, cudaMemcpyDefault, sout);
+        if (e == cudaSuccess)
+            e = cudaMemcpy2DAsync(dL_dpx_host + d0, (size_t)D * sizeof(float), dpx_dev, (size_t)dn * sizeof(float),
+                                  (size_t)dn * sizeof(float), (size_t)B * T * G, cudaMemcpyDefault, sout);
+        if (e == cudaSuccess) e = cudaEventRecord(ev_out[k], sout);
+        if (e != cudaSuccess) break;
+    }
+    cudaEvent_t done[3] = {ev_in[0], ev_comp[0], ev_out[0]};
+    cudaStream_t ss[3] = {sin, scomp, sout};
+    for (int j = 0; j < 3 && e == cudaSuccess; ++j) {
+        e = cudaEventRecord(done[j], ss[j]);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(user, done[j], 0);
+    }
+    cleanup();
+    if (st != PARARNN_OK) return st;
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return hp::fail(PARARNN_ECUDA, "pararnn_newton_step_host: copy or launch failed");
+    }
+    return PARARNN_OK;
+}

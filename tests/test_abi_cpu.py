@@ -173,6 +173,23 @@ def test_host_path_workspace_bytes():
     assert f(gru, 2, 1024, 256, 3, binding.F32, 5) == f(gru, 2, 1024, 256, 3, binding.F32, 2)
 
 
+def test_step_host_workspace_bytes():
+    f = binding.pararnn_newton_step_host_workspace_bytes
+    gru = 1
+    assert f(gru, 2, 1024, 256, 3, 7, 0) == 0  # dtype
+    assert f(9, 2, 1024, 256, 3, binding.F32, 0) == 0  # cell
+    assert f(gru, 2, 1024, 256, 3, binding.F32, 12) == 0  # not a multiple of 8
+    assert f(gru, 2, 1024, 100, 3, binding.F32, 8) == 0  # D not a multiple of 8
+    assert f(gru, 2, 1024, 256, 3, binding.F32, -8) == 0
+    whole = f(gru, 2, 1024, 256, 3, binding.F32, 0)
+    assert whole == f(gru, 2, 1024, 256, 3, binding.F32, 256) == f(gru, 2, 1024, 256, 3, binding.F32, 1000)
+    # three slots of pre-activations, dL/dH, H, dL/dpx (float32) and a solver workspace
+    n = 2 * 1024 * 256
+    assert whole >= 3 * n * (3 * 4 + 4 + 4 + 3 * 4) + 3 * binding.pararnn_workspace_bytes(gru, 2, 1024, 256, 3)
+    assert 0 < f(gru, 2, 1024, 256, 3, binding.F32, 64) < whole
+    assert f(gru, 2, 1024, 256, 3, binding.BF16, 64) < f(gru, 2, 1024, 256, 3, binding.F32, 64)
+
+
 def test_debug_hooks_reject_long_limits():
     # pure host function: it only records the limits for later calls on this thread
     assert binding.pararnn_debug_hooks(20_000_000_000, 0) == binding.EINVAL

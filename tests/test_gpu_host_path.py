@@ -77,3 +77,68 @@ def test_host_path_channel_slices(cell, K, bf16, rows, chans, cuda_device):
     ref = binding.newton_forward(cell, px.to(DEV), w, h0, K=K).cpu()
     H = binding.newton_forward_host(cell, px.pin_memory(), w, h0, K=K, rows_per_slice=rows, channels_per_slice=chans)
     assert torch.equal(H, ref)
+
+
+# ---- forward + adjoint on host buffers (pararnn_newton_step_host) ----------
+
+@pytest.mark.parametrize("cell,K,bf16", [(binding.LINEAR, 1, False), (binding.DIAG_GRU, 3, False),
+                                         (binding.DIAG_GRU, 2, True), (binding.DIAG_LSTM, 3, False),
+                                         (binding.DIAG_LSTM, 0, True)])
+@pytest.mark.parametrize("chans", [0, 8, 64, 136, 48])
+def test_step_host_matches_device_path(cell, K, bf16, chans, cuda_device):
+    # H, dL/dpx and dL/da of the sliced pipeline are the device path's bits
+    B, T, D = 3, 300, 136
+    px, w = _inputs(cell, B, T, D, seed=cell * 7 + chans, bf16=bf16)
+    S = binding.pararnn_state_width(cell)
+    gen = torch.Generator().manual_seed(100 + chans)
+    g = torch.randn((B, T, S, D), generator=gen)
+    h0 = torch.randn((B, S, D), generator=gen).to(DEV)
+    pxd = px.to(DEV)
+    Hd = binding.newton_forward(cell, pxd, w, h0, K=K)
+    dpxd, dad, _ = binding.newton_backward(cell, pxd, Hd, g.to(DEV), w, h0)
+    H, dpx, da = binding.newton_step_host(cell, px.pin_memory(), g.pin_memory(), w, h0, K=K, channels_per_slice=chans)
+    torch.cuda.synchronize()
+    assert torch.equal(H, Hd.cpu())
+    assert torch.equal(dpx, dpxd.cpu())
+    if cell == binding.LINEAR:
+        assert da is None
+    else:
+        assert torch.equal(da.cpu(), dad.cpu())
+
+
+def test_step_host_pageable_memory_without_h0_or_weights(cuda_device):
+    B, T, D = 2, 500, 64
+    px, _ = _inputs(binding.DIAG_GRU, B, T, D, seed=11)
+    g = torch.randn((B, T, 1, D), generator=torch.Generator().manual_seed(12))
+    Hd = binding.newton_forward(binding.DIAG_GRU, px.to(DEV), None, None, K=2)
+    dpxd, dad, _ = binding.newton_backward(binding.DIAG_GRU, px.to(DEV), Hd, g.to(DEV), None, None)
+    H, dpx, da = binding.newton_step_host(binding.DIAG_GRU, px, g, None, None, K=2, channels_per_slice=16)
+    assert torch.equal(H, Hd.cpu()) and torch.equal(dpx, dpxd.cpu()) and torch.equal(da.cpu(), dad.cpu())
+
+
+def test_step_host_reports_nonfinite_and_bad_arguments(cuda_device):
+    B, T, D = 2, 100, 64
+    px, w = _inputs(binding.DIAG_GRU, B, T, D, seed=13)
+    g = torch.randn((B, T, 1, D))
+    g[1, 40, 0, 50] = float("inf")  # in the last of four slices
+    with pytest.raises(binding.PararnnError) as e:
+        binding.newton_step_host(binding.DIAG_GRU, px.pin_memory(), g.pin_memory(), w, None, K=2,
+                                 channels_per_slice=16)
+    assert e.value.status == binding.ENONFINITE
+    g[1, 40, 0, 50] = 0.0
+    n = binding.pararnn_newton_step_host_workspace_bytes(binding.DIAG_GRU, B, T, D, 2, binding.F32, 16)
+    ws = torch.empty(n, dtype=torch.uint8, device=DEV)
+    H, dpx = torch.empty((B, T, 1, D)), torch.empty((B, T, 3, D))
+    da = torch.empty((3, D), device=DEV)
+    f = binding.pararnn_newton_step_host
+    assert f(binding.DIAG_GRU, B, T, D, binding.F32, px, w, None, 2, g, H, dpx, da, ws, n - 256, 16, None) == binding.EINVAL
+    assert f(binding.DIAG_GRU, B, T, D, binding.F32, px, w, None, 2, g, H, dpx, da, ws, n, 12, None) == binding.EINVAL
+    # the weights and dL/da live on the device
+    assert f(binding.DIAG_GRU, B, T, D, binding.F32, px, w.cpu(), None, 2, g, H, dpx, da, ws, n, 16,
+             None) == binding.EINVAL
+    assert f(binding.DIAG_GRU, B, T, D, binding.F32, px, w, None, 2, g, H, dpx, da.cpu(), ws, n, 16,
+             None) == binding.EINVAL
+    assert f(binding.DIAG_GRU, B, T, D, binding.F32, px, w, None, 2, None, H, dpx, da, ws, n, 16,
+             None) == binding.EINVAL
+    assert f(binding.DIAG_GRU, B, T, D, binding.F32, px, w, None, 2, g, H, dpx, da, ws, n, 16, None) == binding.OK
+    assert binding.pararnn_status_sync(ws, None) == binding.OK
