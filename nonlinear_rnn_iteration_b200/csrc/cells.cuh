@@ -54,8 +54,10 @@ struct CellGRU {
     static constexpr bool kNonlinear = true;
 
     static __device__ __forceinline__ void warm(const float (&p)[G], const float (&)[G], float (&f)[S]) {
-        // h = 0: z = sig(p_z), c = tanh(p_c), f = z c
-        f[0] = sigmoid_f(p[0]) * tanh_f(p[2]);
+        // h = 0: z = sig(p_z), c = tanh(p_c), f = z c; z and c share a reciprocal
+        float z, ic;
+        inv_pair(sig_den(p[0]), tanh_den(p[2]), z, ic);
+        f[0] = z * tanh_from_inv(p[2], ic);
     }
     // z, r, c and the chain-rule factors G_z = df/dp_z, G_r = df/dp_r, G_c = df/dp_c
     static __device__ __forceinline__ void gates(const float (&p)[G], const float (&w)[G], float h, float& z,
@@ -70,8 +72,10 @@ struct CellGRU {
     static __device__ __forceinline__ void elem(const float (&p)[G], const float (&w)[G], const float (&sp)[S],
                                                 float (&f)[S], float (&A)[S * S], float (&beta)[S]) {
         const float h = sp[0];
-        const float z = sigmoid_f(__fmaf_rn(w[0], h, p[0]));
-        const float r = sigmoid_f(__fmaf_rn(w[1], h, p[1]));
+        // the update and reset gates share a reciprocal; the candidate
+        // depends on r and takes its own
+        float z, r;
+        inv_pair(sig_den(__fmaf_rn(w[0], h, p[0])), sig_den(__fmaf_rn(w[1], h, p[1])), z, r);
         const float wr = w[2] * r;
         const float c = tanh_f(__fmaf_rn(wr, h, p[2]));
         const float ch = c - h;
@@ -97,10 +101,12 @@ struct CellGRU {
     }
     // warm() on a pair of channels
     static __device__ __forceinline__ void warm2(const f2 (&p)[G], f2 (&f)[S]) {
-        f[0] = mul2(sigmoid2(p[0]), tanh2(p[2]));
+        f2 z, ic;
+        inv_pair2(sig_den2(p[0]), tanh_den2(p[2]), z, ic);
+        f[0] = mul2(z, tanh2_from_inv(p[2], ic));
     }
     // elem() on a pair of channels.  No packed negation exists, so the gates
-    // are formed negated, nz = -z and nr = -r (neg_sigmoid2), and every sign
+    // are formed negated, nz = -z and nr = -r (from negated denominators), and every sign
     // is carried by the algebra:
     //   f      = z (c - h) + h            = nz (h - c) + h
     //   a_c r  = (-a_c) nr
@@ -116,8 +122,10 @@ struct CellGRU {
         elem2(p, w, sp[0], f[0], A[0], beta[0]);
     }
     static __device__ __forceinline__ void elem2(const f2 (&p)[G], const W2& w, f2 h, f2& f, f2& A, f2& beta) {
-        const f2 nz = neg_sigmoid2(fma2(w.w0, h, p[0]));
-        const f2 nr = neg_sigmoid2(fma2(w.w1, h, p[1]));
+        // -z and -r from one reciprocal of (-1 - e_z)(-1 - e_r), which is
+        // the product elem() inverts, exactly
+        f2 nz, nr;
+        inv_pair2(neg_sig_den2(fma2(w.w0, h, p[0])), neg_sig_den2(fma2(w.w1, h, p[1])), nz, nr);
         const f2 wr = mul2(w.nw2, nr);
         const f2 c = tanh2(fma2(wr, h, p[2]));
         const f2 hc = sub2(h, c);

@@ -158,6 +158,46 @@ __device__ __forceinline__ float tanh_f(float x) {
     return fabsf(x) < 0.0625f ? poly : big;
 }
 
+// ---- gates that share one reciprocal ---------------------------------------
+// Two gates that do not depend on one another need the reciprocals of two
+// denominators 1 + e^u at once.  Simultaneous inversion (P. L. Montgomery,
+// "Speeding the Pollard and elliptic curve methods of factorization", Math.
+// Comp. 48 (1987)) forms both from one reciprocal of their product,
+// 1/a = b (1/(ab)) and 1/b = a (1/(ab)), trading a reciprocal on the
+// special-function unit (which also feeds the MIO queue) for two multiplies
+// on the FMA pipe.  Each exponent is capped at 2^62 so that the product stays
+// below 2^125 and its reciprocal is a normal float: a sigmoid below 2^-62
+// (an argument below about -43) is returned as 2^-62, less than 2.2e-19 from
+// its exact value, and a tanh whose exponent is capped (an argument above
+// about 21.5) still rounds to exactly 1.  The cap is taken with min.NaN, so a
+// NaN argument stays NaN.
+constexpr float kExpCap = 62.0f;
+
+__device__ __forceinline__ float min_nan(float a, float b) {
+    float d;
+    asm("min.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+    return d;
+}
+// 1 + e^{-x}, so sigma(x) = 1 / sig_den(x)
+__device__ __forceinline__ float sig_den(float x) { return 1.0f + exp2_approx(min_nan(x * -kLog2e, kExpCap)); }
+// 1 + e^{2x}, so tanh(x) = 1 - 2 / tanh_den(x)
+__device__ __forceinline__ float tanh_den(float x) {
+    return exp2_approx(min_nan(x * (2.0f * kLog2e), kExpCap)) + 1.0f;
+}
+// tanh(x) from inv = 1 / tanh_den(x), with tanh_f's Taylor branch near 0
+__device__ __forceinline__ float tanh_from_inv(float x, float inv) {
+    const float big = __fmaf_rn(-2.0f, inv, 1.0f);
+    const float x2 = x * x;
+    const float poly = x * __fmaf_rn(x2, __fmaf_rn(x2, 2.0f / 15.0f, -1.0f / 3.0f), 1.0f);
+    return fabsf(x) < 0.0625f ? poly : big;
+}
+// 1/a and 1/b from one reciprocal
+__device__ __forceinline__ void inv_pair(float a, float b, float& ia, float& ib) {
+    const float q = rcp_approx(a * b);
+    ia = b * q;
+    ib = a * q;
+}
+
 // ---- packed pairs: two channels per instruction ----------------------------
 // sm_100a's fma / add / sub / mul .rn.f32x2 operate on two floats held in a
 // register pair and round each half exactly like the scalar instruction, so a
@@ -225,6 +265,33 @@ __device__ __forceinline__ f2 tanh2(f2 x) {
     const f2 x2 = mul2(x, x);
     const f2 poly = mul2(x, fma2(x2, fma2(x2, splat2(2.0f / 15.0f), splat2(-1.0f / 3.0f)), splat2(1.0f)));
     return f2{fabsf(x.x) < 0.0625f ? poly.x : big.x, fabsf(x.y) < 0.0625f ? poly.y : big.y};
+}
+
+// the shared-reciprocal helpers above on pairs, with the same operations in
+// the same order, so that each half gives the scalar helper's bits
+__device__ __forceinline__ f2 min_nan2(f2 a, float b) { return f2{min_nan(a.x, b), min_nan(a.y, b)}; }
+__device__ __forceinline__ f2 sig_den2(f2 x) {
+    return add2(splat2(1.0f), ex2_2(min_nan2(mul2(x, splat2(-kLog2e)), kExpCap)));
+}
+// -(1 + e^{-x}): sig_den negated exactly (round-to-nearest is symmetric in
+// sign, and so are products and reciprocals), for the sign-free algebra of
+// the GRU, whose callers want -sigma and have no packed negation
+__device__ __forceinline__ f2 neg_sig_den2(f2 x) {
+    return sub2(splat2(-1.0f), ex2_2(min_nan2(mul2(x, splat2(-kLog2e)), kExpCap)));
+}
+__device__ __forceinline__ f2 tanh_den2(f2 x) {
+    return add2(ex2_2(min_nan2(mul2(x, splat2(2.0f * kLog2e)), kExpCap)), splat2(1.0f));
+}
+__device__ __forceinline__ f2 tanh2_from_inv(f2 x, f2 inv) {
+    const f2 big = fma2(splat2(-2.0f), inv, splat2(1.0f));
+    const f2 x2 = mul2(x, x);
+    const f2 poly = mul2(x, fma2(x2, fma2(x2, splat2(2.0f / 15.0f), splat2(-1.0f / 3.0f)), splat2(1.0f)));
+    return f2{fabsf(x.x) < 0.0625f ? poly.x : big.x, fabsf(x.y) < 0.0625f ? poly.y : big.y};
+}
+__device__ __forceinline__ void inv_pair2(f2 a, f2 b, f2& ia, f2& ib) {
+    const f2 q = rcp_2(mul2(a, b));
+    ia = mul2(b, q);
+    ib = mul2(a, q);
 }
 
 // max that keeps a NaN (so a non-finite residual is reported, not hidden)
