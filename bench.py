@@ -76,8 +76,12 @@ def streaming_bytes_per_elem(w, direction):
 # drain beat whole rows (8 slices)
 E2E_CHANNELS = 256
 # channels per slice of the forward + adjoint host-buffer pipeline: each
-# slice holds all B rows, so 4096 channels in slices of 128 make 32 slices
-E2E_STEP_CHANNELS = 128
+# slice holds all B rows.  Measured on the long-sequence GRU (1 x 131072 x
+# 4096): 128 channels 285 ms, 256: 224, 512: 199, 1024: 186, 2048: 214, one
+# slice 254 ms.  Narrow slices of a long sequence leave few channel groups,
+# each with a long chain of tiles, and the solver becomes the bottleneck;
+# wide ones lengthen the pipeline's fill and drain.
+E2E_STEP_CHANNELS = 1024
 
 KERNEL_SOURCES = ["newton_fwd.cuh", "adjoint_bwd.cuh", "lookback.cuh", "cells.cuh", "common.cuh", "tma.cuh", "pararnn_abi.cu"]
 

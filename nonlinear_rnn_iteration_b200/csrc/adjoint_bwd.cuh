@@ -658,8 +658,15 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
     if (is_scan && prev_tile >= 0) store_tile_partial<Sh, PxT>(sm, (it - 1) & 1, prm, prev_tile, lane);
 }
 
-// dL/da[g][d] = sum over batch rows b, then over tiles along time, of the
-// per-tile partials: one thread per (g, d), a fixed summation order.
+// dL/da[g][d] = the sum, over batch rows b and tiles along time, of the
+// per-tile partials.  One block per (channel group, gate), kReduceSplit warps:
+// lane = channel (a warp reads one tile's 32 partials of a gate, 128 bytes,
+// coalesced), warp j sums the tiles q = b * nChunks + pos with q = j mod
+// kReduceSplit in increasing q, and the block adds the warps' sums in warp
+// order.  The order depends only on (B, nChunks), so the result is the same
+// bits on every call and for every slice of channels of the same problem.
+constexpr int kReduceSplit = 8;
+
 struct ReduceParams {
     const float* part;
     float* dLda;
@@ -667,21 +674,46 @@ struct ReduceParams {
     int G, W;
 };
 
-__global__ void reduce_da_kernel(const ReduceParams prm) {
-    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (i >= (int64_t)prm.G * prm.D) return;
-    const int g = (int)(i / prm.D);
-    const int64_t d = i - (int64_t)g * prm.D;
-    const int64_t cg = d / prm.W, ch = d - cg * prm.W;
-    float acc = 0.0f;
-    for (int64_t b = 0; b < prm.B; ++b) {
-        const int64_t gid = b * prm.nCG + cg;
-        for (int64_t pos = 0; pos < prm.nChunks; ++pos) {
-            const int64_t tile = pos * prm.nGroups + gid;
-            acc += prm.part[(tile * prm.G + g) * prm.W + ch];
+__global__ void __launch_bounds__(32 * kReduceSplit) reduce_da_kernel(const ReduceParams prm) {
+    __shared__ float acc_w[kReduceSplit][32];
+    const int64_t cg = blockIdx.x;
+    const int g = blockIdx.y;
+    const int lane = threadIdx.x & 31, j = threadIdx.x >> 5;
+    const int64_t Q = prm.B * prm.nChunks;
+    // W is a multiple of 32: the block covers W / 32 runs of 32 channels
+    for (int c0 = 0; c0 < prm.W; c0 += 32) {
+        const int ch = c0 + lane;
+        float acc = 0.0f;
+        int64_t q = j;
+        // four independent loads in flight per step, added in order
+        for (; q + 3 * kReduceSplit < Q; q += 4 * kReduceSplit) {
+            float v[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int64_t qq = q + u * kReduceSplit;
+                const int64_t b = qq / prm.nChunks, pos = qq - b * prm.nChunks;
+                const int64_t tile = pos * prm.nGroups + b * prm.nCG + cg;
+                v[u] = __ldg(prm.part + (tile * prm.G + g) * prm.W + ch);
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) acc += v[u];
         }
+        for (; q < Q; q += kReduceSplit) {
+            const int64_t b = q / prm.nChunks, pos = q - b * prm.nChunks;
+            const int64_t tile = pos * prm.nGroups + b * prm.nCG + cg;
+            acc += __ldg(prm.part + (tile * prm.G + g) * prm.W + ch);
+        }
+        acc_w[j][lane] = acc;
+        __syncthreads();
+        if (j == 0) {
+            float sum = acc_w[0][lane];
+#pragma unroll
+            for (int k = 1; k < kReduceSplit; ++k) sum += acc_w[k][lane];
+            const int64_t d = cg * prm.W + ch;
+            if (d < prm.D) prm.dLda[g * prm.D + d] = sum;
+        }
+        __syncthreads();
     }
-    prm.dLda[g * prm.D + d] = acc;
 }
 
 }  // namespace pararnn

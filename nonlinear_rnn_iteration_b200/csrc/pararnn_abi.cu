@@ -544,8 +544,8 @@ pararnn_status launch_bwd(const Plan& pl, BwdParams prm, float* dLda, cudaStream
         rp.nGroups = pl.nGroups;
         rp.G = Sh::G;
         rp.W = Sh::W;
-        const int64_t n = (int64_t)Sh::G * prm.D;
-        reduce_da_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(rp);
+        static_assert(Sh::W % 32 == 0, "the reduction takes whole runs of 32 channels");
+        reduce_da_kernel<<<dim3((unsigned)pl.nCG, (unsigned)Sh::G), 32 * kReduceSplit, 0, st>>>(rp);
         e = cudaGetLastError();
         if (e != cudaSuccess) return cuda_fail(e, "dL/da reduction launch");
     }
