@@ -42,6 +42,7 @@ struct BwdParams {
     unsigned* ticket;
     int64_t B, T, D;
     int64_t nCG, nChunks, nTiles;
+    int late_probe;     // probe the predecessor while the tile is evaluated (see the scan warp)
     LookbackCtx lb;     // nSlots = 1
 };
 
@@ -238,7 +239,19 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
             for (int j = 0; j < CPL; ++j)
 #pragma unroll
                 for (int s = 0; s < S; ++s) zero[j][s] = 0.0f;  // mu_T = 0
-            Probe<S, W> pr;  // no early probe: the single pass is too short to hide one
+            // With at least as many channel groups as resident blocks, a tile's
+            // predecessor (one ticket per group earlier) was claimed a whole
+            // round of tiles before it and has usually finished: its state is
+            // then read once the evaluation has started (after the set-up
+            // barrier), and the look-back after the totals barrier is skipped.
+            // With fewer groups the predecessor is still running, the probe
+            // misses, and its reads cost more than they save (measured: the
+            // 8 x 4096 x 2048 GRU adjoint 12 % faster with it, the
+            // 1 x 131072 x 4096 GRU 6 % and the 4 x 32768 x 1024 LSTM 3 %
+            // slower).  The 2 x 2 cell's adjoint is at its register limit,
+            // where even the unused branch costs spills, so it has no late
+            // probe.
+            Probe<S, W> pr;
             pr.st = 0;
             block_sync();  // (1) tile set up
             if (lane == 0) {
@@ -250,6 +263,9 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
                 sm.ticket[sn] = t2;
                 if constexpr (Sh::kTma)
                     if (t2 < prm.nTiles && prev_t < prm.nTiles) issue_bwd_load<Cell, PxT, Sh>(&maps, sm, prm, t2, sn);
+            }
+            if constexpr (S == 1) {
+                if (prm.late_probe) probe_issue<S, W>(prm.lb, tile, pos, 0, lane, pr);
             }
             if (prev_tile >= 0) store_tile_partial<Sh, PxT>(sm, (it - 1) & 1, prm, prev_tile, lane);
             prev_tile = tile;

@@ -530,6 +530,7 @@ pararnn_status launch_bwd(const Plan& pl, BwdParams prm, float* dLda, cudaStream
     unsigned grid = 0;
     pararnn_status s = persistent_grid(kern, Sh::NT, smem, pl.nTiles, grid, "adjoint_bwd");
     if (s != PARARNN_OK) return s;
+    prm.late_probe = pl.nGroups >= (int64_t)grid ? 1 : 0;
     kern<<<grid, Sh::NT, smem, st>>>(maps, prm);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "backward kernel launch");
