@@ -313,9 +313,9 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
             }
         }
     }
-    if (is_scan) {
+    if (is_scan && !kLean) {
         // the first tiles' weights (read by the compute warps after their
-        // set-up barrier)
+        // set-up barrier; the lean linear scan reads none)
         __syncwarp();
 #pragma unroll
         for (int s = 0; s < NSTAGE - 1; ++s) {
@@ -380,7 +380,7 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
             // the claimed tile's weights, into its stage (whose previous
             // readers have passed this tile's set-up barrier); the scan warp
             // waits for them here, while the compute warps evaluate
-            if constexpr (!kCluster) {
+            if constexpr (!kCluster && !kLean) {
                 const int sn = (it + NSTAGE - 1) % NSTAGE;
                 const unsigned t2 = __shfl_sync(0xffffffffu, sm.ticket[sn], 0);
                 const unsigned prev_t = sm.ticket[(it + NSTAGE - 2) % NSTAGE];
