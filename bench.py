@@ -473,13 +473,15 @@ def time_graph(prob, steps=50, replays=4):
     with torch.cuda.graph(g, stream=side):
         for _ in range(steps):
             prob._fwd(*args)
-    g.replay()
-    torch.cuda.synchronize()
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    t0.record(side)
-    for _ in range(replays):
+    # a graph replays on the current stream: replay and time on the side stream
+    with torch.cuda.stream(side):
         g.replay()
-    t1.record(side)
+        torch.cuda.synchronize()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(side)
+        for _ in range(replays):
+            g.replay()
+        t1.record(side)
     torch.cuda.synchronize()
     del g
     prob.check_status()

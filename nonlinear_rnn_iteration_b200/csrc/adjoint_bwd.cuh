@@ -678,10 +678,12 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
 // per-tile partials.  One block per (channel group, gate), kReduceSplit warps:
 // lane = channel (a warp reads one tile's 32 partials of a gate, 128 bytes,
 // coalesced), warp j sums the tiles q = b * nChunks + pos with q = j mod
-// kReduceSplit in increasing q, and the block adds the warps' sums in warp
-// order.  The order depends only on (B, nChunks), so the result is the same
-// bits on every call and for every slice of channels of the same problem.
-constexpr int kReduceSplit = 8;
+// kReduceSplit in increasing q, kReduceAhead loads in flight, and the block
+// adds the warps' sums in warp order.  The order depends only on (B,
+// nChunks), so the result is the same bits on every call and for every slice
+// of channels of the same problem.
+constexpr int kReduceSplit = 16;
+constexpr int kReduceAhead = 8;
 
 struct ReduceParams {
     const float* part;
@@ -696,29 +698,24 @@ __global__ void __launch_bounds__(32 * kReduceSplit) reduce_da_kernel(const Redu
     const int g = blockIdx.y;
     const int lane = threadIdx.x & 31, j = threadIdx.x >> 5;
     const int64_t Q = prm.B * prm.nChunks;
+    auto at = [&](int64_t q, int ch) {
+        const int64_t b = q / prm.nChunks, pos = q - b * prm.nChunks;
+        const int64_t tile = pos * prm.nGroups + b * prm.nCG + cg;
+        return __ldg(prm.part + (tile * prm.G + g) * prm.W + ch);
+    };
     // W is a multiple of 32: the block covers W / 32 runs of 32 channels
     for (int c0 = 0; c0 < prm.W; c0 += 32) {
         const int ch = c0 + lane;
         float acc = 0.0f;
         int64_t q = j;
-        // four independent loads in flight per step, added in order
-        for (; q + 3 * kReduceSplit < Q; q += 4 * kReduceSplit) {
-            float v[4];
+        for (; q + (kReduceAhead - 1) * kReduceSplit < Q; q += kReduceAhead * kReduceSplit) {
+            float v[kReduceAhead];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int64_t qq = q + u * kReduceSplit;
-                const int64_t b = qq / prm.nChunks, pos = qq - b * prm.nChunks;
-                const int64_t tile = pos * prm.nGroups + b * prm.nCG + cg;
-                v[u] = __ldg(prm.part + (tile * prm.G + g) * prm.W + ch);
-            }
+            for (int u = 0; u < kReduceAhead; ++u) v[u] = at(q + u * kReduceSplit, ch);
 #pragma unroll
-            for (int u = 0; u < 4; ++u) acc += v[u];
+            for (int u = 0; u < kReduceAhead; ++u) acc += v[u];
         }
-        for (; q < Q; q += kReduceSplit) {
-            const int64_t b = q / prm.nChunks, pos = q - b * prm.nChunks;
-            const int64_t tile = pos * prm.nGroups + b * prm.nCG + cg;
-            acc += __ldg(prm.part + (tile * prm.G + g) * prm.W + ch);
-        }
+        for (; q < Q; q += kReduceSplit) acc += at(q, ch);
         acc_w[j][lane] = acc;
         __syncthreads();
         if (j == 0) {

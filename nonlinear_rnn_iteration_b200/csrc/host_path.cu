@@ -314,7 +314,12 @@ extern "C" pararnn_status pararnn_newton_step_host(pararnn_cell cell, int64_t B,
     }
     if (!preacts_host || !dL_dH_host || !H_host || !dL_dpx_host)
         return hp::fail(PARARNN_EINVAL, "pararnn_newton_step_host: preacts, dL_dH, H and dL_dpx are required");
-    const int64_t ncs = (D + l.chans - 1) / l.chans;
+    // The copies out (H and dL/dpx, float32) outweigh the copies in, so the
+    // pipeline runs at the pace of the copies out and only the first slice's
+    // copy in is exposed: the first slice takes a quarter of the others'
+    // channels (a multiple of 8), the rest channels_per_slice each.
+    const int64_t first = (l.chans < D && l.chans >= 32) ? ((l.chans / 4 + 7) / 8) * 8 : l.chans;
+    const int64_t ncs = 1 + (D - first + l.chans - 1) / l.chans;
 
     cudaStream_t sin = nullptr, scomp = nullptr, sout = nullptr;
     cudaEvent_t start = nullptr, ev_in[hp::kSlots] = {}, ev_comp[hp::kSlots] = {}, ev_out[hp::kSlots] = {};
@@ -351,7 +356,9 @@ extern "C" pararnn_status pararnn_newton_step_host(pararnn_cell cell, int64_t B,
     pararnn_status st = PARARNN_OK;
     for (int64_t ic = 0; ic < ncs && st == PARARNN_OK; ++ic) {
         const int k = (int)(ic % hp::kSlots);
-        const int64_t d0 = ic * l.chans, dn = (d0 + l.chans <= D) ? l.chans : D - d0;
+        const int64_t d0 = ic == 0 ? 0 : first + (ic - 1) * l.chans;
+        const int64_t want = ic == 0 ? first : l.chans;
+        const int64_t dn = (d0 + want <= D) ? want : D - d0;
         unsigned char* p = ws + 256 + (size_t)k * l.slot_bytes;
         void* sws = p;
         p += hp::align256(l.ws_bytes);
