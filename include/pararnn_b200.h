@@ -322,10 +322,11 @@ pararnn_status pararnn_newton_forward_host(pararnn_cell cell, int64_t B, int64_t
  * pararnn_newton_forward followed by pararnn_newton_backward, with the
  * pre-activations and dL/dH read from host memory and H and dL/dpx written
  * back to it (pinned memory lets the copies overlap).  The channels are cut
- * into slices of channels_per_slice channels, each holding every batch row,
- * that pass through three device slots on three internal streams -- copy in,
- * forward + adjoint, copy out -- so that both PCIe directions and the solver
- * work at once.  A slice's dL/da columns are complete sums over (b, t) and
+ * into slices of channels_per_slice channels (the first slice a quarter of
+ * that, rounded up to a multiple of 8, so that the pipeline fills quickly),
+ * each holding every batch row, that pass through three device slots on
+ * three internal streams -- copy in, forward + adjoint, copy out -- so that
+ * both PCIe directions and the solver work at once.  A slice's dL/da columns are complete sums over (b, t) and
  * are written straight into dL_da.  Channels are independent recurrences and
  * the tiling along T does not depend on the slice, so every output is
  * bit-identical to pararnn_newton_forward + pararnn_newton_backward on the
