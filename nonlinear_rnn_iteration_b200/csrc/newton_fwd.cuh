@@ -268,6 +268,16 @@ __global__ void __launch_bounds__(Sh::NT, Sh::MINB)
     SM& sm = *reinterpret_cast<SM*>(smem_raw);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if constexpr (kCluster) {
+        // Programmatic dependent launch (the cluster path is launched with
+        // it): let the stream's next kernel be launched now, so that its
+        // launch overlaps this one, and wait until the stream's previous
+        // kernel has finished and its writes are visible before reading or
+        // writing global memory.  Without the launch attribute both are
+        // no-ops.
+        asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+    }
     const bool is_scan = warp == NW;
     const int64_t T = prm.T, D = prm.D;
     const PxT* pxg = static_cast<const PxT*>(prm.px);

@@ -433,13 +433,19 @@ pararnn_status launch_fwd_cluster(const Plan& pl, FwdParams prm, const CUtensorM
     cfg.blockDim = dim3(Sh::NT, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
-    cudaLaunchAttribute attr;
-    attr.id = cudaLaunchAttributeClusterDimension;
-    attr.val.clusterDim.x = csize;
-    attr.val.clusterDim.y = 1;
-    attr.val.clusterDim.z = 1;
-    cfg.attrs = &attr;
-    cfg.numAttrs = 1;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = csize;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    // programmatic dependent launch: the kernel may be launched while the
+    // stream's previous kernel is still running, if that kernel allows it
+    // (the cluster forward allows it as it starts); it waits for that kernel
+    // to finish, and its memory to be visible, before touching global memory
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
     if (log_enabled())
         fprintf(stderr, "pararnn: newton_fwd(cluster) grid=%lld cluster=%d threads=%d smem=%zu\n",
                 (long long)pl.nTiles, csize, Sh::NT, smem);
