@@ -117,3 +117,32 @@ def test_cluster_status_is_tagged_per_call(cuda_device):
     assert run(x["pxt"], 0) == binding.OK              # cluster path after a look-back call
     assert run(bad, 0) == binding.ENONFINITE
     assert run(x["pxt"], NO_CLUSTER) == binding.OK     # look-back path clears the header
+
+
+def test_back_to_back_calls_read_the_previous_calls_output():
+    # The cluster kernel is launched with programmatic dependent launch: a
+    # call may be launched while the previous one runs, and must still see
+    # everything it wrote.  Chain two calls with no host synchronisation,
+    # the second reading the first's output as its pre-activations (H of the
+    # first is written over the start of the second's px buffer), and
+    # compare with the same calls separated by a synchronisation.
+    cell, B, T, D, K = oracle.DIAG_GRU, 1, 1024, 64, 3
+    x = _inputs(cell, B, T, D, seed=41)
+    s = torch.cuda.current_stream()
+    px2_ref = torch.from_numpy(_inputs(cell, B, T, D, seed=42)["px"]).to(DEV)
+    H1 = binding.newton_forward(cell, x["pxt"], x["wt"], None, K=K)
+    torch.cuda.synchronize()
+    px2_ref.view(-1)[: B * T * D].copy_(H1.view(-1))
+    torch.cuda.synchronize()
+    ref = binding.newton_forward(cell, px2_ref, x["wt"], None, K=K)
+    torch.cuda.synchronize()
+    for rep in range(5):
+        px2 = torch.from_numpy(_inputs(cell, B, T, D, seed=42)["px"]).to(DEV)
+        torch.cuda.synchronize()
+        H1_into_px2 = px2.view(-1)[: B * T * D].view(B, T, 1, D)
+        # the first call writes straight into px2; the second reads px2
+        binding.newton_forward(cell, x["pxt"], x["wt"], None, K=K, out=H1_into_px2, sync_status=False)
+        H2 = binding.newton_forward(cell, px2, x["wt"], None, K=K, sync_status=False)
+        torch.cuda.synchronize()
+        assert torch.equal(px2, px2_ref), rep
+        assert torch.equal(H2, ref), rep
