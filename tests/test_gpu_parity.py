@@ -157,6 +157,23 @@ def test_linear_any_k_is_one_scan(cuda_device):
     assert np.all(to_np(r4)[1:] == to_np(r1)[1])
 
 
+@pytest.mark.parametrize("case", [(oracle.DIAG_GRU, 3, 12000, 100), (oracle.DIAG_LSTM, 2, 9000, 40)],
+                         ids=lambda c: "cell%d_B%dT%dD%d" % c)
+def test_backward_many_tiles(case, cuda_device):
+    # hundreds of tiles per channel group and several batch rows: the dL/da
+    # reduction's interleaved per-warp chains and the look-back over many
+    # tiles, against the oracle, with ragged channel groups
+    cell, B, T, D = case
+    K = 2
+    x = _inputs(cell, B, T, D, seed=B * 13 + T + D, h0=True, grad=True)
+    H = binding.newton_forward(cell, x["pxt"], x["wt"], x["h0t"], K=K)
+    dpx, da, dh0 = binding.newton_backward(cell, x["pxt"], H, x["gt"], x["wt"], x["h0t"], want_dh0=True)
+    dpxo, dao, dh0o = oracle.adjoint(cell, x["px"], x["w"], x["h0"], to_np(H), x["g"])
+    assert rel_err(to_np(dpx), dpxo) <= TOL_G
+    assert rel_err(to_np(dh0), dh0o) <= TOL_G
+    assert rel_err(to_np(da), dao) <= TOL_G
+
+
 def test_newton_reaches_unroll(cuda_device):
     # prefix exactness: K = T Newton steps reproduce the sequential unroll
     for cell in (oracle.DIAG_GRU, oracle.DIAG_LSTM):
