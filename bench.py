@@ -690,7 +690,10 @@ def run_native(args):
     else:
         e2e_ms, h2d, d2h = time_e2e(prob, steps=3)
         e2e = {"value": w.elements / (e2e_ms / 1e3) * world, "unit": UNIT, "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 3)}
+               "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 3),
+               "path": ("pararnn_newton_step_host, %d-channel slices" % E2E_STEP_CHANNELS if w.backward
+                        else "pararnn_newton_forward_host, 1-row x %d-channel slices" % E2E_CHANNELS),
+               "host_memory": "pinned"}
     step = "forward (K=%d Newton iterations)" % w.K if w.cell != "linear" else "forward (one exact scan)"
     if w.backward:
         step += " + adjoint backward"
