@@ -541,6 +541,7 @@ def time_e2e(prob, steps):
 
         h2d = px_host.numel() * px_host.element_size() + g_host.numel() * 4
         d2h = H_host.numel() * 4 + dpx_host.numel() * 4
+        path = "pararnn_newton_step_host, %s" % ("%d-channel slices" % chans if chans else "one slice")
     else:
         # slices of one batch row and E2E_CHANNELS channels
         chans = E2E_CHANNELS if (w.D % 8 == 0 and w.D > E2E_CHANNELS) else 0
@@ -555,6 +556,7 @@ def time_e2e(prob, steps):
 
         h2d = px_host.numel() * px_host.element_size()
         d2h = H_host.numel() * 4
+        path = "pararnn_newton_forward_host, one-row %s" % ("x %d-channel slices" % chans if chans else "slices")
     one()
     torch.cuda.synchronize()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -566,7 +568,7 @@ def time_e2e(prob, steps):
     st = binding.pararnn_status_sync(ws_host, s)
     if st != binding.OK:
         raise RuntimeError("host-buffer step device status %s" % binding.STATUS[st])
-    return t0.elapsed_time(t1) / steps, h2d, d2h
+    return t0.elapsed_time(t1) / steps, h2d, d2h, path
 
 
 def cpu_baseline(w, device, seed, target_s=12.0, max_bytes=2.0e9):
@@ -688,12 +690,10 @@ def run_native(args):
     if args.quick:
         e2e = None
     else:
-        e2e_ms, h2d, d2h = time_e2e(prob, steps=3)
+        e2e_ms, h2d, d2h, e2e_path = time_e2e(prob, steps=3)
         e2e = {"value": w.elements / (e2e_ms / 1e3) * world, "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 3),
-               "path": ("pararnn_newton_step_host, %d-channel slices" % E2E_STEP_CHANNELS if w.backward
-                        else "pararnn_newton_forward_host, 1-row x %d-channel slices" % E2E_CHANNELS),
-               "host_memory": "pinned"}
+               "path": e2e_path, "host_memory": "pinned"}
     step = "forward (K=%d Newton iterations)" % w.K if w.cell != "linear" else "forward (one exact scan)"
     if w.backward:
         step += " + adjoint backward"
